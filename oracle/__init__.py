@@ -1,0 +1,239 @@
+"""CPU oracle for the gated delta-rule recurrence (KDA / Complex KDA / RDA / GDN-2).
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline / reference leg of ``bench.py``.  The GPU library never
+imports it and it never imports the GPU library; the two share only the seeded
+input generators in ``workloads``.
+
+Three independent formulations, all float64:
+
+* ``recurrence`` -- the plain-C step recurrence in ``kda_oracle.c`` (decay,
+  residual u = m - S'^T a~, rank-one write, readout o_t = S_t^T q_t), OpenMP
+  over (sequence, head).  This is THE oracle the GPU path is compared with.
+* ``literal_recurrence`` -- NumPy, the state updates exactly as the
+  Raon-1-mini-preview discussion page prints them: explicit d_k x d_k
+  transition matrices (I - beta k k^T) Diag(alpha), (I - e k k^T) Diag(alpha),
+  (I - k (b (.) k)^T) Diag(alpha) and write terms beta k v^T, w k v^T,
+  k (w (.) v)^T.  Small inputs only.
+* ``brute_force`` -- NumPy dense closed form of the unrolled recurrence,
+  S_t = (prod_{s<=t} A_s) S_0 + sum_{s<=t} (prod_{s<r<=t} A_r) W_s, evaluated
+  from scratch for every t.  Tiny inputs only.
+
+Every function is pinned by ``tests/test_oracle_pins.py`` against properties
+the pages fix (RDA = KDA when e = w; GDN-2 = RDA for constant vectors;
+non-expansive Complex-KDA transitions; the exact 2D rotation) and textbook
+special cases (causal linear attention, gated linear attention, overwrite
+memory, Householder reflection).  No function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+VARIANT_CODE = {"kda": 0, "rda": 1, "gdn2": 2}
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (float64, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off",
+                               "-fno-fast-math", "-shared", "-fPIC", _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_recurrence.restype = ctypes.c_int
+        lib.oracle_recurrence.argtypes = [ctypes.c_int] * 6 + [dp] * 6 + [ip, ctypes.c_int] + [dp] * 3 + [ctypes.c_int]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _f64(x) -> Optional[np.ndarray]:
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor: exact upcast of bf16 / fp32
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a):
+    if a is None:
+        return ctypes.POINTER(ctypes.c_double)()
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def recurrence_arrays(variant: str, q, k, v, alpha, g1, g2=None, cu_seqlens=None,
+                      initial_state=None, threads: int = 0):
+    """Step recurrence on float64 arrays with the library's layouts.
+
+    q,k,alpha [B,T,H,dk]; v [B,T,H,dv]; g1/g2 per the variant; cu_seqlens
+    optional int offsets (B must be 1); initial_state [N,H,dk,dv] or None.
+    Returns (o [B,T,H,dv], final_state [N,H,dk,dv]) as float64.
+    """
+    q, k, v, alpha, g1, g2 = (_f64(x) for x in (q, k, v, alpha, g1, g2))
+    s0 = _f64(initial_state)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = None
+    N = B
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+                                             dtype=np.int32))
+        N = cu.size - 1
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    sf = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().oracle_recurrence(
+        VARIANT_CODE[variant], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(g1), _ptr(g2),
+        cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int)) if cu is not None else ctypes.POINTER(ctypes.c_int)(),
+        N, _ptr(s0), _ptr(sf), _ptr(o), int(threads))
+    if rc != 0:
+        raise ValueError("oracle_recurrence rejected its arguments")
+    return o, sf
+
+
+def recurrence(inp, seqs: Optional[Sequence[int]] = None, heads: Optional[Sequence[int]] = None,
+               threads: int = 0):
+    """Oracle on a ``workloads.ChunkInputs`` problem, optionally restricted to
+    some sequences and heads (they are independent, so a restriction is exact).
+
+    Returns (o, final_state) float64.  Without a restriction o is [B,T,H,dv]
+    and final_state [N,H,dk,dv]; with one, o is a dict {(n, h): [len, dv]} and
+    final_state a dict {(n, h): [dk, dv]}.
+    """
+    if seqs is None and heads is None:
+        return recurrence_arrays(inp.variant, inp.q, inp.k, inp.v, inp.alpha, inp.g1, inp.g2,
+                                 inp.cu_seqlens, inp.initial_state, threads)
+    seqs = list(range(inp.num_seqs)) if seqs is None else list(seqs)
+    heads = list(range(inp.H)) if heads is None else list(heads)
+    # gather every requested (sequence, head) as its own batch row, padded to the
+    # longest length (padding rows are never read: cu_seqlens bounds them)
+    parts = []
+    for n in seqs:
+        b, t0, ln = inp.seq_bounds(n)
+        for h in heads:
+            parts.append((n, h, b, t0, ln))
+    lens = [p[4] for p in parts]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    tot = int(cu[-1])
+
+    def gather(x, last):
+        if x is None:
+            return None
+        out = np.zeros((1, tot, 1) + ((last,) if last else ()), dtype=np.float64)
+        for i, (n, h, b, t0, ln) in enumerate(parts):
+            sl = x[b, t0:t0 + ln, h]
+            out[0, cu[i]:cu[i + 1], 0] = sl.detach().cpu().double().numpy() if hasattr(sl, "detach") else sl
+        return out
+
+    dk, dv = inp.d_k, inp.d_v
+    g_last1 = dk if inp.variant == "gdn2" else 0
+    g_last2 = dv if inp.variant == "gdn2" else 0
+    s0 = None
+    if inp.initial_state is not None:
+        s0 = np.stack([inp.initial_state[n, h].double().numpy() for (n, h, *_r) in parts])[:, None]
+    o, sf = recurrence_arrays(inp.variant, gather(inp.q, dk), gather(inp.k, dk), gather(inp.v, dv),
+                              gather(inp.alpha, dk), gather(inp.g1, g_last1), gather(inp.g2, g_last2),
+                              cu, s0, threads)
+    o_d, s_d = {}, {}
+    for i, (n, h, *_r) in enumerate(parts):
+        o_d[(n, h)] = o[0, cu[i]:cu[i + 1], 0]
+        s_d[(n, h)] = sf[i, 0]
+    return o_d, s_d
+
+
+# ---------------------------------------------------------------------------
+# Literal product form and brute force (small inputs)
+# ---------------------------------------------------------------------------
+
+def transition_and_write(variant: str, k, v, alpha, g1, g2):
+    """The pages' transition A_t (d_k x d_k) and write term W_t (d_k x d_v) for
+    one token, exactly as the three update equations print them."""
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    D = np.diag(np.asarray(alpha, dtype=np.float64))
+    I = np.eye(k.size)
+    if variant == "kda":        # S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T
+        beta = float(g1)
+        return (I - beta * np.outer(k, k)) @ D, beta * np.outer(k, v)
+    if variant == "rda":        # S_t = (I - e k k^T) Diag(alpha) S_{t-1} + w k v^T
+        e, w = float(g1), float(g2)
+        return (I - e * np.outer(k, k)) @ D, w * np.outer(k, v)
+    if variant == "gdn2":       # S_t = (I - k (b (.) k)^T) Diag(alpha) S_{t-1} + k (w (.) v)^T
+        b, w = np.asarray(g1, dtype=np.float64), np.asarray(g2, dtype=np.float64)
+        return (I - np.outer(k, b * k)) @ D, np.outer(k, w * v)
+    raise ValueError(variant)
+
+
+def _tok(x, b, t, h):
+    if x is None:
+        return None
+    y = x[b, t, h]
+    return y.detach().cpu().double().numpy() if hasattr(y, "detach") else np.asarray(y, dtype=np.float64)
+
+
+def literal_recurrence(variant: str, q, k, v, alpha, g1, g2=None, initial_state=None):
+    """Fixed-length batches only.  Returns (o [B,T,H,dv], S_T [B,H,dk,dv])."""
+    B, T, H, dk = tuple(q.shape)
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    sf = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if initial_state is None else _f64(initial_state[b, h])
+            for t in range(T):
+                A, W = transition_and_write(variant, _tok(k, b, t, h), _tok(v, b, t, h), _tok(alpha, b, t, h),
+                                            _tok(g1, b, t, h), _tok(g2, b, t, h))
+                S = A @ S + W
+                o[b, t, h] = S.T @ _tok(q, b, t, h)
+            sf[b, h] = S
+    return o, sf
+
+
+def brute_force(variant: str, q, k, v, alpha, g1, g2=None, initial_state=None):
+    """Dense unrolled form, recomputed from scratch at every t.  Returns (o, S_T)."""
+    B, T, H, dk = tuple(q.shape)
+    dv = v.shape[-1]
+    o = np.zeros((B, T, H, dv))
+    sf = np.zeros((B, H, dk, dv))
+    for b in range(B):
+        for h in range(H):
+            S0 = np.zeros((dk, dv)) if initial_state is None else _f64(initial_state[b, h])
+            mats = [transition_and_write(variant, _tok(k, b, t, h), _tok(v, b, t, h), _tok(alpha, b, t, h),
+                                         _tok(g1, b, t, h), _tok(g2, b, t, h)) for t in range(T)]
+            for t in range(T):
+                # S_t = (A_t ... A_0) S_0 + sum_s (A_t ... A_{s+1}) W_s
+                P = np.eye(dk)
+                for r in range(t + 1):
+                    P = mats[r][0] @ P
+                St = P @ S0
+                for s in range(t + 1):
+                    Q = np.eye(dk)
+                    for r in range(s + 1, t + 1):
+                        Q = mats[r][0] @ Q
+                    St = St + Q @ mats[s][1]
+                o[b, t, h] = St.T @ _tok(q, b, t, h)
+                if t == T - 1:
+                    sf[b, h] = St
+    return o, sf

@@ -1,0 +1,271 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test ties the oracle to something other than itself: the pages' own
+product form, a property the pages state, a closed form, or a textbook special
+case.  A plausible slip anywhere in the oracle (a dropped term, a wrong sign,
+decay applied after the erase instead of before, a transposed state, a readout
+on the pre-update state, a gate read at the wrong index) fails at least one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import make_chunk_inputs, tiny_ckda
+
+RNG = np.random.default_rng(1234)
+
+
+def _small(variant, rng_seed, B=2, T=9, H=2, dk=5, dv=3, gate_range="standard", init="random"):
+    return make_chunk_inputs(variant, gate_range, "f32", B=B, T=T, H=H, d_k=dk, d_v=dv,
+                             seed=rng_seed, init_state=init, init_std=0.5)
+
+
+@pytest.mark.parametrize("variant", ["kda", "rda", "gdn2"])
+@pytest.mark.parametrize("gate_range", ["standard", "extended"])
+def test_step_recurrence_equals_literal_product_form(variant, gate_range):
+    """C step recurrence == the update equations exactly as printed
+    (Raon-1-mini-preview discussion: KDA, RDA, GDN-2 equations)."""
+    inp = _small(variant, 7, gate_range=gate_range)
+    o, sf = oracle.recurrence(inp)
+    o2, sf2 = oracle.literal_recurrence(variant, inp.q, inp.k, inp.v, inp.alpha, inp.g1, inp.g2,
+                                        inp.initial_state)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sf, sf2, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("variant", ["kda", "rda", "gdn2"])
+def test_step_recurrence_equals_brute_force(variant):
+    """Dense unrolled closed form on tiny inputs, recomputed for every t."""
+    inp = _small(variant, 11, B=1, T=6, H=1, dk=4, dv=3, gate_range="extended")
+    o, sf = oracle.recurrence(inp)
+    o2, sf2 = oracle.brute_force(variant, inp.q, inp.k, inp.v, inp.alpha, inp.g1, inp.g2, inp.initial_state)
+    np.testing.assert_allclose(o, o2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sf, sf2, rtol=0, atol=1e-12)
+
+
+def test_rda_reduces_to_kda_when_e_equals_w():
+    """'RDA reduces to KDA when e_t = w_t' (Raon-1-mini-preview discussion)."""
+    kda = _small("kda", 3, gate_range="extended")
+    o_k, s_k = oracle.recurrence(kda)
+    o_r, s_r = oracle.recurrence_arrays("rda", kda.q, kda.k, kda.v, kda.alpha, kda.g1, kda.g1,
+                                        None, kda.initial_state)
+    assert np.array_equal(o_k, o_r) and np.array_equal(s_k, s_r)
+    # and a genuinely different w changes the result (the write gate is read)
+    o_r2, _ = oracle.recurrence_arrays("rda", kda.q, kda.k, kda.v, kda.alpha, kda.g1, kda.g1 * 0.5,
+                                       None, kda.initial_state)
+    assert not np.allclose(o_k, o_r2)
+
+
+def test_gdn2_reduces_to_rda_for_constant_vectors():
+    """GDN-2 with b_t = e_t 1 and w_t = w_t 1 is RDA (the two equations on the
+    discussion page coincide term by term)."""
+    rda = _small("rda", 5, dk=6, dv=4)
+    b = rda.g1[..., None].expand(*rda.g1.shape, rda.d_k).contiguous()
+    w = rda.g2[..., None].expand(*rda.g2.shape, rda.d_v).contiguous()
+    o_r, s_r = oracle.recurrence(rda)
+    o_g, s_g = oracle.recurrence_arrays("gdn2", rda.q, rda.k, rda.v, rda.alpha, b, w, None, rda.initial_state)
+    np.testing.assert_allclose(o_g, o_r, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(s_g, s_r, rtol=0, atol=1e-14)
+    # channel-wise gates that are NOT constant give a different answer
+    b2 = b.clone()
+    b2[..., 0] = 0.0
+    o_g2, _ = oracle.recurrence_arrays("gdn2", rda.q, rda.k, rda.v, rda.alpha, b2, w, None, rda.initial_state)
+    assert not np.allclose(o_g2, o_r)
+
+
+def _transitions_from_oracle(k, alpha, beta):
+    """Read the oracle's transition matrices: start each sequence from S_0 = I
+    (d_v = d_k) with v = 0, run one token; then S_1 = A_1 I = A_1."""
+    n, d = k.shape
+    z = np.zeros((n, 1, 1, d))
+    s0 = np.broadcast_to(np.eye(d), (n, 1, d, d)).copy()
+    _, sf = oracle.recurrence_arrays("kda", z, k.reshape(n, 1, 1, d), z, alpha.reshape(n, 1, 1, d),
+                                     beta.reshape(n, 1, 1), None, None, s0)
+    return sf[:, 0]
+
+
+def test_ckda_transitions_are_non_expansive():
+    """Complex KDA transitions (I - beta k k^T) Diag(alpha) with unit k,
+    alpha in [-1,1]^d and beta in [0,2] have spectral norm <= 1 (abstract:
+    'transitions that remain diagonal-plus-rank-one and non-expansive')."""
+    n, d = 10000, 8
+    k = RNG.standard_normal((n, d))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    alpha = RNG.uniform(-1, 1, (n, d))
+    alpha[: n // 10] = np.sign(alpha[: n // 10])          # include the orthogonal corner |alpha| = 1
+    beta = RNG.uniform(0, 2, n)
+    beta[: n // 20] = 2.0
+    A = _transitions_from_oracle(k, alpha, beta)
+    sv = np.linalg.svd(A, compute_uv=False)[:, 0]
+    assert sv.max() <= 1.0 + 1e-12
+    assert sv.max() >= 1.0 - 1e-9        # the bound is attained (reflection x sign gate)
+    # outside the extended range the bound fails, so the check has teeth
+    A_bad = _transitions_from_oracle(k[:2000], alpha[:2000], np.full(2000, 2.5))
+    assert np.linalg.svd(A_bad, compute_uv=False)[:, 0].max() > 1.0 + 1e-3
+
+
+def _rot(phi):
+    return np.array([[math.cos(phi), -math.sin(phi)], [math.sin(phi), math.cos(phi)]])
+
+
+@pytest.mark.parametrize("theta", [0.0, 0.3, 1.1, -2.0, math.pi / 4])
+def test_reflection_times_gate_is_exact_2d_rotation(theta):
+    """d_k = 2, alpha = (1,-1), beta = 2, k = (cos th, sin th): the delta-rule
+    reflection times the sign-flip gate is the rotation R(2 th + pi)
+    (abstract: 'realize 2D rotations by combining a single delta-rule
+    transformation with a second reflection supplied by its channel-wise
+    gate')."""
+    k = np.array([[math.cos(theta), math.sin(theta)]])
+    A = _transitions_from_oracle(k, np.array([[1.0, -1.0]]), np.array([2.0]))[0]
+    np.testing.assert_allclose(A, _rot(2 * theta + math.pi), atol=1e-15)
+    np.testing.assert_allclose(A @ A.T, np.eye(2), atol=1e-15)
+    assert abs(np.linalg.det(A) - 1.0) < 1e-15
+    # many steps with v = 0: S_T = R(T (2 th + pi)) S_0
+    T = 37
+    s0 = RNG.standard_normal((1, 1, 2, 3))
+    z2 = np.zeros((1, T, 1, 2))
+    z3 = np.zeros((1, T, 1, 3))
+    kk = np.broadcast_to(k, (1, T, 1, 2)).copy()
+    al = np.broadcast_to([1.0, -1.0], (1, T, 1, 2)).copy()
+    _, sf = oracle.recurrence_arrays("kda", z2, kk, z3, al, np.full((1, T, 1), 2.0), None, None, s0)
+    np.testing.assert_allclose(sf[0, 0], _rot(T * (2 * theta + math.pi)) @ s0[0, 0], atol=1e-12)
+
+
+def test_no_erase_no_decay_keeps_state():
+    """beta = 0 and alpha = 1: S_t = S_0 and o_t = S_0^T q_t."""
+    inp = _small("kda", 21, init="random")
+    inp.alpha = torch.ones_like(inp.alpha)
+    inp.g1 = torch.zeros_like(inp.g1)
+    o, sf = oracle.recurrence(inp)
+    s0 = inp.initial_state.double().numpy()
+    np.testing.assert_allclose(sf, s0, atol=0)
+    ref = np.einsum("bthi,bhij->bthj", inp.q.double().numpy(), s0)
+    np.testing.assert_allclose(o, ref, atol=1e-13)
+
+
+def test_rda_without_erase_is_causal_linear_attention():
+    """RDA with e = 0 and alpha = 1 is plain causal linear attention:
+    o = ((Q K^T) (.) causal mask (.) w) V + Q S_0, a dense-matrix formula."""
+    inp = _small("rda", 31, B=1, T=23, H=2, dk=6, dv=4)
+    inp.alpha = torch.ones_like(inp.alpha)
+    inp.g1 = torch.zeros_like(inp.g1)
+    o, _ = oracle.recurrence(inp)
+    for h in range(inp.H):
+        Q, K, V = (x[0, :, h].double().numpy() for x in (inp.q, inp.k, inp.v))
+        w = inp.g2[0, :, h].double().numpy()
+        L = np.tril(Q @ K.T) * w[None, :]
+        ref = L @ V + Q @ inp.initial_state[0, h].double().numpy()
+        np.testing.assert_allclose(o[0, :, h], ref, atol=1e-12)
+
+
+def test_rda_without_erase_is_gated_linear_attention():
+    """RDA with e = 0: gated linear attention with channel-wise decay (the
+    Lightning-style recurrence without the v - Sk correction):
+    o_t = sum_{s<=t} w_s sum_c q_tc (prod_{s<r<=t} alpha_rc) k_sc v_s
+          + sum_c q_tc (prod_{r<=t} alpha_rc) S_0[c,:]."""
+    inp = _small("rda", 41, B=1, T=12, H=1, dk=5, dv=3, gate_range="extended")
+    inp.g1 = torch.zeros_like(inp.g1)
+    o, _ = oracle.recurrence(inp)
+    Q, K, V, Al = (x[0, :, 0].double().numpy() for x in (inp.q, inp.k, inp.v, inp.alpha))
+    w = inp.g2[0, :, 0].double().numpy()
+    S0 = inp.initial_state[0, 0].double().numpy()
+    T = Q.shape[0]
+    for t in range(T):
+        acc = np.zeros(V.shape[1])
+        for s in range(t + 1):
+            lam = np.prod(Al[s + 1:t + 1], axis=0) if t > s else np.ones(K.shape[1])
+            acc += w[s] * np.sum(Q[t] * lam * K[s]) * V[s]
+        acc += (Q[t] * np.prod(Al[:t + 1], axis=0)) @ S0
+        np.testing.assert_allclose(o[0, t, 0], acc, atol=1e-12)
+
+
+def test_unit_erase_on_one_hot_key_overwrites_row():
+    """beta = 1, alpha = 1, k = e_i: row i of the state is replaced by v_t
+    exactly, other rows untouched (the notebook analogy on the openarchlab
+    page: erase the old number on that line, then write the new one)."""
+    dk, dv, T = 6, 4, 5
+    s0 = RNG.standard_normal((1, 1, dk, dv))
+    idx = [2, 0, 2, 5, 3]
+    k = np.zeros((1, T, 1, dk))
+    for t, i in enumerate(idx):
+        k[0, t, 0, i] = 1.0
+    v = RNG.standard_normal((1, T, 1, dv))
+    S = s0[0, 0].copy()
+    for t in range(T):
+        _, sf = oracle.recurrence_arrays("kda", np.zeros((1, t + 1, 1, dk)), k[:, :t + 1], v[:, :t + 1],
+                                         np.ones((1, t + 1, 1, dk)), np.ones((1, t + 1, 1)), None, None, s0)
+        S[idx[t]] = v[0, t, 0]
+        np.testing.assert_allclose(sf[0, 0], S, atol=1e-15)
+
+
+def test_householder_reflection_preserves_frobenius_norm():
+    """beta = 2, alpha = 1, v = 0: each step applies I - 2 k k^T (unit k), an
+    orthogonal reflection, so ||S_t||_F = ||S_0||_F."""
+    dk, dv, T = 7, 5, 40
+    k = RNG.standard_normal((1, T, 1, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    s0 = RNG.standard_normal((1, 1, dk, dv))
+    _, sf = oracle.recurrence_arrays("kda", np.zeros((1, T, 1, dk)), k, np.zeros((1, T, 1, dv)),
+                                     np.ones((1, T, 1, dk)), np.full((1, T, 1), 2.0), None, None, s0)
+    assert abs(np.linalg.norm(sf) - np.linalg.norm(s0)) < 1e-12
+
+
+def test_zero_gate_erases_channel_exactly():
+    """alpha_t = 0 wipes the decayed state, so S_t = k_t m_t^T exactly
+    (u = m because S' = 0)."""
+    inp = _small("gdn2", 51, B=1, T=4, H=1, dk=5, dv=3)
+    inp.alpha[0, -1] = 0.0
+    _, sf = oracle.recurrence(inp)
+    k = inp.k[0, -1, 0].double().numpy()
+    m = inp.g2[0, -1, 0].double().numpy() * inp.v[0, -1, 0].double().numpy()
+    np.testing.assert_array_equal(sf[0, 0], np.outer(k, m))
+
+
+def test_state_continuation_and_varlen_packing():
+    """Running [0,t) then [t,T) from the carried state equals [0,T); packing
+    documents with cu_seqlens equals running them separately (document reset,
+    openarchlab page sec. 3)."""
+    inp = _small("rda", 61, B=1, T=20, H=3, dk=4, dv=5, gate_range="extended")
+    o, sf = oracle.recurrence(inp)
+    t = 7
+    a = [x[:, :t] for x in (inp.q, inp.k, inp.v, inp.alpha, inp.g1, inp.g2)]
+    b = [x[:, t:] for x in (inp.q, inp.k, inp.v, inp.alpha, inp.g1, inp.g2)]
+    oa, sa = oracle.recurrence_arrays("rda", *a, None, inp.initial_state)
+    ob, sb = oracle.recurrence_arrays("rda", *b, None, sa)
+    assert np.array_equal(np.concatenate([oa, ob], axis=1), o) and np.array_equal(sb, sf)
+    # varlen: three documents packed along T
+    lens = [5, 1, 9]
+    pk = make_chunk_inputs("gdn2", "extended", "f32", H=2, d_k=4, d_v=3, seed=71, doc_lens=lens,
+                           init_state="random", init_std=0.3)
+    o_p, s_p = oracle.recurrence(pk)
+    start = 0
+    for n, ln in enumerate(lens):
+        parts = [x[:, start:start + ln] for x in (pk.q, pk.k, pk.v, pk.alpha, pk.g1, pk.g2)]
+        o_n, s_n = oracle.recurrence_arrays("gdn2", *parts, None, pk.initial_state[n:n + 1])
+        assert np.array_equal(o_p[:, start:start + ln], o_n)
+        assert np.array_equal(s_p[n], s_n[0])
+        start += ln
+
+
+def test_sampled_restriction_matches_full_run():
+    pk = make_chunk_inputs("kda", "extended", "f32", H=3, d_k=4, d_v=3, seed=81, doc_lens=[4, 7, 2],
+                           init_state="random")
+    o, sf = oracle.recurrence(pk)
+    o_d, s_d = oracle.recurrence(pk, seqs=[2, 0], heads=[1, 2])
+    cu = pk.cu_seqlens.numpy()
+    for (n, h), on in o_d.items():
+        np.testing.assert_array_equal(on, o[0, cu[n]:cu[n + 1], h])
+        np.testing.assert_array_equal(s_d[(n, h)], sf[n, h])
+
+
+def test_tiny_ckda_inputs_match_recipe():
+    """The tiny Complex-KDA workload: shapes, ranges and unit-norm keys."""
+    inp = tiny_ckda()
+    assert tuple(inp.q.shape) == (1, 64, 2, 16) and inp.chunk_size == 16
+    assert inp.q.dtype == torch.float32 and inp.initial_state is None
+    assert float(inp.alpha.min()) >= -1 and float(inp.alpha.max()) <= 1 and float(inp.alpha.min()) < 0
+    assert float(inp.g1.min()) >= 0 and float(inp.g1.max()) <= 2 and float(inp.g1.max()) > 1
+    np.testing.assert_allclose(inp.k.double().norm(dim=-1).numpy(), 1.0, atol=1e-6)
