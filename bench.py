@@ -1,0 +1,460 @@
+"""Benchmark of the gated delta-rule recurrence on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--extra]
+
+A step is one pass of the hot path over one batch of synthetic input: one
+chunked forward (``kda_chunk_fwd``) over the KDA-range bf16 workload
+B=4, H=16, T=4096, d_k=d_v=128, chunk 64 (seeded inputs, resident in HBM).
+The single-token decode step (256 x 32 heads, d=128, fp32 state 512 MiB in
+place, Complex-KDA range) is timed in the same run and reported under
+"decode".  With --extra the Complex-KDA 8x16x8192 and the RDA / GDN-2 varlen
+workloads are timed too (under "also").
+
+Multi-GPU (torchrun): every rank runs its own independent batch (different
+seed): the work shards over (sequence, head) units with no collective on the
+data path, so scaling is weak; ranks only meet at barriers and at the final
+max-over-ranks of the device times.
+
+Rank 0 prints one JSON line.  All device times come from CUDA events on the
+launching stream; clocks are sampled with nvidia-smi during the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "chunked fwd tokens/s & % tensor-core peak; decode step HBM GB/s (1×B200)"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work per workload (bytes and flops the path must move / do)
+# ---------------------------------------------------------------------------
+
+def chunk_algorithmic(inp) -> dict:
+    """Bytes: every input read once, o written once, states read/written once.
+    Flops: WY chunk form per head-token, triangles counted as half:
+    6*dk*dv + 2*C*(dk+dv) + C^2/3."""
+    head_tokens = inp.B * inp.T * inp.H
+    C, dk, dv = inp.chunk_size, inp.d_k, inp.d_v
+    in_bytes = inp.nbytes()
+    o_bytes = inp.B * inp.T * inp.H * dv * inp.q.element_size()
+    n_states = inp.num_seqs * inp.H
+    state_bytes = n_states * dk * dv * 4 * (2 if inp.initial_state is not None else 1)
+    flops = head_tokens * (6 * dk * dv + 2 * C * (dk + dv) + C * C / 3.0)
+    return {"bytes": in_bytes + o_bytes + state_bytes, "flops": flops, "head_tokens": head_tokens,
+            "tokens": inp.B * inp.T}
+
+
+def decode_algorithmic(N, H, dk, dv, elem=2, variant="kda") -> dict:
+    state = 2 * N * H * dk * dv * 4
+    per_head_in = (3 * dk + dv) * elem + (elem if variant != "gdn2" else (dk + dv) * elem)
+    if variant == "rda":
+        per_head_in += elem
+    io = N * H * (per_head_in + dv * elem)
+    return {"bytes": state + io, "flops": N * H * 7 * dk * dv, "tokens": N}
+
+
+# ---------------------------------------------------------------------------
+# Device helpers
+# ---------------------------------------------------------------------------
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.25)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# Timed regions
+# ---------------------------------------------------------------------------
+
+def time_launches(fn, steps: int, warmup: int, world: int, stream):
+    """W untimed steps, then K steps bracketed by barrier + synchronize; per-launch
+    CUDA events on the launching stream.  Returns (total_s, per_launch_s list)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start_all = torch.cuda.Event(enable_timing=True)
+    end_all = torch.cuda.Event(enable_timing=True)
+    start_all.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        fn()
+        ev[i][1].record(stream)
+    end_all.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total = start_all.elapsed_time(end_all) / 1e3
+    per = [a.elapsed_time(b) / 1e3 for a, b in ev]
+    return total, per
+
+
+def pct(xs, p):
+    return float(np.percentile(np.asarray(xs), p))
+
+
+def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True):
+    import linear_rnn_delta_b200 as kda
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    d = {n: (None if getattr(inp, n) is None else getattr(inp, n).to(dev)) for n in
+         ("q", "k", "v", "alpha", "g1", "g2")}
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.to(dev)
+    s0 = None if inp.initial_state is None else inp.initial_state.to(dev)
+    N = inp.num_seqs
+    o = torch.empty((inp.B, inp.T, inp.H, inp.d_v), dtype=d["q"].dtype, device=dev)
+    sf = torch.empty((N, inp.H, inp.d_k, inp.d_v), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.kda_chunk_fwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"],
+                          cu_seqlens=cu, initial_state=s0, final_state=sf, o=o, chunk_size=inp.chunk_size,
+                          stream=stream)
+
+    if sampler:
+        sampler.start()
+    total, per = time_launches(step, steps, warmup, world, stream)
+    clocks = sampler.stop() if sampler else None
+    total = max_over_ranks(total, world)
+    alg = chunk_algorithmic(inp)
+    avg = sum(per) / len(per)
+    res = {"tokens_per_step": alg["tokens"], "total_s": total, "avg_launch_s": avg,
+           "p50_ms": pct(per, 50) * 1e3, "p95_ms": pct(per, 95) * 1e3, "p99_ms": pct(per, 99) * 1e3,
+           "alg": alg, "clocks": clocks}
+    gbs = alg["bytes"] / avg / 1e9
+    tfs = alg["flops"] / avg / 1e12
+    res["hbm"] = {"achieved": gbs, "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"]}
+    res["tensor"] = {"achieved": tfs, "peak": peaks["bf16_tflops"], "frac": tfs / peaks["bf16_tflops"]}
+    if e2e:
+        res["e2e"] = chunk_e2e(inp, d, cu, s0, o, sf, steps, warmup, world, stream)
+    return res
+
+
+def chunk_e2e(inp, d, cu, s0, o, sf, steps, warmup, world, stream):
+    """Same step through the public API with pinned host buffers: H2D of the
+    step's inputs, the kernel, D2H of o and the final state, all timed."""
+    import linear_rnn_delta_b200 as kda
+    host = {n: (None if getattr(inp, n) is None else getattr(inp, n).pin_memory()) for n in
+            ("q", "k", "v", "alpha", "g1", "g2")}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    sf_h = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = o.numel() * o.element_size() + sf.numel() * sf.element_size()
+
+    def step():
+        for n, t in host.items():
+            if t is not None:
+                d[n].copy_(t, non_blocking=True)
+        kda.kda_chunk_fwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"],
+                          cu_seqlens=cu, initial_state=s0, final_state=sf, o=o, chunk_size=inp.chunk_size,
+                          stream=stream)
+        o_h.copy_(o, non_blocking=True)
+        sf_h.copy_(sf, non_blocking=True)
+
+    total, _ = time_launches(step, steps, max(1, warmup), world, stream)
+    total = max_over_ranks(total, world)
+    return {"total_s": total, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_decode_workload(steps, warmup, world, peaks, rank, N=256, H=32, dk=128, dv=128, e2e=True):
+    import linear_rnn_delta_b200 as kda
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    state = W.decode_initial_state(N, H, dk, dv, seed=rank).to(dev)
+    n_inputs = 8   # distinct per-step inputs cycled through the timed steps
+    inputs = []
+    for s in range(n_inputs):
+        st = W.decode_step_inputs(s, "kda", "extended", "bf16", N, H, dk, dv, seed=rank)
+        inputs.append([None if t is None else t.to(dev) for t in (st.q, st.k, st.v, st.alpha, st.g1, st.g2)])
+    o = torch.empty((N, H, dv), dtype=torch.bfloat16, device=dev)
+    it = [0]
+
+    def step():
+        x = inputs[it[0] % n_inputs]
+        it[0] += 1
+        kda.kda_decode_step("kda", "extended", *x, state, o=o, stream=stream)
+
+    total, per = time_launches(step, steps, warmup, world, stream)
+    total = max_over_ranks(total, world)
+    alg = decode_algorithmic(N, H, dk, dv)
+    avg = sum(per) / len(per)
+    gbs = alg["bytes"] / avg / 1e9
+    res = {"value": N * world * steps / total, "unit": "tokens/s", "workload":
+           f"decode Complex-KDA N={N} H={H} d_k=d_v={dk} fp32 state in place, bf16 inputs",
+           "ms_per_step": total / steps * 1e3, "p50_ms": pct(per, 50) * 1e3, "p95_ms": pct(per, 95) * 1e3,
+           "p99_ms": pct(per, 99) * 1e3,
+           "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                        "peak_source": peaks["source"]},
+           "bytes_per_step": alg["bytes"], "gpu_launches": steps}
+    if e2e:
+        host = [None if t is None else t.cpu().pin_memory() for t in inputs[0]]
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host if t is not None)
+
+        def step_e2e():
+            x = inputs[0]
+            for dst, src in zip(x, host):
+                if src is not None:
+                    dst.copy_(src, non_blocking=True)
+            kda.kda_decode_step("kda", "extended", *x, state, o=o, stream=stream)
+            o_h.copy_(o, non_blocking=True)
+
+        tot_e2e, _ = time_launches(step_e2e, steps, warmup, world, stream)
+        tot_e2e = max_over_ranks(tot_e2e, world)
+        res["e2e"] = {"value": N * world * steps / tot_e2e, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": o.numel() * o.element_size()}
+    return res
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(inp, target_s=12.0, threads=0):
+    """Tokens/s of the float64 oracle on a bounded sample of the workload:
+    whole sequences of a few heads, scaled to the metric's unit (a token is a
+    position of the batch across all H heads)."""
+    import oracle
+    cores = threads or oracle.max_threads()
+    pairs = []
+    n_seq, H = inp.num_seqs, inp.H
+    # one head first, to size the sample
+    t0 = time.perf_counter()
+    oracle.recurrence(inp, seqs=[0], heads=[0], threads=1)
+    one = max(time.perf_counter() - t0, 1e-4)
+    per_head_tokens = inp.seq_bounds(0)[2]
+    n_pairs = int(max(1, min(n_seq * H, (target_s * cores) / one)))
+    rng = np.random.default_rng(0)
+    flat = rng.permutation(n_seq * H)[:n_pairs]
+    pairs = sorted({(int(f) // H, int(f) % H) for f in flat})
+    seqs = sorted({n for n, _ in pairs})
+    heads = sorted({h for _, h in pairs})
+    t0 = time.perf_counter()
+    oracle.recurrence(inp, seqs=seqs, heads=heads, threads=threads)
+    dt = time.perf_counter() - t0
+    head_tokens = sum(inp.seq_bounds(n)[2] for n in seqs) * len(heads)
+    rate = head_tokens / inp.H / dt
+    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(seqs)} sequences x {len(heads)} heads of the workload ({head_tokens} head-tokens, "
+                      f"{dt:.1f} s float64 on {cores} host threads); tokens = head-tokens / H",
+            "seconds": dt, "single_head_s": one, "per_head_tokens": per_head_tokens}
+
+
+def reference_arm(args, world, rank):
+    """The oracle, as it stands, on the host cores: the same workload, metric and unit."""
+    if rank != 0:
+        return
+    inp = W.kda_bf16(0)
+    rates = []
+    samples = None
+    # each step is a bounded sample of the workload; sized so the whole run ends within minutes
+    per_step_target = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample_rate(inp, target_s=per_step_target)
+        if i >= args.warmup:
+            rates.append(r["value"])
+            samples = r
+    value = statistics.median(rates)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": inp.B * inp.T / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded numpy, cast to bf16; the oracle reads the same values in float64)",
+            "config": {"workload": "KDA-range chunked forward B=4 H=16 T=4096 d_k=d_v=128 chunk=64 bf16",
+                       "global_batch": inp.B, "seq_len": inp.T, "heads": inp.H, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples["cores"], "kind": "oracle",
+                             "sample": samples["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--extra", action="store_true", help="also time Complex-KDA 8x16x8192 and varlen RDA/GDN-2")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=200)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world, rank, local = dist_setup() if args.impl == "ours" else (int(os.environ.get("WORLD_SIZE", "1")),
+                                                                   int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        reference_arm(args, world, rank)
+        return
+
+    import linear_rnn_delta_b200  # noqa: F401  (fails loudly if the library is missing)
+    peaks = load_peaks()
+    inp = W.kda_bf16(seed=rank)
+    sampler = ClockSampler(local) if rank == 0 else None
+    main_res = run_chunk_workload(inp, args.steps, args.warmup, world, peaks, sampler=sampler)
+    decode = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank)
+    also = []
+    if args.extra:
+        for name, mk in (("Complex-KDA chunked forward B=8 H=16 T=8192 d=128 chunk=64 bf16", lambda: W.ckda_bf16(rank)),
+                         ("RDA varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("rda", rank)),
+                         ("GDN-2 varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("gdn2", rank))):
+            x = mk()
+            r = run_chunk_workload(x, max(5, args.steps // 2), args.warmup, world, peaks, e2e=False)
+            also.append({"workload": name, "value": r["tokens_per_step"] * world * max(5, args.steps // 2) / r["total_s"],
+                         "unit": UNIT, "ms_per_step": r["avg_launch_s"] * 1e3, "hbm_frac": r["hbm"]["frac"],
+                         "tensor_frac": r["tensor"]["frac"], "achieved_gbs": r["hbm"]["achieved"],
+                         "achieved_tflops": r["tensor"]["achieved"]})
+            del x
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample_rate(inp)
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    tokens = main_res["tokens_per_step"] * world
+    value = tokens * args.steps / main_res["total_s"]
+    e2e = main_res["e2e"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": main_res["total_s"] / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded numpy draws, bf16; per-rank seed)",
+        "config": {"workload": "KDA-range chunked forward B=4 H=16 T=4096 d_k=d_v=128 chunk=64 bf16, "
+                               "fp32 state, zero initial state",
+                   "global_batch": inp.B * world, "seq_len": inp.T, "heads": inp.H, "parallelism": f"dp{world}",
+                   "l2": f"inputs {inp.nbytes() / 1e6:.0f} MB > L2 126 MB, no flush"},
+        "p50_ms": main_res["p50_ms"], "p95_ms": main_res["p95_ms"], "p99_ms": main_res["p99_ms"],
+        "roofline": {"bound": "hbm", "achieved": main_res["hbm"]["achieved"], "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": main_res["hbm"]["frac"], "traffic": None,
+                     "peak_source": peaks["source"],
+                     "kernel": "kda_chunk_fwd (one launch per step)",
+                     "alg_bytes_per_launch": main_res["alg"]["bytes"]},
+        "tensor": {"achieved": main_res["tensor"]["achieved"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                   "frac": main_res["tensor"]["frac"], "alg_flops_per_launch": main_res["alg"]["flops"]},
+        "e2e": {"value": tokens * args.steps / e2e["total_s"], "unit": UNIT,
+                "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]},
+        "gpu_launches": args.steps,
+        "clocks": main_res["clocks"],
+        "decode": decode,
+        "cpu_baseline": cpu and {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+    }
+    if also:
+        line["also"] = also
+    print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

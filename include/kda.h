@@ -1,0 +1,143 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) library for the gated delta-rule
+ * recurrence with channel-wise decay: KDA, Complex KDA, RDA and GDN-2.
+ *
+ * The operation (update equations on the Raon-1-mini-preview discussion page,
+ * range extension in the "Complex KDA" arXiv abstract).  For each sequence n,
+ * head h and token t, with the state S in R^{d_k x d_v} (rows = key channel):
+ *
+ *   KDA / Complex KDA : S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   RDA               : S_t = (I - e_t k_t k_t^T) Diag(alpha_t) S_{t-1} + w_t k_t v_t^T
+ *   GDN-2             : S_t = (I - k_t (b_t (.) k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t (.) v_t)^T
+ *   readout           : o_t = S_t^T q_t     (post-update state, no scaling; a
+ *                                            caller wanting 1/sqrt(d_k) pre-scales q)
+ *
+ * KDA range: alpha in (0,1], beta in [0,1].  Complex KDA (KDA_RANGE_EXTENDED):
+ * alpha in [-1,1], beta in [0,2].  The kernels never take a logarithm of
+ * alpha and never divide by a product of alphas, so negative and zero gates
+ * are computed exactly as the recurrence defines them; the range argument
+ * only declares the caller's contract.
+ *
+ * Memory model.  Every tensor pointer is a DEVICE pointer owned by the
+ * caller, 16-byte aligned, densely packed in the row-major layouts below.
+ * The library allocates no device memory, never frees caller memory, keeps
+ * no state between calls (it is reentrant and thread-safe) and enqueues all
+ * work asynchronously on `stream` (a cudaStream_t; NULL = legacy default
+ * stream).  A call returns after the launch: asynchronous kernel faults
+ * surface at the caller's next synchronisation, as with any CUDA launch.
+ *
+ * Errors.  Every entry point validates all arguments on the host before it
+ * launches anything; on a bad argument it returns a KDA_ERR_* code and has
+ * no side effect.  A failed launch returns KDA_ERR_CUDA (detail in
+ * kda_last_error_detail()).
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Variants: which erase direction a~ and written value m the update uses.
+ *   KDA  : a~ = beta k,  m = beta v      g1 = beta [..,H],      g2 = NULL
+ *   RDA  : a~ = e k,     m = w v         g1 = e    [..,H],      g2 = w [..,H]
+ *   GDN2 : a~ = b (.) k, m = w (.) v     g1 = b    [..,H,d_k],  g2 = w [..,H,d_v]  */
+enum kda_variant { KDA_VARIANT_KDA = 0, KDA_VARIANT_RDA = 1, KDA_VARIANT_GDN2 = 2 };
+
+/* Declared gate range (not clamped; kda_check_gates tests inputs against it). */
+enum kda_gate_range {
+    KDA_RANGE_STANDARD = 0, /* alpha in (0,1], beta/e in [0,1]    (KDA)          */
+    KDA_RANGE_EXTENDED = 1  /* alpha in [-1,1], beta/e in [0,2]   (Complex KDA)  */
+};
+
+/* Element type of q, k, v, alpha, g1, g2 and o.  States are always fp32. */
+enum kda_dtype { KDA_DTYPE_BF16 = 0, KDA_DTYPE_F32 = 1 };
+
+enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_seqlens */
+    KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dims, chunk size) */
+    KDA_ERR_RANGE = 3,         /* reserved: a gate outside the declared range */
+    KDA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed */
+};
+
+/* Flags.  (Gate ranges are checked on request by kda_check_gates, which
+ * writes its verdict to caller memory; the forward calls never check them.) */
+#define KDA_FLAG_FORCE_SCAN     2u  /* use the token-by-token CUDA scan kernel even where the
+                                       tensor-core chunked kernel applies (testing aid) */
+
+/*
+ * kda_chunk_fwd -- chunked-parallel forward over whole sequences.
+ *
+ * Shapes (row-major):
+ *   q, k, alpha : [B,T,H,d_k]        v, o : [B,T,H,d_v]
+ *   g1, g2      : per the variant table above, leading dims [B,T,H]
+ *   cu_seqlens  : NULL -> B independent sequences of length T (N = B);
+ *                 else int32 DEVICE array of num_seqs+1 non-decreasing offsets
+ *                 with cu[0] = 0 and cu[num_seqs] = T, B must be 1, and
+ *                 sequence n is tokens [cu[n], cu[n+1]) of the packed batch.
+ *                 Each sequence starts from its own initial state ("document
+ *                 reset", openarchlab page on GDN/KDA state updates, sec. 3);
+ *                 there is no padding inside packed input.
+ *   initial_state : [N,H,d_k,d_v] fp32 or NULL (zero state)
+ *   final_state   : [N,H,d_k,d_v] fp32 or NULL (not written); may alias
+ *                   initial_state (each sequence reads its state before writing it)
+ *   o             : [B,T,H,d_v] output, same dtype as q
+ * Sizes: B >= 1, T >= 0, H >= 1, d_k and d_v in {16, 32, 64, 128},
+ * chunk_size in {16, 32, 64, 128}.  With bf16, d_k = d_v = 128 and
+ * chunk_size = 64 the tcgen05 tensor-core chunked kernel runs (WY/UT form,
+ * fp32 accumulation, fp32 state kept on chip); every other accepted case
+ * runs the token-by-token fp32 CUDA scan, whose result does not depend on
+ * chunk_size.  Results of the two agree to rounding.
+ * Returns KDA_OK or a KDA_ERR_* code.
+ */
+int kda_chunk_fwd(int variant, int gate_range, int dtype,
+                  int B, int T, int H, int d_k, int d_v,
+                  const void *q, const void *k, const void *v, const void *alpha,
+                  const void *g1, const void *g2,
+                  const int32_t *cu_seqlens, int num_seqs,
+                  const float *initial_state, float *final_state,
+                  void *o, int chunk_size, unsigned flags, void *stream);
+
+/*
+ * kda_decode_step -- one recurrent step for N sequences (single-token decode;
+ * the fixed-size state of the openarchlab page, sec. 1 and 3).
+ *
+ *   q, k, alpha : [N,H,d_k]     v, o : [N,H,d_v]     g1, g2 : per variant, [N,H](,d)
+ *   state       : [N,H,d_k,d_v] fp32, read and overwritten IN PLACE with S_t
+ *   o           : [N,H,d_v] = S_t^T q_t, same dtype as q
+ * Sizes: N >= 1, H >= 1, d_k and d_v in {16, 32, 64, 128}.
+ * The state is streamed once (read, update, write).  Returns KDA_OK or KDA_ERR_*.
+ */
+int kda_decode_step(int variant, int gate_range, int dtype,
+                    int N, int H, int d_k, int d_v,
+                    const void *q, const void *k, const void *v, const void *alpha,
+                    const void *g1, const void *g2,
+                    float *state, void *o, unsigned flags, void *stream);
+
+/*
+ * kda_check_gates -- count gates outside the declared range on the device.
+ * Checks alpha [n_tok*d_k] against the range's alpha interval and g1 (beta/e,
+ * n_tok values; GDN-2 b, n_tok*d_k values, against [0, 2] for the extended
+ * range and [0, 1] otherwise).  Writes the count of violations to the device
+ * int `d_count` (caller-owned, overwritten).  NaN counts as a violation.
+ */
+int kda_check_gates(int variant, int gate_range, int dtype, long long n_tok, int d_k,
+                    const void *alpha, const void *g1, int *d_count, void *stream);
+
+/* Static description of a status code (never NULL). */
+const char *kda_error_string(int code);
+
+/* Detail of the last KDA_ERR_CUDA / KDA_ERR_INVALID_ARG on the calling thread. */
+const char *kda_last_error_detail(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,216 @@
+"""B200 (sm_100a) library for the gated delta-rule recurrence with channel-wise
+decay: KDA, Complex KDA, RDA and GDN-2.
+
+This module is a thin ctypes binding over the C ABI in ``include/kda.h``
+(``libkda.so``, built in-tree by ``python -m linear_rnn_delta_b200.build``).
+It only marshals arguments: it reads shapes and device pointers off torch
+tensors, picks the caller's current CUDA stream, and allocates outputs the
+caller did not pass.  Every step of the recurrence runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback, and importing this module
+fails if the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Union
+
+import torch
+
+__all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_version",
+           "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_FORCE_SCAN"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+
+VARIANTS = {"kda": 0, "rda": 1, "gdn2": 2}
+RANGES = {"standard": 0, "extended": 1}
+_DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+FLAG_FORCE_SCAN = 2
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_rnn_delta_b200.build` "
+                          "(the recurrence has no implementation other than its CUDA kernels)")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.kda_chunk_fwd.restype = _i
+    lib.kda_chunk_fwd.argtypes = [_i] * 8 + [_vp] * 6 + [_vp, _i, _vp, _vp, _vp, _i, ctypes.c_uint, _vp]
+    lib.kda_decode_step.restype = _i
+    lib.kda_decode_step.argtypes = [_i] * 7 + [_vp] * 6 + [_vp, _vp, ctypes.c_uint, _vp]
+    lib.kda_check_gates.restype = _i
+    lib.kda_check_gates.argtypes = [_i, _i, _i, ctypes.c_longlong, _i, _vp, _vp, _vp, _vp]
+    lib.kda_error_string.restype = ctypes.c_char_p
+    lib.kda_error_string.argtypes = [_i]
+    lib.kda_last_error_detail.restype = ctypes.c_char_p
+    lib.kda_last_error_detail.argtypes = []
+    lib.kda_version.restype = _i
+    lib.kda_version.argtypes = []
+    return lib
+
+
+lib = _load()
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        detail = lib.kda_last_error_detail().decode(errors="replace")
+        super().__init__(f"{where}: {lib.kda_error_string(code).decode()} -- {detail}")
+
+
+def kda_error_string(code: int) -> str:
+    return lib.kda_error_string(int(code)).decode()
+
+
+def kda_version() -> int:
+    return int(lib.kda_version())
+
+
+def _code(table, x, what):
+    if isinstance(x, str):
+        if x not in table:
+            raise ValueError(f"unknown {what} {x!r}; expected one of {sorted(table)}")
+        return table[x]
+    return int(x)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else _vp(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return _vp(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(t: Optional[torch.Tensor], name: str, dtype, shape, device):
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torch.Tensor, k: torch.Tensor,
+                  v: torch.Tensor, alpha: torch.Tensor, g1: torch.Tensor, g2: Optional[torch.Tensor] = None,
+                  cu_seqlens: Optional[torch.Tensor] = None, initial_state: Optional[torch.Tensor] = None,
+                  final_state: Union[torch.Tensor, bool, None] = True, o: Optional[torch.Tensor] = None,
+                  chunk_size: int = 64, flags: int = 0, stream=None):
+    """Chunked forward of the recurrence over whole sequences (C: kda_chunk_fwd).
+
+    q, k, alpha [B,T,H,d_k]; v [B,T,H,d_v]; g1/g2 per variant (KDA: beta
+    [B,T,H], g2 None; RDA: e, w [B,T,H]; GDN-2: b [B,T,H,d_k], w [B,T,H,d_v]);
+    cu_seqlens int32 [N+1] (B == 1) or None; initial_state fp32 [N,H,d_k,d_v]
+    or None.  ``final_state`` True allocates it, a tensor is written in place,
+    None/False skips it.  Returns (o, final_state or None).
+    """
+    var = _code(VARIANTS, variant, "variant")
+    rng = _code(RANGES, gate_range, "gate_range")
+    if q.dim() != 4:
+        raise ValueError("q must be [B,T,H,d_k]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"dtype {dt} unsupported (bf16 or fp32)")
+    _check(q, "q", dt, (B, T, H, dk), dev)
+    _check(k, "k", dt, (B, T, H, dk), dev)
+    _check(v, "v", dt, (B, T, H, dv), dev)
+    _check(alpha, "alpha", dt, (B, T, H, dk), dev)
+    if var == 2:
+        _check(g1, "g1 (b)", dt, (B, T, H, dk), dev)
+        _check(g2, "g2 (w)", dt, (B, T, H, dv), dev)
+    else:
+        _check(g1, "g1", dt, (B, T, H), dev)
+        if var == 1:
+            _check(g2, "g2 (w)", dt, (B, T, H), dev)
+    if var != 0 and g2 is None:
+        raise ValueError("RDA and GDN-2 need g2 (write gate)")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    _check(initial_state, "initial_state", torch.float32, (N, H, dk, dv), dev)
+    if final_state is True:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    elif final_state is False:
+        final_state = None
+    _check(final_state, "final_state", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _check(o, "o", dt, (B, T, H, dv), dev)
+    rc = lib.kda_chunk_fwd(var, rng, _DTYPES[dt], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                           _ptr(g1), _ptr(g2), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(final_state),
+                           _ptr(o), int(chunk_size), int(flags), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_chunk_fwd")
+    return o, final_state
+
+
+def kda_decode_step(variant: Union[str, int], gate_range: Union[str, int], q: torch.Tensor, k: torch.Tensor,
+                    v: torch.Tensor, alpha: torch.Tensor, g1: torch.Tensor, g2: Optional[torch.Tensor],
+                    state: torch.Tensor, o: Optional[torch.Tensor] = None, stream=None):
+    """One decode step for N sequences (C: kda_decode_step); ``state`` fp32
+    [N,H,d_k,d_v] is updated in place.  q, k, alpha [N,H,d_k]; v [N,H,d_v].
+    Returns o [N,H,d_v]."""
+    var = _code(VARIANTS, variant, "variant")
+    rng = _code(RANGES, gate_range, "gate_range")
+    if q.dim() != 3:
+        raise ValueError("q must be [N,H,d_k]")
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"dtype {dt} unsupported (bf16 or fp32)")
+    _check(q, "q", dt, (N, H, dk), dev)
+    _check(k, "k", dt, (N, H, dk), dev)
+    _check(v, "v", dt, (N, H, dv), dev)
+    _check(alpha, "alpha", dt, (N, H, dk), dev)
+    if var == 2:
+        _check(g1, "g1 (b)", dt, (N, H, dk), dev)
+        _check(g2, "g2 (w)", dt, (N, H, dv), dev)
+    else:
+        _check(g1, "g1", dt, (N, H), dev)
+        if var == 1:
+            _check(g2, "g2 (w)", dt, (N, H), dev)
+    if var != 0 and g2 is None:
+        raise ValueError("RDA and GDN-2 need g2 (write gate)")
+    _check(state, "state", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=dt, device=dev)
+    _check(o, "o", dt, (N, H, dv), dev)
+    rc = lib.kda_decode_step(var, rng, _DTYPES[dt], N, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                             _ptr(g1), _ptr(g2), _ptr(state), _ptr(o), 0, _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_decode_step")
+    return o
+
+
+def kda_check_gates(variant: Union[str, int], gate_range: Union[str, int], alpha: torch.Tensor,
+                    g1: torch.Tensor, stream=None) -> int:
+    """Number of gate values outside the declared range (C: kda_check_gates).
+    Synchronises the stream to read the count back."""
+    var = _code(VARIANTS, variant, "variant")
+    rng = _code(RANGES, gate_range, "gate_range")
+    dk = alpha.shape[-1]
+    n_tok = alpha.numel() // dk
+    dev = alpha.device
+    count = torch.empty((1,), dtype=torch.int32, device=dev)
+    st = _stream(stream, dev)
+    rc = lib.kda_check_gates(var, rng, _DTYPES[alpha.dtype], n_tok, dk, _ptr(alpha.contiguous()),
+                             _ptr(g1.contiguous()), _ptr(count), st)
+    if rc != 0:
+        raise KdaError(rc, "kda_check_gates")
+    return int(count.item())

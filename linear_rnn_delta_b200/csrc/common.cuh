@@ -1,0 +1,37 @@
+// Shared device helpers and internal launch declarations of the kda library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace kda {
+
+enum Variant { KDA = 0, RDA = 1, GDN2 = 2 };
+
+// Element loads/stores in the input dtype, arithmetic in fp32.
+__device__ __forceinline__ float ld_f32(const float *p) { return *p; }
+__device__ __forceinline__ float ld_f32(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void st_out(float *p, float x) { *p = x; }
+__device__ __forceinline__ void st_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+
+// Arguments shared by the forward kernels (device pointers, see include/kda.h).
+struct FwdArgs {
+    int variant;
+    int B, T, H, dk, dv;
+    const void *q, *k, *v, *alpha, *g1, *g2;
+    const int32_t *cu_seqlens;
+    int num_seqs;
+    const float *s0;
+    float *sf;
+    void *o;
+};
+
+// Internal launchers; each returns cudaSuccess or the launch error.
+cudaError_t launch_scan_fwd(const FwdArgs &a, bool bf16, cudaStream_t st);
+cudaError_t launch_decode_step(const FwdArgs &a, bool bf16, cudaStream_t st);
+cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st);
+cudaError_t launch_check_gates(int variant, int gate_range, bool bf16, long long n_tok, int dk,
+                               const void *alpha, const void *g1, int *d_count, cudaStream_t st);
+
+}  // namespace kda

@@ -1,0 +1,159 @@
+// C ABI of the kda library: host-side argument checks and kernel dispatch.
+// Declarations, layouts and error semantics: include/kda.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstdint>
+
+#include "../../include/kda.h"
+#include "common.cuh"
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+int fail(int code, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where)
+{
+    return fail(KDA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64 || c == 128; }
+
+// Checks shared by the forward and decode calls: enums, head dims, pointers.
+int check_common(int variant, int gate_range, int dtype, int d_k, int d_v,
+                 const void *q, const void *k, const void *v, const void *alpha,
+                 const void *g1, const void *g2, const void *o, bool need_data)
+{
+    if (variant < KDA_VARIANT_KDA || variant > KDA_VARIANT_GDN2)
+        return fail(KDA_ERR_INVALID_ARG, "variant %d is not KDA(0), RDA(1) or GDN2(2)", variant);
+    if (gate_range != KDA_RANGE_STANDARD && gate_range != KDA_RANGE_EXTENDED)
+        return fail(KDA_ERR_INVALID_ARG, "gate_range %d is not STANDARD(0) or EXTENDED(1)", gate_range);
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_F32)
+        return fail(KDA_ERR_INVALID_ARG, "dtype %d is not BF16(0) or F32(1)", dtype);
+    if (d_k < 1 || d_v < 1) return fail(KDA_ERR_INVALID_ARG, "head dims must be positive (d_k=%d, d_v=%d)", d_k, d_v);
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "head dims d_k=%d, d_v=%d: supported are 16, 32, 64, 128", d_k, d_v);
+    if (!need_data) return KDA_OK;
+    const void *ptrs[] = {q, k, v, alpha, g1, o};
+    const char *names[] = {"q", "k", "v", "alpha", "g1", "o"};
+    for (int i = 0; i < 6; ++i) {
+        if (!ptrs[i]) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+        if (!aligned16(ptrs[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+    }
+    if (variant != KDA_VARIANT_KDA) {
+        if (!g2) return fail(KDA_ERR_INVALID_ARG, "g2 (write gate) is NULL for RDA/GDN2");
+        if (!aligned16(g2)) return fail(KDA_ERR_INVALID_ARG, "g2 is not 16-byte aligned");
+    }
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
+                             int B, int T, int H, int d_k, int d_v,
+                             const void *q, const void *k, const void *v, const void *alpha,
+                             const void *g1, const void *g2,
+                             const int32_t *cu_seqlens, int num_seqs,
+                             const float *initial_state, float *final_state,
+                             void *o, int chunk_size, unsigned flags, void *stream)
+{
+    if (B < 1 || T < 0 || H < 1)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d (need B>=1, T>=0, H>=1)", B, T, H);
+    if ((unsigned long long)B * (unsigned long long)T * H * 128ull > (1ull << 46))
+        return fail(KDA_ERR_INVALID_ARG, "problem too large (B*T*H=%llu)", (unsigned long long)B * T * H);
+    int rc = check_common(variant, gate_range, dtype, d_k, d_v, q, k, v, alpha, g1, g2, o, T > 0);
+    if (rc != KDA_OK) return rc;
+    if (!chunk_ok(chunk_size))
+        return fail(KDA_ERR_UNSUPPORTED, "chunk_size %d: supported are 16, 32, 64, 128", chunk_size);
+    if (flags & ~KDA_FLAG_FORCE_SCAN) return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    int N = B;
+    if (cu_seqlens) {
+        if (B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (got B=%d)", B);
+        if (num_seqs < 1) return fail(KDA_ERR_INVALID_ARG, "num_seqs must be >= 1 with cu_seqlens (got %d)", num_seqs);
+        if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)
+            return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+        N = num_seqs;
+    }
+    if (initial_state && !aligned16(initial_state))
+        return fail(KDA_ERR_INVALID_ARG, "initial_state is not 16-byte aligned");
+    if (final_state && !aligned16(final_state))
+        return fail(KDA_ERR_INVALID_ARG, "final_state is not 16-byte aligned");
+
+    kda::FwdArgs a{variant, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens, N,
+                   initial_state, final_state, o};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    cudaError_t e;
+#ifdef KDA_WITH_SM100_CHUNK
+    if (bf16 && d_k == 128 && d_v == 128 && chunk_size == 64 && !(flags & KDA_FLAG_FORCE_SCAN))
+        e = kda::launch_chunk_fwd_sm100(a, st);
+    else
+#endif
+        e = kda::launch_scan_fwd(a, bf16, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd launch");
+    return KDA_OK;
+}
+
+extern "C" int kda_decode_step(int variant, int gate_range, int dtype,
+                               int N, int H, int d_k, int d_v,
+                               const void *q, const void *k, const void *v, const void *alpha,
+                               const void *g1, const void *g2,
+                               float *state, void *o, unsigned flags, void *stream)
+{
+    if (N < 1 || H < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes N=%d H=%d (need >= 1)", N, H);
+    int rc = check_common(variant, gate_range, dtype, d_k, d_v, q, k, v, alpha, g1, g2, o, true);
+    if (rc != KDA_OK) return rc;
+    if (!state) return fail(KDA_ERR_INVALID_ARG, "state is NULL");
+    if (!aligned16(state)) return fail(KDA_ERR_INVALID_ARG, "state is not 16-byte aligned");
+    if (flags) return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((unsigned long long)N * H > (1ull << 31) - 1)
+        return fail(KDA_ERR_INVALID_ARG, "N*H too large for one launch");
+    kda::FwdArgs a{variant, N, 1, H, d_k, d_v, q, k, v, alpha, g1, g2, nullptr, N, state, state, o};
+    cudaError_t e = kda::launch_decode_step(a, dtype == KDA_DTYPE_BF16, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
+    return KDA_OK;
+}
+
+extern "C" int kda_check_gates(int variant, int gate_range, int dtype, long long n_tok, int d_k,
+                               const void *alpha, const void *g1, int *d_count, void *stream)
+{
+    if (variant < KDA_VARIANT_KDA || variant > KDA_VARIANT_GDN2)
+        return fail(KDA_ERR_INVALID_ARG, "variant %d is not KDA(0), RDA(1) or GDN2(2)", variant);
+    if (gate_range != KDA_RANGE_STANDARD && gate_range != KDA_RANGE_EXTENDED)
+        return fail(KDA_ERR_INVALID_ARG, "gate_range %d is not STANDARD(0) or EXTENDED(1)", gate_range);
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_F32)
+        return fail(KDA_ERR_INVALID_ARG, "dtype %d is not BF16(0) or F32(1)", dtype);
+    if (n_tok < 0 || d_k < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes n_tok=%lld d_k=%d", n_tok, d_k);
+    if (!d_count) return fail(KDA_ERR_INVALID_ARG, "d_count is NULL");
+    if (n_tok > 0 && (!alpha || !g1)) return fail(KDA_ERR_INVALID_ARG, "alpha or g1 is NULL");
+    cudaError_t e = kda::launch_check_gates(variant, gate_range, dtype == KDA_DTYPE_BF16, n_tok, d_k,
+                                            alpha, g1, d_count, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_check_gates launch");
+    return KDA_OK;
+}
+
+extern "C" const char *kda_error_string(int code)
+{
+    switch (code) {
+    case KDA_OK: return "KDA_OK: success";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG: invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: valid but unsupported size or option";
+    case KDA_ERR_RANGE: return "KDA_ERR_RANGE: gate outside the declared range";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime or launch failure";
+    }
+    return "unknown kda status code";
+}
+
+extern "C" const char *kda_last_error_detail(void) { return g_detail; }
+
+extern "C" int kda_version(void) { return 100; }
