@@ -36,6 +36,15 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
+// 128-byte-swizzle variant (layout type 2).  K-major: rows 128 B apart,
+// SBO = 1024 (8-row atom), LBO unused (16).  MN-major: SBO = 1024 (8 K-rows),
+// LBO = byte stride between 64-element MN panels.  Atoms must be 1024-byte
+// aligned; a K step inside a K-major 128-byte row advances the start by 32 B.
+__device__ __forceinline__ uint64_t make_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo = 1024)
+{
+    return make_desc(saddr, lbo, sbo) | ((uint64_t)2 << 61);
+}
+
 // ---- instruction descriptor, kind::f16 with bf16 A/B and fp32 D -----------
 // bits 4-5 D fmt (1 = f32), 7-9 A fmt (1 = bf16), 10-12 B fmt (1 = bf16),
 // 13/14 negate A/B, 15/16 A/B major (0 = K, 1 = MN), 17-22 N>>3, 24-28 M>>4.
@@ -100,13 +109,22 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t *mbar, uint32_t parit
         : "=r"(ok) : "r"(smem_u32(mbar)), "r"(parity) : "memory");
     return ok;
 }
-// Bounded wait: returns false (and the caller records an error) if the phase
-// did not complete within `limit` polls.  Never traps, never spins forever.
+// Bounded wait: returns false if the phase did not complete within
+// `limit` polls (the caller then records the failure and winds down).
+// Never traps, never spins forever.
 __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint32_t limit = (1u << 26))
 {
     for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(mbar, parity)) return true;
     return false;
+}
+// Bounded wait measured in SM clock cycles (about `cycles` / 1.9e9 seconds).
+__device__ __forceinline__ bool mbar_wait_cycles(uint64_t *mbar, uint32_t parity, long long cycles)
+{
+    const long long t0 = clock64();
+    while (!mbar_try_wait(mbar, parity))
+        if (clock64() - t0 > cycles) return false;
+    return true;
 }
 
 // ---- TMEM <-> registers (32 lanes x N columns of 32 bit per warp) ---------
@@ -131,6 +149,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *r)
         :: "r"(taddr), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
            "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
         : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *r)
+{
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15]),
+          "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]),
+          "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+        : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
