@@ -6,39 +6,47 @@
 //   o_t = S_t^T q_t,
 // with (a~, m) = (beta k, beta v) for KDA / Complex KDA, (e k, w v) for RDA and
 // (b (.) k, w (.) v) for GDN-2.  Unrolled over a chunk of C tokens that starts
-// from state S0 (positions r, s in 0..C-1, all products forward, never divided):
-//   Gamma_r      = prod_{t<=r} alpha_t                      (per key channel)
-//   Lam_{r,s}    = prod_{s<t<=r} alpha_t
-//   A_{r,s}      = sum_c a~_{r,c} Lam_{r,s,c} k_{s,c}        (s < r)
-//   P_{r,s}      = sum_c q_{r,c}  Lam_{r,s,c} k_{s,c}        (s <= r)
-//   T            = (I + A)^{-1}                             (UT transform)
-//   W            = T (Gamma (.) A~),    U = T M - W S0        (WY form)
-//   O            = (Gamma (.) Q) S0 + P U
-//   S_C          = Diag(Gamma_C) S0 + Kbar^T U,   Kbar_s = Lam_{C-1,s} (.) k_s
-// Because alpha may be negative or zero (Complex KDA gates in [-1,1]), no
-// log-space cumulative sum and no ratio Gamma_r / Gamma_s is ever formed:
-// A and P are built from "anchored" forward products.  At level L = 1..6 the
-// chunk is cut into blocks of 2h tokens (h = 32 >> (L-1)); for a row r in a
-// block's second half and a column s in its first half, with anchor
-// a = last token of the first half,
-//   Lam_{r,s} = (prod_{a<t<=r} alpha_t) (.) (prod_{s<t<=a} alpha_t),
-// so that level's pairs are one dense product of "row factors" and "column
-// factors" (a tensor-core GEMM with K = d_k).  The six levels cover every
-// pair s < r exactly once; the diagonal P_{r,r} = q_r . k_r is a dot product.
+// from state S0 (positions r, s in 0..C-1; every product taken forward):
+//   Gamma_r   = prod_{t<=r} alpha_t                 (per key channel)
+//   Lam_{r,s} = prod_{s<t<=r} alpha_t
+//   A_{r,s}   = sum_c a~_{r,c} Lam_{r,s,c} k_{s,c}   (s < r)
+//   P_{r,s}   = sum_c q_{r,c}  Lam_{r,s,c} k_{s,c}   (s <= r)
+//   T         = (I + A)^{-1}                        (UT transform)
+//   W         = T (Gamma (.) A~),   U = T M - W S0  (WY form)
+//   O         = (Gamma (.) Q) S0 + P U
+//   S_C       = Diag(Gamma_C) S0 + Kbar^T U,   Kbar_s = Lam_{C-1,s} (.) k_s
 //
-// One CTA per (sequence, head); the d_k x d_v fp32 state lives in tensor
-// memory (TMEM) for the whole sequence, transposed (lane = value column j,
-// column = key channel i), so every state-dependent GEMM has M = d_v = 128.
-// q, k, v, alpha tiles arrive by TMA; every other operand is produced on chip
-// in 128-byte-swizzled shared-memory tiles.  Per chunk:
-//   1. TMA raw tiles -> decay products, Gamma(.)Q, Gamma(.)A~, Kbar, M
-//   2. level factors -> three tcgen05 GEMMs (M=128, N=64) -> A, P
-//   3. T = (I + A)^{-1} by blocked forward substitution (fp32, SIMT)
-//   4. tcgen05: W = T (Gamma(.)A~);  U^T = M^T T^T
-//   5. tcgen05: U^T -= S0^T W^T;  O^T = S0^T (Gamma(.)Q)^T;  S^T *= Gamma_C
-//   6. tcgen05: O^T += U^T P^T;  S^T += U^T Kbar  -> o to HBM, S^T -> bf16 copy
-// The next chunk's TMA loads are issued as soon as step 2 has consumed the
-// raw tiles.
+// Sign-safe decay.  Complex-KDA gates lie in [-1,1], so cumulative products can
+// be negative, zero or vanishingly small; no logarithm of alpha is ever taken.
+// A and P are formed one of two ways, decided per chunk for the whole CTA:
+//  * fast path, when every |alpha| <= 1 and every channel's chunk product
+//    satisfies |Gamma_C| >= 2^-110: Lam_{r,s} = (Gamma_r / Gamma_C) Lam_{C-1,s},
+//    so [A; P] is ONE tensor-core GEMM of the row operand
+//    [Gamma (.) A~ / Gamma_C ; Gamma (.) Q / Gamma_C] with Kbar (K = d_k).  The
+//    only division is by Gamma_C, which is bounded away from zero.  The state
+//    operand is then the scaled state Diag(Gamma_C) S0, which makes
+//    W S0 = (W / Gamma_C)(Gamma_C S0) and (Gamma Q) S0 = (Gamma Q / Gamma_C)(Gamma_C S0).
+//  * anchored path otherwise (zero or tiny gates): at level L = 1..6 the chunk
+//    is cut into blocks of 2h tokens (h = 32 >> (L-1)); for r in a block's
+//    second half and s in its first half, with a = last token of the first half,
+//      Lam_{r,s} = (prod_{a<t<=r} alpha_t) (.) (prod_{s<t<=a} alpha_t),
+//    a product of forward "row" and "column" factors, so each level's pairs are
+//    one dense GEMM.  Six levels cover every pair s < r once; P_{r,r} = q_r . k_r.
+//    Nothing is divided, so zeros and signs propagate exactly.
+//
+// One CTA per (sequence, head); the fp32 state lives in tensor memory (TMEM)
+// for the whole sequence, transposed (lane = value column j, column = key
+// channel i), so every state-dependent GEMM has M = d_v = 128.  q, k, v,
+// alpha arrive by TMA; every other operand is built on chip in 128-byte
+// swizzled shared-memory tiles.  Per chunk:
+//   1. TMA raw tiles -> block totals, Gamma_C, M, Kbar, row operands
+//   2. A, P  (one GEMM on the fast path, three on the anchored path)
+//   3. T = (I + A)^{-1}: 16x16 diagonal blocks, then two recursive-doubling merges
+//   4. tcgen05: W = T (row operand a~ part);  U^T = M^T T^T
+//   5. state pass: S^T *= Gamma_C in TMEM and its bf16 copy (scaled or not)
+//   6. tcgen05: U^T -= S^T W^T;  O^T = S^T Q^T
+//   7. tcgen05: O^T += U^T P^T;  S^T += U^T Kbar;  o -> HBM
+// The next chunk's TMA loads start as soon as step 2 has consumed the raw tiles.
 #include <cuda.h>
 #include <cstring>
 #include <mutex>
@@ -55,48 +63,51 @@ constexpr int D = 128;   // d_k = d_v
 constexpr int NT = 256;  // threads per CTA
 
 // ---- shared memory map (offsets from a 1024-byte aligned base) ------------
-constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_V = 32768, RAW_A = 49152;  // TMA tiles [64][128] bf16
-constexpr uint32_t OFF_S0T = 65536;   // S^T bf16, 128 x 128, K-major (rows j, K = i)
-constexpr uint32_t OFF_QG = 98304;    // Gamma (.) q      [token][channel] tile
-constexpr uint32_t OFF_KB = 114688;   // Kbar             [token][channel]
-constexpr uint32_t OFF_AG = 131072;   // Gamma (.) a~     [token][channel]; later W
-constexpr uint32_t OFF_MT = 147456;   // M                [token][channel]; later U^T (128 x 64)
-constexpr uint32_t OFF_F = 163840;    // level factors; later A, T (fp32), T, P (bf16)
-constexpr uint32_t OFF_FA = OFF_F;            // 128 rows x 128 ch (32 KB)
-constexpr uint32_t OFF_FB = OFF_F + 32768;    // 64 rows x 128 ch (16 KB)
-constexpr uint32_t OFF_AF32 = OFF_F;          // A  fp32 [64][65]
-constexpr uint32_t OFF_TF32 = OFF_F + 16640;  // T  fp32 [64][65]
-constexpr uint32_t OFF_X = OFF_F + 33280;     // 3 x 16 x 16 fp32 scratch of the block solve
-constexpr uint32_t OFF_TBF = OFF_F + 36864;   // T bf16 64 x 64 K-major
-constexpr uint32_t OFF_PBF = OFF_F + 45056;   // P bf16 64 x 64 K-major
-constexpr uint32_t OFF_MISC = OFF_F + 53248;
+constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_A = 49152;  // TMA tiles [64][128] bf16, row-major
+constexpr uint32_t OFF_UT = 32768;   // T Diag(w) bf16 64 x 64 (step 4), then U^T 128 x 64 (steps 6-7)
+constexpr uint32_t OFF_S0T = 65536;   // state operand bf16, 128 x 128, K-major (rows j, K = i)
+constexpr uint32_t OFF_QA = 98304;    // 128-row tile: rows 0-63 a~ operand (later W), rows 64-127 q operand
+constexpr uint32_t OFF_KB = 131072;   // Kbar [token][channel]
+constexpr uint32_t OFF_MT = 147456;   // M [token][channel]: v by 128B-swizzled TMA (GDN-2: scaled by w in place)
+constexpr uint32_t OFF_F = 163840;    // anchored-path level factors | A, T fp32, T, P bf16 | o staging
+constexpr uint32_t OFF_LA = OFF_F;            // level row factors: 128 rows x 128 ch
+constexpr uint32_t OFF_LB = OFF_F + 32768;    // level column factors: 64 rows x 128 ch
+constexpr uint32_t OFF_AF32 = OFF_F;          // A fp32 [64][65]
+constexpr uint32_t OFF_TF32 = OFF_F + 16640;  // T fp32 [64][65]
+constexpr uint32_t OFF_X = OFF_F + 33280;     // 32 x 32 fp32 scratch of the block solve
+constexpr uint32_t OFF_TBF = OFF_F + 37888;   // T Diag(e) bf16 64 x 64 K-major
+constexpr uint32_t OFF_PBF = OFF_F + 46080;   // P bf16 64 x 64 K-major
+constexpr uint32_t OFF_OST = OFF_F;           // o staging [64][128] bf16 (A, T dead by then)
+constexpr uint32_t OFF_MISC = OFF_F + 54272;
+constexpr int PBAND = 5;   // P_{r,s} for r-4 <= s <= r computed exactly (SIMT) from the bf16 inputs
 constexpr uint32_t M_G1 = OFF_MISC, M_G2 = OFF_MISC + 256, M_GAMC = OFF_MISC + 512, M_TOT = OFF_MISC + 1024,
-                   M_PDIAG = OFF_MISC + 5120, M_BAR = OFF_MISC + 5376, M_TMEM = OFF_MISC + 5408,
-                   M_FLAG = OFF_MISC + 5412;
-constexpr uint32_t SMEM_USED = OFF_MISC + 5440;
+                   M_PBAND = OFF_MISC + 5120, M_BAR = OFF_MISC + 6400, M_TMEM = OFF_MISC + 6432;
+constexpr uint32_t SMEM_USED = OFF_MISC + 6464;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack for aligning the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert((OFF_TBF & 1023) == 0 && (OFF_PBF & 1023) == 0 && (OFF_QA & 1023) == 0, "swizzle atoms");
 
 // ---- TMEM columns ---------------------------------------------------------
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 192, TM_W = 256;
-__device__ __forceinline__ uint32_t tm_ap(int p) { return p == 0 ? 384u : (p == 1 ? 448u : 256u); }
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 192, TM_W = 256, TM_AP = 384;
+__device__ __forceinline__ uint32_t tm_lvl(int p) { return p == 0 ? 384u : (p == 1 ? 448u : 256u); }
 
 constexpr long long WAIT_CYCLES = 4000000000ll;  // ~2 s: only a broken pipeline gets near it
+constexpr float FAST_MIN_GAMMA = 7.703719777548943e-34f;  // 2^-110
 
 struct ChunkParams {
-    CUtensorMap tq, tk, tv, ta;  // [B*T][H][128] bf16, box {128, 1, 64}
+    CUtensorMap tq, tk, ta;  // [B*T][H][128] bf16, box {128, 1, 64}, no swizzle
+    CUtensorMap tv;          // same tensor shape, box {64, 1, 64}, 128-byte swizzle
     FwdArgs a;
 };
 
 // ---- small helpers --------------------------------------------------------
 __device__ __forceinline__ void unpack8(const uint4 &u, float *f)
 {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float2 x = __bfloat1622float2(h[i]);
-        f[2 * i] = x.x;
-        f[2 * i + 1] = x.y;
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
 }
 __device__ __forceinline__ uint4 pack8(const float *f)
@@ -104,34 +115,160 @@ __device__ __forceinline__ uint4 pack8(const float *f)
     return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
 }
 // 16-byte chunk kc (8 consecutive K elements) of row `row` in a K-major
-// 128B-swizzled tile with `rows` rows: 64-element panels of rows*128 bytes.
-__device__ __forceinline__ uint32_t sw_chunk(uint32_t rows, uint32_t row, uint32_t kc)
+// 128B-swizzled tile whose 64-element panels are `pstride` bytes apart.
+__device__ __forceinline__ uint32_t sw_chunk(uint32_t pstride, uint32_t row, uint32_t kc)
 {
-    return (kc >> 3) * (rows * 128u) + row * 128u + ((((kc & 7u) ^ (row & 7u))) << 4);
+    return (kc >> 3) * pstride + row * 128u + ((((kc & 7u) ^ (row & 7u))) << 4);
 }
-__device__ __forceinline__ uint32_t sw_elem(uint32_t rows, uint32_t row, uint32_t k)
+__device__ __forceinline__ uint32_t sw_elem(uint32_t pstride, uint32_t row, uint32_t k)
 {
-    return sw_chunk(rows, row, k >> 3) + (k & 7u) * 2u;
+    return sw_chunk(pstride, row, k >> 3) + (k & 7u) * 2u;
 }
 // raw TMA tile: row-major [64][128] bf16
 __device__ __forceinline__ uint4 raw_row(const uint8_t *sm, uint32_t base, int r, int cg)
 {
     return *reinterpret_cast<const uint4 *>(sm + base + r * 256 + cg * 16);
 }
-
-// K-major descriptor of a 128B-swizzled tile, K step kk (16 elements)
-__device__ __forceinline__ uint64_t dK(uint32_t base, uint32_t rows, int kk)
+// K-major descriptor, K step kk (16 elements), panels `pstride` bytes apart
+__device__ __forceinline__ uint64_t dK(uint32_t base, uint32_t pstride, int kk)
 {
-    return make_desc_sw128(base + (uint32_t)(kk >> 2) * rows * 128u + (uint32_t)(kk & 3) * 32u, 16);
+    return make_desc_sw128(base + (uint32_t)(kk >> 2) * pstride + (uint32_t)(kk & 3) * 32u, 16);
 }
-// MN-major descriptor of a [token][channel] tile (MN = 128 channels in two
-// 64-wide panels 8 KB apart, K = tokens), K step kk (16 tokens)
-__device__ __forceinline__ uint64_t dMN(uint32_t base, int kk)
+// MN-major descriptor of a [token][channel] tile (channels in two 64-wide
+// panels `pstride` bytes apart, K = tokens), K step kk (16 tokens)
+__device__ __forceinline__ uint64_t dMN(uint32_t base, uint32_t pstride, int kk)
 {
-    return make_desc_sw128(base + (uint32_t)kk * 2048u, 8192);
+    return make_desc_sw128(base + (uint32_t)kk * 2048u, pstride);
+}
+__device__ __forceinline__ float bf2f(const __nv_bfloat16 *p, size_t i)
+{
+    return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short *>(p + i)) << 16);
+}
+__device__ __forceinline__ void load_tot(const float *s_tot, int g, int cg, float *t8)
+{
+    *reinterpret_cast<float4 *>(t8) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8);
+    *reinterpret_cast<float4 *>(t8 + 4) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8 + 4);
 }
 
-__device__ __forceinline__ float g_scalar(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
+struct ChunkCtx {
+    uint8_t *sm;
+    const float *s_tot, *s_g1;
+    const __nv_bfloat16 *g1p;
+    size_t rowbase;
+    int H, h, nvalid;
+    bool gdn2;
+};
+
+// Channel-wise part of the erase direction of row r (GDN-2: the vector b;
+// 1 otherwise, because the scalar erase gate is folded into the rows of A and
+// the columns of T instead of into the bf16 operands).
+__device__ __forceinline__ void erase_gate(const ChunkCtx &x, int r, int cg, float *e)
+{
+    if (x.gdn2 && r < x.nvalid) {
+        unpack8(*reinterpret_cast<const uint4 *>(x.g1p + ((x.rowbase + r) * x.H + x.h) * D + cg * 8), e);
+    } else {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) e[c] = 1.f;
+    }
+}
+
+// Anchored path: row and column factors of one level (block half HH) for the
+// 8-token x 8-channel item (tg, cg), into level slot `slot` (0 or 1).
+template <int HH>
+__device__ __forceinline__ void build_level(const ChunkCtx &x, int slot, int tg, int cg)
+{
+    constexpr int BS = 2 * HH;
+    uint8_t *sm = x.sm;
+    float cpre[8], csuf[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) { cpre[c] = 1.f; csuf[c] = 1.f; }
+    if (HH >= 8) {  // carries over whole 8-token blocks
+        const int r0 = tg * 8, pos0 = r0 % BS;
+        const int gs = (r0 - pos0 + HH) >> 3, ge = (r0 - pos0 + HH - 1) >> 3;
+        for (int g = 0; g < 8; ++g) {
+            const bool in_pre = pos0 >= HH && g >= gs && g < tg;
+            const bool in_suf = pos0 < HH && g > tg && g <= ge;
+            if (in_pre || in_suf) {
+                float t8[8];
+                load_tot(x.s_tot, g, cg, t8);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (in_pre) cpre[c] *= t8[c];
+                    if (in_suf) csuf[c] *= t8[c];
+                }
+            }
+        }
+    }
+    float run[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) run[c] = cpre[c];
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i) {  // second-half rows: prefix from the half start
+        const int r = tg * 8 + i, pos = r % BS;
+        if (HH < 8 && pos == HH) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) run[c] = 1.f;
+        }
+        if (pos < HH) continue;
+        const bool v = r < x.nvalid;
+        float al[8], qv[8], kv[8], e[8], fa[8], fp[8];
+        unpack8(raw_row(sm, RAW_A, r, cg), al);
+        unpack8(raw_row(sm, RAW_Q, r, cg), qv);
+        unpack8(raw_row(sm, RAW_K, r, cg), kv);
+        erase_gate(x, r, cg, e);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            run[c] *= v ? al[c] : 1.f;
+            fa[c] = v ? run[c] * e[c] * kv[c] : 0.f;
+            fp[c] = v ? run[c] * qv[c] : 0.f;
+        }
+        const int idx = (r / BS) * HH + (pos - HH);
+        *reinterpret_cast<uint4 *>(sm + OFF_LA + sw_chunk(16384, slot * 32 + idx, cg)) = pack8(fa);
+        *reinterpret_cast<uint4 *>(sm + OFF_LA + sw_chunk(16384, 64 + slot * 32 + idx, cg)) = pack8(fp);
+    }
+    float sx[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) sx[c] = csuf[c];
+#pragma unroll 1
+    for (int i = 7; i >= 0; --i) {  // first-half columns: exclusive suffix to the half end
+        const int r = tg * 8 + i, pos = r % BS;
+        if (pos >= HH) continue;
+        if (HH < 8 && pos == HH - 1) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sx[c] = 1.f;
+        }
+        const bool v = r < x.nvalid;
+        float al[8], kv[8], fc[8];
+        unpack8(raw_row(sm, RAW_A, r, cg), al);
+        unpack8(raw_row(sm, RAW_K, r, cg), kv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            fc[c] = v ? sx[c] * kv[c] : 0.f;
+            sx[c] *= v ? al[c] : 1.f;
+        }
+        const int idx = (r / BS) * HH + pos;
+        *reinterpret_cast<uint4 *>(sm + OFF_LB + sw_chunk(8192, slot * 32 + idx, cg)) = pack8(fc);
+    }
+}
+
+// Anchored path: scatter one level's A or P entries from the 32 TMEM columns
+// the calling warp loaded (rows of this lane's level list).
+template <int HH>
+__device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const float *s_e, bool isP, int lane,
+                                              const float *v)
+{
+    constexpr int BS = 2 * HH;
+    const int r = (lane / HH) * BS + HH + (lane % HH);
+    const int c0 = (r / BS) * HH;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        if (c >= c0 && c < c0 + HH) {
+            const int s = (c / HH) * BS + (c % HH);
+            if (!isP) Af[r * 65 + s] = v[c] * s_e[r];
+            else *reinterpret_cast<unsigned short *>(sm + OFF_PBF + sw_elem(8192, r, s)) = bf16_bits(v[c]);
+        }
+    }
+}
 
 // ---- the kernel -------------------------------------------------------------
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant__ ChunkParams P)
@@ -141,7 +278,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     const uint32_t sb = smem_u32(sm);
     const FwdArgs &a = P.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quarter = warp & 3;                      // TMEM lane quarter of this warp
+    const int quarter = warp & 3;       // TMEM lane quarter of this warp
+    const int half = warp >> 2;         // warps 0-3 / 4-7 split TMEM columns
     const int H = a.H;
     const int n = blockIdx.x / H, h = blockIdx.x % H;
     int b, t0, len;
@@ -152,23 +290,25 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     float *s_g1 = reinterpret_cast<float *>(sm + M_G1);
     float *s_g2 = reinterpret_cast<float *>(sm + M_G2);
     float *s_gamC = reinterpret_cast<float *>(sm + M_GAMC);
-    float *s_tot = reinterpret_cast<float *>(sm + M_TOT);   // [8][128]
-    float *s_pdiag = reinterpret_cast<float *>(sm + M_PDIAG);
+    float *s_tot = reinterpret_cast<float *>(sm + M_TOT);   // [8][128] block totals of alpha
+    float *s_pband = reinterpret_cast<float *>(sm + M_PBAND);   // [64][PBAND]: P_{r, r-w}
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + M_BAR);
     uint64_t *bar_mma = bar_tma + 1;
+    uint64_t *bar_v = bar_tma + 2;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + M_TMEM);
     float *Af = reinterpret_cast<float *>(sm + OFF_AF32);
     float *Tf = reinterpret_cast<float *>(sm + OFF_TF32);
     float *Xs = reinterpret_cast<float *>(sm + OFF_X);
 
     const __nv_bfloat16 *g1p = (const __nv_bfloat16 *)a.g1, *g2p = (const __nv_bfloat16 *)a.g2;
-    __nv_bfloat16 *op = (__nv_bfloat16 *)a.o;
+    uint8_t *op = (uint8_t *)a.o;
     const bool gdn2 = a.variant == GDN2;
 
     if (warp == 0) tmem_alloc(s_tmem, 512);
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_v, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
@@ -176,510 +316,555 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     tc_fence_after();
     const uint32_t tbase = *s_tmem;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    uint32_t ph_tma = 0, ph_mma = 0;
+    const int jcol = quarter * 32 + lane;   // value column j = TMEM lane of this thread
+    uint32_t ph_tma = 0, ph_mma = 0, ph_v = 0;
     bool ok = true;
 
     const CUtensorMap *map_q = &P.tq, *map_k = &P.tk, *map_v = &P.tv, *map_a = &P.ta;
-    auto issue_tma = [&](int chunk) {
+    auto issue_tma = [&](int chunk) {   // q, k, alpha of a chunk
         const int g = b * a.T + t0 + chunk * C;  // token row of the packed [B*T] axis
-        mbar_expect_tx(bar_tma, 4 * 16384);
+        mbar_expect_tx(bar_tma, 3 * 16384);
         tma_load_3d(sm + RAW_Q, map_q, bar_tma, 0, h, g);
         tma_load_3d(sm + RAW_K, map_k, bar_tma, 0, h, g);
-        tma_load_3d(sm + RAW_V, map_v, bar_tma, 0, h, g);
         tma_load_3d(sm + RAW_A, map_a, bar_tma, 0, h, g);
     };
-    // all threads: wait for the MMAs committed so far, then order TMEM reads after them
-    auto wait_mma = [&]() {
+    auto issue_tma_v = [&](int chunk) { // v, straight into its swizzled operand layout (two 64-channel panels)
+        const int g = b * a.T + t0 + chunk * C;
+        mbar_expect_tx(bar_v, 16384);
+        tma_load_3d(sm + OFF_MT, map_v, bar_v, 0, h, g);
+        tma_load_3d(sm + OFF_MT + 8192, map_v, bar_v, 64, h, g);
+    };
+    auto wait_mma = [&]() {     // all threads: MMAs committed so far are complete
         if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
         ph_mma ^= 1;
         tc_fence_after();
     };
-    // all threads: publish shared-memory / TMEM writes to the tensor core, then barrier
-    auto publish = [&]() {
+    auto publish = [&]() {      // all threads: make smem / TMEM writes visible to the tensor core
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
     };
 
-    if (nchunks > 0 && tid == 0) issue_tma(0);
+    if (nchunks > 0 && tid == 0) {
+        issue_tma(0);
+        issue_tma_v(0);
+    }
 
-    // ---- initial state -> TMEM (fp32) and S0^T (bf16) ----------------------
+    // ---- initial state -> TMEM (fp32) ----------------------------------------
     {
         const size_t soff = ((size_t)n * H + h) * D * D;
-        const int j = quarter * 32 + lane;          // value column = TMEM lane
-        const int ihalf = warp >> 2;                // key channels [64*ihalf, +64)
         for (int c16 = 0; c16 < 4; ++c16) {
             float v[16];
-            const int i0 = ihalf * 64 + c16 * 16;
+            const int i0 = half * 64 + c16 * 16;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = a.s0 ? a.s0[soff + (size_t)(i0 + e) * D + j] : 0.f;
+            for (int e = 0; e < 16; ++e) v[e] = a.s0 ? a.s0[soff + (size_t)(i0 + e) * D + jcol] : 0.f;
             tmem_st16(tbase + lane_base + TM_S + i0, v);
-            *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(128, j, i0 >> 3)) = pack8(v);
-            *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(128, j, (i0 >> 3) + 1)) = pack8(v + 8);
         }
         tmem_wait_st();
     }
-    publish();
+    tc_fence_before();
+    __syncthreads();
 
     for (int ch = 0; ch < nchunks && ok; ++ch) {
         const int tok0 = t0 + ch * C;
         const int nvalid = min(C, len - ch * C);
         const size_t rowbase = (size_t)b * a.T + tok0;   // packed token index of chunk row 0
+        const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
 
-        // gate scalars (masked to 0 past the sequence end)
-        if (tid < C) {
+        if (tid < C) {  // scalar erase / write gates (1 for GDN-2), 0 past the sequence end
             const bool v = tid < nvalid;
             const size_t tok = (rowbase + tid) * H + h;
-            if (!gdn2) {
-                s_g1[tid] = v ? g_scalar(g1p, tok) : 0.f;
-                s_g2[tid] = v ? (a.variant == KDA ? g_scalar(g1p, tok) : g_scalar(g2p, tok)) : 0.f;
+            if (gdn2) {
+                s_g1[tid] = v ? 1.f : 0.f;
+                s_g2[tid] = v ? 1.f : 0.f;
+            } else {
+                s_g1[tid] = v ? bf2f(g1p, tok) : 0.f;
+                s_g2[tid] = v ? (a.variant == KDA ? bf2f(g1p, tok) : bf2f(g2p, tok)) : 0.f;
             }
         }
         if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
         ph_tma ^= 1;
-        __syncthreads();  // gate scalars visible to every thread
+        if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
+        ph_v ^= 1;
+        __syncthreads();
 
-        // ===== 1a. block totals of alpha; M; diagonal of P ====================
+        // ===== 1a. block totals of alpha (and range check) | M ================
+        bool in_range = true;
         if (tid < 128) {
             const int tg = tid >> 4, cg = tid & 15;
             float tot[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) tot[c] = 1.f;
+#pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int r = tg * 8 + i;
                 if (r < nvalid) {
                     float al[8];
                     unpack8(raw_row(sm, RAW_A, r, cg), al);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) tot[c] *= al[c];
+                    for (int c = 0; c < 8; ++c) {
+                        tot[c] *= al[c];
+                        in_range = in_range && (fabsf(al[c]) <= 1.f);
+                    }
                 }
             }
             *reinterpret_cast<float4 *>(s_tot + tg * 128 + cg * 8) = make_float4(tot[0], tot[1], tot[2], tot[3]);
             *reinterpret_cast<float4 *>(s_tot + tg * 128 + cg * 8 + 4) = make_float4(tot[4], tot[5], tot[6], tot[7]);
         } else {
             const int u = tid - 128, tg = u >> 4, cg = u & 15;
-            for (int i = 0; i < 8; ++i) {
-                const int r = tg * 8 + i;
-                float mv[8], vv[8];
-                unpack8(raw_row(sm, RAW_V, r, cg), vv);
-                if (r < nvalid) {
-                    if (gdn2) {
-                        float wv[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(g2p + ((rowbase + r) * H + h) * D + cg * 8), wv);
+            {   // band of P: P_{r,r-w} = sum_c q_rc (alpha_r ... alpha_{r-w+1})_c k_{r-w,c}, w = 0..4,
+                // from the bf16 inputs in fp32 (the entries the bf16 GEMM would round most
+                // harmfully); two threads per row, 64 channels each
+                const int r = u >> 1, hf = u & 1;
+                float acc[PBAND];
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) mv[c] = wv[c] * vv[c];
-                    } else {
-                        const float g = s_g2[r];
+                for (int w = 0; w < PBAND; ++w) acc[w] = 0.f;
+                for (int cc = 0; cc < 8; ++cc) {
+                    const int cgx = hf * 8 + ((cc + r) & 7);   // staggered by row: conflict-free loads
+                    float hv[8], kv[8], av[8];
+                    unpack8(raw_row(sm, RAW_Q, r, cgx), hv);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) mv[c] = g * vv[c];
-                    }
-                } else {
+                    for (int w = 0; w < PBAND; ++w) {
+                        if (r - w >= 0) {
+                            unpack8(raw_row(sm, RAW_K, r - w, cgx), kv);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) mv[c] = 0.f;
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_MT + sw_chunk(64, r, cg)) = pack8(mv);
-            }
-            // P_{r,r} = q_r . k_r : two threads per row
-            const int r = u >> 1, hf = u & 1;
-            float acc = 0.f;
-            for (int cc = 0; cc < 8; ++cc) {
-                float qv[8], kv[8];
-                unpack8(raw_row(sm, RAW_Q, r, hf * 8 + cc), qv);
-                unpack8(raw_row(sm, RAW_K, r, hf * 8 + cc), kv);
+                            for (int c = 0; c < 8; ++c) acc[w] = fmaf(hv[c], kv[c], acc[w]);
+                            if (w + 1 < PBAND && r - w - 1 >= 0) {
+                                unpack8(raw_row(sm, RAW_A, r - w, cgx), av);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc = fmaf(qv[c], kv[c], acc);
-            }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            if (hf == 0) s_pdiag[r] = (r < nvalid) ? acc : 0.f;
-        }
-        __syncthreads();
-
-        // ===== 1b. Gamma (.) q, Gamma (.) a~, Kbar, Gamma_C ==================
-        if (tid < 128) {
-            const int tg = tid >> 4, cg = tid & 15;
-            float pre[8], suf[8], run[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) { pre[c] = 1.f; suf[c] = 1.f; run[c] = 1.f; }
-            for (int g = 0; g < 8; ++g) {
-                float t8[8];
-                *reinterpret_cast<float4 *>(t8) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8);
-                *reinterpret_cast<float4 *>(t8 + 4) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8 + 4);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (g < tg) pre[c] *= t8[c];
-                    if (g > tg) suf[c] *= t8[c];
-                }
-            }
-            for (int i = 0; i < 8; ++i) {
-                const int r = tg * 8 + i;
-                const bool v = r < nvalid;
-                float al[8], qv[8], kv[8], gq[8], ga[8];
-                unpack8(raw_row(sm, RAW_A, r, cg), al);
-                unpack8(raw_row(sm, RAW_Q, r, cg), qv);
-                unpack8(raw_row(sm, RAW_K, r, cg), kv);
-                float e[8];
-                if (gdn2) {
-                    if (v) unpack8(*reinterpret_cast<const uint4 *>(g1p + ((rowbase + r) * H + h) * D + cg * 8), e);
-                    else {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) e[c] = 0.f;
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) e[c] = s_g1[r];
-                }
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const float alc = v ? al[c] : 1.f;
-                    run[c] *= alc;
-                    const float gam = pre[c] * run[c];
-                    gq[c] = v ? gam * qv[c] : 0.f;
-                    ga[c] = v ? gam * (e[c] * kv[c]) : 0.f;
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_QG + sw_chunk(64, r, cg)) = pack8(gq);
-                *reinterpret_cast<uint4 *>(sm + OFF_AG + sw_chunk(64, r, cg)) = pack8(ga);
-            }
-            // exclusive suffix inside the block, times the later blocks' totals
-            float sx[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) sx[c] = 1.f;
-            for (int i = 7; i >= 0; --i) {
-                const int r = tg * 8 + i;
-                const bool v = r < nvalid;
-                float al[8], kv[8], kb[8];
-                unpack8(raw_row(sm, RAW_A, r, cg), al);
-                unpack8(raw_row(sm, RAW_K, r, cg), kv);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    kb[c] = v ? suf[c] * sx[c] * kv[c] : 0.f;
-                    sx[c] *= v ? al[c] : 1.f;
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_KB + sw_chunk(64, r, cg)) = pack8(kb);
-            }
-            if (tg == 0) {
-                // Gamma_C = product of all block totals = own block total (sx) x later blocks (suf)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) s_gamC[cg * 8 + c] = sx[c] * suf[c];
-            }
-        }
-
-        // ===== 2. A and P by anchored levels on the tensor core ===============
-        for (int p = 0; p < 3; ++p) {
-            // threads 0..127 build level 2p+1, threads 128..255 level 2p+2
-            {
-                const int lvl = 2 * p + 1 + (tid >> 7);
-                const int hh = 32 >> (lvl - 1);
-                const int slot = tid >> 7;                 // 0: first level of the pair, 1: second
-                const int u = tid & 127, tg = u >> 4, cg = u & 15;
-                // carries over whole 8-token blocks (levels 1-3 only)
-                float cpre[8], csuf[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) { cpre[c] = 1.f; csuf[c] = 1.f; }
-                if (hh >= 8) {
-                    const int r0 = tg * 8, pos0 = r0 % (2 * hh);
-                    const int gs = (r0 - pos0 + hh) >> 3;       // first block of the second half
-                    const int ge = (r0 - pos0 + hh - 1) >> 3;   // last block of the first half
-                    for (int g = 0; g < 8; ++g) {
-                        const bool in_pre = pos0 >= hh && g >= gs && g < tg;
-                        const bool in_suf = pos0 < hh && g > tg && g <= ge;
-                        if (in_pre || in_suf) {
-                            float t8[8];
-                            *reinterpret_cast<float4 *>(t8) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8);
-                            *reinterpret_cast<float4 *>(t8 + 4) =
-                                *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8 + 4);
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) {
-                                if (in_pre) cpre[c] *= t8[c];
-                                if (in_suf) csuf[c] *= t8[c];
+                                for (int c = 0; c < 8; ++c) hv[c] *= av[c];
                             }
                         }
                     }
                 }
-                // forward: second-half rows, prefix from the half start
-                float run[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) run[c] = cpre[c];
+                for (int w = 0; w < PBAND; ++w) {
+                    const float tot = acc[w] + __shfl_xor_sync(0xffffffffu, acc[w], 1);
+                    if (hf == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? tot : 0.f;
+                }
+            }
+            if (gdn2) {   // M = w (.) v, in place in the swizzled v tile (rows past the end -> 0)
+#pragma unroll 2
                 for (int i = 0; i < 8; ++i) {
-                    const int r = tg * 8 + i, pos = r % (2 * hh);
-                    if (pos == hh && hh < 8) {
+                    const int r = tg * 8 + i;
+                    uint4 *pv = reinterpret_cast<uint4 *>(sm + OFF_MT + sw_chunk(8192, r, cg));
+                    float mv[8], vv[8], wv[8];
+                    unpack8(*pv, vv);
+                    if (r < nvalid) {
+                        unpack8(*reinterpret_cast<const uint4 *>(g2p + ((rowbase + r) * H + h) * D + cg * 8), wv);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) run[c] = 1.f;
+                        for (int c = 0; c < 8; ++c) mv[c] = wv[c] * vv[c];
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) mv[c] = 0.f;
                     }
-                    if (pos < hh) continue;
+                    *pv = pack8(mv);
+                }
+            }
+        }
+        in_range = __syncthreads_and(in_range) != 0;
+
+        // ===== Gamma_C and the per-chunk path decision ========================
+        bool gam_ok = true;
+        if (tid < 16) {
+            const int cg = tid;
+            float gc[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) gc[c] = 1.f;
+            for (int g = 0; g < 8; ++g) {
+                float t8[8];
+                load_tot(s_tot, g, cg, t8);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) gc[c] *= t8[c];
+            }
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                s_gamC[cg * 8 + c] = gc[c];
+                gam_ok = gam_ok && (fabsf(gc[c]) >= FAST_MIN_GAMMA);
+            }
+        }
+        const bool fast = (__syncthreads_and(gam_ok) != 0) && in_range;
+
+        // ===== 1b. row operands (Gamma a~, Gamma q, scaled on the fast path) | Kbar
+        {
+            const int u = tid & 127, tg = u >> 4, cg = u & 15;
+            float pre[8], suf[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) { pre[c] = 1.f; suf[c] = 1.f; }
+            for (int g = 0; g < 8; ++g) {
+                if (g == tg) continue;
+                float t8[8];
+                load_tot(s_tot, g, cg, t8);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (g < tg) pre[c] *= t8[c];
+                    else suf[c] *= t8[c];
+                }
+            }
+            if (tid < 128) {
+                float sc[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) sc[c] = fast ? pre[c] * (1.0f / s_gamC[cg * 8 + c]) : pre[c];
+#pragma unroll 2
+                for (int i = 0; i < 8; ++i) {
+                    const int r = tg * 8 + i;
                     const bool v = r < nvalid;
-                    float al[8], qv[8], kv[8], fa[8], fp[8], e[8];
+                    float al[8], qv[8], kv[8], e[8], ga[8], gq[8];
                     unpack8(raw_row(sm, RAW_A, r, cg), al);
                     unpack8(raw_row(sm, RAW_Q, r, cg), qv);
                     unpack8(raw_row(sm, RAW_K, r, cg), kv);
-                    if (gdn2) {
-                        if (v) unpack8(*reinterpret_cast<const uint4 *>(g1p + ((rowbase + r) * H + h) * D + cg * 8), e);
-                        else {
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) e[c] = 0.f;
-                        }
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) e[c] = s_g1[r];
-                    }
+                    erase_gate(x, r, cg, e);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        run[c] *= v ? al[c] : 1.f;
-                        fa[c] = v ? run[c] * e[c] * kv[c] : 0.f;
-                        fp[c] = v ? run[c] * qv[c] : 0.f;
+                        sc[c] *= v ? al[c] : 1.f;
+                        ga[c] = v ? sc[c] * (e[c] * kv[c]) : 0.f;
+                        gq[c] = v ? sc[c] * qv[c] : 0.f;
                     }
-                    const int idx = (r / (2 * hh)) * hh + (pos - hh);
-                    *reinterpret_cast<uint4 *>(sm + OFF_FA + sw_chunk(128, slot * 32 + idx, cg)) = pack8(fa);
-                    *reinterpret_cast<uint4 *>(sm + OFF_FA + sw_chunk(128, 64 + slot * 32 + idx, cg)) = pack8(fp);
+                    *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, r, cg)) = pack8(ga);
+                    *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, 64 + r, cg)) = pack8(gq);
                 }
-                // backward: first-half columns, exclusive suffix to the half end
+            } else {
                 float sx[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) sx[c] = csuf[c];
+                for (int c = 0; c < 8; ++c) sx[c] = suf[c];
+#pragma unroll 2
                 for (int i = 7; i >= 0; --i) {
-                    const int r = tg * 8 + i, pos = r % (2 * hh);
-                    if (pos == 2 * hh - 1 && hh < 8) {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) sx[c] = 1.f;
-                    }
-                    if (pos >= hh) continue;
-                    if (pos == hh - 1 && hh < 8) {
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) sx[c] = 1.f;
-                    }
+                    const int r = tg * 8 + i;
                     const bool v = r < nvalid;
-                    float al[8], kv[8], fc[8];
+                    float al[8], kv[8], kb[8];
                     unpack8(raw_row(sm, RAW_A, r, cg), al);
                     unpack8(raw_row(sm, RAW_K, r, cg), kv);
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        fc[c] = v ? sx[c] * kv[c] : 0.f;
+                        kb[c] = v ? sx[c] * kv[c] : 0.f;
                         sx[c] *= v ? al[c] : 1.f;
                     }
-                    const int idx = (r / (2 * hh)) * hh + pos;
-                    *reinterpret_cast<uint4 *>(sm + OFF_FB + sw_chunk(64, slot * 32 + idx, cg)) = pack8(fc);
+                    *reinterpret_cast<uint4 *>(sm + OFF_KB + sw_chunk(8192, r, cg)) = pack8(kb);
                 }
             }
+        }
+
+        // ===== 2. A and P ======================================================
+        if (fast) {
             publish();
             if (tid == 0) {
                 tc_fence_after();
                 const uint32_t idesc = idesc_bf16(128, 64, false, false);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tbase + tm_ap(p), dK(sb + OFF_FA, 128, kk), dK(sb + OFF_FB, 64, kk), idesc, kk > 0);
+                    mma_bf16(tbase + TM_AP, dK(sb + OFF_QA, 16384, kk), dK(sb + OFF_KB, 8192, kk), idesc, kk > 0);
                 mma_commit(bar_mma);
             }
             wait_mma();
-        }
-        // raw tiles consumed: prefetch the next chunk
-        __syncthreads();
-        if (tid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);
-
-        // ===== 2b. read A, P out of TMEM ======================================
-        for (int e = tid; e < 64 * 65; e += NT) { Af[e] = 0.f; Tf[e] = 0.f; }
-        for (int e = tid; e < 512; e += NT) *reinterpret_cast<uint4 *>(sm + OFF_PBF + e * 16) = make_uint4(0, 0, 0, 0);
-        __syncthreads();
-        for (int p = (warp >> 2); p < 3; p += 2) {
-            const int lvl = 2 * p + 1 + (quarter & 1);
-            const int hh = 32 >> (lvl - 1);
-            const bool isP = quarter >= 2;
+            if (tid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
+            // rows 0-63: A (strictly lower), rows 64-127: P (lower incl. diagonal)
             float v[32];
-            tmem_ld32(tbase + lane_base + tm_ap(p) + (quarter & 1) * 32, v);
+            tmem_ld32(tbase + lane_base + TM_AP + half * 32, v);
             tmem_wait_ld();
-            const int r = (lane / hh) * 2 * hh + hh + (lane % hh);
-            const int c0 = (r / (2 * hh)) * hh;
+            const int rr = jcol & 63;
+            if (jcol < 64) {
+                const float er = s_g1[rr];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                if (c >= c0 && c < c0 + hh) {
-                    const int s = (c / hh) * 2 * hh + (c % hh);
-                    if (!isP) Af[r * 65 + s] = v[c];
-                    else *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_PBF + sw_elem(64, r, s)) = __float2bfloat16_rn(v[c]);
+                for (int c = 0; c < 32; ++c) {
+                    const int s = half * 32 + c;
+                    Af[rr * 65 + s] = (s < rr) ? v[c] * er : 0.f;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const int s = half * 32 + c;
+                    const int w = rr - s;
+                    v[c] = (w >= PBAND) ? v[c] : ((w >= 0) ? s_pband[rr * PBAND + w] : 0.f);
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(sm + OFF_PBF + sw_chunk(8192, rr, half * 4 + q4)) = pack8(v + q4 * 8);
+            }
+        } else {
+            // anchored levels: three GEMMs of two levels each
+            for (int p = 0; p < 3; ++p) {
+                const int lvl = 2 * p + 1 + (tid >> 7), slot = tid >> 7;
+                const int u = tid & 127, tg = u >> 4, cg = u & 15;
+                switch (lvl) {
+                case 1: build_level<32>(x, slot, tg, cg); break;
+                case 2: build_level<16>(x, slot, tg, cg); break;
+                case 3: build_level<8>(x, slot, tg, cg); break;
+                case 4: build_level<4>(x, slot, tg, cg); break;
+                case 5: build_level<2>(x, slot, tg, cg); break;
+                default: build_level<1>(x, slot, tg, cg); break;
+                }
+                publish();
+                if (tid == 0) {
+                    tc_fence_after();
+                    const uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(tbase + tm_lvl(p), dK(sb + OFF_LA, 16384, kk), dK(sb + OFF_LB, 8192, kk), idesc,
+                                 kk > 0);
+                    mma_commit(bar_mma);
+                }
+                wait_mma();
+            }
+            if (tid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
+            for (int e = tid; e < 64 * 65; e += NT) Af[e] = 0.f;
+            for (int e = tid; e < 512; e += NT)
+                *reinterpret_cast<uint4 *>(sm + OFF_PBF + e * 16) = make_uint4(0, 0, 0, 0);
+            __syncthreads();
+            for (int p = half; p < 3; p += 2) {
+                const int lvl = 2 * p + 1 + (quarter & 1);
+                const bool isP = quarter >= 2;
+                float v[32];
+                tmem_ld32(tbase + lane_base + tm_lvl(p) + (quarter & 1) * 32, v);
+                tmem_wait_ld();
+                switch (lvl) {
+                case 1: scatter_level<32>(sm, Af, s_g1, isP, lane, v); break;
+                case 2: scatter_level<16>(sm, Af, s_g1, isP, lane, v); break;
+                case 3: scatter_level<8>(sm, Af, s_g1, isP, lane, v); break;
+                case 4: scatter_level<4>(sm, Af, s_g1, isP, lane, v); break;
+                case 5: scatter_level<2>(sm, Af, s_g1, isP, lane, v); break;
+                default: scatter_level<1>(sm, Af, s_g1, isP, lane, v); break;
                 }
             }
+            __syncthreads();
+            if (tid < C) {
+#pragma unroll
+                for (int w = 0; w < PBAND; ++w)
+                    if (tid - w >= 0)
+                        *reinterpret_cast<unsigned short *>(sm + OFF_PBF + sw_elem(8192, tid, tid - w)) =
+                            bf16_bits(s_pband[tid * PBAND + w]);
+            }
         }
-        if (tid < C) *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_PBF + sw_elem(64, tid, tid)) =
-            __float2bfloat16_rn(s_pdiag[tid]);
         tc_fence_before();
         __syncthreads();
 
-        // ===== 3. T = (I + A)^{-1}: 16x16 diagonal blocks, then block rows ====
-        if (tid < 64) {
+        // ===== 3. T = (I + A)^{-1} =============================================
+        if (tid < 64) {   // 16x16 diagonal blocks by forward substitution, one column per thread
             const int I = tid >> 4, c = tid & 15;
-            float x[16];
+            float xv[16];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                if (rr < c) x[rr] = 0.f;
-                else if (rr == c) x[rr] = 1.f;
+            for (int r2 = 0; r2 < 16; ++r2) {
+                if (r2 < c) xv[r2] = 0.f;
+                else if (r2 == c) xv[r2] = 1.f;
                 else {
-                    float acc = 0.f;
+                    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                    for (int ss = 0; ss < rr; ++ss) acc = fmaf(Af[(16 * I + rr) * 65 + 16 * I + ss], x[ss], acc);
-                    x[rr] = -acc;
+                    for (int s2 = 0; s2 < r2; s2 += 2) {
+                        acc0 = fmaf(Af[(16 * I + r2) * 65 + 16 * I + s2], xv[s2], acc0);
+                        if (s2 + 1 < r2) acc1 = fmaf(Af[(16 * I + r2) * 65 + 16 * I + s2 + 1], xv[s2 + 1], acc1);
+                    }
+                    xv[r2] = -(acc0 + acc1);
                 }
             }
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) Tf[(16 * I + rr) * 65 + 16 * I + c] = x[rr];
+            for (int r2 = 0; r2 < 16; ++r2) Tf[(16 * I + r2) * 65 + 16 * I + c] = xv[r2];
+            // zeros above the diagonal blocks, so the merges below can run over full ranges
+            for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * 65 + 16 * I + c] = 0.f;
         }
         __syncthreads();
-        for (int d = 1; d < 4; ++d) {
-            const int nel = (4 - d) * 256;
-            for (int e = tid; e < nel; e += NT) {
-                const int J = e >> 8, I = J + d, rr = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-                for (int uu = 16 * J; uu < 16 * I; ++uu)
-                    acc = fmaf(Af[(16 * I + rr) * 65 + uu], Tf[uu * 65 + 16 * J + cc], acc);
-                Xs[e] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nel; e += NT) {
-                const int J = e >> 8, I = J + d, rr = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(Tf[(16 * I + rr) * 65 + 16 * I + m], Xs[(J << 8) + m * 16 + cc], acc);
-                Tf[(16 * I + rr) * 65 + 16 * J + cc] = -acc;
-            }
-            __syncthreads();
-        }
+        // 32x32 diagonal blocks: T[16(I+1):, 16I:] = -D_{I+1} A_{I+1,I} D_I, I = 0, 2 (two outputs per thread)
         {
+            const int r2 = (tid >> 4) & 15, c2 = tid & 15;
+            float acc[2] = {0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+                    const int I = 2 * blk;
+                    acc[blk] = fmaf(Af[(16 * I + 16 + r2) * 65 + 16 * I + m], Tf[(16 * I + m) * 65 + 16 * I + c2], acc[blk]);
+                }
+            }
+            Xs[tid] = acc[0];
+            Xs[256 + tid] = acc[1];
+        }
+        __syncthreads();
+        {
+            const int r2 = (tid >> 4) & 15, c2 = tid & 15;
+            float acc[2] = {0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+#pragma unroll
+                for (int blk = 0; blk < 2; ++blk) {
+                    const int I = 2 * blk;
+                    acc[blk] = fmaf(Tf[(16 * I + 16 + r2) * 65 + 16 * I + 16 + m], Xs[(blk << 8) + m * 16 + c2], acc[blk]);
+                }
+            }
+            Tf[(16 + r2) * 65 + c2] = -acc[0];
+            Tf[(48 + r2) * 65 + 32 + c2] = -acc[1];
+        }
+        __syncthreads();
+        // T[32:, :32] = -T2 A21 T1 (four outputs per thread: rows r0 + 8k, column c2)
+        {
+            const int r0 = tid >> 5, c2 = tid & 31;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const float t = Tf[m * 65 + c2];
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) acc[k4] = fmaf(Af[(32 + r0 + 8 * k4) * 65 + m], t, acc[k4]);
+            }
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) Xs[(r0 + 8 * k4) * 32 + c2] = acc[k4];
+        }
+        __syncthreads();
+        {
+            const int r0 = tid >> 5, c2 = tid & 31;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                const float xm = Xs[m * 32 + c2];
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) acc[k4] = fmaf(Tf[(32 + r0 + 8 * k4) * 65 + 32 + m], xm, acc[k4]);
+            }
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + r0 + 8 * k4) * 65 + c2] = -acc[k4];
+        }
+        __syncthreads();
+        {   // bf16 K-major copies T Diag(e) and T Diag(w), zero above the diagonal
             const int r = tid >> 2, kc0 = (tid & 3) * 2;
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
-                float t8[8];
+                float te[8], tw[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) t8[c] = Tf[r * 65 + (kc0 + q2) * 8 + c];
-                *reinterpret_cast<uint4 *>(sm + OFF_TBF + sw_chunk(64, r, kc0 + q2)) = pack8(t8);
+                for (int c = 0; c < 8; ++c) {
+                    const int s = (kc0 + q2) * 8 + c;
+                    const float t = (s <= r) ? Tf[r * 65 + s] : 0.f;
+                    te[c] = t * s_g1[s];
+                    tw[c] = t * s_g2[s];
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_TBF + sw_chunk(8192, r, kc0 + q2)) = pack8(te);
+                *reinterpret_cast<uint4 *>(sm + OFF_UT + sw_chunk(8192, r, kc0 + q2)) = pack8(tw);
             }
         }
         publish();
 
-        // ===== 4. W = T (Gamma (.) A~)  and  U^T = M^T T^T ====================
+        // ===== 4. W = T (row operand a~ part);  U^T = M^T T^T ================
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id_w = idesc_bf16(64, 128, false, true);
             const uint32_t id_u = idesc_bf16(128, 64, true, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16(tbase + TM_W, dK(sb + OFF_TBF, 64, kk), dMN(sb + OFF_AG, kk), id_w, kk > 0);
-                mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, kk), dK(sb + OFF_TBF, 64, kk), id_u, kk > 0);
+                mma_bf16(tbase + TM_W, dK(sb + OFF_TBF, 8192, kk), dMN(sb + OFF_QA, 16384, kk), id_w, kk > 0);
+                mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_UT, 8192, kk), id_u, kk > 0);
             }
             mma_commit(bar_mma);
         }
+        // ===== 5. state pass (overlaps the MMAs above: D_S is not an operand) ===
+        {
+#pragma unroll
+            for (int c32 = 0; c32 < 2; ++c32) {
+                const int i0 = half * 64 + c32 * 32;
+                float s[32], t[32];
+                tmem_ld32(tbase + lane_base + TM_S + i0, s);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    t[e] = s[e] * s_gamC[i0 + e];
+                    if (fast) s[e] = t[e];
+                }
+                // bf16 operand copy of the state (scaled on the fast path)
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
+                tmem_st16(tbase + lane_base + TM_S + i0, t);
+                tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
+            }
+            tmem_wait_st();
+        }
         wait_mma();
-        // W (M = 64 layout: rows 16q..16q+15 in lanes 0..15 of quarter q) -> [token][channel] tile
+        if (tid == 0 && ch + 1 < nchunks) issue_tma_v(ch + 1);   // v consumed by U^T = M^T T^T
+        // W (M = 64 layout: rows 16q..16q+15 in lanes 0..15 of quarter q) -> rows 0-63 of QA
         {
             const int r = quarter * 16 + (lane & 15);
-            const int chalf = warp >> 2;
 #pragma unroll
             for (int c32 = 0; c32 < 2; ++c32) {
                 float v[32];
-                tmem_ld32(tbase + lane_base + TM_W + chalf * 64 + c32 * 32, v);
+                tmem_ld32(tbase + lane_base + TM_W + half * 64 + c32 * 32, v);
                 tmem_wait_ld();
                 if (lane < 16) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int kc = chalf * 8 + c32 * 4 + q4;
-                        *reinterpret_cast<uint4 *>(sm + OFF_AG + sw_chunk(64, r, kc)) = pack8(v + q4 * 8);
-                    }
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, r, half * 8 + c32 * 4 + q4)) =
+                            pack8(v + q4 * 8);
                 }
             }
         }
         publish();
 
-        // ===== 5. U^T -= S0^T W^T ;  O^T = S0^T (Gamma (.) Q)^T ==============
+        // ===== 6. U^T -= S^T W^T ;  O^T = S^T Q^T =============================
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id_neg = idesc_bf16(128, 64, false, false, true);
             const uint32_t id_pos = idesc_bf16(128, 64, false, false);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16(tbase + TM_U, dK(sb + OFF_S0T, 128, kk), dK(sb + OFF_AG, 64, kk), id_neg, 1);
-                mma_bf16(tbase + TM_O, dK(sb + OFF_S0T, 128, kk), dK(sb + OFF_QG, 64, kk), id_pos, kk > 0);
+                mma_bf16(tbase + TM_U, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA, 16384, kk), id_neg, 1);
+                mma_bf16(tbase + TM_O, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA + 8192, 16384, kk), id_pos,
+                         kk > 0);
             }
             mma_commit(bar_mma);
         }
         wait_mma();
-        {
-            const int j = quarter * 32 + lane, shalf = warp >> 2;
-            // U^T row j, tokens [32*shalf, +32) -> bf16 K-major tile (rows j, K = token)
+        {   // U^T row j, tokens [32*half, +32) -> bf16 K-major tile (rows j, K = token)
             float v[32];
-            tmem_ld32(tbase + lane_base + TM_U + shalf * 32, v);
+            tmem_ld32(tbase + lane_base + TM_U + half * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4 *>(sm + OFF_MT + sw_chunk(128, j, shalf * 4 + q4)) = pack8(v + q4 * 8);
-            // S^T row j, key channels [64*shalf, +64): scale by Gamma_C
-#pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
-                const int i0 = shalf * 64 + c32 * 32;
-                float s[32];
-                tmem_ld32(tbase + lane_base + TM_S + i0, s);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[e] *= s_gamC[i0 + e];
-                tmem_st16(tbase + lane_base + TM_S + i0, s);
-                tmem_st16(tbase + lane_base + TM_S + i0 + 16, s + 16);
-            }
-            tmem_wait_st();
+                *reinterpret_cast<uint4 *>(sm + OFF_UT + sw_chunk(16384, jcol, half * 4 + q4)) = pack8(v + q4 * 8);
         }
         publish();
 
-        // ===== 6. O^T += U^T P^T ;  S^T += U^T Kbar ==========================
+        // ===== 7. O^T += U^T P^T ;  S^T += U^T Kbar ===========================
         if (tid == 0) {
             tc_fence_after();
             const uint32_t id_o = idesc_bf16(128, 64, false, false);
             const uint32_t id_s = idesc_bf16(128, 128, false, true);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16(tbase + TM_O, dK(sb + OFF_MT, 128, kk), dK(sb + OFF_PBF, 64, kk), id_o, 1);
-                mma_bf16(tbase + TM_S, dK(sb + OFF_MT, 128, kk), dMN(sb + OFF_KB, kk), id_s, 1);
+                mma_bf16(tbase + TM_O, dK(sb + OFF_UT, 16384, kk), dK(sb + OFF_PBF, 8192, kk), id_o, 1);
+                mma_bf16(tbase + TM_S, dK(sb + OFF_UT, 16384, kk), dMN(sb + OFF_KB, 8192, kk), id_s, 1);
             }
             mma_commit(bar_mma);
         }
         wait_mma();
-        {
-            const int j = quarter * 32 + lane, shalf = warp >> 2;
+        {   // o: TMEM (lane j, column r) -> bf16 staging [r][j] -> 16-byte rows to HBM
             float v[32];
-            tmem_ld32(tbase + lane_base + TM_O + shalf * 32, v);
+            tmem_ld32(tbase + lane_base + TM_O + half * 32, v);
             tmem_wait_ld();
+            unsigned short *ost = reinterpret_cast<unsigned short *>(sm + OFF_OST);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int r = shalf * 32 + e;
-                if (r < nvalid) op[((rowbase + r) * H + h) * D + j] = __float2bfloat16_rn(v[e]);
-            }
-#pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
-                const int i0 = shalf * 64 + c32 * 32;
-                float s[32];
-                tmem_ld32(tbase + lane_base + TM_S + i0, s);
-                tmem_wait_ld();
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(128, j, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
-            }
+            for (int e = 0; e < 32; ++e) ost[(half * 32 + e) * 128 + jcol] = bf16_bits(v[e]);
+        }
+        __syncthreads();
+        for (int e = tid; e < nvalid * 16; e += NT) {
+            const int r = e >> 4, cgo = e & 15;
+            *reinterpret_cast<uint4 *>(op + (((rowbase + r) * H + h) * D + cgo * 8) * 2) =
+                *reinterpret_cast<const uint4 *>(sm + OFF_OST + r * 256 + cgo * 16);
         }
         fence_async_smem();
         tc_fence_before();
         ok = __syncthreads_and(ok) != 0;  // every thread leaves the loop together
     }
 
-    // ---- final state (or NaN if an internal wait timed out) ----------------
+    // ---- final state (NaN if an internal wait timed out) ----------------------
     tc_fence_after();
     if (a.sf) {
         const size_t soff = ((size_t)n * H + h) * D * D;
-        const int j = quarter * 32 + lane, shalf = warp >> 2;
 #pragma unroll
         for (int c32 = 0; c32 < 2; ++c32) {
-            const int i0 = shalf * 64 + c32 * 32;
+            const int i0 = half * 64 + c32 * 32;
             float s[32];
             tmem_ld32(tbase + lane_base + TM_S + i0, s);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) a.sf[soff + (size_t)(i0 + e) * D + j] = ok ? s[e] : __int_as_float(0x7fc00000);
+            for (int e = 0; e < 32; ++e)
+                a.sf[soff + (size_t)(i0 + e) * D + jcol] = ok ? s[e] : __int_as_float(0x7fc00000);
         }
     }
-    if (!ok) {
-        // drain any TMA still in flight (bounded) before the CTA's shared memory is released
+    if (!ok) {  // drain TMA still in flight (bounded)
         mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
+        mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
     }
     tc_fence_before();
     __syncthreads();
@@ -705,16 +890,18 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-bool make_map(CUtensorMap *m, const void *base, long long rows, int H)
+// [rows = B*T][H][128] bf16; box {inner, 1, 64}; inner 128 without swizzle (row-major
+// tile) or 64 with the 128-byte swizzle (one K-major / MN-major operand panel)
+bool make_map(CUtensorMap *m, const void *base, long long rows, int H, bool swizzle)
 {
     cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
     cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    cuuint32_t box[3] = {128, 1, 64}, es[3] = {1, 1, 1};
+    cuuint32_t box[3] = {swizzle ? 64u : 128u, 1, 64}, es[3] = {1, 1, 1};
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -741,8 +928,8 @@ cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
     p.a = a;
     const long long rows = (long long)a.B * a.T;
     if (rows > 0) {
-        if (!make_map(&p.tq, a.q, rows, a.H) || !make_map(&p.tk, a.k, rows, a.H) ||
-            !make_map(&p.tv, a.v, rows, a.H) || !make_map(&p.ta, a.alpha, rows, a.H))
+        if (!make_map(&p.tq, a.q, rows, a.H, false) || !make_map(&p.tk, a.k, rows, a.H, false) ||
+            !make_map(&p.tv, a.v, rows, a.H, true) || !make_map(&p.ta, a.alpha, rows, a.H, false))
             return cudaErrorInvalidValue;
     }
     const int N = a.cu_seqlens ? a.num_seqs : a.B;
