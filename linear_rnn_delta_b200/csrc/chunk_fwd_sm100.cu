@@ -72,13 +72,14 @@ constexpr uint32_t OFF_MT = 147456;   // M [token][channel]: v by 128B-swizzled 
 constexpr uint32_t OFF_F = 163840;    // anchored-path level factors | A, T fp32, T, P bf16 | o staging
 constexpr uint32_t OFF_LA = OFF_F;            // level row factors: 128 rows x 128 ch
 constexpr uint32_t OFF_LB = OFF_F + 32768;    // level column factors: 64 rows x 128 ch
-constexpr uint32_t OFF_AF32 = OFF_F;          // A fp32 [64][65]
-constexpr uint32_t OFF_TF32 = OFF_F + 16640;  // T fp32 [64][65]
-constexpr uint32_t OFF_X = OFF_F + 33280;     // 32 x 32 fp32 scratch of the block solve
-constexpr uint32_t OFF_TBF = OFF_F + 37888;   // T Diag(e) bf16 64 x 64 K-major
-constexpr uint32_t OFF_PBF = OFF_F + 46080;   // P bf16 64 x 64 K-major
+constexpr int TP = 68;                        // pitch (floats) of the fp32 A and T tiles: 16-byte rows
+constexpr uint32_t OFF_AF32 = OFF_F;          // A fp32 [64][TP]
+constexpr uint32_t OFF_TF32 = OFF_F + 17408;  // T fp32 [64][TP]
+constexpr uint32_t OFF_X = OFF_F + 34816;     // 32 x 32 fp32 scratch of the block solve
+constexpr uint32_t OFF_TBF = OFF_F + 38912;   // T Diag(e) bf16 64 x 64 K-major
+constexpr uint32_t OFF_PBF = OFF_F + 47104;   // P bf16 64 x 64 K-major
 constexpr uint32_t OFF_OST = OFF_F;           // o staging [64][128] bf16 (A, T dead by then)
-constexpr uint32_t OFF_MISC = OFF_F + 54272;
+constexpr uint32_t OFF_MISC = OFF_F + 55296;
 constexpr int PBAND = 5;   // P_{r,s} for r-4 <= s <= r computed exactly (SIMT) from the bf16 inputs
 constexpr uint32_t M_G1 = OFF_MISC, M_G2 = OFF_MISC + 256, M_GAMC = OFF_MISC + 512, M_TOT = OFF_MISC + 1024,
                    M_PBAND = OFF_MISC + 5120, M_BAR = OFF_MISC + 6400, M_TMEM = OFF_MISC + 6432;
@@ -264,7 +265,7 @@ __device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const floa
     for (int c = 0; c < 32; ++c) {
         if (c >= c0 && c < c0 + HH) {
             const int s = (c / HH) * BS + (c % HH);
-            if (!isP) Af[r * 65 + s] = v[c] * s_e[r];
+            if (!isP) Af[r * TP + s] = v[c] * s_e[r];
             else *reinterpret_cast<unsigned short *>(sm + OFF_PBF + sw_elem(8192, r, s)) = bf16_bits(v[c]);
         }
     }
@@ -365,22 +366,31 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     tc_fence_before();
     __syncthreads();
 
+    // scalar erase / write gates of a chunk's row `tid` (1 for GDN-2, 0 past the end),
+    // fetched one chunk ahead into registers so the load latency is hidden
+    auto fetch_gates = [&](int chunk, float &ge, float &gw) {
+        const int r = tid, nv = min(C, len - chunk * C);
+        const size_t tok = ((size_t)b * a.T + t0 + chunk * C + r) * H + h;
+        const bool v = r < nv;
+        if (gdn2) { ge = v ? 1.f : 0.f; gw = ge; }
+        else {
+            ge = v ? bf2f(g1p, tok) : 0.f;
+            gw = v ? (a.variant == KDA ? ge : bf2f(g2p, tok)) : 0.f;
+        }
+    };
+    float gate_e = 0.f, gate_w = 0.f;
+    if (tid < C && nchunks > 0) fetch_gates(0, gate_e, gate_w);
+
     for (int ch = 0; ch < nchunks && ok; ++ch) {
         const int tok0 = t0 + ch * C;
         const int nvalid = min(C, len - ch * C);
         const size_t rowbase = (size_t)b * a.T + tok0;   // packed token index of chunk row 0
         const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
 
-        if (tid < C) {  // scalar erase / write gates (1 for GDN-2), 0 past the sequence end
-            const bool v = tid < nvalid;
-            const size_t tok = (rowbase + tid) * H + h;
-            if (gdn2) {
-                s_g1[tid] = v ? 1.f : 0.f;
-                s_g2[tid] = v ? 1.f : 0.f;
-            } else {
-                s_g1[tid] = v ? bf2f(g1p, tok) : 0.f;
-                s_g2[tid] = v ? (a.variant == KDA ? bf2f(g1p, tok) : bf2f(g2p, tok)) : 0.f;
-            }
+        if (tid < C) {
+            s_g1[tid] = gate_e;
+            s_g2[tid] = gate_w;
+            if (ch + 1 < nchunks) fetch_gates(ch + 1, gate_e, gate_w);
         }
         if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
         ph_tma ^= 1;
@@ -412,37 +422,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             *reinterpret_cast<float4 *>(s_tot + tg * 128 + cg * 8 + 4) = make_float4(tot[4], tot[5], tot[6], tot[7]);
         } else {
             const int u = tid - 128, tg = u >> 4, cg = u & 15;
-            {   // band of P: P_{r,r-w} = sum_c q_rc (alpha_r ... alpha_{r-w+1})_c k_{r-w,c}, w = 0..4,
-                // from the bf16 inputs in fp32 (the entries the bf16 GEMM would round most
-                // harmfully); two threads per row, 64 channels each
-                const int r = u >> 1, hf = u & 1;
-                float acc[PBAND];
-#pragma unroll
-                for (int w = 0; w < PBAND; ++w) acc[w] = 0.f;
-                for (int cc = 0; cc < 8; ++cc) {
-                    const int cgx = hf * 8 + ((cc + r) & 7);   // staggered by row: conflict-free loads
-                    float hv[8], kv[8], av[8];
-                    unpack8(raw_row(sm, RAW_Q, r, cgx), hv);
-#pragma unroll
-                    for (int w = 0; w < PBAND; ++w) {
-                        if (r - w >= 0) {
-                            unpack8(raw_row(sm, RAW_K, r - w, cgx), kv);
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) acc[w] = fmaf(hv[c], kv[c], acc[w]);
-                            if (w + 1 < PBAND && r - w - 1 >= 0) {
-                                unpack8(raw_row(sm, RAW_A, r - w, cgx), av);
-#pragma unroll
-                                for (int c = 0; c < 8; ++c) hv[c] *= av[c];
-                            }
-                        }
-                    }
-                }
-#pragma unroll
-                for (int w = 0; w < PBAND; ++w) {
-                    const float tot = acc[w] + __shfl_xor_sync(0xffffffffu, acc[w], 1);
-                    if (hf == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? tot : 0.f;
-                }
-            }
             if (gdn2) {   // M = w (.) v, in place in the swizzled v tile (rows past the end -> 0)
 #pragma unroll 2
                 for (int i = 0; i < 8; ++i) {
@@ -485,9 +464,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
         }
         const bool fast = (__syncthreads_and(gam_ok) != 0) && in_range;
 
-        // ===== 1b. row operands (Gamma a~, Gamma q, scaled on the fast path) | Kbar
+        // ===== 1b. row operands (Gamma a~ | Gamma q, scaled on the fast path), Kbar, band of P
         {
             const int u = tid & 127, tg = u >> 4, cg = u & 15;
+            const bool grp0 = tid < 128;
             float pre[8], suf[8];
 #pragma unroll
             for (int c = 0; c < 8; ++c) { pre[c] = 1.f; suf[c] = 1.f; }
@@ -501,33 +481,35 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     else suf[c] *= t8[c];
                 }
             }
-            if (tid < 128) {
+            {   // forward: group 0 writes rows 0-63 (Gamma a~), group 1 rows 64-127 (Gamma q)
                 float sc[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) sc[c] = fast ? pre[c] * (1.0f / s_gamC[cg * 8 + c]) : pre[c];
-#pragma unroll 2
+#pragma unroll 4
                 for (int i = 0; i < 8; ++i) {
                     const int r = tg * 8 + i;
                     const bool v = r < nvalid;
-                    float al[8], qv[8], kv[8], e[8], ga[8], gq[8];
+                    float al[8], xv[8], e[8], o8[8];
                     unpack8(raw_row(sm, RAW_A, r, cg), al);
-                    unpack8(raw_row(sm, RAW_Q, r, cg), qv);
-                    unpack8(raw_row(sm, RAW_K, r, cg), kv);
-                    erase_gate(x, r, cg, e);
+                    unpack8(raw_row(sm, grp0 ? RAW_K : RAW_Q, r, cg), xv);
+                    if (grp0) erase_gate(x, r, cg, e);
+                    else {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) e[c] = 1.f;
+                    }
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         sc[c] *= v ? al[c] : 1.f;
-                        ga[c] = v ? sc[c] * (e[c] * kv[c]) : 0.f;
-                        gq[c] = v ? sc[c] * qv[c] : 0.f;
+                        o8[c] = v ? sc[c] * (e[c] * xv[c]) : 0.f;
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, r, cg)) = pack8(ga);
-                    *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, 64 + r, cg)) = pack8(gq);
+                    *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, (grp0 ? 0 : 64) + r, cg)) = pack8(o8);
                 }
-            } else {
+            }
+            if (grp0) {   // backward: Kbar_s = (prod_{s<t<C} alpha_t) (.) k_s
                 float sx[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) sx[c] = suf[c];
-#pragma unroll 2
+#pragma unroll 4
                 for (int i = 7; i >= 0; --i) {
                     const int r = tg * 8 + i;
                     const bool v = r < nvalid;
@@ -542,7 +524,42 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     *reinterpret_cast<uint4 *>(sm + OFF_KB + sw_chunk(8192, r, cg)) = pack8(kb);
                 }
             }
+            {   // band of P: P_{r,r-w} = sum_c q_rc (alpha_r ... alpha_{r-w+1})_c k_{r-w,c}, w = 0..4,
+                // from the bf16 inputs in fp32: the entries whose bf16 GEMM rounding would hurt most.
+                // Four threads per row (32 channels each), chunk order staggered by row so the
+                // loads are bank-conflict free; rows below w are clamped and masked afterwards.
+                const int r = tid >> 2, cq = tid & 3;
+                float acc[PBAND];
+#pragma unroll
+                for (int w = 0; w < PBAND; ++w) acc[w] = 0.f;
+#pragma unroll 2
+                for (int j = 0; j < 4; ++j) {
+                    const int cgx = cq * 4 + ((j + r) & 3);
+                    float hv[8];
+                    unpack8(raw_row(sm, RAW_Q, r, cgx), hv);
+#pragma unroll
+                    for (int w = 0; w < PBAND; ++w) {
+                        float kv[8];
+                        unpack8(raw_row(sm, RAW_K, max(r - w, 0), cgx), kv);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) acc[w] = fmaf(hv[c], kv[c], acc[w]);
+                        if (w + 1 < PBAND) {
+                            float av[8];
+                            unpack8(raw_row(sm, RAW_A, max(r - w, 0), cgx), av);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) hv[c] *= av[c];
+                        }
+                    }
+                }
+#pragma unroll
+                for (int w = 0; w < PBAND; ++w) {
+                    float t = acc[w] + __shfl_xor_sync(0xffffffffu, acc[w], 1);
+                    t += __shfl_xor_sync(0xffffffffu, t, 2);
+                    if (cq == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? t : 0.f;
+                }
+            }
         }
+        __syncthreads();   // band and row operands complete before either A/P path reads them
 
         // ===== 2. A and P ======================================================
         if (fast) {
@@ -567,7 +584,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 #pragma unroll
                 for (int c = 0; c < 32; ++c) {
                     const int s = half * 32 + c;
-                    Af[rr * 65 + s] = (s < rr) ? v[c] * er : 0.f;
+                    Af[rr * TP + s] = (s < rr) ? v[c] * er : 0.f;
                 }
             } else {
 #pragma unroll
@@ -606,7 +623,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                 wait_mma();
             }
             if (tid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
-            for (int e = tid; e < 64 * 65; e += NT) Af[e] = 0.f;
+            for (int e = tid; e < 64 * TP; e += NT) Af[e] = 0.f;
             for (int e = tid; e < 512; e += NT)
                 *reinterpret_cast<uint4 *>(sm + OFF_PBF + e * 16) = make_uint4(0, 0, 0, 0);
             __syncthreads();
@@ -638,85 +655,110 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
         __syncthreads();
 
         // ===== 3. T = (I + A)^{-1} =============================================
-        if (tid < 64) {   // 16x16 diagonal blocks by forward substitution, one column per thread
+        // 16x16 diagonal blocks by forward substitution (one column per thread), then
+        // recursive doubling: T[16(I+1):, 16I:] = -D_{I+1} A_{I+1,I} D_I for I = 0, 2, and
+        // T[32:, :32] = -T2 A21 T1.  fp32 throughout; A rows read four at a time.
+        if (tid < 64) {
             const int I = tid >> 4, c = tid & 15;
             float xv[16];
 #pragma unroll
             for (int r2 = 0; r2 < 16; ++r2) {
-                if (r2 < c) xv[r2] = 0.f;
-                else if (r2 == c) xv[r2] = 1.f;
-                else {
-                    float acc0 = 0.f, acc1 = 0.f;
+                float arow[16];
 #pragma unroll
-                    for (int s2 = 0; s2 < r2; s2 += 2) {
-                        acc0 = fmaf(Af[(16 * I + r2) * 65 + 16 * I + s2], xv[s2], acc0);
-                        if (s2 + 1 < r2) acc1 = fmaf(Af[(16 * I + r2) * 65 + 16 * I + s2 + 1], xv[s2 + 1], acc1);
-                    }
-                    xv[r2] = -(acc0 + acc1);
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<float4 *>(arow + 4 * q4) =
+                        *reinterpret_cast<const float4 *>(Af + (16 * I + r2) * TP + 16 * I + 4 * q4);
+                float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int s2 = 0; s2 < r2; ++s2) {
+                    if (s2 & 1) acc1 = fmaf(arow[s2], xv[s2], acc1);
+                    else acc0 = fmaf(arow[s2], xv[s2], acc0);
                 }
+                xv[r2] = (r2 < c) ? 0.f : ((r2 == c) ? 1.f : -(acc0 + acc1));
             }
 #pragma unroll
-            for (int r2 = 0; r2 < 16; ++r2) Tf[(16 * I + r2) * 65 + 16 * I + c] = xv[r2];
-            // zeros above the diagonal blocks, so the merges below can run over full ranges
-            for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * 65 + 16 * I + c] = 0.f;
+            for (int r2 = 0; r2 < 16; ++r2) Tf[(16 * I + r2) * TP + 16 * I + c] = xv[r2];
+            for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * TP + 16 * I + c] = 0.f;  // above the block
         }
         __syncthreads();
-        // 32x32 diagonal blocks: T[16(I+1):, 16I:] = -D_{I+1} A_{I+1,I} D_I, I = 0, 2 (two outputs per thread)
-        {
+        {   // X = A_{I+1,I} D_I for I = 0, 2 (two outputs per thread)
             const int r2 = (tid >> 4) & 15, c2 = tid & 15;
             float acc[2] = {0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
+            for (int m4 = 0; m4 < 4; ++m4) {
 #pragma unroll
                 for (int blk = 0; blk < 2; ++blk) {
                     const int I = 2 * blk;
-                    acc[blk] = fmaf(Af[(16 * I + 16 + r2) * 65 + 16 * I + m], Tf[(16 * I + m) * 65 + 16 * I + c2], acc[blk]);
+                    const float4 av = *reinterpret_cast<const float4 *>(Af + (16 * I + 16 + r2) * TP + 16 * I + 4 * m4);
+                    const float *tcol = Tf + (16 * I + 4 * m4) * TP + 16 * I + c2;
+                    acc[blk] = fmaf(av.x, tcol[0], acc[blk]);
+                    acc[blk] = fmaf(av.y, tcol[TP], acc[blk]);
+                    acc[blk] = fmaf(av.z, tcol[2 * TP], acc[blk]);
+                    acc[blk] = fmaf(av.w, tcol[3 * TP], acc[blk]);
                 }
             }
             Xs[tid] = acc[0];
             Xs[256 + tid] = acc[1];
         }
         __syncthreads();
-        {
+        {   // T_{I+1,I} = -D_{I+1} X
             const int r2 = (tid >> 4) & 15, c2 = tid & 15;
             float acc[2] = {0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
+            for (int m4 = 0; m4 < 4; ++m4) {
 #pragma unroll
                 for (int blk = 0; blk < 2; ++blk) {
                     const int I = 2 * blk;
-                    acc[blk] = fmaf(Tf[(16 * I + 16 + r2) * 65 + 16 * I + 16 + m], Xs[(blk << 8) + m * 16 + c2], acc[blk]);
+                    const float4 tv = *reinterpret_cast<const float4 *>(Tf + (16 * I + 16 + r2) * TP + 16 * I + 16 + 4 * m4);
+                    const float *xcol = Xs + (blk << 8) + (4 * m4) * 16 + c2;
+                    acc[blk] = fmaf(tv.x, xcol[0], acc[blk]);
+                    acc[blk] = fmaf(tv.y, xcol[16], acc[blk]);
+                    acc[blk] = fmaf(tv.z, xcol[32], acc[blk]);
+                    acc[blk] = fmaf(tv.w, xcol[48], acc[blk]);
                 }
             }
-            Tf[(16 + r2) * 65 + c2] = -acc[0];
-            Tf[(48 + r2) * 65 + 32 + c2] = -acc[1];
+            Tf[(16 + r2) * TP + c2] = -acc[0];
+            Tf[(48 + r2) * TP + 32 + c2] = -acc[1];
         }
         __syncthreads();
-        // T[32:, :32] = -T2 A21 T1 (four outputs per thread: rows r0 + 8k, column c2)
-        {
+        {   // X = A21 T1 (rows r0 + 8k, column c2)
             const int r0 = tid >> 5, c2 = tid & 31;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const float t = Tf[m * 65 + c2];
+            for (int m4 = 0; m4 < 8; ++m4) {
+                const float *tcol = Tf + (4 * m4) * TP + c2;
+                const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) acc[k4] = fmaf(Af[(32 + r0 + 8 * k4) * 65 + m], t, acc[k4]);
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + r0 + 8 * k4) * TP + 4 * m4);
+                    acc[k4] = fmaf(av.x, t0v, acc[k4]);
+                    acc[k4] = fmaf(av.y, t1v, acc[k4]);
+                    acc[k4] = fmaf(av.z, t2v, acc[k4]);
+                    acc[k4] = fmaf(av.w, t3v, acc[k4]);
+                }
             }
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) Xs[(r0 + 8 * k4) * 32 + c2] = acc[k4];
         }
         __syncthreads();
-        {
+        {   // T21 = -T2 X
             const int r0 = tid >> 5, c2 = tid & 31;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                const float xm = Xs[m * 32 + c2];
+            for (int m4 = 0; m4 < 8; ++m4) {
+                const float *xcol = Xs + (4 * m4) * 32 + c2;
+                const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) acc[k4] = fmaf(Tf[(32 + r0 + 8 * k4) * 65 + 32 + m], xm, acc[k4]);
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 tv = *reinterpret_cast<const float4 *>(Tf + (32 + r0 + 8 * k4) * TP + 32 + 4 * m4);
+                    acc[k4] = fmaf(tv.x, x0, acc[k4]);
+                    acc[k4] = fmaf(tv.y, x1, acc[k4]);
+                    acc[k4] = fmaf(tv.z, x2, acc[k4]);
+                    acc[k4] = fmaf(tv.w, x3, acc[k4]);
+                }
             }
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + r0 + 8 * k4) * 65 + c2] = -acc[k4];
+            for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + r0 + 8 * k4) * TP + c2] = -acc[k4];
         }
         __syncthreads();
         {   // bf16 K-major copies T Diag(e) and T Diag(w), zero above the diagonal
@@ -727,7 +769,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const int s = (kc0 + q2) * 8 + c;
-                    const float t = (s <= r) ? Tf[r * 65 + s] : 0.f;
+                    const float t = (s <= r) ? Tf[r * TP + s] : 0.f;
                     te[c] = t * s_g1[s];
                     tw[c] = t * s_g2[s];
                 }

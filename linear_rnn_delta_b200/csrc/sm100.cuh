@@ -177,21 +177,17 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, ui
         :: "r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(mbar)), "r"(c0), "r"(c1), "r"(c2) : "memory");
 }
 
-// fp32 -> bf16 round-to-nearest-even on the integer ALU (finite inputs; keeps
-// the conversion off the XU pipe).  Adding 0x7FFF plus the lowest kept bit to
-// the fp32 bit pattern and truncating is exactly RNE for finite values.
-__device__ __forceinline__ uint32_t bf16_rne_bits(float x)
-{
-    const uint32_t u = __float_as_uint(x);
-    return u + 0x7FFFu + ((u >> 16) & 1u);
-}
+// fp32 -> bf16 round-to-nearest-even: two values per instruction (lo in the
+// low half).
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
 {
-    return __byte_perm(bf16_rne_bits(lo), bf16_rne_bits(hi), 0x7632);
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
 }
 __device__ __forceinline__ unsigned short bf16_bits(float x)
 {
-    return (unsigned short)(bf16_rne_bits(x) >> 16);
+    return (unsigned short)(pack_bf16(x, 0.f) & 0xFFFFu);
 }
 
 }  // namespace sm100
