@@ -74,6 +74,33 @@ def decode_algorithmic(N, H, dk, dv, elem=2, variant="kda") -> dict:
 # Device helpers
 # ---------------------------------------------------------------------------
 
+def source_digest(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+CHUNK_SOURCES = ["linear_rnn_delta_b200/csrc/chunk_fwd_sm100.cu", "linear_rnn_delta_b200/csrc/sm100.cuh",
+                 "linear_rnn_delta_b200/csrc/common.cuh"]
+DECODE_SOURCES = ["linear_rnn_delta_b200/csrc/decode_step.cu", "linear_rnn_delta_b200/csrc/common.cuh"]
+
+
+def measured_traffic(name: str, sources) -> dict:
+    """DRAM bytes per launch from a committed ncu summary (profiles/traffic.json),
+    only while the kernel's sources still hash to what was profiled."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return {}
+    with open(p) as f:
+        d = json.load(f).get(name)
+    if not d or d.get("source_sha256") != source_digest(sources):
+        return {}
+    return d
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -97,13 +124,20 @@ class ClockSampler:
         self.path = None
 
     def start(self):
+        """Start sampling and wait until the first sample is written, so that
+        nvidia-smi's start-up never overlaps the timed region."""
         try:
             fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.25)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while time.time() - t0 < 20.0:
+                if os.path.getsize(self.path) > 0:
+                    break
+                time.sleep(0.05)
+            time.sleep(0.2)
         except Exception:
             self.proc = None
 
@@ -160,12 +194,20 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Slowest rank's time: the job finishes when every rank has."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_workload_seed(rank: int) -> int:
+    """Weak scaling: every rank owns an independent batch of (sequence, head)
+    units drawn with its own seed; no data crosses ranks."""
+    return rank
 
 
 # ---------------------------------------------------------------------------
@@ -290,7 +332,8 @@ def run_decode_workload(steps, warmup, world, peaks, rank, N=256, H=32, dk=128, 
            "ms_per_step": total / steps * 1e3, "p50_ms": pct(per, 50) * 1e3, "p95_ms": pct(per, 95) * 1e3,
            "p99_ms": pct(per, 99) * 1e3,
            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                        "frac": gbs / peaks["hbm_gbs"],
+                        "traffic": measured_traffic("decode_ckda_256x32", DECODE_SOURCES).get("dram_bytes_per_launch"),
                         "peak_source": peaks["source"]},
            "bytes_per_step": alg["bytes"], "gpu_launches": steps}
     if e2e:
@@ -379,12 +422,12 @@ def reference_arm(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--extra", action="store_true", help="also time Complex-KDA 8x16x8192 and varlen RDA/GDN-2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--decode-steps", type=int, default=1024)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -397,7 +440,7 @@ def main():
 
     import linear_rnn_delta_b200  # noqa: F401  (fails loudly if the library is missing)
     peaks = load_peaks()
-    inp = W.kda_bf16(seed=rank)
+    inp = W.kda_bf16(seed=rank_workload_seed(rank))
     sampler = ClockSampler(local) if rank == 0 else None
     main_res = run_chunk_workload(inp, args.steps, args.warmup, world, peaks, sampler=sampler)
     decode = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank)
@@ -435,7 +478,8 @@ def main():
                    "l2": f"inputs {inp.nbytes() / 1e6:.0f} MB > L2 126 MB, no flush"},
         "p50_ms": main_res["p50_ms"], "p95_ms": main_res["p95_ms"], "p99_ms": main_res["p99_ms"],
         "roofline": {"bound": "hbm", "achieved": main_res["hbm"]["achieved"], "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": main_res["hbm"]["frac"], "traffic": None,
+                     "unit": "GB/s", "frac": main_res["hbm"]["frac"],
+                     "traffic": measured_traffic("chunk_fwd_kda_4x16x4096", CHUNK_SOURCES).get("dram_bytes_per_launch"),
                      "peak_source": peaks["source"],
                      "kernel": "kda_chunk_fwd (one launch per step)",
                      "alg_bytes_per_launch": main_res["alg"]["bytes"]},

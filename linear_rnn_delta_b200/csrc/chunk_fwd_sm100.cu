@@ -367,18 +367,21 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     __syncthreads();
 
     // scalar erase / write gates of a chunk's row `tid` (1 for GDN-2, 0 past the end),
-    // fetched one chunk ahead into registers so the load latency is hidden
-    auto fetch_gates = [&](int chunk, float &ge, float &gw) {
+    // fetched one chunk ahead as raw bf16 bits so the load latency is hidden; the
+    // conversion happens when the next chunk stores them to shared memory
+    auto fetch_gates = [&](int chunk, uint32_t &ge, uint32_t &gw) {
         const int r = tid, nv = min(C, len - chunk * C);
         const size_t tok = ((size_t)b * a.T + t0 + chunk * C + r) * H + h;
         const bool v = r < nv;
-        if (gdn2) { ge = v ? 1.f : 0.f; gw = ge; }
+        const unsigned short *g1u = reinterpret_cast<const unsigned short *>(g1p);
+        const unsigned short *g2u = reinterpret_cast<const unsigned short *>(g2p);
+        if (gdn2) { ge = v ? 0x3F80u : 0u; gw = ge; }   // bf16 1.0 / 0.0
         else {
-            ge = v ? bf2f(g1p, tok) : 0.f;
-            gw = v ? (a.variant == KDA ? ge : bf2f(g2p, tok)) : 0.f;
+            ge = v ? (uint32_t)g1u[tok] : 0u;
+            gw = v ? (uint32_t)(a.variant == KDA ? g1u[tok] : g2u[tok]) : 0u;
         }
     };
-    float gate_e = 0.f, gate_w = 0.f;
+    uint32_t gate_e = 0u, gate_w = 0u;
     if (tid < C && nchunks > 0) fetch_gates(0, gate_e, gate_w);
 
     for (int ch = 0; ch < nchunks && ok; ++ch) {
@@ -388,8 +391,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
         const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
 
         if (tid < C) {
-            s_g1[tid] = gate_e;
-            s_g2[tid] = gate_w;
+            s_g1[tid] = __uint_as_float(gate_e << 16);
+            s_g2[tid] = __uint_as_float(gate_w << 16);
             if (ch + 1 < nchunks) fetch_gates(ch + 1, gate_e, gate_w);
         }
         if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
