@@ -34,7 +34,7 @@
 //    one dense GEMM.  Six levels cover every pair s < r once; P_{r,r} = q_r . k_r.
 //    Nothing is divided, so zeros and signs propagate exactly.
 //
-// One CTA per (sequence, head); the fp32 state lives in tensor memory (TMEM)
+// One CTA of 512 threads per (sequence, head); the fp32 state lives in tensor memory (TMEM)
 // for the whole sequence, transposed (lane = value column j, column = key
 // channel i), so every state-dependent GEMM has M = d_v = 128.  q, k, v,
 // alpha arrive by TMA; every other operand is built on chip in 128-byte
@@ -60,11 +60,11 @@ using namespace sm100;
 
 constexpr int C = 64;    // chunk length
 constexpr int D = 128;   // d_k = d_v
-constexpr int NT = 256;  // threads per CTA
+constexpr int NT = 384;  // threads per CTA: 4 chain warps + 8 prep warps
 
 // ---- shared memory map (offsets from a 1024-byte aligned base) ------------
 constexpr uint32_t RAW_Q = 0, RAW_K = 16384, RAW_A = 49152;  // TMA tiles [64][128] bf16, row-major
-constexpr uint32_t OFF_UT = 32768;   // T Diag(w) bf16 64 x 64 (step 4), then U^T 128 x 64 (steps 6-7)
+constexpr uint32_t OFF_UT = 32768;   // U^T bf16 128 x 64 (chain steps 6-7), then o staging [64][128]
 constexpr uint32_t OFF_S0T = 65536;   // state operand bf16, 128 x 128, K-major (rows j, K = i)
 constexpr uint32_t OFF_QA = 98304;    // 128-row tile: rows 0-63 a~ operand (later W), rows 64-127 q operand
 constexpr uint32_t OFF_KB = 131072;   // Kbar [token][channel]
@@ -76,14 +76,14 @@ constexpr int TP = 68;                        // pitch (floats) of the fp32 A an
 constexpr uint32_t OFF_AF32 = OFF_F;          // A fp32 [64][TP]
 constexpr uint32_t OFF_TF32 = OFF_F + 17408;  // T fp32 [64][TP]
 constexpr uint32_t OFF_X = OFF_F + 34816;     // 32 x 32 fp32 scratch of the block solve
-constexpr uint32_t OFF_TBF = OFF_F + 38912;   // T Diag(e) bf16 64 x 64 K-major
+constexpr uint32_t OFF_TBF = OFF_F + 38912;   // T Diag(e) / T Diag(w) bf16 64 x 64 K-major
 constexpr uint32_t OFF_PBF = OFF_F + 47104;   // P bf16 64 x 64 K-major
-constexpr uint32_t OFF_OST = OFF_F;           // o staging [64][128] bf16 (A, T dead by then)
 constexpr uint32_t OFF_MISC = OFF_F + 55296;
 constexpr int PBAND = 5;   // P_{r,s} for r-4 <= s <= r computed exactly (SIMT) from the bf16 inputs
-constexpr uint32_t M_G1 = OFF_MISC, M_G2 = OFF_MISC + 256, M_GAMC = OFF_MISC + 512, M_TOT = OFF_MISC + 1024,
-                   M_PBAND = OFF_MISC + 5120, M_BAR = OFF_MISC + 6400, M_TMEM = OFF_MISC + 6432;
-constexpr uint32_t SMEM_USED = OFF_MISC + 6464;
+constexpr uint32_t M_G1 = OFF_MISC, M_G2 = OFF_MISC + 256, M_GAMC = OFF_MISC + 512, M_TOT = OFF_MISC + 1536,
+                   M_PBAND = OFF_MISC + 5632, M_FAST = OFF_MISC + 6912, M_BAR = OFF_MISC + 6920,
+                   M_TMEM = OFF_MISC + 6976;
+constexpr uint32_t SMEM_USED = OFF_MISC + 6992;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack for aligning the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert((OFF_TBF & 1023) == 0 && (OFF_PBF & 1023) == 0 && (OFF_QA & 1023) == 0, "swizzle atoms");
@@ -102,14 +102,23 @@ struct ChunkParams {
 };
 
 // ---- small helpers --------------------------------------------------------
+// Elementwise work is done in "items" of 8 tokens x 4 channels (one 8-byte
+// half of a 16-byte chunk per row): 256 items cover a 64 x 128 tile.
+__device__ __forceinline__ void unpack4(const uint2 &u, float *f)
+{
+    f[0] = __uint_as_float(u.x << 16);
+    f[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(u.y << 16);
+    f[3] = __uint_as_float(u.y & 0xFFFF0000u);
+}
+__device__ __forceinline__ uint2 pack4(const float *f)
+{
+    return make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+}
 __device__ __forceinline__ void unpack8(const uint4 &u, float *f)
 {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
+    unpack4(make_uint2(u.x, u.y), f);
+    unpack4(make_uint2(u.z, u.w), f + 4);
 }
 __device__ __forceinline__ uint4 pack8(const float *f)
 {
@@ -121,6 +130,11 @@ __device__ __forceinline__ uint32_t sw_chunk(uint32_t pstride, uint32_t row, uin
 {
     return (kc >> 3) * pstride + row * 128u + ((((kc & 7u) ^ (row & 7u))) << 4);
 }
+// 8-byte half-chunk of channel quad cq (channels 4cq .. 4cq+3)
+__device__ __forceinline__ uint32_t sw_half(uint32_t pstride, uint32_t row, uint32_t cq)
+{
+    return sw_chunk(pstride, row, cq >> 1) + (cq & 1u) * 8u;
+}
 __device__ __forceinline__ uint32_t sw_elem(uint32_t pstride, uint32_t row, uint32_t k)
 {
     return sw_chunk(pstride, row, k >> 3) + (k & 7u) * 2u;
@@ -129,6 +143,10 @@ __device__ __forceinline__ uint32_t sw_elem(uint32_t pstride, uint32_t row, uint
 __device__ __forceinline__ uint4 raw_row(const uint8_t *sm, uint32_t base, int r, int cg)
 {
     return *reinterpret_cast<const uint4 *>(sm + base + r * 256 + cg * 16);
+}
+__device__ __forceinline__ uint2 raw_quad(const uint8_t *sm, uint32_t base, int r, int cq)
+{
+    return *reinterpret_cast<const uint2 *>(sm + base + r * 256 + cq * 8);
 }
 // K-major descriptor, K step kk (16 elements), panels `pstride` bytes apart
 __device__ __forceinline__ uint64_t dK(uint32_t base, uint32_t pstride, int kk)
@@ -141,14 +159,9 @@ __device__ __forceinline__ uint64_t dMN(uint32_t base, uint32_t pstride, int kk)
 {
     return make_desc_sw128(base + (uint32_t)kk * 2048u, pstride);
 }
-__device__ __forceinline__ float bf2f(const __nv_bfloat16 *p, size_t i)
+__device__ __forceinline__ void load_tot4(const float *s_tot, int g, int cq, float *t4)
 {
-    return __uint_as_float((uint32_t)(*reinterpret_cast<const unsigned short *>(p + i)) << 16);
-}
-__device__ __forceinline__ void load_tot(const float *s_tot, int g, int cg, float *t8)
-{
-    *reinterpret_cast<float4 *>(t8) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8);
-    *reinterpret_cast<float4 *>(t8 + 4) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cg * 8 + 4);
+    *reinterpret_cast<float4 *>(t4) = *reinterpret_cast<const float4 *>(s_tot + g * 128 + cq * 4);
 }
 
 struct ChunkCtx {
@@ -160,29 +173,29 @@ struct ChunkCtx {
     bool gdn2;
 };
 
-// Channel-wise part of the erase direction of row r (GDN-2: the vector b;
-// 1 otherwise, because the scalar erase gate is folded into the rows of A and
-// the columns of T instead of into the bf16 operands).
-__device__ __forceinline__ void erase_gate(const ChunkCtx &x, int r, int cg, float *e)
+// Channel-wise part of the erase direction of row r for 4 channels (GDN-2:
+// the vector b; 1 otherwise, because the scalar erase gate is folded into the
+// rows of A and the columns of T instead of into the bf16 operands).
+__device__ __forceinline__ void erase_gate4(const ChunkCtx &x, int r, int cq, float *e)
 {
     if (x.gdn2 && r < x.nvalid) {
-        unpack8(*reinterpret_cast<const uint4 *>(x.g1p + ((x.rowbase + r) * x.H + x.h) * D + cg * 8), e);
+        unpack4(*reinterpret_cast<const uint2 *>(x.g1p + ((x.rowbase + r) * x.H + x.h) * D + cq * 4), e);
     } else {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) e[c] = 1.f;
+        for (int c = 0; c < 4; ++c) e[c] = 1.f;
     }
 }
 
 // Anchored path: row and column factors of one level (block half HH) for the
-// 8-token x 8-channel item (tg, cg), into level slot `slot` (0 or 1).
+// 8-token x 4-channel item (tg, cq), into level slot `slot` (0 or 1).
 template <int HH>
-__device__ __forceinline__ void build_level(const ChunkCtx &x, int slot, int tg, int cg)
+__device__ __forceinline__ void build_level(const ChunkCtx &x, int slot, int tg, int cq)
 {
     constexpr int BS = 2 * HH;
     uint8_t *sm = x.sm;
-    float cpre[8], csuf[8];
+    float cpre[4], csuf[4];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) { cpre[c] = 1.f; csuf[c] = 1.f; }
+    for (int c = 0; c < 4; ++c) { cpre[c] = 1.f; csuf[c] = 1.f; }
     if (HH >= 8) {  // carries over whole 8-token blocks
         const int r0 = tg * 8, pos0 = r0 % BS;
         const int gs = (r0 - pos0 + HH) >> 3, ge = (r0 - pos0 + HH - 1) >> 3;
@@ -190,65 +203,65 @@ __device__ __forceinline__ void build_level(const ChunkCtx &x, int slot, int tg,
             const bool in_pre = pos0 >= HH && g >= gs && g < tg;
             const bool in_suf = pos0 < HH && g > tg && g <= ge;
             if (in_pre || in_suf) {
-                float t8[8];
-                load_tot(x.s_tot, g, cg, t8);
+                float t4[4];
+                load_tot4(x.s_tot, g, cq, t4);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (in_pre) cpre[c] *= t8[c];
-                    if (in_suf) csuf[c] *= t8[c];
+                for (int c = 0; c < 4; ++c) {
+                    if (in_pre) cpre[c] *= t4[c];
+                    if (in_suf) csuf[c] *= t4[c];
                 }
             }
         }
     }
-    float run[8];
+    float run[4];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) run[c] = cpre[c];
+    for (int c = 0; c < 4; ++c) run[c] = cpre[c];
 #pragma unroll 1
     for (int i = 0; i < 8; ++i) {  // second-half rows: prefix from the half start
         const int r = tg * 8 + i, pos = r % BS;
         if (HH < 8 && pos == HH) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) run[c] = 1.f;
+            for (int c = 0; c < 4; ++c) run[c] = 1.f;
         }
         if (pos < HH) continue;
         const bool v = r < x.nvalid;
-        float al[8], qv[8], kv[8], e[8], fa[8], fp[8];
-        unpack8(raw_row(sm, RAW_A, r, cg), al);
-        unpack8(raw_row(sm, RAW_Q, r, cg), qv);
-        unpack8(raw_row(sm, RAW_K, r, cg), kv);
-        erase_gate(x, r, cg, e);
+        float al[4], qv[4], kv[4], e[4], fa[4], fp[4];
+        unpack4(raw_quad(sm, RAW_A, r, cq), al);
+        unpack4(raw_quad(sm, RAW_Q, r, cq), qv);
+        unpack4(raw_quad(sm, RAW_K, r, cq), kv);
+        erase_gate4(x, r, cq, e);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
             run[c] *= v ? al[c] : 1.f;
             fa[c] = v ? run[c] * e[c] * kv[c] : 0.f;
             fp[c] = v ? run[c] * qv[c] : 0.f;
         }
         const int idx = (r / BS) * HH + (pos - HH);
-        *reinterpret_cast<uint4 *>(sm + OFF_LA + sw_chunk(16384, slot * 32 + idx, cg)) = pack8(fa);
-        *reinterpret_cast<uint4 *>(sm + OFF_LA + sw_chunk(16384, 64 + slot * 32 + idx, cg)) = pack8(fp);
+        *reinterpret_cast<uint2 *>(sm + OFF_LA + sw_half(16384, slot * 32 + idx, cq)) = pack4(fa);
+        *reinterpret_cast<uint2 *>(sm + OFF_LA + sw_half(16384, 64 + slot * 32 + idx, cq)) = pack4(fp);
     }
-    float sx[8];
+    float sx[4];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) sx[c] = csuf[c];
+    for (int c = 0; c < 4; ++c) sx[c] = csuf[c];
 #pragma unroll 1
     for (int i = 7; i >= 0; --i) {  // first-half columns: exclusive suffix to the half end
         const int r = tg * 8 + i, pos = r % BS;
         if (pos >= HH) continue;
         if (HH < 8 && pos == HH - 1) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) sx[c] = 1.f;
+            for (int c = 0; c < 4; ++c) sx[c] = 1.f;
         }
         const bool v = r < x.nvalid;
-        float al[8], kv[8], fc[8];
-        unpack8(raw_row(sm, RAW_A, r, cg), al);
-        unpack8(raw_row(sm, RAW_K, r, cg), kv);
+        float al[4], kv[4], fc[4];
+        unpack4(raw_quad(sm, RAW_A, r, cq), al);
+        unpack4(raw_quad(sm, RAW_K, r, cq), kv);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
             fc[c] = v ? sx[c] * kv[c] : 0.f;
             sx[c] *= v ? al[c] : 1.f;
         }
         const int idx = (r / BS) * HH + pos;
-        *reinterpret_cast<uint4 *>(sm + OFF_LB + sw_chunk(8192, slot * 32 + idx, cg)) = pack8(fc);
+        *reinterpret_cast<uint2 *>(sm + OFF_LB + sw_half(8192, slot * 32 + idx, cq)) = pack4(fc);
     }
 }
 
@@ -272,6 +285,20 @@ __device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const floa
 }
 
 // ---- the kernel -------------------------------------------------------------
+// Warp roles.  Warps 0-3 (CHAIN, 128 threads) own the state: for chunk n they
+// scale S by Gamma_C and copy it to bf16, run U^T -= S^T W^T, O^T = S^T Q^T,
+// read U^T out, run O^T += U^T P^T, S^T += U^T Kbar, and write o.  Warps 4-11
+// (PREP, 256 threads) build chunk n+1's operands meanwhile: decay products,
+// row operands, Kbar, the band of P, A and P, T = (I+A)^{-1}, W and U'^T.
+// Hand-offs go through mbarriers; each buffer the two groups share is
+// released by the step that last reads it:
+//   ready  : prep(n) -> chain(n)   (QA = [W'; Q'], Kbar, P, U' in TMEM, Gamma_C)
+//   s6     : chain(n) GEMMs of step 6 done -> prep(n+1) may rewrite QA
+//   s7     : chain(n) GEMMs of step 7 done -> prep(n+1) may rewrite Kbar, P, levels
+//   ufree  : chain(n) has read U^T out of TMEM -> prep(n+1) may write U'^T
+constexpr int NCHAIN = 128, NPREP = 256;
+constexpr uint32_t BAR_PREP = 1, BAR_CHAIN = 2;
+
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant__ ChunkParams P)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -280,7 +307,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     const FwdArgs &a = P.a;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;       // TMEM lane quarter of this warp
-    const int half = warp >> 2;         // warps 0-3 / 4-7 split TMEM columns
     const int H = a.H;
     const int n = blockIdx.x / H, h = blockIdx.x % H;
     int b, t0, len;
@@ -290,12 +316,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 
     float *s_g1 = reinterpret_cast<float *>(sm + M_G1);
     float *s_g2 = reinterpret_cast<float *>(sm + M_G2);
-    float *s_gamC = reinterpret_cast<float *>(sm + M_GAMC);
-    float *s_tot = reinterpret_cast<float *>(sm + M_TOT);   // [8][128] block totals of alpha
+    float *s_gamC = reinterpret_cast<float *>(sm + M_GAMC);     // [2][128]: chunk parity
+    float *s_tot = reinterpret_cast<float *>(sm + M_TOT);       // [8][128] block totals of alpha
     float *s_pband = reinterpret_cast<float *>(sm + M_PBAND);   // [64][PBAND]: P_{r, r-w}
-    uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + M_BAR);
-    uint64_t *bar_mma = bar_tma + 1;
-    uint64_t *bar_v = bar_tma + 2;
+    int *s_fast = reinterpret_cast<int *>(sm + M_FAST);         // [2]: chunk parity
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + M_BAR);
+    uint64_t *bar_tma = bars + 0, *bar_v = bars + 1, *bar_pmma = bars + 2, *bar_ready = bars + 3;
+    uint64_t *bar_s6 = bars + 4, *bar_s7 = bars + 5, *bar_ufree = bars + 6;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + M_TMEM);
     float *Af = reinterpret_cast<float *>(sm + OFF_AF32);
     float *Tf = reinterpret_cast<float *>(sm + OFF_TF32);
@@ -304,12 +331,11 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     const __nv_bfloat16 *g1p = (const __nv_bfloat16 *)a.g1, *g2p = (const __nv_bfloat16 *)a.g2;
     uint8_t *op = (uint8_t *)a.o;
     const bool gdn2 = a.variant == GDN2;
+    const bool same_gates = a.variant != RDA;   // erase and write gates coincide: one T copy serves both
 
     if (warp == 0) tmem_alloc(s_tmem, 512);
     if (tid == 0) {
-        mbar_init(bar_tma, 1);
-        mbar_init(bar_mma, 1);
-        mbar_init(bar_v, 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
@@ -317,227 +343,325 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     tc_fence_after();
     const uint32_t tbase = *s_tmem;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int jcol = quarter * 32 + lane;   // value column j = TMEM lane of this thread
-    uint32_t ph_tma = 0, ph_mma = 0, ph_v = 0;
     bool ok = true;
 
-    const CUtensorMap *map_q = &P.tq, *map_k = &P.tk, *map_v = &P.tv, *map_a = &P.ta;
-    auto issue_tma = [&](int chunk) {   // q, k, alpha of a chunk
-        const int g = b * a.T + t0 + chunk * C;  // token row of the packed [B*T] axis
-        mbar_expect_tx(bar_tma, 3 * 16384);
-        tma_load_3d(sm + RAW_Q, map_q, bar_tma, 0, h, g);
-        tma_load_3d(sm + RAW_K, map_k, bar_tma, 0, h, g);
-        tma_load_3d(sm + RAW_A, map_a, bar_tma, 0, h, g);
-    };
-    auto issue_tma_v = [&](int chunk) { // v, straight into its swizzled operand layout (two 64-channel panels)
-        const int g = b * a.T + t0 + chunk * C;
-        mbar_expect_tx(bar_v, 16384);
-        tma_load_3d(sm + OFF_MT, map_v, bar_v, 0, h, g);
-        tma_load_3d(sm + OFF_MT + 8192, map_v, bar_v, 64, h, g);
-    };
-    auto wait_mma = [&]() {     // all threads: MMAs committed so far are complete
-        if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
-        ph_mma ^= 1;
-        tc_fence_after();
-    };
-    auto publish = [&]() {      // all threads: make smem / TMEM writes visible to the tensor core
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-    };
-
-    if (nchunks > 0 && tid == 0) {
-        issue_tma(0);
-        issue_tma_v(0);
-    }
-
-    // ---- initial state -> TMEM (fp32) ----------------------------------------
-    {
-        const size_t soff = ((size_t)n * H + h) * D * D;
-        for (int c16 = 0; c16 < 4; ++c16) {
-            float v[16];
-            const int i0 = half * 64 + c16 * 16;
+    if (warp < 4) {
+        // =====================================================================
+        // CHAIN group
+        // =====================================================================
+        const int jcol = tid;   // value column j = TMEM lane
+        {   // initial state -> TMEM (fp32)
+            const size_t soff = ((size_t)n * H + h) * D * D;
+#pragma unroll 1
+            for (int c16 = 0; c16 < 8; ++c16) {
+                float v[16];
+                const int i0 = c16 * 16;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = a.s0 ? a.s0[soff + (size_t)(i0 + e) * D + jcol] : 0.f;
-            tmem_st16(tbase + lane_base + TM_S + i0, v);
+                for (int e = 0; e < 16; ++e) v[e] = a.s0 ? a.s0[soff + (size_t)(i0 + e) * D + jcol] : 0.f;
+                tmem_st16(tbase + lane_base + TM_S + i0, v);
+            }
+            tmem_wait_st();
         }
-        tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // scalar erase / write gates of a chunk's row `tid` (1 for GDN-2, 0 past the end),
-    // fetched one chunk ahead as raw bf16 bits so the load latency is hidden; the
-    // conversion happens when the next chunk stores them to shared memory
-    auto fetch_gates = [&](int chunk, uint32_t &ge, uint32_t &gw) {
-        const int r = tid, nv = min(C, len - chunk * C);
-        const size_t tok = ((size_t)b * a.T + t0 + chunk * C + r) * H + h;
-        const bool v = r < nv;
-        const unsigned short *g1u = reinterpret_cast<const unsigned short *>(g1p);
-        const unsigned short *g2u = reinterpret_cast<const unsigned short *>(g2p);
-        if (gdn2) { ge = v ? 0x3F80u : 0u; gw = ge; }   // bf16 1.0 / 0.0
-        else {
-            ge = v ? (uint32_t)g1u[tok] : 0u;
-            gw = v ? (uint32_t)(a.variant == KDA ? g1u[tok] : g2u[tok]) : 0u;
-        }
-    };
-    uint32_t gate_e = 0u, gate_w = 0u;
-    if (tid < C && nchunks > 0) fetch_gates(0, gate_e, gate_w);
-
-    for (int ch = 0; ch < nchunks && ok; ++ch) {
-        const int tok0 = t0 + ch * C;
-        const int nvalid = min(C, len - ch * C);
-        const size_t rowbase = (size_t)b * a.T + tok0;   // packed token index of chunk row 0
-        const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
-
-        if (tid < C) {
-            s_g1[tid] = __uint_as_float(gate_e << 16);
-            s_g2[tid] = __uint_as_float(gate_w << 16);
-            if (ch + 1 < nchunks) fetch_gates(ch + 1, gate_e, gate_w);
-        }
-        if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
-        ph_tma ^= 1;
-        if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
-        ph_v ^= 1;
-        __syncthreads();
-
-        // ===== 1a. block totals of alpha (and range check) | M ================
-        bool in_range = true;
-        if (tid < 128) {
-            const int tg = tid >> 4, cg = tid & 15;
-            float tot[8];
+        for (int ch = 0; ch < nchunks && ok; ++ch) {
+            const uint32_t par = ch & 1;
+            const int nvalid = min(C, len - ch * C);
+            const size_t rowbase = (size_t)b * a.T + t0 + ch * C;
+            if (!mbar_wait_cycles(bar_ready, par, WAIT_CYCLES)) ok = false;
+            tc_fence_after();
+            const bool fast = s_fast[par] != 0;
+            const float *gamC = s_gamC + par * 128;
+            // ---- state pass: S^T *= Gamma_C in TMEM; bf16 operand copy (scaled on the fast path)
+#pragma unroll 1
+            for (int c32 = 0; c32 < 4; ++c32) {
+                const int i0 = c32 * 32;
+                float s[32], t[32];
+                tmem_ld32(tbase + lane_base + TM_S + i0, s);
+                tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 8; ++c) tot[c] = 1.f;
+                for (int e = 0; e < 32; ++e) {
+                    t[e] = s[e] * gamC[i0 + e];
+                    if (fast) s[e] = t[e];
+                }
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = tg * 8 + i;
-                if (r < nvalid) {
-                    float al[8];
-                    unpack8(raw_row(sm, RAW_A, r, cg), al);
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
+                tmem_st16(tbase + lane_base + TM_S + i0, t);
+                tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            group_sync(BAR_CHAIN, NCHAIN);
+            // ---- step 6: U^T -= S^T W^T ; O^T = S^T Q^T
+            if (tid == 0) {
+                tc_fence_after();
+                const uint32_t id_neg = idesc_bf16(128, 64, false, false, true);
+                const uint32_t id_pos = idesc_bf16(128, 64, false, false);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        tot[c] *= al[c];
-                        in_range = in_range && (fabsf(al[c]) <= 1.f);
-                    }
+                for (int kk = 0; kk < 8; ++kk) {
+                    mma_bf16(tbase + TM_U, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA, 16384, kk), id_neg, 1);
+                    mma_bf16(tbase + TM_O, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA + 8192, 16384, kk), id_pos,
+                             kk > 0);
+                }
+                mma_commit(bar_s6);
+            }
+            if (!mbar_wait_cycles(bar_s6, par, WAIT_CYCLES)) ok = false;
+            tc_fence_after();
+            // ---- U^T row j -> bf16 K-major tile (rows j, K = token); then release TMEM U
+#pragma unroll
+            for (int c32 = 0; c32 < 2; ++c32) {
+                float v[32];
+                tmem_ld32(tbase + lane_base + TM_U + c32 * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(sm + OFF_UT + sw_chunk(16384, jcol, c32 * 4 + q4)) = pack8(v + q4 * 8);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            group_sync(BAR_CHAIN, NCHAIN);
+            // ---- step 7: O^T += U^T P^T ; S^T += U^T Kbar
+            if (tid == 0) {
+                mbar_arrive(bar_ufree);
+                tc_fence_after();
+                const uint32_t id_o = idesc_bf16(128, 64, false, false);
+                const uint32_t id_s = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    mma_bf16(tbase + TM_O, dK(sb + OFF_UT, 16384, kk), dK(sb + OFF_PBF, 8192, kk), id_o, 1);
+                    mma_bf16(tbase + TM_S, dK(sb + OFF_UT, 16384, kk), dMN(sb + OFF_KB, 8192, kk), id_s, 1);
+                }
+                mma_commit(bar_s7);
+            }
+            if (!mbar_wait_cycles(bar_s7, par, WAIT_CYCLES)) ok = false;
+            tc_fence_after();
+            // ---- o: TMEM (lane j, column r) -> bf16 staging [r][j] in the U^T slot -> HBM
+            unsigned short *ost = reinterpret_cast<unsigned short *>(sm + OFF_UT);
+#pragma unroll
+            for (int c32 = 0; c32 < 2; ++c32) {
+                float v[32];
+                tmem_ld32(tbase + lane_base + TM_O + c32 * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const uint32_t pk = pack_bf16(v[e], v[e + 1]);
+                    ost[(c32 * 32 + e) * 128 + jcol] = (unsigned short)(pk & 0xFFFFu);
+                    ost[(c32 * 32 + e + 1) * 128 + jcol] = (unsigned short)(pk >> 16);
                 }
             }
-            *reinterpret_cast<float4 *>(s_tot + tg * 128 + cg * 8) = make_float4(tot[0], tot[1], tot[2], tot[3]);
-            *reinterpret_cast<float4 *>(s_tot + tg * 128 + cg * 8 + 4) = make_float4(tot[4], tot[5], tot[6], tot[7]);
-        } else {
-            const int u = tid - 128, tg = u >> 4, cg = u & 15;
-            if (gdn2) {   // M = w (.) v, in place in the swizzled v tile (rows past the end -> 0)
+            tc_fence_before();
+            group_sync(BAR_CHAIN, NCHAIN);
+            for (int e = tid; e < nvalid * 16; e += NCHAIN) {
+                const int r = e >> 4, cgo = e & 15;
+                *reinterpret_cast<uint4 *>(op + (((rowbase + r) * H + h) * D + cgo * 8) * 2) =
+                    *reinterpret_cast<const uint4 *>(sm + OFF_UT + r * 256 + cgo * 16);
+            }
+            ok = group_sync_and(BAR_CHAIN, NCHAIN, ok);   // staging read before the next U^T write
+        }
+    } else {
+        // =====================================================================
+        // PREP group
+        // =====================================================================
+        const int ptid = tid - NCHAIN, pw = warp - 4;
+        const int phalf = pw >> 2;              // the two prep warps of a lane quarter split columns
+        const int jrow = quarter * 32 + lane;   // TMEM lane of this thread
+        const int tg = ptid >> 5, cq = ptid & 31;   // elementwise item: 8 tokens x 4 channels
+        uint32_t ph_tma = 0, ph_v = 0, ph_pmma = 0;
+
+        const CUtensorMap *map_q = &P.tq, *map_k = &P.tk, *map_v = &P.tv, *map_a = &P.ta;
+        auto issue_tma = [&](int chunk) {   // q, k, alpha of a chunk
+            const int g = b * a.T + t0 + chunk * C;
+            mbar_expect_tx(bar_tma, 3 * 16384);
+            tma_load_3d(sm + RAW_Q, map_q, bar_tma, 0, h, g);
+            tma_load_3d(sm + RAW_K, map_k, bar_tma, 0, h, g);
+            tma_load_3d(sm + RAW_A, map_a, bar_tma, 0, h, g);
+        };
+        auto issue_tma_v = [&](int chunk) { // v, straight into its swizzled operand layout
+            const int g = b * a.T + t0 + chunk * C;
+            mbar_expect_tx(bar_v, 16384);
+            tma_load_3d(sm + OFF_MT, map_v, bar_v, 0, h, g);
+            tma_load_3d(sm + OFF_MT + 8192, map_v, bar_v, 64, h, g);
+        };
+        auto wait_pmma = [&]() {
+            if (!mbar_wait_cycles(bar_pmma, ph_pmma, WAIT_CYCLES)) ok = false;
+            ph_pmma ^= 1;
+            tc_fence_after();
+        };
+        auto publish = [&]() {
+            fence_async_smem();
+            tc_fence_before();
+            group_sync(BAR_PREP, NPREP);
+        };
+        // scalar gates of a chunk's row `ptid` as raw bf16 bits, fetched one chunk ahead
+        auto fetch_gates = [&](int chunk, uint32_t &ge, uint32_t &gw) {
+            const int r = ptid, nv = min(C, len - chunk * C);
+            const size_t tok = ((size_t)b * a.T + t0 + chunk * C + r) * H + h;
+            const bool v = r < nv;
+            const unsigned short *g1u = reinterpret_cast<const unsigned short *>(g1p);
+            const unsigned short *g2u = reinterpret_cast<const unsigned short *>(g2p);
+            if (gdn2) { ge = v ? 0x3F80u : 0u; gw = ge; }   // bf16 1.0 / 0.0
+            else {
+                ge = v ? (uint32_t)g1u[tok] : 0u;
+                gw = v ? (uint32_t)(a.variant == KDA ? g1u[tok] : g2u[tok]) : 0u;
+            }
+        };
+
+        if (nchunks > 0 && ptid == 0) {
+            issue_tma(0);
+            issue_tma_v(0);
+        }
+        uint32_t gate_e = 0u, gate_w = 0u;
+        if (ptid < C && nchunks > 0) fetch_gates(0, gate_e, gate_w);
+
+        for (int ch = 0; ch < nchunks && ok; ++ch) {
+            const uint32_t par = ch & 1, ppar = (ch - 1) & 1;
+            const int nvalid = min(C, len - ch * C);
+            const size_t rowbase = (size_t)b * a.T + t0 + ch * C;
+            const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
+
+            if (ptid < C) {
+                s_g1[ptid] = __uint_as_float(gate_e << 16);
+                s_g2[ptid] = __uint_as_float(gate_w << 16);
+                if (ch + 1 < nchunks) fetch_gates(ch + 1, gate_e, gate_w);
+            }
+            if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
+            ph_tma ^= 1;
+            if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
+            ph_v ^= 1;
+            group_sync(BAR_PREP, NPREP);
+
+            // ===== 1a. block totals of alpha (and range check) | GDN-2: M = w (.) v
+            bool in_range = true;
+            {
+                float tot[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = tg * 8 + i;
+                    if (r < nvalid) {
+                        float al[4];
+                        unpack4(raw_quad(sm, RAW_A, r, cq), al);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            tot[c] *= al[c];
+                            in_range = in_range && (fabsf(al[c]) <= 1.f);
+                        }
+                    }
+                }
+                *reinterpret_cast<float4 *>(s_tot + tg * 128 + cq * 4) = make_float4(tot[0], tot[1], tot[2], tot[3]);
+            }
+            if (gdn2) {   // in place in the swizzled v tile; rows past the end -> 0
 #pragma unroll 2
                 for (int i = 0; i < 8; ++i) {
                     const int r = tg * 8 + i;
-                    uint4 *pv = reinterpret_cast<uint4 *>(sm + OFF_MT + sw_chunk(8192, r, cg));
-                    float mv[8], vv[8], wv[8];
-                    unpack8(*pv, vv);
+                    uint2 *pv = reinterpret_cast<uint2 *>(sm + OFF_MT + sw_half(8192, r, cq));
+                    float mv[4], vv[4], wv[4];
+                    unpack4(*pv, vv);
                     if (r < nvalid) {
-                        unpack8(*reinterpret_cast<const uint4 *>(g2p + ((rowbase + r) * H + h) * D + cg * 8), wv);
+                        unpack4(*reinterpret_cast<const uint2 *>(g2p + ((rowbase + r) * H + h) * D + cq * 4), wv);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) mv[c] = wv[c] * vv[c];
+                        for (int c = 0; c < 4; ++c) mv[c] = wv[c] * vv[c];
                     } else {
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) mv[c] = 0.f;
+                        for (int c = 0; c < 4; ++c) mv[c] = 0.f;
                     }
-                    *pv = pack8(mv);
+                    *pv = pack4(mv);
                 }
             }
-        }
-        in_range = __syncthreads_and(in_range) != 0;
+            in_range = group_sync_and(BAR_PREP, NPREP, in_range);
 
-        // ===== Gamma_C and the per-chunk path decision ========================
-        bool gam_ok = true;
-        if (tid < 16) {
-            const int cg = tid;
-            float gc[8];
+            // ===== Gamma_C and the per-chunk path decision ========================
+            bool gam_ok = true;
+            if (ptid < 32) {
+                float gc[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
-            for (int c = 0; c < 8; ++c) gc[c] = 1.f;
-            for (int g = 0; g < 8; ++g) {
-                float t8[8];
-                load_tot(s_tot, g, cg, t8);
+                for (int g = 0; g < 8; ++g) {
+                    float t4[4];
+                    load_tot4(s_tot, g, ptid, t4);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) gc[c] *= t8[c];
-            }
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                s_gamC[cg * 8 + c] = gc[c];
-                gam_ok = gam_ok && (fabsf(gc[c]) >= FAST_MIN_GAMMA);
-            }
-        }
-        const bool fast = (__syncthreads_and(gam_ok) != 0) && in_range;
-
-        // ===== 1b. row operands (Gamma a~ | Gamma q, scaled on the fast path), Kbar, band of P
-        {
-            const int u = tid & 127, tg = u >> 4, cg = u & 15;
-            const bool grp0 = tid < 128;
-            float pre[8], suf[8];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) { pre[c] = 1.f; suf[c] = 1.f; }
-            for (int g = 0; g < 8; ++g) {
-                if (g == tg) continue;
-                float t8[8];
-                load_tot(s_tot, g, cg, t8);
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    if (g < tg) pre[c] *= t8[c];
-                    else suf[c] *= t8[c];
+                    for (int c = 0; c < 4; ++c) gc[c] *= t4[c];
                 }
-            }
-            {   // forward: group 0 writes rows 0-63 (Gamma a~), group 1 rows 64-127 (Gamma q)
-                float sc[8];
+                *reinterpret_cast<float4 *>(s_gamC + par * 128 + ptid * 4) = make_float4(gc[0], gc[1], gc[2], gc[3]);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) sc[c] = fast ? pre[c] * (1.0f / s_gamC[cg * 8 + c]) : pre[c];
-#pragma unroll 4
-                for (int i = 0; i < 8; ++i) {
+                for (int c = 0; c < 4; ++c) gam_ok = gam_ok && (fabsf(gc[c]) >= FAST_MIN_GAMMA);
+            }
+            const bool fast = group_sync_and(BAR_PREP, NPREP, gam_ok) && in_range;
+            if (ptid == 0) s_fast[par] = fast ? 1 : 0;
+
+            // the previous chunk's chain must be done with QA (step 6) and with Kbar / P (step 7)
+            if (ch > 0) {
+                if (!mbar_wait_cycles(bar_s6, ppar, WAIT_CYCLES)) ok = false;
+                if (!mbar_wait_cycles(bar_s7, ppar, WAIT_CYCLES)) ok = false;
+            }
+
+            // ===== 1b. row operands (Gamma a~ | Gamma q, scaled on the fast path), Kbar, band of P
+            {
+                float pre[4] = {1.f, 1.f, 1.f, 1.f}, suf[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    if (g == tg) continue;
+                    float t4[4];
+                    load_tot4(s_tot, g, cq, t4);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (g < tg) pre[c] *= t4[c];
+                        else suf[c] *= t4[c];
+                    }
+                }
+                float sc[4];
+                if (fast) {
+                    const float4 gc4 = *reinterpret_cast<const float4 *>(s_gamC + par * 128 + cq * 4);
+                    sc[0] = pre[0] / gc4.x; sc[1] = pre[1] / gc4.y; sc[2] = pre[2] / gc4.z; sc[3] = pre[3] / gc4.w;
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sc[c] = pre[c];
+                }
+#pragma unroll 2
+                for (int i = 0; i < 8; ++i) {   // forward: rows 0-63 Gamma a~, rows 64-127 Gamma q
                     const int r = tg * 8 + i;
                     const bool v = r < nvalid;
-                    float al[8], xv[8], e[8], o8[8];
-                    unpack8(raw_row(sm, RAW_A, r, cg), al);
-                    unpack8(raw_row(sm, grp0 ? RAW_K : RAW_Q, r, cg), xv);
-                    if (grp0) erase_gate(x, r, cg, e);
-                    else {
+                    float al[4], kv[4], qv[4], e[4], oa[4], oq[4];
+                    unpack4(raw_quad(sm, RAW_A, r, cq), al);
+                    unpack4(raw_quad(sm, RAW_K, r, cq), kv);
+                    unpack4(raw_quad(sm, RAW_Q, r, cq), qv);
+                    erase_gate4(x, r, cq, e);
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) e[c] = 1.f;
-                    }
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         sc[c] *= v ? al[c] : 1.f;
-                        o8[c] = v ? sc[c] * (e[c] * xv[c]) : 0.f;
+                        oa[c] = v ? sc[c] * (e[c] * kv[c]) : 0.f;
+                        oq[c] = v ? sc[c] * qv[c] : 0.f;
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, (grp0 ? 0 : 64) + r, cg)) = pack8(o8);
+                    *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, r, cq)) = pack4(oa);
+                    *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, 64 + r, cq)) = pack4(oq);
                 }
-            }
-            if (grp0) {   // backward: Kbar_s = (prod_{s<t<C} alpha_t) (.) k_s
-                float sx[8];
+                float sx[4];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) sx[c] = suf[c];
-#pragma unroll 4
-                for (int i = 7; i >= 0; --i) {
+                for (int c = 0; c < 4; ++c) sx[c] = suf[c];
+#pragma unroll 2
+                for (int i = 7; i >= 0; --i) {   // backward: Kbar_s = (prod_{s<t<C} alpha_t) (.) k_s
                     const int r = tg * 8 + i;
                     const bool v = r < nvalid;
-                    float al[8], kv[8], kb[8];
-                    unpack8(raw_row(sm, RAW_A, r, cg), al);
-                    unpack8(raw_row(sm, RAW_K, r, cg), kv);
+                    float al[4], kv[4], kb[4];
+                    unpack4(raw_quad(sm, RAW_A, r, cq), al);
+                    unpack4(raw_quad(sm, RAW_K, r, cq), kv);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         kb[c] = v ? sx[c] * kv[c] : 0.f;
                         sx[c] *= v ? al[c] : 1.f;
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_KB + sw_chunk(8192, r, cg)) = pack8(kb);
+                    *reinterpret_cast<uint2 *>(sm + OFF_KB + sw_half(8192, r, cq)) = pack4(kb);
                 }
             }
             {   // band of P: P_{r,r-w} = sum_c q_rc (alpha_r ... alpha_{r-w+1})_c k_{r-w,c}, w = 0..4,
                 // from the bf16 inputs in fp32: the entries whose bf16 GEMM rounding would hurt most.
-                // Four threads per row (32 channels each), chunk order staggered by row so the
-                // loads are bank-conflict free; rows below w are clamped and masked afterwards.
-                const int r = tid >> 2, cq = tid & 3;
+                // Four threads per row (32 channels each), chunk order staggered by row so the loads
+                // are bank-conflict free; rows below w are clamped and masked afterwards.
+                const int r = ptid >> 2, c4 = ptid & 3;
                 float acc[PBAND];
 #pragma unroll
                 for (int w = 0; w < PBAND; ++w) acc[w] = 0.f;
-#pragma unroll 2
+#pragma unroll 1
                 for (int j = 0; j < 4; ++j) {
-                    const int cgx = cq * 4 + ((j + r) & 3);
+                    const int cgx = c4 * 4 + ((j + r) & 3);
                     float hv[8];
                     unpack8(raw_row(sm, RAW_Q, r, cgx), hv);
 #pragma unroll
@@ -558,347 +682,301 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                 for (int w = 0; w < PBAND; ++w) {
                     float t = acc[w] + __shfl_xor_sync(0xffffffffu, acc[w], 1);
                     t += __shfl_xor_sync(0xffffffffu, t, 2);
-                    if (cq == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? t : 0.f;
+                    if (c4 == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? t : 0.f;
                 }
             }
-        }
-        __syncthreads();   // band and row operands complete before either A/P path reads them
+            group_sync(BAR_PREP, NPREP);   // band and row operands complete before either A/P path reads them
 
-        // ===== 2. A and P ======================================================
-        if (fast) {
-            publish();
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t idesc = idesc_bf16(128, 64, false, false);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(tbase + TM_AP, dK(sb + OFF_QA, 16384, kk), dK(sb + OFF_KB, 8192, kk), idesc, kk > 0);
-                mma_commit(bar_mma);
-            }
-            wait_mma();
-            if (tid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
-            // rows 0-63: A (strictly lower), rows 64-127: P (lower incl. diagonal)
-            float v[32];
-            tmem_ld32(tbase + lane_base + TM_AP + half * 32, v);
-            tmem_wait_ld();
-            const int rr = jcol & 63;
-            if (jcol < 64) {
-                const float er = s_g1[rr];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int s = half * 32 + c;
-                    Af[rr * TP + s] = (s < rr) ? v[c] * er : 0.f;
-                }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const int s = half * 32 + c;
-                    const int w = rr - s;
-                    v[c] = (w >= PBAND) ? v[c] : ((w >= 0) ? s_pband[rr * PBAND + w] : 0.f);
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_PBF + sw_chunk(8192, rr, half * 4 + q4)) = pack8(v + q4 * 8);
-            }
-        } else {
-            // anchored levels: three GEMMs of two levels each
-            for (int p = 0; p < 3; ++p) {
-                const int lvl = 2 * p + 1 + (tid >> 7), slot = tid >> 7;
-                const int u = tid & 127, tg = u >> 4, cg = u & 15;
-                switch (lvl) {
-                case 1: build_level<32>(x, slot, tg, cg); break;
-                case 2: build_level<16>(x, slot, tg, cg); break;
-                case 3: build_level<8>(x, slot, tg, cg); break;
-                case 4: build_level<4>(x, slot, tg, cg); break;
-                case 5: build_level<2>(x, slot, tg, cg); break;
-                default: build_level<1>(x, slot, tg, cg); break;
-                }
+            // ===== 2. A and P ======================================================
+            if (fast) {
                 publish();
-                if (tid == 0) {
+                if (ptid == 0) {
                     tc_fence_after();
                     const uint32_t idesc = idesc_bf16(128, 64, false, false);
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tbase + tm_lvl(p), dK(sb + OFF_LA, 16384, kk), dK(sb + OFF_LB, 8192, kk), idesc,
-                                 kk > 0);
-                    mma_commit(bar_mma);
+                        mma_bf16(tbase + TM_AP, dK(sb + OFF_QA, 16384, kk), dK(sb + OFF_KB, 8192, kk), idesc, kk > 0);
+                    mma_commit(bar_pmma);
                 }
-                wait_mma();
-            }
-            if (tid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
-            for (int e = tid; e < 64 * TP; e += NT) Af[e] = 0.f;
-            for (int e = tid; e < 512; e += NT)
-                *reinterpret_cast<uint4 *>(sm + OFF_PBF + e * 16) = make_uint4(0, 0, 0, 0);
-            __syncthreads();
-            for (int p = half; p < 3; p += 2) {
-                const int lvl = 2 * p + 1 + (quarter & 1);
-                const bool isP = quarter >= 2;
+                wait_pmma();
+                if (ptid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
+                // rows 0-63: A (strictly lower, scaled by e_r), rows 64-127: P (band exact)
                 float v[32];
-                tmem_ld32(tbase + lane_base + tm_lvl(p) + (quarter & 1) * 32, v);
+                tmem_ld32(tbase + lane_base + TM_AP + phalf * 32, v);
                 tmem_wait_ld();
-                switch (lvl) {
-                case 1: scatter_level<32>(sm, Af, s_g1, isP, lane, v); break;
-                case 2: scatter_level<16>(sm, Af, s_g1, isP, lane, v); break;
-                case 3: scatter_level<8>(sm, Af, s_g1, isP, lane, v); break;
-                case 4: scatter_level<4>(sm, Af, s_g1, isP, lane, v); break;
-                case 5: scatter_level<2>(sm, Af, s_g1, isP, lane, v); break;
-                default: scatter_level<1>(sm, Af, s_g1, isP, lane, v); break;
-                }
-            }
-            __syncthreads();
-            if (tid < C) {
+                const int rr = jrow & 63;
+                if (jrow < 64) {
+                    const float er = s_g1[rr];
 #pragma unroll
-                for (int w = 0; w < PBAND; ++w)
-                    if (tid - w >= 0)
-                        *reinterpret_cast<unsigned short *>(sm + OFF_PBF + sw_elem(8192, tid, tid - w)) =
-                            bf16_bits(s_pband[tid * PBAND + w]);
-            }
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        // ===== 3. T = (I + A)^{-1} =============================================
-        // 16x16 diagonal blocks by forward substitution (one column per thread), then
-        // recursive doubling: T[16(I+1):, 16I:] = -D_{I+1} A_{I+1,I} D_I for I = 0, 2, and
-        // T[32:, :32] = -T2 A21 T1.  fp32 throughout; A rows read four at a time.
-        if (tid < 64) {
-            const int I = tid >> 4, c = tid & 15;
-            float xv[16];
+                    for (int c = 0; c < 32; ++c) {
+                        const int s = phalf * 32 + c;
+                        v[c] = (s < rr) ? v[c] * er : 0.f;
+                    }
 #pragma unroll
-            for (int r2 = 0; r2 < 16; ++r2) {
-                float arow[16];
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        *reinterpret_cast<float4 *>(Af + rr * TP + phalf * 32 + 4 * q4) =
+                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                } else {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<float4 *>(arow + 4 * q4) =
-                        *reinterpret_cast<const float4 *>(Af + (16 * I + r2) * TP + 16 * I + 4 * q4);
-                float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                for (int s2 = 0; s2 < r2; ++s2) {
-                    if (s2 & 1) acc1 = fmaf(arow[s2], xv[s2], acc1);
-                    else acc0 = fmaf(arow[s2], xv[s2], acc0);
-                }
-                xv[r2] = (r2 < c) ? 0.f : ((r2 == c) ? 1.f : -(acc0 + acc1));
-            }
-#pragma unroll
-            for (int r2 = 0; r2 < 16; ++r2) Tf[(16 * I + r2) * TP + 16 * I + c] = xv[r2];
-            for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * TP + 16 * I + c] = 0.f;  // above the block
-        }
-        __syncthreads();
-        {   // X = A_{I+1,I} D_I for I = 0, 2 (two outputs per thread)
-            const int r2 = (tid >> 4) & 15, c2 = tid & 15;
-            float acc[2] = {0.f, 0.f};
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-#pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    const int I = 2 * blk;
-                    const float4 av = *reinterpret_cast<const float4 *>(Af + (16 * I + 16 + r2) * TP + 16 * I + 4 * m4);
-                    const float *tcol = Tf + (16 * I + 4 * m4) * TP + 16 * I + c2;
-                    acc[blk] = fmaf(av.x, tcol[0], acc[blk]);
-                    acc[blk] = fmaf(av.y, tcol[TP], acc[blk]);
-                    acc[blk] = fmaf(av.z, tcol[2 * TP], acc[blk]);
-                    acc[blk] = fmaf(av.w, tcol[3 * TP], acc[blk]);
-                }
-            }
-            Xs[tid] = acc[0];
-            Xs[256 + tid] = acc[1];
-        }
-        __syncthreads();
-        {   // T_{I+1,I} = -D_{I+1} X
-            const int r2 = (tid >> 4) & 15, c2 = tid & 15;
-            float acc[2] = {0.f, 0.f};
-#pragma unroll
-            for (int m4 = 0; m4 < 4; ++m4) {
-#pragma unroll
-                for (int blk = 0; blk < 2; ++blk) {
-                    const int I = 2 * blk;
-                    const float4 tv = *reinterpret_cast<const float4 *>(Tf + (16 * I + 16 + r2) * TP + 16 * I + 16 + 4 * m4);
-                    const float *xcol = Xs + (blk << 8) + (4 * m4) * 16 + c2;
-                    acc[blk] = fmaf(tv.x, xcol[0], acc[blk]);
-                    acc[blk] = fmaf(tv.y, xcol[16], acc[blk]);
-                    acc[blk] = fmaf(tv.z, xcol[32], acc[blk]);
-                    acc[blk] = fmaf(tv.w, xcol[48], acc[blk]);
-                }
-            }
-            Tf[(16 + r2) * TP + c2] = -acc[0];
-            Tf[(48 + r2) * TP + 32 + c2] = -acc[1];
-        }
-        __syncthreads();
-        {   // X = A21 T1 (rows r0 + 8k, column c2)
-            const int r0 = tid >> 5, c2 = tid & 31;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m4 = 0; m4 < 8; ++m4) {
-                const float *tcol = Tf + (4 * m4) * TP + c2;
-                const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + r0 + 8 * k4) * TP + 4 * m4);
-                    acc[k4] = fmaf(av.x, t0v, acc[k4]);
-                    acc[k4] = fmaf(av.y, t1v, acc[k4]);
-                    acc[k4] = fmaf(av.z, t2v, acc[k4]);
-                    acc[k4] = fmaf(av.w, t3v, acc[k4]);
-                }
-            }
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) Xs[(r0 + 8 * k4) * 32 + c2] = acc[k4];
-        }
-        __syncthreads();
-        {   // T21 = -T2 X
-            const int r0 = tid >> 5, c2 = tid & 31;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int m4 = 0; m4 < 8; ++m4) {
-                const float *xcol = Xs + (4 * m4) * 32 + c2;
-                const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 tv = *reinterpret_cast<const float4 *>(Tf + (32 + r0 + 8 * k4) * TP + 32 + 4 * m4);
-                    acc[k4] = fmaf(tv.x, x0, acc[k4]);
-                    acc[k4] = fmaf(tv.y, x1, acc[k4]);
-                    acc[k4] = fmaf(tv.z, x2, acc[k4]);
-                    acc[k4] = fmaf(tv.w, x3, acc[k4]);
-                }
-            }
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + r0 + 8 * k4) * TP + c2] = -acc[k4];
-        }
-        __syncthreads();
-        {   // bf16 K-major copies T Diag(e) and T Diag(w), zero above the diagonal
-            const int r = tid >> 2, kc0 = (tid & 3) * 2;
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-                float te[8], tw[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int s = (kc0 + q2) * 8 + c;
-                    const float t = (s <= r) ? Tf[r * TP + s] : 0.f;
-                    te[c] = t * s_g1[s];
-                    tw[c] = t * s_g2[s];
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_TBF + sw_chunk(8192, r, kc0 + q2)) = pack8(te);
-                *reinterpret_cast<uint4 *>(sm + OFF_UT + sw_chunk(8192, r, kc0 + q2)) = pack8(tw);
-            }
-        }
-        publish();
-
-        // ===== 4. W = T (row operand a~ part);  U^T = M^T T^T ================
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id_w = idesc_bf16(64, 128, false, true);
-            const uint32_t id_u = idesc_bf16(128, 64, true, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16(tbase + TM_W, dK(sb + OFF_TBF, 8192, kk), dMN(sb + OFF_QA, 16384, kk), id_w, kk > 0);
-                mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_UT, 8192, kk), id_u, kk > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        // ===== 5. state pass (overlaps the MMAs above: D_S is not an operand) ===
-        {
-#pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
-                const int i0 = half * 64 + c32 * 32;
-                float s[32], t[32];
-                tmem_ld32(tbase + lane_base + TM_S + i0, s);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    t[e] = s[e] * s_gamC[i0 + e];
-                    if (fast) s[e] = t[e];
-                }
-                // bf16 operand copy of the state (scaled on the fast path)
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
-                tmem_st16(tbase + lane_base + TM_S + i0, t);
-                tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
-            }
-            tmem_wait_st();
-        }
-        wait_mma();
-        if (tid == 0 && ch + 1 < nchunks) issue_tma_v(ch + 1);   // v consumed by U^T = M^T T^T
-        // W (M = 64 layout: rows 16q..16q+15 in lanes 0..15 of quarter q) -> rows 0-63 of QA
-        {
-            const int r = quarter * 16 + (lane & 15);
-#pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
-                float v[32];
-                tmem_ld32(tbase + lane_base + TM_W + half * 64 + c32 * 32, v);
-                tmem_wait_ld();
-                if (lane < 16) {
+                    for (int c = 0; c < 32; ++c) {
+                        const int s = phalf * 32 + c;
+                        const int w = rr - s;
+                        v[c] = (w >= PBAND) ? v[c] : ((w >= 0) ? s_pband[rr * PBAND + w] : 0.f);
+                    }
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, r, half * 8 + c32 * 4 + q4)) =
-                            pack8(v + q4 * 8);
+                        *reinterpret_cast<uint4 *>(sm + OFF_PBF + sw_chunk(8192, rr, phalf * 4 + q4)) = pack8(v + q4 * 8);
+                }
+            } else {
+                // anchored levels: three GEMMs of two levels each
+                for (int p = 0; p < 3; ++p) {
+#pragma unroll 1
+                    for (int slot = 0; slot < 2; ++slot) {
+                        switch (2 * p + 1 + slot) {
+                        case 1: build_level<32>(x, slot, tg, cq); break;
+                        case 2: build_level<16>(x, slot, tg, cq); break;
+                        case 3: build_level<8>(x, slot, tg, cq); break;
+                        case 4: build_level<4>(x, slot, tg, cq); break;
+                        case 5: build_level<2>(x, slot, tg, cq); break;
+                        default: build_level<1>(x, slot, tg, cq); break;
+                        }
+                    }
+                    publish();
+                    if (ptid == 0) {
+                        tc_fence_after();
+                        const uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_bf16(tbase + tm_lvl(p), dK(sb + OFF_LA, 16384, kk), dK(sb + OFF_LB, 8192, kk), idesc,
+                                     kk > 0);
+                        mma_commit(bar_pmma);
+                    }
+                    wait_pmma();
+                }
+                if (ptid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
+                for (int e = ptid; e < 64 * TP; e += NPREP) Af[e] = 0.f;
+                for (int e = ptid; e < 512; e += NPREP)
+                    *reinterpret_cast<uint4 *>(sm + OFF_PBF + e * 16) = make_uint4(0, 0, 0, 0);
+                group_sync(BAR_PREP, NPREP);
+                for (int p = phalf; p < 3; p += 2) {   // the two warps of a lane quarter share the pairs
+                    const int lvl = 2 * p + 1 + (quarter & 1);
+                    const bool isP = quarter >= 2;
+                    float v[32];
+                    tmem_ld32(tbase + lane_base + tm_lvl(p) + (quarter & 1) * 32, v);
+                    tmem_wait_ld();
+                    switch (lvl) {
+                    case 1: scatter_level<32>(sm, Af, s_g1, isP, lane, v); break;
+                    case 2: scatter_level<16>(sm, Af, s_g1, isP, lane, v); break;
+                    case 3: scatter_level<8>(sm, Af, s_g1, isP, lane, v); break;
+                    case 4: scatter_level<4>(sm, Af, s_g1, isP, lane, v); break;
+                    case 5: scatter_level<2>(sm, Af, s_g1, isP, lane, v); break;
+                    default: scatter_level<1>(sm, Af, s_g1, isP, lane, v); break;
+                    }
+                }
+                group_sync(BAR_PREP, NPREP);
+                if (ptid < C) {
+#pragma unroll
+                    for (int w = 0; w < PBAND; ++w)
+                        if (ptid - w >= 0)
+                            *reinterpret_cast<unsigned short *>(sm + OFF_PBF + sw_elem(8192, ptid, ptid - w)) =
+                                bf16_bits(s_pband[ptid * PBAND + w]);
                 }
             }
-        }
-        publish();
+            tc_fence_before();
+            group_sync(BAR_PREP, NPREP);
 
-        // ===== 6. U^T -= S^T W^T ;  O^T = S^T Q^T =============================
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id_neg = idesc_bf16(128, 64, false, false, true);
-            const uint32_t id_pos = idesc_bf16(128, 64, false, false);
+            // ===== 3. T = (I + A)^{-1} =============================================
+            // 16x16 diagonal blocks by forward substitution (one column per thread), then
+            // recursive doubling: T[16(I+1):, 16I:] = -D_{I+1} A_{I+1,I} D_I for I = 0, 2, and
+            // T[32:, :32] = -T2 A21 T1.  fp32 throughout; A rows read four at a time.
+            if (ptid < 64) {
+                const int I = ptid >> 4, c = ptid & 15;
+                float xv[16];
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16(tbase + TM_U, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA, 16384, kk), id_neg, 1);
-                mma_bf16(tbase + TM_O, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA + 8192, 16384, kk), id_pos,
-                         kk > 0);
+                for (int r2 = 0; r2 < 16; ++r2) {
+                    float arow[16];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<float4 *>(arow + 4 * q4) =
+                            *reinterpret_cast<const float4 *>(Af + (16 * I + r2) * TP + 16 * I + 4 * q4);
+                    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                    for (int s2 = 0; s2 < r2; ++s2) {
+                        if (s2 & 1) acc1 = fmaf(arow[s2], xv[s2], acc1);
+                        else acc0 = fmaf(arow[s2], xv[s2], acc0);
+                    }
+                    xv[r2] = (r2 < c) ? 0.f : ((r2 == c) ? 1.f : -(acc0 + acc1));
+                }
+#pragma unroll
+                for (int r2 = 0; r2 < 16; ++r2) Tf[(16 * I + r2) * TP + 16 * I + c] = xv[r2];
+                for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * TP + 16 * I + c] = 0.f;  // above the block
             }
-            mma_commit(bar_mma);
-        }
-        wait_mma();
-        {   // U^T row j, tokens [32*half, +32) -> bf16 K-major tile (rows j, K = token)
-            float v[32];
-            tmem_ld32(tbase + lane_base + TM_U + half * 32, v);
-            tmem_wait_ld();
+            group_sync(BAR_PREP, NPREP);
+            {   // X = A_{I+1,I} D_I for I = 0, 2 (two outputs per thread)
+                const int r2 = (ptid >> 4) & 15, c2 = ptid & 15;
+                float acc[2] = {0.f, 0.f};
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4 *>(sm + OFF_UT + sw_chunk(16384, jcol, half * 4 + q4)) = pack8(v + q4 * 8);
-        }
-        publish();
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 av = *reinterpret_cast<const float4 *>(Af + (16 * I + 16 + r2) * TP + 16 * I + 4 * m4);
+                        const float *tcol = Tf + (16 * I + 4 * m4) * TP + 16 * I + c2;
+                        acc[blk] = fmaf(av.x, tcol[0], acc[blk]);
+                        acc[blk] = fmaf(av.y, tcol[TP], acc[blk]);
+                        acc[blk] = fmaf(av.z, tcol[2 * TP], acc[blk]);
+                        acc[blk] = fmaf(av.w, tcol[3 * TP], acc[blk]);
+                    }
+                }
+                Xs[ptid] = acc[0];
+                Xs[256 + ptid] = acc[1];
+            }
+            group_sync(BAR_PREP, NPREP);
+            {   // T_{I+1,I} = -D_{I+1} X
+                const int r2 = (ptid >> 4) & 15, c2 = ptid & 15;
+                float acc[2] = {0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 tv = *reinterpret_cast<const float4 *>(Tf + (16 * I + 16 + r2) * TP + 16 * I + 16 + 4 * m4);
+                        const float *xcol = Xs + (blk << 8) + (4 * m4) * 16 + c2;
+                        acc[blk] = fmaf(tv.x, xcol[0], acc[blk]);
+                        acc[blk] = fmaf(tv.y, xcol[16], acc[blk]);
+                        acc[blk] = fmaf(tv.z, xcol[32], acc[blk]);
+                        acc[blk] = fmaf(tv.w, xcol[48], acc[blk]);
+                    }
+                }
+                Tf[(16 + r2) * TP + c2] = -acc[0];
+                Tf[(48 + r2) * TP + 32 + c2] = -acc[1];
+            }
+            group_sync(BAR_PREP, NPREP);
+            {   // X = A21 T1 (rows r0 + 8k, column c2)
+                const int r0 = ptid >> 5, c2 = ptid & 31;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *tcol = Tf + (4 * m4) * TP + c2;
+                    const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + r0 + 8 * k4) * TP + 4 * m4);
+                        acc[k4] = fmaf(av.x, t0v, acc[k4]);
+                        acc[k4] = fmaf(av.y, t1v, acc[k4]);
+                        acc[k4] = fmaf(av.z, t2v, acc[k4]);
+                        acc[k4] = fmaf(av.w, t3v, acc[k4]);
+                    }
+                }
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) Xs[(r0 + 8 * k4) * 32 + c2] = acc[k4];
+            }
+            group_sync(BAR_PREP, NPREP);
+            {   // T21 = -T2 X
+                const int r0 = ptid >> 5, c2 = ptid & 31;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *xcol = Xs + (4 * m4) * 32 + c2;
+                    const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 tv = *reinterpret_cast<const float4 *>(Tf + (32 + r0 + 8 * k4) * TP + 32 + 4 * m4);
+                        acc[k4] = fmaf(tv.x, x0, acc[k4]);
+                        acc[k4] = fmaf(tv.y, x1, acc[k4]);
+                        acc[k4] = fmaf(tv.z, x2, acc[k4]);
+                        acc[k4] = fmaf(tv.w, x3, acc[k4]);
+                    }
+                }
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + r0 + 8 * k4) * TP + c2] = -acc[k4];
+            }
+            group_sync(BAR_PREP, NPREP);
 
-        // ===== 7. O^T += U^T P^T ;  S^T += U^T Kbar ===========================
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id_o = idesc_bf16(128, 64, false, false);
-            const uint32_t id_s = idesc_bf16(128, 128, false, true);
+            // ===== 4. W = T Diag(e) (row operand a~ part);  U'^T = M^T (T Diag(w))^T ==
+            // T copies go through one bf16 tile: T Diag(e) for W, then (RDA only, whose two
+            // gates differ) T Diag(w) for U' once the W GEMM has read the first copy.
+            auto write_t_copy = [&](const float *gate) {
+                const int r = ptid >> 2, kc0 = (ptid & 3) * 2;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                mma_bf16(tbase + TM_O, dK(sb + OFF_UT, 16384, kk), dK(sb + OFF_PBF, 8192, kk), id_o, 1);
-                mma_bf16(tbase + TM_S, dK(sb + OFF_UT, 16384, kk), dMN(sb + OFF_KB, 8192, kk), id_s, 1);
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    float te[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int s = (kc0 + q2) * 8 + c;
+                        te[c] = (s <= r) ? Tf[r * TP + s] * gate[s] : 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_TBF + sw_chunk(8192, r, kc0 + q2)) = pack8(te);
+                }
+            };
+            write_t_copy(s_g1);
+            publish();
+            // U'^T overwrites TMEM U: the chain must have read the previous chunk's U out
+            if (ch > 0 && !mbar_wait_cycles(bar_ufree, ppar, WAIT_CYCLES)) ok = false;
+            if (ptid == 0) {
+                tc_fence_after();
+                const uint32_t id_w = idesc_bf16(64, 128, false, true);
+                const uint32_t id_u = idesc_bf16(128, 64, true, false);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    mma_bf16(tbase + TM_W, dK(sb + OFF_TBF, 8192, kk), dMN(sb + OFF_QA, 16384, kk), id_w, kk > 0);
+                    if (same_gates)
+                        mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_TBF, 8192, kk), id_u, kk > 0);
+                }
+                mma_commit(bar_pmma);
             }
-            mma_commit(bar_mma);
-        }
-        wait_mma();
-        {   // o: TMEM (lane j, column r) -> bf16 staging [r][j] -> 16-byte rows to HBM
-            float v[32];
-            tmem_ld32(tbase + lane_base + TM_O + half * 32, v);
-            tmem_wait_ld();
-            unsigned short *ost = reinterpret_cast<unsigned short *>(sm + OFF_OST);
+            wait_pmma();
+            if (!same_gates) {
+                write_t_copy(s_g2);
+                publish();
+                if (ptid == 0) {
+                    tc_fence_after();
+                    const uint32_t id_u = idesc_bf16(128, 64, true, false);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ost[(half * 32 + e) * 128 + jcol] = bf16_bits(v[e]);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_TBF, 8192, kk), id_u, kk > 0);
+                    mma_commit(bar_pmma);
+                }
+                wait_pmma();
+            }
+            if (ptid == 0 && ch + 1 < nchunks) issue_tma_v(ch + 1);   // v consumed by U'^T = M^T T^T
+            // W (M = 64 layout: rows 16q..16q+15 in lanes 0..15 of quarter q) -> rows 0-63 of QA
+            {
+                const int r = quarter * 16 + (lane & 15);
+#pragma unroll
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    float v[32];
+                    tmem_ld32(tbase + lane_base + TM_W + phalf * 64 + c32 * 32, v);
+                    tmem_wait_ld();
+                    if (lane < 16) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, r, phalf * 8 + c32 * 4 + q4)) =
+                                pack8(v + q4 * 8);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            ok = group_sync_and(BAR_PREP, NPREP, ok);
+            if (ptid == 0) mbar_arrive(bar_ready);   // chunk ch's operands are ready for the chain
         }
-        __syncthreads();
-        for (int e = tid; e < nvalid * 16; e += NT) {
-            const int r = e >> 4, cgo = e & 15;
-            *reinterpret_cast<uint4 *>(op + (((rowbase + r) * H + h) * D + cgo * 8) * 2) =
-                *reinterpret_cast<const uint4 *>(sm + OFF_OST + r * 256 + cgo * 16);
+        if (!ok) {  // drain TMA still in flight (bounded)
+            mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
+            mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
         }
-        fence_async_smem();
-        tc_fence_before();
-        ok = __syncthreads_and(ok) != 0;  // every thread leaves the loop together
     }
 
     // ---- final state (NaN if an internal wait timed out) ----------------------
+    __syncthreads();
     tc_fence_after();
-    if (a.sf) {
+    ok = __syncthreads_and(ok) != 0;
+    if (warp < 4 && a.sf) {
         const size_t soff = ((size_t)n * H + h) * D * D;
-#pragma unroll
-        for (int c32 = 0; c32 < 2; ++c32) {
-            const int i0 = half * 64 + c32 * 32;
+        const int jcol = tid;
+#pragma unroll 1
+        for (int c32 = 0; c32 < 4; ++c32) {
+            const int i0 = c32 * 32;
             float s[32];
             tmem_ld32(tbase + lane_base + TM_S + i0, s);
             tmem_wait_ld();
@@ -906,10 +984,6 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             for (int e = 0; e < 32; ++e)
                 a.sf[soff + (size_t)(i0 + e) * D + jcol] = ok ? s[e] : __int_as_float(0x7fc00000);
         }
-    }
-    if (!ok) {  // drain TMA still in flight (bounded)
-        mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
-        mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
     }
     tc_fence_before();
     __syncthreads();

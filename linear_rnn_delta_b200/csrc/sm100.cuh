@@ -127,6 +127,29 @@ __device__ __forceinline__ bool mbar_wait_cycles(uint64_t *mbar, uint32_t parity
     return true;
 }
 
+// ---- named barriers (one group of warps; id 0 is __syncthreads) -----------
+__device__ __forceinline__ void group_sync(uint32_t id, uint32_t nthreads)
+{
+    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(nthreads) : "memory");
+}
+// barrier over `nthreads` that also returns the AND of `pred` over them
+__device__ __forceinline__ bool group_sync_and(uint32_t id, uint32_t nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(nthreads) : "memory");
+    return r != 0;
+}
+// one arrival on an mbarrier (count-based phase)
+__device__ __forceinline__ void mbar_arrive(uint64_t *mbar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(mbar)) : "memory");
+}
+
 // ---- TMEM <-> registers (32 lanes x N columns of 32 bit per warp) ---------
 // Warp w may only touch lanes 32*(w%4) .. 32*(w%4)+31; thread t gets lane
 // 32*(w%4)+t.  taddr = (lane << 16) | column.
