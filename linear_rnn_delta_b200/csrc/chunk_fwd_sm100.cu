@@ -593,33 +593,53 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                 if (!mbar_wait_cycles(bar_s7, ppar, WAIT_CYCLES)) ok = false;
             }
 
-            // ===== 1b. row operands (Gamma a~ | Gamma q, scaled on the fast path), Kbar, band of P
-            {
-                float pre[4] = {1.f, 1.f, 1.f, 1.f}, suf[4] = {1.f, 1.f, 1.f, 1.f};
+            // ===== 1b. row operands, Kbar and the exact band of P ================
+            if (fast) {
+                // Fast path, one forward sweep.  sc = Gamma_r / Gamma_C, |sc| >= 1 (all |alpha| <= 1), so
+                //   row operands  Gamma a~ / Gamma_C = sc (.) a~,  Gamma q / Gamma_C = sc (.) q,
+                //   Kbar_r = Lam_{C-1,r} (.) k_r = k_r / sc   (divisor bounded away from zero),
+                // and the band P_{r,r-w} = sum_c (sc q)_r (Kbar)_{r-w} comes exactly from these fp32
+                // values: a sliding window keeps Kbar of the four previous rows, and each row's five
+                // partial sums over this lane's 4 channels are reduce-scattered across the warp (the
+                // 32 lanes of a warp are the 32 channel quads of one 8-token block).
+                float pre[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
-                    if (g == tg) continue;
+                    if (g >= tg) break;
                     float t4[4];
                     load_tot4(s_tot, g, cq, t4);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        if (g < tg) pre[c] *= t4[c];
-                        else suf[c] *= t4[c];
+                    for (int c = 0; c < 4; ++c) pre[c] *= t4[c];
+                }
+                const float4 gc4 = *reinterpret_cast<const float4 *>(s_gamC + par * 128 + cq * 4);
+                float sc[4] = {pre[0] / gc4.x, pre[1] / gc4.y, pre[2] / gc4.z, pre[3] / gc4.w};
+                float kw[4][4];   // Kbar of rows r-4 .. r-1
+                {
+                    float sb4[4] = {sc[0], sc[1], sc[2], sc[3]};   // Gamma_{8tg-1} / Gamma_C
+#pragma unroll
+                    for (int j = 3; j >= 0; --j) {
+                        const int rp = tg * 8 - 4 + j;
+                        if (rp >= 0) {
+                            float kv[4], av[4];
+                            unpack4(raw_quad(sm, RAW_K, rp, cq), kv);
+                            unpack4(raw_quad(sm, RAW_A, rp, cq), av);
+                            const bool v = rp < nvalid;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                kw[j][c] = v ? __fdividef(kv[c], sb4[c]) : 0.f;
+                                sb4[c] = v ? __fdividef(sb4[c], av[c]) : sb4[c];
+                            }
+                        } else {
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) kw[j][c] = 0.f;
+                        }
                     }
                 }
-                float sc[4];
-                if (fast) {
-                    const float4 gc4 = *reinterpret_cast<const float4 *>(s_gamC + par * 128 + cq * 4);
-                    sc[0] = pre[0] / gc4.x; sc[1] = pre[1] / gc4.y; sc[2] = pre[2] / gc4.z; sc[3] = pre[3] / gc4.w;
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) sc[c] = pre[c];
-                }
-#pragma unroll 2
-                for (int i = 0; i < 8; ++i) {   // forward: rows 0-63 Gamma a~, rows 64-127 Gamma q
+#pragma unroll 1
+                for (int i = 0; i < 8; ++i) {
                     const int r = tg * 8 + i;
                     const bool v = r < nvalid;
-                    float al[4], kv[4], qv[4], e[4], oa[4], oq[4];
+                    float al[4], kv[4], qv[4], e[4], oa[4], oq[4], kb[4];
                     unpack4(raw_quad(sm, RAW_A, r, cq), al);
                     unpack4(raw_quad(sm, RAW_K, r, cq), kv);
                     unpack4(raw_quad(sm, RAW_Q, r, cq), qv);
@@ -629,60 +649,134 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                         sc[c] *= v ? al[c] : 1.f;
                         oa[c] = v ? sc[c] * (e[c] * kv[c]) : 0.f;
                         oq[c] = v ? sc[c] * qv[c] : 0.f;
+                        kb[c] = v ? __fdividef(kv[c], sc[c]) : 0.f;
                     }
                     *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, r, cq)) = pack4(oa);
                     *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, 64 + r, cq)) = pack4(oq);
-                }
-                float sx[4];
+                    *reinterpret_cast<uint2 *>(sm + OFF_KB + sw_half(8192, r, cq)) = pack4(kb);
+                    // partial sums of P_{r,r-w} over this lane's channels, slots 5-7 unused
+                    float pv[8];
+                    pv[0] = oq[0] * kb[0] + oq[1] * kb[1] + oq[2] * kb[2] + oq[3] * kb[3];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) sx[c] = suf[c];
-#pragma unroll 2
-                for (int i = 7; i >= 0; --i) {   // backward: Kbar_s = (prod_{s<t<C} alpha_t) (.) k_s
-                    const int r = tg * 8 + i;
-                    const bool v = r < nvalid;
-                    float al[4], kv[4], kb[4];
-                    unpack4(raw_quad(sm, RAW_A, r, cq), al);
-                    unpack4(raw_quad(sm, RAW_K, r, cq), kv);
+                    for (int w = 1; w < PBAND; ++w)
+                        pv[w] = oq[0] * kw[4 - w][0] + oq[1] * kw[4 - w][1] + oq[2] * kw[4 - w][2] + oq[3] * kw[4 - w][3];
+                    pv[5] = pv[6] = pv[7] = 0.f;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        kb[c] = v ? sx[c] * kv[c] : 0.f;
-                        sx[c] *= v ? al[c] : 1.f;
+                        kw[0][c] = kw[1][c]; kw[1][c] = kw[2][c]; kw[2][c] = kw[3][c]; kw[3][c] = kb[c];
                     }
-                    *reinterpret_cast<uint2 *>(sm + OFF_KB + sw_half(8192, r, cq)) = pack4(kb);
+                    // reduce-scatter of 8 slots over 32 lanes: lane keeps slot 4*b4 + 2*b3 + b2
+                    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float send = b4 ? pv[k] : pv[k + 4];
+                        pv[k] = (b4 ? pv[k + 4] : pv[k]) + __shfl_xor_sync(0xffffffffu, send, 16);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        const float send = b3 ? pv[k] : pv[k + 2];
+                        pv[k] = (b3 ? pv[k + 2] : pv[k]) + __shfl_xor_sync(0xffffffffu, send, 8);
+                    }
+                    {
+                        const float send = b2 ? pv[0] : pv[1];
+                        pv[0] = (b2 ? pv[1] : pv[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+                    }
+                    pv[0] += __shfl_xor_sync(0xffffffffu, pv[0], 2);
+                    pv[0] += __shfl_xor_sync(0xffffffffu, pv[0], 1);
+                    const int slot = (b4 ? 4 : 0) + (b3 ? 2 : 0) + (b2 ? 1 : 0);
+                    if ((lane & 3) == 0 && slot < PBAND) s_pband[r * PBAND + slot] = (v && r - slot >= 0) ? pv[0] : 0.f;
                 }
-            }
-            {   // band of P: P_{r,r-w} = sum_c q_rc (alpha_r ... alpha_{r-w+1})_c k_{r-w,c}, w = 0..4,
-                // from the bf16 inputs in fp32: the entries whose bf16 GEMM rounding would hurt most.
-                // Four threads per row (32 channels each), chunk order staggered by row so the loads
-                // are bank-conflict free; rows below w are clamped and masked afterwards.
-                const int r = ptid >> 2, c4 = ptid & 3;
-                float acc[PBAND];
+            } else {
+            {
+                    float pre[4] = {1.f, 1.f, 1.f, 1.f}, suf[4] = {1.f, 1.f, 1.f, 1.f};
 #pragma unroll
-                for (int w = 0; w < PBAND; ++w) acc[w] = 0.f;
-#pragma unroll 1
-                for (int j = 0; j < 4; ++j) {
-                    const int cgx = c4 * 4 + ((j + r) & 3);
-                    float hv[8];
-                    unpack8(raw_row(sm, RAW_Q, r, cgx), hv);
+                    for (int g = 0; g < 8; ++g) {
+                        if (g == tg) continue;
+                        float t4[4];
+                        load_tot4(s_tot, g, cq, t4);
 #pragma unroll
-                    for (int w = 0; w < PBAND; ++w) {
-                        float kv[8];
-                        unpack8(raw_row(sm, RAW_K, max(r - w, 0), cgx), kv);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) acc[w] = fmaf(hv[c], kv[c], acc[w]);
-                        if (w + 1 < PBAND) {
-                            float av[8];
-                            unpack8(raw_row(sm, RAW_A, max(r - w, 0), cgx), av);
-#pragma unroll
-                            for (int c = 0; c < 8; ++c) hv[c] *= av[c];
+                        for (int c = 0; c < 4; ++c) {
+                            if (g < tg) pre[c] *= t4[c];
+                            else suf[c] *= t4[c];
                         }
                     }
-                }
+                    float sc[4];
+                    if (fast) {
+                        const float4 gc4 = *reinterpret_cast<const float4 *>(s_gamC + par * 128 + cq * 4);
+                        sc[0] = pre[0] / gc4.x; sc[1] = pre[1] / gc4.y; sc[2] = pre[2] / gc4.z; sc[3] = pre[3] / gc4.w;
+                    } else {
 #pragma unroll
-                for (int w = 0; w < PBAND; ++w) {
-                    float t = acc[w] + __shfl_xor_sync(0xffffffffu, acc[w], 1);
-                    t += __shfl_xor_sync(0xffffffffu, t, 2);
-                    if (c4 == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? t : 0.f;
+                        for (int c = 0; c < 4; ++c) sc[c] = pre[c];
+                    }
+#pragma unroll 2
+                    for (int i = 0; i < 8; ++i) {   // forward: rows 0-63 Gamma a~, rows 64-127 Gamma q
+                        const int r = tg * 8 + i;
+                        const bool v = r < nvalid;
+                        float al[4], kv[4], qv[4], e[4], oa[4], oq[4];
+                        unpack4(raw_quad(sm, RAW_A, r, cq), al);
+                        unpack4(raw_quad(sm, RAW_K, r, cq), kv);
+                        unpack4(raw_quad(sm, RAW_Q, r, cq), qv);
+                        erase_gate4(x, r, cq, e);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            sc[c] *= v ? al[c] : 1.f;
+                            oa[c] = v ? sc[c] * (e[c] * kv[c]) : 0.f;
+                            oq[c] = v ? sc[c] * qv[c] : 0.f;
+                        }
+                        *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, r, cq)) = pack4(oa);
+                        *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, 64 + r, cq)) = pack4(oq);
+                    }
+                    float sx[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sx[c] = suf[c];
+#pragma unroll 2
+                    for (int i = 7; i >= 0; --i) {   // backward: Kbar_s = (prod_{s<t<C} alpha_t) (.) k_s
+                        const int r = tg * 8 + i;
+                        const bool v = r < nvalid;
+                        float al[4], kv[4], kb[4];
+                        unpack4(raw_quad(sm, RAW_A, r, cq), al);
+                        unpack4(raw_quad(sm, RAW_K, r, cq), kv);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            kb[c] = v ? sx[c] * kv[c] : 0.f;
+                            sx[c] *= v ? al[c] : 1.f;
+                        }
+                        *reinterpret_cast<uint2 *>(sm + OFF_KB + sw_half(8192, r, cq)) = pack4(kb);
+                    }
+                }
+                {   // band of P: P_{r,r-w} = sum_c q_rc (alpha_r ... alpha_{r-w+1})_c k_{r-w,c}, w = 0..4,
+                    // from the bf16 inputs in fp32: the entries whose bf16 GEMM rounding would hurt most.
+                    // Four threads per row (32 channels each), chunk order staggered by row so the loads
+                    // are bank-conflict free; rows below w are clamped and masked afterwards.
+                    const int r = ptid >> 2, c4 = ptid & 3;
+                    float acc[PBAND];
+#pragma unroll
+                    for (int w = 0; w < PBAND; ++w) acc[w] = 0.f;
+#pragma unroll 1
+                    for (int j = 0; j < 4; ++j) {
+                        const int cgx = c4 * 4 + ((j + r) & 3);
+                        float hv[8];
+                        unpack8(raw_row(sm, RAW_Q, r, cgx), hv);
+#pragma unroll
+                        for (int w = 0; w < PBAND; ++w) {
+                            float kv[8];
+                            unpack8(raw_row(sm, RAW_K, max(r - w, 0), cgx), kv);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) acc[w] = fmaf(hv[c], kv[c], acc[w]);
+                            if (w + 1 < PBAND) {
+                                float av[8];
+                                unpack8(raw_row(sm, RAW_A, max(r - w, 0), cgx), av);
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) hv[c] *= av[c];
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int w = 0; w < PBAND; ++w) {
+                        float t = acc[w] + __shfl_xor_sync(0xffffffffu, acc[w], 1);
+                        t += __shfl_xor_sync(0xffffffffu, t, 2);
+                        if (c4 == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? t : 0.f;
+                    }
                 }
             }
             group_sync(BAR_PREP, NPREP);   // band and row operands complete before either A/P path reads them
