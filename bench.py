@@ -242,7 +242,20 @@ def pct(xs, p):
     return float(np.percentile(np.asarray(xs), p))
 
 
-def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True):
+FORM_FLAGS = {"auto": 0, "fused": 4, "split": 8}
+
+
+def chunk_form(inp, flags=0) -> str:
+    """Which form of the tensor-core path the library runs for this workload:
+    it needs a workspace exactly when it runs the split form."""
+    import linear_rnn_delta_b200 as kda
+    ws = kda.lib.kda_chunk_fwd_workspace_size(0 if inp.dtype == "bf16" else 1, inp.B, inp.T, inp.H, inp.d_k,
+                                              inp.d_v, int(inp.cu_seqlens is not None), inp.num_seqs,
+                                              inp.chunk_size, flags)
+    return "split" if ws else "fused"
+
+
+def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True, flags=0):
     import linear_rnn_delta_b200 as kda
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
@@ -257,7 +270,7 @@ def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True)
     def step():
         kda.kda_chunk_fwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"],
                           cu_seqlens=cu, initial_state=s0, final_state=sf, o=o, chunk_size=inp.chunk_size,
-                          stream=stream)
+                          flags=flags, stream=stream)
 
     if sampler:
         sampler.start()
@@ -266,7 +279,9 @@ def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True)
     total = max_over_ranks(total, world)
     alg = chunk_algorithmic(inp)
     avg = sum(per) / len(per)
-    res = {"tokens_per_step": alg["tokens"], "total_s": total, "avg_launch_s": avg,
+    form = chunk_form(inp, flags)
+    res = {"tokens_per_step": alg["tokens"], "total_s": total, "avg_launch_s": avg, "form": form,
+           "kernels_per_step": 2 if form == "split" else 1,
            "p50_ms": pct(per, 50) * 1e3, "p95_ms": pct(per, 95) * 1e3, "p99_ms": pct(per, 99) * 1e3,
            "alg": alg, "clocks": clocks}
     gbs = alg["bytes"] / avg / 1e9
@@ -274,11 +289,11 @@ def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True)
     res["hbm"] = {"achieved": gbs, "peak": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"]}
     res["tensor"] = {"achieved": tfs, "peak": peaks["bf16_tflops"], "frac": tfs / peaks["bf16_tflops"]}
     if e2e:
-        res["e2e"] = chunk_e2e(inp, d, cu, s0, o, sf, steps, warmup, world, stream)
+        res["e2e"] = chunk_e2e(inp, d, cu, s0, o, sf, steps, warmup, world, stream, flags)
     return res
 
 
-def chunk_e2e(inp, d, cu, s0, o, sf, steps, warmup, world, stream):
+def chunk_e2e(inp, d, cu, s0, o, sf, steps, warmup, world, stream, flags=0):
     """Same step through the public API with pinned host buffers: H2D of the
     step's inputs, the kernel, D2H of o and the final state, all timed."""
     import linear_rnn_delta_b200 as kda
@@ -295,7 +310,7 @@ def chunk_e2e(inp, d, cu, s0, o, sf, steps, warmup, world, stream):
                 d[n].copy_(t, non_blocking=True)
         kda.kda_chunk_fwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"],
                           cu_seqlens=cu, initial_state=s0, final_state=sf, o=o, chunk_size=inp.chunk_size,
-                          stream=stream)
+                          flags=flags, stream=stream)
         o_h.copy_(o, non_blocking=True)
         sf_h.copy_(sf, non_blocking=True)
 
@@ -428,6 +443,8 @@ def main():
     ap.add_argument("--extra", action="store_true", help="also time Complex-KDA 8x16x8192 and varlen RDA/GDN-2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--form", choices=sorted(FORM_FLAGS), default="auto",
+                    help="form of the tensor-core chunked path (auto = the library's shape-based choice)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -442,7 +459,8 @@ def main():
     peaks = load_peaks()
     inp = W.kda_bf16(seed=rank_workload_seed(rank))
     sampler = ClockSampler(local) if rank == 0 else None
-    main_res = run_chunk_workload(inp, args.steps, args.warmup, world, peaks, sampler=sampler)
+    fflags = FORM_FLAGS[args.form]
+    main_res = run_chunk_workload(inp, args.steps, args.warmup, world, peaks, sampler=sampler, flags=fflags)
     decode = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank)
     also = []
     if args.extra:
@@ -450,9 +468,10 @@ def main():
                          ("RDA varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("rda", rank)),
                          ("GDN-2 varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("gdn2", rank))):
             x = mk()
-            r = run_chunk_workload(x, max(5, args.steps // 2), args.warmup, world, peaks, e2e=False)
+            r = run_chunk_workload(x, max(5, args.steps // 2), args.warmup, world, peaks, e2e=False, flags=fflags)
             also.append({"workload": name, "value": r["tokens_per_step"] * world * max(5, args.steps // 2) / r["total_s"],
-                         "unit": UNIT, "ms_per_step": r["avg_launch_s"] * 1e3, "hbm_frac": r["hbm"]["frac"],
+                         "unit": UNIT, "ms_per_step": r["avg_launch_s"] * 1e3, "form": r["form"],
+                         "hbm_frac": r["hbm"]["frac"],
                          "tensor_frac": r["tensor"]["frac"], "achieved_gbs": r["hbm"]["achieved"],
                          "achieved_tflops": r["tensor"]["achieved"]})
             del x
@@ -479,15 +498,18 @@ def main():
         "p50_ms": main_res["p50_ms"], "p95_ms": main_res["p95_ms"], "p99_ms": main_res["p99_ms"],
         "roofline": {"bound": "hbm", "achieved": main_res["hbm"]["achieved"], "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": main_res["hbm"]["frac"],
-                     "traffic": measured_traffic("chunk_fwd_kda_4x16x4096", CHUNK_SOURCES).get("dram_bytes_per_launch"),
+                     "traffic": measured_traffic(f"chunk_fwd_kda_4x16x4096_{main_res['form']}",
+                                                 CHUNK_SOURCES).get("dram_bytes_per_launch"),
                      "peak_source": peaks["source"],
-                     "kernel": "kda_chunk_fwd (one launch per step)",
+                     "kernel": ("kda_chunk_fwd, split form: preparation + chain kernels timed as one call"
+                                if main_res["form"] == "split" else "kda_chunk_fwd, fused form: one kernel"),
+                     "form": main_res["form"],
                      "alg_bytes_per_launch": main_res["alg"]["bytes"]},
         "tensor": {"achieved": main_res["tensor"]["achieved"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                    "frac": main_res["tensor"]["frac"], "alg_flops_per_launch": main_res["alg"]["flops"]},
         "e2e": {"value": tokens * args.steps / e2e["total_s"], "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * main_res["kernels_per_step"],
         "clocks": main_res["clocks"],
         "decode": decode,
         "cpu_baseline": cpu and {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},

@@ -34,6 +34,7 @@
 #ifndef KDA_H_
 #define KDA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -67,6 +68,8 @@ enum kda_status {
  * writes its verdict to caller memory; the forward calls never check them.) */
 #define KDA_FLAG_FORCE_SCAN     2u  /* use the token-by-token CUDA scan kernel even where the
                                        tensor-core chunked kernel applies (testing aid) */
+#define KDA_FLAG_FORCE_FUSED    4u  /* tensor-core path: force the single fused kernel */
+#define KDA_FLAG_FORCE_SPLIT    8u  /* tensor-core path: force the two-kernel path */
 
 /*
  * kda_chunk_fwd -- chunked-parallel forward over whole sequences.
@@ -87,10 +90,22 @@ enum kda_status {
  *   o             : [B,T,H,d_v] output, same dtype as q
  * Sizes: B >= 1, T >= 0, H >= 1, d_k and d_v in {16, 32, 64, 128},
  * chunk_size in {16, 32, 64, 128}.  With bf16, d_k = d_v = 128 and
- * chunk_size = 64 the tcgen05 tensor-core chunked kernel runs (WY/UT form,
+ * chunk_size = 64 the tcgen05 tensor-core chunked path runs (WY/UT form,
  * fp32 accumulation, fp32 state kept on chip); every other accepted case
  * runs the token-by-token fp32 CUDA scan, whose result does not depend on
  * chunk_size.  Results of the two agree to rounding.
+ * The tensor-core path has two forms with bit-identical results:
+ *   fused -- one kernel, one CTA per (sequence, head) builds each chunk's
+ *            operands and runs the state chain; no workspace;
+ *   split -- a persistent kernel over all SMs builds every chunk's operands
+ *            into a workspace, then one CTA per (sequence, head) runs the
+ *            chain.  Its workspace holds about 81 KiB per (chunk, head); here
+ *            it is allocated stream-ordered (cudaMallocAsync) on `stream`
+ *            and freed on it before the call returns, and if that fails the
+ *            fused form runs instead.  kda_chunk_fwd_ws takes a caller-owned
+ *            workspace instead.
+ * The form is chosen by problem shape unless KDA_FLAG_FORCE_FUSED or
+ * KDA_FLAG_FORCE_SPLIT (mutually exclusive) names one.
  * Returns KDA_OK or a KDA_ERR_* code.
  */
 int kda_chunk_fwd(int variant, int gate_range, int dtype,
@@ -100,6 +115,36 @@ int kda_chunk_fwd(int variant, int gate_range, int dtype,
                   const int32_t *cu_seqlens, int num_seqs,
                   const float *initial_state, float *final_state,
                   void *o, int chunk_size, unsigned flags, void *stream);
+
+/*
+ * kda_chunk_fwd_workspace_size -- bytes of workspace kda_chunk_fwd_ws needs
+ * for these sizes and flags: (N + ceil(B*T / 64)) * H * 82944 when the split
+ * form would run, N = num_seqs with cu_seqlens (has_cu_seqlens = 1) or B
+ * without; 0 when another form runs (scan: dtype, head dims or chunk size;
+ * fused: chosen by shape on the current device or forced) and when an
+ * argument is out of range.  By shape, the split form is chosen when
+ * 2 * N * H <= the device's SM count.
+ */
+size_t kda_chunk_fwd_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
+                                    int has_cu_seqlens, int num_seqs, int chunk_size, unsigned flags);
+
+/*
+ * kda_chunk_fwd_ws -- kda_chunk_fwd with a caller-owned DEVICE workspace of
+ * `workspace_bytes` bytes (16-byte aligned; not read before it is written,
+ * contents undefined afterwards; it must stay allocated until the call's
+ * work on `stream` has finished).  The split form runs when chosen and the
+ * workspace holds at least kda_chunk_fwd_workspace_size(...) bytes;
+ * otherwise the fused form runs (KDA_FLAG_FORCE_SPLIT with a NULL or short
+ * workspace is KDA_ERR_INVALID_ARG).  Nothing is allocated.
+ */
+int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
+                     int B, int T, int H, int d_k, int d_v,
+                     const void *q, const void *k, const void *v, const void *alpha,
+                     const void *g1, const void *g2,
+                     const int32_t *cu_seqlens, int num_seqs,
+                     const float *initial_state, float *final_state,
+                     void *o, int chunk_size, void *workspace, size_t workspace_bytes,
+                     unsigned flags, void *stream);
 
 /*
  * kda_decode_step -- one recurrent step for N sequences (single-token decode;

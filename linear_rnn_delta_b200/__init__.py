@@ -2,7 +2,7 @@
 decay: KDA, Complex KDA, RDA and GDN-2.
 
 This module is a thin ctypes binding over the C ABI in ``include/kda.h``
-(``libkda.so``, built in-tree by ``python -m linear_rnn_delta_b200.build``).
+(``libkda.so``, built in-tree by ``python linear_rnn_delta_b200/build.py``).
 It only marshals arguments: it reads shapes and device pointers off torch
 tensors, picks the caller's current CUDA stream, and allocates outputs the
 caller did not pass.  Every step of the recurrence runs in the library's
@@ -18,14 +18,17 @@ from typing import Optional, Union
 import torch
 
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_version",
-           "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_FORCE_SCAN"]
+           "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_FORCE_SCAN", "FLAG_FORCE_FUSED",
+           "FLAG_FORCE_SPLIT"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
 VARIANTS = {"kda": 0, "rda": 1, "gdn2": 2}
 RANGES = {"standard": 0, "extended": 1}
 _DTYPES = {torch.bfloat16: 0, torch.float32: 1}
-FLAG_FORCE_SCAN = 2
+FLAG_FORCE_SCAN = 2    # token-by-token CUDA scan even where the tensor-core path applies
+FLAG_FORCE_FUSED = 4   # tensor-core path, single fused kernel
+FLAG_FORCE_SPLIT = 8   # tensor-core path, preparation kernel + chain kernel
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -33,11 +36,21 @@ _i = ctypes.c_int
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_rnn_delta_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python linear_rnn_delta_b200/build.py` "
                           "(the recurrence has no implementation other than its CUDA kernels)")
     lib = ctypes.CDLL(LIB_PATH)
+    for name in ("kda_chunk_fwd", "kda_chunk_fwd_ws", "kda_chunk_fwd_workspace_size", "kda_decode_step",
+                 "kda_check_gates", "kda_error_string", "kda_last_error_detail", "kda_version"):
+        if not hasattr(lib, name):
+            raise ImportError(f"{LIB_PATH} lacks {name}: it is stale, rebuild it with "
+                              "`python linear_rnn_delta_b200/build.py`")
     lib.kda_chunk_fwd.restype = _i
     lib.kda_chunk_fwd.argtypes = [_i] * 8 + [_vp] * 6 + [_vp, _i, _vp, _vp, _vp, _i, ctypes.c_uint, _vp]
+    lib.kda_chunk_fwd_ws.restype = _i
+    lib.kda_chunk_fwd_ws.argtypes = ([_i] * 8 + [_vp] * 6 + [_vp, _i, _vp, _vp, _vp, _i, _vp, ctypes.c_size_t,
+                                                            ctypes.c_uint, _vp])
+    lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.kda_chunk_fwd_workspace_size.argtypes = [_i] * 9 + [ctypes.c_uint]
     lib.kda_decode_step.restype = _i
     lib.kda_decode_step.argtypes = [_i] * 7 + [_vp] * 6 + [_vp, _vp, ctypes.c_uint, _vp]
     lib.kda_check_gates.restype = _i
@@ -105,7 +118,8 @@ def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torc
                   cu_seqlens: Optional[torch.Tensor] = None, initial_state: Optional[torch.Tensor] = None,
                   final_state: Union[torch.Tensor, bool, None] = True, o: Optional[torch.Tensor] = None,
                   chunk_size: int = 64, flags: int = 0, stream=None):
-    """Chunked forward of the recurrence over whole sequences (C: kda_chunk_fwd).
+    """Chunked forward of the recurrence over whole sequences (C: kda_chunk_fwd_ws,
+    with the split form's workspace taken from torch's caching allocator).
 
     q, k, alpha [B,T,H,d_k]; v [B,T,H,d_v]; g1/g2 per variant (KDA: beta
     [B,T,H], g2 None; RDA: e, w [B,T,H]; GDN-2: b [B,T,H,d_k], w [B,T,H,d_v]);
@@ -151,9 +165,18 @@ def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torc
     if o is None:
         o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
     _check(o, "o", dt, (B, T, H, dv), dev)
-    rc = lib.kda_chunk_fwd(var, rng, _DTYPES[dt], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                           _ptr(g1), _ptr(g2), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(final_state),
-                           _ptr(o), int(chunk_size), int(flags), _stream(stream, dev))
+    # workspace of the split form, from torch's caching allocator (no per-call device allocation)
+    ws_bytes = lib.kda_chunk_fwd_workspace_size(_DTYPES[dt], B, T, H, dk, dv, int(cu_seqlens is not None), N,
+                                                int(chunk_size), int(flags))
+    ws = None
+    if ws_bytes:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        if stream is not None and stream != torch.cuda.current_stream(dev):
+            ws.record_stream(stream)
+    rc = lib.kda_chunk_fwd_ws(var, rng, _DTYPES[dt], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                              _ptr(g1), _ptr(g2), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(final_state),
+                              _ptr(o), int(chunk_size), _ptr(ws), ws_bytes if ws is not None else 0, int(flags),
+                              _stream(stream, dev))
     if rc != 0:
         raise KdaError(rc, "kda_chunk_fwd")
     return o, final_state

@@ -1,6 +1,8 @@
 """Build the kda C-ABI shared library (libkda.so) for sm_100a, in-tree.
 
-    python -m linear_rnn_delta_b200.build [--force] [--verbose]
+    python linear_rnn_delta_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package loads the library, which may not exist yet)
 
 Every ``csrc/*.cu`` is compiled with nvcc for ``sm_100a`` only and linked
 into ``linear_rnn_delta_b200/libkda.so`` (CUDA runtime linked statically, so

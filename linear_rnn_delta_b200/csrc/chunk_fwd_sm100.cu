@@ -34,11 +34,11 @@
 //    one dense GEMM.  Six levels cover every pair s < r once; P_{r,r} = q_r . k_r.
 //    Nothing is divided, so zeros and signs propagate exactly.
 //
-// One CTA of 512 threads per (sequence, head); the fp32 state lives in tensor memory (TMEM)
-// for the whole sequence, transposed (lane = value column j, column = key
-// channel i), so every state-dependent GEMM has M = d_v = 128.  q, k, v,
-// alpha arrive by TMA; every other operand is built on chip in 128-byte
-// swizzled shared-memory tiles.  Per chunk:
+// Fused form: one CTA of 384 threads per (sequence, head); the fp32 state
+// lives in tensor memory (TMEM) for the whole sequence, transposed (lane =
+// value column j, column = key channel i), so every state-dependent GEMM has
+// M = d_v = 128.  q, k, v, alpha arrive by TMA; every other operand is built
+// on chip in 128-byte swizzled shared-memory tiles.  Per chunk:
 //   1. TMA raw tiles -> block totals, Gamma_C, M, Kbar, row operands
 //   2. A, P  (one GEMM on the fast path, three on the anchored path)
 //   3. T = (I + A)^{-1}: 16x16 diagonal blocks, then two recursive-doubling merges
@@ -47,7 +47,15 @@
 //   6. tcgen05: U^T -= S^T W^T;  O^T = S^T Q^T
 //   7. tcgen05: O^T += U^T P^T;  S^T += U^T Kbar;  o -> HBM
 // The next chunk's TMA loads start as soon as step 2 has consumed the raw tiles.
+//
+// Split form: steps 1-4 do not depend on the state, so a persistent kernel
+// (the same code, SPLIT = true) runs them for every (chunk, head) on all SMs
+// and stores each chunk's operand tiles to a workspace slot; a chain kernel
+// per (sequence, head) then runs steps 5-7 from those slots.  Same arithmetic
+// in the same order: the two forms give identical bits.
 #include <cuda.h>
+#include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -99,7 +107,70 @@ struct ChunkParams {
     CUtensorMap tq, tk, ta;  // [B*T][H][128] bf16, box {128, 1, 64}, no swizzle
     CUtensorMap tv;          // same tensor shape, box {64, 1, 64}, 128-byte swizzle
     FwdArgs a;
+    uint8_t *ws;             // split path: chunk operand slots
+    int nslots;              // slots per head
+    uint32_t epoch;          // split path: tag of this call's slots
 };
+
+// ---- split path: per-chunk operand slots in global memory -------------------
+// Chunk c of sequence n (first global row R_n) has slot s = n + floor(R_n / C) + c:
+// unique, increasing within a sequence, and below N + ceil(rows / C).
+// A slot (one per head) holds byte images of the shared-memory operand tiles,
+// laid out so the chain kernel loads one contiguous block:
+constexpr uint32_t SL_QA = 0;         // [W'; Q'] 128-row K-major tile (32 KiB)
+constexpr uint32_t SL_KB = 32768;     // Kbar (16 KiB)
+constexpr uint32_t SL_PBF = 49152;    // P bf16 (8 KiB)
+constexpr uint32_t SL_TBF = 57344;    // T Diag(w) bf16 (8 KiB)
+constexpr uint32_t SL_META = 65536;   // Gamma_C fp32 [128], status word, epoch tag
+constexpr uint32_t SL_META_BYTES = 528;
+constexpr uint32_t SL_OPS = 66560;    // bytes the chain kernel loads for every variant
+constexpr uint32_t SL_M = 66560;      // GDN-2: M = w (.) v, 128B-swizzled [token][channel] (16 KiB)
+constexpr uint32_t SLOT_BYTES = 82944;
+constexpr int META_FAST = 1;          // status word bits
+constexpr int META_OK = 2;
+
+__device__ __forceinline__ int seq_row0(const FwdArgs &a, int n) { return a.cu_seqlens ? a.cu_seqlens[n] : n * a.T; }
+__device__ __forceinline__ int seq_len(const FwdArgs &a, int n)
+{
+    return a.cu_seqlens ? a.cu_seqlens[n + 1] - a.cu_seqlens[n] : a.T;
+}
+__device__ __forceinline__ int slot_base(const FwdArgs &a, int n) { return n + seq_row0(a, n) / C; }
+
+// One chunk of work for the preparation role.
+struct Item {
+    int n, h, c, row0, len;   // sequence, head, chunk, first global row of the sequence, its length
+    int slot;
+    bool valid;
+};
+// Split path: work index w = slot * H + h -> chunk, or invalid when the slot is empty.
+__device__ __forceinline__ Item decode_item(const FwdArgs &a, int N, int w)
+{
+    Item it;
+    it.h = w % a.H;
+    it.slot = w / a.H;
+    int lo = 0, hi = N - 1;   // last sequence whose first slot is <= slot
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (slot_base(a, mid) <= it.slot) lo = mid;
+        else hi = mid - 1;
+    }
+    it.n = lo;
+    it.row0 = seq_row0(a, lo);
+    it.len = seq_len(a, lo);
+    it.c = it.slot - slot_base(a, lo);
+    it.valid = it.c >= 0 && it.c * C < it.len;
+    return it;
+}
+__device__ __forceinline__ Item next_split_item(const FwdArgs &a, int N, int nwork, int &w)
+{
+    for (; w < nwork; w += gridDim.x) {
+        const Item it = decode_item(a, N, w);
+        if (it.valid) return it;
+    }
+    Item none{};
+    none.valid = false;
+    return none;
+}
 
 // ---- small helpers --------------------------------------------------------
 // Elementwise work is done in "items" of 8 tokens x 4 channels (one 8-byte
@@ -299,7 +370,11 @@ __device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const floa
 constexpr int NCHAIN = 128, NPREP = 256;
 constexpr uint32_t BAR_PREP = 1, BAR_CHAIN = 2;
 
-__global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant__ ChunkParams P)
+// SPLIT = false: the fused kernel, one CTA per (sequence, head), both roles.
+// SPLIT = true: the preparation role alone (256 threads), persistent over all
+// chunks of all sequences and heads; each chunk's operands go to its slot.
+template <bool SPLIT>
+__global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __grid_constant__ ChunkParams P)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -308,10 +383,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;       // TMEM lane quarter of this warp
     const int H = a.H;
-    const int n = blockIdx.x / H, h = blockIdx.x % H;
-    int b, t0, len;
-    if (a.cu_seqlens) { b = 0; t0 = a.cu_seqlens[n]; len = a.cu_seqlens[n + 1] - t0; }
-    else { b = n; t0 = 0; len = a.T; }
+    const int N = a.cu_seqlens ? a.num_seqs : a.B;
+    const int n = blockIdx.x / H, h = blockIdx.x % H;   // fused kernel: this CTA's sequence and head
+    const int len = SPLIT ? 0 : seq_len(a, n);
     const int nchunks = (len + C - 1) / C;
 
     float *s_g1 = reinterpret_cast<float *>(sm + M_G1);
@@ -345,7 +419,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
 
-    if (warp < 4) {
+    if (!SPLIT && warp < 4) {
         // =====================================================================
         // CHAIN group
         // =====================================================================
@@ -365,7 +439,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
         for (int ch = 0; ch < nchunks && ok; ++ch) {
             const uint32_t par = ch & 1;
             const int nvalid = min(C, len - ch * C);
-            const size_t rowbase = (size_t)b * a.T + t0 + ch * C;
+            const size_t rowbase = (size_t)seq_row0(a, n) + ch * C;
             if (!mbar_wait_cycles(bar_ready, par, WAIT_CYCLES)) ok = false;
             tc_fence_after();
             const bool fast = s_fast[par] != 0;
@@ -462,25 +536,28 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
         // =====================================================================
         // PREP group
         // =====================================================================
-        const int ptid = tid - NCHAIN, pw = warp - 4;
+        const int ptid = SPLIT ? tid : tid - NCHAIN, pw = SPLIT ? warp : warp - 4;
         const int phalf = pw >> 2;              // the two prep warps of a lane quarter split columns
         const int jrow = quarter * 32 + lane;   // TMEM lane of this thread
         const int tg = ptid >> 5, cq = ptid & 31;   // elementwise item: 8 tokens x 4 channels
         uint32_t ph_tma = 0, ph_v = 0, ph_pmma = 0;
 
         const CUtensorMap *map_q = &P.tq, *map_k = &P.tk, *map_v = &P.tv, *map_a = &P.ta;
-        auto issue_tma = [&](int chunk) {   // q, k, alpha of a chunk
-            const int g = b * a.T + t0 + chunk * C;
+        // M tile: the fused kernel has one; the split kernel (GDN-2) alternates two by item
+        // parity, since an item's M is still being stored while the next item's v arrives
+        auto mt_off = [&](uint32_t parity) -> uint32_t { return (SPLIT && parity) ? OFF_S0T : OFF_MT; };
+        auto issue_tma = [&](const Item &it) {   // q, k, alpha of a chunk
+            const int g = it.row0 + it.c * C;
             mbar_expect_tx(bar_tma, 3 * 16384);
-            tma_load_3d(sm + RAW_Q, map_q, bar_tma, 0, h, g);
-            tma_load_3d(sm + RAW_K, map_k, bar_tma, 0, h, g);
-            tma_load_3d(sm + RAW_A, map_a, bar_tma, 0, h, g);
+            tma_load_3d(sm + RAW_Q, map_q, bar_tma, 0, it.h, g);
+            tma_load_3d(sm + RAW_K, map_k, bar_tma, 0, it.h, g);
+            tma_load_3d(sm + RAW_A, map_a, bar_tma, 0, it.h, g);
         };
-        auto issue_tma_v = [&](int chunk) { // v, straight into its swizzled operand layout
-            const int g = b * a.T + t0 + chunk * C;
+        auto issue_tma_v = [&](const Item &it, uint32_t parity) { // v, straight into its swizzled operand layout
+            const int g = it.row0 + it.c * C;
             mbar_expect_tx(bar_v, 16384);
-            tma_load_3d(sm + OFF_MT, map_v, bar_v, 0, h, g);
-            tma_load_3d(sm + OFF_MT + 8192, map_v, bar_v, 64, h, g);
+            tma_load_3d(sm + mt_off(parity), map_v, bar_v, 0, it.h, g);
+            tma_load_3d(sm + mt_off(parity) + 8192, map_v, bar_v, 64, it.h, g);
         };
         auto wait_pmma = [&]() {
             if (!mbar_wait_cycles(bar_pmma, ph_pmma, WAIT_CYCLES)) ok = false;
@@ -493,9 +570,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             group_sync(BAR_PREP, NPREP);
         };
         // scalar gates of a chunk's row `ptid` as raw bf16 bits, fetched one chunk ahead
-        auto fetch_gates = [&](int chunk, uint32_t &ge, uint32_t &gw) {
-            const int r = ptid, nv = min(C, len - chunk * C);
-            const size_t tok = ((size_t)b * a.T + t0 + chunk * C + r) * H + h;
+        auto fetch_gates = [&](const Item &it, uint32_t &ge, uint32_t &gw) {
+            const int r = ptid, nv = min(C, it.len - it.c * C);
+            const size_t tok = ((size_t)it.row0 + it.c * C + r) * H + it.h;
             const bool v = r < nv;
             const unsigned short *g1u = reinterpret_cast<const unsigned short *>(g1p);
             const unsigned short *g2u = reinterpret_cast<const unsigned short *>(g2p);
@@ -506,28 +583,45 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             }
         };
 
-        if (nchunks > 0 && ptid == 0) {
-            issue_tma(0);
-            issue_tma_v(0);
+        // the chain of items this role prepares
+        const int nwork = SPLIT ? P.nslots * H : 0;
+        int wnext = blockIdx.x;
+        auto fused_item = [&](int c) {
+            Item it{n, h, c, 0, len, 0, c < nchunks};
+            it.row0 = seq_row0(a, n);
+            return it;
+        };
+        Item cur = SPLIT ? next_split_item(a, N, nwork, wnext) : fused_item(0);
+        const bool need_v = !SPLIT || gdn2;   // the split kernel leaves U' to the chain kernel
+        if (cur.valid && ptid == 0) {
+            issue_tma(cur);
+            if (need_v) issue_tma_v(cur, 0);
         }
         uint32_t gate_e = 0u, gate_w = 0u;
-        if (ptid < C && nchunks > 0) fetch_gates(0, gate_e, gate_w);
+        if (ptid < C && cur.valid) fetch_gates(cur, gate_e, gate_w);
 
-        for (int ch = 0; ch < nchunks && ok; ++ch) {
+        for (int ch = 0; cur.valid && ok; ++ch) {
             const uint32_t par = ch & 1, ppar = (ch - 1) & 1;
-            const int nvalid = min(C, len - ch * C);
-            const size_t rowbase = (size_t)b * a.T + t0 + ch * C;
+            if (SPLIT) wnext += gridDim.x;
+            const Item nxt = SPLIT ? next_split_item(a, N, nwork, wnext) : fused_item(ch + 1);
+            const int h = cur.h;
+            const int nvalid = min(C, cur.len - cur.c * C);
+            const size_t rowbase = (size_t)cur.row0 + cur.c * C;
             const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
+            const uint32_t OFF_MTC = mt_off(par);
+            float *gamc = SPLIT ? reinterpret_cast<float *>(sm + OFF_UT) : s_gamC + par * 128;
 
             if (ptid < C) {
                 s_g1[ptid] = __uint_as_float(gate_e << 16);
                 s_g2[ptid] = __uint_as_float(gate_w << 16);
-                if (ch + 1 < nchunks) fetch_gates(ch + 1, gate_e, gate_w);
+                if (nxt.valid) fetch_gates(nxt, gate_e, gate_w);
             }
             if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
             ph_tma ^= 1;
-            if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
-            ph_v ^= 1;
+            if (need_v) {
+                if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
+                ph_v ^= 1;
+            }
             group_sync(BAR_PREP, NPREP);
 
             // ===== 1a. block totals of alpha (and range check) | GDN-2: M = w (.) v
@@ -553,7 +647,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 #pragma unroll 2
                 for (int i = 0; i < 8; ++i) {
                     const int r = tg * 8 + i;
-                    uint2 *pv = reinterpret_cast<uint2 *>(sm + OFF_MT + sw_half(8192, r, cq));
+                    uint2 *pv = reinterpret_cast<uint2 *>(sm + OFF_MTC + sw_half(8192, r, cq));
                     float mv[4], vv[4], wv[4];
                     unpack4(*pv, vv);
                     if (r < nvalid) {
@@ -566,6 +660,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     }
                     *pv = pack4(mv);
                 }
+            }
+            if (SPLIT && ptid == 0) {
+                bulk_wait_read();   // the previous item's slot stores have read their tiles
+                if (gdn2 && nxt.valid) issue_tma_v(nxt, par ^ 1u);
             }
             in_range = group_sync_and(BAR_PREP, NPREP, in_range);
 
@@ -580,7 +678,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 #pragma unroll
                     for (int c = 0; c < 4; ++c) gc[c] *= t4[c];
                 }
-                *reinterpret_cast<float4 *>(s_gamC + par * 128 + ptid * 4) = make_float4(gc[0], gc[1], gc[2], gc[3]);
+                *reinterpret_cast<float4 *>(gamc + ptid * 4) = make_float4(gc[0], gc[1], gc[2], gc[3]);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) gam_ok = gam_ok && (fabsf(gc[c]) >= FAST_MIN_GAMMA);
             }
@@ -588,7 +686,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             if (ptid == 0) s_fast[par] = fast ? 1 : 0;
 
             // the previous chunk's chain must be done with QA (step 6) and with Kbar / P (step 7)
-            if (ch > 0) {
+            if (!SPLIT && ch > 0) {
                 if (!mbar_wait_cycles(bar_s6, ppar, WAIT_CYCLES)) ok = false;
                 if (!mbar_wait_cycles(bar_s7, ppar, WAIT_CYCLES)) ok = false;
             }
@@ -611,7 +709,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 #pragma unroll
                     for (int c = 0; c < 4; ++c) pre[c] *= t4[c];
                 }
-                const float4 gc4 = *reinterpret_cast<const float4 *>(s_gamC + par * 128 + cq * 4);
+                const float4 gc4 = *reinterpret_cast<const float4 *>(gamc + cq * 4);
                 float sc[4] = {pre[0] / gc4.x, pre[1] / gc4.y, pre[2] / gc4.z, pre[3] / gc4.w};
                 float kw[4][4];   // Kbar of rows r-4 .. r-1
                 {
@@ -702,7 +800,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     }
                     float sc[4];
                     if (fast) {
-                        const float4 gc4 = *reinterpret_cast<const float4 *>(s_gamC + par * 128 + cq * 4);
+                        const float4 gc4 = *reinterpret_cast<const float4 *>(gamc + cq * 4);
                         sc[0] = pre[0] / gc4.x; sc[1] = pre[1] / gc4.y; sc[2] = pre[2] / gc4.z; sc[3] = pre[3] / gc4.w;
                     } else {
 #pragma unroll
@@ -793,7 +891,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     mma_commit(bar_pmma);
                 }
                 wait_pmma();
-                if (ptid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
+                if (ptid == 0 && nxt.valid) issue_tma(nxt);   // raw tiles consumed
                 // rows 0-63: A (strictly lower, scaled by e_r), rows 64-127: P (band exact)
                 float v[32];
                 tmem_ld32(tbase + lane_base + TM_AP + phalf * 32, v);
@@ -847,7 +945,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     }
                     wait_pmma();
                 }
-                if (ptid == 0 && ch + 1 < nchunks) issue_tma(ch + 1);   // raw tiles consumed
+                if (ptid == 0 && nxt.valid) issue_tma(nxt);   // raw tiles consumed
                 for (int e = ptid; e < 64 * TP; e += NPREP) Af[e] = 0.f;
                 for (int e = ptid; e < 512; e += NPREP)
                     *reinterpret_cast<uint4 *>(sm + OFF_PBF + e * 16) = make_uint4(0, 0, 0, 0);
@@ -1006,7 +1104,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             write_t_copy(s_g1);
             publish();
             // U'^T overwrites TMEM U: the chain must have read the previous chunk's U out
-            if (ch > 0 && !mbar_wait_cycles(bar_ufree, ppar, WAIT_CYCLES)) ok = false;
+            // (the split kernel leaves U' to the chain kernel and stores T Diag(w) instead)
+            if (!SPLIT && ch > 0 && !mbar_wait_cycles(bar_ufree, ppar, WAIT_CYCLES)) ok = false;
             if (ptid == 0) {
                 tc_fence_after();
                 const uint32_t id_w = idesc_bf16(64, 128, false, true);
@@ -1014,7 +1113,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     mma_bf16(tbase + TM_W, dK(sb + OFF_TBF, 8192, kk), dMN(sb + OFF_QA, 16384, kk), id_w, kk > 0);
-                    if (same_gates)
+                    if (!SPLIT && same_gates)
                         mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_TBF, 8192, kk), id_u, kk > 0);
                 }
                 mma_commit(bar_pmma);
@@ -1023,7 +1122,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             if (!same_gates) {
                 write_t_copy(s_g2);
                 publish();
-                if (ptid == 0) {
+                if (!SPLIT && ptid == 0) {
                     tc_fence_after();
                     const uint32_t id_u = idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -1031,9 +1130,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                         mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_TBF, 8192, kk), id_u, kk > 0);
                     mma_commit(bar_pmma);
                 }
-                wait_pmma();
+                if (!SPLIT) wait_pmma();
             }
-            if (ptid == 0 && ch + 1 < nchunks) issue_tma_v(ch + 1);   // v consumed by U'^T = M^T T^T
+            if (!SPLIT && ptid == 0 && nxt.valid) issue_tma_v(nxt, 0);   // v consumed by U'^T = M^T T^T
             // W (M = 64 layout: rows 16q..16q+15 in lanes 0..15 of quarter q) -> rows 0-63 of QA
             {
                 const int r = quarter * 16 + (lane & 15);
@@ -1050,22 +1149,38 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     }
                 }
             }
+            if (SPLIT && ptid == 0) {   // status word and epoch tag of the slot
+                int *meta = reinterpret_cast<int *>(sm + OFF_UT);
+                meta[128] = META_OK | (fast ? META_FAST : 0);
+                meta[129] = (int)P.epoch;
+            }
             fence_async_smem();
             tc_fence_before();
             ok = group_sync_and(BAR_PREP, NPREP, ok);
-            if (ptid == 0) mbar_arrive(bar_ready);   // chunk ch's operands are ready for the chain
+            if (!SPLIT && ptid == 0) mbar_arrive(bar_ready);   // chunk ch's operands are ready for the chain
+            if (SPLIT && ptid == 0 && ok) {   // the slot: operand tiles, meta block, GDN-2 M
+                uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
+                bulk_store(slot + SL_QA, sm + OFF_QA, 49152);   // QA and Kbar are adjacent
+                bulk_store(slot + SL_PBF, sm + OFF_PBF, 8192);
+                bulk_store(slot + SL_TBF, sm + OFF_TBF, 8192);
+                bulk_store(slot + SL_META, sm + OFF_UT, SL_META_BYTES);
+                if (gdn2) bulk_store(slot + SL_M, sm + OFF_MTC, 16384);
+                bulk_commit();
+            }
+            cur = nxt;
         }
         if (!ok) {  // drain TMA still in flight (bounded)
             mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
-            mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
+            if (need_v) mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
         }
+        if (SPLIT && ptid == 0) bulk_wait_all();
     }
 
     // ---- final state (NaN if an internal wait timed out) ----------------------
     __syncthreads();
     tc_fence_after();
     ok = __syncthreads_and(ok) != 0;
-    if (warp < 4 && a.sf) {
+    if (!SPLIT && warp < 4 && a.sf) {
         const size_t soff = ((size_t)n * H + h) * D * D;
         const int jcol = tid;
 #pragma unroll 1
@@ -1082,6 +1197,217 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+// ---- chain kernel (split path) ----------------------------------------------
+// One CTA of 256 threads per (sequence, head) runs steps 5-7 over the chunks
+// whose operands the preparation kernel stored in their slots: two slot
+// buffers in shared memory, the next-but-one chunk loading while a chunk is
+// processed.  Warps w and w + 4 share TMEM lane quarter w (value columns
+// 32w .. 32w+31) and split the TMEM columns of every tile between them.
+constexpr int CK_NT = 256;
+constexpr uint32_t CK_BUF = SLOT_BYTES;        // a slot image; M (or v) at SL_M
+constexpr uint32_t CK_S0T = 2 * CK_BUF;         // state operand bf16 128 x 128, K-major
+constexpr uint32_t CK_UT = CK_S0T + 32768;      // U^T bf16 128 x 64, then o staging
+constexpr uint32_t CK_BAR = CK_UT + 16384;      // mbarriers: load[2], mma
+constexpr uint32_t CK_TMEM = CK_BAR + 32;
+constexpr uint32_t CK_ALLOC = CK_BAR + 64 + 1024;
+static_assert(CK_ALLOC <= 232448, "shared memory budget");
+static_assert((CK_BUF & 1023) == 0 && (CK_S0T & 1023) == 0 && (CK_UT & 1023) == 0, "swizzle atoms");
+
+__global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_constant__ ChunkParams P)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sb = smem_u32(sm);
+    const FwdArgs &a = P.a;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int half = warp >> 2;   // which half of a tile's TMEM columns this warp handles
+    const int H = a.H;
+    const int n = blockIdx.x / H, h = blockIdx.x % H;
+    const int row0 = seq_row0(a, n), len = seq_len(a, n), sbase = slot_base(a, n);
+    const int nchunks = (len + C - 1) / C;
+    const bool gdn2 = a.variant == GDN2;
+    uint64_t *bar_load = reinterpret_cast<uint64_t *>(sm + CK_BAR), *bar_mma = bar_load + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + CK_TMEM);
+    uint8_t *op = (uint8_t *)a.o;
+
+    if (warp == 0) tmem_alloc(s_tmem, 256);
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init(bar_load + i, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int jcol = (warp & 3) * 32 + lane;   // value column j = TMEM lane
+    bool ok = true;
+
+    // chunk c's slot (operands, meta, GDN-2 M) and, except for GDN-2, its v tile
+    auto issue_load = [&](int c, int buf) {
+        uint8_t *dst = sm + buf * CK_BUF;
+        const uint8_t *slot = P.ws + ((size_t)(sbase + c) * H + h) * SLOT_BYTES;
+        mbar_expect_tx(bar_load + buf, SL_OPS + 16384);
+        bulk_load(dst, slot, SL_OPS, bar_load + buf);
+        if (gdn2) {
+            bulk_load(dst + SL_M, slot + SL_M, 16384, bar_load + buf);
+        } else {
+            const int g = row0 + c * C;
+            tma_load_3d(dst + SL_M, &P.tv, bar_load + buf, 0, h, g);
+            tma_load_3d(dst + SL_M + 8192, &P.tv, bar_load + buf, 64, h, g);
+        }
+    };
+    if (tid == 0) {
+        if (nchunks > 0) issue_load(0, 0);
+        if (nchunks > 1) issue_load(1, 1);
+    }
+    {   // initial state -> TMEM (fp32), key channels 64 half .. 64 half + 63
+        const size_t soff = ((size_t)n * H + h) * D * D;
+#pragma unroll 1
+        for (int c16 = 0; c16 < 4; ++c16) {
+            float v[16];
+            const int i0 = half * 64 + c16 * 16;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = a.s0 ? a.s0[soff + (size_t)(i0 + e) * D + jcol] : 0.f;
+            tmem_st16(tbase + lane_base + TM_S + i0, v);
+        }
+        tmem_wait_st();
+    }
+    uint32_t ph_mma = 0;
+    int ch = 0;
+    for (; ch < nchunks && ok; ++ch) {
+        const int buf = ch & 1;
+        const uint32_t bufa = sb + buf * CK_BUF;
+        const int nvalid = min(C, len - ch * C);
+        const size_t rowbase = (size_t)row0 + ch * C;
+        if (!mbar_wait_cycles(bar_load + buf, (ch >> 1) & 1, WAIT_CYCLES)) ok = false;
+        tc_fence_after();
+        const int *meta = reinterpret_cast<const int *>(sm + buf * CK_BUF + SL_META);
+        const float *gamC = reinterpret_cast<const float *>(meta);
+        // a slot this call's preparation kernel did not complete reads as a failure
+        ok = __syncthreads_and(ok && (meta[128] & META_OK) && meta[129] == (int)P.epoch) != 0;
+        if (!ok) break;
+        const bool fast = (meta[128] & META_FAST) != 0;
+        if (tid == 0) {   // U'^T = M^T (T Diag(w))^T: independent of the state, issued first
+            tc_fence_after();
+            const uint32_t id_u = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tbase + TM_U, dMN(bufa + SL_M, 8192, kk), dK(bufa + SL_TBF, 8192, kk), id_u, kk > 0);
+        }
+        // ---- state pass: S^T *= Gamma_C in TMEM; bf16 operand copy (scaled on the fast path)
+#pragma unroll 1
+        for (int c32 = 0; c32 < 2; ++c32) {
+            const int i0 = half * 64 + c32 * 32;
+            float s[32], t[32];
+            tmem_ld32(tbase + lane_base + TM_S + i0, s);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                t[e] = s[e] * gamC[i0 + e];
+                if (fast) s[e] = t[e];
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4 *>(sm + CK_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
+            tmem_st16(tbase + lane_base + TM_S + i0, t);
+            tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
+        }
+        tmem_wait_st();
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- step 6: U^T -= S^T W^T ; O^T = S^T Q^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_neg = idesc_bf16(128, 64, false, false, true);
+            const uint32_t id_pos = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                mma_bf16(tbase + TM_U, dK(sb + CK_S0T, 16384, kk), dK(bufa + SL_QA, 16384, kk), id_neg, 1);
+                mma_bf16(tbase + TM_O, dK(sb + CK_S0T, 16384, kk), dK(bufa + SL_QA + 8192, 16384, kk), id_pos,
+                         kk > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
+        ph_mma ^= 1;
+        tc_fence_after();
+        // ---- U^T row j -> bf16 K-major tile (rows j, K = token); tokens 32 half .. 32 half + 31
+        {
+            float v[32];
+            tmem_ld32(tbase + lane_base + TM_U + half * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                *reinterpret_cast<uint4 *>(sm + CK_UT + sw_chunk(16384, jcol, half * 4 + q4)) = pack8(v + q4 * 8);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        // ---- step 7: O^T += U^T P^T ; S^T += U^T Kbar
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id_o = idesc_bf16(128, 64, false, false);
+            const uint32_t id_s = idesc_bf16(128, 128, false, true);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                mma_bf16(tbase + TM_O, dK(sb + CK_UT, 16384, kk), dK(bufa + SL_PBF, 8192, kk), id_o, 1);
+                mma_bf16(tbase + TM_S, dK(sb + CK_UT, 16384, kk), dMN(bufa + SL_KB, 8192, kk), id_s, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
+        ph_mma ^= 1;
+        tc_fence_after();
+        // every read of this buffer is done: load chunk ch + 2 into it
+        if (tid == 0 && ok && ch + 2 < nchunks) issue_load(ch + 2, buf);
+        // ---- o: TMEM (lane j, column r) -> bf16 staging [r][j] in the U^T slot -> HBM
+        unsigned short *ost = reinterpret_cast<unsigned short *>(sm + CK_UT);
+        {
+            float v[32];
+            tmem_ld32(tbase + lane_base + TM_O + half * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+                const uint32_t pk = pack_bf16(v[e], v[e + 1]);
+                ost[(half * 32 + e) * 128 + jcol] = (unsigned short)(pk & 0xFFFFu);
+                ost[(half * 32 + e + 1) * 128 + jcol] = (unsigned short)(pk >> 16);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        for (int e = tid; e < nvalid * 16; e += CK_NT) {
+            const int r = e >> 4, cgo = e & 15;
+            *reinterpret_cast<uint4 *>(op + (((rowbase + r) * H + h) * D + cgo * 8) * 2) =
+                *reinterpret_cast<const uint4 *>(sm + CK_UT + r * 256 + cgo * 16);
+        }
+        ok = __syncthreads_and(ok) != 0;   // staging read before the next U^T write
+    }
+    if (!ok && tid == 0) {   // drain loads still in flight (bounded)
+        for (int c = ch; c < nchunks && c < ch + 2; ++c) mbar_wait_cycles(bar_load + (c & 1), (c >> 1) & 1, WAIT_CYCLES);
+    }
+    // ---- final state (NaN if a wait timed out or a slot was missing)
+    __syncthreads();
+    tc_fence_after();
+    if (a.sf) {
+        const size_t soff = ((size_t)n * H + h) * D * D;
+#pragma unroll 1
+        for (int c32 = 0; c32 < 2; ++c32) {
+            const int i0 = half * 64 + c32 * 32;
+            float s[32];
+            tmem_ld32(tbase + lane_base + TM_S + i0, s);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                a.sf[soff + (size_t)(i0 + e) * D + jcol] = ok ? s[e] : __int_as_float(0x7fc00000);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 256);
 }
 
 // ---- host side --------------------------------------------------------------
@@ -1119,24 +1445,33 @@ bool make_map(CUtensorMap *m, const void *base, long long rows, int H, bool swiz
 
 }  // namespace
 
-cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
+namespace {
+// Per-device one-time set-up: dynamic shared-memory opt-ins and the SM count.
+cudaError_t device_setup(int &num_sms)
 {
-    // the dynamic shared-memory opt-in is per device; set it once per device
     static std::mutex mu;
-    static bool attr_done[64] = {};
+    static int sms[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-        if (!attr_done[dev]) {
-            e = cudaFuncSetAttribute(chunk_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_ALLOC);
-            if (e != cudaSuccess) return e;
-            attr_done[dev] = true;
-        }
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!sms[dev]) {
+        if ((e = cudaFuncSetAttribute(chunk_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      SMEM_ALLOC)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      SMEM_ALLOC)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CK_ALLOC)) !=
+                cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
     }
-    ChunkParams p;
+    num_sms = sms[dev];
+    return cudaSuccess;
+}
+
+cudaError_t make_params(ChunkParams &p, const FwdArgs &a)
+{
     memset(&p, 0, sizeof(p));
     p.a = a;
     const long long rows = (long long)a.B * a.T;
@@ -1145,8 +1480,63 @@ cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
             !make_map(&p.tv, a.v, rows, a.H, true) || !make_map(&p.ta, a.alpha, rows, a.H, false))
             return cudaErrorInvalidValue;
     }
+    return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
+{
+    int num_sms = 0;
+    cudaError_t e = device_setup(num_sms);
+    if (e != cudaSuccess) return e;
+    ChunkParams p;
+    if ((e = make_params(p, a)) != cudaSuccess) return e;
     const int N = a.cu_seqlens ? a.num_seqs : a.B;
-    chunk_fwd_kernel<<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
+    chunk_fwd_kernel<false><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
+    return cudaGetLastError();
+}
+
+bool chunk_prefer_split(const FwdArgs &a)
+{
+    // The fused kernel runs one CTA per (sequence, head) for the whole sequence.
+    // When those CTAs would leave at least half of the SMs idle, spreading the
+    // operand preparation over every SM outweighs the workspace round trip.
+    int num_sms = 0;
+    if (device_setup(num_sms) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    const long long N = a.cu_seqlens ? a.num_seqs : a.B;
+    return N * a.H * 2 <= num_sms;
+}
+
+size_t chunk_split_workspace_bytes(const FwdArgs &a)
+{
+    const long long N = a.cu_seqlens ? a.num_seqs : a.B;
+    const long long rows = (long long)a.B * a.T;
+    return (size_t)(N + (rows + C - 1) / C) * a.H * SLOT_BYTES;
+}
+
+cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st)
+{
+    int num_sms = 0;
+    cudaError_t e = device_setup(num_sms);
+    if (e != cudaSuccess) return e;
+    ChunkParams p;
+    if ((e = make_params(p, a)) != cudaSuccess) return e;
+    static std::atomic<uint32_t> epoch{0};
+    const int N = a.cu_seqlens ? a.num_seqs : a.B;
+    const long long rows = (long long)a.B * a.T;
+    p.ws = static_cast<uint8_t *>(ws);
+    p.nslots = (int)(N + (rows + C - 1) / C);
+    p.epoch = epoch.fetch_add(1) + 1;
+    const long long nwork = (long long)p.nslots * a.H;
+    if (rows > 0 && nwork > 0) {
+        const unsigned grid = (unsigned)std::min<long long>(nwork, num_sms);
+        chunk_fwd_kernel<true><<<grid, NPREP, SMEM_ALLOC, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    chunk_chain_kernel<<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);
     return cudaGetLastError();
 }
 

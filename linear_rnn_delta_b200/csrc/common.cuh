@@ -31,6 +31,10 @@ struct FwdArgs {
 cudaError_t launch_scan_fwd(const FwdArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_decode_step(const FwdArgs &a, bool bf16, cudaStream_t st);
 cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st);
+// Two-kernel chunked path: `ws` holds chunk_split_workspace_bytes(a) bytes.
+bool chunk_prefer_split(const FwdArgs &a);   // the shape-based default choice of form
+size_t chunk_split_workspace_bytes(const FwdArgs &a);
+cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st);
 cudaError_t launch_check_gates(int variant, int gate_range, bool bf16, long long n_tok, int dk,
                                const void *alpha, const void *g1, int *d_count, cudaStream_t st);
 

@@ -57,15 +57,25 @@ int check_common(int variant, int gate_range, int dtype, int d_k, int d_v,
     return KDA_OK;
 }
 
-}  // namespace
+// Form of the tensor-core path: the fused kernel (no workspace) or the split
+// preparation + chain kernels; by shape unless a flag forces one.
+bool use_split(const kda::FwdArgs &a, unsigned flags)
+{
+    if (flags & KDA_FLAG_FORCE_FUSED) return false;
+    if (flags & KDA_FLAG_FORCE_SPLIT) return true;
+#ifdef KDA_WITH_SM100_CHUNK
+    return kda::chunk_prefer_split(a);
+#else
+    (void)a;
+    return false;
+#endif
+}
 
-extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
-                             int B, int T, int H, int d_k, int d_v,
-                             const void *q, const void *k, const void *v, const void *alpha,
-                             const void *g1, const void *g2,
-                             const int32_t *cu_seqlens, int num_seqs,
-                             const float *initial_state, float *final_state,
-                             void *o, int chunk_size, unsigned flags, void *stream)
+// Validated forward arguments; returns KDA_OK or the error code (detail set).
+int chunk_args(kda::FwdArgs &a, int variant, int gate_range, int dtype, int B, int T, int H, int d_k, int d_v,
+               const void *q, const void *k, const void *v, const void *alpha, const void *g1, const void *g2,
+               const int32_t *cu_seqlens, int num_seqs, const float *initial_state, float *final_state, void *o,
+               int chunk_size, unsigned flags)
 {
     if (B < 1 || T < 0 || H < 1)
         return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d (need B>=1, T>=0, H>=1)", B, T, H);
@@ -75,7 +85,10 @@ extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
     if (rc != KDA_OK) return rc;
     if (!chunk_ok(chunk_size))
         return fail(KDA_ERR_UNSUPPORTED, "chunk_size %d: supported are 16, 32, 64, 128", chunk_size);
-    if (flags & ~KDA_FLAG_FORCE_SCAN) return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if (flags & ~(KDA_FLAG_FORCE_SCAN | KDA_FLAG_FORCE_FUSED | KDA_FLAG_FORCE_SPLIT))
+        return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if ((flags & KDA_FLAG_FORCE_FUSED) && (flags & KDA_FLAG_FORCE_SPLIT))
+        return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_FORCE_FUSED and KDA_FLAG_FORCE_SPLIT exclude each other");
     int N = B;
     if (cu_seqlens) {
         if (B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (got B=%d)", B);
@@ -88,20 +101,119 @@ extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
         return fail(KDA_ERR_INVALID_ARG, "initial_state is not 16-byte aligned");
     if (final_state && !aligned16(final_state))
         return fail(KDA_ERR_INVALID_ARG, "final_state is not 16-byte aligned");
+    a = kda::FwdArgs{variant, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens, N,
+                     initial_state, final_state, o};
+    return KDA_OK;
+}
 
-    kda::FwdArgs a{variant, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens, N,
-                   initial_state, final_state, o};
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool bf16 = dtype == KDA_DTYPE_BF16;
-    cudaError_t e;
+bool tensor_core_path(const kda::FwdArgs &a, int dtype, int chunk_size, unsigned flags)
+{
 #ifdef KDA_WITH_SM100_CHUNK
-    if (bf16 && d_k == 128 && d_v == 128 && chunk_size == 64 && !(flags & KDA_FLAG_FORCE_SCAN))
-        e = kda::launch_chunk_fwd_sm100(a, st);
-    else
+    return dtype == KDA_DTYPE_BF16 && a.dk == 128 && a.dv == 128 && chunk_size == 64 &&
+           !(flags & KDA_FLAG_FORCE_SCAN);
+#else
+    (void)a; (void)dtype; (void)chunk_size; (void)flags;
+    return false;
 #endif
-        e = kda::launch_scan_fwd(a, bf16, st);
+}
+
+// Launches the chosen path; `ws` (may be NULL) holds `ws_bytes` bytes.
+int chunk_launch(const kda::FwdArgs &a, int dtype, int chunk_size, unsigned flags, void *ws, size_t ws_bytes,
+                 cudaStream_t st)
+{
+    cudaError_t e = cudaSuccess;
+    if (tensor_core_path(a, dtype, chunk_size, flags)) {
+#ifdef KDA_WITH_SM100_CHUNK
+        if (use_split(a, flags) && ws && ws_bytes >= kda::chunk_split_workspace_bytes(a))
+            e = kda::launch_chunk_split_sm100(a, ws, st);
+        else
+            e = kda::launch_chunk_fwd_sm100(a, st);
+#endif
+    } else {
+        e = kda::launch_scan_fwd(a, dtype == KDA_DTYPE_BF16, st);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd launch");
     return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" size_t kda_chunk_fwd_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
+                                               int has_cu_seqlens, int num_seqs, int chunk_size, unsigned flags)
+{
+    if (B < 1 || T < 0 || H < 1 || (has_cu_seqlens && (B != 1 || num_seqs < 1))) return 0;
+    if ((unsigned long long)B * (unsigned long long)T * H * 128ull > (1ull << 46)) return 0;
+    if ((flags & KDA_FLAG_FORCE_FUSED) && (flags & KDA_FLAG_FORCE_SPLIT)) return 0;
+    kda::FwdArgs a{};
+    a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v;
+    a.num_seqs = has_cu_seqlens ? num_seqs : B;
+    a.cu_seqlens = has_cu_seqlens ? reinterpret_cast<const int32_t *>(16) : nullptr;  // presence only
+    if (!tensor_core_path(a, dtype, chunk_size, flags) || !use_split(a, flags)) return 0;
+#ifdef KDA_WITH_SM100_CHUNK
+    return kda::chunk_split_workspace_bytes(a);
+#else
+    return 0;
+#endif
+}
+
+extern "C" int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
+                                int B, int T, int H, int d_k, int d_v,
+                                const void *q, const void *k, const void *v, const void *alpha,
+                                const void *g1, const void *g2,
+                                const int32_t *cu_seqlens, int num_seqs,
+                                const float *initial_state, float *final_state,
+                                void *o, int chunk_size, void *workspace, size_t workspace_bytes,
+                                unsigned flags, void *stream)
+{
+    kda::FwdArgs a;
+    int rc = chunk_args(a, variant, gate_range, dtype, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens,
+                        num_seqs, initial_state, final_state, o, chunk_size, flags);
+    if (rc != KDA_OK) return rc;
+    if (workspace && !aligned16(workspace)) return fail(KDA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    if ((flags & KDA_FLAG_FORCE_SPLIT) && tensor_core_path(a, dtype, chunk_size, flags)) {
+        size_t need = 0;
+#ifdef KDA_WITH_SM100_CHUNK
+        need = kda::chunk_split_workspace_bytes(a);
+#endif
+        if (!workspace || workspace_bytes < need)
+            return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_FORCE_SPLIT needs a workspace of %zu bytes (got %zu)", need,
+                        workspace ? workspace_bytes : (size_t)0);
+    }
+    return chunk_launch(a, dtype, chunk_size, flags, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
+                             int B, int T, int H, int d_k, int d_v,
+                             const void *q, const void *k, const void *v, const void *alpha,
+                             const void *g1, const void *g2,
+                             const int32_t *cu_seqlens, int num_seqs,
+                             const float *initial_state, float *final_state,
+                             void *o, int chunk_size, unsigned flags, void *stream)
+{
+    kda::FwdArgs a;
+    int rc = chunk_args(a, variant, gate_range, dtype, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens,
+                        num_seqs, initial_state, final_state, o, chunk_size, flags);
+    if (rc != KDA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+#ifdef KDA_WITH_SM100_CHUNK
+    if (tensor_core_path(a, dtype, chunk_size, flags) && use_split(a, flags)) {
+        // stream-ordered workspace; without it the fused kernel runs
+        ws_bytes = kda::chunk_split_workspace_bytes(a);
+        if (cudaMallocAsync(&ws, ws_bytes, st) != cudaSuccess) {
+            (void)cudaGetLastError();
+            ws = nullptr;
+            ws_bytes = 0;
+        }
+    }
+#endif
+    rc = chunk_launch(a, dtype, chunk_size, flags, ws, ws_bytes, st);
+    if (ws) {
+        const cudaError_t ef = cudaFreeAsync(ws, st);
+        if (rc == KDA_OK && ef != cudaSuccess) rc = cuda_fail(ef, "kda_chunk_fwd workspace release");
+    }
+    return rc;
 }
 
 extern "C" int kda_decode_step(int variant, int gate_range, int dtype,

@@ -200,6 +200,27 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, ui
         :: "r"(smem_u32(smem_dst)), "l"(tmap), "r"(smem_u32(mbar)), "r"(c0), "r"(c1), "r"(c2) : "memory");
 }
 
+// ---- untiled bulk copies (no multicast) ------------------------------------
+// Both addresses 16-byte aligned, `bytes` a multiple of 16.
+// global -> shared, completion counted in bytes on `mbar`
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *mbar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(smem_dst)), "l"(gsrc), "r"(bytes), "r"(smem_u32(mbar)) : "memory");
+}
+// shared -> global in the issuing thread's bulk async-group
+__device__ __forceinline__ void bulk_store(void *gdst, const void *smem_src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(gdst), "r"(smem_u32(smem_src)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the issuing thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // fp32 -> bf16 round-to-nearest-even: two values per instruction (lo in the
 // low half).
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)

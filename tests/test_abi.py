@@ -17,7 +17,11 @@ HEADER = os.path.join(ROOT, "include", "kda.h")
 
 @pytest.fixture(scope="module")
 def lib():
-    from linear_rnn_delta_b200 import build
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("linear_rnn_delta_b200_build",
+                                                  os.path.join(ROOT, "linear_rnn_delta_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)   # by path: importing the package loads the library being built
     build.build()
     import linear_rnn_delta_b200 as k
     return k.lib
@@ -62,6 +66,49 @@ def fwd(lib, **kw):
                              a["sf"], a["o"], a["chunk"], a["flags"], a["stream"])
 
 
+def fwd_ws(lib, ws=None, ws_bytes=0, **kw):
+    a = dict(variant=0, gate_range=0, dtype=0, B=1, T=8, H=1, dk=128, dv=128, q=P, k=P, v=P, alpha=P, g1=P,
+             g2=None, cu=None, nseq=0, s0=None, sf=None, o=P, chunk=64, flags=0, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_fwd_ws(a["variant"], a["gate_range"], a["dtype"], a["B"], a["T"], a["H"], a["dk"],
+                                a["dv"], a["q"], a["k"], a["v"], a["alpha"], a["g1"], a["g2"], a["cu"], a["nseq"],
+                                a["s0"], a["sf"], a["o"], a["chunk"], ws, ws_bytes, a["flags"], a["stream"])
+
+
+SLOT_BYTES = 82944
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((0, 4, 4096, 16, 128, 128, 0, 0, 64), (4 + 4 * 4096 // 64) * 16 * SLOT_BYTES),   # fixed length: N = B
+    ((0, 1, 1000, 32, 128, 128, 1, 16, 64), (16 + 16) * 32 * SLOT_BYTES),           # varlen: N = num_seqs
+    ((0, 2, 65, 3, 128, 128, 0, 0, 64), (2 + 3) * 3 * SLOT_BYTES),                    # ragged: ceil(130 / 64)
+    ((0, 2, 0, 3, 128, 128, 0, 0, 64), 2 * 3 * SLOT_BYTES),                           # T = 0
+    ((1, 4, 4096, 16, 128, 128, 0, 0, 64), 0),      # fp32: token scan, no workspace
+    ((0, 4, 4096, 16, 64, 128, 0, 0, 64), 0),       # d_k = 64: token scan
+    ((0, 4, 4096, 16, 128, 128, 0, 0, 32), 0),      # chunk 32: token scan
+    ((0, 2, 64, 2, 128, 128, 1, 3, 64), 0),         # cu_seqlens with B != 1
+    ((0, 0, 64, 2, 128, 128, 0, 0, 64), 0),         # B = 0
+])
+def test_workspace_size_of_the_split_form(lib, args, expect):
+    assert lib.kda_chunk_fwd_workspace_size(*args, 8) == expect
+
+
+def test_workspace_size_other_forms(lib):
+    args = (0, 4, 4096, 16, 128, 128, 0, 0, 64)
+    assert lib.kda_chunk_fwd_workspace_size(*args, 4) == 0       # fused forced
+    assert lib.kda_chunk_fwd_workspace_size(*args, 2) == 0       # scan forced
+    assert lib.kda_chunk_fwd_workspace_size(*args, 4 | 8) == 0   # contradictory flags
+
+
+def test_forced_split_needs_a_workspace(lib):
+    need = lib.kda_chunk_fwd_workspace_size(0, 1, 8, 1, 128, 128, 0, 0, 64, 8)
+    assert fwd_ws(lib, flags=8) == INVALID                          # none
+    assert fwd_ws(lib, ws=P, ws_bytes=need - 16, flags=8) == INVALID  # too small
+    assert fwd_ws(lib, ws=BAD, ws_bytes=need, flags=8) == INVALID     # misaligned
+    assert fwd_ws(lib, ws=P, ws_bytes=need, flags=4 | 8) == INVALID   # both forms forced
+    assert fwd_ws(lib, flags=1 << 9) == INVALID
+
+
 def dec(lib, **kw):
     a = dict(variant=0, gate_range=1, dtype=0, N=4, H=2, dk=128, dv=128, q=P, k=P, v=P, alpha=P, g1=P, g2=None,
              state=P, o=P, flags=0, stream=None)
@@ -84,6 +131,7 @@ INVALID, UNSUPPORTED = 1, 2
     (dict(variant=2, g2=BAD), INVALID),     # GDN-2 with misaligned g2
     (dict(chunk=48), UNSUPPORTED), (dict(chunk=256), UNSUPPORTED),
     (dict(flags=1 << 7), INVALID),
+    (dict(flags=4 | 8), INVALID),           # fused and split forms both forced
     (dict(cu=P, nseq=2, B=2), INVALID),     # cu_seqlens needs B == 1
     (dict(cu=P, nseq=0), INVALID),
     (dict(cu=ctypes.c_void_p(0x10002), nseq=1), INVALID),
