@@ -147,6 +147,35 @@ int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
                      unsigned flags, void *stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- the split form of the tensor-core chunked forward
+ * for callers that cannot allocate device memory at call time: an engine
+ * whose allocator already owns all of HBM, a runtime with a fixed device
+ * memory budget, or a latency-critical loop that cannot take cudaMalloc's
+ * cost and the device synchronisation it may cause.  The pages have no
+ * counterpart; this is a deployment entry point, not part of the method.
+ *
+ * Arguments and results are those of kda_chunk_fwd with chunk_size 64 and
+ * no flags (flags must be 0).  It serves bf16 with d_k = d_v = 128 only
+ * (else KDA_ERR_UNSUPPORTED) and allocates nothing: its workspace is a fixed
+ * 64 MiB device array inside the library, held by every GPU that loads the
+ * library until the process exits.  Problems needing more,
+ * (N + ceil(B*T/64)) * H > 809, are rejected with KDA_ERR_UNSUPPORTED.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the array: calls that overlap on the GPU (other
+ * streams, other host threads) race and give wrong results; calls in order
+ * on one stream are safe.  The array's earlier contents never leak into a
+ * result (each call tags its slots).
+ */
+int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
+                          int B, int T, int H, int d_k, int d_v,
+                          const void *q, const void *k, const void *v, const void *alpha,
+                          const void *g1, const void *g2,
+                          const int32_t *cu_seqlens, int num_seqs,
+                          const float *initial_state, float *final_state,
+                          void *o, unsigned flags, void *stream);
+
+/*
  * kda_decode_step -- one recurrent step for N sequences (single-token decode;
  * the fixed-size state of the openarchlab page, sec. 1 and 3).
  *

@@ -35,6 +35,9 @@ cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st);
 bool chunk_prefer_split(const FwdArgs &a);   // the shape-based default choice of form
 size_t chunk_split_workspace_bytes(const FwdArgs &a);
 cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st);
+// Split form with the fixed device scratch array as its workspace (no allocation).
+size_t chunk_noalloc_capacity();
+cudaError_t launch_chunk_split_noalloc(const FwdArgs &a, cudaStream_t st);
 cudaError_t launch_check_gates(int variant, int gate_range, bool bf16, long long n_tok, int dk,
                                const void *alpha, const void *g1, int *d_count, cudaStream_t st);
 

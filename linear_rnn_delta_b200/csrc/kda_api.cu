@@ -216,6 +216,36 @@ extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
     return rc;
 }
 
+extern "C" int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
+                                     int B, int T, int H, int d_k, int d_v,
+                                     const void *q, const void *k, const void *v, const void *alpha,
+                                     const void *g1, const void *g2,
+                                     const int32_t *cu_seqlens, int num_seqs,
+                                     const float *initial_state, float *final_state,
+                                     void *o, unsigned flags, void *stream)
+{
+    kda::FwdArgs a;
+    int rc = chunk_args(a, variant, gate_range, dtype, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens,
+                        num_seqs, initial_state, final_state, o, 64, 0u);
+    if (rc != KDA_OK) return rc;
+    if (flags != 0) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_noalloc takes no flags (got 0x%x)", flags);
+#ifdef KDA_WITH_SM100_CHUNK
+    if (!tensor_core_path(a, dtype, 64, 0u))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_noalloc serves bf16 with d_k = d_v = 128 only "
+                                         "(got dtype %d, d_k %d, d_v %d)", dtype, d_k, d_v);
+    const size_t need = kda::chunk_split_workspace_bytes(a), cap = kda::chunk_noalloc_capacity();
+    if (need > cap)
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_noalloc: this problem needs %zu bytes of scratch, "
+                                         "the fixed array holds %zu ((N + ceil(B*T/64)) * H must be <= %zu)",
+                    need, cap, cap / 82944);
+    const cudaError_t e = kda::launch_chunk_split_noalloc(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_noalloc launch");
+    return KDA_OK;
+#else
+    return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_noalloc: built without the sm_100a chunked kernels");
+#endif
+}
+
 extern "C" int kda_decode_step(int variant, int gate_range, int dtype,
                                int N, int H, int d_k, int d_v,
                                const void *q, const void *k, const void *v, const void *alpha,
