@@ -195,6 +195,11 @@ __device__ __forceinline__ uint4 pack8(const float *f)
 {
     return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
 }
+__device__ __forceinline__ uint4 pack8_neg(const float *f)   // -f, exact
+{
+    return make_uint4(pack_bf16(-f[0], -f[1]), pack_bf16(-f[2], -f[3]), pack_bf16(-f[4], -f[5]),
+                      pack_bf16(-f[6], -f[7]));
+}
 // 16-byte chunk kc (8 consecutive K elements) of row `row` in a K-major
 // 128B-swizzled tile whose 64-element panels are `pstride` bytes apart.
 __device__ __forceinline__ uint32_t sw_chunk(uint32_t pstride, uint32_t row, uint32_t kc)
@@ -219,16 +224,19 @@ __device__ __forceinline__ uint2 raw_quad(const uint8_t *sm, uint32_t base, int 
 {
     return *reinterpret_cast<const uint2 *>(sm + base + r * 256 + cq * 8);
 }
-// K-major descriptor, K step kk (16 elements), panels `pstride` bytes apart
+// K-major descriptor, K step kk (16 elements), panels `pstride` bytes apart.
+// The step only moves the start address (bits 0-13, in 16-byte units; shared
+// addresses stay below 2^18 bytes, so the field cannot overflow): the base
+// descriptor is computed once and each step adds a constant.
 __device__ __forceinline__ uint64_t dK(uint32_t base, uint32_t pstride, int kk)
 {
-    return make_desc_sw128(base + (uint32_t)(kk >> 2) * pstride + (uint32_t)(kk & 3) * 32u, 16);
+    return make_desc_sw128(base, 16) + (uint64_t)(((uint32_t)(kk >> 2) * pstride + (uint32_t)(kk & 3) * 32u) >> 4);
 }
 // MN-major descriptor of a [token][channel] tile (channels in two 64-wide
 // panels `pstride` bytes apart, K = tokens), K step kk (16 tokens)
 __device__ __forceinline__ uint64_t dMN(uint32_t base, uint32_t pstride, int kk)
 {
-    return make_desc_sw128(base + (uint32_t)kk * 2048u, pstride);
+    return make_desc_sw128(base, pstride) + (uint64_t)((uint32_t)kk * (2048u >> 4));
 }
 __device__ __forceinline__ void load_tot4(const float *s_tot, int g, int cq, float *t4)
 {
@@ -254,6 +262,119 @@ __device__ __forceinline__ void erase_gate4(const ChunkCtx &x, int r, int cq, fl
     } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c) e[c] = 1.f;
+    }
+}
+
+// Step 6 of the chain: U^T += S^T (-W)^T and O^T = S^T Q^T.  The operand tile
+// qa holds [-W; Q'] as 128 K-major rows and U^T, O^T are adjacent in TMEM, so
+// after the first K step (U^T accumulates onto U'^T, O^T starts fresh) both
+// run as one N = 128 GEMM.
+__device__ __forceinline__ void step6_mmas(uint32_t tbase, uint32_t s0t, uint32_t qa)
+{
+    const uint32_t id64 = idesc_bf16(128, 64, false, false), id128 = idesc_bf16(128, 128, false, false);
+    mma_bf16(tbase + TM_U, dK(s0t, 16384, 0), dK(qa, 16384, 0), id64, 1);
+    mma_bf16(tbase + TM_O, dK(s0t, 16384, 0), dK(qa + 8192, 16384, 0), id64, 0);
+#pragma unroll
+    for (int kk = 1; kk < 8; ++kk) mma_bf16(tbase + TM_U, dK(s0t, 16384, kk), dK(qa, 16384, kk), id128, 1);
+}
+
+// Fast path, step 1b for the item (tg, cq): one forward sweep over the item's
+// 8 rows.  With sc = Gamma_r / Gamma_C (|sc| >= 1 since every |alpha| <= 1):
+//   row operands  Gamma a~ / Gamma_C = sc (.) a~,   Gamma q / Gamma_C = sc (.) q,
+//   Kbar_r = Lam_{C-1,r} (.) k_r = k_r / sc   (the divisor is bounded away from zero).
+// The band of P, P_{r,r-w} = sum_c (sc q)_{r,c} Kbar_{r-w,c} for w = 0..4, is
+// formed from these fp32 values: a window keeps Kbar of the four previous
+// rows, and each lane's 4-channel partial sums go to band_part[r][w][lane]
+// (summed over the 32 lanes = 128 channels by band_reduce).
+// FULL: all 64 rows valid (no masking).  EVEC: channel-wise erase vector
+// (GDN-2).  UNROLL: rows per unrolled step (register budget permitting).
+template <bool FULL, bool EVEC, int UNROLL>
+__device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot, const float *gamc,
+                                          float *band_part, int tg, int cq, int lane)
+{
+    uint8_t *sm = x.sm;
+    const int nvalid = x.nvalid;
+    float pre[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+        if (g >= tg) break;
+        float t4[4];
+        load_tot4(s_tot, g, cq, t4);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) pre[c] *= t4[c];
+    }
+    const float4 gc4 = *reinterpret_cast<const float4 *>(gamc + cq * 4);
+    float sc[4] = {pre[0] / gc4.x, pre[1] / gc4.y, pre[2] / gc4.z, pre[3] / gc4.w};
+    float kw[4][4];   // Kbar of rows r-4 .. r-1
+    {
+        float sb4[4] = {sc[0], sc[1], sc[2], sc[3]};   // Gamma_{8tg-1} / Gamma_C
+#pragma unroll
+        for (int j = 3; j >= 0; --j) {
+            const int rp = tg * 8 - 4 + j;
+            if (rp >= 0) {
+                float kv[4], av[4];
+                unpack4(raw_quad(sm, RAW_K, rp, cq), kv);
+                unpack4(raw_quad(sm, RAW_A, rp, cq), av);
+                const bool v = FULL || rp < nvalid;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    kw[j][c] = v ? __fdividef(kv[c], sb4[c]) : 0.f;
+                    sb4[c] = v ? __fdividef(sb4[c], av[c]) : sb4[c];
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) kw[j][c] = 0.f;
+            }
+        }
+    }
+#pragma unroll UNROLL
+    for (int i = 0; i < 8; ++i) {
+        const int r = tg * 8 + i;
+        const bool v = FULL || r < nvalid;
+        float al[4], kv[4], qv[4], oa[4], oq[4], kb[4];
+        unpack4(raw_quad(sm, RAW_A, r, cq), al);
+        unpack4(raw_quad(sm, RAW_K, r, cq), kv);
+        unpack4(raw_quad(sm, RAW_Q, r, cq), qv);
+        float e[4] = {1.f, 1.f, 1.f, 1.f};
+        if (EVEC) erase_gate4(x, r, cq, e);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            sc[c] *= v ? al[c] : 1.f;
+            const float ek = EVEC ? e[c] * kv[c] : kv[c];
+            oa[c] = v ? sc[c] * ek : 0.f;
+            oq[c] = v ? sc[c] * qv[c] : 0.f;
+            kb[c] = v ? __fdividef(kv[c], sc[c]) : 0.f;
+        }
+        *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, r, cq)) = pack4(oa);
+        *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, 64 + r, cq)) = pack4(oq);
+        *reinterpret_cast<uint2 *>(sm + OFF_KB + sw_half(8192, r, cq)) = pack4(kb);
+        float *bp = band_part + r * (PBAND * 32) + lane;
+        bp[0] = oq[0] * kb[0] + oq[1] * kb[1] + oq[2] * kb[2] + oq[3] * kb[3];
+#pragma unroll
+        for (int w = 1; w < PBAND; ++w)
+            bp[w * 32] = oq[0] * kw[4 - w][0] + oq[1] * kw[4 - w][1] + oq[2] * kw[4 - w][2] + oq[3] * kw[4 - w][3];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            kw[0][c] = kw[1][c]; kw[1][c] = kw[2][c]; kw[2][c] = kw[3][c]; kw[3][c] = kb[c];
+        }
+    }
+}
+
+// Fast path: P_{r,r-w} = sum over the 32 lanes of band_part[r][w][lane] for
+// the 64 x PBAND band entries (masked past the valid rows and above row 0).
+// Lanes start their eight 16-byte reads at rotated offsets: conflict-free.
+__device__ __forceinline__ void band_reduce(const float *band_part, float *s_pband, int nvalid, int ptid, int nthreads)
+{
+    for (int idx = ptid; idx < C * PBAND; idx += nthreads) {
+        const float4 *src = reinterpret_cast<const float4 *>(band_part + idx * 32);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 t = src[(j + idx) & 7];
+            acc[j & 3] += (t.x + t.y) + (t.z + t.w);
+        }
+        const int r = idx / PBAND, w = idx - r * PBAND;
+        s_pband[idx] = (r < nvalid && r - w >= 0) ? (acc[0] + acc[1]) + (acc[2] + acc[3]) : 0.f;
     }
 }
 
@@ -469,14 +590,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             // ---- step 6: U^T -= S^T W^T ; O^T = S^T Q^T
             if (tid == 0) {
                 tc_fence_after();
-                const uint32_t id_neg = idesc_bf16(128, 64, false, false, true);
-                const uint32_t id_pos = idesc_bf16(128, 64, false, false);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    mma_bf16(tbase + TM_U, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA, 16384, kk), id_neg, 1);
-                    mma_bf16(tbase + TM_O, dK(sb + OFF_S0T, 16384, kk), dK(sb + OFF_QA + 8192, 16384, kk), id_pos,
-                             kk > 0);
-                }
+                step6_mmas(tbase, sb + OFF_S0T, sb + OFF_QA);
                 mma_commit(bar_s6);
             }
             if (!mbar_wait_cycles(bar_s6, par, WAIT_CYCLES)) ok = false;
@@ -693,96 +807,13 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
 
             // ===== 1b. row operands, Kbar and the exact band of P ================
             if (fast) {
-                // Fast path, one forward sweep.  sc = Gamma_r / Gamma_C, |sc| >= 1 (all |alpha| <= 1), so
-                //   row operands  Gamma a~ / Gamma_C = sc (.) a~,  Gamma q / Gamma_C = sc (.) q,
-                //   Kbar_r = Lam_{C-1,r} (.) k_r = k_r / sc   (divisor bounded away from zero),
-                // and the band P_{r,r-w} = sum_c (sc q)_r (Kbar)_{r-w} comes exactly from these fp32
-                // values: a sliding window keeps Kbar of the four previous rows, and each row's five
-                // partial sums over this lane's 4 channels are reduce-scattered across the warp (the
-                // 32 lanes of a warp are the 32 channel quads of one 8-token block).
-                float pre[4] = {1.f, 1.f, 1.f, 1.f};
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    if (g >= tg) break;
-                    float t4[4];
-                    load_tot4(s_tot, g, cq, t4);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) pre[c] *= t4[c];
-                }
-                const float4 gc4 = *reinterpret_cast<const float4 *>(gamc + cq * 4);
-                float sc[4] = {pre[0] / gc4.x, pre[1] / gc4.y, pre[2] / gc4.z, pre[3] / gc4.w};
-                float kw[4][4];   // Kbar of rows r-4 .. r-1
-                {
-                    float sb4[4] = {sc[0], sc[1], sc[2], sc[3]};   // Gamma_{8tg-1} / Gamma_C
-#pragma unroll
-                    for (int j = 3; j >= 0; --j) {
-                        const int rp = tg * 8 - 4 + j;
-                        if (rp >= 0) {
-                            float kv[4], av[4];
-                            unpack4(raw_quad(sm, RAW_K, rp, cq), kv);
-                            unpack4(raw_quad(sm, RAW_A, rp, cq), av);
-                            const bool v = rp < nvalid;
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                kw[j][c] = v ? __fdividef(kv[c], sb4[c]) : 0.f;
-                                sb4[c] = v ? __fdividef(sb4[c], av[c]) : sb4[c];
-                            }
-                        } else {
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) kw[j][c] = 0.f;
-                        }
-                    }
-                }
-#pragma unroll 1
-                for (int i = 0; i < 8; ++i) {
-                    const int r = tg * 8 + i;
-                    const bool v = r < nvalid;
-                    float al[4], kv[4], qv[4], e[4], oa[4], oq[4], kb[4];
-                    unpack4(raw_quad(sm, RAW_A, r, cq), al);
-                    unpack4(raw_quad(sm, RAW_K, r, cq), kv);
-                    unpack4(raw_quad(sm, RAW_Q, r, cq), qv);
-                    erase_gate4(x, r, cq, e);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        sc[c] *= v ? al[c] : 1.f;
-                        oa[c] = v ? sc[c] * (e[c] * kv[c]) : 0.f;
-                        oq[c] = v ? sc[c] * qv[c] : 0.f;
-                        kb[c] = v ? __fdividef(kv[c], sc[c]) : 0.f;
-                    }
-                    *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, r, cq)) = pack4(oa);
-                    *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, 64 + r, cq)) = pack4(oq);
-                    *reinterpret_cast<uint2 *>(sm + OFF_KB + sw_half(8192, r, cq)) = pack4(kb);
-                    // partial sums of P_{r,r-w} over this lane's channels, slots 5-7 unused
-                    float pv[8];
-                    pv[0] = oq[0] * kb[0] + oq[1] * kb[1] + oq[2] * kb[2] + oq[3] * kb[3];
-#pragma unroll
-                    for (int w = 1; w < PBAND; ++w)
-                        pv[w] = oq[0] * kw[4 - w][0] + oq[1] * kw[4 - w][1] + oq[2] * kw[4 - w][2] + oq[3] * kw[4 - w][3];
-                    pv[5] = pv[6] = pv[7] = 0.f;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        kw[0][c] = kw[1][c]; kw[1][c] = kw[2][c]; kw[2][c] = kw[3][c]; kw[3][c] = kb[c];
-                    }
-                    // reduce-scatter of 8 slots over 32 lanes: lane keeps slot 4*b4 + 2*b3 + b2
-                    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float send = b4 ? pv[k] : pv[k + 4];
-                        pv[k] = (b4 ? pv[k + 4] : pv[k]) + __shfl_xor_sync(0xffffffffu, send, 16);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 2; ++k) {
-                        const float send = b3 ? pv[k] : pv[k + 2];
-                        pv[k] = (b3 ? pv[k + 2] : pv[k]) + __shfl_xor_sync(0xffffffffu, send, 8);
-                    }
-                    {
-                        const float send = b2 ? pv[0] : pv[1];
-                        pv[0] = (b2 ? pv[1] : pv[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
-                    }
-                    pv[0] += __shfl_xor_sync(0xffffffffu, pv[0], 2);
-                    pv[0] += __shfl_xor_sync(0xffffffffu, pv[0], 1);
-                    const int slot = (b4 ? 4 : 0) + (b3 ? 2 : 0) + (b2 ? 1 : 0);
-                    if ((lane & 3) == 0 && slot < PBAND) s_pband[r * PBAND + slot] = (v && r - slot >= 0) ? pv[0] : 0.f;
+                // one forward sweep per item; band partials to the F region, reduced after the A/P GEMM issue
+                float *band_part = reinterpret_cast<float *>(sm + OFF_F);
+                if (nvalid == C) {
+                    if (gdn2) fast_rows<true, true, SPLIT ? 4 : 1>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    else fast_rows<true, false, SPLIT ? 4 : 1>(x, s_tot, gamc, band_part, tg, cq, lane);
+                } else {
+                    fast_rows<false, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
                 }
             } else {
             {
@@ -890,6 +921,9 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                         mma_bf16(tbase + TM_AP, dK(sb + OFF_QA, 16384, kk), dK(sb + OFF_KB, 8192, kk), idesc, kk > 0);
                     mma_commit(bar_pmma);
                 }
+                // band of P while the GEMM runs; the partials' F region is rewritten by the read-out below
+                band_reduce(reinterpret_cast<const float *>(sm + OFF_F), s_pband, nvalid, ptid, NPREP);
+                group_sync(BAR_PREP, NPREP);
                 wait_pmma();
                 if (ptid == 0 && nxt.valid) issue_tma(nxt);   // raw tiles consumed
                 // rows 0-63: A (strictly lower, scaled by e_r), rows 64-127: P (band exact)
@@ -1145,7 +1179,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
 #pragma unroll
                         for (int q4 = 0; q4 < 4; ++q4)
                             *reinterpret_cast<uint4 *>(sm + OFF_QA + sw_chunk(16384, r, phalf * 8 + c32 * 4 + q4)) =
-                                pack8(v + q4 * 8);
+                                pack8_neg(v + q4 * 8);
                     }
                 }
             }
@@ -1205,6 +1239,9 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
 // buffers in shared memory, the next-but-one chunk loading while a chunk is
 // processed.  Warps w and w + 4 share TMEM lane quarter w (value columns
 // 32w .. 32w+31) and split the TMEM columns of every tile between them.
+// Chunk c's o is staged in shared memory after its step-7 GEMMs and goes to
+// HBM while the step-6 GEMMs of chunk c + 1 run (global stores, no tensor
+// memory traffic next to the GEMMs).
 constexpr int CK_NT = 256;
 constexpr uint32_t CK_BUF = SLOT_BYTES;        // a slot image; M (or v) at SL_M
 constexpr uint32_t CK_S0T = 2 * CK_BUF;         // state operand bf16 128 x 128, K-major
@@ -1212,6 +1249,7 @@ constexpr uint32_t CK_UT = CK_S0T + 32768;      // U^T bf16 128 x 64, then o sta
 constexpr uint32_t CK_BAR = CK_UT + 16384;      // mbarriers: load[2], mma
 constexpr uint32_t CK_TMEM = CK_BAR + 32;
 constexpr uint32_t CK_ALLOC = CK_BAR + 64 + 1024;
+constexpr uint32_t CK_TMEM_COLS = 256;   // S^T [0,128), U^T [128,192), O^T [192,256)
 static_assert(CK_ALLOC <= 232448, "shared memory budget");
 static_assert((CK_BUF & 1023) == 0 && (CK_S0T & 1023) == 0 && (CK_UT & 1023) == 0, "swizzle atoms");
 
@@ -1232,7 +1270,7 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + CK_TMEM);
     uint8_t *op = (uint8_t *)a.o;
 
-    if (warp == 0) tmem_alloc(s_tmem, 256);
+    if (warp == 0) tmem_alloc(s_tmem, CK_TMEM_COLS);
     if (tid == 0) {
         for (int i = 0; i < 3; ++i) mbar_init(bar_load + i, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1259,6 +1297,29 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
             tma_load_3d(dst + SL_M + 8192, &P.tv, bar_load + buf, 64, h, g);
         }
     };
+    // o of chunk c: TMEM O^T -> bf16 staging [token][j] in the U^T tile (free once the step-7
+    // GEMMs have read it), then 16-byte rows to HBM
+    unsigned short *ost = reinterpret_cast<unsigned short *>(sm + CK_UT);
+    auto stage_o = [&]() {
+        float v[32];
+        tmem_ld32(tbase + lane_base + TM_O + half * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const uint32_t pk = pack_bf16(v[e], v[e + 1]);
+            ost[(half * 32 + e) * 128 + jcol] = (unsigned short)(pk & 0xFFFFu);
+            ost[(half * 32 + e + 1) * 128 + jcol] = (unsigned short)(pk >> 16);
+        }
+    };
+    auto store_o = [&](int c) {
+        const int nv = min(C, len - c * C);
+        const size_t rb = (size_t)row0 + c * C;
+        for (int e = tid; e < nv * 16; e += CK_NT) {
+            const int r = e >> 4, cgo = e & 15;
+            *reinterpret_cast<uint4 *>(op + (((rb + r) * H + h) * D + cgo * 8) * 2) =
+                *reinterpret_cast<const uint4 *>(sm + CK_UT + r * 256 + cgo * 16);
+        }
+    };
     if (tid == 0) {
         if (nchunks > 0) issue_load(0, 0);
         if (nchunks > 1) issue_load(1, 1);
@@ -1276,44 +1337,49 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
         tmem_wait_st();
     }
     uint32_t ph_mma = 0;
+    bool mma_pending = false;   // thread 0: GEMMs issued but not yet committed and waited for
     int ch = 0;
     for (; ch < nchunks && ok; ++ch) {
         const int buf = ch & 1;
         const uint32_t bufa = sb + buf * CK_BUF;
-        const int nvalid = min(C, len - ch * C);
-        const size_t rowbase = (size_t)row0 + ch * C;
         if (!mbar_wait_cycles(bar_load + buf, (ch >> 1) & 1, WAIT_CYCLES)) ok = false;
         tc_fence_after();
+        if (tid == 0 && ok) {   // U'^T = M^T (T Diag(w))^T: independent of the state, issued first
+            const uint32_t id_u = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tbase + TM_U, dMN(bufa + SL_M, 8192, kk), dK(bufa + SL_TBF, 8192, kk), id_u, kk > 0);
+            mma_pending = true;   // completed by the step-6 commit
+        }
         const int *meta = reinterpret_cast<const int *>(sm + buf * CK_BUF + SL_META);
         const float *gamC = reinterpret_cast<const float *>(meta);
         // a slot this call's preparation kernel did not complete reads as a failure
         ok = __syncthreads_and(ok && (meta[128] & META_OK) && meta[129] == (int)P.epoch) != 0;
         if (!ok) break;
         const bool fast = (meta[128] & META_FAST) != 0;
-        if (tid == 0) {   // U'^T = M^T (T Diag(w))^T: independent of the state, issued first
-            tc_fence_after();
-            const uint32_t id_u = idesc_bf16(128, 64, true, false);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tbase + TM_U, dMN(bufa + SL_M, 8192, kk), dK(bufa + SL_TBF, 8192, kk), id_u, kk > 0);
-        }
         // ---- state pass: S^T *= Gamma_C in TMEM; bf16 operand copy (scaled on the fast path)
-#pragma unroll 1
-        for (int c32 = 0; c32 < 2; ++c32) {
-            const int i0 = half * 64 + c32 * 32;
-            float s[32], t[32];
-            tmem_ld32(tbase + lane_base + TM_S + i0, s);
+        {
+            float s[64];
+            tmem_ld32(tbase + lane_base + TM_S + half * 64, s);
+            tmem_ld32(tbase + lane_base + TM_S + half * 64 + 32, s + 32);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                t[e] = s[e] * gamC[i0 + e];
-                if (fast) s[e] = t[e];
-            }
+            for (int c32 = 0; c32 < 2; ++c32) {
+                const int i0 = half * 64 + c32 * 32;
+                float *sv = s + c32 * 32;
+                float t[32];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4 *>(sm + CK_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
-            tmem_st16(tbase + lane_base + TM_S + i0, t);
-            tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
+                for (int e = 0; e < 32; ++e) {
+                    t[e] = sv[e] * gamC[i0 + e];
+                    if (fast) sv[e] = t[e];
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                    *reinterpret_cast<uint4 *>(sm + CK_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) =
+                        pack8(sv + q4 * 8);
+                tmem_st16(tbase + lane_base + TM_S + i0, t);
+                tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
+            }
         }
         tmem_wait_st();
         fence_async_smem();
@@ -1322,19 +1388,16 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
         // ---- step 6: U^T -= S^T W^T ; O^T = S^T Q^T
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t id_neg = idesc_bf16(128, 64, false, false, true);
-            const uint32_t id_pos = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                mma_bf16(tbase + TM_U, dK(sb + CK_S0T, 16384, kk), dK(bufa + SL_QA, 16384, kk), id_neg, 1);
-                mma_bf16(tbase + TM_O, dK(sb + CK_S0T, 16384, kk), dK(bufa + SL_QA + 8192, 16384, kk), id_pos,
-                         kk > 0);
-            }
+            step6_mmas(tbase, sb + CK_S0T, bufa + SL_QA);
             mma_commit(bar_mma);
         }
+        // ---- o of the previous chunk, staged in the U^T tile, to HBM while the step-6 GEMMs run
+        if (ch > 0) store_o(ch - 1);
         if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
         ph_mma ^= 1;
+        mma_pending = false;
         tc_fence_after();
+        __syncthreads();   // staging read before the U^T tile is rewritten
         // ---- U^T row j -> bf16 K-major tile (rows j, K = token); tokens 32 half .. 32 half + 31
         {
             float v[32];
@@ -1364,30 +1427,17 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
         tc_fence_after();
         // every read of this buffer is done: load chunk ch + 2 into it
         if (tid == 0 && ok && ch + 2 < nchunks) issue_load(ch + 2, buf);
-        // ---- o: TMEM (lane j, column r) -> bf16 staging [r][j] in the U^T slot -> HBM
-        unsigned short *ost = reinterpret_cast<unsigned short *>(sm + CK_UT);
-        {
-            float v[32];
-            tmem_ld32(tbase + lane_base + TM_O + half * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-                const uint32_t pk = pack_bf16(v[e], v[e + 1]);
-                ost[(half * 32 + e) * 128 + jcol] = (unsigned short)(pk & 0xFFFFu);
-                ost[(half * 32 + e + 1) * 128 + jcol] = (unsigned short)(pk >> 16);
-            }
-        }
+        stage_o();   // the U^T tile is free: the step-7 GEMMs are done
         tc_fence_before();
-        __syncthreads();
-        for (int e = tid; e < nvalid * 16; e += CK_NT) {
-            const int r = e >> 4, cgo = e & 15;
-            *reinterpret_cast<uint4 *>(op + (((rowbase + r) * H + h) * D + cgo * 8) * 2) =
-                *reinterpret_cast<const uint4 *>(sm + CK_UT + r * 256 + cgo * 16);
-        }
-        ok = __syncthreads_and(ok) != 0;   // staging read before the next U^T write
+        ok = __syncthreads_and(ok) != 0;
     }
-    if (!ok && tid == 0) {   // drain loads still in flight (bounded)
+    if (ok && nchunks > 0) store_o(nchunks - 1);
+    if (!ok && tid == 0) {   // drain loads and an uncommitted GEMM still in flight (bounded)
         for (int c = ch; c < nchunks && c < ch + 2; ++c) mbar_wait_cycles(bar_load + (c & 1), (c >> 1) & 1, WAIT_CYCLES);
+        if (mma_pending) {
+            mma_commit(bar_mma);
+            mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES);
+        }
     }
     // ---- final state (NaN if a wait timed out or a slot was missing)
     __syncthreads();
@@ -1407,7 +1457,7 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tbase, 256);
+    if (warp == 0) tmem_dealloc(tbase, CK_TMEM_COLS);
 }
 
 // ---- host side --------------------------------------------------------------
