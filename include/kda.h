@@ -20,10 +20,13 @@
  *
  * Memory model.  Every tensor pointer is a DEVICE pointer owned by the
  * caller, 16-byte aligned, densely packed in the row-major layouts below.
- * The library allocates no device memory, never frees caller memory, keeps
- * no state between calls (it is reentrant and thread-safe) and enqueues all
- * work asynchronously on `stream` (a cudaStream_t; NULL = legacy default
- * stream).  A call returns after the launch: asynchronous kernel faults
+ * The library never frees caller memory and enqueues all work
+ * asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream).
+ * Only kda_chunk_fwd allocates device memory: the split form's workspace,
+ * stream-ordered and released within the call (kda_chunk_fwd_ws takes it
+ * from the caller instead).  Between calls the library keeps only per-device
+ * set-up (kernel attributes, SM count, the fixed scratch array of
+ * kda_chunk_fwd_noalloc); it is reentrant and thread-safe.  A call returns after the launch: asynchronous kernel faults
  * surface at the caller's next synchronisation, as with any CUDA launch.
  *
  * Errors.  Every entry point validates all arguments on the host before it
@@ -122,8 +125,10 @@ int kda_chunk_fwd(int variant, int gate_range, int dtype,
  * form would run, N = num_seqs with cu_seqlens (has_cu_seqlens = 1) or B
  * without; 0 when another form runs (scan: dtype, head dims or chunk size;
  * fused: chosen by shape on the current device or forced) and when an
- * argument is out of range.  By shape, the split form is chosen when
- * 2 * N * H <= the device's SM count.
+ * argument is out of range.  By shape, the split form is chosen for packed
+ * (cu_seqlens) batches and, for B equal-length sequences, when a cost model
+ * of measured per-chunk times favours it (for example B*H <= about 0.8x the
+ * SM count, or a last partial wave of the fused kernel).
  */
 size_t kda_chunk_fwd_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
                                     int has_cu_seqlens, int num_seqs, int chunk_size, unsigned flags);

@@ -56,6 +56,7 @@
 #include <cuda.h>
 #include <algorithm>
 #include <atomic>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -91,7 +92,9 @@ constexpr int PBAND = 5;   // P_{r,s} for r-4 <= s <= r computed exactly (SIMT) 
 constexpr uint32_t M_G1 = OFF_MISC, M_G2 = OFF_MISC + 256, M_GAMC = OFF_MISC + 512, M_TOT = OFF_MISC + 1536,
                    M_PBAND = OFF_MISC + 5632, M_FAST = OFF_MISC + 6912, M_BAR = OFF_MISC + 6920,
                    M_TMEM = OFF_MISC + 6976;
-constexpr uint32_t SMEM_USED = OFF_MISC + 6992;
+constexpr uint32_t M_G1B = OFF_MISC + 6992, M_G2B = OFF_MISC + 7248;   // gates of the other item parity
+constexpr uint32_t M_ITEM = OFF_MISC + 7504;                            // split: decoded items [2][8] int
+constexpr uint32_t SMEM_USED = OFF_MISC + 7568;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack for aligning the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert((OFF_TBF & 1023) == 0 && (OFF_PBF & 1023) == 0 && (OFF_QA & 1023) == 0, "swizzle atoms");
@@ -509,8 +512,10 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
     const int len = SPLIT ? 0 : seq_len(a, n);
     const int nchunks = (len + C - 1) / C;
 
-    float *s_g1 = reinterpret_cast<float *>(sm + M_G1);
-    float *s_g2 = reinterpret_cast<float *>(sm + M_G2);
+    // scalar gates, per item parity (filled one item ahead)
+    auto s_g1buf = [&](uint32_t parity) { return reinterpret_cast<float *>(sm + (parity ? M_G1B : M_G1)); };
+    auto s_g2buf = [&](uint32_t parity) { return reinterpret_cast<float *>(sm + (parity ? M_G2B : M_G2)); };
+    int *s_items = reinterpret_cast<int *>(sm + M_ITEM);
     float *s_gamC = reinterpret_cast<float *>(sm + M_GAMC);     // [2][128]: chunk parity
     float *s_tot = reinterpret_cast<float *>(sm + M_TOT);       // [8][128] block totals of alpha
     float *s_pband = reinterpret_cast<float *>(sm + M_PBAND);   // [64][PBAND]: P_{r, r-w}
@@ -683,18 +688,36 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             tc_fence_before();
             group_sync(BAR_PREP, NPREP);
         };
-        // scalar gates of a chunk's row `ptid` as raw bf16 bits, fetched one chunk ahead
-        auto fetch_gates = [&](const Item &it, uint32_t &ge, uint32_t &gw) {
-            const int r = ptid, nv = min(C, it.len - it.c * C);
+        // scalar gates of row r of a chunk into the gate arrays of item parity `parity`
+        // (0 past the chunk's end; GDN-2 keeps its gates channel-wise: 1 here)
+        auto fetch_gates = [&](const Item &it, int r, uint32_t parity) {
+            const int nv = min(C, it.len - it.c * C);
             const size_t tok = ((size_t)it.row0 + it.c * C + r) * H + it.h;
             const bool v = r < nv;
             const unsigned short *g1u = reinterpret_cast<const unsigned short *>(g1p);
             const unsigned short *g2u = reinterpret_cast<const unsigned short *>(g2p);
+            uint32_t ge, gw;
             if (gdn2) { ge = v ? 0x3F80u : 0u; gw = ge; }   // bf16 1.0 / 0.0
             else {
                 ge = v ? (uint32_t)g1u[tok] : 0u;
                 gw = v ? (uint32_t)(a.variant == KDA ? g1u[tok] : g2u[tok]) : 0u;
             }
+            s_g1buf(parity)[r] = __uint_as_float(ge << 16);
+            s_g2buf(parity)[r] = __uint_as_float(gw << 16);
+        };
+        // split: decoded items travel through shared memory, two ahead (decoded by one
+        // thread while most warps wait in the T solve)
+        auto put_item = [&](const Item &it, uint32_t slot) {
+            int *d = s_items + slot * 8;
+            d[0] = it.n; d[1] = it.h; d[2] = it.c; d[3] = it.row0; d[4] = it.len; d[5] = it.slot;
+            d[6] = it.valid ? 1 : 0;
+        };
+        auto get_item = [&](uint32_t slot) {
+            const int *d = s_items + slot * 8;
+            Item it;
+            it.n = d[0]; it.h = d[1]; it.c = d[2]; it.row0 = d[3]; it.len = d[4]; it.slot = d[5];
+            it.valid = d[6] != 0;
+            return it;
         };
 
         // the chain of items this role prepares
@@ -706,30 +729,30 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             return it;
         };
         Item cur = SPLIT ? next_split_item(a, N, nwork, wnext) : fused_item(0);
+        Item nxt_boot{};
+        if (SPLIT) {   // the first two items are decoded by every thread
+            wnext += gridDim.x;
+            nxt_boot = next_split_item(a, N, nwork, wnext);
+        }
         const bool need_v = !SPLIT || gdn2;   // the split kernel leaves U' to the chain kernel
         if (cur.valid && ptid == 0) {
             issue_tma(cur);
             if (need_v) issue_tma_v(cur, 0);
         }
-        uint32_t gate_e = 0u, gate_w = 0u;
-        if (ptid < C && cur.valid) fetch_gates(cur, gate_e, gate_w);
+        if (ptid < C && cur.valid) fetch_gates(cur, ptid, 0);
 
         for (int ch = 0; cur.valid && ok; ++ch) {
             const uint32_t par = ch & 1, ppar = (ch - 1) & 1;
-            if (SPLIT) wnext += gridDim.x;
-            const Item nxt = SPLIT ? next_split_item(a, N, nwork, wnext) : fused_item(ch + 1);
+            const Item nxt = !SPLIT ? fused_item(ch + 1) : (ch == 0 ? nxt_boot : get_item((ch + 1) & 1));
             const int h = cur.h;
             const int nvalid = min(C, cur.len - cur.c * C);
             const size_t rowbase = (size_t)cur.row0 + cur.c * C;
+            float *const s_g1 = s_g1buf(par);
+            float *const s_g2 = s_g2buf(par);
             const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
             const uint32_t OFF_MTC = mt_off(par);
             float *gamc = SPLIT ? reinterpret_cast<float *>(sm + OFF_UT) : s_gamC + par * 128;
 
-            if (ptid < C) {
-                s_g1[ptid] = __uint_as_float(gate_e << 16);
-                s_g2[ptid] = __uint_as_float(gate_w << 16);
-                if (nxt.valid) fetch_gates(nxt, gate_e, gate_w);
-            }
             if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
             ph_tma ^= 1;
             if (need_v) {
@@ -775,11 +798,10 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                     *pv = pack4(mv);
                 }
             }
-            if (SPLIT && ptid == 0) {
-                bulk_wait_read();   // the previous item's slot stores have read their tiles
-                if (gdn2 && nxt.valid) issue_tma_v(nxt, par ^ 1u);
-            }
+            if (SPLIT && lane == 0 && pw < 5) bulk_wait_read();   // the previous item's slot stores
             in_range = group_sync_and(BAR_PREP, NPREP, in_range);
+            // GDN-2: the next item's v into the M tile the previous item stored (read: waited above)
+            if (SPLIT && ptid == 0 && gdn2 && nxt.valid) issue_tma_v(nxt, par ^ 1u);
 
             // ===== Gamma_C and the per-chunk path decision ========================
             bool gam_ok = true;
@@ -1036,6 +1058,11 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
 #pragma unroll
                 for (int r2 = 0; r2 < 16; ++r2) Tf[(16 * I + r2) * TP + 16 * I + c] = xv[r2];
                 for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * TP + 16 * I + c] = 0.f;  // above the block
+            } else if (ptid < 64 + C) {   // meanwhile: the next item's gates
+                if (nxt.valid) fetch_gates(nxt, ptid - 64, par ^ 1u);
+            } else if (SPLIT && ptid == 64 + C) {   // and the item after it
+                wnext += gridDim.x;
+                put_item(nxt.valid ? next_split_item(a, N, nwork, wnext) : Item{}, par);
             }
             group_sync(BAR_PREP, NPREP);
             {   // X = A_{I+1,I} D_I for I = 0, 2 (two outputs per thread)
@@ -1192,13 +1219,16 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             tc_fence_before();
             ok = group_sync_and(BAR_PREP, NPREP, ok);
             if (!SPLIT && ptid == 0) mbar_arrive(bar_ready);   // chunk ch's operands are ready for the chain
-            if (SPLIT && ptid == 0 && ok) {   // the slot: operand tiles, meta block, GDN-2 M
+            if (SPLIT && ok && lane == 0 && pw < 5) {   // the slot, one bulk store per warp
                 uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
-                bulk_store(slot + SL_QA, sm + OFF_QA, 49152);   // QA and Kbar are adjacent
-                bulk_store(slot + SL_PBF, sm + OFF_PBF, 8192);
-                bulk_store(slot + SL_TBF, sm + OFF_TBF, 8192);
-                bulk_store(slot + SL_META, sm + OFF_UT, SL_META_BYTES);
-                if (gdn2) bulk_store(slot + SL_M, sm + OFF_MTC, 16384);
+                if (pw == 0) bulk_store(slot + SL_QA, sm + OFF_QA, 32768);
+                else if (pw == 1) bulk_store(slot + SL_KB, sm + OFF_KB, 16384);
+                else if (pw == 2) bulk_store(slot + SL_PBF, sm + OFF_PBF, 8192);
+                else if (pw == 3) bulk_store(slot + SL_TBF, sm + OFF_TBF, 8192);
+                else {
+                    bulk_store(slot + SL_META, sm + OFF_UT, SL_META_BYTES);
+                    if (gdn2) bulk_store(slot + SL_M, sm + OFF_MTC, 16384);
+                }
                 bulk_commit();
             }
             cur = nxt;
@@ -1207,7 +1237,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
             if (need_v) mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
         }
-        if (SPLIT && ptid == 0) bulk_wait_all();
+        if (SPLIT && lane == 0 && pw < 5) bulk_wait_all();
     }
 
     // ---- final state (NaN if an internal wait timed out) ----------------------
@@ -1548,16 +1578,21 @@ cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
 
 bool chunk_prefer_split(const FwdArgs &a)
 {
-    // The fused kernel runs one CTA per (sequence, head) for the whole sequence.
-    // When those CTAs would leave at least half of the SMs idle, spreading the
-    // operand preparation over every SM outweighs the workspace round trip.
+    // Cost model from measured per-chunk times on B200 (SM cycles): preparation of one
+    // (chunk, head) ~13.8 K, the split chain ~4.1 K, the fused kernel's critical path ~15.4 K.
+    // With U = N*H units on S SMs and W = ceil(U / S) waves of the per-unit kernels:
+    //   fused ~ W * 15.4,   split ~ (U / S) * 13.8 + W * 4.1   (per chunk of a unit).
+    // Packed (varlen) batches take the split form: the fused kernel's time is that of the
+    // longest sequence per CTA, while the preparation kernel balances chunks over all SMs.
     int num_sms = 0;
     if (device_setup(num_sms) != cudaSuccess) {
         (void)cudaGetLastError();
         return false;
     }
-    const long long N = a.cu_seqlens ? a.num_seqs : a.B;
-    return N * a.H * 2 <= num_sms;
+    if (a.cu_seqlens) return true;
+    const double U = (double)a.B * a.H, S = num_sms;
+    const double W = std::ceil(U / S);
+    return (U / S) * 13.8 + W * 4.1 < W * 15.4;
 }
 
 size_t chunk_split_workspace_bytes(const FwdArgs &a)
