@@ -464,11 +464,17 @@ def main():
     decode = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank)
     also = []
     if args.extra:
-        for name, mk in (("Complex-KDA chunked forward B=8 H=16 T=8192 d=128 chunk=64 bf16", lambda: W.ckda_bf16(rank)),
-                         ("RDA varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("rda", rank)),
-                         ("GDN-2 varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("gdn2", rank))):
+        prep = lambda: W.make_chunk_inputs("kda", "standard", "bf16", B=4, T=4096, H=16, d_k=128, d_v=128,
+                                           seed=rank_workload_seed(rank), logits=True, raw_k=True)
+        for name, mk, xflags in (
+                ("Complex-KDA chunked forward B=8 H=16 T=8192 d=128 chunk=64 bf16", lambda: W.ckda_bf16(rank), 0),
+                ("RDA varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("rda", rank), 0),
+                ("GDN-2 varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("gdn2", rank), 0),
+                ("KDA B=4 H=16 T=4096 bf16 from gate logits and raw keys (in-kernel activations, L2 norm)",
+                 prep, 16 | 32)):
             x = mk()
-            r = run_chunk_workload(x, max(5, args.steps // 2), args.warmup, world, peaks, e2e=False, flags=fflags)
+            r = run_chunk_workload(x, max(5, args.steps // 2), args.warmup, world, peaks, e2e=False,
+                                   flags=fflags | xflags)
             also.append({"workload": name, "value": r["tokens_per_step"] * world * max(5, args.steps // 2) / r["total_s"],
                          "unit": UNIT, "ms_per_step": r["avg_launch_s"] * 1e3, "form": r["form"],
                          "hbm_frac": r["hbm"]["frac"],

@@ -73,6 +73,16 @@ enum kda_status {
                                        tensor-core chunked kernel applies (testing aid) */
 #define KDA_FLAG_FORCE_FUSED    4u  /* tensor-core path: force the single fused kernel */
 #define KDA_FLAG_FORCE_SPLIT    8u  /* tensor-core path: force the two-kernel path */
+/* Input preparation inside the kernels (chunked forward and decode), saving
+ * the separate passes over HBM a model would otherwise run first:
+ *   KDA_FLAG_GATE_LOGITS -- alpha, g1 and g2 hold logits.  Standard range:
+ *       alpha = exp(-softplus(x)) = 1/(1+e^x), beta / e / w / b = sigmoid(y);
+ *       extended range: alpha = tanh(x), beta / e / w / b = 2 sigmoid(y).
+ *   KDA_FLAG_L2NORM_K -- k_t is replaced by k_t / max(||k_t||_2, 1e-6) per
+ *       token and head.
+ * Both are computed in fp32 from the stored inputs. */
+#define KDA_FLAG_GATE_LOGITS   16u
+#define KDA_FLAG_L2NORM_K      32u
 
 /*
  * kda_chunk_fwd -- chunked-parallel forward over whole sequences.

@@ -19,7 +19,7 @@ import torch
 
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_version",
            "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_FORCE_SCAN", "FLAG_FORCE_FUSED",
-           "FLAG_FORCE_SPLIT"]
+           "FLAG_FORCE_SPLIT", "FLAG_GATE_LOGITS", "FLAG_L2NORM_K"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
@@ -29,6 +29,8 @@ _DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 FLAG_FORCE_SCAN = 2    # token-by-token CUDA scan even where the tensor-core path applies
 FLAG_FORCE_FUSED = 4   # tensor-core path, single fused kernel
 FLAG_FORCE_SPLIT = 8   # tensor-core path, preparation kernel + chain kernel
+FLAG_GATE_LOGITS = 16  # alpha and gates given as logits; the kernels apply the activations
+FLAG_L2NORM_K = 32     # k given unnormalised; the kernels L2-normalise it per token and head
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -184,7 +186,7 @@ def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torc
 
 def kda_decode_step(variant: Union[str, int], gate_range: Union[str, int], q: torch.Tensor, k: torch.Tensor,
                     v: torch.Tensor, alpha: torch.Tensor, g1: torch.Tensor, g2: Optional[torch.Tensor],
-                    state: torch.Tensor, o: Optional[torch.Tensor] = None, stream=None):
+                    state: torch.Tensor, o: Optional[torch.Tensor] = None, flags: int = 0, stream=None):
     """One decode step for N sequences (C: kda_decode_step); ``state`` fp32
     [N,H,d_k,d_v] is updated in place.  q, k, alpha [N,H,d_k]; v [N,H,d_v].
     Returns o [N,H,d_v]."""
@@ -215,7 +217,7 @@ def kda_decode_step(variant: Union[str, int], gate_range: Union[str, int], q: to
         o = torch.empty((N, H, dv), dtype=dt, device=dev)
     _check(o, "o", dt, (N, H, dv), dev)
     rc = lib.kda_decode_step(var, rng, _DTYPES[dt], N, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
-                             _ptr(g1), _ptr(g2), _ptr(state), _ptr(o), 0, _stream(stream, dev))
+                             _ptr(g1), _ptr(g2), _ptr(state), _ptr(o), int(flags), _stream(stream, dev))
     if rc != 0:
         raise KdaError(rc, "kda_decode_step")
     return o

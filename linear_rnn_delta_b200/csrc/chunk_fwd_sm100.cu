@@ -253,6 +253,7 @@ struct ChunkCtx {
     size_t rowbase;
     int H, h, nvalid;
     bool gdn2;
+    bool logits, ext;   // input preparation: GDN-2's erase vector arrives as logits; extended range
 };
 
 // Channel-wise part of the erase direction of row r for 4 channels (GDN-2:
@@ -262,6 +263,10 @@ __device__ __forceinline__ void erase_gate4(const ChunkCtx &x, int r, int cq, fl
 {
     if (x.gdn2 && r < x.nvalid) {
         unpack4(*reinterpret_cast<const uint2 *>(x.g1p + ((x.rowbase + r) * x.H + x.h) * D + cq * 4), e);
+        if (x.logits) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) e[c] = round_bf16(prep_gate(e[c], x.ext));
+        }
     } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c) e[c] = 1.f;
@@ -497,7 +502,9 @@ constexpr uint32_t BAR_PREP = 1, BAR_CHAIN = 2;
 // SPLIT = false: the fused kernel, one CTA per (sequence, head), both roles.
 // SPLIT = true: the preparation role alone (256 threads), persistent over all
 // chunks of all sequences and heads; each chunk's operands go to its slot.
-template <bool SPLIT>
+// PREP: input preparation requested (gate logits and / or raw keys); without
+// it the preparation code is compiled out.
+template <bool SPLIT, bool PREP>
 __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __grid_constant__ ChunkParams P)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -532,6 +539,8 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
     uint8_t *op = (uint8_t *)a.o;
     const bool gdn2 = a.variant == GDN2;
     const bool same_gates = a.variant != RDA;   // erase and write gates coincide: one T copy serves both
+    const bool logits = PREP && (a.prep & PREP_LOGITS) != 0, l2k = PREP && (a.prep & PREP_L2NORM_K) != 0;
+    const bool ext = a.ext != 0;
 
     if (warp == 0) tmem_alloc(s_tmem, 512);
     if (tid == 0) {
@@ -702,8 +711,13 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                 ge = v ? (uint32_t)g1u[tok] : 0u;
                 gw = v ? (uint32_t)(a.variant == KDA ? g1u[tok] : g2u[tok]) : 0u;
             }
-            s_g1buf(parity)[r] = __uint_as_float(ge << 16);
-            s_g2buf(parity)[r] = __uint_as_float(gw << 16);
+            float fe = __uint_as_float(ge << 16), fw = __uint_as_float(gw << 16);
+            if (logits && !gdn2 && v) {
+                fe = round_bf16(prep_gate(fe, ext));
+                fw = round_bf16(prep_gate(fw, ext));
+            }
+            s_g1buf(parity)[r] = fe;
+            s_g2buf(parity)[r] = fw;
         };
         // split: decoded items travel through shared memory, two ahead (decoded by one
         // thread while most warps wait in the T solve)
@@ -749,7 +763,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             const size_t rowbase = (size_t)cur.row0 + cur.c * C;
             float *const s_g1 = s_g1buf(par);
             float *const s_g2 = s_g2buf(par);
-            const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2};
+            const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2, logits, ext};
             const uint32_t OFF_MTC = mt_off(par);
             float *gamc = SPLIT ? reinterpret_cast<float *>(sm + OFF_UT) : s_gamC + par * 128;
 
@@ -760,6 +774,58 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                 ph_v ^= 1;
             }
             group_sync(BAR_PREP, NPREP);
+
+            // ===== 0. input preparation, in place in the raw tiles (this thread's 8 rows x 4 channels),
+            // rounded to bf16 as a separate activation / normalisation pass would have stored them
+            if (PREP && logits) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint2 *pa = reinterpret_cast<uint2 *>(sm + RAW_A + (tg * 8 + i) * 256 + cq * 8);
+                    float al[4];
+                    unpack4(*pa, al);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) al[c] = prep_alpha(al[c], ext);
+                    *pa = pack4(al);
+                }
+            }
+            if (PREP && l2k) {   // 1 / ||k_r|| of this warp's 8 rows: 4-channel partial sums, reduce-scattered
+                float ss[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float kv[4];
+                    unpack4(raw_quad(sm, RAW_K, tg * 8 + i, cq), kv);
+                    ss[i] = kv[0] * kv[0] + kv[1] * kv[1] + kv[2] * kv[2] + kv[3] * kv[3];
+                }
+                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float send = b4 ? ss[i] : ss[i + 4];
+                    ss[i] = (b4 ? ss[i + 4] : ss[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float send = b3 ? ss[i] : ss[i + 2];
+                    ss[i] = (b3 ? ss[i + 2] : ss[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+                {
+                    const float send = b2 ? ss[0] : ss[1];
+                    ss[0] = (b2 ? ss[1] : ss[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+                }
+                ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], 2);
+                ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], 1);
+                // lane 4 i holds row i's sum (i = 4 b4 + 2 b3 + b2): hand each lane its rows' scales
+                const float sc = prep_kscale(ss[0]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float sci = __shfl_sync(0xffffffffu, sc, ((i & 4) ? 16 : 0) + ((i & 2) ? 8 : 0) + ((i & 1) ? 4 : 0));
+                    uint2 *pk = reinterpret_cast<uint2 *>(sm + RAW_K + (tg * 8 + i) * 256 + cq * 8);
+                    float kv[4];
+                    unpack4(*pk, kv);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) kv[c] *= sci;
+                    *pk = pack4(kv);
+                }
+            }
 
             // ===== 1a. block totals of alpha (and range check) | GDN-2: M = w (.) v
             bool in_range = true;
@@ -790,7 +856,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                     if (r < nvalid) {
                         unpack4(*reinterpret_cast<const uint2 *>(g2p + ((rowbase + r) * H + h) * D + cq * 4), wv);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) mv[c] = wv[c] * vv[c];
+                        for (int c = 0; c < 4; ++c) mv[c] = (logits ? round_bf16(prep_gate(wv[c], ext)) : wv[c]) * vv[c];
                     } else {
 #pragma unroll
                         for (int c = 0; c < 4; ++c) mv[c] = 0.f;
@@ -1537,9 +1603,13 @@ cudaError_t device_setup(int &num_sms)
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!sms[dev]) {
-        if ((e = cudaFuncSetAttribute(chunk_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(chunk_fwd_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       SMEM_ALLOC)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(chunk_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            (e = cudaFuncSetAttribute(chunk_fwd_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      SMEM_ALLOC)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_fwd_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      SMEM_ALLOC)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_fwd_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       SMEM_ALLOC)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CK_ALLOC)) !=
                 cudaSuccess ||
@@ -1572,7 +1642,8 @@ cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
     ChunkParams p;
     if ((e = make_params(p, a)) != cudaSuccess) return e;
     const int N = a.cu_seqlens ? a.num_seqs : a.B;
-    chunk_fwd_kernel<false><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
+    if (a.prep) chunk_fwd_kernel<false, true><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
+    else chunk_fwd_kernel<false, false><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -1618,7 +1689,8 @@ cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st
     const long long nwork = (long long)p.nslots * a.H;
     if (rows > 0 && nwork > 0) {
         const unsigned grid = (unsigned)std::min<long long>(nwork, num_sms);
-        chunk_fwd_kernel<true><<<grid, NPREP, SMEM_ALLOC, st>>>(p);
+        if (a.prep) chunk_fwd_kernel<true, true><<<grid, NPREP, SMEM_ALLOC, st>>>(p);
+        else chunk_fwd_kernel<true, false><<<grid, NPREP, SMEM_ALLOC, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     chunk_chain_kernel<<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);

@@ -25,7 +25,37 @@ struct FwdArgs {
     const float *s0;
     float *sf;
     void *o;
+    unsigned prep = 0;   // PREP_* bits: input preparation done by the kernels
+    int ext = 0;         // extended (Complex KDA) gate range: selects the activations
 };
+
+// ---- input preparation (optional, applied once where the kernels read their inputs) ----
+// PREP_LOGITS: alpha and the gates arrive as logits.  Standard range:
+//   alpha = exp(-softplus(x)) = 1 / (1 + e^x),  gate = sigmoid(y);
+// extended range: alpha = tanh(x),  gate = 2 sigmoid(y).
+// PREP_L2NORM_K: k_t is replaced by k_t / max(||k_t||_2, 1e-6) per token and head.
+// Prepared values are computed in fp32 and rounded to the input dtype, as a
+// separate activation / normalisation pass would have stored them.
+constexpr unsigned PREP_LOGITS = 1u, PREP_L2NORM_K = 2u;
+constexpr float K_NORM_FLOOR = 1e-6f;
+
+__device__ __forceinline__ float prep_alpha(float x, bool ext)
+{
+    return ext ? tanhf(x) : __fdividef(1.f, 1.f + __expf(x));   // e^x = inf -> 0
+}
+__device__ __forceinline__ float prep_gate(float y, bool ext)
+{
+    const float s = __fdividef(1.f, 1.f + __expf(-y));
+    return ext ? 2.f * s : s;
+}
+__device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+template <typename T> __device__ __forceinline__ float round_to(float x) { return x; }
+template <> __device__ __forceinline__ float round_to<__nv_bfloat16>(float x) { return round_bf16(x); }
+// 1 / max(||k||, floor) from the sum of squares
+__device__ __forceinline__ float prep_kscale(float sumsq)
+{
+    return 1.f / fmaxf(sqrtf(sumsq), K_NORM_FLOOR);
+}
 
 // Internal launchers; each returns cudaSuccess or the launch error.
 cudaError_t launch_scan_fwd(const FwdArgs &a, bool bf16, cudaStream_t st);

@@ -28,7 +28,8 @@ struct DecodeShape {
     static_assert(RPT * RP == DK, "rows must divide evenly");
 };
 
-template <int DK, int DV, typename TIn>
+// PREP: input preparation requested; without it that code is compiled out.
+template <int DK, int DV, typename TIn, bool PREP>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::THREADS)
 decode_step_kernel(FwdArgs a)
 {
@@ -36,7 +37,7 @@ decode_step_kernel(FwdArgs a)
     constexpr int RP = Sh::RP, RPT = Sh::RPT, CT = Sh::CT;
     __shared__ __align__(16) float s_q[DK], s_k[DK], s_al[DK], s_at[DK], s_m[DV];
     __shared__ __align__(16) float s_red[2][RP][DV];
-    __shared__ float s_u[DV], s_p[DV], s_kq;
+    __shared__ float s_u[DV], s_p[DV], s_kq, s_ksc;
 
     const int nh = blockIdx.x;
     const int tid = threadIdx.x;
@@ -52,22 +53,45 @@ decode_step_kernel(FwdArgs a)
     const TIn *q = (const TIn *)a.q + (size_t)nh * DK, *k = (const TIn *)a.k + (size_t)nh * DK;
     const TIn *al = (const TIn *)a.alpha + (size_t)nh * DK, *v = (const TIn *)a.v + (size_t)nh * DV;
     const TIn *g1 = (const TIn *)a.g1, *g2 = (const TIn *)a.g2;
+    const bool logits = PREP && (a.prep & PREP_LOGITS), l2k = PREP && (a.prep & PREP_L2NORM_K), ext = a.ext != 0;
+    auto erase_gate = [&](int i) {   // beta / e, or GDN-2's b_i (activated from its logit on request)
+        const float g = (a.variant == GDN2) ? ld_f32(g1 + (size_t)nh * DK + i) : ld_f32(g1 + nh);
+        return logits ? round_to<TIn>(prep_gate(g, ext)) : g;
+    };
     for (int i = tid; i < DK; i += Sh::THREADS) {
         const float kk = ld_f32(k + i);
-        const float g = (a.variant == GDN2) ? ld_f32(g1 + (size_t)nh * DK + i) : ld_f32(g1 + nh);
+        float ai = ld_f32(al + i);
+        if (logits) ai = round_to<TIn>(prep_alpha(ai, ext));
         s_q[i] = ld_f32(q + i);
         s_k[i] = kk;
-        s_al[i] = ld_f32(al + i);
-        s_at[i] = g * kk;
+        s_al[i] = ai;
+        s_at[i] = erase_gate(i) * kk;
     }
     for (int j = tid; j < DV; j += Sh::THREADS) {
         float g;
         if (a.variant == KDA) g = ld_f32(g1 + nh);
         else if (a.variant == RDA) g = ld_f32(g2 + nh);
         else g = ld_f32(g2 + (size_t)nh * DV + j);
+        if (logits) g = round_to<TIn>(prep_gate(g, ext));
         s_m[j] = g * ld_f32(v + j);
     }
     __syncthreads();
+    if (l2k) {   // k / ||k|| (rounded to the input dtype); a~ = g (.) k with the normalised k
+        if (tid < 32) {
+            float ss = 0.f;
+            for (int i = tid; i < DK; i += 32) ss = fmaf(s_k[i], s_k[i], ss);
+#pragma unroll
+            for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+            if (tid == 0) s_ksc = prep_kscale(ss);
+        }
+        __syncthreads();
+        for (int i = tid; i < DK; i += Sh::THREADS) {
+            const float kn = round_to<TIn>(s_k[i] * s_ksc);
+            s_k[i] = kn;
+            s_at[i] = erase_gate(i) * kn;
+        }
+        __syncthreads();
+    }
 
     // 3. decay in registers; partial S'^T a~ and S'^T q over this thread's rows
     float pu[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -122,8 +146,13 @@ template <int DK, int DV>
 cudaError_t launch_dims(const FwdArgs &a, bool bf16, cudaStream_t st)
 {
     dim3 grid((unsigned)(a.B * a.H)), block(DecodeShape<DK, DV>::THREADS);
-    if (bf16) decode_step_kernel<DK, DV, __nv_bfloat16><<<grid, block, 0, st>>>(a);
-    else decode_step_kernel<DK, DV, float><<<grid, block, 0, st>>>(a);
+    if (bf16) {
+        if (a.prep) decode_step_kernel<DK, DV, __nv_bfloat16, true><<<grid, block, 0, st>>>(a);
+        else decode_step_kernel<DK, DV, __nv_bfloat16, false><<<grid, block, 0, st>>>(a);
+    } else {
+        if (a.prep) decode_step_kernel<DK, DV, float, true><<<grid, block, 0, st>>>(a);
+        else decode_step_kernel<DK, DV, float, false><<<grid, block, 0, st>>>(a);
+    }
     return cudaGetLastError();
 }
 

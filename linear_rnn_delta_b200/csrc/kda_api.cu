@@ -26,6 +26,14 @@ int cuda_fail(cudaError_t e, const char *where)
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Input-preparation flags and their kernel-side bits.
+constexpr unsigned PREP_FLAGS = KDA_FLAG_GATE_LOGITS | KDA_FLAG_L2NORM_K;
+unsigned prep_bits(unsigned flags)
+{
+    return ((flags & KDA_FLAG_GATE_LOGITS) ? kda::PREP_LOGITS : 0u) |
+           ((flags & KDA_FLAG_L2NORM_K) ? kda::PREP_L2NORM_K : 0u);
+}
 bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64 || c == 128; }
 
@@ -85,7 +93,7 @@ int chunk_args(kda::FwdArgs &a, int variant, int gate_range, int dtype, int B, i
     if (rc != KDA_OK) return rc;
     if (!chunk_ok(chunk_size))
         return fail(KDA_ERR_UNSUPPORTED, "chunk_size %d: supported are 16, 32, 64, 128", chunk_size);
-    if (flags & ~(KDA_FLAG_FORCE_SCAN | KDA_FLAG_FORCE_FUSED | KDA_FLAG_FORCE_SPLIT))
+    if (flags & ~(KDA_FLAG_FORCE_SCAN | KDA_FLAG_FORCE_FUSED | KDA_FLAG_FORCE_SPLIT | PREP_FLAGS))
         return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
     if ((flags & KDA_FLAG_FORCE_FUSED) && (flags & KDA_FLAG_FORCE_SPLIT))
         return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_FORCE_FUSED and KDA_FLAG_FORCE_SPLIT exclude each other");
@@ -102,7 +110,7 @@ int chunk_args(kda::FwdArgs &a, int variant, int gate_range, int dtype, int B, i
     if (final_state && !aligned16(final_state))
         return fail(KDA_ERR_INVALID_ARG, "final_state is not 16-byte aligned");
     a = kda::FwdArgs{variant, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens, N,
-                     initial_state, final_state, o};
+                     initial_state, final_state, o, prep_bits(flags), gate_range == KDA_RANGE_EXTENDED};
     return KDA_OK;
 }
 
@@ -257,10 +265,11 @@ extern "C" int kda_decode_step(int variant, int gate_range, int dtype,
     if (rc != KDA_OK) return rc;
     if (!state) return fail(KDA_ERR_INVALID_ARG, "state is NULL");
     if (!aligned16(state)) return fail(KDA_ERR_INVALID_ARG, "state is not 16-byte aligned");
-    if (flags) return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if (flags & ~PREP_FLAGS) return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
     if ((unsigned long long)N * H > (1ull << 31) - 1)
         return fail(KDA_ERR_INVALID_ARG, "N*H too large for one launch");
-    kda::FwdArgs a{variant, N, 1, H, d_k, d_v, q, k, v, alpha, g1, g2, nullptr, N, state, state, o};
+    kda::FwdArgs a{variant, N, 1, H, d_k, d_v, q, k, v, alpha, g1, g2, nullptr, N, state, state, o,
+                   prep_bits(flags), gate_range == KDA_RANGE_EXTENDED};
     cudaError_t e = kda::launch_decode_step(a, dtype == KDA_DTYPE_BF16, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
     return KDA_OK;

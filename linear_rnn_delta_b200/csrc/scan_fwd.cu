@@ -15,7 +15,8 @@
 //   S_ij = alpha_i S_ij + k_i u_j
 //   o_j  = sum_i q_i S_ij
 // Token vectors are staged TB tokens at a time in shared memory so the inner
-// loop runs without barriers.
+// loop runs without barriers; optional input preparation (gate activations,
+// L2 norm of k) is applied while staging.
 #include "common.cuh"
 
 namespace kda {
@@ -23,7 +24,8 @@ namespace {
 
 constexpr int TB = 16;  // tokens staged per barrier
 
-template <int DK, int DV, typename TIn>
+// PREP: input preparation requested; without it that code is compiled out.
+template <int DK, int DV, typename TIn, bool PREP>
 __global__ void __launch_bounds__(DV)
 scan_fwd_kernel(FwdArgs a)
 {
@@ -32,6 +34,7 @@ scan_fwd_kernel(FwdArgs a)
     __shared__ __align__(16) float s_k[TB][DK];
     __shared__ __align__(16) float s_q[TB][DK];
     __shared__ __align__(16) float s_m[TB][DV];
+    __shared__ float s_ksc[TB];   // 1 / ||k_t|| (input preparation)
 
     const int n = blockIdx.x / a.H, h = blockIdx.x % a.H;
     const int j = threadIdx.x;
@@ -47,17 +50,23 @@ scan_fwd_kernel(FwdArgs a)
 #pragma unroll
     for (int i = 0; i < DK; ++i) S[i] = a.s0 ? a.s0[soff + (size_t)i * DV + j] : 0.f;
 
+    const bool logits = PREP && (a.prep & PREP_LOGITS), l2k = PREP && (a.prep & PREP_L2NORM_K), ext = a.ext != 0;
     for (int base = 0; base < len; base += TB) {
         const int nt = min(TB, len - base);
         __syncthreads();  // previous block of tokens fully consumed
         for (int e = j; e < nt * DK; e += DV) {
             const int tt = e / DK, i = e % DK;
             const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
-            const float kk = ld_f32(k + tok * DK + i), aa = ld_f32(al + tok * DK + i);
-            const float g = (a.variant == GDN2) ? ld_f32(g1 + tok * DK + i) : ld_f32(g1 + tok);
+            const float kk = ld_f32(k + tok * DK + i);
+            float aa = ld_f32(al + tok * DK + i);
+            float g = (a.variant == GDN2) ? ld_f32(g1 + tok * DK + i) : ld_f32(g1 + tok);
+            if (logits) {
+                aa = round_to<TIn>(prep_alpha(aa, ext));
+                g = round_to<TIn>(prep_gate(g, ext));
+            }
             s_k[tt][i] = kk;
             s_al[tt][i] = aa;
-            s_aa[tt][i] = aa * (g * kk);
+            s_aa[tt][i] = l2k ? aa * g : aa * (g * kk);   // times k once it is normalised
             s_q[tt][i] = ld_f32(q + tok * DK + i);
         }
         for (int e = j; e < nt * DV; e += DV) {
@@ -67,9 +76,25 @@ scan_fwd_kernel(FwdArgs a)
             if (a.variant == KDA) g = ld_f32(g1 + tok);
             else if (a.variant == RDA) g = ld_f32(g2 + tok);
             else g = ld_f32(g2 + tok * DV + jj);
+            if (logits) g = round_to<TIn>(prep_gate(g, ext));
             s_m[tt][jj] = g * ld_f32(v + tok * DV + jj);
         }
         __syncthreads();
+        if (l2k) {   // k_t / ||k_t||, then a~ = (alpha g) (.) k
+            for (int tt = j; tt < nt; tt += DV) {
+                float ss = 0.f;
+                for (int i = 0; i < DK; ++i) ss = fmaf(s_k[tt][i], s_k[tt][i], ss);
+                s_ksc[tt] = prep_kscale(ss);
+            }
+            __syncthreads();
+            for (int e = j; e < nt * DK; e += DV) {
+                const int tt = e / DK, i = e % DK;
+                const float kn = round_to<TIn>(s_k[tt][i] * s_ksc[tt]);
+                s_k[tt][i] = kn;
+                s_aa[tt][i] *= kn;
+            }
+            __syncthreads();
+        }
         for (int tt = 0; tt < nt; ++tt) {
             float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
@@ -111,8 +136,13 @@ cudaError_t launch_dims(const FwdArgs &a, bool bf16, cudaStream_t st)
 {
     const int N = a.cu_seqlens ? a.num_seqs : a.B;
     dim3 grid((unsigned)(N * a.H)), block(DV);
-    if (bf16) scan_fwd_kernel<DK, DV, __nv_bfloat16><<<grid, block, 0, st>>>(a);
-    else scan_fwd_kernel<DK, DV, float><<<grid, block, 0, st>>>(a);
+    if (bf16) {
+        if (a.prep) scan_fwd_kernel<DK, DV, __nv_bfloat16, true><<<grid, block, 0, st>>>(a);
+        else scan_fwd_kernel<DK, DV, __nv_bfloat16, false><<<grid, block, 0, st>>>(a);
+    } else {
+        if (a.prep) scan_fwd_kernel<DK, DV, float, true><<<grid, block, 0, st>>>(a);
+        else scan_fwd_kernel<DK, DV, float, false><<<grid, block, 0, st>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -18,6 +18,9 @@ Three independent formulations, all float64:
 * ``brute_force`` -- NumPy dense closed form of the unrolled recurrence,
   S_t = (prod_{s<=t} A_s) S_0 + sum_{s<=t} (prod_{s<r<=t} A_r) W_s, evaluated
   from scratch for every t.  Tiny inputs only.
+* ``prepare`` -- the optional input preparation (gate activations from
+  logits, L2 normalisation of k) in float64, applied before ``recurrence``
+  when a problem stores logits or raw keys.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against properties
 the pages fix (RDA = KDA when e = w; GDN-2 = RDA for constant vectors;
@@ -84,15 +87,64 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
+def _sigmoid(y: np.ndarray) -> np.ndarray:
+    # 1 / (1 + e^-y) without overflow for large |y|
+    e = np.exp(-np.abs(y))
+    return np.where(y >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def _round_to(x, dtype: Optional[str]):
+    if x is None or dtype is None:
+        return x
+    if dtype == "bf16":   # round to nearest even, as the input dtype stores it
+        import torch
+        return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).double().numpy()
+    if dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+def prepare(gate_range: str, k, alpha, g1, g2=None, logits: bool = False, l2norm_k: bool = False,
+            round_to: Optional[str] = None):
+    """Input preparation on request, float64, from the stored values.
+
+    ``logits``: alpha, g1, g2 hold logits.  Standard range: alpha =
+    exp(-softplus(x)) and every gate (beta, e, w, GDN-2's b and w) =
+    sigmoid(y); extended (Complex-KDA) range: alpha = tanh(x), gate =
+    2 sigmoid(y) -- the gates' ranges (0,1] / [-1,1] and [0,1] / [0,2].
+    ``l2norm_k``: k_t / max(||k_t||_2, 1e-6) along the last axis.
+    ``round_to`` ("bf16" / "f32"): the prepared values are rounded to the
+    input dtype, as a separate preparation pass would store them.
+    Returns (k, alpha, g1, g2) as float64 arrays (g2 may be None).
+    """
+    k, alpha, g1, g2 = (_f64(x) for x in (k, alpha, g1, g2))
+    if logits:
+        ext = gate_range == "extended"
+        alpha = np.tanh(alpha) if ext else np.exp(-np.logaddexp(0.0, alpha))
+        scale = 2.0 if ext else 1.0
+        g1 = scale * _sigmoid(g1)
+        g2 = None if g2 is None else scale * _sigmoid(g2)
+        alpha, g1, g2 = (_round_to(x, round_to) for x in (alpha, g1, g2))
+    if l2norm_k:
+        norm = np.sqrt(np.sum(k * k, axis=-1, keepdims=True))
+        k = _round_to(k / np.maximum(norm, 1e-6), round_to)
+    return k, alpha, g1, g2
+
+
 def recurrence_arrays(variant: str, q, k, v, alpha, g1, g2=None, cu_seqlens=None,
-                      initial_state=None, threads: int = 0):
+                      initial_state=None, threads: int = 0, gate_range: str = "standard",
+                      logits: bool = False, l2norm_k: bool = False, round_to: Optional[str] = None):
     """Step recurrence on float64 arrays with the library's layouts.
 
     q,k,alpha [B,T,H,dk]; v [B,T,H,dv]; g1/g2 per the variant; cu_seqlens
     optional int offsets (B must be 1); initial_state [N,H,dk,dv] or None.
-    Returns (o [B,T,H,dv], final_state [N,H,dk,dv]) as float64.
+    ``logits`` / ``l2norm_k`` run ``prepare`` first (``gate_range`` picks the
+    activations, ``round_to`` the stored dtype of the prepared values).
+    Returns (o [B,T,H,dv], final_state [N,H,dk,dv]) float64.
     """
     q, k, v, alpha, g1, g2 = (_f64(x) for x in (q, k, v, alpha, g1, g2))
+    if logits or l2norm_k:
+        k, alpha, g1, g2 = prepare(gate_range, k, alpha, g1, g2, logits, l2norm_k, round_to)
     s0 = _f64(initial_state)
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -122,9 +174,11 @@ def recurrence(inp, seqs: Optional[Sequence[int]] = None, heads: Optional[Sequen
     and final_state [N,H,dk,dv]; with one, o is a dict {(n, h): [len, dv]} and
     final_state a dict {(n, h): [dk, dv]}.
     """
+    pk = dict(gate_range=inp.gate_range, logits=getattr(inp, "logits", False),
+              l2norm_k=getattr(inp, "l2norm_k", False), round_to=inp.dtype)
     if seqs is None and heads is None:
         return recurrence_arrays(inp.variant, inp.q, inp.k, inp.v, inp.alpha, inp.g1, inp.g2,
-                                 inp.cu_seqlens, inp.initial_state, threads)
+                                 inp.cu_seqlens, inp.initial_state, threads, **pk)
     seqs = list(range(inp.num_seqs)) if seqs is None else list(seqs)
     heads = list(range(inp.H)) if heads is None else list(heads)
     # gather every requested (sequence, head) as its own batch row, padded to the
@@ -155,7 +209,7 @@ def recurrence(inp, seqs: Optional[Sequence[int]] = None, heads: Optional[Sequen
         s0 = np.stack([inp.initial_state[n, h].double().numpy() for (n, h, *_r) in parts])[:, None]
     o, sf = recurrence_arrays(inp.variant, gather(inp.q, dk), gather(inp.k, dk), gather(inp.v, dv),
                               gather(inp.alpha, dk), gather(inp.g1, g_last1), gather(inp.g2, g_last2),
-                              cu, s0, threads)
+                              cu, s0, threads, **pk)
     o_d, s_d = {}, {}
     for i, (n, h, *_r) in enumerate(parts):
         o_d[(n, h)] = o[0, cu[i]:cu[i + 1], 0]

@@ -269,3 +269,87 @@ def test_tiny_ckda_inputs_match_recipe():
     assert float(inp.alpha.min()) >= -1 and float(inp.alpha.max()) <= 1 and float(inp.alpha.min()) < 0
     assert float(inp.g1.min()) >= 0 and float(inp.g1.max()) <= 2 and float(inp.g1.max()) > 1
     np.testing.assert_allclose(inp.k.double().norm(dim=-1).numpy(), 1.0, atol=1e-6)
+
+
+# ---- input preparation (gate logits, L2-normalised k) -------------------------------------
+
+def test_prepare_at_zero_logits():
+    """sigmoid(0) = 1/2, exp(-softplus(0)) = 1/2, tanh(0) = 0: the activations' fixed values."""
+    z = np.zeros((1, 1, 1, 4))
+    zs = np.zeros((1, 1, 1))
+    _, a, g1, g2 = oracle.prepare("standard", z + 1.0, z, zs, zs, logits=True)
+    assert np.allclose(a, 0.5) and np.allclose(g1, 0.5) and np.allclose(g2, 0.5)
+    _, a, g1, g2 = oracle.prepare("extended", z + 1.0, z, zs, zs, logits=True)
+    assert np.allclose(a, 0.0) and np.allclose(g1, 1.0) and np.allclose(g2, 1.0)
+
+
+def test_prepare_inverts_the_activations():
+    """Logits written with the inverse functions come back as the gates they encode."""
+    rng = np.random.default_rng(11)
+    a = rng.uniform(0.01, 0.99, (2, 5, 3, 8))
+    g = rng.uniform(0.01, 0.99, (2, 5, 3))
+    x = np.log((1.0 - a) / a)                  # exp(-softplus(x)) = 1 / (1 + e^x) = a
+    y = np.log(g / (1.0 - g))                  # sigmoid(y) = g
+    k = rng.standard_normal((2, 5, 3, 8))
+    _, a2, g2, _ = oracle.prepare("standard", k, x, y, None, logits=True)
+    assert np.allclose(a2, a, rtol=1e-12, atol=1e-14) and np.allclose(g2, g, rtol=1e-12, atol=1e-14)
+    ae = rng.uniform(-0.99, 0.99, (2, 5, 3, 8))
+    ge = rng.uniform(0.02, 1.98, (2, 5, 3))
+    _, a3, g3, _ = oracle.prepare("extended", k, np.arctanh(ae), np.log((ge / 2) / (1 - ge / 2)), None,
+                                  logits=True)
+    assert np.allclose(a3, ae, rtol=1e-12, atol=1e-14) and np.allclose(g3, ge, rtol=1e-12, atol=1e-14)
+    # GDN-2 vectors take the gate activation elementwise
+    b = rng.uniform(0.01, 0.99, (2, 5, 3, 8))
+    _, _, b2, w2 = oracle.prepare("standard", k, x, np.log(b / (1 - b)), np.log(b / (1 - b)), logits=True)
+    assert np.allclose(b2, b, rtol=1e-12) and np.allclose(w2, b, rtol=1e-12)
+
+
+def test_prepare_saturates_without_overflow():
+    big = np.array([[[[800.0, -800.0]]]])
+    with np.errstate(over="raise", invalid="raise", divide="raise"):
+        _, a, g, _ = oracle.prepare("standard", big, big, big[..., 0], None, logits=True)
+    assert a[0, 0, 0, 0] == 0.0 and a[0, 0, 0, 1] == 1.0 and g[0, 0, 0] == 1.0
+
+
+def test_prepare_l2_normalises_k():
+    rng = np.random.default_rng(12)
+    k = rng.standard_normal((2, 7, 3, 16)) * 5.0
+    k[0, 0, 0] = 0.0                                       # a zero key stays zero (norm floor)
+    kn, a, g1, _ = oracle.prepare("standard", k, np.ones((2, 7, 3, 16)), np.ones((2, 7, 3)), l2norm_k=True)
+    n = np.linalg.norm(kn, axis=-1)
+    assert np.allclose(n[n > 0], 1.0, rtol=1e-13) and n[0, 0, 0] == 0.0
+    assert np.allclose(np.sum(kn * k, axis=-1), np.linalg.norm(k, axis=-1), rtol=1e-12)   # same direction
+    assert np.array_equal(a, np.ones((2, 7, 3, 16))) and np.array_equal(g1, np.ones((2, 7, 3)))  # untouched
+
+
+@pytest.mark.parametrize("variant,gate_range", [("kda", "standard"), ("kda", "extended"), ("rda", "extended"),
+                                                ("gdn2", "standard")])
+def test_recurrence_with_preparation_equals_prepared_inputs(variant, gate_range):
+    """The oracle's prepared path is the recurrence on the activated, normalised inputs."""
+    inp = make_chunk_inputs(variant, gate_range, "f32", B=2, T=23, H=2, d_k=8, d_v=4, seed=5,
+                              logits=True, raw_k=True, init_state="random", init_std=0.3)
+    o1, s1 = oracle.recurrence(inp)
+    k, a, g1, g2 = oracle.prepare(gate_range, inp.k, inp.alpha, inp.g1, inp.g2, logits=True, l2norm_k=True,
+                                  round_to=inp.dtype)
+    o2, s2 = oracle.recurrence_arrays(variant, inp.q, k, inp.v, a, g1, g2, None, inp.initial_state)
+    assert np.array_equal(o1, o2) and np.array_equal(s1, s2)
+    # and the raw inputs give a different answer (the preparation is not a no-op)
+    o3, _ = oracle.recurrence_arrays(variant, inp.q, inp.k, inp.v, inp.alpha, inp.g1, inp.g2, None,
+                                     inp.initial_state)
+    assert not np.allclose(o1, o3)
+
+
+def test_prepare_rounds_to_the_input_dtype():
+    """Rounded preparation: bf16-representable values within half a bf16 ulp of the exact ones."""
+    rng = np.random.default_rng(13)
+    k = rng.standard_normal((1, 9, 2, 16)) * 3
+    x = rng.standard_normal((1, 9, 2, 16)) * 2
+    y = rng.standard_normal((1, 9, 2))
+    ex = oracle.prepare("standard", k, x, y, None, logits=True, l2norm_k=True)
+    rd = oracle.prepare("standard", k, x, y, None, logits=True, l2norm_k=True, round_to="bf16")
+    for e, r in zip(ex[:3], rd[:3]):
+        back = torch.from_numpy(r).to(torch.bfloat16).double().numpy()
+        assert np.array_equal(back, r)                                   # representable in bf16
+        assert np.all(np.abs(r - e) <= np.abs(e) * 2.0 ** -8 + 1e-300)  # RNE: half an ulp (8 bits)
+    f = oracle.prepare("extended", k, x, y, None, logits=True, round_to="f32")
+    assert np.array_equal(f[1], f[1].astype(np.float32).astype(np.float64))

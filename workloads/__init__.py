@@ -68,6 +68,8 @@ class ChunkInputs:
     cu_seqlens: Optional[torch.Tensor]
     initial_state: Optional[torch.Tensor]
     chunk_size: int = 64
+    logits: bool = False     # alpha and gates are stored as logits (KDA_FLAG_GATE_LOGITS)
+    l2norm_k: bool = False   # k is stored unnormalised (KDA_FLAG_L2NORM_K)
 
     @property
     def num_seqs(self) -> int:
@@ -103,9 +105,25 @@ def _cast(x: Optional[np.ndarray], dtype: str) -> Optional[torch.Tensor]:
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(DTYPES[dtype])
 
 
-def _alpha_gates(rng, variant, gate_range, lead, d_k, d_v, uniform_tiny=False):
-    """Draw alpha and the variant's gates for leading shape ``lead``."""
+def _alpha_gates(rng, variant, gate_range, lead, d_k, d_v, uniform_tiny=False, logits=False):
+    """Draw alpha and the variant's gates for leading shape ``lead``.  With
+    ``logits`` the same draws are returned as logits (alpha's logit x with
+    alpha = exp(-softplus(x)), or tanh(x) for the extended range; gate logits
+    y with gate = sigmoid(y), or 2 sigmoid(y) extended)."""
     a_pre = rng.standard_normal(lead + (d_k,), dtype=np.float32)
+    if logits:
+        if uniform_tiny:
+            raise ValueError("uniform_tiny draws have no logits")
+        ext = gate_range == "extended"
+        x = (2.0 * a_pre if ext else a_pre).astype(np.float32)
+        if variant == "kda":
+            return x, rng.standard_normal(lead, dtype=np.float32), None
+        if variant == "rda":
+            return x, rng.standard_normal(lead, dtype=np.float32), rng.standard_normal(lead, dtype=np.float32)
+        if variant == "gdn2":
+            return (x, rng.standard_normal(lead + (d_k,), dtype=np.float32),
+                    rng.standard_normal(lead + (d_v,), dtype=np.float32))
+        raise ValueError(f"unknown variant {variant!r}")
     if uniform_tiny:
         alpha = rng.uniform(-1.0, 1.0, lead + (d_k,)).astype(np.float32)
         g1 = rng.uniform(0.0, 2.0, lead).astype(np.float32)
@@ -136,13 +154,15 @@ def make_chunk_inputs(variant: str = "kda", gate_range: str = "standard", dtype:
                       B: int = 1, T: int = 64, H: int = 2, d_k: int = 16, d_v: int = 16,
                       seed: int = 0, chunk_size: int = 64, doc_lens=None,
                       init_state: str = "zero", init_std: float = 0.02,
-                      uniform_tiny: bool = False) -> ChunkInputs:
+                      uniform_tiny: bool = False, logits: bool = False, raw_k: bool = False) -> ChunkInputs:
     """Draw one chunked-forward problem.
 
     ``doc_lens`` packs documents of those lengths along T (B must be 1) and
     returns the matching ``cu_seqlens`` (int32, exclusive prefix sum).
     ``init_state`` is "zero" (None is passed, the library starts from 0) or
-    "random" (fp32 N(0, init_std) per sequence and head).
+    "random" (fp32 N(0, init_std) per sequence and head).  ``logits`` stores
+    alpha and the gates as logits, ``raw_k`` stores k unnormalised (the
+    library's input preparation turns them into the recurrence's inputs).
     """
     rng = np.random.default_rng(seed)
     cu = None
@@ -154,8 +174,9 @@ def make_chunk_inputs(variant: str = "kda", gate_range: str = "standard", dtype:
     q = rng.standard_normal(lead + (d_k,), dtype=np.float32)
     k = rng.standard_normal(lead + (d_k,), dtype=np.float32)
     v = rng.standard_normal(lead + (d_v,), dtype=np.float32)
-    alpha, g1, g2 = _alpha_gates(rng, variant, gate_range, lead, d_k, d_v, uniform_tiny)
-    k = _l2norm_rows(k)
+    alpha, g1, g2 = _alpha_gates(rng, variant, gate_range, lead, d_k, d_v, uniform_tiny, logits)
+    if not raw_k:
+        k = _l2norm_rows(k)
     n_seqs = B if cu is None else len(doc_lens)
     s0 = None
     if init_state == "random":
@@ -165,7 +186,7 @@ def make_chunk_inputs(variant: str = "kda", gate_range: str = "standard", dtype:
         raise ValueError(init_state)
     return ChunkInputs(variant, gate_range, dtype, B, T, H, d_k, d_v,
                        _cast(q, dtype), _cast(k, dtype), _cast(v, dtype), _cast(alpha, dtype),
-                       _cast(g1, dtype), _cast(g2, dtype), cu, s0, chunk_size)
+                       _cast(g1, dtype), _cast(g2, dtype), cu, s0, chunk_size, logits, raw_k)
 
 
 # ---------------------------------------------------------------------------
@@ -222,6 +243,8 @@ class DecodeInputs:
     alpha: torch.Tensor
     g1: torch.Tensor
     g2: Optional[torch.Tensor]
+    logits: bool = False
+    l2norm_k: bool = False
 
     def tensors(self):
         return [t for t in (self.q, self.k, self.v, self.alpha, self.g1, self.g2) if t is not None]
@@ -239,7 +262,7 @@ def decode_initial_state(N: int = 256, H: int = 32, d_k: int = 128, d_v: int = 1
 
 def decode_step_inputs(step: int, variant: str = "kda", gate_range: str = "extended",
                        dtype: str = "bf16", N: int = 256, H: int = 32, d_k: int = 128,
-                       d_v: int = 128, seed: int = 0) -> DecodeInputs:
+                       d_v: int = 128, seed: int = 0, logits: bool = False, raw_k: bool = False) -> DecodeInputs:
     """Per-step decode inputs from ``default_rng((seed, step))`` so any step can be
     regenerated independently (Complex KDA range by default)."""
     rng = np.random.default_rng((seed, step))
@@ -247,7 +270,8 @@ def decode_step_inputs(step: int, variant: str = "kda", gate_range: str = "exten
     q = rng.standard_normal(lead + (d_k,), dtype=np.float32)
     k = rng.standard_normal(lead + (d_k,), dtype=np.float32)
     v = rng.standard_normal(lead + (d_v,), dtype=np.float32)
-    alpha, g1, g2 = _alpha_gates(rng, variant, gate_range, lead, d_k, d_v)
-    k = _l2norm_rows(k)
+    alpha, g1, g2 = _alpha_gates(rng, variant, gate_range, lead, d_k, d_v, logits=logits)
+    if not raw_k:
+        k = _l2norm_rows(k)
     return DecodeInputs(variant, gate_range, dtype, N, H, d_k, d_v, _cast(q, dtype), _cast(k, dtype),
-                        _cast(v, dtype), _cast(alpha, dtype), _cast(g1, dtype), _cast(g2, dtype))
+                        _cast(v, dtype), _cast(alpha, dtype), _cast(g1, dtype), _cast(g2, dtype), logits, raw_k)
