@@ -255,7 +255,7 @@ def chunk_form(inp, flags=0) -> str:
     return "split" if ws else "fused"
 
 
-def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True, flags=0):
+def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True, flags=0, states=False):
     import linear_rnn_delta_b200 as kda
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
@@ -266,11 +266,15 @@ def run_chunk_workload(inp, steps, warmup, world, peaks, sampler=None, e2e=True,
     N = inp.num_seqs
     o = torch.empty((inp.B, inp.T, inp.H, inp.d_v), dtype=d["q"].dtype, device=dev)
     sf = torch.empty((N, inp.H, inp.d_k, inp.d_v), dtype=torch.float32, device=dev)
+    cs = None
+    if states:   # state snapshots after every 64 tokens
+        cs = torch.empty((kda.num_chunk_slots(inp.B, inp.T, N), inp.H, inp.d_k, inp.d_v), dtype=torch.float32,
+                         device=dev)
 
     def step():
         kda.kda_chunk_fwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"],
                           cu_seqlens=cu, initial_state=s0, final_state=sf, o=o, chunk_size=inp.chunk_size,
-                          flags=flags, stream=stream)
+                          flags=flags, stream=stream, chunk_states=cs)
 
     if sampler:
         sampler.start()
@@ -471,10 +475,12 @@ def main():
                 ("RDA varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("rda", rank), 0),
                 ("GDN-2 varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("gdn2", rank), 0),
                 ("KDA B=4 H=16 T=4096 bf16 from gate logits and raw keys (in-kernel activations, L2 norm)",
-                 prep, 16 | 32)):
+                 prep, 16 | 32),
+                ("KDA B=4 H=16 T=4096 bf16 with fp32 state snapshots after every 64 tokens",
+                 lambda: W.kda_bf16(seed=rank_workload_seed(rank)), "states")):
             x = mk()
             r = run_chunk_workload(x, max(5, args.steps // 2), args.warmup, world, peaks, e2e=False,
-                                   flags=fflags | xflags)
+                                   flags=fflags | (xflags if xflags != "states" else 0), states=xflags == "states")
             also.append({"workload": name, "value": r["tokens_per_step"] * world * max(5, args.steps // 2) / r["total_s"],
                          "unit": UNIT, "ms_per_step": r["avg_launch_s"] * 1e3, "form": r["form"],
                          "hbm_frac": r["hbm"]["frac"],

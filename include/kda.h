@@ -151,13 +151,24 @@ size_t kda_chunk_fwd_workspace_size(int dtype, int B, int T, int H, int d_k, int
  * workspace holds at least kda_chunk_fwd_workspace_size(...) bytes;
  * otherwise the fused form runs (KDA_FLAG_FORCE_SPLIT with a NULL or short
  * workspace is KDA_ERR_INVALID_ARG).  Nothing is allocated.
+ *
+ * chunk_states (optional, NULL = none): fp32 [num_slots][H][d_k][d_v] with
+ * num_slots = N + ceil(B*T / 64), receives the state after every 64 tokens
+ * of each sequence and after its last token, for prefix caching ("state
+ * snapshots", openarchlab page on GDN/KDA state updates, sec. 3): the state
+ * after chunk c (tokens [64c, min(64c+64, len))) of sequence n goes to slot
+ * n + floor(R_n / 64) + c, R_n its first token's row in the packed [B*T]
+ * token order (cu[n], or n*T without cu_seqlens).  Slots that belong to no
+ * chunk are not written.  Every path writes them (fused, split, scan); the
+ * last chunk's entry equals final_state.  Appending tokens to a cached
+ * prefix is a forward call with initial_state = that entry.
  */
 int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
                      int B, int T, int H, int d_k, int d_v,
                      const void *q, const void *k, const void *v, const void *alpha,
                      const void *g1, const void *g2,
                      const int32_t *cu_seqlens, int num_seqs,
-                     const float *initial_state, float *final_state,
+                     const float *initial_state, float *final_state, float *chunk_states,
                      void *o, int chunk_size, void *workspace, size_t workspace_bytes,
                      unsigned flags, void *stream);
 

@@ -19,7 +19,7 @@ import torch
 
 __all__ = ["kda_chunk_fwd", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_version",
            "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_FORCE_SCAN", "FLAG_FORCE_FUSED",
-           "FLAG_FORCE_SPLIT", "FLAG_GATE_LOGITS", "FLAG_L2NORM_K"]
+           "FLAG_FORCE_SPLIT", "FLAG_GATE_LOGITS", "FLAG_L2NORM_K", "num_chunk_slots", "chunk_slot"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
@@ -49,7 +49,7 @@ def _load():
     lib.kda_chunk_fwd.restype = _i
     lib.kda_chunk_fwd.argtypes = [_i] * 8 + [_vp] * 6 + [_vp, _i, _vp, _vp, _vp, _i, ctypes.c_uint, _vp]
     lib.kda_chunk_fwd_ws.restype = _i
-    lib.kda_chunk_fwd_ws.argtypes = ([_i] * 8 + [_vp] * 6 + [_vp, _i, _vp, _vp, _vp, _i, _vp, ctypes.c_size_t,
+    lib.kda_chunk_fwd_ws.argtypes = ([_i] * 8 + [_vp] * 6 + [_vp, _i, _vp, _vp, _vp, _vp, _i, _vp, ctypes.c_size_t,
                                                             ctypes.c_uint, _vp])
     lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_fwd_workspace_size.argtypes = [_i] * 9 + [ctypes.c_uint]
@@ -119,7 +119,8 @@ def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torc
                   v: torch.Tensor, alpha: torch.Tensor, g1: torch.Tensor, g2: Optional[torch.Tensor] = None,
                   cu_seqlens: Optional[torch.Tensor] = None, initial_state: Optional[torch.Tensor] = None,
                   final_state: Union[torch.Tensor, bool, None] = True, o: Optional[torch.Tensor] = None,
-                  chunk_size: int = 64, flags: int = 0, stream=None):
+                  chunk_size: int = 64, flags: int = 0, stream=None,
+                  chunk_states: Union[torch.Tensor, bool, None] = None):
     """Chunked forward of the recurrence over whole sequences (C: kda_chunk_fwd_ws,
     with the split form's workspace taken from torch's caching allocator).
 
@@ -127,7 +128,10 @@ def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torc
     [B,T,H], g2 None; RDA: e, w [B,T,H]; GDN-2: b [B,T,H,d_k], w [B,T,H,d_v]);
     cu_seqlens int32 [N+1] (B == 1) or None; initial_state fp32 [N,H,d_k,d_v]
     or None.  ``final_state`` True allocates it, a tensor is written in place,
-    None/False skips it.  Returns (o, final_state or None).
+    None/False skips it.  ``chunk_states`` (True allocates fp32
+    [num_chunk_slots(B, T, N), H, d_k, d_v]) receives the state after every 64
+    tokens of each sequence and after its last token, at ``chunk_slot``.
+    Returns (o, final_state or None), plus chunk_states when requested.
     """
     var = _code(VARIANTS, variant, "variant")
     rng = _code(RANGES, gate_range, "gate_range")
@@ -167,6 +171,12 @@ def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torc
     if o is None:
         o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
     _check(o, "o", dt, (B, T, H, dv), dev)
+    want_states = chunk_states is not None and chunk_states is not False
+    if chunk_states is True:
+        chunk_states = torch.empty((num_chunk_slots(B, T, N), H, dk, dv), dtype=torch.float32, device=dev)
+    elif chunk_states is False:
+        chunk_states = None
+    _check(chunk_states, "chunk_states", torch.float32, (num_chunk_slots(B, T, N), H, dk, dv), dev)
     # workspace of the split form, from torch's caching allocator (no per-call device allocation)
     ws_bytes = lib.kda_chunk_fwd_workspace_size(_DTYPES[dt], B, T, H, dk, dv, int(cu_seqlens is not None), N,
                                                 int(chunk_size), int(flags))
@@ -177,11 +187,24 @@ def kda_chunk_fwd(variant: Union[str, int], gate_range: Union[str, int], q: torc
             ws.record_stream(stream)
     rc = lib.kda_chunk_fwd_ws(var, rng, _DTYPES[dt], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
                               _ptr(g1), _ptr(g2), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(final_state),
-                              _ptr(o), int(chunk_size), _ptr(ws), ws_bytes if ws is not None else 0, int(flags),
-                              _stream(stream, dev))
+                              _ptr(chunk_states), _ptr(o), int(chunk_size), _ptr(ws),
+                              ws_bytes if ws is not None else 0, int(flags), _stream(stream, dev))
     if rc != 0:
         raise KdaError(rc, "kda_chunk_fwd")
+    if want_states:
+        return o, final_state, chunk_states
     return o, final_state
+
+
+def num_chunk_slots(B: int, T: int, N: int) -> int:
+    """Chunk slots of a [B, T] token layout with N sequences: N + ceil(B*T / 64)."""
+    return N + (B * T + 63) // 64
+
+
+def chunk_slot(n: int, c: int, row0: int) -> int:
+    """Slot of chunk c (tokens [64c, 64c+64)) of sequence n whose first token
+    is row ``row0`` of the packed token order (cu_seqlens[n], or n*T)."""
+    return n + row0 // 64 + c
 
 
 def kda_decode_step(variant: Union[str, int], gate_range: Union[str, int], q: torch.Tensor, k: torch.Tensor,

@@ -132,12 +132,6 @@ constexpr uint32_t SLOT_BYTES = 82944;
 constexpr int META_FAST = 1;          // status word bits
 constexpr int META_OK = 2;
 
-__device__ __forceinline__ int seq_row0(const FwdArgs &a, int n) { return a.cu_seqlens ? a.cu_seqlens[n] : n * a.T; }
-__device__ __forceinline__ int seq_len(const FwdArgs &a, int n)
-{
-    return a.cu_seqlens ? a.cu_seqlens[n + 1] - a.cu_seqlens[n] : a.T;
-}
-__device__ __forceinline__ int slot_base(const FwdArgs &a, int n) { return n + seq_row0(a, n) / C; }
 
 // One chunk of work for the preparation role.
 struct Item {
@@ -284,6 +278,23 @@ __device__ __forceinline__ void step6_mmas(uint32_t tbase, uint32_t s0t, uint32_
     mma_bf16(tbase + TM_O, dK(s0t, 16384, 0), dK(qa + 8192, 16384, 0), id64, 0);
 #pragma unroll
     for (int kk = 1; kk < 8; ++kk) mma_bf16(tbase + TM_U, dK(s0t, 16384, kk), dK(qa, 16384, kk), id128, 1);
+}
+
+// State snapshot after a chunk: S^T (TMEM lane j = value column j, fp32) ->
+// snap[slot][h][i][j] for the key channels of 32-column blocks c32 in
+// [c32a, c32a + n32); for a fixed i a warp writes 128 contiguous bytes.
+__device__ __forceinline__ void snapshot_state(const FwdArgs &a, uint32_t tlane, int slot, int h, int c32a, int n32,
+                                               int jcol)
+{
+    float *dst = a.snap + ((size_t)slot * a.H + h) * D * D + jcol;
+#pragma unroll 1
+    for (int c32 = c32a; c32 < c32a + n32; ++c32) {
+        float s[32];
+        tmem_ld32(tlane + TM_S + c32 * 32, s);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) dst[(size_t)(c32 * 32 + e) * D] = s[e];
+    }
 }
 
 // Fast path, step 1b for the item (tg, cq): one forward sweep over the item's
@@ -637,6 +648,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             }
             if (!mbar_wait_cycles(bar_s7, par, WAIT_CYCLES)) ok = false;
             tc_fence_after();
+            if (a.snap) snapshot_state(a, tbase + lane_base, slot_base(a, n) + ch, h, 0, 4, jcol);
             // ---- o: TMEM (lane j, column r) -> bf16 staging [r][j] in the U^T slot -> HBM
             unsigned short *ost = reinterpret_cast<unsigned short *>(sm + OFF_UT);
 #pragma unroll
@@ -1521,6 +1533,7 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
         if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
         ph_mma ^= 1;
         tc_fence_after();
+        if (a.snap) snapshot_state(a, tbase + lane_base, sbase + ch, h, half * 2, 2, jcol);
         // every read of this buffer is done: load chunk ch + 2 into it
         if (tid == 0 && ok && ch + 2 < nchunks) issue_load(ch + 2, buf);
         stage_o();   // the U^T tile is free: the step-7 GEMMs are done

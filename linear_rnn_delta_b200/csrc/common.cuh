@@ -27,7 +27,19 @@ struct FwdArgs {
     void *o;
     unsigned prep = 0;   // PREP_* bits: input preparation done by the kernels
     int ext = 0;         // extended (Complex KDA) gate range: selects the activations
+    float *snap = nullptr;   // optional: state after every 64 tokens, [slot][H][dk][dv] (chunk slots)
 };
+
+// Chunk slot of chunk c (64 tokens) of sequence n whose first token is global
+// row R_n: n + floor(R_n / 64) + c -- unique, increasing within a sequence and
+// below N + ceil(rows / 64).  Workspace slots and state snapshots use it.
+constexpr int SLOT_TOKENS = 64;
+__device__ __forceinline__ int seq_row0(const FwdArgs &a, int n) { return a.cu_seqlens ? a.cu_seqlens[n] : n * a.T; }
+__device__ __forceinline__ int seq_len(const FwdArgs &a, int n)
+{
+    return a.cu_seqlens ? a.cu_seqlens[n + 1] - a.cu_seqlens[n] : a.T;
+}
+__device__ __forceinline__ int slot_base(const FwdArgs &a, int n) { return n + seq_row0(a, n) / SLOT_TOKENS; }
 
 // ---- input preparation (optional, applied once where the kernels read their inputs) ----
 // PREP_LOGITS: alpha and the gates arrive as logits.  Standard range:

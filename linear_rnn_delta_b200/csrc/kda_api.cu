@@ -169,7 +169,7 @@ extern "C" int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
                                 const void *q, const void *k, const void *v, const void *alpha,
                                 const void *g1, const void *g2,
                                 const int32_t *cu_seqlens, int num_seqs,
-                                const float *initial_state, float *final_state,
+                                const float *initial_state, float *final_state, float *chunk_states,
                                 void *o, int chunk_size, void *workspace, size_t workspace_bytes,
                                 unsigned flags, void *stream)
 {
@@ -177,6 +177,9 @@ extern "C" int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
     int rc = chunk_args(a, variant, gate_range, dtype, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens,
                         num_seqs, initial_state, final_state, o, chunk_size, flags);
     if (rc != KDA_OK) return rc;
+    if (chunk_states && !aligned16(chunk_states))
+        return fail(KDA_ERR_INVALID_ARG, "chunk_states is not 16-byte aligned");
+    a.snap = chunk_states;
     if (workspace && !aligned16(workspace)) return fail(KDA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
     if ((flags & KDA_FLAG_FORCE_SPLIT) && tensor_core_path(a, dtype, chunk_size, flags)) {
         size_t need = 0;

@@ -123,6 +123,12 @@ scan_fwd_kernel(FwdArgs a)
             }
             const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
             st_out((TIn *)a.o + tok * DV + j, (o0 + o1) + (o2 + o3));
+            const int t = base + tt;   // token index within the sequence
+            if (a.snap && ((t + 1) % SLOT_TOKENS == 0 || t + 1 == len)) {   // state after a 64-token chunk
+                float *dst = a.snap + ((size_t)(slot_base(a, n) + t / SLOT_TOKENS) * a.H + h) * DK * DV + j;
+#pragma unroll
+                for (int i = 0; i < DK; ++i) dst[(size_t)i * DV] = S[i];
+            }
         }
     }
     if (a.sf) {

@@ -291,3 +291,26 @@ def brute_force(variant: str, q, k, v, alpha, g1, g2=None, initial_state=None):
                 if t == T - 1:
                     sf[b, h] = St
     return o, sf
+
+
+def chunk_states(inp, every: int = 64, threads: int = 0):
+    """State after every ``every`` tokens of each sequence and after its last
+    token, by running the step recurrence piece by piece from the previous
+    piece's final state (continuation is exact).  Returns a dict
+    {(n, c): [H, dk, dv] float64} for chunk c of sequence n.
+    """
+    names = ("q", "k", "v", "alpha", "g1", "g2")
+    out = {}
+    for n in range(inp.num_seqs):
+        b, t0, ln = inp.seq_bounds(n)
+        s = None if inp.initial_state is None else inp.initial_state[n:n + 1]
+        for c in range((ln + every - 1) // every):
+            a, e = t0 + c * every, t0 + min(ln, (c + 1) * every)
+            piece = {nm: (None if getattr(inp, nm) is None else getattr(inp, nm)[b:b + 1, a:e]) for nm in names}
+            _, sf = recurrence_arrays(inp.variant, piece["q"], piece["k"], piece["v"], piece["alpha"],
+                                      piece["g1"], piece["g2"], None, s, threads, gate_range=inp.gate_range,
+                                      logits=getattr(inp, "logits", False), l2norm_k=getattr(inp, "l2norm_k", False),
+                                      round_to=inp.dtype)
+            out[(n, c)] = sf[0]
+            s = sf
+    return out

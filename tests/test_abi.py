@@ -72,7 +72,8 @@ def fwd_ws(lib, ws=None, ws_bytes=0, **kw):
     a.update(kw)
     return lib.kda_chunk_fwd_ws(a["variant"], a["gate_range"], a["dtype"], a["B"], a["T"], a["H"], a["dk"],
                                 a["dv"], a["q"], a["k"], a["v"], a["alpha"], a["g1"], a["g2"], a["cu"], a["nseq"],
-                                a["s0"], a["sf"], a["o"], a["chunk"], ws, ws_bytes, a["flags"], a["stream"])
+                                a["s0"], a["sf"], a.get("cs"), a["o"], a["chunk"], ws, ws_bytes, a["flags"],
+                                a["stream"])
 
 
 SLOT_BYTES = 82944
@@ -107,6 +108,7 @@ def test_forced_split_needs_a_workspace(lib):
     assert fwd_ws(lib, ws=BAD, ws_bytes=need, flags=8) == INVALID     # misaligned
     assert fwd_ws(lib, ws=P, ws_bytes=need, flags=4 | 8) == INVALID   # both forms forced
     assert fwd_ws(lib, flags=1 << 9) == INVALID
+    assert fwd_ws(lib, cs=BAD) == INVALID                            # misaligned chunk_states
 
 
 def dec(lib, **kw):

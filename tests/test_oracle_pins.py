@@ -353,3 +353,23 @@ def test_prepare_rounds_to_the_input_dtype():
         assert np.all(np.abs(r - e) <= np.abs(e) * 2.0 ** -8 + 1e-300)  # RNE: half an ulp (8 bits)
     f = oracle.prepare("extended", k, x, y, None, logits=True, round_to="f32")
     assert np.array_equal(f[1], f[1].astype(np.float32).astype(np.float64))
+
+
+def test_chunk_states_are_prefix_runs():
+    """The oracle's state after chunk c is the final state of a run over the first 64(c+1) tokens."""
+    inp = make_chunk_inputs("gdn2", "extended", "f32", H=2, d_k=8, d_v=4, seed=31, doc_lens=[150, 64, 0, 9],
+                            init_state="random", init_std=0.3)
+    cs = oracle.chunk_states(inp)
+    assert sorted(cs) == [(0, 0), (0, 1), (0, 2), (1, 0), (3, 0)]
+    _, s_full = oracle.recurrence(inp)
+    for n, c in cs:
+        b, t0, ln = inp.seq_bounds(n)
+        e = min(ln, 64 * (c + 1))
+        cut = make_chunk_inputs("gdn2", "extended", "f32", H=2, d_k=8, d_v=4, seed=31, doc_lens=[150, 64, 0, 9],
+                                init_state="random", init_std=0.3)
+        _, sp = oracle.recurrence_arrays("gdn2", cut.q[:, t0:t0 + e], cut.k[:, t0:t0 + e], cut.v[:, t0:t0 + e],
+                                         cut.alpha[:, t0:t0 + e], cut.g1[:, t0:t0 + e], cut.g2[:, t0:t0 + e],
+                                         None, cut.initial_state[n:n + 1])
+        assert np.allclose(cs[(n, c)], sp[0], rtol=1e-12, atol=1e-14)
+        if 64 * (c + 1) >= ln:                       # the last chunk's state is the final state
+            assert np.allclose(cs[(n, c)], s_full[n], rtol=1e-12, atol=1e-14)
