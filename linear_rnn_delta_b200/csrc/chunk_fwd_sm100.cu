@@ -44,9 +44,11 @@
 //   3. T = (I + A)^{-1}: 16x16 diagonal blocks, then two recursive-doubling merges
 //   4. tcgen05: W = T (row operand a~ part);  U^T = M^T T^T
 //   5. state pass: S^T *= Gamma_C in TMEM and its bf16 copy (scaled or not)
-//   6. tcgen05: U^T -= S^T W^T;  O^T = S^T Q^T
+//   6. tcgen05: U^T -= S^T W^T;  O^T = S^T Q^T  (one N = 128 GEMM over [-W; Q'])
 //   7. tcgen05: O^T += U^T P^T;  S^T += U^T Kbar;  o -> HBM
 // The next chunk's TMA loads start as soon as step 2 has consumed the raw tiles.
+// Optional input preparation (gate logits, raw keys) rewrites the raw tiles in
+// place before step 1 (a compile-time variant, PREP).
 //
 // Split form: steps 1-4 do not depend on the state, so a persistent kernel
 // (the same code, SPLIT = true) runs them for every (chunk, head) on all SMs
@@ -120,7 +122,7 @@ struct ChunkParams {
 // unique, increasing within a sequence, and below N + ceil(rows / C).
 // A slot (one per head) holds byte images of the shared-memory operand tiles,
 // laid out so the chain kernel loads one contiguous block:
-constexpr uint32_t SL_QA = 0;         // [W'; Q'] 128-row K-major tile (32 KiB)
+constexpr uint32_t SL_QA = 0;         // [-W'; Q'] 128-row K-major tile (32 KiB)
 constexpr uint32_t SL_KB = 32768;     // Kbar (16 KiB)
 constexpr uint32_t SL_PBF = 49152;    // P bf16 (8 KiB)
 constexpr uint32_t SL_TBF = 57344;    // T Diag(w) bf16 (8 KiB)
@@ -503,7 +505,7 @@ __device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const floa
 // row operands, Kbar, the band of P, A and P, T = (I+A)^{-1}, W and U'^T.
 // Hand-offs go through mbarriers; each buffer the two groups share is
 // released by the step that last reads it:
-//   ready  : prep(n) -> chain(n)   (QA = [W'; Q'], Kbar, P, U' in TMEM, Gamma_C)
+//   ready  : prep(n) -> chain(n)   (QA = [-W'; Q'], Kbar, P, U' in TMEM, Gamma_C)
 //   s6     : chain(n) GEMMs of step 6 done -> prep(n+1) may rewrite QA
 //   s7     : chain(n) GEMMs of step 7 done -> prep(n+1) may rewrite Kbar, P, levels
 //   ufree  : chain(n) has read U^T out of TMEM -> prep(n+1) may write U'^T
