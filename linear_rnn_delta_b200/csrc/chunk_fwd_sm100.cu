@@ -878,7 +878,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                     *pv = pack4(mv);
                 }
             }
-            if (SPLIT && lane == 0 && pw < 5) bulk_wait_read();   // the previous item's slot stores
+            if (SPLIT && lane == 0) bulk_wait_read();   // the previous item's slot stores
             in_range = group_sync_and(BAR_PREP, NPREP, in_range);
             // GDN-2: the next item's v into the M tile the previous item stored (read: waited above)
             if (SPLIT && ptid == 0 && gdn2 && nxt.valid) issue_tma_v(nxt, par ^ 1u);
@@ -1113,6 +1113,16 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             tc_fence_before();
             group_sync(BAR_PREP, NPREP);
 
+            // split: Q' (rows 64-127 of both panels) and Kbar are final -- to the slot now, so that
+            // less is left to read out of shared memory at the end of the item
+            if (SPLIT && ok && lane == 0 && pw >= 5) {
+                uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
+                if (pw == 5) bulk_store(slot + SL_QA + 8192, sm + OFF_QA + 8192, 8192);
+                else if (pw == 6) bulk_store(slot + SL_QA + 24576, sm + OFF_QA + 24576, 8192);
+                else bulk_store(slot + SL_KB, sm + OFF_KB, 16384);
+                bulk_commit();
+            }
+
             // ===== 3. T = (I + A)^{-1} =============================================
             // 16x16 diagonal blocks by forward substitution (one column per thread), then
             // recursive doubling: T[16(I+1):, 16I:] = -D_{I+1} A_{I+1,I} D_I for I = 0, 2, and
@@ -1299,10 +1309,10 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             tc_fence_before();
             ok = group_sync_and(BAR_PREP, NPREP, ok);
             if (!SPLIT && ptid == 0) mbar_arrive(bar_ready);   // chunk ch's operands are ready for the chain
-            if (SPLIT && ok && lane == 0 && pw < 5) {   // the slot, one bulk store per warp
+            if (SPLIT && ok && lane == 0 && pw < 5) {   // the rest of the slot, one bulk store per warp
                 uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
-                if (pw == 0) bulk_store(slot + SL_QA, sm + OFF_QA, 32768);
-                else if (pw == 1) bulk_store(slot + SL_KB, sm + OFF_KB, 16384);
+                if (pw == 0) bulk_store(slot + SL_QA, sm + OFF_QA, 8192);                     // -W', panel 0
+                else if (pw == 1) bulk_store(slot + SL_QA + 16384, sm + OFF_QA + 16384, 8192);   // -W', panel 1
                 else if (pw == 2) bulk_store(slot + SL_PBF, sm + OFF_PBF, 8192);
                 else if (pw == 3) bulk_store(slot + SL_TBF, sm + OFF_TBF, 8192);
                 else {
@@ -1317,7 +1327,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
             if (need_v) mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
         }
-        if (SPLIT && lane == 0 && pw < 5) bulk_wait_all();
+        if (SPLIT && lane == 0) bulk_wait_all();
     }
 
     // ---- final state (NaN if an internal wait timed out) ----------------------
