@@ -1674,10 +1674,10 @@ cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
 
 bool chunk_prefer_split(const FwdArgs &a)
 {
-    // Cost model from measured per-chunk times on B200 (SM cycles): preparation of one
-    // (chunk, head) ~13.8 K, the split chain ~4.1 K, the fused kernel's critical path ~15.4 K.
-    // With U = N*H units on S SMs and W = ceil(U / S) waves of the per-unit kernels:
-    //   fused ~ W * 15.4,   split ~ (U / S) * 13.8 + W * 4.1   (per chunk of a unit).
+    // Cost model from measured kernel times on B200 (thousands of SM cycles per chunk):
+    // preparation of one (chunk, head) ~15.0, the split chain ~4.4, the fused kernel's
+    // critical path ~16.3.  With U = N*H units on S SMs and W = ceil(U / S) waves of the
+    // per-unit kernels:  fused ~ W * 16.3,  split ~ (U / S) * 15.0 + W * 4.4  (per chunk).
     // Packed (varlen) batches take the split form: the fused kernel's time is that of the
     // longest sequence per CTA, while the preparation kernel balances chunks over all SMs.
     int num_sms = 0;
@@ -1688,7 +1688,7 @@ bool chunk_prefer_split(const FwdArgs &a)
     if (a.cu_seqlens) return true;
     const double U = (double)a.B * a.H, S = num_sms;
     const double W = std::ceil(U / S);
-    return (U / S) * 13.8 + W * 4.1 < W * 15.4;
+    return (U / S) * 15.0 + W * 4.4 < W * 16.3;
 }
 
 size_t chunk_split_workspace_bytes(const FwdArgs &a)
