@@ -1373,6 +1373,8 @@ constexpr uint32_t CK_TMEM_COLS = 256;   // S^T [0,128), U^T [128,192), O^T [192
 static_assert(CK_ALLOC <= 232448, "shared memory budget");
 static_assert((CK_BUF & 1023) == 0 && (CK_S0T & 1023) == 0 && (CK_UT & 1023) == 0, "swizzle atoms");
 
+// SNAP: state snapshots requested (compiled out otherwise)
+template <bool SNAP>
 __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_constant__ ChunkParams P)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -1545,7 +1547,7 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
         if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
         ph_mma ^= 1;
         tc_fence_after();
-        if (a.snap) snapshot_state(a, tbase + lane_base, sbase + ch, h, half * 2, 2, jcol);
+        if (SNAP) snapshot_state(a, tbase + lane_base, sbase + ch, h, half * 2, 2, jcol);
         // every read of this buffer is done: load chunk ch + 2 into it
         if (tid == 0 && ok && ch + 2 < nchunks) issue_load(ch + 2, buf);
         stage_o();   // the U^T tile is free: the step-7 GEMMs are done
@@ -1636,8 +1638,10 @@ cudaError_t device_setup(int &num_sms)
                                       SMEM_ALLOC)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(chunk_fwd_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       SMEM_ALLOC)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(chunk_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CK_ALLOC)) !=
-                cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      CK_ALLOC)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      CK_ALLOC)) != cudaSuccess ||
             (e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return e;
     }
@@ -1718,7 +1722,8 @@ cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st
         else chunk_fwd_kernel<true, false><<<grid, NPREP, SMEM_ALLOC, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    chunk_chain_kernel<<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);
+    if (a.snap) chunk_chain_kernel<true><<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);
+    else chunk_chain_kernel<false><<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);
     return cudaGetLastError();
 }
 
