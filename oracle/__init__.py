@@ -314,3 +314,72 @@ def chunk_states(inp, every: int = 64, threads: int = 0):
             out[(n, c)] = sf[0]
             s = sf
     return out
+
+
+# ---------------------------------------------------------------------------
+# Gradients (reverse mode of the step recurrence)
+# ---------------------------------------------------------------------------
+
+def _gates(variant, k, v, g1, g2):
+    """Erase direction a~ and written value m of every token (float64)."""
+    if variant == "kda":
+        return g1[..., None] * k, g1[..., None] * v
+    if variant == "rda":
+        return g1[..., None] * k, g2[..., None] * v
+    return g1 * k, g2 * v
+
+
+def recurrence_grad(variant: str, q, k, v, alpha, g1, g2, initial_state, do, dsf=None):
+    """Gradients of L = sum(do * o) + sum(dsf * S_T) for ONE sequence and head.
+
+    q, k, alpha [T, dk]; v [T, dv]; g1 / g2 per the variant ([T] scalars or
+    [T, d] vectors, g2 None for KDA); initial_state [dk, dv] or None; do
+    [T, dv]; dsf [dk, dv] or None.  Reverse mode of the step recurrence
+      S' = Diag(alpha) S,  u = m - S'^T a~,  S = S' + k u^T,  o = S^T q,
+    taken step by step backwards (the adjoint of each step written out).
+    Returns a dict of float64 arrays: dq, dk, dv, dalpha, dg1, dg2 (None for
+    KDA), ds0.
+    """
+    q, k, v, alpha, g1, g2, do = (_f64(x) for x in (q, k, v, alpha, g1, g2, do))
+    T, dk = q.shape
+    dv = v.shape[-1]
+    at, m = _gates(variant, k, v, g1, g2)
+    S = np.zeros((dk, dv)) if initial_state is None else _f64(initial_state).copy()
+    states, us = [S.copy()], []
+    for t in range(T):                                   # forward, keeping S_{t-1} and u_t
+        Sp = alpha[t][:, None] * S
+        u = m[t] - Sp.T @ at[t]
+        S = Sp + np.outer(k[t], u)
+        states.append(S.copy())
+        us.append(u)
+    G = np.zeros((dk, dv)) if dsf is None else _f64(dsf).copy()
+    dq, dk_, dv_, da = (np.zeros_like(x) for x in (q, k, v, alpha))
+    dat, dm = np.zeros_like(at), np.zeros_like(m)
+    for t in range(T - 1, -1, -1):
+        S_prev, S_t, u = states[t], states[t + 1], us[t]
+        G = G + np.outer(q[t], do[t])                    # o_t = S_t^T q_t
+        dq[t] = S_t @ do[t]
+        du = G.T @ k[t]                                  # S_t = S' + k u^T
+        dk_[t] = G @ u
+        dSp = G - np.outer(at[t], du)                    # u = m - S'^T a~
+        dm[t] = du
+        Sp = alpha[t][:, None] * S_prev
+        dat[t] = -(Sp @ du)
+        da[t] = np.sum(S_prev * dSp, axis=1)             # S' = Diag(alpha) S_{t-1}
+        G = alpha[t][:, None] * dSp
+    if variant == "kda":
+        dg1 = np.sum(k * dat, axis=1) + np.sum(v * dm, axis=1)
+        dk_ += g1[:, None] * dat
+        dv_ = g1[:, None] * dm
+        dg2 = None
+    elif variant == "rda":
+        dg1 = np.sum(k * dat, axis=1)
+        dg2 = np.sum(v * dm, axis=1)
+        dk_ += g1[:, None] * dat
+        dv_ = g2[:, None] * dm
+    else:
+        dg1 = k * dat
+        dg2 = v * dm
+        dk_ += g1 * dat
+        dv_ = g2 * dm
+    return {"dq": dq, "dk": dk_, "dv": dv_, "dalpha": da, "dg1": dg1, "dg2": dg2, "ds0": G}

@@ -373,3 +373,60 @@ def test_chunk_states_are_prefix_runs():
         assert np.allclose(cs[(n, c)], sp[0], rtol=1e-12, atol=1e-14)
         if 64 * (c + 1) >= ln:                       # the last chunk's state is the final state
             assert np.allclose(cs[(n, c)], s_full[n], rtol=1e-12, atol=1e-14)
+
+
+# ---- gradients ------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("variant,gate_range", [("kda", "standard"), ("kda", "extended"), ("rda", "extended"),
+                                                ("gdn2", "standard")])
+def test_recurrence_grad_matches_central_differences(variant, gate_range):
+    """Every input's gradient against central differences of the forward oracle (float64)."""
+    inp = make_chunk_inputs(variant, gate_range, "f32", B=1, T=7, H=1, d_k=4, d_v=3, seed=43,
+                            init_state="random", init_std=0.5)
+    f = lambda x: x[0, :, 0].double().numpy()
+    arrs = {"q": f(inp.q), "k": f(inp.k), "v": f(inp.v), "alpha": f(inp.alpha), "g1": f(inp.g1),
+            "g2": None if inp.g2 is None else f(inp.g2)}
+    s0 = inp.initial_state[0, 0].double().numpy()
+    rng = np.random.default_rng(3)
+    do = rng.standard_normal((7, 3))
+    dsf = rng.standard_normal((4, 3))
+
+    def loss(a, s):
+        o, sf = oracle.recurrence_arrays(variant, *(None if a[n] is None else a[n][None, :, None]
+                                                     for n in ("q", "k", "v", "alpha", "g1", "g2")),
+                                         None, s[None, None])
+        return float(np.sum(o[0, :, 0] * do) + np.sum(sf[0, 0] * dsf))
+
+    g = oracle.recurrence_grad(variant, arrs["q"], arrs["k"], arrs["v"], arrs["alpha"], arrs["g1"], arrs["g2"],
+                               s0, do, dsf)
+    eps = 1e-6
+    for name, gname in (("q", "dq"), ("k", "dk"), ("v", "dv"), ("alpha", "dalpha"), ("g1", "dg1"), ("g2", "dg2")):
+        if arrs[name] is None:
+            assert g[gname] is None
+            continue
+        fd = np.zeros_like(arrs[name])
+        for idx in np.ndindex(arrs[name].shape):
+            a_p = {n: (None if x is None else x.copy()) for n, x in arrs.items()}
+            a_m = {n: (None if x is None else x.copy()) for n, x in arrs.items()}
+            a_p[name][idx] += eps
+            a_m[name][idx] -= eps
+            fd[idx] = (loss(a_p, s0) - loss(a_m, s0)) / (2 * eps)
+        assert np.allclose(g[gname], fd, rtol=1e-6, atol=1e-7), name
+    fd0 = np.zeros_like(s0)
+    for idx in np.ndindex(s0.shape):
+        sp, sm = s0.copy(), s0.copy()
+        sp[idx] += eps
+        sm[idx] -= eps
+        fd0[idx] = (loss(arrs, sp) - loss(arrs, sm)) / (2 * eps)
+    assert np.allclose(g["ds0"], fd0, rtol=1e-6, atol=1e-7)
+
+
+def test_recurrence_grad_of_linear_attention_closed_form():
+    """alpha = 1, beta = 0 (no erase, no write): o_t = S_0^T q_t, so dq_t = S_0 do_t and dS_0 = sum_t q_t do_t^T."""
+    rng = np.random.default_rng(4)
+    T, dk, dv = 6, 5, 3
+    q, k = rng.standard_normal((T, dk)), rng.standard_normal((T, dk))
+    v, s0, do = rng.standard_normal((T, dv)), rng.standard_normal((dk, dv)), rng.standard_normal((T, dv))
+    g = oracle.recurrence_grad("kda", q, k, v, np.ones((T, dk)), np.zeros(T), None, s0, do)
+    assert np.allclose(g["dq"], do @ s0.T) and np.allclose(g["ds0"], q.T @ do)
+    assert np.allclose(g["dv"], 0) and np.allclose(g["dk"], 0)
