@@ -202,6 +202,36 @@ int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
                           void *o, unsigned flags, void *stream);
 
 /*
+ * kda_chunk_bwd -- gradients of the forward recurrence (backward pass), for
+ * L with dL/do = d_o and dL/dS_final = d_final_state (NULL = 0):
+ *   dq, dk, alpha-, g1-, g2-gradients and dL/dS_initial, all fp32, in the
+ *   layouts of the corresponding inputs (dg1: beta / e [B,T,H] or GDN-2's b
+ *   [B,T,H,d_k]; dg2: w [B,T,H] (RDA) or [B,T,H,d_v] (GDN-2), NULL for KDA;
+ *   d_initial_state [N,H,d_k,d_v] or NULL).
+ * Inputs as for kda_chunk_fwd (d_o in the input dtype, [B,T,H,d_v]); no
+ * flags (the inputs are the recurrence's own: no logits, normalised keys).
+ * The gradient is that of the exact recurrence: an fp32 adjoint scan replays
+ * each 64-token chunk forward from an fp32 checkpoint (a forward scan's state
+ * snapshots) and walks it backwards (adjoint of one step:
+ *   G_{t-1} = Diag(alpha_t) (I - a~_t k_t^T) (G_t + q_t do_t^T)).
+ * Token-serial per (sequence, head); far slower than the forward.
+ * workspace: caller-owned, 16-byte aligned, at least
+ * kda_chunk_bwd_workspace_size(...) bytes: (N + ceil(B*T/64)) * H * d_k * d_v
+ * * 4 for the checkpoints plus N * H * 64 * d_k * d_v * 4.
+ */
+size_t kda_chunk_bwd_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
+                                    int has_cu_seqlens, int num_seqs);
+int kda_chunk_bwd(int variant, int gate_range, int dtype,
+                  int B, int T, int H, int d_k, int d_v,
+                  const void *q, const void *k, const void *v, const void *alpha,
+                  const void *g1, const void *g2,
+                  const int32_t *cu_seqlens, int num_seqs, const float *initial_state,
+                  const void *d_o, const float *d_final_state,
+                  float *dq, float *dk, float *dv, float *dalpha, float *dg1, float *dg2,
+                  float *d_initial_state, void *workspace, size_t workspace_bytes,
+                  unsigned flags, void *stream);
+
+/*
  * kda_decode_step -- one recurrent step for N sequences (single-token decode;
  * the fixed-size state of the openarchlab page, sec. 1 and 3).
  *

@@ -257,6 +257,77 @@ extern "C" int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
 #endif
 }
 
+// Backward workspace: the forward's state snapshots (chunk slots) and each
+// CTA's per-chunk states.
+size_t bwd_workspace_bytes(const kda::FwdArgs &a)
+{
+    const long long N = a.cu_seqlens ? a.num_seqs : a.B;
+    const long long slots = N + ((long long)a.B * a.T + 63) / 64;
+    return (size_t)slots * a.H * a.dk * a.dv * sizeof(float) + kda::scan_bwd_scratch_bytes(a);
+}
+
+extern "C" size_t kda_chunk_bwd_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
+                                               int has_cu_seqlens, int num_seqs)
+{
+    if (B < 1 || T < 0 || H < 1 || (has_cu_seqlens && (B != 1 || num_seqs < 1))) return 0;
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_F32) return 0;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return 0;
+    if ((unsigned long long)B * (unsigned long long)T * H * 128ull > (1ull << 46)) return 0;
+    kda::FwdArgs a{};
+    a.B = B; a.T = T; a.H = H; a.dk = d_k; a.dv = d_v;
+    a.num_seqs = has_cu_seqlens ? num_seqs : B;
+    a.cu_seqlens = has_cu_seqlens ? reinterpret_cast<const int32_t *>(16) : nullptr;   // presence only
+    return bwd_workspace_bytes(a);
+}
+
+extern "C" int kda_chunk_bwd(int variant, int gate_range, int dtype,
+                             int B, int T, int H, int d_k, int d_v,
+                             const void *q, const void *k, const void *v, const void *alpha,
+                             const void *g1, const void *g2,
+                             const int32_t *cu_seqlens, int num_seqs, const float *initial_state,
+                             const void *d_o, const float *d_final_state,
+                             float *dq, float *dk, float *dv, float *dalpha, float *dg1, float *dg2,
+                             float *d_initial_state, void *workspace, size_t workspace_bytes,
+                             unsigned flags, void *stream)
+{
+    kda::FwdArgs a;
+    int rc = chunk_args(a, variant, gate_range, dtype, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens,
+                        num_seqs, initial_state, nullptr, d_o ? const_cast<void *>(d_o) : workspace, 64, 0u);
+    if (rc != KDA_OK) return rc;
+    if (flags) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd takes no flags (got 0x%x)", flags);
+    if (T > 0) {
+        const void *need[] = {d_o, dq, dk, dv, dalpha, dg1};
+        const char *names[] = {"d_o", "dq", "dk", "dv", "dalpha", "dg1"};
+        for (int i = 0; i < 6; ++i) {
+            if (!need[i]) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+            if (!aligned16(need[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+        }
+        if (variant != KDA_VARIANT_KDA && (!dg2 || !aligned16(dg2)))
+            return fail(KDA_ERR_INVALID_ARG, "dg2 is NULL or misaligned (RDA and GDN-2 have a write gate)");
+    }
+    if ((d_final_state && !aligned16(d_final_state)) || (d_initial_state && !aligned16(d_initial_state)))
+        return fail(KDA_ERR_INVALID_ARG, "d_final_state / d_initial_state is not 16-byte aligned");
+    const size_t need_ws = bwd_workspace_bytes(a);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need_ws)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd needs a 16-byte aligned workspace of %zu bytes", need_ws);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    // 1. forward scan in fp32, keeping only the state after every 64 tokens (the checkpoints)
+    a.o = nullptr;
+    a.sf = nullptr;
+    a.snap = static_cast<float *>(workspace);
+    const long long N = a.cu_seqlens ? a.num_seqs : a.B;
+    const size_t snap_bytes = (size_t)(N + ((long long)a.B * a.T + 63) / 64) * a.H * a.dk * a.dv * sizeof(float);
+    cudaError_t e = kda::launch_scan_fwd(a, bf16, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd forward replay");
+    // 2. adjoint scan
+    kda::BwdArgs g{d_o, d_final_state, dq, dk, dv, dalpha, dg1, dg2, d_initial_state,
+                   reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + snap_bytes)};
+    e = kda::launch_scan_bwd(a, g, bf16, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd launch");
+    return KDA_OK;
+}
+
 extern "C" int kda_decode_step(int variant, int gate_range, int dtype,
                                int N, int H, int d_k, int d_v,
                                const void *q, const void *k, const void *v, const void *alpha,

@@ -122,7 +122,7 @@ scan_fwd_kernel(FwdArgs a)
                 o3 = fmaf(qv.w, S[i + 3], o3);
             }
             const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
-            st_out((TIn *)a.o + tok * DV + j, (o0 + o1) + (o2 + o3));
+            if (a.o) st_out((TIn *)a.o + tok * DV + j, (o0 + o1) + (o2 + o3));   // null: states only
             const int t = base + tt;   // token index within the sequence
             if (a.snap && ((t + 1) % SLOT_TOKENS == 0 || t + 1 == len)) {   // state after a 64-token chunk
                 float *dst = a.snap + ((size_t)(slot_base(a, n) + t / SLOT_TOKENS) * a.H + h) * DK * DV + j;

@@ -192,6 +192,19 @@ def make_chunk_inputs(variant: str = "kda", gate_range: str = "standard", dtype:
 # ---------------------------------------------------------------------------
 # The named workloads (shapes and distributions of the recurrence's benchmark
 # configurations).  Each returns ChunkInputs; the decode workload is separate.
+def grad_outputs(inp: ChunkInputs, seed: int = 0, d_final: bool = True):
+    """Incoming gradients for a backward pass over ``inp``: d_o [B,T,H,d_v]
+    ~ N(0,1) in the run dtype and dL/dS_final fp32 [N,H,d_k,d_v] ~ N(0, 0.1^2)
+    (None unless ``d_final``), from ``default_rng((seed, 7))``."""
+    rng = np.random.default_rng((seed, 7))
+    d_o = _cast(rng.standard_normal((inp.B, inp.T, inp.H, inp.d_v), dtype=np.float32), inp.dtype)
+    dsf = None
+    if d_final:
+        dsf = torch.from_numpy(0.1 * rng.standard_normal((inp.num_seqs, inp.H, inp.d_k, inp.d_v),
+                                                         dtype=np.float32))
+    return d_o, dsf
+
+
 # ---------------------------------------------------------------------------
 
 def tiny_ckda(seed: int = 0) -> ChunkInputs:
