@@ -5,7 +5,7 @@
 #include <cstdint>
 
 #include "../../include/kda.h"
-#include "common.cuh"
+#include "scan_bwd.cuh"
 
 namespace {
 

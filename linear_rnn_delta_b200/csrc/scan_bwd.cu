@@ -16,7 +16,7 @@
 // shared memory (rows padded to DV + 1 floats: row-wise and column-wise sweeps
 // are both bank-conflict free); row sums (over value columns j) and column
 // sums (over key channels i) are split over the CTA's 256 threads.
-#include "common.cuh"
+#include "scan_bwd.cuh"
 
 namespace kda {
 namespace {

@@ -36,6 +36,8 @@ def _close(g, r, what):
     g2 = g.reshape(-1, g.shape[-1]) if g.ndim > 1 else g.reshape(-1, 1)
     r2 = r.reshape(-1, r.shape[-1]) if r.ndim > 1 else r.reshape(-1, 1)
     assert np.all(np.isfinite(g2)), f"{what}: non-finite"
+    if g2.size == 0:
+        return
     err = np.abs(g2 - r2).max(axis=1)
     scale = np.maximum(1.0, np.abs(r2).max(axis=1))
     worst = int(np.argmax(err / scale))
