@@ -9,14 +9,26 @@
 //   G <- Diag(alpha) dS'   (dL/dS_{t-1}),
 // followed by the variant's gate algebra ((a~, m) = (beta k, beta v),
 // (e k, w v) or (b (.) k, w (.) v)).  The backward needs S_{t-1} at every
-// token: one CTA per (sequence, head) walks the sequence's 64-token chunks
-// from last to first; each chunk is replayed forward from its checkpoint (the
-// state snapshot the forward scan stored after the previous chunk), keeping
-// every S_{t-1} and u_t of the chunk, then walked backwards.  S and G live in
-// shared memory (rows padded to DV + 1 floats: row-wise and column-wise sweeps
-// are both bank-conflict free); row sums (over value columns j) and column
-// sums (over key channels i) are split over the CTA's 256 threads.
+// token: each sequence's 64-token chunks are walked from last to first; each
+// chunk is replayed forward from its checkpoint (the state snapshot the forward
+// scan stored after the previous chunk), then walked backwards.
+//
+// Both directions act on the columns of S and G independently (the left
+// factors Diag(alpha) and I - k a~^T are shared by all value columns; m_j and
+// do_j touch column j only).  The main kernel (d_k >= 32) therefore splits the
+// d_v columns over a cluster of CTAs, 32 columns each, and gives every thread
+// one row of S and G in registers: sums over columns are in-thread, sums over
+// rows are a warp reduce-scatter plus one CTA barrier.  The per-row results
+// (dq, dk, dalpha, da~) are partial sums over the CTA's columns; the cluster
+// adds them through distributed shared memory every 8 tokens, in a fixed order
+// (deterministic results).  The replay keeps S_{t-1} only every 4 tokens
+// (global scratch) with u_t in shared memory; the backward walk recomputes the
+// states in between with the same fused multiply-adds, so they are bitwise
+// those of the replay.  d_k = 16 uses a plain shared-memory kernel (one CTA per
+// sequence and head).
 #include "scan_bwd.cuh"
+
+#include <cooperative_groups.h>
 
 namespace kda {
 namespace {
@@ -286,21 +298,418 @@ cudaError_t launch_bwd_dv(const FwdArgs &a, const BwdArgs &g, bool bf16, cudaStr
     return cudaErrorInvalidValue;
 }
 
+// ---------------------------------------------------------------------------
+// Row-resident kernel: a cluster of DV / DVB CTAs per (sequence, head), DK
+// threads per CTA (thread i = row i), DVB value columns per CTA.
+
+namespace cg = cooperative_groups;
+
+constexpr int CKP = 4;   // tokens between stored states within a chunk
+constexpr int RTB = 8;   // tokens per cross-CTA reduction block
+
+template <int DK, int DVB>
+struct RowSmem {
+    static constexpr int NW = DK / 32;
+    static constexpr size_t U = 0;                               // [BC][DVB] u_t of the chunk
+    static constexpr size_t DO = U + (size_t)BC * DVB;           // [BC][DVB] do_t
+    static constexpr size_t VV = DO + (size_t)BC * DVB;          // [BC][DVB] v_t
+    static constexpr size_t WW = VV + (size_t)BC * DVB;          // [BC][DVB] write gate (scalar gates broadcast)
+    static constexpr size_t PART = WW + (size_t)BC * DVB;        // [2][NW][DVB] per-warp column sums
+    static constexpr size_t FIN = PART + 2 * NW * DVB;           // [NW][DVB] column totals, one copy per warp
+    static constexpr size_t RING = FIN + NW * DVB;               // [2][RTB][4][DK] per-token row partials
+    static constexpr size_t RINGV = RING + 2 * RTB * 4 * DK;     // [2][RTB] partial sum_j v_j du_j
+    static constexpr size_t SRED = RINGV + 2 * RTB;              // [RTB][NW] warp sums of k_i da~_i
+    static constexpr size_t TOK = SRED + RTB * NW;               // [2][RTB] token index (int)
+    static constexpr size_t CKB = TOK + 2 * RTB;                 // [2][DVB/4][DK] float4: a group's stored state
+    static constexpr size_t RSM = CKB + 2 * (size_t)DVB * DK;    // [CKP][4][DK] row scalars of a group
+    static constexpr size_t FLOATS = RSM + (size_t)CKP * 4 * DK;
+};
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Sums x over the warp's 32 lanes for every column: on return x[0] holds the
+// total of column lane / (32 / L) (a butterfly that halves the vector at each
+// exchange; the last exchanges, when L < 32, add duplicates).
+template <int L>
+__device__ __forceinline__ void reduce_scatter(float (&x)[L], int lane)
+{
+#pragma unroll
+    for (int half = L / 2, off = 16; half >= 1; half /= 2, off /= 2) {
+        const bool upper = lane & off;
+#pragma unroll
+        for (int e = 0; e < half; ++e) {
+            const float send = upper ? x[e] : x[e + half];
+            const float keep = upper ? x[e + half] : x[e];
+            x[e] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+    }
+#pragma unroll
+    for (int off = 16 / L; off >= 1; off /= 2) x[0] += __shfl_xor_sync(0xffffffffu, x[0], off);
+}
+
+template <int DK, int DVB, typename TIn>
+__global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
+{
+    using L = RowSmem<DK, DVB>;
+    constexpr int NW = L::NW, LPC = 32 / DVB, NQ = DVB / 4;
+    extern __shared__ __align__(16) float smf[];
+    float *sU = smf + L::U, *sDO = smf + L::DO, *sV = smf + L::VV, *sW = smf + L::WW;
+    int *tokrow = reinterpret_cast<int *>(smf + L::TOK);
+    cg::cluster_group cl = cg::this_cluster();
+    const int NB = a.dv / DVB;
+    const int rank = (int)cl.block_rank();
+    const int hh = blockIdx.x / NB, jb = blockIdx.x % NB;
+    const int n = hh / a.H, h = hh % a.H;
+    const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+    const bool owner = lane % LPC == 0;   // holds column lane / LPC after a reduce-scatter
+    const int col = lane / LPC;
+    const int row0 = seq_row0(a, n), len = seq_len(a, n);
+    const TIn *q = (const TIn *)a.q, *k = (const TIn *)a.k, *v = (const TIn *)a.v;
+    const TIn *al = (const TIn *)a.alpha, *g1 = (const TIn *)a.g1, *g2 = (const TIn *)a.g2;
+    const TIn *dO = (const TIn *)g.d_o;
+    const bool vec_gate = a.variant == GDN2;
+    // row i of this CTA's column block in a [dk][dv] state
+    const size_t srow = (((size_t)n * a.H + h) * DK + i) * a.dv + (size_t)jb * DVB;
+    float4 *scr = reinterpret_cast<float4 *>(g.scratch) + (size_t)blockIdx.x * (BC / CKP) * NQ * DK;
+
+    float S[DVB], G[DVB];
+    auto load_row = [&](float (&dst)[DVB], const float *src) {
+#pragma unroll
+        for (int c4 = 0; c4 < NQ; ++c4) {
+            const float4 x = src ? reinterpret_cast<const float4 *>(src)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+            dst[4 * c4] = x.x; dst[4 * c4 + 1] = x.y; dst[4 * c4 + 2] = x.z; dst[4 * c4 + 3] = x.w;
+        }
+    };
+    auto tok_of = [&](int t) { return ((size_t)row0 + t) * a.H + h; };
+    auto gate_e = [&](size_t tok) { return vec_gate ? ld_f32(g1 + tok * DK + i) : ld_f32(g1 + tok); };
+    // column sums over the CTA's rows of x (destroyed); returns nothing, leaves the
+    // totals in `fin` (this warp's copy) after a CTA barrier and a warp barrier
+    unsigned red_count = 0;
+    auto column_sums = [&](float (&x)[DVB]) -> float * {
+        reduce_scatter<DVB>(x, lane);
+        float *part = smf + L::PART + (red_count & 1) * NW * DVB;
+        ++red_count;
+        if (owner) part[warp * DVB + col] = x[0];
+        __syncthreads();
+        float *fin = smf + L::FIN + warp * DVB;
+        if (owner) {
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) acc += part[w * DVB + col];
+            fin[col] = acc;
+        }
+        __syncwarp();
+        return fin;
+    };
+
+    load_row(G, g.d_sf ? g.d_sf + srow : nullptr);
+    int blk = 0, pos = 0;   // cross-CTA reduction block and position in it
+    const int nchunks = (len + BC - 1) / BC;
+    for (int c = nchunks - 1; c >= 0; --c) {
+        const int t0 = c * BC, nt = min(BC, len - t0);
+        __syncthreads();   // the previous chunk's readers of the staged vectors are done
+        for (int e = i; e < nt * DVB; e += DK) {
+            const int tt = e / DVB, j = e % DVB;
+            const size_t tok = tok_of(t0 + tt);
+            const size_t cj = tok * a.dv + (size_t)jb * DVB + j;
+            float w;
+            if (a.variant == KDA) w = ld_f32(g1 + tok);
+            else if (a.variant == RDA) w = ld_f32(g2 + tok);
+            else w = ld_f32(g2 + cj);
+            sV[e] = ld_f32(v + cj);
+            sW[e] = w;
+            sDO[e] = ld_f32(dO + cj);
+        }
+        load_row(S, c == 0 ? (a.s0 ? a.s0 + srow : nullptr)
+                           : a.snap + (((size_t)(slot_base(a, n) + c - 1) * a.H + h) * DK + i) * a.dv +
+                                 (size_t)jb * DVB);
+        __syncthreads();
+        // ---- replay: u_t into shared memory, S_{t-1} every CKP tokens into scratch
+        float n_al = 0.f, n_k = 0.f, n_e = 0.f;
+        if (nt > 0) {
+            const size_t tok = tok_of(t0);
+            n_al = ld_f32(al + tok * DK + i); n_k = ld_f32(k + tok * DK + i); n_e = gate_e(tok);
+        }
+        for (int tt = 0; tt < nt; ++tt) {
+            const float alpha_i = n_al, k_i = n_k, e_i = n_e;
+            if (tt + 1 < nt) {
+                const size_t tok = tok_of(t0 + tt + 1);
+                n_al = ld_f32(al + tok * DK + i); n_k = ld_f32(k + tok * DK + i); n_e = gate_e(tok);
+            }
+            if (tt % CKP == 0) {
+#pragma unroll
+                for (int c4 = 0; c4 < NQ; ++c4)
+                    scr[((size_t)(tt / CKP) * NQ + c4) * DK + i] =
+                        make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
+            }
+            float x[DVB];
+            const float aa = alpha_i * (e_i * k_i);   // alpha_i a~_i
+#pragma unroll
+            for (int j = 0; j < DVB; ++j) x[j] = aa * S[j];
+            float *fin = column_sums(x);
+            if (owner) {   // u_j = m_j - sum_i alpha_i a~_i S_ij
+                const float u = sW[tt * DVB + col] * sV[tt * DVB + col] - fin[col];
+                fin[col] = u;
+                if (warp == 0) sU[tt * DVB + col] = u;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int c4 = 0; c4 < NQ; ++c4) {
+                const float4 u4 = reinterpret_cast<const float4 *>(fin)[c4];
+                S[4 * c4] = fmaf(alpha_i, S[4 * c4], k_i * u4.x);
+                S[4 * c4 + 1] = fmaf(alpha_i, S[4 * c4 + 1], k_i * u4.y);
+                S[4 * c4 + 2] = fmaf(alpha_i, S[4 * c4 + 2], k_i * u4.z);
+                S[4 * c4 + 3] = fmaf(alpha_i, S[4 * c4 + 3], k_i * u4.w);
+            }
+        }
+        __syncthreads();   // u_t of the chunk visible to every warp
+        // ---- backward walk, last token first, in groups of CKP tokens (one stored state each)
+        const int ngrp = (nt + CKP - 1) / CKP;
+        float4 *ckb = reinterpret_cast<float4 *>(smf + L::CKB);   // [2][NQ][DK]: each thread its own row
+        float c_al[CKP], c_k[CKP];   // alpha_i, k_i of the current group's tokens (recompute steps)
+        float *rsm = smf + L::RSM;   // [CKP][4][DK]: alpha, k, q, e of the group's tokens, own row only
+        float f_al[CKP] = {}, f_k[CKP] = {}, f_q[CKP] = {}, f_e[CKP] = {};   // of the next group (prefetched)
+        // pass gi fetches group gi - 1 (stored state by cp.async, row scalars into
+        // registers) while it works on group gi, fetched by the pass before
+        for (int gi = ngrp; gi >= 0; --gi) {
+            const int grp = gi, buf = gi & 1;
+#pragma unroll
+            for (int s = 0; s < CKP; ++s) {
+                c_al[s] = f_al[s];
+                c_k[s] = f_k[s];
+                rsm[(s * 4 + 0) * DK + i] = f_al[s];
+                rsm[(s * 4 + 1) * DK + i] = f_k[s];
+                rsm[(s * 4 + 2) * DK + i] = f_q[s];
+                rsm[(s * 4 + 3) * DK + i] = f_e[s];
+            }
+            cp_async_wait_all();
+            if (gi > 0) {
+                const int fg = gi - 1, fb = fg & 1;
+#pragma unroll
+                for (int c4 = 0; c4 < NQ; ++c4)
+                    cp_async16(&ckb[((size_t)fb * NQ + c4) * DK + i], &scr[((size_t)fg * NQ + c4) * DK + i]);
+                cp_async_commit();
+                const int fn = min(CKP, nt - fg * CKP);
+#pragma unroll
+                for (int s = 0; s < CKP; ++s) {
+                    if (s < fn) {
+                        const size_t tok = tok_of(t0 + fg * CKP + s);
+                        f_al[s] = ld_f32(al + tok * DK + i);
+                        f_k[s] = ld_f32(k + tok * DK + i);
+                        f_q[s] = ld_f32(q + tok * DK + i);
+                        f_e[s] = gate_e(tok);
+                    }
+                }
+            }
+            if (gi == ngrp) continue;
+            const int ntok = min(CKP, nt - grp * CKP);
+            for (int r = ntok - 1; r >= 0; --r) {
+                const int tt = grp * CKP + r;
+                // S_{t-1}: the group's stored state advanced over its first r tokens (the replay's own steps)
+#pragma unroll
+                for (int c4 = 0; c4 < NQ; ++c4) {
+                    const float4 x = ckb[((size_t)buf * NQ + c4) * DK + i];
+                    S[4 * c4] = x.x; S[4 * c4 + 1] = x.y; S[4 * c4 + 2] = x.z; S[4 * c4 + 3] = x.w;
+                }
+                const float alpha_i = rsm[(r * 4 + 0) * DK + i], k_i = rsm[(r * 4 + 1) * DK + i];
+                const float q_i = rsm[(r * 4 + 2) * DK + i], e_i = rsm[(r * 4 + 3) * DK + i];
+#pragma unroll
+                for (int s = 0; s < CKP - 1; ++s) {
+                    if (s < r) {
+                        const float4 *u4p = reinterpret_cast<const float4 *>(sU + (grp * CKP + s) * DVB);
+#pragma unroll
+                        for (int c4 = 0; c4 < NQ; ++c4) {
+                            const float4 u4 = u4p[c4];
+                            S[4 * c4] = fmaf(c_al[s], S[4 * c4], c_k[s] * u4.x);
+                            S[4 * c4 + 1] = fmaf(c_al[s], S[4 * c4 + 1], c_k[s] * u4.y);
+                            S[4 * c4 + 2] = fmaf(c_al[s], S[4 * c4 + 2], c_k[s] * u4.z);
+                            S[4 * c4 + 3] = fmaf(c_al[s], S[4 * c4 + 3], c_k[s] * u4.w);
+                        }
+                    }
+                }
+                const int t = t0 + tt;
+                const size_t tok = tok_of(t);
+                const float4 *do4 = reinterpret_cast<const float4 *>(sDO + tt * DVB);
+                const float4 *u4p = reinterpret_cast<const float4 *>(sU + tt * DVB);
+                // G += q do^T;  row partials of S_t do (= alpha S_{t-1} do + k (u.do)) and G u
+                float sdo[2] = {0.f, 0.f}, udo[2] = {0.f, 0.f}, gu[2] = {0.f, 0.f};
+#pragma unroll
+                for (int c4 = 0; c4 < NQ; ++c4) {
+                    const float4 d4 = do4[c4], u4 = u4p[c4];
+                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w}, uu[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * c4 + e;
+                        G[j] = fmaf(q_i, dd[e], G[j]);
+                        sdo[e & 1] = fmaf(S[j], dd[e], sdo[e & 1]);
+                        udo[e & 1] = fmaf(uu[e], dd[e], udo[e & 1]);
+                        gu[e & 1] = fmaf(G[j], uu[e], gu[e & 1]);
+                    }
+                }
+                // du_j = sum_i k_i G_ij
+                float x[DVB];
+#pragma unroll
+                for (int j = 0; j < DVB; ++j) x[j] = k_i * G[j];
+                float *fin = column_sums(x);
+                if (warp == 0) {   // per-column outputs: dv = w du;  GDN-2 dw = v du;  scalar gates: sum_j v_j du_j
+                    float vdu = 0.f;
+                    if (owner) {
+                        const float du = fin[col], vj = sV[tt * DVB + col];
+                        const size_t cj = tok * a.dv + (size_t)jb * DVB + col;
+                        g.dv[cj] = sW[tt * DVB + col] * du;
+                        if (vec_gate) g.dg2[cj] = vj * du;
+                        vdu = vj * du;
+                    }
+                    if (!vec_gate) {
+#pragma unroll
+                        for (int off = 16; off; off >>= 1) vdu += __shfl_xor_sync(0xffffffffu, vdu, off);
+                        if (lane == 0) smf[L::RINGV + (blk & 1) * RTB + pos] = vdu;
+                    }
+                }
+                // dS' = G - a~ du^T;  dalpha = rowsum(S_{t-1} dS');  S_{t-1} du;  G <- Diag(alpha) dS'
+                const float at = e_i * k_i;
+                float sds[2] = {0.f, 0.f}, sdu[2] = {0.f, 0.f};
+#pragma unroll
+                for (int c4 = 0; c4 < NQ; ++c4) {
+                    const float4 du4 = reinterpret_cast<const float4 *>(fin)[c4];
+                    const float du[4] = {du4.x, du4.y, du4.z, du4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * c4 + e;
+                        G[j] = fmaf(-at, du[e], G[j]);
+                        sds[e & 1] = fmaf(S[j], G[j], sds[e & 1]);
+                        sdu[e & 1] = fmaf(S[j], du[e], sdu[e & 1]);
+                        G[j] *= alpha_i;
+                    }
+                }
+                // this CTA's parts (its value columns) of dq, dk, dalpha and k (.) da~, da~ = -Diag(alpha) S_{t-1} du
+                const float datp = -alpha_i * (sdu[0] + sdu[1]);
+                float *ring = smf + L::RING + ((size_t)((blk & 1) * RTB + pos) * 4) * DK;
+                ring[i] = fmaf(alpha_i, sdo[0] + sdo[1], k_i * (udo[0] + udo[1]));
+                ring[DK + i] = fmaf(e_i, datp, gu[0] + gu[1]);   // a~ = e (.) k: dk = G u + e da~
+                ring[2 * DK + i] = sds[0] + sds[1];
+                ring[3 * DK + i] = k_i * datp;
+                if (i == 0) tokrow[(blk & 1) * RTB + pos] = t;
+                ++pos;
+                if (pos == RTB || (c == 0 && tt == 0)) {   // add the cluster's parts for this block of tokens
+                    const int rb = blk & 1, cnt = pos;
+                    cl.sync();
+                    for (int p = rank; p < cnt; p += NB) {
+                        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (int cr = 0; cr < NB; ++cr) {
+                            const float *rr =
+                                cl.map_shared_rank(smf + L::RING + (size_t)((rb * RTB + p) * 4) * DK, cr);
+#pragma unroll
+                            for (int qd = 0; qd < 4; ++qd) sum[qd] += rr[qd * DK + i];
+                        }
+                        const size_t tk = tok_of(tokrow[rb * RTB + p]);
+                        g.dq[tk * DK + i] = sum[0];
+                        g.dk[tk * DK + i] = sum[1];
+                        g.dalpha[tk * DK + i] = sum[2];
+                        if (vec_gate) {
+                            g.dg1[tk * DK + i] = sum[3];   // db_i = k_i da~_i
+                        } else {
+                            float sk = sum[3];
+#pragma unroll
+                            for (int off = 16; off; off >>= 1) sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                            if (lane == 0) smf[L::SRED + p * NW + warp] = sk;
+                        }
+                    }
+                    if (!vec_gate) {
+                        __syncthreads();
+                        if (i < cnt && i % NB == rank) {   // scalar gates of token position i
+                            const int p = i;
+                            float sk = 0.f, sv = 0.f;
+#pragma unroll
+                            for (int w = 0; w < NW; ++w) sk += smf[L::SRED + p * NW + w];
+                            for (int cr = 0; cr < NB; ++cr)
+                                sv += *cl.map_shared_rank(smf + L::RINGV + rb * RTB + p, cr);
+                            const size_t tk = tok_of(tokrow[rb * RTB + p]);
+                            if (a.variant == KDA) {
+                                g.dg1[tk] = sk + sv;   // a~ = beta k, m = beta v
+                            } else {
+                                g.dg1[tk] = sk;        // RDA: a~ = e k, m = w v
+                                g.dg2[tk] = sv;
+                            }
+                        }
+                    }
+                    ++blk;
+                    pos = 0;
+                }
+            }
+        }
+    }
+    if (g.d_s0) {
+        float4 *dst = reinterpret_cast<float4 *>(g.d_s0 + srow);
+#pragma unroll
+        for (int c4 = 0; c4 < NQ; ++c4) dst[c4] = make_float4(G[4 * c4], G[4 * c4 + 1], G[4 * c4 + 2], G[4 * c4 + 3]);
+    }
+    cl.sync();   // no CTA leaves while the cluster may still read its shared memory
+}
+
+template <int DK, int DVB>
+cudaError_t launch_rows_dims(const FwdArgs &a, const BwdArgs &g, bool bf16, cudaStream_t st)
+{
+    const size_t smem = RowSmem<DK, DVB>::FLOATS * sizeof(float);
+    const int N = a.cu_seqlens ? a.num_seqs : a.B;
+    const int NB = a.dv / DVB;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(N * a.H * NB));
+    cfg.blockDim = dim3(DK);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = NB;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (bf16) {
+        auto *kern = scan_bwd_rows_kernel<DK, DVB, __nv_bfloat16>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        e = cudaLaunchKernelEx(&cfg, kern, a, g);
+    } else {
+        auto *kern = scan_bwd_rows_kernel<DK, DVB, float>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+            return e;
+        e = cudaLaunchKernelEx(&cfg, kern, a, g);
+    }
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int DK>
+cudaError_t launch_rows_dv(const FwdArgs &a, const BwdArgs &g, bool bf16, cudaStream_t st)
+{
+    // 16 columns per CTA for d_v = 16, else 32 (clusters of 1, 2 or 4 CTAs)
+    return a.dv == 16 ? launch_rows_dims<DK, 16>(a, g, bf16, st) : launch_rows_dims<DK, 32>(a, g, bf16, st);
+}
+
 }  // namespace
 
 size_t scan_bwd_scratch_bytes(const FwdArgs &a)
 {
+    // d_k = 16: every S_{t-1} of a chunk; otherwise every CKP-th
     const long long N = a.cu_seqlens ? a.num_seqs : a.B;
-    return (size_t)N * a.H * BC * a.dk * a.dv * sizeof(float);
+    return (size_t)N * a.H * (a.dk == 16 ? BC : BC / CKP) * a.dk * a.dv * sizeof(float);
 }
 
 cudaError_t launch_scan_bwd(const FwdArgs &a, const BwdArgs &g, bool bf16, cudaStream_t st)
 {
+    if (a.dv % 16 != 0 || a.dv < 16 || a.dv > 128) return cudaErrorInvalidValue;
     switch (a.dk) {
     case 16: return launch_bwd_dv<16>(a, g, bf16, st);
-    case 32: return launch_bwd_dv<32>(a, g, bf16, st);
-    case 64: return launch_bwd_dv<64>(a, g, bf16, st);
-    case 128: return launch_bwd_dv<128>(a, g, bf16, st);
+    case 32: return launch_rows_dv<32>(a, g, bf16, st);
+    case 64: return launch_rows_dv<64>(a, g, bf16, st);
+    case 128: return launch_rows_dv<128>(a, g, bf16, st);
     }
     return cudaErrorInvalidValue;
 }

@@ -82,7 +82,7 @@ def test_bwd_varlen_f32_small_heads(variant):
     _check(inp, _bwd(inp, d_o, dsf), d_o, dsf)
 
 
-@pytest.mark.parametrize("dk,dv", [(16, 128), (128, 16), (32, 64)])
+@pytest.mark.parametrize("dk,dv", [(16, 128), (128, 16), (32, 64), (64, 64)])
 def test_bwd_head_dims_no_initial_state(dk, dv):
     inp = W.make_chunk_inputs("gdn2", "standard", "f32", B=1, T=97, H=2, d_k=dk, d_v=dv, seed=71)
     d_o, _ = W.grad_outputs(inp, seed=71, d_final=False)
