@@ -7,8 +7,10 @@ chunked forward (``kda_chunk_fwd``) over the KDA-range bf16 workload
 B=4, H=16, T=4096, d_k=d_v=128, chunk 64 (seeded inputs, resident in HBM).
 The single-token decode step (256 x 32 heads, d=128, fp32 state 512 MiB in
 place, Complex-KDA range) is timed in the same run and reported under
-"decode".  With --extra the Complex-KDA 8x16x8192 and the RDA / GDN-2 varlen
-workloads are timed too (under "also").
+"decode", and the backward pass (``kda_chunk_bwd``: every gradient of the
+same chunked workload, fp32 arithmetic) under "backward".  With --extra the
+Complex-KDA 8x16x8192 and the RDA / GDN-2 varlen workloads are timed too
+(under "also").
 
 Multi-GPU (torchrun): every rank runs its own independent batch (different
 seed): the work shards over (sequence, head) units with no collective on the
@@ -73,6 +75,21 @@ def decode_algorithmic(N, H, dk, dv, elem=2, variant="kda") -> dict:
 # ---------------------------------------------------------------------------
 # Device helpers
 # ---------------------------------------------------------------------------
+
+# fp32 FMA peak of the SIMT cores: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def backward_algorithmic(inp) -> dict:
+    """Arithmetic of the backward as built, per head-token: the checkpoint scan
+    (u and the state update: 2 d_k d_v FMAs), the replay of each chunk (the same
+    2) and the adjoint step (G += q do^T, the row sums S do, G u, S dS', S du,
+    the column sum k^T G, dS' and G <- Diag(alpha) dS': 7.5 d_k d_v FMAs), i.e.
+    23 d_k d_v flops.  The recomputation of states between stored ones is not
+    counted."""
+    heads_tokens = inp.B * inp.T * inp.H
+    return {"tokens": inp.B * inp.T, "flops": 23.0 * inp.d_k * inp.d_v * heads_tokens}
+
 
 def source_digest(paths) -> str:
     import hashlib
@@ -379,6 +396,36 @@ def run_decode_workload(steps, warmup, world, peaks, rank, N=256, H=32, dk=128, 
 # CPU oracle timing (baseline and reference arm)
 # ---------------------------------------------------------------------------
 
+def run_backward_workload(inp, steps, warmup, world, rank):
+    """kda_chunk_bwd over the chunked workload with seeded d_o and dL/dS_final."""
+    import linear_rnn_delta_b200 as kda
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    d = {n: (None if getattr(inp, n) is None else getattr(inp, n).to(dev)) for n in
+         ("q", "k", "v", "alpha", "g1", "g2")}
+    d_o, dsf = W.grad_outputs(inp, seed=rank_workload_seed(rank))
+    d_o, dsf = d_o.to(dev), dsf.to(dev)
+
+    def step():
+        kda.kda_chunk_bwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"], d_o,
+                          dsf, stream=stream)
+
+    total, per = time_launches(step, steps, warmup, world, stream)
+    total = max_over_ranks(total, world)
+    alg = backward_algorithmic(inp)
+    avg = sum(per) / len(per)
+    tfs = alg["flops"] / avg / 1e12
+    return {"workload": "backward (all gradients) of the KDA-range chunked workload B=4 H=16 T=4096 d=128 bf16 "
+                        "inputs, fp32 arithmetic; seeded d_o ~ N(0,1), dL/dS_final ~ N(0, 0.01)",
+            "value": alg["tokens"] * world * steps / total, "unit": UNIT, "ms_per_step": total / steps * 1e3,
+            "p50_ms": pct(per, 50) * 1e3, "kernels_per_step": 2, "gpu_launches": 2 * steps,
+            "roofline": {"bound": "alu", "achieved": tfs, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                         "frac": tfs / FP32_ALU_TFLOPS, "traffic": None,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz",
+                         "alg_flops_per_launch": alg["flops"],
+                         "kernel": "kda_chunk_bwd: checkpoint scan + cluster adjoint scan timed as one call"}}
+
+
 def oracle_sample_rate(inp, target_s=12.0, threads=0):
     """Tokens/s of the float64 oracle on a bounded sample of the workload:
     whole sequences of a few heads, scaled to the metric's unit (a token is a
@@ -447,6 +494,7 @@ def main():
     ap.add_argument("--extra", action="store_true", help="also time Complex-KDA 8x16x8192 and varlen RDA/GDN-2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--backward-steps", type=int, default=20)
     ap.add_argument("--form", choices=sorted(FORM_FLAGS), default="auto",
                     help="form of the tensor-core chunked path (auto = the library's shape-based choice)")
     args = ap.parse_args()
@@ -466,6 +514,7 @@ def main():
     fflags = FORM_FLAGS[args.form]
     main_res = run_chunk_workload(inp, args.steps, args.warmup, world, peaks, sampler=sampler, flags=fflags)
     decode = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank)
+    backward = run_backward_workload(inp, args.backward_steps, args.warmup, world, rank)
     also = []
     if args.extra:
         prep = lambda: W.make_chunk_inputs("kda", "standard", "bf16", B=4, T=4096, H=16, d_k=128, d_v=128,
@@ -524,6 +573,7 @@ def main():
         "gpu_launches": args.steps * main_res["kernels_per_step"],
         "clocks": main_res["clocks"],
         "decode": decode,
+        "backward": backward,
         "cpu_baseline": cpu and {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
     }
     if also:
