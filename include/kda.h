@@ -210,14 +210,22 @@ int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
  *   d_initial_state [N,H,d_k,d_v] or NULL).
  * Inputs as for kda_chunk_fwd (d_o in the input dtype, [B,T,H,d_v]); no
  * flags (the inputs are the recurrence's own: no logits, normalised keys).
- * The gradient is that of the exact recurrence: an fp32 adjoint scan replays
- * each 64-token chunk forward from an fp32 checkpoint (a forward scan's state
- * snapshots) and walks it backwards (adjoint of one step:
- *   G_{t-1} = Diag(alpha_t) (I - a~_t k_t^T) (G_t + q_t do_t^T)).
- * Token-serial per (sequence, head); far slower than the forward.
+ * Defined by the update equations of the Raon-1-mini-preview discussion page
+ * (the pages give no gradient formulas; training keeping checkpoints and the
+ * chunk/scan intermediates is named on the openarchlab page, section 3).
+ * The gradient is that of the exact recurrence, in fp32 arithmetic (adjoint of
+ * one step: G_{t-1} = Diag(alpha_t) (I - a~_t k_t^T) (G_t + q_t do_t^T)).  Two
+ * launches on `stream`: a token scan stores the fp32 state after every 64
+ * tokens; then a cluster of d_v/32 CTAs per (sequence, head) replays each
+ * chunk from its checkpoint and walks it backwards.  Results are
+ * deterministic (fixed summation order).
  * workspace: caller-owned, 16-byte aligned, at least
  * kda_chunk_bwd_workspace_size(...) bytes: (N + ceil(B*T/64)) * H * d_k * d_v
- * * 4 for the checkpoints plus N * H * 64 * d_k * d_v * 4.
+ * * 4 for the checkpoints plus N * H * 16 * d_k * d_v * 4 (N * H * 64 * d_k *
+ * d_v * 4 at d_k = 16) for the states kept during the replay.
+ * Errors: as kda_chunk_fwd; KDA_ERR_INVALID_ARG also for nonzero flags, a NULL
+ * or misaligned gradient pointer (dg2 only for RDA and GDN-2) or a workspace
+ * that is NULL, misaligned or too small.
  */
 size_t kda_chunk_bwd_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
                                     int has_cu_seqlens, int num_seqs);
