@@ -21,6 +21,11 @@ Three independent formulations, all float64:
 * ``prepare`` -- the optional input preparation (gate activations from
   logits, L2 normalisation of k) in float64, applied before ``recurrence``
   when a problem stores logits or raw keys.
+* ``recurrence_grad`` -- NumPy reverse mode of the step recurrence (every
+  gradient of one sequence and head).
+* ``recurrence_rank2`` -- NumPy rank-2 (DeltaProduct_2-style) steps: the
+  decay once per token, then two erase/write sub-steps with their own keys,
+  values and gates, then the readout.
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against properties
 the pages fix (RDA = KDA when e = w; GDN-2 = RDA for constant vectors;
@@ -383,3 +388,49 @@ def recurrence_grad(variant: str, q, k, v, alpha, g1, g2, initial_state, do, dsf
         dk_ += g1 * dat
         dv_ = g2 * dm
     return {"dq": dq, "dk": dk_, "dv": dv_, "dalpha": da, "dg1": dg1, "dg2": dg2, "ds0": G}
+
+
+def recurrence_rank2(variant: str, q, k, v, alpha, g1, g2=None, cu_seqlens=None, initial_state=None):
+    """Rank-2 steps (two delta-rule transitions composed in one recurrent
+    update, named as prior work in the Complex KDA arXiv abstract), with the
+    channel-wise decay applied once per token, before the first sub-step:
+
+      S <- Diag(alpha_t) S
+      for s in (1, 2):  u = m_{t,s} - S^T a~_{t,s};  S <- S + k_{t,s} u^T
+      o_t = S^T q_t
+
+    (a~, m) per sub-step as in the rank-1 variants.  Layouts: q, alpha
+    [B,T,H,dk]; k [B,T,2,H,dk]; v [B,T,2,H,dv]; g1 [B,T,2,H] (KDA beta, RDA e)
+    or [B,T,2,H,dk] (GDN-2 b); g2 None (KDA), [B,T,2,H] (RDA w) or
+    [B,T,2,H,dv] (GDN-2 w); cu_seqlens optional (B = 1); initial_state
+    [N,H,dk,dv] or None.  Returns (o [B,T,H,dv], final_state [N,H,dk,dv]).
+    Small inputs only (NumPy loop over tokens).
+    """
+    q, k, v, alpha, g1, g2 = (_f64(x) for x in (q, k, v, alpha, g1, g2))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is not None:
+        cu = [int(x) for x in np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens)]
+        seqs = [(0, cu[n], cu[n + 1]) for n in range(len(cu) - 1)]
+    else:
+        seqs = [(b, 0, T) for b in range(B)]
+    s0 = _f64(initial_state)
+    o = np.zeros((B, T, H, dv))
+    sf = np.zeros((len(seqs), H, dk, dv))
+    for n, (b, t0, t1) in enumerate(seqs):
+        S = np.zeros((H, dk, dv)) if s0 is None else s0[n].copy()
+        for t in range(t0, t1):
+            S = alpha[b, t][:, :, None] * S                                 # decay, once per token
+            for sub in range(2):
+                kk, vv = k[b, t, sub], v[b, t, sub]                         # [H, dk], [H, dv]
+                if variant == "kda":
+                    at, m = g1[b, t, sub][:, None] * kk, g1[b, t, sub][:, None] * vv
+                elif variant == "rda":
+                    at, m = g1[b, t, sub][:, None] * kk, g2[b, t, sub][:, None] * vv
+                else:
+                    at, m = g1[b, t, sub] * kk, g2[b, t, sub] * vv
+                u = m - np.einsum("hij,hi->hj", S, at)                      # residual
+                S = S + kk[:, :, None] * u[:, None, :]                      # rank-one write
+            o[b, t] = np.einsum("hij,hi->hj", S, q[b, t])                   # readout after both sub-steps
+        sf[n] = S
+    return o, sf

@@ -430,3 +430,70 @@ def test_recurrence_grad_of_linear_attention_closed_form():
     g = oracle.recurrence_grad("kda", q, k, v, np.ones((T, dk)), np.zeros(T), None, s0, do)
     assert np.allclose(g["dq"], do @ s0.T) and np.allclose(g["ds0"], q.T @ do)
     assert np.allclose(g["dv"], 0) and np.allclose(g["dk"], 0)
+
+
+# ---- rank-2 (DeltaProduct_2-style) steps ----------------------------------------------------
+
+def _rank2_inputs(variant, B=2, T=9, H=2, dk=6, dv=5, seed=51):
+    rng = np.random.default_rng(seed)
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q = rng.standard_normal((B, T, H, dk))
+    k = unit(rng.standard_normal((B, T, 2, H, dk)))
+    v = rng.standard_normal((B, T, 2, H, dv))
+    alpha = np.tanh(rng.standard_normal((B, T, H, dk)))
+    if variant == "gdn2":
+        g1, g2 = rng.uniform(0, 1, (B, T, 2, H, dk)), rng.uniform(0, 1, (B, T, 2, H, dv))
+    else:
+        g1 = rng.uniform(0, 2, (B, T, 2, H))
+        g2 = rng.uniform(0, 1, (B, T, 2, H)) if variant == "rda" else None
+    s0 = rng.standard_normal((B, H, dk, dv))
+    return q, k, v, alpha, g1, g2, s0
+
+
+@pytest.mark.parametrize("variant", ["kda", "rda", "gdn2"])
+def test_rank2_with_silent_second_step_is_rank1(variant):
+    """Second sub-step with zero erase and write gates: exactly the rank-1 recurrence on the first."""
+    q, k, v, alpha, g1, g2, s0 = _rank2_inputs(variant)
+    g1[:, :, 1] = 0
+    if g2 is not None:
+        g2[:, :, 1] = 0
+    o2, s2 = oracle.recurrence_rank2(variant, q, k, v, alpha, g1, g2, initial_state=s0)
+    o1, s1 = oracle.recurrence_arrays(variant, q, k[:, :, 0], v[:, :, 0], alpha, g1[:, :, 0],
+                                      None if g2 is None else g2[:, :, 0], initial_state=s0)
+    assert np.allclose(o2, o1, rtol=1e-12, atol=1e-12) and np.allclose(s2, s1, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("variant", ["kda", "rda", "gdn2"])
+def test_rank2_equals_two_rank1_tokens_without_decay_in_between(variant):
+    """A rank-2 step is two rank-1 steps of the C oracle, the second with alpha = 1, read out after the
+    second; packed documents double their offsets."""
+    q, k, v, alpha, g1, g2, s0 = _rank2_inputs(variant, B=1, T=11)
+    cu = np.array([0, 4, 4, 11])
+    s0 = s0[:1].repeat(3, axis=0) * np.array([1.0, -0.5, 2.0])[:, None, None, None]
+    o2, s2 = oracle.recurrence_rank2(variant, q, k, v, alpha, g1, g2, cu_seqlens=cu, initial_state=s0)
+    B, T, H, dk = q.shape
+    inter = lambda x: x.reshape(B, 2 * T, *x.shape[3:])        # [B,T,2,...] is [B,2T,...] in memory
+    a2 = np.ones((B, T, 2, H, dk))
+    a2[:, :, 0] = alpha
+    q2 = np.stack([np.zeros_like(q), q], axis=2)
+    o1, s1 = oracle.recurrence_arrays(variant, inter(q2), inter(k), inter(v), inter(a2), inter(g1),
+                                      None if g2 is None else inter(g2), cu_seqlens=2 * cu, initial_state=s0)
+    assert np.allclose(o2, o1.reshape(B, T, 2, H, -1)[:, :, 1], rtol=1e-12, atol=1e-12)
+    assert np.allclose(s2, s1, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("a,b", [(0.2, 0.9), (1.1, -0.4)])
+def test_rank2_two_reflections_make_a_rotation(a, b):
+    """beta = 2 on both sub-steps, unit keys at angles a and b, alpha = 1, v = 0: each step applies the
+    Householder reflections H(k1) then H(k2), whose product turns the plane by 2 (b - a); T steps turn
+    the state's rows by 2 T (b - a)."""
+    T = 5
+    k = np.zeros((1, T, 2, 1, 2))
+    k[0, :, 0, 0] = [np.cos(a), np.sin(a)]
+    k[0, :, 1, 0] = [np.cos(b), np.sin(b)]
+    s0 = np.random.default_rng(6).standard_normal((1, 1, 2, 3))
+    _, sf = oracle.recurrence_rank2("kda", np.zeros((1, T, 1, 2)), k, np.zeros((1, T, 2, 1, 3)),
+                                    np.ones((1, T, 1, 2)), np.full((1, T, 2, 1), 2.0), None, initial_state=s0)
+    phi = 2 * T * (b - a)
+    R = np.array([[np.cos(phi), -np.sin(phi)], [np.sin(phi), np.cos(phi)]])
+    assert np.allclose(sf[0, 0], R @ s0[0, 0], rtol=1e-12, atol=1e-12)
