@@ -426,6 +426,25 @@ def run_backward_workload(inp, steps, warmup, world, rank):
                          "kernel": "kda_chunk_bwd: checkpoint scan + cluster adjoint scan timed as one call"}}
 
 
+def run_rank2_workload(inp, steps, warmup, world):
+    """kda_chunk_fwd_rank2 (two sub-steps per token) over a rank-2 workload."""
+    import linear_rnn_delta_b200 as kda
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    d = {n: (None if getattr(inp, n) is None else getattr(inp, n).to(dev)) for n in
+         ("q", "k", "v", "alpha", "g1", "g2")}
+    o = torch.empty((inp.B, inp.T, inp.H, inp.d_v), dtype=d["q"].dtype, device=dev)
+    sf = torch.empty((inp.B, inp.H, inp.d_k, inp.d_v), dtype=torch.float32, device=dev)
+
+    def step():
+        kda.kda_chunk_fwd_rank2(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"],
+                                final_state=sf, o=o, stream=stream)
+
+    total, per = time_launches(step, steps, warmup, world, stream)
+    total = max_over_ranks(total, world)
+    return {"tokens_per_step": inp.B * inp.T, "total_s": total, "avg_launch_s": sum(per) / len(per)}
+
+
 def oracle_sample_rate(inp, target_s=12.0, threads=0):
     """Tokens/s of the float64 oracle on a bounded sample of the workload:
     whole sequences of a few heads, scaled to the metric's unit (a token is a
@@ -536,6 +555,14 @@ def main():
                          "tensor_frac": r["tensor"]["frac"], "achieved_gbs": r["hbm"]["achieved"],
                          "achieved_tflops": r["tensor"]["achieved"]})
             del x
+        x = W.make_rank2_inputs("kda", "standard", "bf16", B=4, T=2048, H=16, d_k=128, d_v=128,
+                                seed=rank_workload_seed(rank))
+        r = run_rank2_workload(x, max(5, args.steps // 2), args.warmup, world)
+        also.append({"workload": "KDA rank-2 steps (two sub-steps per token) B=4 H=16 T=2048 d=128 bf16: "
+                                 "q/alpha expansion + chunked forward over 4096 sub-tokens + o gather",
+                     "value": r["tokens_per_step"] * world * max(5, args.steps // 2) / r["total_s"], "unit": UNIT,
+                     "ms_per_step": r["avg_launch_s"] * 1e3})
+        del x
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample_rate(inp)

@@ -17,7 +17,7 @@ from typing import Optional, Union
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "KdaChunkFunction", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_version",
+__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "KdaChunkFunction", "kda_chunk_fwd_rank2", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_version",
            "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_FORCE_SCAN", "FLAG_FORCE_FUSED",
            "FLAG_FORCE_SPLIT", "FLAG_GATE_LOGITS", "FLAG_L2NORM_K", "num_chunk_slots", "chunk_slot"]
 
@@ -42,7 +42,8 @@ def _load():
                           "(the recurrence has no implementation other than its CUDA kernels)")
     lib = ctypes.CDLL(LIB_PATH)
     for name in ("kda_chunk_fwd", "kda_chunk_fwd_ws", "kda_chunk_fwd_workspace_size", "kda_chunk_bwd",
-                 "kda_chunk_bwd_workspace_size", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_last_error_detail", "kda_version"):
+                 "kda_chunk_bwd_workspace_size", "kda_chunk_fwd_rank2", "kda_chunk_fwd_rank2_workspace_size",
+                 "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_last_error_detail", "kda_version"):
         if not hasattr(lib, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: it is stale, rebuild it with "
                               "`python linear_rnn_delta_b200/build.py`")
@@ -58,6 +59,11 @@ def _load():
                                   [_vp, ctypes.c_size_t, ctypes.c_uint, _vp])
     lib.kda_chunk_bwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_bwd_workspace_size.argtypes = [_i] * 8
+    lib.kda_chunk_fwd_rank2.restype = _i
+    lib.kda_chunk_fwd_rank2.argtypes = ([_i] * 8 + [_vp] * 6 + [_vp, _i, _vp, _vp, _vp, _i, _vp, ctypes.c_size_t,
+                                         ctypes.c_uint, _vp])
+    lib.kda_chunk_fwd_rank2_workspace_size.restype = ctypes.c_size_t
+    lib.kda_chunk_fwd_rank2_workspace_size.argtypes = [_i] * 9 + [ctypes.c_uint]
     lib.kda_decode_step.restype = _i
     lib.kda_decode_step.argtypes = [_i] * 7 + [_vp] * 6 + [_vp, _vp, ctypes.c_uint, _vp]
     lib.kda_check_gates.restype = _i
@@ -279,6 +285,64 @@ class KdaChunkFunction(torch.autograd.Function):
         casts = [None if g is None else g.to(x.dtype)
                  for g, x in zip(grads, (q, k, v, alpha, g1, g2, initial_state))]
         return (None, None, *casts[:6], None, casts[6])
+
+
+def kda_chunk_fwd_rank2(variant: Union[str, int], gate_range: Union[str, int], q: torch.Tensor, k: torch.Tensor,
+                        v: torch.Tensor, alpha: torch.Tensor, g1: torch.Tensor, g2: Optional[torch.Tensor] = None,
+                        cu_seqlens: Optional[torch.Tensor] = None, initial_state: Optional[torch.Tensor] = None,
+                        final_state: Union[torch.Tensor, bool, None] = True, o: Optional[torch.Tensor] = None,
+                        chunk_size: int = 64, flags: int = 0, stream=None):
+    """Rank-2 steps (C: kda_chunk_fwd_rank2): per token the decay alpha_t,
+    then two erase/write sub-steps, then o_t = S_t^T q_t.  q, alpha
+    [B,T,H,d_k]; k [B,T,2,H,d_k]; v [B,T,2,H,d_v]; g1 / g2 with the sub-step
+    axis after T ([B,T,2,H] or GDN-2's [B,T,2,H,d]).  Other arguments as for
+    kda_chunk_fwd (no gate logits).  Returns (o, final_state or None)."""
+    var = _code(VARIANTS, variant, "variant")
+    rng = _code(RANGES, gate_range, "gate_range")
+    if q.dim() != 4 or k.dim() != 5:
+        raise ValueError("q must be [B,T,H,d_k] and k [B,T,2,H,d_k]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"dtype {dt} unsupported (bf16 or fp32)")
+    _check(q, "q", dt, (B, T, H, dk), dev)
+    _check(alpha, "alpha", dt, (B, T, H, dk), dev)
+    _check(k, "k", dt, (B, T, 2, H, dk), dev)
+    _check(v, "v", dt, (B, T, 2, H, dv), dev)
+    _check(g1, "g1", dt, (B, T, 2, H, dk) if var == 2 else (B, T, 2, H), dev)
+    if var != 0:
+        if g2 is None:
+            raise ValueError("RDA and GDN-2 need g2 (write gate)")
+        _check(g2, "g2", dt, (B, T, 2, H, dv) if var == 2 else (B, T, 2, H), dev)
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    _check(initial_state, "initial_state", torch.float32, (N, H, dk, dv), dev)
+    if final_state is True:
+        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    elif final_state is False:
+        final_state = None
+    _check(final_state, "final_state", torch.float32, (N, H, dk, dv), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dt, device=dev)
+    _check(o, "o", dt, (B, T, H, dv), dev)
+    ws_bytes = lib.kda_chunk_fwd_rank2_workspace_size(_DTYPES[dt], B, T, H, dk, dv, int(cu_seqlens is not None), N,
+                                                      int(chunk_size), int(flags))
+    if ws_bytes == 0:
+        raise KdaError(1, "kda_chunk_fwd_rank2_workspace_size")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if stream is not None and stream != torch.cuda.current_stream(dev):
+        ws.record_stream(stream)
+    rc = lib.kda_chunk_fwd_rank2(var, rng, _DTYPES[dt], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                 _ptr(g1), _ptr(g2), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(final_state),
+                                 _ptr(o), int(chunk_size), _ptr(ws), ws_bytes, int(flags), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_chunk_fwd_rank2")
+    return o, final_state
 
 
 def num_chunk_slots(B: int, T: int, N: int) -> int:

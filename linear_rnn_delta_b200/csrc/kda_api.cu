@@ -6,6 +6,7 @@
 
 #include "../../include/kda.h"
 #include "scan_bwd.cuh"
+#include "rank2.cuh"
 
 namespace {
 
@@ -257,6 +258,8 @@ extern "C" int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
 #endif
 }
 
+namespace {
+
 // Backward workspace: the forward's state snapshots (chunk slots) and each
 // CTA's per-chunk states.
 size_t bwd_workspace_bytes(const kda::FwdArgs &a)
@@ -265,6 +268,8 @@ size_t bwd_workspace_bytes(const kda::FwdArgs &a)
     const long long slots = N + ((long long)a.B * a.T + 63) / 64;
     return (size_t)slots * a.H * a.dk * a.dv * sizeof(float) + kda::scan_bwd_scratch_bytes(a);
 }
+
+}  // namespace
 
 extern "C" size_t kda_chunk_bwd_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
                                                int has_cu_seqlens, int num_seqs)
@@ -325,6 +330,104 @@ extern "C" int kda_chunk_bwd(int variant, int gate_range, int dtype,
                    reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + snap_bytes)};
     e = kda::launch_scan_bwd(a, g, bf16, st);
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd launch");
+    return KDA_OK;
+}
+
+namespace {
+
+// Rank-2 steps: workspace regions (256-byte aligned) for the sub-token problem
+// of B x 2T tokens: q2, alpha2 [B,2T,H,d_k], o2 [B,2T,H,d_v], doubled
+// cu_seqlens, then the chunked path's own workspace.
+struct Rank2Layout {
+    size_t q2, a2, o2, cu2, chunk, chunk_bytes, total;
+};
+
+Rank2Layout rank2_layout(int dtype, int B, int T, int H, int d_k, int d_v, int has_cu, int num_seqs, int chunk_size,
+                         unsigned flags)
+{
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    const size_t tok2 = (size_t)B * 2 * (size_t)T * H;
+    Rank2Layout L;
+    L.q2 = 0;
+    L.a2 = up(tok2 * d_k * es);
+    L.o2 = L.a2 + up(tok2 * d_k * es);
+    L.cu2 = L.o2 + up(tok2 * d_v * es);
+    L.chunk = L.cu2 + up(has_cu ? (size_t)(num_seqs + 1) * 4 : 0);
+    L.chunk_bytes = kda_chunk_fwd_workspace_size(dtype, B, 2 * T, H, d_k, d_v, has_cu, num_seqs, chunk_size, flags);
+    L.total = L.chunk + up(L.chunk_bytes);
+    return L;
+}
+
+bool rank2_sizes_ok(int dtype, int B, int T, int H, int d_k, int d_v, int has_cu, int num_seqs)
+{
+    if (B < 1 || T < 0 || T > (1 << 29) || H < 1 || (has_cu && (B != 1 || num_seqs < 1))) return false;
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_F32) return false;
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v)) return false;
+    return (unsigned long long)B * (2ull * (unsigned long long)T) * H * 128ull <= (1ull << 46);
+}
+
+}  // namespace
+
+extern "C" size_t kda_chunk_fwd_rank2_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
+                                                     int has_cu_seqlens, int num_seqs, int chunk_size, unsigned flags)
+{
+    if (!rank2_sizes_ok(dtype, B, T, H, d_k, d_v, has_cu_seqlens, num_seqs)) return 0;
+    if ((flags & KDA_FLAG_FORCE_FUSED) && (flags & KDA_FLAG_FORCE_SPLIT)) return 0;
+    return rank2_layout(dtype, B, T, H, d_k, d_v, has_cu_seqlens, num_seqs, chunk_size, flags).total;
+}
+
+extern "C" int kda_chunk_fwd_rank2(int variant, int gate_range, int dtype,
+                                   int B, int T, int H, int d_k, int d_v,
+                                   const void *q, const void *k, const void *v, const void *alpha,
+                                   const void *g1, const void *g2,
+                                   const int32_t *cu_seqlens, int num_seqs,
+                                   const float *initial_state, float *final_state,
+                                   void *o, int chunk_size, void *workspace, size_t workspace_bytes,
+                                   unsigned flags, void *stream)
+{
+    if (flags & KDA_FLAG_GATE_LOGITS)
+        return fail(KDA_ERR_UNSUPPORTED, "rank-2 steps take gate values, not logits "
+                                         "(the second sub-step's alpha = 1 has no finite logit)");
+    if (B < 1 || T < 0 || H < 1 || T > (1 << 29))
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d (need B>=1, 0<=T<=2^29, H>=1)", B, T, H);
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_F32) return fail(KDA_ERR_INVALID_ARG, "bad dtype %d", dtype);
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "head dims d_k=%d d_v=%d: supported are 16, 32, 64, 128", d_k, d_v);
+    if (!rank2_sizes_ok(dtype, B, T, H, d_k, d_v, cu_seqlens != nullptr, num_seqs))
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d num_seqs=%d (cu_seqlens needs B == 1)", B, T, H,
+                    num_seqs);
+    if (T > 0) {
+        const void *need[] = {q, alpha, o};
+        const char *names[] = {"q", "alpha", "o"};
+        for (int i = 0; i < 3; ++i) {
+            if (!need[i]) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+            if (!aligned16(need[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+        }
+    }
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+    const Rank2Layout L = rank2_layout(dtype, B, T, H, d_k, d_v, cu_seqlens != nullptr, num_seqs, chunk_size, flags);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < L.total)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_fwd_rank2 needs a 16-byte aligned workspace of %zu bytes",
+                    L.total);
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    int32_t *cu2 = cu_seqlens ? reinterpret_cast<int32_t *>(w + L.cu2) : nullptr;
+    // the sub-token problem: k, v and the gates are already [B,2T,H,.]; q, alpha and o live in the workspace
+    kda::FwdArgs a;
+    int rc = chunk_args(a, variant, gate_range, dtype, B, 2 * T, H, d_k, d_v, w + L.q2, k, v, w + L.a2, g1, g2,
+                        cu2, num_seqs, initial_state, final_state, w + L.o2, chunk_size, flags);
+    if (rc != KDA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    const long long tokens = (long long)B * T;
+    cudaError_t e = kda::launch_rank2_expand(bf16, q, alpha, w + L.q2, w + L.a2, tokens, H * d_k, cu_seqlens, cu2,
+                                             cu_seqlens ? num_seqs + 1 : 0, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_rank2 expand");
+    rc = chunk_launch(a, dtype, chunk_size, flags, w + L.chunk, L.chunk_bytes, st);
+    if (rc != KDA_OK) return rc;
+    e = kda::launch_rank2_gather(bf16, w + L.o2, o, tokens, H * d_v, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_rank2 gather");
     return KDA_OK;
 }
 

@@ -170,3 +170,39 @@ def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+# ---- rank-2 steps ---------------------------------------------------------------------------
+
+def test_rank2_workspace_size(lib):
+    # fp32 (token scan: no chunk workspace): q2, alpha2 [1,200,3,64], o2 [1,200,3,32], doubled cu_seqlens
+    up = lambda x: (x + 255) // 256 * 256
+    expect = 2 * up(600 * 64 * 4) + up(600 * 32 * 4) + up(5 * 4)
+    assert lib.kda_chunk_fwd_rank2_workspace_size(1, 1, 100, 3, 64, 32, 1, 4, 64, 0) == expect
+    assert lib.kda_chunk_fwd_rank2_workspace_size(1, 2, 100, 3, 64, 32, 1, 4, 64, 0) == 0    # cu_seqlens, B != 1
+    assert lib.kda_chunk_fwd_rank2_workspace_size(1, 1, -1, 3, 64, 32, 0, 1, 64, 0) == 0
+    assert lib.kda_chunk_fwd_rank2_workspace_size(1, 1, 8, 3, 48, 32, 0, 1, 64, 0) == 0      # d_k = 48
+    assert lib.kda_chunk_fwd_rank2_workspace_size(0, 1, 8, 3, 128, 128, 0, 1, 64, 4 | 8) == 0
+
+
+def r2(lib, **kw):
+    a = dict(variant=0, gate_range=0, dtype=1, B=1, T=8, H=2, dk=64, dv=32, q=P, k=P, v=P, alpha=P, g1=P, g2=None,
+             cu=None, nseq=1, s0=None, sf=None, o=P, chunk=64, ws=P, ws_bytes=0, flags=0, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_fwd_rank2(a["variant"], a["gate_range"], a["dtype"], a["B"], a["T"], a["H"], a["dk"],
+                                   a["dv"], a["q"], a["k"], a["v"], a["alpha"], a["g1"], a["g2"], a["cu"], a["nseq"],
+                                   a["s0"], a["sf"], a["o"], a["chunk"], a["ws"], a["ws_bytes"], a["flags"],
+                                   a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(flags=16), UNSUPPORTED),           # gate logits: the second sub-step's alpha = 1 has none
+    (dict(T=-1), INVALID), (dict(B=0), INVALID), (dict(dtype=7), INVALID), (dict(dk=48), UNSUPPORTED),
+    (dict(q=None), INVALID), (dict(alpha=BAD), INVALID), (dict(o=None), INVALID),
+    (dict(cu=ctypes.c_void_p(0x10002), nseq=1), INVALID),
+    (dict(ws=None), INVALID),                # no workspace
+    (dict(ws_bytes=16), INVALID),            # workspace too small
+])
+def test_rank2_rejects_bad_arguments(lib, kw, code):
+    assert r2(lib, **kw) == code
+    assert len(lib.kda_last_error_detail()) > 0

@@ -189,9 +189,6 @@ def make_chunk_inputs(variant: str = "kda", gate_range: str = "standard", dtype:
                        _cast(g1, dtype), _cast(g2, dtype), cu, s0, chunk_size, logits, raw_k)
 
 
-# ---------------------------------------------------------------------------
-# The named workloads (shapes and distributions of the recurrence's benchmark
-# configurations).  Each returns ChunkInputs; the decode workload is separate.
 def grad_outputs(inp: ChunkInputs, seed: int = 0, d_final: bool = True):
     """Incoming gradients for a backward pass over ``inp``: d_o [B,T,H,d_v]
     ~ N(0,1) in the run dtype and dL/dS_final fp32 [N,H,d_k,d_v] ~ N(0, 0.1^2)
@@ -205,6 +202,44 @@ def grad_outputs(inp: ChunkInputs, seed: int = 0, d_final: bool = True):
     return d_o, dsf
 
 
+@dataclasses.dataclass
+class Rank2Inputs(ChunkInputs):
+    """A rank-2 (two sub-steps per token) problem.  q, alpha [B,T,H,d_k] per
+    token; k [B,T,2,H,d_k], v [B,T,2,H,d_v] and the gates ([B,T,2,H] scalars
+    or [B,T,2,H,d] GDN-2 vectors) carry the sub-step axis after T."""
+
+
+def make_rank2_inputs(variant: str = "kda", gate_range: str = "standard", dtype: str = "bf16",
+                      B: int = 1, T: int = 64, H: int = 2, d_k: int = 16, d_v: int = 16, seed: int = 0,
+                      doc_lens=None, init_state: str = "zero", init_std: float = 0.02) -> Rank2Inputs:
+    """Draw one rank-2 problem with the rank-1 recipe: q, then k and v of both
+    sub-steps, then alpha per token, then the gates per sub-step (same
+    distributions as ``make_chunk_inputs``); keys L2-normalised per sub-step;
+    from ``default_rng((seed, 2))``."""
+    rng = np.random.default_rng((seed, 2))
+    cu = None
+    if doc_lens is not None:
+        doc_lens = [int(x) for x in doc_lens]
+        B, T = 1, int(sum(doc_lens))
+        cu = torch.tensor(np.concatenate([[0], np.cumsum(doc_lens)]).astype(np.int32))
+    q = rng.standard_normal((B, T, H, d_k), dtype=np.float32)
+    k = _l2norm_rows(rng.standard_normal((B, T, 2, H, d_k), dtype=np.float32))
+    v = rng.standard_normal((B, T, 2, H, d_v), dtype=np.float32)
+    alpha, _, _ = _alpha_gates(rng, variant, gate_range, (B, T, H), d_k, d_v)
+    _, g1, g2 = _alpha_gates(rng, variant, gate_range, (B, T, 2, H), d_k, d_v)
+    n_seqs = B if cu is None else len(doc_lens)
+    s0 = None
+    if init_state == "random":
+        s0 = torch.from_numpy(init_std * rng.standard_normal((n_seqs, H, d_k, d_v), dtype=np.float32))
+    elif init_state != "zero":
+        raise ValueError(init_state)
+    return Rank2Inputs(variant, gate_range, dtype, B, T, H, d_k, d_v, _cast(q, dtype), _cast(k, dtype),
+                       _cast(v, dtype), _cast(alpha, dtype), _cast(g1, dtype), _cast(g2, dtype), cu, s0)
+
+
+# ---------------------------------------------------------------------------
+# The named workloads (shapes and distributions of the recurrence's benchmark
+# configurations).  Each returns ChunkInputs; the decode workload is separate.
 # ---------------------------------------------------------------------------
 
 def tiny_ckda(seed: int = 0) -> ChunkInputs:
