@@ -353,6 +353,12 @@ __device__ __forceinline__ void reduce_scatter(float (&x)[L], int lane)
     for (int off = 16 / L; off >= 1; off /= 2) x[0] += __shfl_xor_sync(0xffffffffu, x[0], off);
 }
 
+// Prefetched scalars stay in the input dtype until used: widening a bf16 load
+// right away would wait for the load inside the barrier-delimited region that
+// issued it.
+__device__ __forceinline__ float widen(float x) { return x; }
+__device__ __forceinline__ float widen(__nv_bfloat16 x) { return __bfloat162float(x); }
+
 template <int DK, int DVB, typename TIn>
 __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
 {
@@ -387,7 +393,7 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
         }
     };
     auto tok_of = [&](int t) { return ((size_t)row0 + t) * a.H + h; };
-    auto gate_e = [&](size_t tok) { return vec_gate ? ld_f32(g1 + tok * DK + i) : ld_f32(g1 + tok); };
+    auto gate_raw = [&](size_t tok) { return vec_gate ? g1[tok * DK + i] : g1[tok]; };
     // column sums over the CTA's rows of x (destroyed); returns nothing, leaves the
     // totals in `fin` (this warp's copy) after a CTA barrier and a warp barrier
     unsigned red_count = 0;
@@ -414,33 +420,45 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
     for (int c = nchunks - 1; c >= 0; --c) {
         const int t0 = c * BC, nt = min(BC, len - t0);
         __syncthreads();   // the previous chunk's readers of the staged vectors are done
-        for (int e = i; e < nt * DVB; e += DK) {
-            const int tt = e / DVB, j = e % DVB;
-            const size_t tok = tok_of(t0 + tt);
-            const size_t cj = tok * a.dv + (size_t)jb * DVB + j;
-            float w;
-            if (a.variant == KDA) w = ld_f32(g1 + tok);
-            else if (a.variant == RDA) w = ld_f32(g2 + tok);
-            else w = ld_f32(g2 + cj);
-            sV[e] = ld_f32(v + cj);
-            sW[e] = w;
-            sDO[e] = ld_f32(dO + cj);
+        constexpr int SB = 8;   // elements per thread loaded before any is widened
+        for (int e0 = i; e0 < nt * DVB; e0 += DK * SB) {
+            TIn rv[SB], rw[SB], rd[SB];
+#pragma unroll
+            for (int b = 0; b < SB; ++b) {
+                const int e = e0 + b * DK;
+                if (e < nt * DVB) {
+                    const size_t tok = tok_of(t0 + e / DVB);
+                    const size_t cj = tok * a.dv + (size_t)jb * DVB + e % DVB;
+                    rv[b] = v[cj];
+                    rw[b] = a.variant == KDA ? g1[tok] : (a.variant == RDA ? g2[tok] : g2[cj]);
+                    rd[b] = dO[cj];
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < SB; ++b) {
+                const int e = e0 + b * DK;
+                if (e < nt * DVB) {
+                    sV[e] = widen(rv[b]);
+                    sW[e] = widen(rw[b]);
+                    sDO[e] = widen(rd[b]);
+                }
+            }
         }
         load_row(S, c == 0 ? (a.s0 ? a.s0 + srow : nullptr)
                            : a.snap + (((size_t)(slot_base(a, n) + c - 1) * a.H + h) * DK + i) * a.dv +
                                  (size_t)jb * DVB);
         __syncthreads();
         // ---- replay: u_t into shared memory, S_{t-1} every CKP tokens into scratch
-        float n_al = 0.f, n_k = 0.f, n_e = 0.f;
+        TIn n_al = TIn(0.f), n_k = TIn(0.f), n_e = TIn(0.f);   // next token's row scalars, raw
         if (nt > 0) {
             const size_t tok = tok_of(t0);
-            n_al = ld_f32(al + tok * DK + i); n_k = ld_f32(k + tok * DK + i); n_e = gate_e(tok);
+            n_al = al[tok * DK + i]; n_k = k[tok * DK + i]; n_e = gate_raw(tok);
         }
         for (int tt = 0; tt < nt; ++tt) {
-            const float alpha_i = n_al, k_i = n_k, e_i = n_e;
+            const float alpha_i = widen(n_al), k_i = widen(n_k), e_i = widen(n_e);
             if (tt + 1 < nt) {
                 const size_t tok = tok_of(t0 + tt + 1);
-                n_al = ld_f32(al + tok * DK + i); n_k = ld_f32(k + tok * DK + i); n_e = gate_e(tok);
+                n_al = al[tok * DK + i]; n_k = k[tok * DK + i]; n_e = gate_raw(tok);
             }
             if (tt % CKP == 0) {
 #pragma unroll
@@ -474,19 +492,21 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
         float4 *ckb = reinterpret_cast<float4 *>(smf + L::CKB);   // [2][NQ][DK]: each thread its own row
         float c_al[CKP], c_k[CKP];   // alpha_i, k_i of the current group's tokens (recompute steps)
         float *rsm = smf + L::RSM;   // [CKP][4][DK]: alpha, k, q, e of the group's tokens, own row only
-        float f_al[CKP] = {}, f_k[CKP] = {}, f_q[CKP] = {}, f_e[CKP] = {};   // of the next group (prefetched)
+        TIn f_al[CKP], f_k[CKP], f_q[CKP], f_e[CKP];   // of the next group (prefetched, raw)
+#pragma unroll
+        for (int s = 0; s < CKP; ++s) f_al[s] = f_k[s] = f_q[s] = f_e[s] = TIn(0.f);
         // pass gi fetches group gi - 1 (stored state by cp.async, row scalars into
         // registers) while it works on group gi, fetched by the pass before
         for (int gi = ngrp; gi >= 0; --gi) {
             const int grp = gi, buf = gi & 1;
 #pragma unroll
             for (int s = 0; s < CKP; ++s) {
-                c_al[s] = f_al[s];
-                c_k[s] = f_k[s];
-                rsm[(s * 4 + 0) * DK + i] = f_al[s];
-                rsm[(s * 4 + 1) * DK + i] = f_k[s];
-                rsm[(s * 4 + 2) * DK + i] = f_q[s];
-                rsm[(s * 4 + 3) * DK + i] = f_e[s];
+                c_al[s] = widen(f_al[s]);
+                c_k[s] = widen(f_k[s]);
+                rsm[(s * 4 + 0) * DK + i] = c_al[s];
+                rsm[(s * 4 + 1) * DK + i] = c_k[s];
+                rsm[(s * 4 + 2) * DK + i] = widen(f_q[s]);
+                rsm[(s * 4 + 3) * DK + i] = widen(f_e[s]);
             }
             cp_async_wait_all();
             if (gi > 0) {
@@ -500,10 +520,10 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                 for (int s = 0; s < CKP; ++s) {
                     if (s < fn) {
                         const size_t tok = tok_of(t0 + fg * CKP + s);
-                        f_al[s] = ld_f32(al + tok * DK + i);
-                        f_k[s] = ld_f32(k + tok * DK + i);
-                        f_q[s] = ld_f32(q + tok * DK + i);
-                        f_e[s] = gate_e(tok);
+                        f_al[s] = al[tok * DK + i];
+                        f_k[s] = k[tok * DK + i];
+                        f_q[s] = q[tok * DK + i];
+                        f_e[s] = gate_raw(tok);
                     }
                 }
             }
