@@ -23,6 +23,10 @@ namespace kda {
 namespace {
 
 constexpr int TB = 16;  // tokens staged per barrier
+constexpr int SB = 4;   // elements per thread loaded before any is widened (staging)
+
+__device__ __forceinline__ float widen(float x) { return x; }
+__device__ __forceinline__ float widen(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // PREP: input preparation requested; without it that code is compiled out.
 template <int DK, int DV, typename TIn, bool PREP>
@@ -54,30 +58,61 @@ scan_fwd_kernel(FwdArgs a)
     for (int base = 0; base < len; base += TB) {
         const int nt = min(TB, len - base);
         __syncthreads();  // previous block of tokens fully consumed
-        for (int e = j; e < nt * DK; e += DV) {
-            const int tt = e / DK, i = e % DK;
-            const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
-            const float kk = ld_f32(k + tok * DK + i);
-            float aa = ld_f32(al + tok * DK + i);
-            float g = (a.variant == GDN2) ? ld_f32(g1 + tok * DK + i) : ld_f32(g1 + tok);
-            if (logits) {
-                aa = round_to<TIn>(prep_alpha(aa, ext));
-                g = round_to<TIn>(prep_gate(g, ext));
+        // loads are issued SB elements at a time and widened afterwards: widening
+        // each one as it arrives would wait out every load's latency in turn
+        for (int e0 = j; e0 < nt * DK; e0 += DV * SB) {
+            TIn rk[SB], ra[SB], rg[SB], rq[SB];
+#pragma unroll
+            for (int bb = 0; bb < SB; ++bb) {
+                const int e = e0 + bb * DV;
+                if (e < nt * DK) {
+                    const int tt = e / DK, i = e % DK;
+                    const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
+                    rk[bb] = k[tok * DK + i];
+                    ra[bb] = al[tok * DK + i];
+                    rg[bb] = (a.variant == GDN2) ? g1[tok * DK + i] : g1[tok];
+                    rq[bb] = q[tok * DK + i];
+                }
             }
-            s_k[tt][i] = kk;
-            s_al[tt][i] = aa;
-            s_aa[tt][i] = l2k ? aa * g : aa * (g * kk);   // times k once it is normalised
-            s_q[tt][i] = ld_f32(q + tok * DK + i);
+#pragma unroll
+            for (int bb = 0; bb < SB; ++bb) {
+                const int e = e0 + bb * DV;
+                if (e < nt * DK) {
+                    const int tt = e / DK, i = e % DK;
+                    const float kk = widen(rk[bb]);
+                    float aa = widen(ra[bb]), g = widen(rg[bb]);
+                    if (logits) {
+                        aa = round_to<TIn>(prep_alpha(aa, ext));
+                        g = round_to<TIn>(prep_gate(g, ext));
+                    }
+                    s_k[tt][i] = kk;
+                    s_al[tt][i] = aa;
+                    s_aa[tt][i] = l2k ? aa * g : aa * (g * kk);   // times k once it is normalised
+                    s_q[tt][i] = widen(rq[bb]);
+                }
+            }
         }
-        for (int e = j; e < nt * DV; e += DV) {
-            const int tt = e / DV, jj = e % DV;
-            const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
-            float g;
-            if (a.variant == KDA) g = ld_f32(g1 + tok);
-            else if (a.variant == RDA) g = ld_f32(g2 + tok);
-            else g = ld_f32(g2 + tok * DV + jj);
-            if (logits) g = round_to<TIn>(prep_gate(g, ext));
-            s_m[tt][jj] = g * ld_f32(v + tok * DV + jj);
+        for (int e0 = j; e0 < nt * DV; e0 += DV * SB) {
+            TIn rv[SB], rw[SB];
+#pragma unroll
+            for (int bb = 0; bb < SB; ++bb) {
+                const int e = e0 + bb * DV;
+                if (e < nt * DV) {
+                    const int tt = e / DV, jj = e % DV;
+                    const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
+                    rw[bb] = a.variant == KDA ? g1[tok] : (a.variant == RDA ? g2[tok] : g2[tok * DV + jj]);
+                    rv[bb] = v[tok * DV + jj];
+                }
+            }
+#pragma unroll
+            for (int bb = 0; bb < SB; ++bb) {
+                const int e = e0 + bb * DV;
+                if (e < nt * DV) {
+                    float g = widen(rw[bb]);
+                    if (logits) g = round_to<TIn>(prep_gate(g, ext));
+                    s_m[e / DV][e % DV] = g * widen(rv[bb]);
+                }
+            }
         }
         __syncthreads();
         if (l2k) {   // k_t / ||k_t||, then a~ = (alpha g) (.) k
