@@ -295,11 +295,13 @@ extern "C" int kda_chunk_bwd(int variant, int gate_range, int dtype,
                              float *d_initial_state, void *workspace, size_t workspace_bytes,
                              unsigned flags, void *stream)
 {
+    if (flags) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd takes no flags (got 0x%x)", flags);
+    if (T > 0 && !d_o) return fail(KDA_ERR_INVALID_ARG, "d_o is NULL");
+    // d_o has o's layout and dtype: the forward's checks cover it in o's place
     kda::FwdArgs a;
     int rc = chunk_args(a, variant, gate_range, dtype, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens,
-                        num_seqs, initial_state, nullptr, d_o ? const_cast<void *>(d_o) : workspace, 64, 0u);
+                        num_seqs, initial_state, nullptr, const_cast<void *>(d_o), 64, 0u);
     if (rc != KDA_OK) return rc;
-    if (flags) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd takes no flags (got 0x%x)", flags);
     if (T > 0) {
         const void *need[] = {d_o, dq, dk, dv, dalpha, dg1};
         const char *names[] = {"d_o", "dq", "dk", "dv", "dalpha", "dg1"};

@@ -195,14 +195,55 @@ def r2(lib, **kw):
                                    a["stream"])
 
 
-@pytest.mark.parametrize("kw,code", [
-    (dict(flags=16), UNSUPPORTED),           # gate logits: the second sub-step's alpha = 1 has none
-    (dict(T=-1), INVALID), (dict(B=0), INVALID), (dict(dtype=7), INVALID), (dict(dk=48), UNSUPPORTED),
-    (dict(q=None), INVALID), (dict(alpha=BAD), INVALID), (dict(o=None), INVALID),
-    (dict(cu=ctypes.c_void_p(0x10002), nseq=1), INVALID),
-    (dict(ws=None), INVALID),                # no workspace
-    (dict(ws_bytes=16), INVALID),            # workspace too small
+# As for the backward: the default workspace is too small, and the detail names the check that fired.
+@pytest.mark.parametrize("kw,code,detail", [
+    (dict(flags=16), UNSUPPORTED, b"logits"),   # the second sub-step's alpha = 1 has no logit
+    (dict(T=-1), INVALID, b"T=-1"), (dict(B=0), INVALID, b"B=0"), (dict(dtype=7), INVALID, b"dtype"),
+    (dict(dk=48), UNSUPPORTED, b"d_k=48"),
+    (dict(q=None), INVALID, b"q is NULL"), (dict(alpha=BAD), INVALID, b"alpha"), (dict(o=None), INVALID, b"o is"),
+    (dict(cu=ctypes.c_void_p(0x10002), nseq=1), INVALID, b"cu_seqlens"),
+    (dict(ws=None), INVALID, b"workspace"),
+    (dict(ws_bytes=16), INVALID, b"workspace"),
 ])
-def test_rank2_rejects_bad_arguments(lib, kw, code):
+def test_rank2_rejects_bad_arguments(lib, kw, code, detail):
     assert r2(lib, **kw) == code
-    assert len(lib.kda_last_error_detail()) > 0
+    assert detail in lib.kda_last_error_detail()
+
+
+# ---- backward -------------------------------------------------------------------------------
+
+def test_bwd_workspace_size(lib):
+    # checkpoints: (N + ceil(B*T/64)) slots x H x d_k x d_v fp32, plus N*H*16*d_k*d_v fp32 replay states
+    assert lib.kda_chunk_bwd_workspace_size(0, 2, 100, 3, 128, 128, 0, 2) == \
+        (2 + 4) * 3 * 128 * 128 * 4 + 2 * 3 * 16 * 128 * 128 * 4
+    assert lib.kda_chunk_bwd_workspace_size(1, 1, 10, 1, 16, 32, 1, 3) == \
+        (3 + 1) * 1 * 16 * 32 * 4 + 3 * 1 * 64 * 16 * 32 * 4     # d_k = 16: every state of a chunk
+    assert lib.kda_chunk_bwd_workspace_size(0, 2, 100, 3, 48, 128, 0, 2) == 0
+    assert lib.kda_chunk_bwd_workspace_size(0, 2, 100, 3, 128, 128, 1, 2) == 0   # cu_seqlens needs B == 1
+
+
+def bwd(lib, **kw):
+    a = dict(variant=0, gate_range=0, dtype=0, B=1, T=8, H=2, dk=128, dv=128, q=P, k=P, v=P, alpha=P, g1=P,
+             g2=None, cu=None, nseq=1, s0=None, d_o=P, dsf=None, dq=P, dk_=P, dv_=P, dalpha=P, dg1=P, dg2=None,
+             ds0=None, ws=P, ws_bytes=16, flags=0, stream=None)
+    a.update(kw)
+    return lib.kda_chunk_bwd(a["variant"], a["gate_range"], a["dtype"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                             a["q"], a["k"], a["v"], a["alpha"], a["g1"], a["g2"], a["cu"], a["nseq"], a["s0"],
+                             a["d_o"], a["dsf"], a["dq"], a["dk_"], a["dv_"], a["dalpha"], a["dg1"], a["dg2"],
+                             a["ds0"], a["ws"], a["ws_bytes"], a["flags"], a["stream"])
+
+
+# Every call keeps a far too small workspace, so nothing could launch even if a check were missing;
+# the error detail shows which check fired.
+@pytest.mark.parametrize("kw,code,detail", [
+    (dict(flags=16), INVALID, b"flags"), (dict(d_o=None), INVALID, b"d_o"), (dict(d_o=BAD), INVALID, b"o is not"),
+    (dict(dq=None), INVALID, b"dq"), (dict(dalpha=BAD), INVALID, b"dalpha"),
+    (dict(variant=1, g2=P), INVALID, b"dg2"),        # RDA without dg2
+    (dict(dsf=BAD), INVALID, b"d_final_state"), (dict(ds0=BAD), INVALID, b"d_initial_state"),
+    (dict(dk=48), UNSUPPORTED, b"d_k"), (dict(T=-1), INVALID, b"T=-1"),
+    (dict(ws=None), INVALID, b"workspace"), (dict(ws=BAD), INVALID, b"workspace"),
+    (dict(ws_bytes=16), INVALID, b"workspace"),
+])
+def test_bwd_rejects_bad_arguments(lib, kw, code, detail):
+    assert bwd(lib, **kw) == code
+    assert detail in lib.kda_last_error_detail()
