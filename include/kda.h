@@ -26,8 +26,19 @@
  * stream-ordered and released within the call (kda_chunk_fwd_ws takes it
  * from the caller instead).  Between calls the library keeps only per-device
  * set-up (kernel attributes, SM count, the fixed scratch array of
- * kda_chunk_fwd_noalloc); it is reentrant and thread-safe.  A call returns after the launch: asynchronous kernel faults
- * surface at the caller's next synchronisation, as with any CUDA launch.
+ * kda_chunk_fwd_noalloc); it is reentrant and thread-safe.  A call returns
+ * after the launch: asynchronous kernel faults surface at the caller's next
+ * synchronisation, as with any CUDA launch.
+ *
+ * Entry points.
+ *   kda_chunk_fwd, kda_chunk_fwd_ws, kda_chunk_fwd_noalloc
+ *                           chunked forward over whole sequences (o, final
+ *                           state, optional snapshots every 64 tokens)
+ *   kda_chunk_bwd           every gradient of that forward (fp32)
+ *   kda_chunk_fwd_rank2     two erase/write sub-steps per token
+ *   kda_decode_step         one token per (sequence, head), state in place
+ *   *_workspace_size        bytes of the caller-owned workspace of each call
+ *   kda_check_gates, kda_error_string, kda_last_error_detail, kda_version
  *
  * Errors.  Every entry point validates all arguments on the host before it
  * launches anything; on a bad argument it returns a KDA_ERR_* code and has
