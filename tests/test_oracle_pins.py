@@ -377,8 +377,8 @@ def test_chunk_states_are_prefix_runs():
 
 # ---- gradients ------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("variant,gate_range", [("kda", "standard"), ("kda", "extended"), ("rda", "extended"),
-                                                ("gdn2", "standard")])
+@pytest.mark.parametrize("variant,gate_range", [("kda", "standard"), ("kda", "extended"), ("rda", "standard"),
+                                                ("rda", "extended"), ("gdn2", "standard"), ("gdn2", "extended")])
 def test_recurrence_grad_matches_central_differences(variant, gate_range):
     """Every input's gradient against central differences of the forward oracle (float64)."""
     inp = make_chunk_inputs(variant, gate_range, "f32", B=1, T=7, H=1, d_k=4, d_v=3, seed=43,
