@@ -34,8 +34,10 @@ def _worker(rank, world, port, out):
         seed = bench.rank_workload_seed(rank)
         inp = W.make_chunk_inputs("kda", "extended", "f32", B=2, T=24, H=2, d_k=8, d_v=4, seed=seed)
         o, sf = oracle.recurrence(inp)
-        digest = torch.tensor([float(np.abs(o).sum()), float(np.abs(sf).sum())], dtype=torch.float64)
-        gathered = [torch.zeros(2, dtype=torch.float64) for _ in range(world)]
+        d_o, _ = W.grad_outputs(inp, seed=seed)          # the backward leg's incoming gradient, per rank
+        digest = torch.tensor([float(np.abs(o).sum()), float(np.abs(sf).sum()), float(d_o.abs().sum())],
+                              dtype=torch.float64)
+        gathered = [torch.zeros(3, dtype=torch.float64) for _ in range(world)]
         dist.all_gather(gathered, digest)
         # max over ranks of a per-rank "device time"
         t = bench.max_over_ranks(0.5 + rank, world)
@@ -55,6 +57,7 @@ def test_two_ranks_own_distinct_units_and_agree_on_slowest_time():
     g0, g1 = out[0][1], out[1][1]
     assert g0 == g1                       # everyone saw the same gathered digests
     assert g0[0] != g0[1]                 # ...and the two ranks' units differ
+    assert g0[0][2] != g0[1][2]           # including the backward's incoming gradients
     assert out[0][2] == out[1][2] == 1.5  # max over ranks
 
 
