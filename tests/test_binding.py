@@ -55,3 +55,26 @@ def test_autograd_function_is_exported(kda):
     assert issubclass(kda.KdaChunkFunction, torch.autograd.Function)
     for name in ("kda_chunk_bwd", "kda_chunk_fwd_rank2", "KdaChunkFunction"):
         assert name in kda.__all__
+
+
+def test_chunk_slots_are_unique_increasing_and_in_range(kda):
+    """Slot of chunk c of sequence n (first packed row R_n): n + floor(R_n / 64) + c.  For random packings,
+    every (sequence, chunk) gets its own slot, slots increase within a sequence and stay below
+    num_chunk_slots(B, T, N) = N + ceil(B*T / 64)."""
+    import numpy as np
+    rng = np.random.default_rng(5)
+    for _ in range(200):
+        lens = rng.integers(0, 300, size=int(rng.integers(1, 12)))
+        rows = np.concatenate([[0], np.cumsum(lens)])
+        N, total = len(lens), int(rows[-1])
+        seen = set()
+        for n, ln in enumerate(lens):
+            slots = [kda.chunk_slot(n, c, int(rows[n])) for c in range((int(ln) + 63) // 64)]
+            assert slots == sorted(slots) and len(set(slots)) == len(slots)
+            seen.update(slots)
+            assert all(0 <= s < kda.num_chunk_slots(1, total, N) for s in slots)
+        assert len(seen) == sum((int(ln) + 63) // 64 for ln in lens)
+    # fixed-length batches: sequence n starts at row n*T
+    B, T = 3, 130
+    slots = [kda.chunk_slot(n, c, n * T) for n in range(B) for c in range(3)]
+    assert len(set(slots)) == len(slots) and max(slots) < kda.num_chunk_slots(B, T, B)
