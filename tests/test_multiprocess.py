@@ -49,7 +49,7 @@ def _worker(rank, world, port, out):
 def test_two_ranks_own_distinct_units_and_agree_on_slowest_time():
     world = 2
     port = _free_port()
-    manager = mp.Manager()
+    manager = mp.get_context("spawn").Manager()   # no fork of a process that may hold threads or a CUDA context
     out = manager.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     seeds = [out[r][0] for r in range(world)]
