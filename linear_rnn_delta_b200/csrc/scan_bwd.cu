@@ -16,10 +16,11 @@
 // Both directions act on the columns of S and G independently (the left
 // factors Diag(alpha) and I - k a~^T are shared by all value columns; m_j and
 // do_j touch column j only).  The main kernel (d_k >= 32) therefore splits the
-// d_v columns over a cluster of CTAs, 32 columns each, and gives every thread
-// one row of S and G in registers: sums over columns are in-thread, sums over
-// rows are a warp reduce-scatter plus one CTA barrier.  The per-row results
-// (dq, dk, dalpha, da~) are partial sums over the CTA's columns; the cluster
+// d_v columns over a cluster of CTAs, 32 columns each (16 at d_v = 16), and
+// gives every thread one row of S and G in registers: sums over value columns
+// are in-thread, sums over key rows are a warp reduce-scatter plus one CTA
+// barrier.  The per-row results (dq, dk, dalpha, k (.) da~) are partial sums
+// over the CTA's columns; the cluster
 // adds them through distributed shared memory every 8 tokens, in a fixed order
 // (deterministic results).  The replay keeps S_{t-1} only every 4 tokens
 // (global scratch) with u_t in shared memory; the backward walk recomputes the
