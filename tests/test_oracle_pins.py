@@ -497,3 +497,42 @@ def test_rank2_two_reflections_make_a_rotation(a, b):
     phi = 2 * T * (b - a)
     R = np.array([[np.cos(phi), -np.sin(phi)], [np.sin(phi), np.cos(phi)]])
     assert np.allclose(sf[0, 0], R @ s0[0, 0], rtol=1e-12, atol=1e-12)
+
+
+def test_rank2_gradient_is_the_rank1_reverse_mode_over_sub_tokens():
+    """The gradient of rank-2 steps equals the rank-1 reverse mode over the 2T sub-tokens (the first carries
+    the token's decay and q = 0, the second alpha = 1 and the token's q), mapped back: dq from the second
+    sub-tokens, dalpha from the first; k, v and gate gradients keep the sub-token layout.  Checked against
+    central differences of ``recurrence_rank2``."""
+    rng = np.random.default_rng(21)
+    T, dk, dv = 4, 3, 2
+    q, alpha = rng.standard_normal((T, dk)), np.tanh(rng.standard_normal((T, dk)))
+    k, v = rng.standard_normal((T, 2, dk)), rng.standard_normal((T, 2, dv))
+    g1 = rng.uniform(0, 2, (T, 2))
+    s0, do, dsf = rng.standard_normal((dk, dv)), rng.standard_normal((T, dv)), rng.standard_normal((dk, dv))
+
+    def loss(q_, k_, v_, a_, g_):
+        o, sf = oracle.recurrence_rank2("kda", q_[None, :, None], k_[None, :, :, None], v_[None, :, :, None],
+                                        a_[None, :, None], g_[None, :, :, None], None, initial_state=s0[None, None])
+        return float(np.sum(o[0, :, 0] * do) + np.sum(sf[0, 0] * dsf))
+
+    q2 = np.stack([np.zeros_like(q), q], axis=1).reshape(2 * T, dk)
+    a2 = np.stack([alpha, np.ones_like(alpha)], axis=1).reshape(2 * T, dk)
+    do2 = np.stack([np.zeros_like(do), do], axis=1).reshape(2 * T, dv)
+    g = oracle.recurrence_grad("kda", q2, k.reshape(2 * T, dk), v.reshape(2 * T, dv), a2, g1.reshape(2 * T),
+                               None, s0, do2, dsf)
+    mapped = {"q": g["dq"].reshape(T, 2, dk)[:, 1], "alpha": g["dalpha"].reshape(T, 2, dk)[:, 0],
+              "k": g["dk"].reshape(T, 2, dk), "v": g["dv"].reshape(T, 2, dv), "g1": g["dg1"].reshape(T, 2)}
+    args = {"q": q, "k": k, "v": v, "alpha": alpha, "g1": g1}
+    eps = 1e-6
+    for name, x in args.items():
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            a_p = {**args, name: xp}
+            a_m = {**args, name: xm}
+            fd[idx] = (loss(a_p["q"], a_p["k"], a_p["v"], a_p["alpha"], a_p["g1"])
+                       - loss(a_m["q"], a_m["k"], a_m["v"], a_m["alpha"], a_m["g1"])) / (2 * eps)
+        assert np.allclose(mapped[name], fd, rtol=1e-6, atol=1e-7), name
