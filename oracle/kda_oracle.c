@@ -107,13 +107,15 @@ int oracle_recurrence(int variant, int B, int T, int H, int dk, int dv,
         N = num_seqs;
     }
     long work = (long)N * H;
+    /* the thread count applies to this call only (a num_threads clause, not
+       omp_set_num_threads, which would persist into later calls) */
 #ifdef _OPENMP
-    if (n_threads > 0) omp_set_num_threads(n_threads);
+    const int nt = n_threads > 0 ? n_threads : omp_get_max_threads();
 #else
     (void)n_threads;
 #endif
     int err = 0;
-#pragma omp parallel
+#pragma omp parallel num_threads(nt)
     {
         double *S = (double *)malloc(sizeof(double) * (size_t)dk * dv);
         double *at = (double *)malloc(sizeof(double) * (size_t)dk);
