@@ -323,3 +323,117 @@ def decode_step_inputs(step: int, variant: str = "kda", gate_range: str = "exten
         k = _l2norm_rows(k)
     return DecodeInputs(variant, gate_range, dtype, N, H, d_k, d_v, _cast(q, dtype), _cast(k, dtype),
                         _cast(v, dtype), _cast(alpha, dtype), _cast(g1, dtype), _cast(g2, dtype), logits, raw_k)
+
+
+# ---------------------------------------------------------------------------
+# Planted gates: inputs that force the chunked kernel's division-free
+# (anchored) branch.  That branch serves every chunk in which some channel's
+# chunk product of gates vanishes or underflows; random draws almost never
+# produce one.  Each kind rewrites alpha of an existing problem in place of
+# its draws (same seed -> same planting); nothing else changes.
+# ---------------------------------------------------------------------------
+
+PLANT_KINDS = ("zero", "tiny", "mixed", "negative")
+TINY_GATE = 2.0 ** -6   # 19 such factors already fall below 2^-110; a chunk of 64 underflows fp32
+
+
+def plant_gates(inp: ChunkInputs, kind: str, seed: int = 0, chunk: int = 64) -> ChunkInputs:
+    """A copy of ``inp`` with alpha rewritten so that chosen 64-token chunks
+    of every sequence contain vanishing gates:
+
+    * "zero": alpha = 0 exactly at 3% of the (token, head, channel) entries of
+      every chunk (erases those channels, as the recurrence defines);
+    * "tiny": |alpha| = 2^-6 over whole chunks in 8 channels per head (signs
+      random in the extended range), so their chunk products underflow;
+    * "mixed": "zero" only in the odd chunks of each sequence, so fast and
+      anchored chunks alternate within one sequence;
+    * "negative": runs of 16 tokens with alpha = -1 or -0.999 in a quarter of
+      the channels, plus one exact zero per chunk and head (extended range;
+      in the standard range the runs use +1 and +0.999).
+    Returns a new ChunkInputs; alpha keeps the run dtype (all planted values
+    are bf16-representable except -0.999 / 0.999, rounded like any input)."""
+    if kind not in PLANT_KINDS:
+        raise ValueError(f"unknown planting {kind!r}; expected one of {PLANT_KINDS}")
+    rng = np.random.default_rng((seed, 31))
+    a = inp.alpha.float().numpy().copy()          # [B,T,H,d_k]
+    B, T, H, dk = a.shape
+    ext = inp.gate_range == "extended"
+    starts = []
+    for n in range(inp.num_seqs):
+        b, t0, ln = inp.seq_bounds(n)
+        for c in range((ln + chunk - 1) // chunk):
+            starts.append((b, t0 + c * chunk, min(chunk, ln - c * chunk), c))
+    for b, s, ln, c in starts:
+        blk = a[b, s:s + ln]                       # view [ln, H, d_k]
+        if kind in ("zero", "mixed"):
+            if kind == "mixed" and c % 2 == 0:
+                continue
+            blk[rng.random(blk.shape) < 0.03] = 0.0
+        elif kind == "tiny":
+            for h in range(H):
+                ch = rng.choice(dk, 8, replace=False)
+                sign = rng.choice([-1.0, 1.0], (ln, 8)) if ext else np.ones((ln, 8))
+                blk[:, h, ch] = sign * TINY_GATE
+        else:   # negative
+            mag = np.where(rng.random(blk.shape) < 0.5, 1.0, 0.999)
+            run = np.zeros(blk.shape, dtype=bool)
+            for h in range(H):
+                ch = rng.choice(dk, dk // 4, replace=False)
+                r0 = int(rng.integers(0, max(1, ln - 15)))
+                run[r0:r0 + 16, h, ch] = True
+            blk[run] = ((-1.0 if ext else 1.0) * mag)[run]
+            for h in range(H):
+                blk[int(rng.integers(ln)), h, int(rng.integers(dk))] = 0.0
+    out = dataclasses.replace(inp)
+    out.alpha = _cast(a, inp.dtype)
+    return out
+
+
+def plant_reflections(inp: ChunkInputs, seed: int = 0, chunk: int = 64, every: int = 2) -> ChunkInputs:
+    """A copy of ``inp`` in which every ``every``-th 64-token chunk of each
+    sequence (starting with the first) is rewritten into a run of strong,
+    barely decaying reflections on correlated keys: k_t = normalise(c + 0.05
+    n_t) around one direction c per (sequence, head), |alpha| in [0.97, 1]
+    (random signs in the extended range), and erase gates near their top
+    (beta / e, or every channel of GDN-2's b, in [0.9, 1] x the range's
+    maximum).  The
+    exact result is close to an orthogonal map; the bf16 WY form of such a
+    chunk amplifies its operands' rounding, which is the case the chunked
+    kernel hands to its exact token-by-token path.  Other chunks keep their
+    draws.  Inputs stored as logits (``inp.logits``) get logits of such gates,
+    raw keys (``inp.l2norm_k``) keep a random norm."""
+    rng = np.random.default_rng((seed, 37))
+    k = inp.k.float().numpy().copy()
+    a = inp.alpha.float().numpy().copy()
+    g1 = inp.g1.float().numpy().copy()
+    B, T, H, dk = k.shape
+    ext = inp.gate_range == "extended"
+    top = 2.0 if ext else 1.0
+    for n in range(inp.num_seqs):
+        b, t0, ln = inp.seq_bounds(n)
+        for c in range(0, (ln + chunk - 1) // chunk, every):
+            s, e = t0 + c * chunk, t0 + min(ln, (c + 1) * chunk)
+            L = e - s
+            for h in range(H):
+                cdir = rng.standard_normal(dk)
+                kk = cdir[None, :] + 0.05 * rng.standard_normal((L, dk))
+                kk /= np.linalg.norm(kk, axis=1, keepdims=True)
+                if inp.l2norm_k:
+                    kk *= rng.uniform(0.5, 3.0, (L, 1))
+                k[b, s:e, h] = kk
+                mag = rng.uniform(0.97, 1.0, (L, dk))
+                sign = np.where(rng.random((L, dk)) < 0.3, -1.0, 1.0) if ext else np.ones((L, dk))
+                al = mag * sign
+                if inp.variant == "gdn2":
+                    gate = top * rng.uniform(0.9, 1.0, (L, dk))
+                else:
+                    gate = top * rng.uniform(0.9, 1.0, L)
+                if inp.logits:   # the logits of these gates (the library's activations inverted)
+                    al = np.arctanh(np.clip(al, -0.9999, 0.9999)) if ext else np.log((1.0 - al + 1e-4) / al)
+                    x = gate / top
+                    gate = np.log(x / (1.0 - x + 1e-4))
+                a[b, s:e, h] = al
+                g1[b, s:e, h] = gate
+    out = dataclasses.replace(inp)
+    out.k, out.alpha, out.g1 = _cast(k, inp.dtype), _cast(a, inp.dtype), _cast(g1, inp.dtype)
+    return out
