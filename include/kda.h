@@ -26,9 +26,14 @@
  * stream-ordered and released within the call (kda_chunk_fwd_ws takes it
  * from the caller instead).  Between calls the library keeps only per-device
  * set-up (kernel attributes, SM count, the fixed scratch array of
- * kda_chunk_fwd_noalloc); it is reentrant and thread-safe.  A call returns
- * after the launch: asynchronous kernel faults surface at the caller's next
- * synchronisation, as with any CUDA launch.
+ * kda_chunk_fwd_noalloc) and each device's failure word (kda_device_status).
+ * It is reentrant and thread-safe, with one exception: calls of
+ * kda_chunk_fwd_noalloc share one scratch array, so two of them that overlap
+ * on the GPU race (see there).  A call returns after the launch:
+ * asynchronous kernel faults surface at the caller's next synchronisation, as
+ * with any CUDA launch; a kernel that gives up a bounded wait (or, in the
+ * split form, finds a chunk's operands missing) records it in the device's
+ * failure word, which kda_device_status reads.
  *
  * Entry points.
  *   kda_chunk_fwd, kda_chunk_fwd_ws, kda_chunk_fwd_noalloc
@@ -38,12 +43,16 @@
  *   kda_chunk_fwd_rank2     two erase/write sub-steps per token
  *   kda_decode_step         one token per (sequence, head), state in place
  *   *_workspace_size        bytes of the caller-owned workspace of each call
- *   kda_check_gates, kda_error_string, kda_last_error_detail, kda_version
+ *   kda_check_gates, kda_check_seqlens   device checks of the inputs' contracts
+ *   kda_device_status       failures the kernels recorded on the device
+ *   kda_error_string, kda_last_error_detail, kda_version
  *
  * Errors.  Every entry point validates all arguments on the host before it
  * launches anything; on a bad argument it returns a KDA_ERR_* code and has
  * no side effect.  A failed launch returns KDA_ERR_CUDA (detail in
- * kda_last_error_detail()).
+ * kda_last_error_detail()).  Values that live on the device (gates,
+ * cu_seqlens) are checked only on request: KDA_FLAG_VALIDATE_RANGE, or the
+ * kda_check_* calls.  Device-side failures are reported by kda_device_status.
  */
 #ifndef KDA_H_
 #define KDA_H_
@@ -74,12 +83,25 @@ enum kda_status {
     KDA_OK = 0,
     KDA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, bad cu_seqlens */
     KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dims, chunk size) */
-    KDA_ERR_RANGE = 3,         /* reserved: a gate outside the declared range */
-    KDA_ERR_CUDA = 4           /* a CUDA runtime call or launch failed */
+    KDA_ERR_RANGE = 3,         /* a gate outside the declared range (KDA_FLAG_VALIDATE_RANGE) */
+    KDA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_DEVICE_TIMEOUT = 5 /* kda_device_status: a kernel gave up a bounded wait or found
+                                  a chunk's operands missing; the affected outputs are undefined */
 };
 
-/* Flags.  (Gate ranges are checked on request by kda_check_gates, which
- * writes its verdict to caller memory; the forward calls never check them.) */
+/* Flags. */
+/* KDA_FLAG_VALIDATE_RANGE -- before the work is launched, check on the device
+ * that every gate lies in the declared range (alpha, and beta / e / GDN-2's b,
+ * as kda_check_gates does; NaN fails) and that cu_seqlens keeps its contract
+ * (as kda_check_seqlens does), and WAIT for the verdict: the call then
+ * synchronises `stream`.  A violation returns KDA_ERR_RANGE (gates) or
+ * KDA_ERR_INVALID_ARG (cu_seqlens) and launches nothing.  With
+ * KDA_FLAG_GATE_LOGITS only cu_seqlens is checked (logits have no range).
+ * Accepted by kda_chunk_fwd, kda_chunk_fwd_ws and kda_decode_step.  Without
+ * it no device value is checked: the kernels compute out-of-range gates as
+ * the recurrence defines them, and a cu_seqlens that breaks its contract
+ * makes them read and write out of bounds. */
+#define KDA_FLAG_VALIDATE_RANGE 1u
 #define KDA_FLAG_FORCE_SCAN     2u  /* use the token-by-token CUDA scan kernel even where the
                                        tensor-core chunked kernel applies (testing aid) */
 #define KDA_FLAG_FORCE_FUSED    4u  /* tensor-core path: force the single fused kernel */
@@ -94,6 +116,19 @@ enum kda_status {
  * Both are computed in fp32 from the stored inputs. */
 #define KDA_FLAG_GATE_LOGITS   16u
 #define KDA_FLAG_L2NORM_K      32u
+/* KDA_FLAG_DEBUG_STALL -- testing aid for the failure path (needs
+ * KDA_FLAG_FORCE_SPLIT and the tensor-core path): the chain CTA of
+ * (sequence 0, head 0) never loads its first chunk's operands and gives up
+ * waiting for them after about 1 ms, so that the bounded-wait expiry runs on
+ * demand.  That pair's o is left unwritten and its final state is NaN; every
+ * other pair is computed normally; kda_device_status then reports
+ * KDA_ERR_DEVICE_TIMEOUT with KDA_DEVICE_WAIT_TIMEOUT.  Nothing faults. */
+#define KDA_FLAG_DEBUG_STALL   64u
+
+/* Bits of the device failure word (kda_device_status). */
+#define KDA_DEVICE_WAIT_TIMEOUT 1u  /* a bounded wait inside a kernel ran out (about 2 s) */
+#define KDA_DEVICE_SLOT_MISSING 2u  /* split form: a chunk slot not written by this call's
+                                       preparation kernel */
 
 /*
  * kda_chunk_fwd -- chunked-parallel forward over whole sequences.
@@ -198,8 +233,10 @@ int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
  * library until the process exits.  Problems needing more,
  * (N + ceil(B*T/64)) * H > 809, are rejected with KDA_ERR_UNSUPPORTED.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the array: calls that overlap on the GPU (other
+ * device, with that device current) and keeps it for the life of the
+ * process; make that first call before any stream capture, and do not call
+ * this entry point after cudaDeviceReset on that device (the kept address no
+ * longer names the array there).  All calls share the array: calls that overlap on the GPU (other
  * streams, other host threads) race and give wrong results; calls in order
  * on one stream are safe.  The array's earlier contents never leak into a
  * result (each call tags its slots).
@@ -275,6 +312,34 @@ int kda_decode_step(int variant, int gate_range, int dtype,
  */
 int kda_check_gates(int variant, int gate_range, int dtype, long long n_tok, int d_k,
                     const void *alpha, const void *g1, int *d_count, void *stream);
+
+/*
+ * kda_check_seqlens -- check packed-document offsets on the device: counts
+ * cu_seqlens[0] != 0, each n < num_seqs with cu_seqlens[n+1] < cu_seqlens[n],
+ * and cu_seqlens[num_seqs] != total_tokens (the B*T of the forward call), and
+ * writes the count to the device int `d_count` (caller-owned, overwritten).
+ * cu_seqlens: int32 DEVICE array of num_seqs + 1 entries.  The forward calls
+ * rely on this contract (the "document reset" of the openarchlab page on
+ * GDN/KDA state updates, sec. 3); a batch that breaks it must not be passed
+ * to them.  Asynchronous on `stream`; never traps.
+ */
+int kda_check_seqlens(const int32_t *cu_seqlens, int num_seqs, long long total_tokens, int *d_count,
+                      void *stream);
+
+/*
+ * kda_device_status -- failures the library's kernels recorded on the current
+ * device.  Waits for the work queued on `stream`, then reads and clears the
+ * device's failure word: KDA_OK when it was clear, else KDA_ERR_DEVICE_TIMEOUT
+ * with the KDA_DEVICE_* bits in *bits (when `bits` is not NULL; 0 on
+ * KDA_OK).  The word collects failures of every call on the device since the
+ * previous query, whatever its stream: synchronise other streams first to
+ * attribute theirs.  Failures a kernel records: a bounded mbarrier wait that
+ * ran out (about 2 s; only a broken pipeline gets near it; the kernel then
+ * drains its copies in flight, writes NaN to the final state of its
+ * (sequence, head) and exits), and in the split form a chunk slot that this
+ * call's preparation kernel did not complete.  No kernel traps.
+ */
+int kda_device_status(void *stream, unsigned *bits);
 
 /* Static description of a status code (never NULL). */
 const char *kda_error_string(int code);

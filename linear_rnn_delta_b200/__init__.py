@@ -17,20 +17,26 @@ from typing import Optional, Union
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "KdaChunkFunction", "kda_chunk_fwd_rank2", "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_version",
-           "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_FORCE_SCAN", "FLAG_FORCE_FUSED",
-           "FLAG_FORCE_SPLIT", "FLAG_GATE_LOGITS", "FLAG_L2NORM_K", "num_chunk_slots", "chunk_slot"]
+__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "KdaChunkFunction", "kda_chunk_fwd_rank2", "kda_decode_step",
+           "kda_check_gates", "kda_check_seqlens", "kda_device_status", "kda_error_string", "kda_version",
+           "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_VALIDATE_RANGE", "FLAG_FORCE_SCAN",
+           "FLAG_FORCE_FUSED", "FLAG_FORCE_SPLIT", "FLAG_GATE_LOGITS", "FLAG_L2NORM_K", "FLAG_DEBUG_STALL",
+           "DEVICE_WAIT_TIMEOUT", "DEVICE_SLOT_MISSING", "num_chunk_slots", "chunk_slot"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
 VARIANTS = {"kda": 0, "rda": 1, "gdn2": 2}
 RANGES = {"standard": 0, "extended": 1}
 _DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+FLAG_VALIDATE_RANGE = 1  # check gates and cu_seqlens on the device first (synchronous); refuse on a violation
 FLAG_FORCE_SCAN = 2    # token-by-token CUDA scan even where the tensor-core path applies
 FLAG_FORCE_FUSED = 4   # tensor-core path, single fused kernel
 FLAG_FORCE_SPLIT = 8   # tensor-core path, preparation kernel + chain kernel
 FLAG_GATE_LOGITS = 16  # alpha and gates given as logits; the kernels apply the activations
 FLAG_L2NORM_K = 32     # k given unnormalised; the kernels L2-normalise it per token and head
+FLAG_DEBUG_STALL = 64  # testing aid (with FLAG_FORCE_SPLIT): one chain CTA's first wait runs out
+DEVICE_WAIT_TIMEOUT = 1   # kda_device_status bits
+DEVICE_SLOT_MISSING = 2
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -43,7 +49,8 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     for name in ("kda_chunk_fwd", "kda_chunk_fwd_ws", "kda_chunk_fwd_workspace_size", "kda_chunk_bwd",
                  "kda_chunk_bwd_workspace_size", "kda_chunk_fwd_rank2", "kda_chunk_fwd_rank2_workspace_size",
-                 "kda_decode_step", "kda_check_gates", "kda_error_string", "kda_last_error_detail", "kda_version"):
+                 "kda_decode_step", "kda_check_gates", "kda_check_seqlens", "kda_device_status", "kda_error_string",
+                 "kda_last_error_detail", "kda_version"):
         if not hasattr(lib, name):
             raise ImportError(f"{LIB_PATH} lacks {name}: it is stale, rebuild it with "
                               "`python linear_rnn_delta_b200/build.py`")
@@ -68,6 +75,10 @@ def _load():
     lib.kda_decode_step.argtypes = [_i] * 7 + [_vp] * 6 + [_vp, _vp, ctypes.c_uint, _vp]
     lib.kda_check_gates.restype = _i
     lib.kda_check_gates.argtypes = [_i, _i, _i, ctypes.c_longlong, _i, _vp, _vp, _vp, _vp]
+    lib.kda_check_seqlens.restype = _i
+    lib.kda_check_seqlens.argtypes = [_vp, _i, ctypes.c_longlong, _vp, _vp]
+    lib.kda_device_status.restype = _i
+    lib.kda_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint)]
     lib.kda_error_string.restype = ctypes.c_char_p
     lib.kda_error_string.argtypes = [_i]
     lib.kda_last_error_detail.restype = ctypes.c_char_p
@@ -411,3 +422,31 @@ def kda_check_gates(variant: Union[str, int], gate_range: Union[str, int], alpha
     if rc != 0:
         raise KdaError(rc, "kda_check_gates")
     return int(count.item())
+
+
+def kda_check_seqlens(cu_seqlens: torch.Tensor, total_tokens: int, stream=None) -> int:
+    """Number of violations of the cu_seqlens contract (cu[0] = 0,
+    non-decreasing, cu[N] = total_tokens), counted on the device (C:
+    kda_check_seqlens).  Synchronises the stream to read the count back."""
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+    dev = cu_seqlens.device
+    count = torch.empty((1,), dtype=torch.int32, device=dev)
+    cu = cu_seqlens.contiguous()
+    rc = lib.kda_check_seqlens(_ptr(cu), cu.numel() - 1, int(total_tokens), _ptr(count), _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_check_seqlens")
+    return int(count.item())
+
+
+def kda_device_status(stream=None, device=None):
+    """(status code, failure bits) of the library's kernels on the current
+    device since the previous query (C: kda_device_status): waits for
+    ``stream``, then reads and clears the word.  Code 0 = no failure, 5 =
+    KDA_ERR_DEVICE_TIMEOUT (bits DEVICE_WAIT_TIMEOUT, DEVICE_SLOT_MISSING)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    bits = ctypes.c_uint(0)
+    rc = lib.kda_device_status(_stream(stream, dev), ctypes.byref(bits))
+    if rc not in (0, 5):
+        raise KdaError(rc, "kda_device_status")
+    return rc, int(bits.value)

@@ -1,10 +1,17 @@
-// Device-side check of gate values against the declared range.
+// Device-side checks of the inputs' contracts.
 //
-// KDA range: alpha in (0,1], beta in [0,1]; Complex KDA range: alpha in
-// [-1,1], beta in [0,2] ("Complex KDA" arXiv abstract: gates in [-1,1] and the
-// delta-rule coefficient in [0,2]).  The same intervals are applied to RDA's
-// erase gate e and to GDN-2's erase vector b.  Writes the number of
-// violations (NaN included) to caller memory.
+// Gates against the declared range.  KDA range: alpha in (0,1], beta in
+// [0,1]; Complex KDA range: alpha in [-1,1], beta in [0,2] ("Complex KDA"
+// arXiv abstract: gates in [-1,1] and the delta-rule coefficient in [0,2]).
+// The same intervals are applied to RDA's erase gate e and to GDN-2's erase
+// vector b.  NaN counts as a violation.
+//
+// Packed document offsets (the "document reset" of the openarchlab page on
+// GDN/KDA state updates, sec. 3): cu[0] = 0, cu[n] <= cu[n+1], cu[N] = total.
+//
+// Each check writes a count of violations to device memory and never traps.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace kda {
@@ -32,7 +39,57 @@ __global__ void check_gates_kernel(int variant, int extended, long long n_alpha,
     (void)variant;
 }
 
+// One count per violated condition: cu[0] != 0, each n with cu[n+1] < cu[n], cu[N] != total.
+__global__ void check_seqlens_kernel(const int32_t *cu, int num_seqs, long long total, int *count)
+{
+    int bad = 0;
+    const int stride = gridDim.x * blockDim.x;
+    for (int n = blockIdx.x * blockDim.x + threadIdx.x; n < num_seqs; n += stride)
+        bad += cu[n + 1] < cu[n] ? 1 : 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0)
+        bad += (cu[0] != 0 ? 1 : 0) + ((long long)cu[num_seqs] != total ? 1 : 0);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, off);
+    if ((threadIdx.x & 31) == 0 && bad) atomicAdd(count, bad);
+}
+
+// Counters of the synchronous validation (calls hold the mutex below while they use them).
+__device__ int g_validate_counts[2];
+
 }  // namespace
+
+cudaError_t launch_check_seqlens(const int32_t *cu, int num_seqs, long long total, int *d_count, cudaStream_t st)
+{
+    cudaError_t e = cudaMemsetAsync(d_count, 0, sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    long long blocks = ((long long)num_seqs + 255) / 256;
+    if (blocks > 148 * 8) blocks = 148 * 8;
+    if (blocks < 1) blocks = 1;
+    check_seqlens_kernel<<<(unsigned)blocks, 256, 0, st>>>(cu, num_seqs, total, d_count);
+    return cudaGetLastError();
+}
+
+cudaError_t validate_inputs(int variant, int gate_range, bool bf16, long long n_tok, int dk, const void *alpha,
+                            const void *g1, const int32_t *cu, int num_seqs, long long total, cudaStream_t st,
+                            int *bad_gates, int *bad_seqlens)
+{
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    int *counts = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void **>(&counts), g_validate_counts);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaMemsetAsync(counts, 0, 2 * sizeof(int), st)) != cudaSuccess) return e;
+    if (n_tok > 0 && (e = launch_check_gates(variant, gate_range, bf16, n_tok, dk, alpha, g1, counts, st)) !=
+                         cudaSuccess)
+        return e;
+    if (cu && (e = launch_check_seqlens(cu, num_seqs, total, counts + 1, st)) != cudaSuccess) return e;
+    int h[2] = {0, 0};
+    if ((e = cudaMemcpyAsync(h, counts, sizeof(h), cudaMemcpyDeviceToHost, st)) != cudaSuccess) return e;
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
+    *bad_gates = h[0];
+    *bad_seqlens = h[1];
+    return cudaSuccess;
+}
 
 cudaError_t launch_check_gates(int variant, int gate_range, bool bf16, long long n_tok, int dk,
                                const void *alpha, const void *g1, int *d_count, cudaStream_t st)

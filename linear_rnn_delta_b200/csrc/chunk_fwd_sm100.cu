@@ -115,6 +115,7 @@ struct ChunkParams {
     uint8_t *ws;             // split path: chunk operand slots
     int nslots;              // slots per head
     uint32_t epoch;          // split path: tag of this call's slots
+    int debug_stall;         // split path, testing aid: stall the chain CTA of (sequence 0, head 0)
 };
 
 // ---- split path: per-chunk operand slots in global memory -------------------
@@ -133,6 +134,40 @@ constexpr uint32_t SL_M = 66560;      // GDN-2: M = w (.) v, 128B-swizzled [toke
 constexpr uint32_t SLOT_BYTES = 82944;
 constexpr int META_FAST = 1;          // status word bits
 constexpr int META_OK = 2;
+constexpr int META_EXACT = 4;         // ill-conditioned chunk: the chain runs it token by token
+
+// A chunk is run token by token in fp32 (the exact path below) when the bf16
+// WY form would lose too much to cancellation.  Two signs of it, both from
+// matrices the preparation has in fp32 anyway:
+//  * the UT transform is large: the largest row sum of |T_{r,s}| max(|e_s|,
+//    |w_s|) exceeds EXACT_T_NORM.  Runs of strong, barely decaying
+//    reflections on correlated keys (erase gates near 2) do this; their exact
+//    result is close to an orthogonal map (the 2D rotation of the Complex KDA
+//    abstract), and the rounding of T, W and U reaches the state through
+//    K^T T (.) with no decay to damp it.
+//  * the tokens of the chunk interact strongly: the largest row sum of |A|
+//    (A_{r,s} = e_r sum_c k_{r,c} Lam_{r,s,c} k_{s,c}) exceeds EXACT_A_NORM.
+//    Aligned keys with little decay (erase gates near 1) make each token
+//    overwrite what the previous ones wrote; the readout and the state update
+//    then sum many nearly cancelling terms, and every bf16 rounding point
+//    (operands, P, U) shows in the result.
+// Random chunks of the benchmark recipes stay below 3.1 and 0.9; in emulation
+// of the kernel's rounding, adversarial chunks under both bounds stay within
+// the bf16 tolerance (worst 0.014 of the 0.02 bound).
+constexpr float EXACT_T_NORM = 6.f;
+constexpr float EXACT_A_NORM = 3.f;
+
+// Device-side failure word of this library on each device: bits are OR-ed in
+// by any CTA whose bounded wait ran out or whose input slot was not prepared,
+// and read (and cleared) by kda_device_status.
+__device__ unsigned int g_device_status;
+constexpr unsigned DEV_WAIT_TIMEOUT = 1u, DEV_SLOT_MISSING = 2u;
+__device__ __forceinline__ void report_device_failure(unsigned bits) { atomicOr(&g_device_status, bits); }
+
+// Test-only stall (KDA_FLAG_DEBUG_STALL): the chain CTA of (sequence 0, head 0)
+// does not load its first slot and gives up waiting for it after this many
+// cycles (~1 ms), so that the bounded-wait expiry path runs on demand.
+constexpr long long STALL_WAIT_CYCLES = 1ll << 21;
 
 
 // One chunk of work for the preparation role.
@@ -497,6 +532,182 @@ __device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const floa
     }
 }
 
+// ---- exact path for ill-conditioned chunks ------------------------------------
+// The raw inputs of one chunk, rows 0 .. nv-1 (64 x 128 bf16 each, row-major),
+// copied to shared memory with the input preparation applied as the
+// preparation kernel applies it (alpha activated and k normalised, both
+// rounded to bf16); rows past nv are not written.  All `nthreads` threads
+// from `tid` take part; the caller synchronises afterwards.
+__device__ __forceinline__ void stage_exact_inputs(const FwdArgs &a, size_t tok0, int nv, int h, uint8_t *dq,
+                                                   uint8_t *dk, uint8_t *da, int tid, int nthreads)
+{
+    const int H = a.H;
+    const uint4 *gq = reinterpret_cast<const uint4 *>(a.q), *gk = reinterpret_cast<const uint4 *>(a.k),
+                *ga = reinterpret_cast<const uint4 *>(a.alpha);
+    const bool logits = (a.prep & PREP_LOGITS) != 0, l2k = (a.prep & PREP_L2NORM_K) != 0, ext = a.ext != 0;
+    // four threads per row (adjacent lanes), 32 channels (four 16-byte pieces) each; every lane of
+    // a warp runs the same iterations (nthreads is a multiple of 32), so the row sums can shuffle
+    for (int base = 0; base < nv * 4; base += nthreads) {
+        const int e = base + tid;
+        const bool act = e < nv * 4;
+        const int r = e >> 2, part = e & 3;
+        const size_t g = ((tok0 + r) * H + h) * (D / 8) + part * 4;
+        uint4 qv[4], kv[4], av[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            qv[j] = act ? gq[g + j] : make_uint4(0, 0, 0, 0);
+            kv[j] = act ? gk[g + j] : make_uint4(0, 0, 0, 0);
+            av[j] = act ? ga[g + j] : make_uint4(0, 0, 0, 0);
+        }
+        if (logits) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float f[8];
+                unpack8(av[j], f);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) f[c] = prep_alpha(f[c], ext);
+                av[j] = pack8(f);
+            }
+        }
+        if (l2k) {
+            float ss = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float f[8];
+                unpack8(kv[j], f);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) ss = fmaf(f[c], f[c], ss);
+            }
+            ss += __shfl_xor_sync(0xffffffffu, ss, 1);   // the row's four threads are adjacent lanes
+            ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+            const float sc = prep_kscale(ss);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float f[8];
+                unpack8(kv[j], f);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) f[c] *= sc;
+                kv[j] = pack8(f);
+            }
+        }
+        if (act) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                reinterpret_cast<uint4 *>(dq + r * 256)[part * 4 + j] = qv[j];
+                reinterpret_cast<uint4 *>(dk + r * 256)[part * 4 + j] = kv[j];
+                reinterpret_cast<uint4 *>(da + r * 256)[part * 4 + j] = av[j];
+            }
+        }
+    }
+}
+
+// The recurrence of one chunk token by token, in fp32, on the state in TMEM
+// (lane j = value column j, column i = key channel i): per token
+//   S' = Diag(alpha) S,  u = m - S'^T a~,  S = S' + k u^T,  o = S^T q = S'^T q + (k . q) u.
+// The calling thread owns value column jcol and key channels [i0, i0 + 32 NP)
+// at TMEM address `tstate` (its lane, column 0 of S).  With PAIR the other
+// channels of the column belong to the thread of the other warp of the same
+// TMEM lane quarter; the two add their partial sums through `xch`
+// (float4 [2][2][128]) and named barrier `bar_id` (64 threads).  q, k, alpha
+// rows come from the staging tiles (row-major [64][128] bf16, prepared);
+// v, the gates and GDN-2's erase vector are read from global memory (and
+// activated here when they are logits).  o_t,j goes to bf16 element
+// ost[t * ost_stride + jcol] (a staging tile or o itself) when `write_o`.
+// Every warp of the caller runs the same token loop (the TMEM accesses are
+// warp-wide).
+template <int NP, bool PAIR>
+__device__ __noinline__ void exact_chunk(const FwdArgs &a, uint32_t tstate, int i0, int jcol, int half,
+                                         const uint8_t *sq, const uint8_t *sk, const uint8_t *sa, size_t tok0,
+                                         int nv, int h, float4 *xch, uint32_t bar_id, unsigned short *ost,
+                                         size_t ost_stride, bool write_o)
+{
+    const int H = a.H;
+    const __nv_bfloat16 *g1 = (const __nv_bfloat16 *)a.g1, *g2 = (const __nv_bfloat16 *)a.g2,
+                        *vv = (const __nv_bfloat16 *)a.v;
+    const bool gdn2 = a.variant == GDN2, logits = (a.prep & PREP_LOGITS) != 0, ext = a.ext != 0;
+    auto gate = [&](float x) { return logits ? round_bf16(prep_gate(x, ext)) : x; };
+#pragma unroll 1
+    for (int t = 0; t < nv; ++t) {
+        const size_t tok = (tok0 + t) * H + h;
+        float e, m;
+        const float vj = __bfloat162float(vv[tok * D + jcol]);
+        if (gdn2) {
+            e = 1.f;
+            m = gate(__bfloat162float(g2[tok * D + jcol])) * vj;
+        } else {
+            e = gate(__bfloat162float(g1[tok]));
+            m = (a.variant == KDA ? e : gate(__bfloat162float(g2[tok]))) * vj;
+        }
+        const uint4 *qr = reinterpret_cast<const uint4 *>(sq + t * 256);
+        const uint4 *kr = reinterpret_cast<const uint4 *>(sk + t * 256);
+        const uint4 *ar = reinterpret_cast<const uint4 *>(sa + t * 256);
+        const uint4 *br = gdn2 ? reinterpret_cast<const uint4 *>(g1 + tok * D) : nullptr;
+        float pk = 0.f, pq = 0.f, pkq = 0.f;
+#pragma unroll 1
+        for (int p = 0; p < NP; ++p) {
+            const int c0 = i0 + 32 * p;
+            float s[32];
+            tmem_ld32(tstate + c0, s);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+                float qf[8], kf[8], af[8];
+                unpack8(qr[c0 / 8 + j8], qf);
+                unpack8(kr[c0 / 8 + j8], kf);
+                unpack8(ar[c0 / 8 + j8], af);
+                if (gdn2) {   // erase direction b (.) k
+                    float bf[8];
+                    unpack8(br[c0 / 8 + j8], bf);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float sp = af[c] * s[j8 * 8 + c];
+                        pk = fmaf(gate(bf[c]) * kf[c], sp, pk);
+                        pq = fmaf(qf[c], sp, pq);
+                        pkq = fmaf(qf[c], kf[c], pkq);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float sp = af[c] * s[j8 * 8 + c];
+                        pk = fmaf(kf[c], sp, pk);
+                        pq = fmaf(qf[c], sp, pq);
+                        pkq = fmaf(qf[c], kf[c], pkq);
+                    }
+                }
+            }
+        }
+        if (PAIR) {
+            float4 *mine = xch + (t & 1) * 256;
+            mine[half * 128 + jcol] = make_float4(pk, pq, pkq, 0.f);
+            group_sync(bar_id, 64);
+            const float4 o4 = mine[(half ^ 1) * 128 + jcol];
+            pk += o4.x;
+            pq += o4.y;
+            pkq += o4.z;
+        }
+        const float u = m - e * pk;
+        if (write_o) ost[t * ost_stride + jcol] = bf16_bits(fmaf(pkq, u, pq));
+#pragma unroll 1
+        for (int p = 0; p < NP; ++p) {
+            const int c0 = i0 + 32 * p;
+            float s[32];
+            tmem_ld32(tstate + c0, s);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+                float kf[8], af[8];
+                unpack8(kr[c0 / 8 + j8], kf);
+                unpack8(ar[c0 / 8 + j8], af);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) s[j8 * 8 + c] = fmaf(kf[c], u, af[c] * s[j8 * 8 + c]);
+            }
+            tmem_st16(tstate + c0, s);
+            tmem_st16(tstate + c0 + 16, s + 16);
+        }
+        tmem_wait_st();
+    }
+}
+
 // ---- the kernel -------------------------------------------------------------
 // Warp roles.  Warps 0-3 (CHAIN, 128 threads) own the state: for chunk n they
 // scale S by Gamma_C and copy it to bf16, run U^T -= S^T W^T, O^T = S^T Q^T,
@@ -590,87 +801,113 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             const size_t rowbase = (size_t)seq_row0(a, n) + ch * C;
             if (!mbar_wait_cycles(bar_ready, par, WAIT_CYCLES)) ok = false;
             tc_fence_after();
-            const bool fast = s_fast[par] != 0;
-            const float *gamC = s_gamC + par * 128;
-            // ---- state pass: S^T *= Gamma_C in TMEM; bf16 operand copy (scaled on the fast path)
+            const int cflags = s_fast[par];
+            unsigned short *ost = reinterpret_cast<unsigned short *>(sm + OFF_UT);   // o staging [r][j]
+            const bool exact = ok && (cflags & META_EXACT);
+            if (exact) {
+                // ---- exact path: this chunk token by token in fp32.  None of its prepared operands
+                // is read, so they are released at once; q and k are staged in the state-operand
+                // tile, alpha in the U^T tile (the chain's own shared memory), and o goes straight
+                // to HBM.
+                if (tid == 0) {
+                    mbar_arrive(bar_s6);
+                    mbar_arrive(bar_ufree);
+                    mbar_arrive(bar_s7);
+                }
+                uint8_t *stq = sm + OFF_S0T, *stk = sm + OFF_S0T + 16384, *sta = sm + OFF_UT;
+                stage_exact_inputs(a, rowbase, nvalid, h, stq, stk, sta, tid, NCHAIN);
+                group_sync(BAR_CHAIN, NCHAIN);
+                exact_chunk<4, false>(a, tbase + lane_base + TM_S, 0, jcol, 0, stq, stk, sta, rowbase, nvalid, h,
+                                      nullptr, 0, reinterpret_cast<unsigned short *>(op) + (rowbase * H + h) * D,
+                                      (size_t)H * D, true);
+                tc_fence_before();
+                group_sync(BAR_CHAIN, NCHAIN);
+                tc_fence_after();
+                if (a.snap) snapshot_state(a, tbase + lane_base, slot_base(a, n) + ch, h, 0, 4, jcol);
+            } else {
+                const bool fast = (cflags & META_FAST) != 0;
+                const float *gamC = s_gamC + par * 128;
+                // ---- state pass: S^T *= Gamma_C in TMEM; bf16 operand copy (scaled on the fast path)
 #pragma unroll 1
-            for (int c32 = 0; c32 < 4; ++c32) {
-                const int i0 = c32 * 32;
-                float s[32], t[32];
-                tmem_ld32(tbase + lane_base + TM_S + i0, s);
-                tmem_wait_ld();
+                for (int c32 = 0; c32 < 4; ++c32) {
+                    const int i0 = c32 * 32;
+                    float s[32], t[32];
+                    tmem_ld32(tbase + lane_base + TM_S + i0, s);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    t[e] = s[e] * gamC[i0 + e];
-                    if (fast) s[e] = t[e];
+                    for (int e = 0; e < 32; ++e) {
+                        t[e] = s[e] * gamC[i0 + e];
+                        if (fast) s[e] = t[e];
+                    }
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
+                    tmem_st16(tbase + lane_base + TM_S + i0, t);
+                    tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
                 }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_S0T + sw_chunk(16384, jcol, (i0 >> 3) + q4)) = pack8(s + q4 * 8);
-                tmem_st16(tbase + lane_base + TM_S + i0, t);
-                tmem_st16(tbase + lane_base + TM_S + i0 + 16, t + 16);
-            }
-            tmem_wait_st();
-            fence_async_smem();
-            tc_fence_before();
-            group_sync(BAR_CHAIN, NCHAIN);
-            // ---- step 6: U^T -= S^T W^T ; O^T = S^T Q^T
-            if (tid == 0) {
+                tmem_wait_st();
+                fence_async_smem();
+                tc_fence_before();
+                group_sync(BAR_CHAIN, NCHAIN);
+                // ---- step 6: U^T -= S^T W^T ; O^T = S^T Q^T
+                if (tid == 0) {
+                    tc_fence_after();
+                    step6_mmas(tbase, sb + OFF_S0T, sb + OFF_QA);
+                    mma_commit(bar_s6);
+                }
+                if (!mbar_wait_cycles(bar_s6, par, WAIT_CYCLES)) ok = false;
                 tc_fence_after();
-                step6_mmas(tbase, sb + OFF_S0T, sb + OFF_QA);
-                mma_commit(bar_s6);
-            }
-            if (!mbar_wait_cycles(bar_s6, par, WAIT_CYCLES)) ok = false;
-            tc_fence_after();
-            // ---- U^T row j -> bf16 K-major tile (rows j, K = token); then release TMEM U
+                // ---- U^T row j -> bf16 K-major tile (rows j, K = token); then release TMEM U
 #pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
-                float v[32];
-                tmem_ld32(tbase + lane_base + TM_U + c32 * 32, v);
-                tmem_wait_ld();
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    float v[32];
+                    tmem_ld32(tbase + lane_base + TM_U + c32 * 32, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(sm + OFF_UT + sw_chunk(16384, jcol, c32 * 4 + q4)) = pack8(v + q4 * 8);
-            }
-            fence_async_smem();
-            tc_fence_before();
-            group_sync(BAR_CHAIN, NCHAIN);
-            // ---- step 7: O^T += U^T P^T ; S^T += U^T Kbar
-            if (tid == 0) {
-                mbar_arrive(bar_ufree);
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4 *>(sm + OFF_UT + sw_chunk(16384, jcol, c32 * 4 + q4)) = pack8(v + q4 * 8);
+                }
+                fence_async_smem();
+                tc_fence_before();
+                group_sync(BAR_CHAIN, NCHAIN);
+                // ---- step 7: O^T += U^T P^T ; S^T += U^T Kbar
+                if (tid == 0) {
+                    mbar_arrive(bar_ufree);
+                    tc_fence_after();
+                    const uint32_t id_o = idesc_bf16(128, 64, false, false);
+                    const uint32_t id_s = idesc_bf16(128, 128, false, true);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        mma_bf16(tbase + TM_O, dK(sb + OFF_UT, 16384, kk), dK(sb + OFF_PBF, 8192, kk), id_o, 1);
+                        mma_bf16(tbase + TM_S, dK(sb + OFF_UT, 16384, kk), dMN(sb + OFF_KB, 8192, kk), id_s, 1);
+                    }
+                    mma_commit(bar_s7);
+                }
+                if (!mbar_wait_cycles(bar_s7, par, WAIT_CYCLES)) ok = false;
                 tc_fence_after();
-                const uint32_t id_o = idesc_bf16(128, 64, false, false);
-                const uint32_t id_s = idesc_bf16(128, 128, false, true);
+                if (a.snap) snapshot_state(a, tbase + lane_base, slot_base(a, n) + ch, h, 0, 4, jcol);
+                // ---- o: TMEM (lane j, column r) -> bf16 staging [r][j] in the U^T slot -> HBM
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    mma_bf16(tbase + TM_O, dK(sb + OFF_UT, 16384, kk), dK(sb + OFF_PBF, 8192, kk), id_o, 1);
-                    mma_bf16(tbase + TM_S, dK(sb + OFF_UT, 16384, kk), dMN(sb + OFF_KB, 8192, kk), id_s, 1);
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    float v[32];
+                    tmem_ld32(tbase + lane_base + TM_O + c32 * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const uint32_t pk = pack_bf16(v[e], v[e + 1]);
+                        ost[(c32 * 32 + e) * 128 + jcol] = (unsigned short)(pk & 0xFFFFu);
+                        ost[(c32 * 32 + e + 1) * 128 + jcol] = (unsigned short)(pk >> 16);
+                    }
                 }
-                mma_commit(bar_s7);
-            }
-            if (!mbar_wait_cycles(bar_s7, par, WAIT_CYCLES)) ok = false;
-            tc_fence_after();
-            if (a.snap) snapshot_state(a, tbase + lane_base, slot_base(a, n) + ch, h, 0, 4, jcol);
-            // ---- o: TMEM (lane j, column r) -> bf16 staging [r][j] in the U^T slot -> HBM
-            unsigned short *ost = reinterpret_cast<unsigned short *>(sm + OFF_UT);
-#pragma unroll
-            for (int c32 = 0; c32 < 2; ++c32) {
-                float v[32];
-                tmem_ld32(tbase + lane_base + TM_O + c32 * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const uint32_t pk = pack_bf16(v[e], v[e + 1]);
-                    ost[(c32 * 32 + e) * 128 + jcol] = (unsigned short)(pk & 0xFFFFu);
-                    ost[(c32 * 32 + e + 1) * 128 + jcol] = (unsigned short)(pk >> 16);
-                }
-            }
+            }   // normal (tensor-core) chunk
             tc_fence_before();
             group_sync(BAR_CHAIN, NCHAIN);
-            for (int e = tid; e < nvalid * 16; e += NCHAIN) {
-                const int r = e >> 4, cgo = e & 15;
-                *reinterpret_cast<uint4 *>(op + (((rowbase + r) * H + h) * D + cgo * 8) * 2) =
-                    *reinterpret_cast<const uint4 *>(sm + OFF_UT + r * 256 + cgo * 16);
+            if (!exact) {   // the exact path wrote o itself
+                for (int e = tid; e < nvalid * 16; e += NCHAIN) {
+                    const int r = e >> 4, cgo = e & 15;
+                    *reinterpret_cast<uint4 *>(op + (((rowbase + r) * H + h) * D + cgo * 8) * 2) =
+                        *reinterpret_cast<const uint4 *>(sm + OFF_UT + r * 256 + cgo * 16);
+                }
             }
             ok = group_sync_and(BAR_CHAIN, NCHAIN, ok);   // staging read before the next U^T write
         }
@@ -710,6 +947,11 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             fence_async_smem();
             tc_fence_before();
             group_sync(BAR_PREP, NPREP);
+        };
+        auto publish_and = [&](bool pred) {   // publish, and the AND of pred over the group
+            fence_async_smem();
+            tc_fence_before();
+            return group_sync_and(BAR_PREP, NPREP, pred);
         };
         // scalar gates of row r of a chunk into the gate arrays of item parity `parity`
         // (0 past the chunk's end; GDN-2 keeps its gates channel-wise: 1 here)
@@ -899,7 +1141,6 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                 for (int c = 0; c < 4; ++c) gam_ok = gam_ok && (fabsf(gc[c]) >= FAST_MIN_GAMMA);
             }
             const bool fast = group_sync_and(BAR_PREP, NPREP, gam_ok) && in_range;
-            if (ptid == 0) s_fast[par] = fast ? 1 : 0;
 
             // the previous chunk's chain must be done with QA (step 6) and with Kbar / P (step 7)
             if (!SPLIT && ch > 0) {
@@ -1239,21 +1480,34 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             // ===== 4. W = T Diag(e) (row operand a~ part);  U'^T = M^T (T Diag(w))^T ==
             // T copies go through one bf16 tile: T Diag(e) for W, then (RDA only, whose two
             // gates differ) T Diag(w) for U' once the W GEMM has read the first copy.
+            // Also returns whether row r stays within both bounds of the exact path: its sum of
+            // |T_{r,s}| max(|e_s|, |w_s|) and its sum of |A_{r,s}| (the four threads of a row are
+            // adjacent lanes).
             auto write_t_copy = [&](const float *gate) {
                 const int r = ptid >> 2, kc0 = (ptid & 3) * 2;
+                float tsum = 0.f, asum = 0.f;
 #pragma unroll
                 for (int q2 = 0; q2 < 2; ++q2) {
                     float te[8];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const int s = (kc0 + q2) * 8 + c;
-                        te[c] = (s <= r) ? Tf[r * TP + s] * gate[s] : 0.f;
+                        const float t = (s <= r) ? Tf[r * TP + s] : 0.f;
+                        te[c] = t * gate[s];
+                        tsum += fabsf(t) * fmaxf(fabsf(s_g1[s]), fabsf(s_g2[s]));
+                        asum += fabsf(Af[r * TP + s]);   // zero on and above the diagonal
                     }
                     *reinterpret_cast<uint4 *>(sm + OFF_TBF + sw_chunk(8192, r, kc0 + q2)) = pack8(te);
                 }
+#pragma unroll
+                for (int m = 1; m <= 2; m <<= 1) {
+                    tsum += __shfl_xor_sync(0xffffffffu, tsum, m);
+                    asum += __shfl_xor_sync(0xffffffffu, asum, m);
+                }
+                return tsum <= EXACT_T_NORM && asum <= EXACT_A_NORM;
             };
-            write_t_copy(s_g1);
-            publish();
+            // an ill-conditioned chunk is run token by token by the chain instead (exact path)
+            const bool exact = !publish_and(write_t_copy(s_g1));
             // U'^T overwrites TMEM U: the chain must have read the previous chunk's U out
             // (the split kernel leaves U' to the chain kernel and stores T Diag(w) instead)
             if (!SPLIT && ch > 0 && !mbar_wait_cycles(bar_ufree, ppar, WAIT_CYCLES)) ok = false;
@@ -1302,13 +1556,16 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             }
             if (SPLIT && ptid == 0) {   // status word and epoch tag of the slot
                 int *meta = reinterpret_cast<int *>(sm + OFF_UT);
-                meta[128] = META_OK | (fast ? META_FAST : 0);
+                meta[128] = META_OK | (fast ? META_FAST : 0) | (exact ? META_EXACT : 0);
                 meta[129] = (int)P.epoch;
             }
             fence_async_smem();
             tc_fence_before();
             ok = group_sync_and(BAR_PREP, NPREP, ok);
-            if (!SPLIT && ptid == 0) mbar_arrive(bar_ready);   // chunk ch's operands are ready for the chain
+            if (!SPLIT && ptid == 0) {   // chunk ch's operands are ready for the chain
+                s_fast[par] = (fast ? META_FAST : 0) | (exact ? META_EXACT : 0);
+                mbar_arrive(bar_ready);
+            }
             if (SPLIT && ok && lane == 0 && pw < 5) {   // the rest of the slot, one bulk store per warp
                 uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
                 if (pw == 0) bulk_store(slot + SL_QA, sm + OFF_QA, 8192);                     // -W', panel 0
@@ -1330,10 +1587,12 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
         if (SPLIT && lane == 0) bulk_wait_all();
     }
 
-    // ---- final state (NaN if an internal wait timed out) ----------------------
+    // ---- final state (NaN if an internal wait timed out; the failure is also recorded in the
+    // device status word, where kda_device_status finds it) -------------------------------------
     __syncthreads();
     tc_fence_after();
     ok = __syncthreads_and(ok) != 0;
+    if (!ok && tid == 0) report_device_failure(DEV_WAIT_TIMEOUT);
     if (!SPLIT && warp < 4 && a.sf) {
         const size_t soff = ((size_t)n * H + h) * D * D;
         const int jcol = tid;
@@ -1442,8 +1701,10 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
                 *reinterpret_cast<const uint4 *>(sm + CK_UT + r * 256 + cgo * 16);
         }
     };
+    // testing aid: this CTA never loads its first slot, so that waiting for it runs out
+    const bool stall = P.debug_stall && blockIdx.x == 0;
     if (tid == 0) {
-        if (nchunks > 0) issue_load(0, 0);
+        if (nchunks > 0 && !stall) issue_load(0, 0);
         if (nchunks > 1) issue_load(1, 1);
     }
     {   // initial state -> TMEM (fp32), key channels 64 half .. 64 half + 63
@@ -1460,24 +1721,51 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
     }
     uint32_t ph_mma = 0;
     bool mma_pending = false;   // thread 0: GEMMs issued but not yet committed and waited for
+    bool timed_out = false, slot_missing = false;   // this thread's view of a failure
     int ch = 0;
     for (; ch < nchunks && ok; ++ch) {
         const int buf = ch & 1;
         const uint32_t bufa = sb + buf * CK_BUF;
-        if (!mbar_wait_cycles(bar_load + buf, (ch >> 1) & 1, WAIT_CYCLES)) ok = false;
+        if (!mbar_wait_cycles(bar_load + buf, (ch >> 1) & 1, (stall && ch == 0) ? STALL_WAIT_CYCLES : WAIT_CYCLES))
+            ok = false, timed_out = true;
         tc_fence_after();
-        if (tid == 0 && ok) {   // U'^T = M^T (T Diag(w))^T: independent of the state, issued first
+        const int *meta = reinterpret_cast<const int *>(sm + buf * CK_BUF + SL_META);
+        const float *gamC = reinterpret_cast<const float *>(meta);
+        if (tid == 0 && ok && !(meta[128] & META_EXACT)) {   // U'^T = M^T (T Diag(w))^T: independent of the state
             const uint32_t id_u = idesc_bf16(128, 64, true, false);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
                 mma_bf16(tbase + TM_U, dMN(bufa + SL_M, 8192, kk), dK(bufa + SL_TBF, 8192, kk), id_u, kk > 0);
             mma_pending = true;   // completed by the step-6 commit
         }
-        const int *meta = reinterpret_cast<const int *>(sm + buf * CK_BUF + SL_META);
-        const float *gamC = reinterpret_cast<const float *>(meta);
         // a slot this call's preparation kernel did not complete reads as a failure
-        ok = __syncthreads_and(ok && (meta[128] & META_OK) && meta[129] == (int)P.epoch) != 0;
+        const bool slot_ok = (meta[128] & META_OK) && meta[129] == (int)P.epoch;
+        if (ok && !slot_ok) slot_missing = true;
+        ok = __syncthreads_and(ok && slot_ok) != 0;
         if (!ok) break;
+        if (meta[128] & META_EXACT) {
+            // ---- exact path: this chunk token by token in fp32 from its raw inputs, staged in the
+            // slot buffer (its prepared operands are not needed); o goes to the staging tile once the
+            // previous chunk's o has left it
+            const int nv = min(C, len - ch * C);
+            if (ch > 0) store_o(ch - 1);
+            __syncthreads();
+            uint8_t *stq = sm + buf * CK_BUF, *stk = stq + 16384, *sta = stq + 32768;
+            stage_exact_inputs(a, (size_t)row0 + ch * C, nv, h, stq, stk, sta, tid, CK_NT);
+            __syncthreads();
+            exact_chunk<2, true>(a, tbase + lane_base + TM_S, half * 64, jcol, half, stq, stk, sta,
+                                 (size_t)row0 + ch * C, nv, h, reinterpret_cast<float4 *>(sm + CK_S0T),
+                                 1 + (warp & 3), ost, 128, half == 0);
+            fence_async_smem();   // the staging writes precede the next bulk load into this buffer
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
+            if (SNAP) snapshot_state(a, tbase + lane_base, sbase + ch, h, half * 2, 2, jcol);
+            if (tid == 0 && ok && ch + 2 < nchunks) issue_load(ch + 2, buf);
+            tc_fence_before();
+            ok = __syncthreads_and(ok) != 0;
+            continue;
+        }
         const bool fast = (meta[128] & META_FAST) != 0;
         // ---- state pass: S^T *= Gamma_C in TMEM; bf16 operand copy (scaled on the fast path)
         {
@@ -1515,7 +1803,7 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
         }
         // ---- o of the previous chunk, staged in the U^T tile, to HBM while the step-6 GEMMs run
         if (ch > 0) store_o(ch - 1);
-        if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
+        if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false, timed_out = true;
         ph_mma ^= 1;
         mma_pending = false;
         tc_fence_after();
@@ -1544,7 +1832,7 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
             }
             mma_commit(bar_mma);
         }
-        if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false;
+        if (!mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES)) ok = false, timed_out = true;
         ph_mma ^= 1;
         tc_fence_after();
         if (SNAP) snapshot_state(a, tbase + lane_base, sbase + ch, h, half * 2, 2, jcol);
@@ -1555,8 +1843,11 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
         ok = __syncthreads_and(ok) != 0;
     }
     if (ok && nchunks > 0) store_o(nchunks - 1);
-    if (!ok && tid == 0) {   // drain loads and an uncommitted GEMM still in flight (bounded)
-        for (int c = ch; c < nchunks && c < ch + 2; ++c) mbar_wait_cycles(bar_load + (c & 1), (c >> 1) & 1, WAIT_CYCLES);
+    if (timed_out || slot_missing) report_device_failure((timed_out ? DEV_WAIT_TIMEOUT : 0u) |
+                                                         (slot_missing ? DEV_SLOT_MISSING : 0u));
+    if (!ok && tid == 0) {   // drain loads (those issued) and an uncommitted GEMM still in flight (bounded)
+        for (int c = ch; c < nchunks && c < ch + 2; ++c)
+            if (!(stall && c == 0)) mbar_wait_cycles(bar_load + (c & 1), (c >> 1) & 1, WAIT_CYCLES);
         if (mma_pending) {
             mma_commit(bar_mma);
             mbar_wait_cycles(bar_mma, ph_mma, WAIT_CYCLES);
@@ -1663,6 +1954,26 @@ cudaError_t make_params(ChunkParams &p, const FwdArgs &a)
 }
 }  // namespace
 
+namespace {
+__device__ unsigned int g_status_taken;
+__global__ void take_status_kernel() { g_status_taken = atomicExch(&g_device_status, 0u); }
+}  // namespace
+
+cudaError_t take_device_status(cudaStream_t st, unsigned *bits)
+{
+    static std::mutex mu;   // one reader of the staging word at a time
+    std::lock_guard<std::mutex> lock(mu);
+    take_status_kernel<<<1, 1, 0, st>>>();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    unsigned w = 0;
+    if ((e = cudaMemcpyFromSymbolAsync(&w, g_status_taken, sizeof(w), 0, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        return e;
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return e;
+    *bits = w;
+    return cudaSuccess;
+}
+
 cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
 {
     int num_sms = 0;
@@ -1714,7 +2025,8 @@ cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st
     const long long rows = (long long)a.B * a.T;
     p.ws = static_cast<uint8_t *>(ws);
     p.nslots = (int)(N + (rows + C - 1) / C);
-    p.epoch = epoch.fetch_add(1) + 1;
+    p.epoch = epoch.fetch_add(1) + 1;   // a 32-bit tag: it repeats only after 2^32 split-form calls
+    p.debug_stall = a.debug_stall;
     const long long nwork = (long long)p.nslots * a.H;
     if (rows > 0 && nwork > 0) {
         const unsigned grid = (unsigned)std::min<long long>(nwork, num_sms);

@@ -28,6 +28,7 @@ struct FwdArgs {
     unsigned prep = 0;   // PREP_* bits: input preparation done by the kernels
     int ext = 0;         // extended (Complex KDA) gate range: selects the activations
     float *snap = nullptr;   // optional: state after every 64 tokens, [slot][H][dk][dv] (chunk slots)
+    int debug_stall = 0;     // testing aid (split form): one chain CTA's first wait runs out
 };
 
 // Chunk slot of chunk c (64 tokens) of sequence n whose first token is global
@@ -82,5 +83,14 @@ size_t chunk_noalloc_capacity();
 cudaError_t launch_chunk_split_noalloc(const FwdArgs &a, cudaStream_t st);
 cudaError_t launch_check_gates(int variant, int gate_range, bool bf16, long long n_tok, int dk,
                                const void *alpha, const void *g1, int *d_count, cudaStream_t st);
+cudaError_t launch_check_seqlens(const int32_t *cu, int num_seqs, long long total, int *d_count, cudaStream_t st);
+// Synchronous input validation: counts gates outside the range (*bad_gates) and
+// violations of the cu_seqlens contract (*bad_seqlens; cu may be NULL), waiting
+// for the verdict on `st`.
+cudaError_t validate_inputs(int variant, int gate_range, bool bf16, long long n_tok, int dk, const void *alpha,
+                            const void *g1, const int32_t *cu, int num_seqs, long long total, cudaStream_t st,
+                            int *bad_gates, int *bad_seqlens);
+// Device failure word: read and cleared after `st` has drained.
+cudaError_t take_device_status(cudaStream_t st, unsigned *bits);
 
 }  // namespace kda

@@ -94,10 +94,13 @@ int chunk_args(kda::FwdArgs &a, int variant, int gate_range, int dtype, int B, i
     if (rc != KDA_OK) return rc;
     if (!chunk_ok(chunk_size))
         return fail(KDA_ERR_UNSUPPORTED, "chunk_size %d: supported are 16, 32, 64, 128", chunk_size);
-    if (flags & ~(KDA_FLAG_FORCE_SCAN | KDA_FLAG_FORCE_FUSED | KDA_FLAG_FORCE_SPLIT | PREP_FLAGS))
+    if (flags & ~(KDA_FLAG_VALIDATE_RANGE | KDA_FLAG_FORCE_SCAN | KDA_FLAG_FORCE_FUSED | KDA_FLAG_FORCE_SPLIT |
+                  PREP_FLAGS | KDA_FLAG_DEBUG_STALL))
         return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
     if ((flags & KDA_FLAG_FORCE_FUSED) && (flags & KDA_FLAG_FORCE_SPLIT))
         return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_FORCE_FUSED and KDA_FLAG_FORCE_SPLIT exclude each other");
+    if ((flags & KDA_FLAG_DEBUG_STALL) && !(flags & KDA_FLAG_FORCE_SPLIT))
+        return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_DEBUG_STALL needs KDA_FLAG_FORCE_SPLIT");
     int N = B;
     if (cu_seqlens) {
         if (B != 1) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (got B=%d)", B);
@@ -112,6 +115,28 @@ int chunk_args(kda::FwdArgs &a, int variant, int gate_range, int dtype, int B, i
         return fail(KDA_ERR_INVALID_ARG, "final_state is not 16-byte aligned");
     a = kda::FwdArgs{variant, B, T, H, d_k, d_v, q, k, v, alpha, g1, g2, cu_seqlens, N,
                      initial_state, final_state, o, prep_bits(flags), gate_range == KDA_RANGE_EXTENDED};
+    a.debug_stall = (flags & KDA_FLAG_DEBUG_STALL) ? 1 : 0;
+    return KDA_OK;
+}
+
+// KDA_FLAG_VALIDATE_RANGE: check the gates against the declared range and
+// cu_seqlens against its contract on the device, wait for the verdict, and
+// refuse the call (nothing launched) on a violation.  Gate logits are not
+// gates yet: with KDA_FLAG_GATE_LOGITS only cu_seqlens is checked.
+int validate(const kda::FwdArgs &a, int gate_range, int dtype, unsigned flags, cudaStream_t st)
+{
+    if (!(flags & KDA_FLAG_VALIDATE_RANGE)) return KDA_OK;
+    const long long n_tok = (flags & KDA_FLAG_GATE_LOGITS) ? 0 : (long long)a.B * a.T * a.H;
+    int bad_gates = 0, bad_seqlens = 0;
+    const cudaError_t e = kda::validate_inputs(a.variant, gate_range, dtype == KDA_DTYPE_BF16, n_tok, a.dk, a.alpha,
+                                               a.g1, a.cu_seqlens, a.num_seqs, (long long)a.B * a.T, st, &bad_gates,
+                                               &bad_seqlens);
+    if (e != cudaSuccess) return cuda_fail(e, "input validation");
+    if (bad_seqlens)
+        return fail(KDA_ERR_INVALID_ARG, "cu_seqlens violates cu[0] = 0, cu[n] <= cu[n+1], cu[N] = %lld "
+                                         "(%d violations)", (long long)a.B * a.T, bad_seqlens);
+    if (bad_gates)
+        return fail(KDA_ERR_RANGE, "%d gate values outside the declared range (or NaN)", bad_gates);
     return KDA_OK;
 }
 
@@ -182,6 +207,8 @@ extern "C" int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
         return fail(KDA_ERR_INVALID_ARG, "chunk_states is not 16-byte aligned");
     a.snap = chunk_states;
     if (workspace && !aligned16(workspace)) return fail(KDA_ERR_INVALID_ARG, "workspace is not 16-byte aligned");
+    if ((flags & KDA_FLAG_DEBUG_STALL) && !tensor_core_path(a, dtype, chunk_size, flags))
+        return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_DEBUG_STALL needs the tensor-core split form");
     if ((flags & KDA_FLAG_FORCE_SPLIT) && tensor_core_path(a, dtype, chunk_size, flags)) {
         size_t need = 0;
 #ifdef KDA_WITH_SM100_CHUNK
@@ -191,6 +218,7 @@ extern "C" int kda_chunk_fwd_ws(int variant, int gate_range, int dtype,
             return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_FORCE_SPLIT needs a workspace of %zu bytes (got %zu)", need,
                         workspace ? workspace_bytes : (size_t)0);
     }
+    if ((rc = validate(a, gate_range, dtype, flags, static_cast<cudaStream_t>(stream))) != KDA_OK) return rc;
     return chunk_launch(a, dtype, chunk_size, flags, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -207,6 +235,9 @@ extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
                         num_seqs, initial_state, final_state, o, chunk_size, flags);
     if (rc != KDA_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((flags & KDA_FLAG_DEBUG_STALL) && !tensor_core_path(a, dtype, chunk_size, flags))
+        return fail(KDA_ERR_INVALID_ARG, "KDA_FLAG_DEBUG_STALL needs the tensor-core split form");
+    if ((rc = validate(a, gate_range, dtype, flags, st)) != KDA_OK) return rc;
     void *ws = nullptr;
     size_t ws_bytes = 0;
 #ifdef KDA_WITH_SM100_CHUNK
@@ -220,6 +251,9 @@ extern "C" int kda_chunk_fwd(int variant, int gate_range, int dtype,
         }
     }
 #endif
+    if ((flags & KDA_FLAG_FORCE_SPLIT) && !ws && tensor_core_path(a, dtype, chunk_size, flags) &&
+        (flags & KDA_FLAG_DEBUG_STALL))
+        return fail(KDA_ERR_CUDA, "KDA_FLAG_DEBUG_STALL: the split form's workspace could not be allocated");
     rc = chunk_launch(a, dtype, chunk_size, flags, ws, ws_bytes, st);
     if (ws) {
         const cudaError_t ef = cudaFreeAsync(ws, st);
@@ -391,6 +425,9 @@ extern "C" int kda_chunk_fwd_rank2(int variant, int gate_range, int dtype,
     if (flags & KDA_FLAG_GATE_LOGITS)
         return fail(KDA_ERR_UNSUPPORTED, "rank-2 steps take gate values, not logits "
                                          "(the second sub-step's alpha = 1 has no finite logit)");
+    if (flags & (KDA_FLAG_VALIDATE_RANGE | KDA_FLAG_DEBUG_STALL))
+        return fail(KDA_ERR_UNSUPPORTED, "kda_chunk_fwd_rank2 takes neither KDA_FLAG_VALIDATE_RANGE nor "
+                                         "KDA_FLAG_DEBUG_STALL (check the gates with kda_check_gates)");
     if (B < 1 || T < 0 || H < 1 || T > (1 << 29))
         return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d (need B>=1, 0<=T<=2^29, H>=1)", B, T, H);
     if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_F32) return fail(KDA_ERR_INVALID_ARG, "bad dtype %d", dtype);
@@ -444,11 +481,13 @@ extern "C" int kda_decode_step(int variant, int gate_range, int dtype,
     if (rc != KDA_OK) return rc;
     if (!state) return fail(KDA_ERR_INVALID_ARG, "state is NULL");
     if (!aligned16(state)) return fail(KDA_ERR_INVALID_ARG, "state is not 16-byte aligned");
-    if (flags & ~PREP_FLAGS) return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if (flags & ~(PREP_FLAGS | KDA_FLAG_VALIDATE_RANGE))
+        return fail(KDA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
     if ((unsigned long long)N * H > (1ull << 31) - 1)
         return fail(KDA_ERR_INVALID_ARG, "N*H too large for one launch");
     kda::FwdArgs a{variant, N, 1, H, d_k, d_v, q, k, v, alpha, g1, g2, nullptr, N, state, state, o,
                    prep_bits(flags), gate_range == KDA_RANGE_EXTENDED};
+    if ((rc = validate(a, gate_range, dtype, flags, static_cast<cudaStream_t>(stream))) != KDA_OK) return rc;
     cudaError_t e = kda::launch_decode_step(a, dtype == KDA_DTYPE_BF16, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kda_decode_step launch");
     return KDA_OK;
@@ -472,6 +511,32 @@ extern "C" int kda_check_gates(int variant, int gate_range, int dtype, long long
     return KDA_OK;
 }
 
+extern "C" int kda_check_seqlens(const int32_t *cu_seqlens, int num_seqs, long long total_tokens, int *d_count,
+                                 void *stream)
+{
+    if (num_seqs < 1 || total_tokens < 0)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes num_seqs=%d total_tokens=%lld", num_seqs, total_tokens);
+    if (!cu_seqlens || !d_count) return fail(KDA_ERR_INVALID_ARG, "cu_seqlens or d_count is NULL");
+    if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) || (reinterpret_cast<uintptr_t>(d_count) & 3u))
+        return fail(KDA_ERR_INVALID_ARG, "cu_seqlens or d_count is not 4-byte aligned");
+    const cudaError_t e = kda::launch_check_seqlens(cu_seqlens, num_seqs, total_tokens, d_count,
+                                                    static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kda_check_seqlens launch");
+    return KDA_OK;
+}
+
+extern "C" int kda_device_status(void *stream, unsigned *bits)
+{
+    unsigned w = 0;
+    const cudaError_t e = kda::take_device_status(static_cast<cudaStream_t>(stream), &w);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_device_status");
+    if (bits) *bits = w;
+    if (w) return fail(KDA_ERR_DEVICE_TIMEOUT, "device failure bits 0x%x (%s%s)", w,
+                       (w & KDA_DEVICE_WAIT_TIMEOUT) ? "a bounded wait ran out " : "",
+                       (w & KDA_DEVICE_SLOT_MISSING) ? "a chunk slot was not prepared" : "");
+    return KDA_OK;
+}
+
 extern "C" const char *kda_error_string(int code)
 {
     switch (code) {
@@ -480,10 +545,12 @@ extern "C" const char *kda_error_string(int code)
     case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: valid but unsupported size or option";
     case KDA_ERR_RANGE: return "KDA_ERR_RANGE: gate outside the declared range";
     case KDA_ERR_CUDA: return "KDA_ERR_CUDA: CUDA runtime or launch failure";
+    case KDA_ERR_DEVICE_TIMEOUT:
+        return "KDA_ERR_DEVICE_TIMEOUT: a kernel gave up a bounded wait or found its input missing";
     }
     return "unknown kda status code";
 }
 
 extern "C" const char *kda_last_error_detail(void) { return g_detail; }
 
-extern "C" int kda_version(void) { return 100; }
+extern "C" int kda_version(void) { return 200; }

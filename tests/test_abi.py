@@ -46,7 +46,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_error_strings(lib):
     assert lib.kda_version() >= 100
-    for code in range(5):
+    for code in range(6):
         s = lib.kda_error_string(code).decode()
         assert s.startswith("KDA_")
     assert "unknown" in lib.kda_error_string(99).decode()
@@ -147,7 +147,7 @@ def test_chunk_fwd_rejects_bad_arguments(lib, kw, code):
 @pytest.mark.parametrize("kw,code", [
     (dict(N=0), INVALID), (dict(H=0), INVALID), (dict(variant=9), INVALID), (dict(dk=24), UNSUPPORTED),
     (dict(state=None), INVALID), (dict(state=BAD), INVALID), (dict(o=None), INVALID),
-    (dict(variant=1), INVALID), (dict(flags=1), INVALID), (dict(q=BAD), INVALID),
+    (dict(variant=1), INVALID), (dict(flags=1 << 8), INVALID), (dict(q=BAD), INVALID),
 ])
 def test_decode_step_rejects_bad_arguments(lib, kw, code):
     assert dec(lib, **kw) == code
@@ -247,3 +247,28 @@ def bwd(lib, **kw):
 def test_bwd_rejects_bad_arguments(lib, kw, code, detail):
     assert bwd(lib, **kw) == code
     assert detail in lib.kda_last_error_detail()
+
+
+def test_debug_stall_needs_the_split_form(lib):
+    """The failure-path testing aid only exists in the split form: other forms refuse it on the host."""
+    assert fwd(lib, flags=64) == 1                     # no FORCE_SPLIT
+    assert fwd(lib, flags=64 | 4) == 1                 # fused
+    assert fwd(lib, flags=64 | 8 | 2) == 1             # scan
+    assert "DEBUG_STALL" in lib.kda_last_error_detail().decode()
+    assert fwd_ws(lib, flags=64 | 8, dtype=1) == 1     # fp32 runs the scan
+
+
+def test_validate_flag_is_refused_where_it_has_no_meaning(lib):
+    r2 = lib.kda_chunk_fwd_rank2
+    r2.restype = ctypes.c_int
+    assert r2(0, 0, 0, 1, 8, 1, 128, 128, P, P, P, P, P, None, None, 0, None, None, P, 64, P, 1 << 30, 1,
+              None) == 2
+
+
+def test_check_seqlens_rejects_bad_arguments(lib):
+    lib.kda_check_seqlens.restype = ctypes.c_int
+    assert lib.kda_check_seqlens(None, 2, 10, P, None) == 1
+    assert lib.kda_check_seqlens(P, 0, 10, P, None) == 1
+    assert lib.kda_check_seqlens(P, 2, -1, P, None) == 1
+    assert lib.kda_check_seqlens(P, 2, 10, None, None) == 1
+    assert lib.kda_check_seqlens(ctypes.c_void_p(0x10002), 2, 10, P, None) == 1

@@ -115,17 +115,19 @@ def test_rotation_closed_form_fp32_d128(theta):
     assert torch.equal(s[2:], ref[2:])
 
 
-def test_rotation_tensor_core_path_bf16():
-    """The same construction through the bf16 tensor-core kernel: rows 3..d_k are
-    bitwise unchanged (zero key channels, unit gates), rows 1-2 match the oracle
-    within the bf16 tolerance on a short run.  (Long runs of identical
-    non-decaying reflections cancel heavily in the bf16 WY form: see the
-    precision notes of the chunked kernel.)"""
+@pytest.mark.parametrize("form", ["fused", "split"])
+@pytest.mark.parametrize("T", [4, 64, 128, 256])
+def test_rotation_tensor_core_path_bf16(T, form):
+    """The same construction through the bf16 tensor-core kernel, over one to
+    four whole chunks of identical, non-decaying reflections: rows 3..d_k are
+    bitwise unchanged (zero key channels, unit gates), and rows 1-2 match the
+    oracle within the bf16 tolerance however many chunks the rotation runs."""
     import linear_rnn_delta_b200 as kda
     import oracle
-    T, dk = 4, 128
+    dk = 128
     (q, k, v, al, beta), s0 = _rotation_inputs(0.3, T, dk, "bf16")
-    o, s = kda.kda_chunk_fwd("kda", "extended", q, k, v, al, beta, None, initial_state=s0.cuda())
+    o, s = kda.kda_chunk_fwd("kda", "extended", q, k, v, al, beta, None, initial_state=s0.cuda(),
+                             flags={"fused": 4, "split": 8}[form])
     torch.cuda.synchronize()
     _, s_ref = oracle.recurrence_arrays("kda", q.cpu(), k.cpu(), v.cpu(), al.cpu(), beta.cpu(), None, None, s0)
     assert torch.equal(s.cpu()[0, 0, 2:], s0[0, 0, 2:])
