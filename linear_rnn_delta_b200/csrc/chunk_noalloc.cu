@@ -23,7 +23,9 @@ static __device__ __align__(256) unsigned char g_chunk_scratch[NOALLOC_SCRATCH_B
 
 // Device address of the array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address must come from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, once per device, with that device current.  The
+// address is kept for the life of the process: a cudaDeviceReset, which
+// unloads the module, makes it stale (the header forbids calls after one).
 cudaError_t scratch_address(void **ptr)
 {
     static std::mutex mu;

@@ -2,8 +2,11 @@
 device memory at call time (an engine that owns all of HBM through its own
 allocator, a fixed device-memory budget, a loop that cannot take cudaMalloc's
 latency or synchronisation).  Its workspace is a fixed 64 MiB array inside the
-library, so its results must match the allocating entry point's, including on
-a second call that finds the previous call's slots still in the array.
+library.  It runs the split form of the tensor-core path, so its results must
+equal, bit for bit, those of the allocating entry point forced to the split
+form, on two calls in a row over different slot layouts of the same array (any
+leftover of the first call read by the second would change bits); both are
+also checked against the float64 oracle.
 
 This file is collected last on purpose: a failure here comes after every other
 test has run.
@@ -20,6 +23,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import oracle  # noqa: E402
 import workloads as W  # noqa: E402
 
 _vp, _i = ctypes.c_void_p, ctypes.c_int
@@ -72,12 +76,15 @@ def test_noalloc_matches_the_allocating_entry_point_on_two_calls_in_a_row():
         o = torch.empty((inp.B, inp.T, inp.H, inp.d_v), dtype=torch.bfloat16, device="cuda")
         sf = torch.empty((inp.num_seqs, inp.H, inp.d_k, inp.d_v), dtype=torch.float32, device="cuda")
         assert _noalloc(lib, inp, d, o, sf, stream) == OK, lib.kda_last_error_detail()
-        o_ref, sf_ref = kda.kda_chunk_fwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"],
-                                          d["g1"], d["g2"], cu_seqlens=d["cu_seqlens"],
-                                          initial_state=d["initial_state"])
+        o_ws, sf_ws = kda.kda_chunk_fwd(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"],
+                                        d["g1"], d["g2"], cu_seqlens=d["cu_seqlens"],
+                                        initial_state=d["initial_state"], flags=kda.FLAG_FORCE_SPLIT)
         torch.cuda.synchronize()
-        _close(o, o_ref, 2e-2, "o")
-        _close(sf, sf_ref, 2e-2, "final state")
+        assert torch.equal(o, o_ws), "o differs from the split form's"
+        assert torch.equal(sf, sf_ws), "final state differs from the split form's"
+        o_ref, s_ref = oracle.recurrence(inp)
+        _close(o, torch.from_numpy(o_ref), 2e-2, "o")
+        _close(sf, torch.from_numpy(s_ref), 2e-2, "final state")
 
 
 # A fake, 16-byte-aligned, never-dereferenced device address: the checks below
