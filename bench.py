@@ -3,14 +3,16 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--extra]
 
 A step is one pass of the hot path over one batch of synthetic input: one
-chunked forward (``kda_chunk_fwd``) over the KDA-range bf16 workload
-B=4, H=16, T=4096, d_k=d_v=128, chunk 64 (seeded inputs, resident in HBM).
-The single-token decode step (256 x 32 heads, d=128, fp32 state 512 MiB in
-place, Complex-KDA range) is timed in the same run and reported under
-"decode", and the backward pass (``kda_chunk_bwd``: every gradient of the
-same chunked workload, fp32 arithmetic) under "backward".  With --extra the
-Complex-KDA 8x16x8192 and the RDA / GDN-2 varlen workloads are timed too
-(under "also").
+chunked forward (``kda_chunk_fwd``) over the Complex-KDA bf16 workload
+B=8, H=16, T=8192, d_k=d_v=128, chunk 64 (alpha = tanh(2 N(0,1)), beta =
+2 sigmoid(N(0,1)); seeded inputs resident in HBM) -- the largest of the
+chunked workloads and the one with signed gates.  In the same run, each with
+its own roofline and end-to-end figures, "also" times the KDA-range workload
+B=4, H=16, T=4096 and the RDA and GDN-2 packed workloads (16 documents of
+U[512, 4096] tokens, H=32); "decode" times the single-token step (256 x 32
+heads, d=128, fp32 state 512 MiB in place, Complex-KDA range) and
+"backward" the gradients of the KDA-range workload.  --extra adds the forward
+from gate logits and raw keys, with state snapshots, and rank-2 steps.
 
 Multi-GPU (torchrun): every rank runs its own independent batch (different
 seed): the work shards over (sequence, head) units with no collective on the
@@ -445,61 +447,116 @@ def run_rank2_workload(inp, steps, warmup, world):
     return {"tokens_per_step": inp.B * inp.T, "total_s": total, "avg_launch_s": sum(per) / len(per)}
 
 
-def oracle_sample_rate(inp, target_s=12.0, threads=0):
-    """Tokens/s of the float64 oracle on a bounded sample of the workload:
-    whole sequences of a few heads, scaled to the metric's unit (a token is a
-    position of the batch across all H heads)."""
+def host_cores() -> int:
+    """Cores this process may run on (its CPU affinity)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:   # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_block(inp, n_pairs: int):
+    """A block of about n_pairs (sequence, head) pairs, whole sequences: the
+    first heads, then as many of the first sequences as it takes."""
+    heads = list(range(min(inp.H, max(1, n_pairs))))
+    seqs = list(range(min(inp.num_seqs, -(-max(1, n_pairs) // len(heads)))))
+    return seqs, heads
+
+
+def time_oracle(inp, seqs, heads, threads: int):
+    """Seconds and head-tokens of the float64 oracle over every (sequence, head)
+    of the block."""
     import oracle
-    cores = threads or oracle.max_threads()
-    pairs = []
-    n_seq, H = inp.num_seqs, inp.H
-    # one head first, to size the sample
-    t0 = time.perf_counter()
-    oracle.recurrence(inp, seqs=[0], heads=[0], threads=1)
-    one = max(time.perf_counter() - t0, 1e-4)
-    per_head_tokens = inp.seq_bounds(0)[2]
-    n_pairs = int(max(1, min(n_seq * H, (target_s * cores) / one)))
-    rng = np.random.default_rng(0)
-    flat = rng.permutation(n_seq * H)[:n_pairs]
-    pairs = sorted({(int(f) // H, int(f) % H) for f in flat})
-    seqs = sorted({n for n, _ in pairs})
-    heads = sorted({h for _, h in pairs})
     t0 = time.perf_counter()
     oracle.recurrence(inp, seqs=seqs, heads=heads, threads=threads)
     dt = time.perf_counter() - t0
-    head_tokens = sum(inp.seq_bounds(n)[2] for n in seqs) * len(heads)
-    rate = head_tokens / inp.H / dt
-    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(seqs)} sequences x {len(heads)} heads of the workload ({head_tokens} head-tokens, "
-                      f"{dt:.1f} s float64 on {cores} host threads); tokens = head-tokens / H",
-            "seconds": dt, "single_head_s": one, "per_head_tokens": per_head_tokens}
+    return dt, sum(inp.seq_bounds(n)[2] for n in seqs) * len(heads)
+
+
+def oracle_sample_rate(inp, target_s=10.0):
+    """Tokens/s of the float64 oracle, as it stands, on a bounded sample of the
+    workload (whole sequences of a block of (sequence, head) pairs), on every
+    core this process may use; a token is a position of the batch across all
+    H heads, so the rate is head-tokens / H / seconds.  A one-thread time of
+    one (sequence, head) sizes the sample and is reported beside it."""
+    cores = host_cores()
+    one_s, one_ht = time_oracle(inp, [0], [0], threads=1)
+    seqs, heads = oracle_block(inp, int(max(cores, target_s * cores / max(one_s, 1e-4))))
+    dt, ht = time_oracle(inp, seqs, heads, threads=cores)
+    return {"value": ht / inp.H / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(seqs)} sequences x {len(heads)} heads of the workload, whole sequences ({ht} "
+                      f"head-tokens, {dt:.1f} s of float64 work on {cores} threads); tokens = head-tokens / H",
+            "cpu_model": cpu_model(), "affinity_cores": cores,
+            "single_thread": {"value": one_ht / inp.H / one_s, "unit": "tokens/s",
+                              "sample": f"sequence 0, head 0 ({one_ht} head-tokens, {one_s:.2f} s, 1 thread)"}}
+
+
+HEADLINE = "Complex-KDA chunked forward B=8 H=16 T=8192 d_k=d_v=128 chunk=64 bf16, fp32 state, zero initial state"
 
 
 def reference_arm(args, world, rank):
-    """The oracle, as it stands, on the host cores: the same workload, metric and unit."""
+    """The oracle, as it stands, on the host cores: the headline workload, metric
+    and unit.  A reference step is the float64 recurrence over a fixed sample of
+    the workload -- as many whole (sequence, head) pairs as there are cores, so
+    that each step takes about a second -- and it is timed whole: ms_per_step is
+    the wall time of one such step, value = head-tokens / H / seconds."""
     if rank != 0:
         return
-    inp = W.kda_bf16(0)
-    rates = []
-    samples = None
-    # each step is a bounded sample of the workload; sized so the whole run ends within minutes
-    per_step_target = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    inp = W.ckda_bf16(0)
+    cores = host_cores()
+    seqs, heads = oracle_block(inp, cores)
+    head_tokens = None
+    times = []
     for i in range(args.warmup + args.steps):
-        r = oracle_sample_rate(inp, target_s=per_step_target)
+        dt, head_tokens = time_oracle(inp, seqs, heads, threads=cores)
         if i >= args.warmup:
-            rates.append(r["value"])
-            samples = r
-    value = statistics.median(rates)
+            times.append(dt)
+    total = sum(times)
+    value = head_tokens * len(times) / inp.H / total
+    sample = (f"{len(seqs)} sequences x {len(heads)} heads of the workload per step, whole sequences "
+              f"({head_tokens} head-tokens, float64 on {cores} threads, {cpu_model()}); tokens = head-tokens / H")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": inp.B * inp.T / value * 1e3,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded numpy, cast to bf16; the oracle reads the same values in float64)",
-            "config": {"workload": "KDA-range chunked forward B=4 H=16 T=4096 d_k=d_v=128 chunk=64 bf16",
-                       "global_batch": inp.B, "seq_len": inp.T, "heads": inp.H, "parallelism": "host cores"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples["cores"], "kind": "oracle",
-                             "sample": samples["sample"]},
+            "config": {"workload": HEADLINE, "global_batch": inp.B, "seq_len": inp.T, "heads": inp.H,
+                       "parallelism": "host cores", "step": "a bounded sample of the workload (see cpu_baseline)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line))
+
+
+def chunk_line(name, inp, r, world, steps, traffic_key=None):
+    """The JSON fields of one timed chunked workload."""
+    value = r["tokens_per_step"] * world * steps / r["total_s"]
+    line = {"workload": name, "value": value, "unit": UNIT, "ms_per_step": r["total_s"] / steps * 1e3,
+            "p50_ms": r["p50_ms"], "p95_ms": r["p95_ms"], "p99_ms": r["p99_ms"], "form": r["form"],
+            "gpu_launches": steps * r["kernels_per_step"],
+            "roofline": {"bound": "hbm", "achieved": r["hbm"]["achieved"], "peak": r["hbm"]["peak"], "unit": "GB/s",
+                         "frac": r["hbm"]["frac"],
+                         "traffic": (measured_traffic(traffic_key, CHUNK_SOURCES).get("dram_bytes_per_launch")
+                                     if traffic_key else None),
+                         "kernel": ("kda_chunk_fwd, split form: preparation + chain kernels timed as one call"
+                                    if r["form"] == "split" else "kda_chunk_fwd, fused form: one kernel"),
+                         "alg_bytes_per_launch": r["alg"]["bytes"]},
+            "tensor": {"achieved": r["tensor"]["achieved"], "peak": r["tensor"]["peak"], "unit": "TFLOP/s",
+                       "frac": r["tensor"]["frac"], "alg_flops_per_launch": r["alg"]["flops"]}}
+    if "e2e" in r:
+        e = r["e2e"]
+        line["e2e"] = {"value": r["tokens_per_step"] * world * steps / e["total_s"], "unit": UNIT,
+                       "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"]}
+    return line
 
 
 # ---------------------------------------------------------------------------
@@ -507,10 +564,11 @@ def reference_arm(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--extra", action="store_true", help="also time Complex-KDA 8x16x8192 and varlen RDA/GDN-2")
+    ap.add_argument("--extra", action="store_true",
+                    help="also time the forward from gate logits and raw keys, with state snapshots, and rank-2 steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--backward-steps", type=int, default=20)
@@ -528,83 +586,77 @@ def main():
 
     import linear_rnn_delta_b200  # noqa: F401  (fails loudly if the library is missing)
     peaks = load_peaks()
-    inp = W.kda_bf16(seed=rank_workload_seed(rank))
-    sampler = ClockSampler(local) if rank == 0 else None
+    seed = rank_workload_seed(rank)
     fflags = FORM_FLAGS[args.form]
+    sampler = ClockSampler(local) if rank == 0 else None
+    # the headline: Complex KDA, B=8 H=16 T=8192
+    inp = W.ckda_bf16(seed)
     main_res = run_chunk_workload(inp, args.steps, args.warmup, world, peaks, sampler=sampler, flags=fflags)
-    decode = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank)
-    backward = run_backward_workload(inp, args.backward_steps, args.warmup, world, rank)
-    also = []
-    if args.extra:
-        prep = lambda: W.make_chunk_inputs("kda", "standard", "bf16", B=4, T=4096, H=16, d_k=128, d_v=128,
-                                           seed=rank_workload_seed(rank), logits=True, raw_k=True)
-        for name, mk, xflags in (
-                ("Complex-KDA chunked forward B=8 H=16 T=8192 d=128 chunk=64 bf16", lambda: W.ckda_bf16(rank), 0),
-                ("RDA varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("rda", rank), 0),
-                ("GDN-2 varlen 16 docs U[512,4096] H=32 d=128 bf16", lambda: W.varlen_bf16("gdn2", rank), 0),
-                ("KDA B=4 H=16 T=4096 bf16 from gate logits and raw keys (in-kernel activations, L2 norm)",
-                 prep, 16 | 32),
-                ("KDA B=4 H=16 T=4096 bf16 with fp32 state snapshots after every 64 tokens",
-                 lambda: W.kda_bf16(seed=rank_workload_seed(rank)), "states")):
-            x = mk()
-            r = run_chunk_workload(x, max(5, args.steps // 2), args.warmup, world, peaks, e2e=False,
-                                   flags=fflags | (xflags if xflags != "states" else 0), states=xflags == "states")
-            also.append({"workload": name, "value": r["tokens_per_step"] * world * max(5, args.steps // 2) / r["total_s"],
-                         "unit": UNIT, "ms_per_step": r["avg_launch_s"] * 1e3, "form": r["form"],
-                         "hbm_frac": r["hbm"]["frac"],
-                         "tensor_frac": r["tensor"]["frac"], "achieved_gbs": r["hbm"]["achieved"],
-                         "achieved_tflops": r["tensor"]["achieved"]})
-            del x
-        x = W.make_rank2_inputs("kda", "standard", "bf16", B=4, T=2048, H=16, d_k=128, d_v=128,
-                                seed=rank_workload_seed(rank))
-        r = run_rank2_workload(x, max(5, args.steps // 2), args.warmup, world)
-        also.append({"workload": "KDA rank-2 steps (two sub-steps per token) B=4 H=16 T=2048 d=128 bf16: "
-                                 "q/alpha expansion + chunked forward over 4096 sub-tokens + o gather",
-                     "value": r["tokens_per_step"] * world * max(5, args.steps // 2) / r["total_s"], "unit": UNIT,
-                     "ms_per_step": r["avg_launch_s"] * 1e3})
-        del x
+    head = chunk_line(HEADLINE, inp, main_res, world, args.steps, f"chunk_fwd_ckda_8x16x8192_{main_res['form']}")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample_rate(inp)
+    del inp
+    # the other chunked workloads, each with its own roofline and end-to-end figures
+    also = []
+    for name, mk, key in (
+            ("KDA-range chunked forward B=4 H=16 T=4096 d=128 chunk=64 bf16, zero initial state",
+             lambda: W.kda_bf16(seed), "chunk_fwd_kda_4x16x4096"),
+            ("RDA packed documents: 16 docs of U[512,4096] tokens, H=32 d=128 bf16, random initial states",
+             lambda: W.varlen_bf16("rda", seed), "chunk_fwd_rda_varlen"),
+            ("GDN-2 packed documents: 16 docs of U[512,4096] tokens, H=32 d=128 bf16, random initial states",
+             lambda: W.varlen_bf16("gdn2", seed), "chunk_fwd_gdn2_varlen")):
+        x = mk()
+        r = run_chunk_workload(x, args.steps, args.warmup, world, peaks, flags=fflags)
+        also.append(chunk_line(name, x, r, world, args.steps, f"{key}_{r['form']}"))
+        del x
+    decode = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank)
+    bwd_inp = W.kda_bf16(seed)
+    backward = run_backward_workload(bwd_inp, args.backward_steps, args.warmup, world, rank)
+    del bwd_inp
+    if args.extra:
+        prep = lambda: W.make_chunk_inputs("kda", "standard", "bf16", B=4, T=4096, H=16, d_k=128, d_v=128,
+                                           seed=seed, logits=True, raw_k=True)
+        for name, mk, xflags in (
+                ("KDA B=4 H=16 T=4096 bf16 from gate logits and raw keys (in-kernel activations, L2 norm)",
+                 prep, 16 | 32),
+                ("KDA B=4 H=16 T=4096 bf16 with fp32 state snapshots after every 64 tokens",
+                 lambda: W.kda_bf16(seed), "states")):
+            x = mk()
+            r = run_chunk_workload(x, args.steps, args.warmup, world, peaks, e2e=False,
+                                   flags=fflags | (xflags if xflags != "states" else 0), states=xflags == "states")
+            also.append(chunk_line(name, x, r, world, args.steps))
+            del x
+        x = W.make_rank2_inputs("kda", "standard", "bf16", B=4, T=2048, H=16, d_k=128, d_v=128, seed=seed)
+        r = run_rank2_workload(x, args.steps, args.warmup, world)
+        also.append({"workload": "KDA rank-2 steps (two sub-steps per token) B=4 H=16 T=2048 d=128 bf16: "
+                                 "q/alpha expansion + chunked forward over 4096 sub-tokens + o gather",
+                     "value": r["tokens_per_step"] * world * args.steps / r["total_s"], "unit": UNIT,
+                     "ms_per_step": r["total_s"] / args.steps * 1e3})
+        del x
     if rank != 0:
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
         return
-    tokens = main_res["tokens_per_step"] * world
-    value = tokens * args.steps / main_res["total_s"]
-    e2e = main_res["e2e"]
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": main_res["total_s"] / args.steps * 1e3,
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded numpy draws, bf16; per-rank seed)",
-        "config": {"workload": "KDA-range chunked forward B=4 H=16 T=4096 d_k=d_v=128 chunk=64 bf16, "
-                               "fp32 state, zero initial state",
-                   "global_batch": inp.B * world, "seq_len": inp.T, "heads": inp.H, "parallelism": f"dp{world}",
-                   "l2": f"inputs {inp.nbytes() / 1e6:.0f} MB > L2 126 MB, no flush"},
-        "p50_ms": main_res["p50_ms"], "p95_ms": main_res["p95_ms"], "p99_ms": main_res["p99_ms"],
-        "roofline": {"bound": "hbm", "achieved": main_res["hbm"]["achieved"], "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": main_res["hbm"]["frac"],
-                     "traffic": measured_traffic(f"chunk_fwd_kda_4x16x4096_{main_res['form']}",
-                                                 CHUNK_SOURCES).get("dram_bytes_per_launch"),
-                     "peak_source": peaks["source"],
-                     "kernel": ("kda_chunk_fwd, split form: preparation + chain kernels timed as one call"
-                                if main_res["form"] == "split" else "kda_chunk_fwd, fused form: one kernel"),
-                     "form": main_res["form"],
-                     "alg_bytes_per_launch": main_res["alg"]["bytes"]},
-        "tensor": {"achieved": main_res["tensor"]["achieved"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                   "frac": main_res["tensor"]["frac"], "alg_flops_per_launch": main_res["alg"]["flops"]},
-        "e2e": {"value": tokens * args.steps / e2e["total_s"], "unit": UNIT,
-                "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"]},
-        "gpu_launches": args.steps * main_res["kernels_per_step"],
+        "config": {"workload": HEADLINE, "global_batch": 8 * world, "seq_len": 8192, "heads": 16,
+                   "parallelism": f"dp{world}", "l2": "inputs 1.08 GB per step > L2 126 MB, no flush"},
+        "p50_ms": head["p50_ms"], "p95_ms": head["p95_ms"], "p99_ms": head["p99_ms"],
+        "roofline": dict(head["roofline"], peak_source=peaks["source"], form=head["form"]),
+        "tensor": head["tensor"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
         "clocks": main_res["clocks"],
+        "also": also,
         "decode": decode,
         "backward": backward,
-        "cpu_baseline": cpu and {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+        "cpu_baseline": cpu,
     }
-    if also:
-        line["also"] = also
     print(json.dumps(line))
     if world > 1:
         import torch.distributed as dist
