@@ -51,10 +51,11 @@
 // place before step 1 (a compile-time variant, PREP).
 //
 // Split form: steps 1-4 do not depend on the state, so a persistent kernel
-// (the same code, SPLIT = true) runs them for every (chunk, head) on all SMs
-// and stores each chunk's operand tiles to a workspace slot; a chain kernel
-// per (sequence, head) then runs steps 5-7 from those slots.  Same arithmetic
-// in the same order: the two forms give identical bits.
+// (chunk_prep_kernel, which pipelines two items per SM) runs them for every
+// (chunk, head) on all SMs and stores each chunk's operand tiles to a
+// workspace slot; a chain kernel per (sequence, head) then runs steps 5-7 from
+// those slots.  Same arithmetic on every element: the two forms give identical
+// bits.
 #include <cuda.h>
 #include <algorithm>
 #include <atomic>
@@ -95,8 +96,7 @@ constexpr uint32_t M_G1 = OFF_MISC, M_G2 = OFF_MISC + 256, M_GAMC = OFF_MISC + 5
                    M_PBAND = OFF_MISC + 5632, M_FAST = OFF_MISC + 6912, M_BAR = OFF_MISC + 6920,
                    M_TMEM = OFF_MISC + 6976;
 constexpr uint32_t M_G1B = OFF_MISC + 6992, M_G2B = OFF_MISC + 7248;   // gates of the other item parity
-constexpr uint32_t M_ITEM = OFF_MISC + 7504;                            // split: decoded items [2][8] int
-constexpr uint32_t SMEM_USED = OFF_MISC + 7568;
+constexpr uint32_t SMEM_USED = OFF_MISC + 7504;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack for aligning the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 static_assert((OFF_TBF & 1023) == 0 && (OFF_PBF & 1023) == 0 && (OFF_QA & 1023) == 0, "swizzle atoms");
@@ -176,36 +176,6 @@ struct Item {
     int slot;
     bool valid;
 };
-// Split path: work index w = slot * H + h -> chunk, or invalid when the slot is empty.
-__device__ __forceinline__ Item decode_item(const FwdArgs &a, int N, int w)
-{
-    Item it;
-    it.h = w % a.H;
-    it.slot = w / a.H;
-    int lo = 0, hi = N - 1;   // last sequence whose first slot is <= slot
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (slot_base(a, mid) <= it.slot) lo = mid;
-        else hi = mid - 1;
-    }
-    it.n = lo;
-    it.row0 = seq_row0(a, lo);
-    it.len = seq_len(a, lo);
-    it.c = it.slot - slot_base(a, lo);
-    it.valid = it.c >= 0 && it.c * C < it.len;
-    return it;
-}
-__device__ __forceinline__ Item next_split_item(const FwdArgs &a, int N, int nwork, int &w)
-{
-    for (; w < nwork; w += gridDim.x) {
-        const Item it = decode_item(a, N, w);
-        if (it.valid) return it;
-    }
-    Item none{};
-    none.valid = false;
-    return none;
-}
-
 // ---- small helpers --------------------------------------------------------
 // Elementwise work is done in "items" of 8 tokens x 4 channels (one 8-byte
 // half of a 16-byte chunk per row): 256 items cover a 64 x 128 tile.
@@ -285,6 +255,7 @@ struct ChunkCtx {
     int H, h, nvalid;
     bool gdn2;
     bool logits, ext;   // input preparation: GDN-2's erase vector arrives as logits; extended range
+    uint32_t qa, kb, la, lb;   // shared-memory offsets of the row-operand tile, Kbar and the level factors
 };
 
 // Channel-wise part of the erase direction of row r for 4 channels (GDN-2:
@@ -401,9 +372,9 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
             oq[c] = v ? sc[c] * qv[c] : 0.f;
             kb[c] = v ? __fdividef(kv[c], sc[c]) : 0.f;
         }
-        *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, r, cq)) = pack4(oa);
-        *reinterpret_cast<uint2 *>(sm + OFF_QA + sw_half(16384, 64 + r, cq)) = pack4(oq);
-        *reinterpret_cast<uint2 *>(sm + OFF_KB + sw_half(8192, r, cq)) = pack4(kb);
+        *reinterpret_cast<uint2 *>(sm + x.qa + sw_half(16384, r, cq)) = pack4(oa);
+        *reinterpret_cast<uint2 *>(sm + x.qa + sw_half(16384, 64 + r, cq)) = pack4(oq);
+        *reinterpret_cast<uint2 *>(sm + x.kb + sw_half(8192, r, cq)) = pack4(kb);
         float *bp = band_part + r * (PBAND * 32) + lane;
         bp[0] = oq[0] * kb[0] + oq[1] * kb[1] + oq[2] * kb[2] + oq[3] * kb[3];
 #pragma unroll
@@ -485,8 +456,8 @@ __device__ __forceinline__ void build_level(const ChunkCtx &x, int slot, int tg,
             fp[c] = v ? run[c] * qv[c] : 0.f;
         }
         const int idx = (r / BS) * HH + (pos - HH);
-        *reinterpret_cast<uint2 *>(sm + OFF_LA + sw_half(16384, slot * 32 + idx, cq)) = pack4(fa);
-        *reinterpret_cast<uint2 *>(sm + OFF_LA + sw_half(16384, 64 + slot * 32 + idx, cq)) = pack4(fp);
+        *reinterpret_cast<uint2 *>(sm + x.la + sw_half(16384, slot * 32 + idx, cq)) = pack4(fa);
+        *reinterpret_cast<uint2 *>(sm + x.la + sw_half(16384, 64 + slot * 32 + idx, cq)) = pack4(fp);
     }
     float sx[4];
 #pragma unroll
@@ -509,14 +480,14 @@ __device__ __forceinline__ void build_level(const ChunkCtx &x, int slot, int tg,
             sx[c] *= v ? al[c] : 1.f;
         }
         const int idx = (r / BS) * HH + pos;
-        *reinterpret_cast<uint2 *>(sm + OFF_LB + sw_half(8192, slot * 32 + idx, cq)) = pack4(fc);
+        *reinterpret_cast<uint2 *>(sm + x.lb + sw_half(8192, slot * 32 + idx, cq)) = pack4(fc);
     }
 }
 
 // Anchored path: scatter one level's A or P entries from the 32 TMEM columns
 // the calling warp loaded (rows of this lane's level list).
 template <int HH>
-__device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const float *s_e, bool isP, int lane,
+__device__ __forceinline__ void scatter_level(uint8_t *pbf, float *Af, const float *s_e, bool isP, int lane,
                                               const float *v)
 {
     constexpr int BS = 2 * HH;
@@ -527,7 +498,7 @@ __device__ __forceinline__ void scatter_level(uint8_t *sm, float *Af, const floa
         if (c >= c0 && c < c0 + HH) {
             const int s = (c / HH) * BS + (c % HH);
             if (!isP) Af[r * TP + s] = v[c] * s_e[r];
-            else *reinterpret_cast<unsigned short *>(sm + OFF_PBF + sw_elem(8192, r, s)) = bf16_bits(v[c]);
+            else *reinterpret_cast<unsigned short *>(pbf + sw_elem(8192, r, s)) = bf16_bits(v[c]);
         }
     }
 }
@@ -723,13 +694,11 @@ __device__ __noinline__ void exact_chunk(const FwdArgs &a, uint32_t tstate, int 
 constexpr int NCHAIN = 128, NPREP = 256;
 constexpr uint32_t BAR_PREP = 1, BAR_CHAIN = 2;
 
-// SPLIT = false: the fused kernel, one CTA per (sequence, head), both roles.
-// SPLIT = true: the preparation role alone (256 threads), persistent over all
-// chunks of all sequences and heads; each chunk's operands go to its slot.
+// The fused kernel: one CTA per (sequence, head), both roles.
 // PREP: input preparation requested (gate logits and / or raw keys); without
 // it the preparation code is compiled out.
-template <bool SPLIT, bool PREP>
-__global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __grid_constant__ ChunkParams P)
+template <bool PREP>
+__global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant__ ChunkParams P)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -738,15 +707,13 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3;       // TMEM lane quarter of this warp
     const int H = a.H;
-    const int N = a.cu_seqlens ? a.num_seqs : a.B;
-    const int n = blockIdx.x / H, h = blockIdx.x % H;   // fused kernel: this CTA's sequence and head
-    const int len = SPLIT ? 0 : seq_len(a, n);
+    const int n = blockIdx.x / H, h = blockIdx.x % H;   // this CTA's sequence and head
+    const int len = seq_len(a, n);
     const int nchunks = (len + C - 1) / C;
 
     // scalar gates, per item parity (filled one item ahead)
     auto s_g1buf = [&](uint32_t parity) { return reinterpret_cast<float *>(sm + (parity ? M_G1B : M_G1)); };
     auto s_g2buf = [&](uint32_t parity) { return reinterpret_cast<float *>(sm + (parity ? M_G2B : M_G2)); };
-    int *s_items = reinterpret_cast<int *>(sm + M_ITEM);
     float *s_gamC = reinterpret_cast<float *>(sm + M_GAMC);     // [2][128]: chunk parity
     float *s_tot = reinterpret_cast<float *>(sm + M_TOT);       // [8][128] block totals of alpha
     float *s_pband = reinterpret_cast<float *>(sm + M_PBAND);   // [64][PBAND]: P_{r, r-w}
@@ -778,7 +745,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     bool ok = true;
 
-    if (!SPLIT && warp < 4) {
+    if (warp < 4) {
         // =====================================================================
         // CHAIN group
         // =====================================================================
@@ -915,16 +882,13 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
         // =====================================================================
         // PREP group
         // =====================================================================
-        const int ptid = SPLIT ? tid : tid - NCHAIN, pw = SPLIT ? warp : warp - 4;
+        const int ptid = tid - NCHAIN, pw = warp - 4;
         const int phalf = pw >> 2;              // the two prep warps of a lane quarter split columns
         const int jrow = quarter * 32 + lane;   // TMEM lane of this thread
         const int tg = ptid >> 5, cq = ptid & 31;   // elementwise item: 8 tokens x 4 channels
         uint32_t ph_tma = 0, ph_v = 0, ph_pmma = 0;
 
         const CUtensorMap *map_q = &P.tq, *map_k = &P.tk, *map_v = &P.tv, *map_a = &P.ta;
-        // M tile: the fused kernel has one; the split kernel (GDN-2) alternates two by item
-        // parity, since an item's M is still being stored while the next item's v arrives
-        auto mt_off = [&](uint32_t parity) -> uint32_t { return (SPLIT && parity) ? OFF_S0T : OFF_MT; };
         auto issue_tma = [&](const Item &it) {   // q, k, alpha of a chunk
             const int g = it.row0 + it.c * C;
             mbar_expect_tx(bar_tma, 3 * 16384);
@@ -932,11 +896,11 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             tma_load_3d(sm + RAW_K, map_k, bar_tma, 0, it.h, g);
             tma_load_3d(sm + RAW_A, map_a, bar_tma, 0, it.h, g);
         };
-        auto issue_tma_v = [&](const Item &it, uint32_t parity) { // v, straight into its swizzled operand layout
+        auto issue_tma_v = [&](const Item &it) {   // v, straight into its swizzled operand layout
             const int g = it.row0 + it.c * C;
             mbar_expect_tx(bar_v, 16384);
-            tma_load_3d(sm + mt_off(parity), map_v, bar_v, 0, it.h, g);
-            tma_load_3d(sm + mt_off(parity) + 8192, map_v, bar_v, 64, it.h, g);
+            tma_load_3d(sm + OFF_MT, map_v, bar_v, 0, it.h, g);
+            tma_load_3d(sm + OFF_MT + 8192, map_v, bar_v, 64, it.h, g);
         };
         auto wait_pmma = [&]() {
             if (!mbar_wait_cycles(bar_pmma, ph_pmma, WAIT_CYCLES)) ok = false;
@@ -975,60 +939,35 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             s_g1buf(parity)[r] = fe;
             s_g2buf(parity)[r] = fw;
         };
-        // split: decoded items travel through shared memory, two ahead (decoded by one
-        // thread while most warps wait in the T solve)
-        auto put_item = [&](const Item &it, uint32_t slot) {
-            int *d = s_items + slot * 8;
-            d[0] = it.n; d[1] = it.h; d[2] = it.c; d[3] = it.row0; d[4] = it.len; d[5] = it.slot;
-            d[6] = it.valid ? 1 : 0;
-        };
-        auto get_item = [&](uint32_t slot) {
-            const int *d = s_items + slot * 8;
-            Item it;
-            it.n = d[0]; it.h = d[1]; it.c = d[2]; it.row0 = d[3]; it.len = d[4]; it.slot = d[5];
-            it.valid = d[6] != 0;
-            return it;
-        };
-
-        // the chain of items this role prepares
-        const int nwork = SPLIT ? P.nslots * H : 0;
-        int wnext = blockIdx.x;
+        // the chunks of this CTA's sequence, one after the other
         auto fused_item = [&](int c) {
             Item it{n, h, c, 0, len, 0, c < nchunks};
             it.row0 = seq_row0(a, n);
             return it;
         };
-        Item cur = SPLIT ? next_split_item(a, N, nwork, wnext) : fused_item(0);
-        Item nxt_boot{};
-        if (SPLIT) {   // the first two items are decoded by every thread
-            wnext += gridDim.x;
-            nxt_boot = next_split_item(a, N, nwork, wnext);
-        }
-        const bool need_v = !SPLIT || gdn2;   // the split kernel leaves U' to the chain kernel
+        Item cur = fused_item(0);
         if (cur.valid && ptid == 0) {
             issue_tma(cur);
-            if (need_v) issue_tma_v(cur, 0);
+            issue_tma_v(cur);
         }
         if (ptid < C && cur.valid) fetch_gates(cur, ptid, 0);
 
         for (int ch = 0; cur.valid && ok; ++ch) {
             const uint32_t par = ch & 1, ppar = (ch - 1) & 1;
-            const Item nxt = !SPLIT ? fused_item(ch + 1) : (ch == 0 ? nxt_boot : get_item((ch + 1) & 1));
+            const Item nxt = fused_item(ch + 1);
             const int h = cur.h;
             const int nvalid = min(C, cur.len - cur.c * C);
             const size_t rowbase = (size_t)cur.row0 + cur.c * C;
             float *const s_g1 = s_g1buf(par);
             float *const s_g2 = s_g2buf(par);
-            const ChunkCtx x{sm, s_tot, s_g1, g1p, rowbase, H, h, nvalid, gdn2, logits, ext};
-            const uint32_t OFF_MTC = mt_off(par);
-            float *gamc = SPLIT ? reinterpret_cast<float *>(sm + OFF_UT) : s_gamC + par * 128;
+            const ChunkCtx x{sm,   s_tot, s_g1,   g1p,    rowbase, H,     h,     nvalid,
+                             gdn2, logits, ext, OFF_QA, OFF_KB, OFF_LA, OFF_LB};
+            float *gamc = s_gamC + par * 128;
 
             if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
             ph_tma ^= 1;
-            if (need_v) {
-                if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
-                ph_v ^= 1;
-            }
+            if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
+            ph_v ^= 1;
             group_sync(BAR_PREP, NPREP);
 
             // ===== 0. input preparation, in place in the raw tiles (this thread's 8 rows x 4 channels),
@@ -1106,7 +1045,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
 #pragma unroll 2
                 for (int i = 0; i < 8; ++i) {
                     const int r = tg * 8 + i;
-                    uint2 *pv = reinterpret_cast<uint2 *>(sm + OFF_MTC + sw_half(8192, r, cq));
+                    uint2 *pv = reinterpret_cast<uint2 *>(sm + OFF_MT + sw_half(8192, r, cq));
                     float mv[4], vv[4], wv[4];
                     unpack4(*pv, vv);
                     if (r < nvalid) {
@@ -1120,10 +1059,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                     *pv = pack4(mv);
                 }
             }
-            if (SPLIT && lane == 0) bulk_wait_read();   // the previous item's slot stores
             in_range = group_sync_and(BAR_PREP, NPREP, in_range);
-            // GDN-2: the next item's v into the M tile the previous item stored (read: waited above)
-            if (SPLIT && ptid == 0 && gdn2 && nxt.valid) issue_tma_v(nxt, par ^ 1u);
 
             // ===== Gamma_C and the per-chunk path decision ========================
             bool gam_ok = true;
@@ -1143,7 +1079,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             const bool fast = group_sync_and(BAR_PREP, NPREP, gam_ok) && in_range;
 
             // the previous chunk's chain must be done with QA (step 6) and with Kbar / P (step 7)
-            if (!SPLIT && ch > 0) {
+            if (ch > 0) {
                 if (!mbar_wait_cycles(bar_s6, ppar, WAIT_CYCLES)) ok = false;
                 if (!mbar_wait_cycles(bar_s7, ppar, WAIT_CYCLES)) ok = false;
             }
@@ -1153,8 +1089,8 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                 // one forward sweep per item; band partials to the F region, reduced after the A/P GEMM issue
                 float *band_part = reinterpret_cast<float *>(sm + OFF_F);
                 if (nvalid == C) {
-                    if (gdn2) fast_rows<true, true, SPLIT ? 4 : 1>(x, s_tot, gamc, band_part, tg, cq, lane);
-                    else fast_rows<true, false, SPLIT ? 4 : 1>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    if (gdn2) fast_rows<true, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    else fast_rows<true, false, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
                 } else {
                     fast_rows<false, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
                 }
@@ -1334,12 +1270,12 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                     tmem_ld32(tbase + lane_base + tm_lvl(p) + (quarter & 1) * 32, v);
                     tmem_wait_ld();
                     switch (lvl) {
-                    case 1: scatter_level<32>(sm, Af, s_g1, isP, lane, v); break;
-                    case 2: scatter_level<16>(sm, Af, s_g1, isP, lane, v); break;
-                    case 3: scatter_level<8>(sm, Af, s_g1, isP, lane, v); break;
-                    case 4: scatter_level<4>(sm, Af, s_g1, isP, lane, v); break;
-                    case 5: scatter_level<2>(sm, Af, s_g1, isP, lane, v); break;
-                    default: scatter_level<1>(sm, Af, s_g1, isP, lane, v); break;
+                    case 1: scatter_level<32>(sm + OFF_PBF, Af, s_g1, isP, lane, v); break;
+                    case 2: scatter_level<16>(sm + OFF_PBF, Af, s_g1, isP, lane, v); break;
+                    case 3: scatter_level<8>(sm + OFF_PBF, Af, s_g1, isP, lane, v); break;
+                    case 4: scatter_level<4>(sm + OFF_PBF, Af, s_g1, isP, lane, v); break;
+                    case 5: scatter_level<2>(sm + OFF_PBF, Af, s_g1, isP, lane, v); break;
+                    default: scatter_level<1>(sm + OFF_PBF, Af, s_g1, isP, lane, v); break;
                     }
                 }
                 group_sync(BAR_PREP, NPREP);
@@ -1353,16 +1289,6 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             }
             tc_fence_before();
             group_sync(BAR_PREP, NPREP);
-
-            // split: Q' (rows 64-127 of both panels) and Kbar are final -- to the slot now, so that
-            // less is left to read out of shared memory at the end of the item
-            if (SPLIT && ok && lane == 0 && pw >= 5) {
-                uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
-                if (pw == 5) bulk_store(slot + SL_QA + 8192, sm + OFF_QA + 8192, 8192);
-                else if (pw == 6) bulk_store(slot + SL_QA + 24576, sm + OFF_QA + 24576, 8192);
-                else bulk_store(slot + SL_KB, sm + OFF_KB, 16384);
-                bulk_commit();
-            }
 
             // ===== 3. T = (I + A)^{-1} =============================================
             // 16x16 diagonal blocks by forward substitution (one column per thread), then
@@ -1391,9 +1317,6 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                 for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * TP + 16 * I + c] = 0.f;  // above the block
             } else if (ptid < 64 + C) {   // meanwhile: the next item's gates
                 if (nxt.valid) fetch_gates(nxt, ptid - 64, par ^ 1u);
-            } else if (SPLIT && ptid == 64 + C) {   // and the item after it
-                wnext += gridDim.x;
-                put_item(nxt.valid ? next_split_item(a, N, nwork, wnext) : Item{}, par);
             }
             group_sync(BAR_PREP, NPREP);
             {   // X = A_{I+1,I} D_I for I = 0, 2 (two outputs per thread)
@@ -1510,7 +1433,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             const bool exact = !publish_and(write_t_copy(s_g1));
             // U'^T overwrites TMEM U: the chain must have read the previous chunk's U out
             // (the split kernel leaves U' to the chain kernel and stores T Diag(w) instead)
-            if (!SPLIT && ch > 0 && !mbar_wait_cycles(bar_ufree, ppar, WAIT_CYCLES)) ok = false;
+            if (ch > 0 && !mbar_wait_cycles(bar_ufree, ppar, WAIT_CYCLES)) ok = false;
             if (ptid == 0) {
                 tc_fence_after();
                 const uint32_t id_w = idesc_bf16(64, 128, false, true);
@@ -1518,7 +1441,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     mma_bf16(tbase + TM_W, dK(sb + OFF_TBF, 8192, kk), dMN(sb + OFF_QA, 16384, kk), id_w, kk > 0);
-                    if (!SPLIT && same_gates)
+                    if (same_gates)
                         mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_TBF, 8192, kk), id_u, kk > 0);
                 }
                 mma_commit(bar_pmma);
@@ -1527,7 +1450,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
             if (!same_gates) {
                 write_t_copy(s_g2);
                 publish();
-                if (!SPLIT && ptid == 0) {
+                if (ptid == 0) {
                     tc_fence_after();
                     const uint32_t id_u = idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -1535,9 +1458,9 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                         mma_bf16(tbase + TM_U, dMN(sb + OFF_MT, 8192, kk), dK(sb + OFF_TBF, 8192, kk), id_u, kk > 0);
                     mma_commit(bar_pmma);
                 }
-                if (!SPLIT) wait_pmma();
+                wait_pmma();
             }
-            if (!SPLIT && ptid == 0 && nxt.valid) issue_tma_v(nxt, 0);   // v consumed by U'^T = M^T T^T
+            if (ptid == 0 && nxt.valid) issue_tma_v(nxt);   // v consumed by U'^T = M^T T^T
             // W (M = 64 layout: rows 16q..16q+15 in lanes 0..15 of quarter q) -> rows 0-63 of QA
             {
                 const int r = quarter * 16 + (lane & 15);
@@ -1554,37 +1477,19 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                     }
                 }
             }
-            if (SPLIT && ptid == 0) {   // status word and epoch tag of the slot
-                int *meta = reinterpret_cast<int *>(sm + OFF_UT);
-                meta[128] = META_OK | (fast ? META_FAST : 0) | (exact ? META_EXACT : 0);
-                meta[129] = (int)P.epoch;
-            }
             fence_async_smem();
             tc_fence_before();
             ok = group_sync_and(BAR_PREP, NPREP, ok);
-            if (!SPLIT && ptid == 0) {   // chunk ch's operands are ready for the chain
+            if (ptid == 0) {   // chunk ch's operands are ready for the chain
                 s_fast[par] = (fast ? META_FAST : 0) | (exact ? META_EXACT : 0);
                 mbar_arrive(bar_ready);
-            }
-            if (SPLIT && ok && lane == 0 && pw < 5) {   // the rest of the slot, one bulk store per warp
-                uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
-                if (pw == 0) bulk_store(slot + SL_QA, sm + OFF_QA, 8192);                     // -W', panel 0
-                else if (pw == 1) bulk_store(slot + SL_QA + 16384, sm + OFF_QA + 16384, 8192);   // -W', panel 1
-                else if (pw == 2) bulk_store(slot + SL_PBF, sm + OFF_PBF, 8192);
-                else if (pw == 3) bulk_store(slot + SL_TBF, sm + OFF_TBF, 8192);
-                else {
-                    bulk_store(slot + SL_META, sm + OFF_UT, SL_META_BYTES);
-                    if (gdn2) bulk_store(slot + SL_M, sm + OFF_MTC, 16384);
-                }
-                bulk_commit();
             }
             cur = nxt;
         }
         if (!ok) {  // drain TMA still in flight (bounded)
             mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
-            if (need_v) mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
+            mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
         }
-        if (SPLIT && lane == 0) bulk_wait_all();
     }
 
     // ---- final state (NaN if an internal wait timed out; the failure is also recorded in the
@@ -1593,7 +1498,7 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
     tc_fence_after();
     ok = __syncthreads_and(ok) != 0;
     if (!ok && tid == 0) report_device_failure(DEV_WAIT_TIMEOUT);
-    if (!SPLIT && warp < 4 && a.sf) {
+    if (warp < 4 && a.sf) {
         const size_t soff = ((size_t)n * H + h) * D * D;
         const int jcol = tid;
 #pragma unroll 1
@@ -1607,6 +1512,891 @@ __global__ void __launch_bounds__(SPLIT ? 256 : NT, 1) chunk_fwd_kernel(const __
                 a.sf[soff + (size_t)(i0 + e) * D + jcol] = ok ? s[e] : __int_as_float(0x7fc00000);
         }
     }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tbase, 512);
+}
+
+// ---- split form: the preparation kernel, two items in flight per SM --------
+// Preparing one (chunk, head) item is a chain of short, latency-bound phases
+// (about 15 K cycles per item with one item per SM, most issue slots idle).
+// This kernel overlaps two items on each SM:
+//   FRONT (warps 0-7) runs steps 0-2 of item j+1: input preparation, block
+//     totals, Gamma_C and the path decision, row operands, Kbar and the band
+//     of P, the A/P GEMM(s) and their read-out into A (fp32) and P (bf16);
+//   BACK (warps 8-11) runs the rest of item j: the UT transform T (solved in
+//     place over its copy of A), the exact-path decision, the T Diag(.)
+//     copies, the W GEMM and its read-out into -W'.
+// Each group bulk-stores its own part of the item's slot (front: Q', Kbar, P,
+// GDN-2's M; back: -W', T Diag(w), the meta block).  GDN-2's v arrives in the
+// one M tile; M = w (.) v is stored as soon as it is formed, and the next
+// item's v is loaded once that store has read the tile.  Two mbarriers hand items
+// over: `full` (front -> back: A, the a~' rows of the row-operand tile, the
+// gates, Gamma_C and the path flag of item j are ready) and `taken` (back ->
+// front: the back has copied them into its own buffers, so the front may
+// rewrite them for item j+1).  Items are decoded four ahead by one back
+// thread into a ring in shared memory.  Every element is computed by the same
+// arithmetic as in the fused kernel (only the thread that computes it
+// differs), so the two forms still give identical bits.
+constexpr int PF_FRONT = 256, PF_BACK = 128, PF_NT = PF_FRONT + PF_BACK;
+constexpr uint32_t BAR_FRONT = 1, BAR_BACK = 2;
+// raw TMA tiles [64][128] bf16 at the fused kernel's offsets (the shared helpers read them there)
+constexpr uint32_t P2_RAW_Q = RAW_Q, P2_RAW_K = RAW_K, P2_RAW_A = RAW_A;
+constexpr uint32_t P2_KB = 32768;     // Kbar [token][channel], between the k and alpha tiles
+constexpr uint32_t P2_QA = 65536;     // [a~'; Q'] 128-row K-major tile (A/P GEMM operand)
+constexpr uint32_t P2_AT = 98304;     // back: the a~' rows (2 panels x 64 rows), then -W'
+constexpr uint32_t P2_FR = 114688;    // front: band partials | level factors; then A fp32 and P bf16
+constexpr uint32_t P2_LA = P2_FR, P2_LB = P2_FR + 32768, P2_AF = P2_FR, P2_PBF = P2_FR + 17408;
+constexpr uint32_t P2_TB = 163840;    // back: A, then T in place, fp32 [64][TP]
+constexpr uint32_t P2_TBF = 181248;   // back: the 32 x 32 scratch of the T solve, then T Diag(.) bf16
+constexpr uint32_t P2_X = P2_TBF;
+constexpr uint32_t P2_MT = 189440;    // front, GDN-2: v, then M = w (.) v in place
+constexpr uint32_t P2_MISC = 205824;
+constexpr uint32_t P2_TOT = P2_MISC;                 // float [8][128] block totals of alpha
+constexpr uint32_t P2_PBAND = P2_MISC + 4096;        // float [64][PBAND]
+constexpr uint32_t P2_GATES = P2_MISC + 5376;        // float [4][2][64]: gates by item index mod 4
+constexpr uint32_t P2_GAMC = P2_MISC + 7424;         // float [2][128]: Gamma_C by item parity
+constexpr uint32_t P2_META = P2_MISC + 8448;         // back: Gamma_C fp32 [128], status word, epoch tag
+constexpr uint32_t P2_RING = P2_MISC + 8992;         // int [8][8]: decoded items
+constexpr uint32_t P2_FLAGS = P2_MISC + 9248;        // int [2] path flags by item parity, [1] abort
+constexpr uint32_t P2_BAR = P2_MISC + 9264;          // mbarriers: tma, v, pmma, wmma, full, taken
+constexpr uint32_t P2_TMEM = P2_MISC + 9312;
+constexpr uint32_t P2_ALLOC = P2_MISC + 9328 + 1024;
+static_assert(P2_ALLOC <= 232448, "shared memory budget");
+static_assert(P2_FR + 40960 <= P2_TB && P2_LB + 16384 <= P2_TB && P2_PBF + 8192 <= P2_TB, "front region");
+static_assert(P2_TB + 64 * TP * 4 <= P2_TBF && P2_TBF + 8192 <= P2_MT && P2_MT + 16384 <= P2_MISC, "back region");
+static_assert(((P2_QA | P2_KB | P2_AT | P2_PBF | P2_TBF | P2_MT) & 1023) == 0, "swizzle atoms");
+static_assert(RAW_Q + 16384 <= RAW_K && RAW_K + 16384 <= P2_KB && P2_KB + 16384 <= RAW_A &&
+              RAW_A + 16384 <= P2_QA && P2_QA + 32768 <= P2_AT && P2_AT + 16384 <= P2_FR, "tile map");
+static_assert((P2_META & 15) == 0 && (P2_BAR & 7) == 0, "alignment");
+// TMEM columns: front A/P at TM_AP, anchored levels below; back W at TM_W
+__device__ __forceinline__ uint32_t tm_lvl_split(int p) { return p == 0 ? 384u : (p == 1 ? 448u : 128u); }
+
+// Next valid item at or after work index w (w += gridDim.x), with the sequence
+// found by walking forward from n (items of one CTA come in increasing slot order).
+__device__ __forceinline__ Item next_item_walk(const FwdArgs &a, int N, int nwork, int &w, int &n)
+{
+    for (; w < nwork; w += gridDim.x) {
+        Item it;
+        it.h = w % a.H;
+        it.slot = w / a.H;
+        while (n + 1 < N && slot_base(a, n + 1) <= it.slot) ++n;
+        it.n = n;
+        it.row0 = seq_row0(a, n);
+        it.len = seq_len(a, n);
+        it.c = it.slot - slot_base(a, n);
+        it.valid = it.c >= 0 && it.c * C < it.len;
+        if (it.valid) return it;
+    }
+    Item none{};
+    none.valid = false;
+    return none;
+}
+__device__ __forceinline__ void ring_put(int *ring, int k, const Item &it)
+{
+    int *d = ring + (k & 7) * 8;
+    d[0] = it.n; d[1] = it.h; d[2] = it.c; d[3] = it.row0; d[4] = it.len; d[5] = it.slot; d[6] = it.valid ? 1 : 0;
+}
+__device__ __forceinline__ Item ring_get(const int *ring, int k)
+{
+    const int *d = ring + (k & 7) * 8;
+    Item it;
+    it.n = d[0]; it.h = d[1]; it.c = d[2]; it.row0 = d[3]; it.len = d[4]; it.slot = d[5]; it.valid = d[6] != 0;
+    return it;
+}
+
+template <bool PREP>
+__global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_constant__ ChunkParams P)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sb = smem_u32(sm);
+    const FwdArgs &a = P.a;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3;
+    const int H = a.H;
+    const int N = a.cu_seqlens ? a.num_seqs : a.B;
+    const int nwork = P.nslots * H;
+    float *s_tot = reinterpret_cast<float *>(sm + P2_TOT);
+    float *s_pband = reinterpret_cast<float *>(sm + P2_PBAND);
+    float *s_gates = reinterpret_cast<float *>(sm + P2_GATES);
+    float *s_gamc = reinterpret_cast<float *>(sm + P2_GAMC);
+    int *s_meta = reinterpret_cast<int *>(sm + P2_META);
+    int *s_ring = reinterpret_cast<int *>(sm + P2_RING);
+    int *s_flags = reinterpret_cast<int *>(sm + P2_FLAGS);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + P2_BAR);
+    uint64_t *bar_tma = bars + 0, *bar_v = bars + 1, *bar_pmma = bars + 2, *bar_wmma = bars + 3;
+    uint64_t *bar_full = bars + 4, *bar_taken = bars + 5;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P2_TMEM);
+    const __nv_bfloat16 *g1p = (const __nv_bfloat16 *)a.g1, *g2p = (const __nv_bfloat16 *)a.g2;
+    const bool gdn2 = a.variant == GDN2;
+    const bool same_gates = a.variant != RDA;
+    const bool logits = PREP && (a.prep & PREP_LOGITS) != 0, l2k = PREP && (a.prep & PREP_L2NORM_K) != 0;
+    const bool ext = a.ext != 0;
+    // the item decoder (one back thread) keeps its cursor across the whole kernel
+    const bool decoder = tid == PF_FRONT + 64;
+    int wdec = blockIdx.x, ndec = 0;
+
+    if (warp == 0) tmem_alloc(s_tmem, 512);
+    if (tid == 0) {
+        for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+        s_flags[2] = 0;   // abort
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (decoder) {   // the first four items
+        for (int k = 0; k < 4; ++k) {
+            ring_put(s_ring, k, next_item_walk(a, N, nwork, wdec, ndec));
+            wdec += gridDim.x;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    bool ok = true;
+
+    if (tid < PF_FRONT) {
+        // =====================================================================
+        // FRONT: steps 0-2 of each item
+        // =====================================================================
+        const int ptid = tid, pw = warp;
+        const int phalf = pw >> 2;
+        const int jrow = quarter * 32 + lane;
+        const int tg = ptid >> 5, cq = ptid & 31;
+        uint32_t ph_tma = 0, ph_v = 0, ph_pmma = 0, ph_taken = 0;
+        float *Af = reinterpret_cast<float *>(sm + P2_AF);
+        auto issue_tma = [&](const Item &it) {
+            const int g = it.row0 + it.c * C;
+            mbar_expect_tx(bar_tma, 3 * 16384);
+            tma_load_3d(sm + P2_RAW_Q, &P.tq, bar_tma, 0, it.h, g);
+            tma_load_3d(sm + P2_RAW_K, &P.tk, bar_tma, 0, it.h, g);
+            tma_load_3d(sm + P2_RAW_A, &P.ta, bar_tma, 0, it.h, g);
+        };
+        auto issue_tma_v = [&](const Item &it) {   // GDN-2: v into the M tile
+            const int g = it.row0 + it.c * C;
+            mbar_expect_tx(bar_v, 16384);
+            tma_load_3d(sm + P2_MT, &P.tv, bar_v, 0, it.h, g);
+            tma_load_3d(sm + P2_MT + 8192, &P.tv, bar_v, 64, it.h, g);
+        };
+        auto wait_pmma = [&]() {
+            if (!mbar_wait_cycles(bar_pmma, ph_pmma, WAIT_CYCLES)) ok = false;
+            ph_pmma ^= 1;
+            tc_fence_after();
+        };
+        auto publish = [&]() {
+            fence_async_smem();
+            tc_fence_before();
+            group_sync(BAR_FRONT, PF_FRONT);
+        };
+        auto gates_of = [&](int k) { return s_gates + (k & 3) * 128; };   // g1 [64], then g2 [64]
+        // scalar gates of row r of an item: loaded early (raw bf16 bits), stored later, so that
+        // the global-load latency is not on any barrier's critical path
+        auto load_gates = [&](const Item &it, int r, uint32_t &ge, uint32_t &gw) {
+            const int nv = min(C, it.len - it.c * C);
+            const size_t tok = ((size_t)it.row0 + it.c * C + r) * H + it.h;
+            const bool v = it.valid && r < nv;
+            const unsigned short *g1u = reinterpret_cast<const unsigned short *>(g1p);
+            const unsigned short *g2u = reinterpret_cast<const unsigned short *>(g2p);
+            if (gdn2) { ge = v ? 0x3F80u : 0u; gw = ge; }   // GDN-2 keeps its gates channel-wise: 1 here
+            else {
+                ge = v ? (uint32_t)g1u[tok] : 0u;
+                gw = v ? (uint32_t)(a.variant == KDA ? g1u[tok] : g2u[tok]) : 0u;
+            }
+        };
+        auto store_gates = [&](int r, uint32_t ge, uint32_t gw, bool valid_row, float *dst) {
+            float fe = __uint_as_float(ge << 16), fw = __uint_as_float(gw << 16);
+            if (logits && !gdn2 && valid_row) {
+                fe = round_bf16(prep_gate(fe, ext));
+                fw = round_bf16(prep_gate(fw, ext));
+            }
+            dst[r] = fe;
+            dst[64 + r] = fw;
+        };
+        auto row_valid = [&](const Item &it, int r) { return it.valid && r < min(C, it.len - it.c * C); };
+
+        Item cur = ring_get(s_ring, 0);
+        if (cur.valid && ptid == 0) {
+            issue_tma(cur);
+            if (gdn2) issue_tma_v(cur);
+        }
+        if (ptid < C && cur.valid) {
+            uint32_t ge, gw;
+            load_gates(cur, ptid, ge, gw);
+            store_gates(ptid, ge, gw, row_valid(cur, ptid), gates_of(0));
+        }
+        int j = 0;
+        for (; cur.valid && ok; ++j) {
+            const uint32_t par = j & 1;
+            const Item nxt = ring_get(s_ring, j + 1);
+            const int h = cur.h;
+            const int nvalid = min(C, cur.len - cur.c * C);
+            const size_t rowbase = (size_t)cur.row0 + cur.c * C;
+            float *const s_g1 = gates_of(j);
+            const ChunkCtx x{sm,   s_tot, s_g1,  g1p,   rowbase, H,     h,     nvalid,
+                             gdn2, logits, ext, P2_QA, P2_KB,   P2_LA, P2_LB};
+            float *gamc = s_gamc + par * 128;
+            uint8_t *slot = P.ws + ((size_t)cur.slot * H + h) * SLOT_BYTES;
+            // the next item's gates (threads 64..127) and, for GDN-2, this item's write vector w
+            // (every thread: its 8 rows x 4 channels) are put in flight first
+            uint32_t nge = 0, ngw = 0;
+            if (ptid >= 64 && ptid < 64 + C) load_gates(nxt, ptid - 64, nge, ngw);
+            uint2 wraw[8];
+            if (gdn2) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = tg * 8 + i;
+                    wraw[i] = r < nvalid ? *reinterpret_cast<const uint2 *>(g2p + ((rowbase + r) * H + h) * D + cq * 4)
+                                         : make_uint2(0u, 0u);
+                }
+            }
+
+            if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
+            ph_tma ^= 1;
+            if (gdn2) {
+                if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
+                ph_v ^= 1;
+            }
+            group_sync(BAR_FRONT, PF_FRONT);
+
+            // ===== 0. input preparation, in place in the raw tiles
+            if (PREP && logits) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint2 *pa = reinterpret_cast<uint2 *>(sm + P2_RAW_A + (tg * 8 + i) * 256 + cq * 8);
+                    float al[4];
+                    unpack4(*pa, al);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) al[c] = prep_alpha(al[c], ext);
+                    *pa = pack4(al);
+                }
+            }
+            if (PREP && l2k) {
+                float ss[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float kv[4];
+                    unpack4(raw_quad(sm, P2_RAW_K, tg * 8 + i, cq), kv);
+                    ss[i] = kv[0] * kv[0] + kv[1] * kv[1] + kv[2] * kv[2] + kv[3] * kv[3];
+                }
+                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float send = b4 ? ss[i] : ss[i + 4];
+                    ss[i] = (b4 ? ss[i + 4] : ss[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const float send = b3 ? ss[i] : ss[i + 2];
+                    ss[i] = (b3 ? ss[i + 2] : ss[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+                }
+                {
+                    const float send = b2 ? ss[0] : ss[1];
+                    ss[0] = (b2 ? ss[1] : ss[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+                }
+                ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], 2);
+                ss[0] += __shfl_xor_sync(0xffffffffu, ss[0], 1);
+                const float sc = prep_kscale(ss[0]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float sci = __shfl_sync(0xffffffffu, sc, ((i & 4) ? 16 : 0) + ((i & 2) ? 8 : 0) + ((i & 1) ? 4 : 0));
+                    uint2 *pk = reinterpret_cast<uint2 *>(sm + P2_RAW_K + (tg * 8 + i) * 256 + cq * 8);
+                    float kv[4];
+                    unpack4(*pk, kv);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) kv[c] *= sci;
+                    *pk = pack4(kv);
+                }
+            }
+
+            // ===== 1a. block totals of alpha (and range check) | GDN-2: M = w (.) v
+            bool in_range = true;
+            {
+                float tot[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = tg * 8 + i;
+                    if (r < nvalid) {
+                        float al[4];
+                        unpack4(raw_quad(sm, P2_RAW_A, r, cq), al);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            tot[c] *= al[c];
+                            in_range = in_range && (fabsf(al[c]) <= 1.f);
+                        }
+                    }
+                }
+                *reinterpret_cast<float4 *>(s_tot + tg * 128 + cq * 4) = make_float4(tot[0], tot[1], tot[2], tot[3]);
+            }
+            if (gdn2) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = tg * 8 + i;
+                    uint2 *pv = reinterpret_cast<uint2 *>(sm + P2_MT + sw_half(8192, r, cq));
+                    float mv[4], vv[4], wv[4];
+                    unpack4(*pv, vv);
+                    if (r < nvalid) {
+                        unpack4(wraw[i], wv);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) mv[c] = (logits ? round_bf16(prep_gate(wv[c], ext)) : wv[c]) * vv[c];
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) mv[c] = 0.f;
+                    }
+                    *pv = pack4(mv);
+                }
+            }
+            if (lane == 0) bulk_wait_read();   // this group's stores of the previous item have read their tiles
+            fence_async_smem();
+            in_range = group_sync_and(BAR_FRONT, PF_FRONT, in_range);
+            if (gdn2 && ptid == 128 && ok) {   // M is final: to the slot now; the next v may then follow
+                bulk_store(slot + SL_M, sm + P2_MT, 16384);
+                bulk_commit();
+            }
+
+            // ===== Gamma_C and the path decision; meanwhile the next item's gates
+            bool gam_ok = true;
+            if (ptid < 32) {
+                float gc[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    float t4[4];
+                    load_tot4(s_tot, g, ptid, t4);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) gc[c] *= t4[c];
+                }
+                *reinterpret_cast<float4 *>(gamc + ptid * 4) = make_float4(gc[0], gc[1], gc[2], gc[3]);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) gam_ok = gam_ok && (fabsf(gc[c]) >= FAST_MIN_GAMMA);
+            } else if (ptid >= 64 && ptid < 64 + C) {
+                store_gates(ptid - 64, nge, ngw, row_valid(nxt, ptid - 64), gates_of(j + 1));
+            }
+            const bool fast = group_sync_and(BAR_FRONT, PF_FRONT, gam_ok) && in_range;
+
+            // the back must have taken the previous item's A, a~' rows, gates and Gamma_C
+            if (j > 0) {
+                if (!mbar_wait_cycles(bar_taken, ph_taken, WAIT_CYCLES)) ok = false;
+                ph_taken ^= 1;
+            }
+
+            // ===== 1b. row operands, Kbar and the exact band of P
+            if (fast) {
+                float *band_part = reinterpret_cast<float *>(sm + P2_FR);
+                if (nvalid == C) {
+                    if (gdn2) fast_rows<true, true, 4>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    else fast_rows<true, false, 4>(x, s_tot, gamc, band_part, tg, cq, lane);
+                } else {
+                    fast_rows<false, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
+                }
+            } else {
+                {
+                    float pre[4] = {1.f, 1.f, 1.f, 1.f}, suf[4] = {1.f, 1.f, 1.f, 1.f};
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) {
+                        if (g == tg) continue;
+                        float t4[4];
+                        load_tot4(s_tot, g, cq, t4);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            if (g < tg) pre[c] *= t4[c];
+                            else suf[c] *= t4[c];
+                        }
+                    }
+                    float sc[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sc[c] = pre[c];
+#pragma unroll 2
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = tg * 8 + i;
+                        const bool v = r < nvalid;
+                        float al[4], kv[4], qv[4], e[4], oa[4], oq[4];
+                        unpack4(raw_quad(sm, P2_RAW_A, r, cq), al);
+                        unpack4(raw_quad(sm, P2_RAW_K, r, cq), kv);
+                        unpack4(raw_quad(sm, P2_RAW_Q, r, cq), qv);
+                        erase_gate4(x, r, cq, e);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            sc[c] *= v ? al[c] : 1.f;
+                            oa[c] = v ? sc[c] * (e[c] * kv[c]) : 0.f;
+                            oq[c] = v ? sc[c] * qv[c] : 0.f;
+                        }
+                        *reinterpret_cast<uint2 *>(sm + P2_QA + sw_half(16384, r, cq)) = pack4(oa);
+                        *reinterpret_cast<uint2 *>(sm + P2_QA + sw_half(16384, 64 + r, cq)) = pack4(oq);
+                    }
+                    float sx[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sx[c] = suf[c];
+#pragma unroll 2
+                    for (int i = 7; i >= 0; --i) {
+                        const int r = tg * 8 + i;
+                        const bool v = r < nvalid;
+                        float al[4], kv[4], kb[4];
+                        unpack4(raw_quad(sm, P2_RAW_A, r, cq), al);
+                        unpack4(raw_quad(sm, P2_RAW_K, r, cq), kv);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            kb[c] = v ? sx[c] * kv[c] : 0.f;
+                            sx[c] *= v ? al[c] : 1.f;
+                        }
+                        *reinterpret_cast<uint2 *>(sm + P2_KB + sw_half(8192, r, cq)) = pack4(kb);
+                    }
+                }
+                {   // exact band of P from the bf16 inputs (four threads per row)
+                    const int r = ptid >> 2, c4 = ptid & 3;
+                    float acc[PBAND];
+#pragma unroll
+                    for (int w = 0; w < PBAND; ++w) acc[w] = 0.f;
+#pragma unroll 1
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int cgx = c4 * 4 + ((jj + r) & 3);
+                        float hv[8];
+                        unpack8(raw_row(sm, P2_RAW_Q, r, cgx), hv);
+#pragma unroll
+                        for (int w = 0; w < PBAND; ++w) {
+                            float kv[8];
+                            unpack8(raw_row(sm, P2_RAW_K, max(r - w, 0), cgx), kv);
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) acc[w] = fmaf(hv[c], kv[c], acc[w]);
+                            if (w + 1 < PBAND) {
+                                float av[8];
+                                unpack8(raw_row(sm, P2_RAW_A, max(r - w, 0), cgx), av);
+#pragma unroll
+                                for (int c = 0; c < 8; ++c) hv[c] *= av[c];
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int w = 0; w < PBAND; ++w) {
+                        float t = acc[w] + __shfl_xor_sync(0xffffffffu, acc[w], 1);
+                        t += __shfl_xor_sync(0xffffffffu, t, 2);
+                        if (c4 == 0) s_pband[r * PBAND + w] = (r < nvalid && r - w >= 0) ? t : 0.f;
+                    }
+                }
+            }
+            fence_async_smem();   // Q' and Kbar are final: to the slot now, read by the bulk copies
+            group_sync(BAR_FRONT, PF_FRONT);
+            if (ok && lane == 0 && (pw == 5 || pw == 6 || pw == 7)) {
+                if (pw == 5) bulk_store(slot + SL_QA + 8192, sm + P2_QA + 8192, 8192);          // Q', panel 0
+                else if (pw == 6) bulk_store(slot + SL_QA + 24576, sm + P2_QA + 24576, 8192);   // Q', panel 1
+                else bulk_store(slot + SL_KB, sm + P2_KB, 16384);
+                bulk_commit();
+            }
+            if (gdn2 && ptid == 128 && nxt.valid) {   // the M store has read its tile: the next item's v
+                bulk_wait_read();
+                issue_tma_v(nxt);
+            }
+            // fast path: nothing reads the raw tiles after step 1b -- the next item's may come in now
+            if (fast && ptid == 0 && nxt.valid) issue_tma(nxt);
+
+            // ===== 2. A and P
+            if (fast) {
+                publish();
+                if (ptid == 0) {
+                    tc_fence_after();
+                    const uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_bf16(tbase + TM_AP, dK(sb + P2_QA, 16384, kk), dK(sb + P2_KB, 8192, kk), idesc, kk > 0);
+                    mma_commit(bar_pmma);
+                }
+                band_reduce(reinterpret_cast<const float *>(sm + P2_FR), s_pband, nvalid, ptid, PF_FRONT);
+                group_sync(BAR_FRONT, PF_FRONT);
+                wait_pmma();
+                float v[32];
+                tmem_ld32(tbase + lane_base + TM_AP + phalf * 32, v);
+                tmem_wait_ld();
+                const int rr = jrow & 63;
+                if (jrow < 64) {
+                    const float er = s_g1[rr];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int s = phalf * 32 + c;
+                        v[c] = (s < rr) ? v[c] * er : 0.f;
+                    }
+#pragma unroll
+                    for (int q4 = 0; q4 < 8; ++q4)
+                        *reinterpret_cast<float4 *>(Af + rr * TP + phalf * 32 + 4 * q4) =
+                            make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        const int s = phalf * 32 + c;
+                        const int w = rr - s;
+                        v[c] = (w >= PBAND) ? v[c] : ((w >= 0) ? s_pband[rr * PBAND + w] : 0.f);
+                    }
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4 *>(sm + P2_PBF + sw_chunk(8192, rr, phalf * 4 + q4)) = pack8(v + q4 * 8);
+                }
+            } else {
+                for (int p = 0; p < 3; ++p) {
+#pragma unroll 1
+                    for (int sl = 0; sl < 2; ++sl) {
+                        switch (2 * p + 1 + sl) {
+                        case 1: build_level<32>(x, sl, tg, cq); break;
+                        case 2: build_level<16>(x, sl, tg, cq); break;
+                        case 3: build_level<8>(x, sl, tg, cq); break;
+                        case 4: build_level<4>(x, sl, tg, cq); break;
+                        case 5: build_level<2>(x, sl, tg, cq); break;
+                        default: build_level<1>(x, sl, tg, cq); break;
+                        }
+                    }
+                    publish();
+                    if (ptid == 0) {
+                        tc_fence_after();
+                        const uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_bf16(tbase + tm_lvl_split(p), dK(sb + P2_LA, 16384, kk), dK(sb + P2_LB, 8192, kk),
+                                     idesc, kk > 0);
+                        mma_commit(bar_pmma);
+                    }
+                    wait_pmma();
+                }
+                if (ptid == 0 && nxt.valid) issue_tma(nxt);   // raw tiles consumed
+                for (int e = ptid; e < 64 * TP; e += PF_FRONT) Af[e] = 0.f;
+                for (int e = ptid; e < 512; e += PF_FRONT)
+                    *reinterpret_cast<uint4 *>(sm + P2_PBF + e * 16) = make_uint4(0, 0, 0, 0);
+                group_sync(BAR_FRONT, PF_FRONT);
+                for (int p = phalf; p < 3; p += 2) {
+                    const int lvl = 2 * p + 1 + (quarter & 1);
+                    const bool isP = quarter >= 2;
+                    float v[32];
+                    tmem_ld32(tbase + lane_base + tm_lvl_split(p) + (quarter & 1) * 32, v);
+                    tmem_wait_ld();
+                    uint8_t *pbf = sm + P2_PBF;
+                    switch (lvl) {
+                    case 1: scatter_level<32>(pbf, Af, s_g1, isP, lane, v); break;
+                    case 2: scatter_level<16>(pbf, Af, s_g1, isP, lane, v); break;
+                    case 3: scatter_level<8>(pbf, Af, s_g1, isP, lane, v); break;
+                    case 4: scatter_level<4>(pbf, Af, s_g1, isP, lane, v); break;
+                    case 5: scatter_level<2>(pbf, Af, s_g1, isP, lane, v); break;
+                    default: scatter_level<1>(pbf, Af, s_g1, isP, lane, v); break;
+                    }
+                }
+                group_sync(BAR_FRONT, PF_FRONT);
+                if (ptid < C) {
+#pragma unroll
+                    for (int w = 0; w < PBAND; ++w)
+                        if (ptid - w >= 0)
+                            *reinterpret_cast<unsigned short *>(sm + P2_PBF + sw_elem(8192, ptid, ptid - w)) =
+                                bf16_bits(s_pband[ptid * PBAND + w]);
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            ok = group_sync_and(BAR_FRONT, PF_FRONT, ok);
+
+            // ===== P to the slot (Q', Kbar and GDN-2's M left earlier); then hand the item over
+            if (ok && lane == 0 && pw == 3) {
+                bulk_store(slot + SL_PBF, sm + P2_PBF, 8192);
+                bulk_commit();
+            }
+            if (ptid == 0) {
+                s_flags[par] = fast ? META_FAST : 0;
+                mbar_arrive(bar_full);
+            }
+            cur = nxt;
+        }
+        // no item j for the back: the ring says so (or the abort flag, after a failure).  The back
+        // must have waited for item j-1 first: `full` may run at most one phase ahead of its
+        // waits (a parity wait cannot tell two completed phases from none)
+        if (j > 0) {
+            if (!mbar_wait_cycles(bar_taken, ph_taken, WAIT_CYCLES)) ok = false;
+            ph_taken ^= 1;
+        }
+        if (ptid == 0) {
+            if (!ok) s_flags[2] = 1;
+            mbar_arrive(bar_full);
+        }
+        if (!ok) {   // drain TMA still in flight (bounded)
+            mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
+            if (gdn2) mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
+        }
+        if (lane == 0) bulk_wait_all();
+    } else {
+        // =====================================================================
+        // BACK: T, the exact-path decision, W, and the rest of the slot
+        // =====================================================================
+        const int btid = tid - PF_FRONT, bw = warp - PF_FRONT / 32;
+        uint32_t ph_full = 0, ph_wmma = 0;
+        float *TB = reinterpret_cast<float *>(sm + P2_TB);
+        float *Xs = reinterpret_cast<float *>(sm + P2_X);
+        auto publish_and = [&](bool pred) {
+            fence_async_smem();
+            tc_fence_before();
+            return group_sync_and(BAR_BACK, PF_BACK, pred);
+        };
+        // T Diag(gate) -> TBF (bf16, K-major); two passes cover the 64 rows with the fused
+        // kernel's thread mapping (row ptid'/4, 16 columns).  Returns whether both of this
+        // thread's rows stay within the exact path's |T| bound.
+        auto write_t_copy = [&](const float *gate, const float *s_bg1, const float *s_bg2) {
+            bool well = true;
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {
+                const int pt = btid + PF_BACK * pp;
+                const int r = pt >> 2, kc0 = (pt & 3) * 2;
+                float tsum = 0.f;
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    float te[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int s = (kc0 + q2) * 8 + c;
+                        const float t = (s <= r) ? TB[r * TP + s] : 0.f;
+                        te[c] = t * gate[s];
+                        tsum += fabsf(t) * fmaxf(fabsf(s_bg1[s]), fabsf(s_bg2[s]));
+                    }
+                    *reinterpret_cast<uint4 *>(sm + P2_TBF + sw_chunk(8192, r, kc0 + q2)) = pack8(te);
+                }
+#pragma unroll
+                for (int m = 1; m <= 2; m <<= 1) tsum += __shfl_xor_sync(0xffffffffu, tsum, m);
+                well = well && tsum <= EXACT_T_NORM;
+            }
+            return well;
+        };
+
+        for (int j = 0; ok; ++j) {
+            if (!mbar_wait_cycles(bar_full, ph_full, WAIT_CYCLES)) {
+                ok = false;
+                break;
+            }
+            ph_full ^= 1;
+            const Item it = ring_get(s_ring, j);
+            if (!it.valid || s_flags[2]) break;
+            const uint32_t par = j & 1;
+            if (lane == 0) bulk_wait_read();   // this group's stores of item j-1 have read AT, TBF, meta
+            group_sync(BAR_BACK, PF_BACK);
+            // ---- take item j: A, the a~' rows, gates, Gamma_C, path flag
+            {
+                // all loads of a batch are issued before its stores
+                constexpr int NA = 64 * TP / 4;   // 16-byte pieces of A (1088 = 8.5 per thread)
+                const uint4 *src = reinterpret_cast<const uint4 *>(sm + P2_AF);
+                uint4 *dst = reinterpret_cast<uint4 *>(sm + P2_TB);
+                uint4 buf[9];
+#pragma unroll
+                for (int i = 0; i < 9; ++i) {
+                    const int e = btid + PF_BACK * i;
+                    if (e < NA) buf[i] = src[e];
+                }
+#pragma unroll
+                for (int i = 0; i < 9; ++i) {
+                    const int e = btid + PF_BACK * i;
+                    if (e < NA) dst[e] = buf[i];
+                }
+                uint4 qb[8];   // the a~' rows: 2 panels x 512 pieces
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int e = btid + PF_BACK * i, pnl = e >> 9;
+                    qb[i] = reinterpret_cast<const uint4 *>(sm + P2_QA + pnl * 16384)[e & 511];
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int e = btid + PF_BACK * i, pnl = e >> 9;
+                    reinterpret_cast<uint4 *>(sm + P2_AT + pnl * 8192)[e & 511] = qb[i];
+                }
+                reinterpret_cast<float *>(s_meta)[btid] = s_gamc[par * 128 + btid];
+            }
+            const bool fast = s_flags[par] != 0;
+            // the gates stay where the front put them: their buffer (item index mod 4) is not
+            // rewritten before this item is done
+            const float *s_bg1 = s_gates + (j & 3) * 128, *s_bg2 = s_bg1 + 64;
+            group_sync(BAR_BACK, PF_BACK);
+            if (btid == 0) mbar_arrive(bar_taken);
+            uint8_t *slot = P.ws + ((size_t)it.slot * H + it.h) * SLOT_BYTES;
+
+            // ---- |A| row sums (the exact path's second bound), before T overwrites A
+            bool well_a = true;
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {
+                const int pt = btid + PF_BACK * pp;
+                const int r = pt >> 2, kc0 = (pt & 3) * 2;
+                float asum = 0.f;
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) asum += fabsf(TB[r * TP + (kc0 + q2) * 8 + c]);
+#pragma unroll
+                for (int m = 1; m <= 2; m <<= 1) asum += __shfl_xor_sync(0xffffffffu, asum, m);
+                well_a = well_a && asum <= EXACT_A_NORM;
+            }
+
+            // ===== 3. T = (I + A)^{-1}, in place: 16x16 diagonal blocks, then recursive doubling
+            {
+                float xv[16];
+                const int I = btid >> 4, c = btid & 15;
+                if (btid < 64) {
+#pragma unroll
+                    for (int r2 = 0; r2 < 16; ++r2) {
+                        float arow[16];
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<float4 *>(arow + 4 * q4) =
+                                *reinterpret_cast<const float4 *>(TB + (16 * I + r2) * TP + 16 * I + 4 * q4);
+                        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                        for (int s2 = 0; s2 < r2; ++s2) {
+                            if (s2 & 1) acc1 = fmaf(arow[s2], xv[s2], acc1);
+                            else acc0 = fmaf(arow[s2], xv[s2], acc0);
+                        }
+                        xv[r2] = (r2 < c) ? 0.f : ((r2 == c) ? 1.f : -(acc0 + acc1));
+                    }
+                } else if (decoder) {   // meanwhile: the item four ahead
+                    ring_put(s_ring, j + 4, next_item_walk(a, N, nwork, wdec, ndec));
+                    wdec += gridDim.x;
+                }
+                group_sync(BAR_BACK, PF_BACK);   // every read of the diagonal blocks of A is done
+                if (btid < 64) {
+#pragma unroll
+                    for (int r2 = 0; r2 < 16; ++r2) TB[(16 * I + r2) * TP + 16 * I + c] = xv[r2];
+                }
+            }
+            group_sync(BAR_BACK, PF_BACK);
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {   // X = A_{I+1,I} D_I for I = 0, 2
+                const int pt = btid + PF_BACK * pp;
+                const int r2 = (pt >> 4) & 15, c2 = pt & 15;
+                float acc[2] = {0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 av = *reinterpret_cast<const float4 *>(TB + (16 * I + 16 + r2) * TP + 16 * I + 4 * m4);
+                        const float *tcol = TB + (16 * I + 4 * m4) * TP + 16 * I + c2;
+                        acc[blk] = fmaf(av.x, tcol[0], acc[blk]);
+                        acc[blk] = fmaf(av.y, tcol[TP], acc[blk]);
+                        acc[blk] = fmaf(av.z, tcol[2 * TP], acc[blk]);
+                        acc[blk] = fmaf(av.w, tcol[3 * TP], acc[blk]);
+                    }
+                }
+                Xs[pt] = acc[0];
+                Xs[256 + pt] = acc[1];
+            }
+            group_sync(BAR_BACK, PF_BACK);
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {   // T_{I+1,I} = -D_{I+1} X, over A_{I+1,I}
+                const int pt = btid + PF_BACK * pp;
+                const int r2 = (pt >> 4) & 15, c2 = pt & 15;
+                float acc[2] = {0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 tv = *reinterpret_cast<const float4 *>(TB + (16 * I + 16 + r2) * TP + 16 * I + 16 + 4 * m4);
+                        const float *xcol = Xs + (blk << 8) + (4 * m4) * 16 + c2;
+                        acc[blk] = fmaf(tv.x, xcol[0], acc[blk]);
+                        acc[blk] = fmaf(tv.y, xcol[16], acc[blk]);
+                        acc[blk] = fmaf(tv.z, xcol[32], acc[blk]);
+                        acc[blk] = fmaf(tv.w, xcol[48], acc[blk]);
+                    }
+                }
+                TB[(16 + r2) * TP + c2] = -acc[0];
+                TB[(48 + r2) * TP + 32 + c2] = -acc[1];
+            }
+            group_sync(BAR_BACK, PF_BACK);
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {   // X = A21 T1 (rows r0 + 8k, column c2)
+                const int pt = btid + PF_BACK * pp;
+                const int r0 = pt >> 5, c2 = pt & 31;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *tcol = TB + (4 * m4) * TP + c2;
+                    const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 av = *reinterpret_cast<const float4 *>(TB + (32 + r0 + 8 * k4) * TP + 4 * m4);
+                        acc[k4] = fmaf(av.x, t0v, acc[k4]);
+                        acc[k4] = fmaf(av.y, t1v, acc[k4]);
+                        acc[k4] = fmaf(av.z, t2v, acc[k4]);
+                        acc[k4] = fmaf(av.w, t3v, acc[k4]);
+                    }
+                }
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) Xs[(r0 + 8 * k4) * 32 + c2] = acc[k4];
+            }
+            group_sync(BAR_BACK, PF_BACK);
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {   // T21 = -T2 X, over A21 (read by the previous phase)
+                const int pt = btid + PF_BACK * pp;
+                const int r0 = pt >> 5, c2 = pt & 31;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *xcol = Xs + (4 * m4) * 32 + c2;
+                    const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 tv = *reinterpret_cast<const float4 *>(TB + (32 + r0 + 8 * k4) * TP + 32 + 4 * m4);
+                        acc[k4] = fmaf(tv.x, x0, acc[k4]);
+                        acc[k4] = fmaf(tv.y, x1, acc[k4]);
+                        acc[k4] = fmaf(tv.z, x2, acc[k4]);
+                        acc[k4] = fmaf(tv.w, x3, acc[k4]);
+                    }
+                }
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) TB[(32 + r0 + 8 * k4) * TP + c2] = -acc[k4];
+            }
+            group_sync(BAR_BACK, PF_BACK);
+
+            // ===== 4. T Diag(e) -> W = T Diag(e) a~'; the exact-path decision; T Diag(w) for the slot
+            const bool exact = !publish_and(write_t_copy(s_bg1, s_bg1, s_bg2) && well_a);
+            if (btid == 0) {
+                tc_fence_after();
+                const uint32_t id_w = idesc_bf16(64, 128, false, true);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tbase + TM_W, dK(sb + P2_TBF, 8192, kk), dMN(sb + P2_AT, 8192, kk), id_w, kk > 0);
+                mma_commit(bar_wmma);
+            }
+            if (!mbar_wait_cycles(bar_wmma, ph_wmma, WAIT_CYCLES)) ok = false;
+            ph_wmma ^= 1;
+            tc_fence_after();
+            if (!same_gates) {
+                write_t_copy(s_bg2, s_bg1, s_bg2);
+                fence_async_smem();
+                group_sync(BAR_BACK, PF_BACK);
+            }
+            // W (M = 64 layout: rows 16q..16q+15 in lanes 0..15 of quarter q) -> -W' in AT
+            {
+                const int r = quarter * 16 + (lane & 15);
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    float v[32];
+                    tmem_ld32(tbase + lane_base + TM_W + c4 * 32, v);
+                    tmem_wait_ld();
+                    if (lane < 16) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<uint4 *>(sm + P2_AT + sw_chunk(8192, r, c4 * 4 + q4)) =
+                                pack8_neg(v + q4 * 8);
+                    }
+                }
+            }
+            if (btid == 0) {   // status word and epoch tag of the slot
+                s_meta[128] = META_OK | (fast ? META_FAST : 0) | (exact ? META_EXACT : 0);
+                s_meta[129] = (int)P.epoch;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            ok = group_sync_and(BAR_BACK, PF_BACK, ok);
+            if (ok && lane == 0) {
+                if (bw == 0) bulk_store(slot + SL_QA, sm + P2_AT, 8192);                 // -W', panel 0
+                else if (bw == 1) bulk_store(slot + SL_QA + 16384, sm + P2_AT + 8192, 8192);   // -W', panel 1
+                else if (bw == 2) bulk_store(slot + SL_TBF, sm + P2_TBF, 8192);
+                else bulk_store(slot + SL_META, sm + P2_META, SL_META_BYTES);
+                bulk_commit();
+            }
+        }
+        if (lane == 0) bulk_wait_all();
+    }
+
+    __syncthreads();
+    tc_fence_after();
+    ok = __syncthreads_and(ok) != 0;
+    if (!ok && tid == 0) report_device_failure(DEV_WAIT_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tbase, 512);
@@ -1921,14 +2711,14 @@ cudaError_t device_setup(int &num_sms)
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!sms[dev]) {
-        if ((e = cudaFuncSetAttribute(chunk_fwd_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(chunk_fwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       SMEM_ALLOC)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(chunk_fwd_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            (e = cudaFuncSetAttribute(chunk_fwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       SMEM_ALLOC)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(chunk_fwd_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      SMEM_ALLOC)) != cudaSuccess ||
-            (e = cudaFuncSetAttribute(chunk_fwd_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      SMEM_ALLOC)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_prep_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      P2_ALLOC)) != cudaSuccess ||
+            (e = cudaFuncSetAttribute(chunk_prep_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      P2_ALLOC)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(chunk_chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       CK_ALLOC)) != cudaSuccess ||
             (e = cudaFuncSetAttribute(chunk_chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1982,17 +2772,18 @@ cudaError_t launch_chunk_fwd_sm100(const FwdArgs &a, cudaStream_t st)
     ChunkParams p;
     if ((e = make_params(p, a)) != cudaSuccess) return e;
     const int N = a.cu_seqlens ? a.num_seqs : a.B;
-    if (a.prep) chunk_fwd_kernel<false, true><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
-    else chunk_fwd_kernel<false, false><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
+    if (a.prep) chunk_fwd_kernel<true><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
+    else chunk_fwd_kernel<false><<<(unsigned)(N * a.H), NT, SMEM_ALLOC, st>>>(p);
     return cudaGetLastError();
 }
 
 bool chunk_prefer_split(const FwdArgs &a)
 {
     // Cost model from measured kernel times on B200 (thousands of SM cycles per chunk):
-    // preparation of one (chunk, head) ~15.0, the split chain ~4.4, the fused kernel's
-    // critical path ~16.3.  With U = N*H units on S SMs and W = ceil(U / S) waves of the
-    // per-unit kernels:  fused ~ W * 16.3,  split ~ (U / S) * 15.0 + W * 4.4  (per chunk).
+    // preparation of one (chunk, head) by the two-group split kernel ~12.0, the split chain
+    // ~4.4, the fused kernel's critical path ~16.3.  With U = N*H units on S SMs and
+    // W = ceil(U / S) waves of the per-unit kernels:  fused ~ W * 16.3,
+    // split ~ (U / S) * 12.0 + W * 4.4  (per chunk).
     // Packed (varlen) batches take the split form: the fused kernel's time is that of the
     // longest sequence per CTA, while the preparation kernel balances chunks over all SMs.
     int num_sms = 0;
@@ -2003,7 +2794,7 @@ bool chunk_prefer_split(const FwdArgs &a)
     if (a.cu_seqlens) return true;
     const double U = (double)a.B * a.H, S = num_sms;
     const double W = std::ceil(U / S);
-    return (U / S) * 15.0 + W * 4.4 < W * 16.3;
+    return (U / S) * 12.0 + W * 4.4 < W * 16.3;
 }
 
 size_t chunk_split_workspace_bytes(const FwdArgs &a)
@@ -2030,8 +2821,8 @@ cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st
     const long long nwork = (long long)p.nslots * a.H;
     if (rows > 0 && nwork > 0) {
         const unsigned grid = (unsigned)std::min<long long>(nwork, num_sms);
-        if (a.prep) chunk_fwd_kernel<true, true><<<grid, NPREP, SMEM_ALLOC, st>>>(p);
-        else chunk_fwd_kernel<true, false><<<grid, NPREP, SMEM_ALLOC, st>>>(p);
+        if (a.prep) chunk_prep_kernel<true><<<grid, PF_NT, P2_ALLOC, st>>>(p);
+        else chunk_prep_kernel<false><<<grid, PF_NT, P2_ALLOC, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (a.snap) chunk_chain_kernel<true><<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);
