@@ -561,6 +561,15 @@ def chunk_line(name, inp, r, world, steps, traffic_key=None):
 
 # ---------------------------------------------------------------------------
 
+ONLY = {
+    "ckda": (HEADLINE, lambda seed: W.ckda_bf16(seed)),
+    "kda": ("KDA-range chunked forward B=4 H=16 T=4096 d=128 chunk=64 bf16", lambda seed: W.kda_bf16(seed)),
+    "rda": ("RDA packed documents: 16 docs of U[512,4096] tokens, H=32", lambda seed: W.varlen_bf16("rda", seed)),
+    "gdn2": ("GDN-2 packed documents: 16 docs of U[512,4096] tokens, H=32",
+             lambda seed: W.varlen_bf16("gdn2", seed)),
+}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -574,6 +583,9 @@ def main():
     ap.add_argument("--backward-steps", type=int, default=20)
     ap.add_argument("--form", choices=sorted(FORM_FLAGS), default="auto",
                     help="form of the tensor-core chunked path (auto = the library's shape-based choice)")
+    ap.add_argument("--only", choices=sorted(ONLY) + ["decode"], default=None,
+                    help="time one workload alone (no e2e, no other workloads, no CPU baseline; for profiler "
+                         "captures) and print its line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -588,6 +600,24 @@ def main():
     peaks = load_peaks()
     seed = rank_workload_seed(rank)
     fflags = FORM_FLAGS[args.form]
+    if args.only == "decode":
+        r = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank, e2e=False)
+        if rank == 0:
+            print(json.dumps(r))
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    if args.only:
+        name, mk = ONLY[args.only]
+        x = mk(seed)
+        r = run_chunk_workload(x, args.steps, args.warmup, world, peaks, e2e=False, flags=fflags)
+        if rank == 0:
+            print(json.dumps(chunk_line(name, x, r, world, args.steps)))
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     sampler = ClockSampler(local) if rank == 0 else None
     # the headline: Complex KDA, B=8 H=16 T=8192
     inp = W.ckda_bf16(seed)
