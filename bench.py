@@ -583,7 +583,7 @@ def main():
     ap.add_argument("--backward-steps", type=int, default=20)
     ap.add_argument("--form", choices=sorted(FORM_FLAGS), default="auto",
                     help="form of the tensor-core chunked path (auto = the library's shape-based choice)")
-    ap.add_argument("--only", choices=sorted(ONLY) + ["decode"], default=None,
+    ap.add_argument("--only", choices=sorted(ONLY) + ["backward", "decode"], default=None,
                     help="time one workload alone (no e2e, no other workloads, no CPU baseline; for profiler "
                          "captures) and print its line")
     args = ap.parse_args()
@@ -600,6 +600,14 @@ def main():
     peaks = load_peaks()
     seed = rank_workload_seed(rank)
     fflags = FORM_FLAGS[args.form]
+    if args.only == "backward":
+        r = run_backward_workload(W.kda_bf16(seed), args.backward_steps, args.warmup, world, rank)
+        if rank == 0:
+            print(json.dumps(r))
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     if args.only == "decode":
         r = run_decode_workload(args.decode_steps, args.warmup, world, peaks, rank, e2e=False)
         if rank == 0:
