@@ -41,6 +41,7 @@
  *                           state, optional snapshots every 64 tokens)
  *   kda_chunk_bwd           every gradient of that forward (fp32)
  *   kda_chunk_fwd_rank2     two erase/write sub-steps per token
+ *   kda_chunk_bwd_rank2     every gradient of the rank-2 forward (fp32)
  *   kda_decode_step         one token per (sequence, head), state in place
  *   *_workspace_size        bytes of the caller-owned workspace of each call
  *   kda_check_gates, kda_check_seqlens   device checks of the inputs' contracts
@@ -286,6 +287,36 @@ int kda_chunk_bwd(int variant, int gate_range, int dtype,
                   float *dq, float *dk, float *dv, float *dalpha, float *dg1, float *dg2,
                   float *d_initial_state, void *workspace, size_t workspace_bytes,
                   unsigned flags, void *stream);
+
+/*
+ * kda_chunk_bwd_rank2 -- gradients of kda_chunk_fwd_rank2 (two erase/write
+ * sub-steps per token: the DeltaProduct_2-style composition the "Complex KDA"
+ * arXiv abstract names as prior work), for L with dL/do = d_o [B,T,H,d_v] (the
+ * inputs' dtype) and dL/dS_final = d_final_state (NULL = 0).
+ * Layouts as for kda_chunk_fwd_rank2: q, alpha, d_o and their gradients dq,
+ * dalpha per token [B,T,H,.]; k, v, g1, g2 and their gradients dk, dv, dg1,
+ * dg2 with the sub-step axis after T ([B,T,2,H,.]); all gradients fp32.
+ * A rank-2 step is two rank-1 steps of the same recurrence, the second with
+ * alpha = 1 and the readout after it, so the gradient is the rank-1 backward
+ * (kda_chunk_bwd, same arithmetic and tolerance) over the 2T sub-tokens with
+ * d_o on the second ones, mapped back: dq from the second sub-tokens, dalpha
+ * from the first; the k, v and gate gradients are already in the caller's
+ * layout.  Caller-owned workspace of kda_chunk_bwd_rank2_workspace_size bytes
+ * (16-byte aligned): the expanded q, alpha, d_o, the sub-token dq, dalpha,
+ * the doubled offsets and the rank-1 backward's workspace.  No flags.
+ * Errors as kda_chunk_bwd; everything is checked before anything is launched.
+ */
+size_t kda_chunk_bwd_rank2_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
+                                          int has_cu_seqlens, int num_seqs);
+int kda_chunk_bwd_rank2(int variant, int gate_range, int dtype,
+                        int B, int T, int H, int d_k, int d_v,
+                        const void *q, const void *k, const void *v, const void *alpha,
+                        const void *g1, const void *g2,
+                        const int32_t *cu_seqlens, int num_seqs, const float *initial_state,
+                        const void *d_o, const float *d_final_state,
+                        float *dq, float *dk, float *dv, float *dalpha, float *dg1, float *dg2,
+                        float *d_initial_state, void *workspace, size_t workspace_bytes,
+                        unsigned flags, void *stream);
 
 /*
  * kda_decode_step -- one recurrent step for N sequences (single-token decode;

@@ -17,7 +17,8 @@ from typing import Optional, Union
 
 import torch
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "KdaChunkFunction", "kda_chunk_fwd_rank2", "kda_decode_step",
+__all__ = ["kda_chunk_fwd", "kda_chunk_bwd", "KdaChunkFunction", "kda_chunk_fwd_rank2", "kda_chunk_bwd_rank2",
+           "kda_decode_step",
            "kda_check_gates", "kda_check_seqlens", "kda_device_status", "kda_error_string", "kda_version",
            "KdaError", "VARIANTS", "RANGES", "LIB_PATH", "FLAG_VALIDATE_RANGE", "FLAG_FORCE_SCAN",
            "FLAG_FORCE_FUSED", "FLAG_FORCE_SPLIT", "FLAG_GATE_LOGITS", "FLAG_L2NORM_K", "FLAG_DEBUG_STALL",
@@ -49,6 +50,7 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     for name in ("kda_chunk_fwd", "kda_chunk_fwd_ws", "kda_chunk_fwd_workspace_size", "kda_chunk_bwd",
                  "kda_chunk_bwd_workspace_size", "kda_chunk_fwd_rank2", "kda_chunk_fwd_rank2_workspace_size",
+                 "kda_chunk_bwd_rank2", "kda_chunk_bwd_rank2_workspace_size",
                  "kda_decode_step", "kda_check_gates", "kda_check_seqlens", "kda_device_status", "kda_error_string",
                  "kda_last_error_detail", "kda_version"):
         if not hasattr(lib, name):
@@ -71,6 +73,10 @@ def _load():
                                          ctypes.c_uint, _vp])
     lib.kda_chunk_fwd_rank2_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_fwd_rank2_workspace_size.argtypes = [_i] * 9 + [ctypes.c_uint]
+    lib.kda_chunk_bwd_rank2.restype = _i
+    lib.kda_chunk_bwd_rank2.argtypes = lib.kda_chunk_bwd.argtypes
+    lib.kda_chunk_bwd_rank2_workspace_size.restype = ctypes.c_size_t
+    lib.kda_chunk_bwd_rank2_workspace_size.argtypes = [_i] * 8
     lib.kda_decode_step.restype = _i
     lib.kda_decode_step.argtypes = [_i] * 7 + [_vp] * 6 + [_vp, _vp, ctypes.c_uint, _vp]
     lib.kda_check_gates.restype = _i
@@ -354,6 +360,60 @@ def kda_chunk_fwd_rank2(variant: Union[str, int], gate_range: Union[str, int], q
     if rc != 0:
         raise KdaError(rc, "kda_chunk_fwd_rank2")
     return o, final_state
+
+
+def kda_chunk_bwd_rank2(variant: Union[str, int], gate_range: Union[str, int], q: torch.Tensor, k: torch.Tensor,
+                        v: torch.Tensor, alpha: torch.Tensor, g1: torch.Tensor, g2: Optional[torch.Tensor],
+                        d_o: torch.Tensor, d_final_state: Optional[torch.Tensor] = None,
+                        cu_seqlens: Optional[torch.Tensor] = None, initial_state: Optional[torch.Tensor] = None,
+                        d_initial_state: bool = True, stream=None):
+    """Gradients of rank-2 steps (C: kda_chunk_bwd_rank2).  Inputs as for
+    kda_chunk_fwd_rank2, d_o [B,T,H,d_v] in their dtype, d_final_state fp32
+    [N,H,d_k,d_v] or None.  Returns fp32 (dq, dk, dv, dalpha, dg1, dg2,
+    d_initial_state) shaped like q, k, v, alpha, g1, g2 (None for KDA) and the
+    state (None unless ``d_initial_state``)."""
+    var = _code(VARIANTS, variant, "variant")
+    rng = _code(RANGES, gate_range, "gate_range")
+    if q.dim() != 4 or k.dim() != 5:
+        raise ValueError("q must be [B,T,H,d_k] and k [B,T,2,H,d_k]")
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, dt = q.device, q.dtype
+    if dt not in _DTYPES:
+        raise ValueError(f"dtype {dt} unsupported (bf16 or fp32)")
+    for t, name, shape in ((q, "q", (B, T, H, dk)), (alpha, "alpha", (B, T, H, dk)), (d_o, "d_o", (B, T, H, dv)),
+                           (k, "k", (B, T, 2, H, dk)), (v, "v", (B, T, 2, H, dv)),
+                           (g1, "g1", (B, T, 2, H, dk) if var == 2 else (B, T, 2, H))):
+        _check(t, name, dt, shape, dev)
+    if var != 0:
+        if g2 is None:
+            raise ValueError("RDA and GDN-2 need g2 (write gate)")
+        _check(g2, "g2", dt, (B, T, 2, H, dv) if var == 2 else (B, T, 2, H), dev)
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 CUDA tensor")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    _check(initial_state, "initial_state", torch.float32, (N, H, dk, dv), dev)
+    _check(d_final_state, "d_final_state", torch.float32, (N, H, dk, dv), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    grads = [torch.empty(t.shape, **f32) for t in (q, k, v, alpha, g1)]
+    grads.append(torch.empty(g2.shape, **f32) if var != 0 else None)
+    grads.append(torch.empty((N, H, dk, dv), **f32) if d_initial_state else None)
+    ws_bytes = lib.kda_chunk_bwd_rank2_workspace_size(_DTYPES[dt], B, T, H, dk, dv, int(cu_seqlens is not None), N)
+    if ws_bytes == 0:
+        raise KdaError(1, "kda_chunk_bwd_rank2_workspace_size")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if stream is not None and stream != torch.cuda.current_stream(dev):
+        ws.record_stream(stream)
+    rc = lib.kda_chunk_bwd_rank2(var, rng, _DTYPES[dt], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                 _ptr(g1), _ptr(g2), _ptr(cu_seqlens), N, _ptr(initial_state), _ptr(d_o),
+                                 _ptr(d_final_state), *[_ptr(x) for x in grads], _ptr(ws), ws_bytes, 0,
+                                 _stream(stream, dev))
+    if rc != 0:
+        raise KdaError(rc, "kda_chunk_bwd_rank2")
+    return tuple(grads)
 
 
 def num_chunk_slots(B: int, T: int, N: int) -> int:

@@ -465,8 +465,108 @@ extern "C" int kda_chunk_fwd_rank2(int variant, int gate_range, int dtype,
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_rank2 expand");
     rc = chunk_launch(a, dtype, chunk_size, flags, w + L.chunk, L.chunk_bytes, st);
     if (rc != KDA_OK) return rc;
-    e = kda::launch_rank2_gather(bf16, w + L.o2, o, tokens, H * d_v, st);
+    e = kda::launch_rank2_gather(bf16, w + L.o2, o, tokens, H * d_v, 1, st);
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_fwd_rank2 gather");
+    return KDA_OK;
+}
+
+namespace {
+
+// Gradient of rank-2 steps: workspace regions (256-byte aligned) for the
+// sub-token problem of B x 2T tokens: q2, alpha2 [B,2T,H,d_k] and d_o2
+// [B,2T,H,d_v] in the input dtype, dq2 and dalpha2 [B,2T,H,d_k] fp32, the
+// doubled cu_seqlens, then the rank-1 backward's own workspace.
+struct Rank2BwdLayout {
+    size_t q2, a2, do2, dq2, da2, cu2, bwd, bwd_bytes, total;
+};
+
+Rank2BwdLayout rank2_bwd_layout(int dtype, int B, int T, int H, int d_k, int d_v, int has_cu, int num_seqs)
+{
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    const size_t tok2 = (size_t)B * 2 * (size_t)T * H;
+    Rank2BwdLayout L;
+    L.q2 = 0;
+    L.a2 = up(tok2 * d_k * es);
+    L.do2 = L.a2 + up(tok2 * d_k * es);
+    L.dq2 = L.do2 + up(tok2 * d_v * es);
+    L.da2 = L.dq2 + up(tok2 * d_k * 4);
+    L.cu2 = L.da2 + up(tok2 * d_k * 4);
+    L.bwd = L.cu2 + up(has_cu ? (size_t)(num_seqs + 1) * 4 : 0);
+    L.bwd_bytes = kda_chunk_bwd_workspace_size(dtype, B, 2 * T, H, d_k, d_v, has_cu, num_seqs);
+    L.total = L.bwd + up(L.bwd_bytes);
+    return L;
+}
+
+}  // namespace
+
+extern "C" size_t kda_chunk_bwd_rank2_workspace_size(int dtype, int B, int T, int H, int d_k, int d_v,
+                                                     int has_cu_seqlens, int num_seqs)
+{
+    if (!rank2_sizes_ok(dtype, B, T, H, d_k, d_v, has_cu_seqlens, num_seqs)) return 0;
+    return rank2_bwd_layout(dtype, B, T, H, d_k, d_v, has_cu_seqlens, num_seqs).total;
+}
+
+extern "C" int kda_chunk_bwd_rank2(int variant, int gate_range, int dtype,
+                                   int B, int T, int H, int d_k, int d_v,
+                                   const void *q, const void *k, const void *v, const void *alpha,
+                                   const void *g1, const void *g2,
+                                   const int32_t *cu_seqlens, int num_seqs, const float *initial_state,
+                                   const void *d_o, const float *d_final_state,
+                                   float *dq, float *dk, float *dv, float *dalpha, float *dg1, float *dg2,
+                                   float *d_initial_state, void *workspace, size_t workspace_bytes,
+                                   unsigned flags, void *stream)
+{
+    if (flags) return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_rank2 takes no flags (got 0x%x)", flags);
+    if (B < 1 || T < 0 || H < 1 || T > (1 << 29))
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d (need B>=1, 0<=T<=2^29, H>=1)", B, T, H);
+    if (dtype != KDA_DTYPE_BF16 && dtype != KDA_DTYPE_F32) return fail(KDA_ERR_INVALID_ARG, "bad dtype %d", dtype);
+    if (!head_dim_ok(d_k) || !head_dim_ok(d_v))
+        return fail(KDA_ERR_UNSUPPORTED, "head dims d_k=%d d_v=%d: supported are 16, 32, 64, 128", d_k, d_v);
+    if (!rank2_sizes_ok(dtype, B, T, H, d_k, d_v, cu_seqlens != nullptr, num_seqs))
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%d T=%d H=%d num_seqs=%d (cu_seqlens needs B == 1)", B, T, H,
+                    num_seqs);
+    if (T > 0) {
+        const void *need[] = {q, alpha, d_o, dq, dalpha, dk, dv, dg1};
+        const char *names[] = {"q", "alpha", "d_o", "dq", "dalpha", "dk", "dv", "dg1"};
+        for (int i = 0; i < 8; ++i) {
+            if (!need[i]) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", names[i]);
+            if (!aligned16(need[i])) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+        }
+        if (variant != KDA_VARIANT_KDA && (!dg2 || !aligned16(dg2)))
+            return fail(KDA_ERR_INVALID_ARG, "dg2 is NULL or misaligned (RDA and GDN-2 have a write gate)");
+    }
+    if ((d_final_state && !aligned16(d_final_state)) || (d_initial_state && !aligned16(d_initial_state)))
+        return fail(KDA_ERR_INVALID_ARG, "d_final_state / d_initial_state is not 16-byte aligned");
+    if (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return fail(KDA_ERR_INVALID_ARG, "cu_seqlens is not 4-byte aligned");
+    const Rank2BwdLayout L = rank2_bwd_layout(dtype, B, T, H, d_k, d_v, cu_seqlens != nullptr, num_seqs);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < L.total)
+        return fail(KDA_ERR_INVALID_ARG, "kda_chunk_bwd_rank2 needs a 16-byte aligned workspace of %zu bytes",
+                    L.total);
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    int32_t *cu2 = cu_seqlens ? reinterpret_cast<int32_t *>(w + L.cu2) : nullptr;
+    // the sub-token problem's own checks (k, v, gates; variant, range, sizes) before anything is launched
+    kda::FwdArgs chk;
+    int rc = chunk_args(chk, variant, gate_range, dtype, B, 2 * T, H, d_k, d_v, w + L.q2, k, v, w + L.a2, g1, g2,
+                        cu2, num_seqs, initial_state, nullptr, w + L.do2, 64, 0u);
+    if (rc != KDA_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool bf16 = dtype == KDA_DTYPE_BF16;
+    const long long tokens = (long long)B * T;
+    cudaError_t e = kda::launch_rank2_expand(bf16, q, alpha, w + L.q2, w + L.a2, tokens, H * d_k, cu_seqlens, cu2,
+                                             cu_seqlens ? num_seqs + 1 : 0, st);
+    if (e == cudaSuccess) e = kda::launch_rank2_spread(bf16, d_o, w + L.do2, tokens, H * d_v, st);
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd_rank2 expand");
+    // k, v and the gates (and their gradients) are already in the sub-token layout [B,2T,H,.]
+    rc = kda_chunk_bwd(variant, gate_range, dtype, B, 2 * T, H, d_k, d_v, w + L.q2, k, v, w + L.a2, g1, g2, cu2,
+                       num_seqs, initial_state, w + L.do2, d_final_state, reinterpret_cast<float *>(w + L.dq2), dk,
+                       dv, reinterpret_cast<float *>(w + L.da2), dg1, dg2, d_initial_state, w + L.bwd, L.bwd_bytes,
+                       0u, stream);
+    if (rc != KDA_OK) return rc;
+    e = kda::launch_rank2_gather(false, w + L.dq2, dq, tokens, H * d_k, 1, st);   // q enters the second sub-token
+    if (e == cudaSuccess) e = kda::launch_rank2_gather(false, w + L.da2, dalpha, tokens, H * d_k, 0, st);   // alpha the first
+    if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd_rank2 gather");
     return KDA_OK;
 }
 

@@ -5,8 +5,10 @@
 //   sub-token 2t+1: decay 1, (k, v, gates) of sub-step 2, readout = o_t
 // The caller's k, v and gate tensors carry the sub-step axis after T
 // ([B,T,2,H,.]), which in memory is already the sub-token order [B,2T,H,.];
-// only q and alpha are expanded, and o gathered, by the two copy kernels here
-// (16-byte vectors, grid-stride).
+// only q and alpha are expanded, and o gathered, by the copy kernels here
+// (16-byte vectors, grid-stride).  The gradient of rank-2 steps is the rank-1
+// backward over the same sub-tokens with d_o spread onto the second sub-tokens,
+// mapped back: dq from the second sub-tokens, dalpha from the first.
 #include "rank2.cuh"
 
 namespace kda {
@@ -35,13 +37,26 @@ __global__ void rank2_expand_kernel(const uint4 *q, const uint4 *alpha, uint4 *q
         for (long long i = first; i < n_cu; i += stride) cu2[i] = 2 * cu[i];
 }
 
-__global__ void rank2_gather_kernel(const uint4 *o2, uint4 *o, long long tokens, int row_vecs)
+__global__ void rank2_gather_kernel(const uint4 *o2, uint4 *o, long long tokens, int row_vecs, int parity)
 {
     const long long stride = (long long)gridDim.x * blockDim.x;
     const long long n = tokens * row_vecs;
     for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
         const long long tok = e / row_vecs, r = e % row_vecs;
-        o[e] = o2[(2 * tok + 1) * row_vecs + r];
+        o[e] = o2[(2 * tok + parity) * row_vecs + r];
+    }
+}
+
+// x2[2t] = 0, x2[2t+1] = x[t]: a per-token tensor onto the sub-tokens, present on the second
+__global__ void rank2_spread_kernel(const uint4 *x, uint4 *x2, long long tokens, int row_vecs)
+{
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const long long n = tokens * row_vecs;
+    const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += stride) {
+        const long long tok = e / row_vecs, r = e % row_vecs;
+        x2[2 * tok * row_vecs + r] = zero;
+        x2[(2 * tok + 1) * row_vecs + r] = x[e];
     }
 }
 
@@ -66,12 +81,22 @@ cudaError_t launch_rank2_expand(bool bf16, const void *q, const void *alpha, voi
     return cudaGetLastError();
 }
 
-cudaError_t launch_rank2_gather(bool bf16, const void *o2, void *o, long long tokens, int row_elems, cudaStream_t st)
+cudaError_t launch_rank2_gather(bool bf16, const void *o2, void *o, long long tokens, int row_elems, int parity,
+                                cudaStream_t st)
 {
     const int row_vecs = row_elems * (bf16 ? 2 : 4) / 16;
     if (tokens == 0) return cudaSuccess;
     rank2_gather_kernel<<<blocks_for(tokens * row_vecs), COPY_THREADS, 0, st>>>(
-        static_cast<const uint4 *>(o2), static_cast<uint4 *>(o), tokens, row_vecs);
+        static_cast<const uint4 *>(o2), static_cast<uint4 *>(o), tokens, row_vecs, parity);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rank2_spread(bool bf16, const void *x, void *x2, long long tokens, int row_elems, cudaStream_t st)
+{
+    const int row_vecs = row_elems * (bf16 ? 2 : 4) / 16;
+    if (tokens == 0) return cudaSuccess;
+    rank2_spread_kernel<<<blocks_for(tokens * row_vecs), COPY_THREADS, 0, st>>>(
+        static_cast<const uint4 *>(x), static_cast<uint4 *>(x2), tokens, row_vecs);
     return cudaGetLastError();
 }
 

@@ -272,3 +272,23 @@ def test_check_seqlens_rejects_bad_arguments(lib):
     assert lib.kda_check_seqlens(P, 2, -1, P, None) == 1
     assert lib.kda_check_seqlens(P, 2, 10, None, None) == 1
     assert lib.kda_check_seqlens(ctypes.c_void_p(0x10002), 2, 10, P, None) == 1
+
+
+def test_rank2_bwd_rejects_bad_arguments(lib):
+    """Every check happens before anything is launched (fake pointers never reach a kernel)."""
+    f = lib.kda_chunk_bwd_rank2
+    f.restype = ctypes.c_int
+
+    def call(flags=0, q=P, d_o=P, dq=P, ws=P, ws_bytes=1 << 30, dk=128):
+        return f(0, 0, 0, 1, 8, 1, dk, 128, q, P, P, P, P, None, None, 0, None, d_o, None, dq, P, P, P, P, None,
+                 None, ws, ctypes.c_size_t(ws_bytes), flags, None)
+    assert call(flags=1) == INVALID
+    assert call(q=None) == INVALID
+    assert call(d_o=BAD) == INVALID
+    assert call(dq=None) == INVALID
+    assert call(ws_bytes=16) == INVALID
+    assert call(ws=BAD) == INVALID
+    assert call(dk=48) == UNSUPPORTED
+    lib.kda_chunk_bwd_rank2_workspace_size.restype = ctypes.c_size_t
+    need = lib.kda_chunk_bwd_rank2_workspace_size(0, 1, 8, 1, 128, 128, 0, 1)
+    assert need > lib.kda_chunk_bwd_workspace_size(0, 1, 16, 1, 128, 128, 0, 1)

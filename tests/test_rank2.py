@@ -94,3 +94,92 @@ def test_rank2_empty_batch_passes_state_through():
                               init_state="random")
     o, sf = _run(inp)
     assert o.numel() == 0 and torch.equal(sf.cpu(), inp.initial_state)
+
+
+# ---- gradients of rank-2 steps (kda_chunk_bwd_rank2) --------------------------------------------
+
+GRAD_TOL = 1e-3   # fp32 arithmetic throughout, as for the rank-1 backward
+
+
+def _grad_close(g, r, what):
+    g2 = g.reshape(-1, g.shape[-1]) if g.ndim > 1 else g.reshape(-1, 1)
+    r2 = r.reshape(-1, r.shape[-1]) if r.ndim > 1 else r.reshape(-1, 1)
+    assert np.all(np.isfinite(g2)), f"{what}: non-finite"
+    if g2.size == 0:
+        return
+    err = np.abs(g2 - r2).max(axis=1)
+    scale = np.maximum(1.0, np.abs(r2).max(axis=1))
+    worst = int(np.argmax(err / scale))
+    assert err[worst] <= GRAD_TOL * scale[worst], \
+        f"{what}: row {worst} error {err[worst]:.3e} > {GRAD_TOL} * {scale[worst]:.3e}"
+
+
+def _rank2_grad_ref(inp, d_o, dsf, n, h):
+    """The oracle's reverse mode over the 2T sub-tokens of (sequence n, head h), mapped back."""
+    f64 = lambda t: None if t is None else t.double().numpy()
+    b, t0, ln = inp.seq_bounds(n)
+    s0 = None if inp.initial_state is None else f64(inp.initial_state[n, h])
+    if ln == 0:   # an empty sequence hands dL/dS_final straight to its initial state
+        return {"ds0": np.zeros((inp.d_k, inp.d_v)) if dsf is None else f64(dsf[n, h])}
+    sl = slice(t0, t0 + ln)
+    q, al, do = f64(inp.q[b, sl, h]), f64(inp.alpha[b, sl, h]), f64(d_o[b, sl, h])
+    def sub(t):   # [B,T,2,H,(d)] -> the sequence's 2 ln sub-tokens of head h
+        if t is None:
+            return None
+        x = f64(t[b, sl, :, h])
+        return x.reshape((2 * ln,) + x.shape[2:])
+    k2, v2, g12, g22 = sub(inp.k), sub(inp.v), sub(inp.g1), sub(inp.g2)
+    q2 = np.stack([np.zeros_like(q), q], axis=1).reshape(2 * ln, -1)
+    a2 = np.stack([al, np.ones_like(al)], axis=1).reshape(2 * ln, -1)
+    do2 = np.stack([np.zeros_like(do), do], axis=1).reshape(2 * ln, -1)
+    g = oracle.recurrence_grad(inp.variant, q2, k2, v2, a2, g12, g22, s0, do2, None if dsf is None else f64(dsf[n, h]))
+    pair = lambda x: None if x is None else x.reshape((ln, 2) + x.shape[1:])
+    return {"dq": g["dq"][1::2], "dalpha": g["dalpha"][0::2], "dk": pair(g["dk"]), "dv": pair(g["dv"]),
+            "dg1": pair(g["dg1"]), "dg2": pair(g["dg2"]), "ds0": g["ds0"]}
+
+
+@pytest.mark.parametrize("variant,gate_range", [("kda", "standard"), ("kda", "extended"), ("rda", "standard"),
+                                                ("gdn2", "extended")])
+@pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("f32", 32, 64)])
+def test_rank2_backward_matches_the_oracle(variant, gate_range, dtype, dk, dv):
+    import linear_rnn_delta_b200 as kda
+    inp = W.make_rank2_inputs(variant, gate_range, dtype, H=2, d_k=dk, d_v=dv, seed=93, doc_lens=[70, 0, 1, 33],
+                              init_state="random", init_std=0.2)
+    d_o, dsf = W.grad_outputs(inp, seed=93)
+    c = lambda t: None if t is None else t.cuda().contiguous()
+    got = kda.kda_chunk_bwd_rank2(inp.variant, inp.gate_range, c(inp.q), c(inp.k), c(inp.v), c(inp.alpha),
+                                  c(inp.g1), c(inp.g2), c(d_o), c(dsf), cu_seqlens=c(inp.cu_seqlens),
+                                  initial_state=c(inp.initial_state))
+    torch.cuda.synchronize()
+    names = ("dq", "dk", "dv", "dalpha", "dg1", "dg2", "ds0")
+    got = {nm: (None if t is None else t.double().cpu().numpy()) for nm, t in zip(names, got)}
+    for n in range(inp.num_seqs):
+        b, t0, ln = inp.seq_bounds(n)
+        for h in range(inp.H):
+            ref = _rank2_grad_ref(inp, d_o, dsf, n, h)
+            _grad_close(got["ds0"][n, h], ref["ds0"], f"ds0[{n},{h}]")
+            if ln == 0:
+                continue
+            for nm in ("dq", "dalpha"):
+                _grad_close(got[nm][b, t0:t0 + ln, h], ref[nm], f"{nm}[{n},{h}]")
+            for nm in ("dk", "dv", "dg1", "dg2"):
+                if ref[nm] is not None:
+                    _grad_close(got[nm][b, t0:t0 + ln, :, h], ref[nm], f"{nm}[{n},{h}]")
+
+
+def test_rank2_backward_fixed_length_without_final_gradient():
+    import linear_rnn_delta_b200 as kda
+    inp = W.make_rank2_inputs("rda", "extended", "bf16", B=2, T=45, H=3, d_k=64, d_v=64, seed=94)
+    d_o, _ = W.grad_outputs(inp, seed=94, d_final=False)
+    c = lambda t: None if t is None else t.cuda().contiguous()
+    got = kda.kda_chunk_bwd_rank2(inp.variant, inp.gate_range, c(inp.q), c(inp.k), c(inp.v), c(inp.alpha),
+                                  c(inp.g1), c(inp.g2), c(d_o), None, d_initial_state=False)
+    torch.cuda.synchronize()
+    assert got[6] is None
+    for n in range(inp.B):
+        for h in range(inp.H):
+            ref = _rank2_grad_ref(inp, d_o, None, n, h)
+            _grad_close(got[0][n, :, h].double().cpu().numpy(), ref["dq"], "dq")
+            _grad_close(got[3][n, :, h].double().cpu().numpy(), ref["dalpha"], "dalpha")
+            _grad_close(got[1][n, :, :, h].double().cpu().numpy(), ref["dk"], "dk")
+            _grad_close(got[5][n, :, :, h].double().cpu().numpy(), ref["dg2"], "dg2")
