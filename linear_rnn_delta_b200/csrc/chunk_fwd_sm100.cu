@@ -1561,7 +1561,8 @@ constexpr uint32_t P2_RING = P2_MISC + 8992;         // int [8][8]: decoded item
 constexpr uint32_t P2_FLAGS = P2_MISC + 9248;        // int [2] path flags by item parity, [1] abort
 constexpr uint32_t P2_BAR = P2_MISC + 9264;          // mbarriers: tma, v, pmma, wmma, full, taken
 constexpr uint32_t P2_TMEM = P2_MISC + 9312;
-constexpr uint32_t P2_ALLOC = P2_MISC + 9328 + 1024;
+constexpr uint32_t P2_APART = P2_MISC + 9328;        // float [2][2][64]: |A| half-row sums by item parity
+constexpr uint32_t P2_ALLOC = P2_MISC + 10352 + 1024;
 static_assert(P2_ALLOC <= 232448, "shared memory budget");
 static_assert(P2_FR + 40960 <= P2_TB && P2_LB + 16384 <= P2_TB && P2_PBF + 8192 <= P2_TB, "front region");
 static_assert(P2_TB + 64 * TP * 4 <= P2_TBF && P2_TBF + 8192 <= P2_MT && P2_MT + 16384 <= P2_MISC, "back region");
@@ -1666,6 +1667,7 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
         const int tg = ptid >> 5, cq = ptid & 31;
         uint32_t ph_tma = 0, ph_v = 0, ph_pmma = 0, ph_taken = 0;
         float *Af = reinterpret_cast<float *>(sm + P2_AF);
+        float *s_apart = reinterpret_cast<float *>(sm + P2_APART);
         auto issue_tma = [&](const Item &it) {
             const int g = it.row0 + it.c * C;
             mbar_expect_tx(bar_tma, 3 * 16384);
@@ -2013,6 +2015,14 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                         const int s = phalf * 32 + c;
                         v[c] = (s < rr) ? v[c] * er : 0.f;
                     }
+                    // |A| over this half row, as two 16-column sums (the order the fused kernel adds them in)
+                    float g0 = 0.f, g1s = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        g0 += fabsf(v[c]);
+                        g1s += fabsf(v[16 + c]);
+                    }
+                    s_apart[(par * 2 + phalf) * 64 + rr] = g0 + g1s;
 #pragma unroll
                     for (int q4 = 0; q4 < 8; ++q4)
                         *reinterpret_cast<float4 *>(Af + rr * TP + phalf * 32 + 4 * q4) =
@@ -2081,6 +2091,14 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                         if (ptid - w >= 0)
                             *reinterpret_cast<unsigned short *>(sm + P2_PBF + sw_elem(8192, ptid, ptid - w)) =
                                 bf16_bits(s_pband[ptid * PBAND + w]);
+                }
+                {   // |A| half-row sums: four threads per row, 16 columns each, adjacent lanes paired
+                    const int r = ptid >> 2, m = ptid & 3;
+                    float g = 0.f;
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) g += fabsf(Af[r * TP + 16 * m + c]);
+                    g += __shfl_xor_sync(0xffffffffu, g, 1);
+                    if (!(m & 1)) s_apart[(par * 2 + (m >> 1)) * 64 + r] = g;
                 }
             }
             fence_async_smem();
@@ -2205,20 +2223,15 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
             if (btid == 0) mbar_arrive(bar_taken);
             uint8_t *slot = P.ws + ((size_t)it.slot * H + it.h) * SLOT_BYTES;
 
-            // ---- |A| row sums (the exact path's second bound), before T overwrites A
+            // ---- |A| row sums (the exact path's second bound), from the front's half-row sums
             bool well_a = true;
-#pragma unroll 1
-            for (int pp = 0; pp < 2; ++pp) {
-                const int pt = btid + PF_BACK * pp;
-                const int r = pt >> 2, kc0 = (pt & 3) * 2;
-                float asum = 0.f;
+            {
+                const float *ap = reinterpret_cast<const float *>(sm + P2_APART) + par * 128;
 #pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) asum += fabsf(TB[r * TP + (kc0 + q2) * 8 + c]);
-#pragma unroll
-                for (int m = 1; m <= 2; m <<= 1) asum += __shfl_xor_sync(0xffffffffu, asum, m);
-                well_a = well_a && asum <= EXACT_A_NORM;
+                for (int pp = 0; pp < 2; ++pp) {
+                    const int r = (btid + PF_BACK * pp) >> 2;
+                    well_a = well_a && (ap[r] + ap[64 + r]) <= EXACT_A_NORM;
+                }
             }
 
             // ===== 3. T = (I + A)^{-1}, in place: 16x16 diagonal blocks, then recursive doubling
@@ -2296,48 +2309,50 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                 TB[(48 + r2) * TP + 32 + c2] = -acc[1];
             }
             group_sync(BAR_BACK, PF_BACK);
-#pragma unroll 1
-            for (int pp = 0; pp < 2; ++pp) {   // X = A21 T1 (rows r0 + 8k, column c2)
-                const int pt = btid + PF_BACK * pp;
-                const int r0 = pt >> 5, c2 = pt & 31;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            {   // X = A21 T1: warp bw takes rows bw + 4i (i < 8), lane c2 column c2; a column of T1
+                // serves the warp's eight rows (each output summed in the fused kernel's order)
+                const int c2 = lane;
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
                 for (int m4 = 0; m4 < 8; ++m4) {
                     const float *tcol = TB + (4 * m4) * TP + c2;
                     const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const float4 av = *reinterpret_cast<const float4 *>(TB + (32 + r0 + 8 * k4) * TP + 4 * m4);
-                        acc[k4] = fmaf(av.x, t0v, acc[k4]);
-                        acc[k4] = fmaf(av.y, t1v, acc[k4]);
-                        acc[k4] = fmaf(av.z, t2v, acc[k4]);
-                        acc[k4] = fmaf(av.w, t3v, acc[k4]);
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 av = *reinterpret_cast<const float4 *>(TB + (32 + bw + 4 * i) * TP + 4 * m4);
+                        acc[i] = fmaf(av.x, t0v, acc[i]);
+                        acc[i] = fmaf(av.y, t1v, acc[i]);
+                        acc[i] = fmaf(av.z, t2v, acc[i]);
+                        acc[i] = fmaf(av.w, t3v, acc[i]);
                     }
                 }
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) Xs[(r0 + 8 * k4) * 32 + c2] = acc[k4];
+                for (int i = 0; i < 8; ++i) Xs[(bw + 4 * i) * 32 + c2] = acc[i];
             }
             group_sync(BAR_BACK, PF_BACK);
-#pragma unroll 1
-            for (int pp = 0; pp < 2; ++pp) {   // T21 = -T2 X, over A21 (read by the previous phase)
-                const int pt = btid + PF_BACK * pp;
-                const int r0 = pt >> 5, c2 = pt & 31;
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            {   // T21 = -T2 X, over A21 (read by the previous phase); same row split
+                const int c2 = lane;
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
                 for (int m4 = 0; m4 < 8; ++m4) {
                     const float *xcol = Xs + (4 * m4) * 32 + c2;
                     const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        const float4 tv = *reinterpret_cast<const float4 *>(TB + (32 + r0 + 8 * k4) * TP + 32 + 4 * m4);
-                        acc[k4] = fmaf(tv.x, x0, acc[k4]);
-                        acc[k4] = fmaf(tv.y, x1, acc[k4]);
-                        acc[k4] = fmaf(tv.z, x2, acc[k4]);
-                        acc[k4] = fmaf(tv.w, x3, acc[k4]);
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 tv =
+                            *reinterpret_cast<const float4 *>(TB + (32 + bw + 4 * i) * TP + 32 + 4 * m4);
+                        acc[i] = fmaf(tv.x, x0, acc[i]);
+                        acc[i] = fmaf(tv.y, x1, acc[i]);
+                        acc[i] = fmaf(tv.z, x2, acc[i]);
+                        acc[i] = fmaf(tv.w, x3, acc[i]);
                     }
                 }
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) TB[(32 + r0 + 8 * k4) * TP + c2] = -acc[k4];
+                for (int i = 0; i < 8; ++i) TB[(32 + bw + 4 * i) * TP + c2] = -acc[i];
             }
             group_sync(BAR_BACK, PF_BACK);
 
