@@ -447,6 +447,26 @@ def run_rank2_workload(inp, steps, warmup, world):
     return {"tokens_per_step": inp.B * inp.T, "total_s": total, "avg_launch_s": sum(per) / len(per)}
 
 
+def run_rank2_backward_workload(inp, steps, warmup, world, rank):
+    """kda_chunk_bwd_rank2 (gradients of rank-2 steps) with seeded d_o ~ N(0,1), dL/dS_final ~ N(0, 0.01)."""
+    import linear_rnn_delta_b200 as kda
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    d = {n: (None if getattr(inp, n) is None else getattr(inp, n).to(dev)) for n in
+         ("q", "k", "v", "alpha", "g1", "g2")}
+    g = torch.Generator().manual_seed(rank_workload_seed(rank) * 7 + 3)
+    d_o = torch.randn((inp.B, inp.T, inp.H, inp.d_v), generator=g).to(dev, d["q"].dtype)
+    dsf = (0.1 * torch.randn((inp.B, inp.H, inp.d_k, inp.d_v), generator=g)).to(dev)
+
+    def step():
+        kda.kda_chunk_bwd_rank2(inp.variant, inp.gate_range, d["q"], d["k"], d["v"], d["alpha"], d["g1"], d["g2"],
+                                d_o, dsf, stream=stream)
+
+    total, per = time_launches(step, steps, warmup, world, stream)
+    total = max_over_ranks(total, world)
+    return {"tokens_per_step": inp.B * inp.T, "total_s": total, "avg_launch_s": sum(per) / len(per)}
+
+
 def host_cores() -> int:
     """Cores this process may run on (its CPU affinity)."""
     try:
@@ -671,6 +691,11 @@ def main():
                                  "q/alpha expansion + chunked forward over 4096 sub-tokens + o gather",
                      "value": r["tokens_per_step"] * world * args.steps / r["total_s"], "unit": UNIT,
                      "ms_per_step": r["total_s"] / args.steps * 1e3})
+        r = run_rank2_backward_workload(x, args.backward_steps, args.warmup, world, rank)
+        also.append({"workload": "gradients of KDA rank-2 steps B=4 H=16 T=2048 d=128 bf16 inputs, fp32 "
+                                 "arithmetic: d_o spread + rank-1 backward over 4096 sub-tokens + dq/dalpha gathers",
+                     "value": r["tokens_per_step"] * world * args.backward_steps / r["total_s"], "unit": UNIT,
+                     "ms_per_step": r["total_s"] / args.backward_steps * 1e3})
         del x
     if rank != 0:
         if world > 1:
