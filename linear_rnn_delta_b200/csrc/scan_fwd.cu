@@ -1,14 +1,22 @@
 // Token-by-token fp32 scan of the gated delta-rule recurrence.
 //
 // Serves every shape/dtype the tensor-core chunked kernel does not (fp32
-// inputs, head dims 16..128), and is the exact-order reference path on the
-// GPU.  One CTA per (sequence, head); thread j owns value column j of the
-// state and keeps S[:, j] (d_k fp32) in registers for the whole sequence.
+// inputs, head dims 16..128), writes the backward pass's fp32 checkpoints,
+// and is the exact-order reference path on the GPU.
 // The columns of S evolve independently: the left operator
 // (I - k a~^T) Diag(alpha) acts on every column alike and the written value
 // m enters column j only through m_j (update equations on the
-// Raon-1-mini-preview discussion page), so no thread talks to another except
-// through the shared per-token vectors.
+// Raon-1-mini-preview discussion page), so a column needs nothing from the
+// others but the shared per-token vectors.  Lanes work in groups of KS
+// (16, or d_k / 4 below d_k = 64) adjacent lanes; a group owns CC = 4 (2 for
+// the smallest heads) adjacent value columns, and lane p of it keeps rows
+// i = 4 (m KS + p) + e (e < 4) of them in registers for the whole sequence.  The two sums over key rows are
+// in-thread partial sums and log2(KS) butterfly shuffles, after which every
+// lane of the group holds the same bits.  Per token a lane reads 3 d_k / KS
+// floats of the shared token vectors and uses each for CC columns, so the
+// shared-memory pipe, which bounds this kernel, delivers 3 d_k / CC floats
+// per column and token (one float per lane and wavefront).  A CTA serves 64 columns (all of them when
+// d_v < 64) of one (sequence, head).
 //
 // Per token (decay, residual, write, readout):
 //   u_j  = m_j - sum_i (alpha_i a~_i) S_ij
@@ -16,7 +24,8 @@
 //   o_j  = sum_i q_i S_ij
 // Token vectors are staged TB tokens at a time in shared memory so the inner
 // loop runs without barriers; optional input preparation (gate activations,
-// L2 norm of k) is applied while staging.
+// L2 norm of k) is applied while staging.  Without an output (the backward's
+// checkpoints) the readout is compiled out.
 #include "common.cuh"
 
 namespace kda {
@@ -28,20 +37,63 @@ constexpr int SB = 4;   // elements per thread loaded before any is widened (sta
 __device__ __forceinline__ float widen(float x) { return x; }
 __device__ __forceinline__ float widen(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// PREP: input preparation requested; without it that code is compiled out.
-template <int DK, int DV, typename TIn, bool PREP>
-__global__ void __launch_bounds__(DV)
+template <int DK, int DV> struct ScanShape {
+    static constexpr int KS = DK >= 64 ? 16 : DK / 4;      // lanes per group (rows split KS ways)
+    static constexpr int NG = DK / (4 * KS);               // float4 row groups per lane
+    static constexpr int CB = DV < 64 ? DV : 64;           // value columns per CTA
+    static constexpr int CC = CB / 4 * KS >= 32 ? 4 : 2;   // value columns per group (whole warps)
+    static constexpr int NTH = CB / CC * KS;               // threads per CTA
+    static constexpr int CTAS = DV / CB;                   // CTAs per (sequence, head)
+    static_assert(NG >= 1 && NTH % 32 == 0, "scan shape");
+};
+
+// CC consecutive floats (16- or 8-byte aligned)
+template <int CC> __device__ __forceinline__ void ld_cols(const float *p, float (&x)[CC])
+{
+    if constexpr (CC == 4) {
+        const float4 t = *reinterpret_cast<const float4 *>(p);
+        x[0] = t.x; x[1] = t.y; x[2] = t.z; x[3] = t.w;
+    } else {
+        const float2 t = *reinterpret_cast<const float2 *>(p);
+        x[0] = t.x; x[1] = t.y;
+    }
+}
+template <int CC> __device__ __forceinline__ void st_cols(float *p, const float (&x)[CC])
+{
+    if constexpr (CC == 4) *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    else *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+}
+
+// Sum of x over the KS lanes of a group; every lane gets the same bits (each
+// butterfly step adds the same two values, in one order or the other).
+template <int KS>
+__device__ __forceinline__ float group_sum(float x)
+{
+#pragma unroll
+    for (int off = 1; off < KS; off <<= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+
+// PREP: input preparation requested; OUT: o is written.  Without either, that
+// code is compiled out.
+template <int DK, int DV, typename TIn, bool PREP, bool OUT>
+__global__ void __launch_bounds__(ScanShape<DK, DV>::NTH)
 scan_fwd_kernel(FwdArgs a)
 {
+    using SH = ScanShape<DK, DV>;
+    constexpr int KS = SH::KS, NG = SH::NG, CB = SH::CB, CC = SH::CC, NTH = SH::NTH, CTAS = SH::CTAS;
     __shared__ __align__(16) float s_aa[TB][DK];   // alpha_i * a~_i
     __shared__ __align__(16) float s_al[TB][DK];   // alpha_i
     __shared__ __align__(16) float s_k[TB][DK];
-    __shared__ __align__(16) float s_q[TB][DK];
-    __shared__ __align__(16) float s_m[TB][DV];
+    __shared__ __align__(16) float s_q[OUT ? TB : 1][DK];
+    __shared__ __align__(16) float s_m[TB][CB];
     __shared__ float s_ksc[TB];   // 1 / ||k_t|| (input preparation)
 
-    const int n = blockIdx.x / a.H, h = blockIdx.x % a.H;
-    const int j = threadIdx.x;
+    const int pair = blockIdx.x / CTAS, cblk = blockIdx.x % CTAS;
+    const int n = pair / a.H, h = pair % a.H;
+    const int tid = threadIdx.x, p = tid % KS, grp = tid / KS;
+    const int cl = grp * CC;        // first of the group's columns within the CTA
+    const int j = cblk * CB + cl;   // ... and within the head
     int b, t0, len;
     if (a.cu_seqlens) { b = 0; t0 = a.cu_seqlens[n]; len = a.cu_seqlens[n + 1] - t0; }
     else { b = n; t0 = 0; len = a.T; }
@@ -49,10 +101,21 @@ scan_fwd_kernel(FwdArgs a)
     const TIn *q = (const TIn *)a.q, *k = (const TIn *)a.k, *v = (const TIn *)a.v;
     const TIn *al = (const TIn *)a.alpha, *g1 = (const TIn *)a.g1, *g2 = (const TIn *)a.g2;
     const size_t soff = ((size_t)n * a.H + h) * DK * DV;
+    auto row = [&](int m, int e) { return 4 * (m * KS + p) + e; };
 
-    float S[DK];
+    // S[4 m + e][c] = S_{row(m, e), j + c}
+    float S[4 * NG][CC];
 #pragma unroll
-    for (int i = 0; i < DK; ++i) S[i] = a.s0 ? a.s0[soff + (size_t)i * DV + j] : 0.f;
+    for (int m = 0; m < NG; ++m)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (a.s0) {
+                ld_cols<CC>(a.s0 + soff + (size_t)row(m, e) * DV + j, S[4 * m + e]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < CC; ++c) S[4 * m + e][c] = 0.f;
+            }
+        }
 
     const bool logits = PREP && (a.prep & PREP_LOGITS), l2k = PREP && (a.prep & PREP_L2NORM_K), ext = a.ext != 0;
     for (int base = 0; base < len; base += TB) {
@@ -60,23 +123,23 @@ scan_fwd_kernel(FwdArgs a)
         __syncthreads();  // previous block of tokens fully consumed
         // loads are issued SB elements at a time and widened afterwards: widening
         // each one as it arrives would wait out every load's latency in turn
-        for (int e0 = j; e0 < nt * DK; e0 += DV * SB) {
+        for (int e0 = tid; e0 < nt * DK; e0 += NTH * SB) {
             TIn rk[SB], ra[SB], rg[SB], rq[SB];
 #pragma unroll
             for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * DV;
+                const int e = e0 + bb * NTH;
                 if (e < nt * DK) {
                     const int tt = e / DK, i = e % DK;
                     const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
                     rk[bb] = k[tok * DK + i];
                     ra[bb] = al[tok * DK + i];
                     rg[bb] = (a.variant == GDN2) ? g1[tok * DK + i] : g1[tok];
-                    rq[bb] = q[tok * DK + i];
+                    if (OUT) rq[bb] = q[tok * DK + i];
                 }
             }
 #pragma unroll
             for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * DV;
+                const int e = e0 + bb * NTH;
                 if (e < nt * DK) {
                     const int tt = e / DK, i = e % DK;
                     const float kk = widen(rk[bb]);
@@ -88,17 +151,17 @@ scan_fwd_kernel(FwdArgs a)
                     s_k[tt][i] = kk;
                     s_al[tt][i] = aa;
                     s_aa[tt][i] = l2k ? aa * g : aa * (g * kk);   // times k once it is normalised
-                    s_q[tt][i] = widen(rq[bb]);
+                    if (OUT) s_q[tt][i] = widen(rq[bb]);
                 }
             }
         }
-        for (int e0 = j; e0 < nt * DV; e0 += DV * SB) {
+        for (int e0 = tid; e0 < nt * CB; e0 += NTH * SB) {
             TIn rv[SB], rw[SB];
 #pragma unroll
             for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * DV;
-                if (e < nt * DV) {
-                    const int tt = e / DV, jj = e % DV;
+                const int e = e0 + bb * NTH;
+                if (e < nt * CB) {
+                    const int tt = e / CB, jj = cblk * CB + e % CB;
                     const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
                     rw[bb] = a.variant == KDA ? g1[tok] : (a.variant == RDA ? g2[tok] : g2[tok * DV + jj]);
                     rv[bb] = v[tok * DV + jj];
@@ -106,23 +169,23 @@ scan_fwd_kernel(FwdArgs a)
             }
 #pragma unroll
             for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * DV;
-                if (e < nt * DV) {
+                const int e = e0 + bb * NTH;
+                if (e < nt * CB) {
                     float g = widen(rw[bb]);
                     if (logits) g = round_to<TIn>(prep_gate(g, ext));
-                    s_m[e / DV][e % DV] = g * widen(rv[bb]);
+                    s_m[e / CB][e % CB] = g * widen(rv[bb]);
                 }
             }
         }
         __syncthreads();
         if (l2k) {   // k_t / ||k_t||, then a~ = (alpha g) (.) k
-            for (int tt = j; tt < nt; tt += DV) {
+            for (int tt = tid; tt < nt; tt += NTH) {
                 float ss = 0.f;
                 for (int i = 0; i < DK; ++i) ss = fmaf(s_k[tt][i], s_k[tt][i], ss);
                 s_ksc[tt] = prep_kscale(ss);
             }
             __syncthreads();
-            for (int e = j; e < nt * DK; e += DV) {
+            for (int e = tid; e < nt * DK; e += NTH) {
                 const int tt = e / DK, i = e % DK;
                 const float kn = round_to<TIn>(s_k[tt][i] * s_ksc[tt]);
                 s_k[tt][i] = kn;
@@ -131,59 +194,92 @@ scan_fwd_kernel(FwdArgs a)
             __syncthreads();
         }
         for (int tt = 0; tt < nt; ++tt) {
-            float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+            float r[CC][2];
 #pragma unroll
-            for (int i = 0; i < DK; i += 4) {
-                const float4 c = *reinterpret_cast<const float4 *>(&s_aa[tt][i]);
-                r0 = fmaf(c.x, S[i], r0);
-                r1 = fmaf(c.y, S[i + 1], r1);
-                r2 = fmaf(c.z, S[i + 2], r2);
-                r3 = fmaf(c.w, S[i + 3], r3);
+            for (int c = 0; c < CC; ++c) r[c][0] = r[c][1] = 0.f;
+#pragma unroll
+            for (int m = 0; m < NG; ++m) {
+                const float4 x = *reinterpret_cast<const float4 *>(&s_aa[tt][row(m, 0)]);
+#pragma unroll
+                for (int c = 0; c < CC; ++c) {
+                    r[c][0] = fmaf(x.x, S[4 * m][c], r[c][0]);
+                    r[c][1] = fmaf(x.y, S[4 * m + 1][c], r[c][1]);
+                    r[c][0] = fmaf(x.z, S[4 * m + 2][c], r[c][0]);
+                    r[c][1] = fmaf(x.w, S[4 * m + 3][c], r[c][1]);
+                }
             }
-            const float u = s_m[tt][j] - ((r0 + r1) + (r2 + r3));
-            float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+            float u[CC];
+            ld_cols<CC>(&s_m[tt][cl], u);
 #pragma unroll
-            for (int i = 0; i < DK; i += 4) {
-                const float4 av = *reinterpret_cast<const float4 *>(&s_al[tt][i]);
-                const float4 kv = *reinterpret_cast<const float4 *>(&s_k[tt][i]);
-                const float4 qv = *reinterpret_cast<const float4 *>(&s_q[tt][i]);
-                S[i] = fmaf(av.x, S[i], kv.x * u);
-                S[i + 1] = fmaf(av.y, S[i + 1], kv.y * u);
-                S[i + 2] = fmaf(av.z, S[i + 2], kv.z * u);
-                S[i + 3] = fmaf(av.w, S[i + 3], kv.w * u);
-                o0 = fmaf(qv.x, S[i], o0);
-                o1 = fmaf(qv.y, S[i + 1], o1);
-                o2 = fmaf(qv.z, S[i + 2], o2);
-                o3 = fmaf(qv.w, S[i + 3], o3);
+            for (int c = 0; c < CC; ++c) u[c] -= group_sum<KS>(r[c][0] + r[c][1]);
+            float o[CC][2];
+#pragma unroll
+            for (int c = 0; c < CC; ++c) o[c][0] = o[c][1] = 0.f;
+#pragma unroll
+            for (int m = 0; m < NG; ++m) {
+                const float4 av = *reinterpret_cast<const float4 *>(&s_al[tt][row(m, 0)]);
+                const float4 kv = *reinterpret_cast<const float4 *>(&s_k[tt][row(m, 0)]);
+                const float a4[4] = {av.x, av.y, av.z, av.w}, k4[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+#pragma unroll
+                    for (int c = 0; c < CC; ++c) S[4 * m + e][c] = fmaf(a4[e], S[4 * m + e][c], k4[e] * u[c]);
+                if (OUT) {
+                    const float4 qv = *reinterpret_cast<const float4 *>(&s_q[tt][row(m, 0)]);
+                    const float q4[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+#pragma unroll
+                        for (int c = 0; c < CC; ++c) o[c][e & 1] = fmaf(q4[e], S[4 * m + e][c], o[c][e & 1]);
+                }
             }
             const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
-            if (a.o) st_out((TIn *)a.o + tok * DV + j, (o0 + o1) + (o2 + o3));   // null: states only
+            if (OUT) {
+                float ov[CC];
+#pragma unroll
+                for (int c = 0; c < CC; ++c) ov[c] = group_sum<KS>(o[c][0] + o[c][1]);
+                if (p == 0) {
+#pragma unroll
+                    for (int c = 0; c < CC; ++c) st_out((TIn *)a.o + tok * DV + j + c, ov[c]);
+                }
+            }
             const int t = base + tt;   // token index within the sequence
             if (a.snap && ((t + 1) % SLOT_TOKENS == 0 || t + 1 == len)) {   // state after a 64-token chunk
                 float *dst = a.snap + ((size_t)(slot_base(a, n) + t / SLOT_TOKENS) * a.H + h) * DK * DV + j;
 #pragma unroll
-                for (int i = 0; i < DK; ++i) dst[(size_t)i * DV] = S[i];
+                for (int m = 0; m < NG; ++m)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) st_cols<CC>(dst + (size_t)row(m, e) * DV, S[4 * m + e]);
             }
         }
     }
     if (a.sf) {
 #pragma unroll
-        for (int i = 0; i < DK; ++i) a.sf[soff + (size_t)i * DV + j] = S[i];
+        for (int m = 0; m < NG; ++m)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st_cols<CC>(a.sf + soff + (size_t)row(m, e) * DV + j, S[4 * m + e]);
     }
+}
+
+// Variants launched: with output, with or without input preparation; states
+// only (the backward's checkpoints), without preparation.
+template <int DK, int DV, typename TIn>
+void launch_typed(const FwdArgs &a, dim3 grid, cudaStream_t st)
+{
+    constexpr int NTH = ScanShape<DK, DV>::NTH;
+    if (a.prep) scan_fwd_kernel<DK, DV, TIn, true, true><<<grid, NTH, 0, st>>>(a);
+    else if (a.o) scan_fwd_kernel<DK, DV, TIn, false, true><<<grid, NTH, 0, st>>>(a);
+    else scan_fwd_kernel<DK, DV, TIn, false, false><<<grid, NTH, 0, st>>>(a);
 }
 
 template <int DK, int DV>
 cudaError_t launch_dims(const FwdArgs &a, bool bf16, cudaStream_t st)
 {
+    if (a.prep && !a.o) return cudaErrorInvalidValue;   // no such variant (and no caller)
     const int N = a.cu_seqlens ? a.num_seqs : a.B;
-    dim3 grid((unsigned)(N * a.H)), block(DV);
-    if (bf16) {
-        if (a.prep) scan_fwd_kernel<DK, DV, __nv_bfloat16, true><<<grid, block, 0, st>>>(a);
-        else scan_fwd_kernel<DK, DV, __nv_bfloat16, false><<<grid, block, 0, st>>>(a);
-    } else {
-        if (a.prep) scan_fwd_kernel<DK, DV, float, true><<<grid, block, 0, st>>>(a);
-        else scan_fwd_kernel<DK, DV, float, false><<<grid, block, 0, st>>>(a);
-    }
+    const dim3 grid((unsigned)(N * a.H * ScanShape<DK, DV>::CTAS));
+    if (bf16) launch_typed<DK, DV, __nv_bfloat16>(a, grid, st);
+    else launch_typed<DK, DV, float>(a, grid, st);
     return cudaGetLastError();
 }
 
