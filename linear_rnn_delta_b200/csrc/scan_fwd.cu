@@ -22,17 +22,16 @@
 //   u_j  = m_j - sum_i (alpha_i a~_i) S_ij
 //   S_ij = alpha_i S_ij + k_i u_j
 //   o_j  = sum_i q_i S_ij
-// Token vectors are staged TB tokens at a time in shared memory so the inner
-// loop runs without barriers; optional input preparation (gate activations,
-// L2 norm of k) is applied while staging.  Without an output (the backward's
+// Token vectors are staged TB tokens at a time in shared memory, double
+// buffered, so the inner loop runs without barriers; optional input
+// preparation (gate activations, L2 norm of k) is applied while staging.  Without an output (the backward's
 // checkpoints) the readout is compiled out.
 #include "common.cuh"
 
 namespace kda {
 namespace {
 
-constexpr int TB = 16;  // tokens staged per barrier
-constexpr int SB = 4;   // elements per thread loaded before any is widened (staging)
+constexpr int TB = 8;   // tokens per staged block (two blocks in shared memory)
 
 __device__ __forceinline__ float widen(float x) { return x; }
 __device__ __forceinline__ float widen(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -58,10 +57,10 @@ template <int CC> __device__ __forceinline__ void ld_cols(const float *p, float 
         x[0] = t.x; x[1] = t.y;
     }
 }
-template <int CC> __device__ __forceinline__ void st_cols(float *p, const float (&x)[CC])
+template <int CC> __device__ __forceinline__ void st_cols(float *p, const float2 (&x)[CC / 2])
 {
-    if constexpr (CC == 4) *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
-    else *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+    if constexpr (CC == 4) *reinterpret_cast<float4 *>(p) = make_float4(x[0].x, x[0].y, x[1].x, x[1].y);
+    else *reinterpret_cast<float2 *>(p) = x[0];
 }
 
 // Sum of x over the KS lanes of a group; every lane gets the same bits (each
@@ -82,11 +81,11 @@ scan_fwd_kernel(FwdArgs a)
 {
     using SH = ScanShape<DK, DV>;
     constexpr int KS = SH::KS, NG = SH::NG, CB = SH::CB, CC = SH::CC, NTH = SH::NTH, CTAS = SH::CTAS;
-    __shared__ __align__(16) float s_aa[TB][DK];   // alpha_i * a~_i
-    __shared__ __align__(16) float s_al[TB][DK];   // alpha_i
-    __shared__ __align__(16) float s_k[TB][DK];
-    __shared__ __align__(16) float s_q[OUT ? TB : 1][DK];
-    __shared__ __align__(16) float s_m[TB][CB];
+    __shared__ __align__(16) float s_aa[2][TB][DK];   // alpha_i * a~_i (two blocks of tokens)
+    __shared__ __align__(16) float s_al[2][TB][DK];   // alpha_i
+    __shared__ __align__(16) float s_k[2][TB][DK];
+    __shared__ __align__(16) float s_q[2][OUT ? TB : 1][DK];
+    __shared__ __align__(16) float s_m[2][TB][CB];
     __shared__ float s_ksc[TB];   // 1 / ||k_t|| (input preparation)
 
     const int pair = blockIdx.x / CTAS, cblk = blockIdx.x % CTAS;
@@ -103,141 +102,159 @@ scan_fwd_kernel(FwdArgs a)
     const size_t soff = ((size_t)n * a.H + h) * DK * DV;
     auto row = [&](int m, int e) { return 4 * (m * KS + p) + e; };
 
-    // S[4 m + e][c] = S_{row(m, e), j + c}
-    float S[4 * NG][CC];
+    // S2[4 m + e][c] = (S_{row(m, e), j + 2c}, S_{row(m, e), j + 2c + 1})
+    float2 S2[4 * NG][CC / 2];
 #pragma unroll
     for (int m = 0; m < NG; ++m)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            if (a.s0) {
-                ld_cols<CC>(a.s0 + soff + (size_t)row(m, e) * DV + j, S[4 * m + e]);
-            } else {
+        for (int e = 0; e < 4; ++e)
 #pragma unroll
-                for (int c = 0; c < CC; ++c) S[4 * m + e][c] = 0.f;
-            }
-        }
+            for (int c = 0; c < CC / 2; ++c)
+                S2[4 * m + e][c] = a.s0 ? *reinterpret_cast<const float2 *>(a.s0 + soff + (size_t)row(m, e) * DV + j + 2 * c)
+                                        : make_float2(0.f, 0.f);
 
     const bool logits = PREP && (a.prep & PREP_LOGITS), l2k = PREP && (a.prep & PREP_L2NORM_K), ext = a.ext != 0;
-    for (int base = 0; base < len; base += TB) {
+    // Token vectors of block b+1 are loaded into registers (raw) while block b
+    // is computed, then widened, prepared and stored to the other buffer: the
+    // loads' latency hides behind a block's arithmetic and each block costs
+    // one barrier.
+    constexpr int EK = (TB * DK + NTH - 1) / NTH, EM = (TB * CB + NTH - 1) / NTH;
+    TIn pk[EK], pa[EK], pg[EK], pq[OUT ? EK : 1], pv[EM], pw[EM];
+    auto fetch = [&](int base) {
         const int nt = min(TB, len - base);
-        __syncthreads();  // previous block of tokens fully consumed
-        // loads are issued SB elements at a time and widened afterwards: widening
-        // each one as it arrives would wait out every load's latency in turn
-        for (int e0 = tid; e0 < nt * DK; e0 += NTH * SB) {
-            TIn rk[SB], ra[SB], rg[SB], rq[SB];
 #pragma unroll
-            for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * NTH;
-                if (e < nt * DK) {
-                    const int tt = e / DK, i = e % DK;
-                    const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
-                    rk[bb] = k[tok * DK + i];
-                    ra[bb] = al[tok * DK + i];
-                    rg[bb] = (a.variant == GDN2) ? g1[tok * DK + i] : g1[tok];
-                    if (OUT) rq[bb] = q[tok * DK + i];
-                }
-            }
-#pragma unroll
-            for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * NTH;
-                if (e < nt * DK) {
-                    const int tt = e / DK, i = e % DK;
-                    const float kk = widen(rk[bb]);
-                    float aa = widen(ra[bb]), g = widen(rg[bb]);
-                    if (logits) {
-                        aa = round_to<TIn>(prep_alpha(aa, ext));
-                        g = round_to<TIn>(prep_gate(g, ext));
-                    }
-                    s_k[tt][i] = kk;
-                    s_al[tt][i] = aa;
-                    s_aa[tt][i] = l2k ? aa * g : aa * (g * kk);   // times k once it is normalised
-                    if (OUT) s_q[tt][i] = widen(rq[bb]);
-                }
+        for (int x = 0; x < EK; ++x) {
+            const int e = tid + x * NTH;
+            if (e < nt * DK) {
+                const int tt = e / DK, i = e % DK;
+                const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
+                pk[x] = k[tok * DK + i];
+                pa[x] = al[tok * DK + i];
+                pg[x] = (a.variant == GDN2) ? g1[tok * DK + i] : g1[tok];
+                if (OUT) pq[x] = q[tok * DK + i];
             }
         }
-        for (int e0 = tid; e0 < nt * CB; e0 += NTH * SB) {
-            TIn rv[SB], rw[SB];
 #pragma unroll
-            for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * NTH;
-                if (e < nt * CB) {
-                    const int tt = e / CB, jj = cblk * CB + e % CB;
-                    const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
-                    rw[bb] = a.variant == KDA ? g1[tok] : (a.variant == RDA ? g2[tok] : g2[tok * DV + jj]);
-                    rv[bb] = v[tok * DV + jj];
-                }
-            }
-#pragma unroll
-            for (int bb = 0; bb < SB; ++bb) {
-                const int e = e0 + bb * NTH;
-                if (e < nt * CB) {
-                    float g = widen(rw[bb]);
-                    if (logits) g = round_to<TIn>(prep_gate(g, ext));
-                    s_m[e / CB][e % CB] = g * widen(rv[bb]);
-                }
+        for (int x = 0; x < EM; ++x) {
+            const int e = tid + x * NTH;
+            if (e < nt * CB) {
+                const int tt = e / CB, jj = cblk * CB + e % CB;
+                const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
+                pw[x] = a.variant == KDA ? g1[tok] : (a.variant == RDA ? g2[tok] : g2[tok * DV + jj]);
+                pv[x] = v[tok * DV + jj];
             }
         }
-        __syncthreads();
+    };
+    auto commit = [&](int buf, int base) {
+        const int nt = min(TB, len - base);
+#pragma unroll
+        for (int x = 0; x < EK; ++x) {
+            const int e = tid + x * NTH;
+            if (e < nt * DK) {
+                const int tt = e / DK, i = e % DK;
+                const float kk = widen(pk[x]);
+                float aa = widen(pa[x]), g = widen(pg[x]);
+                if (logits) {
+                    aa = round_to<TIn>(prep_alpha(aa, ext));
+                    g = round_to<TIn>(prep_gate(g, ext));
+                }
+                s_k[buf][tt][i] = kk;
+                s_al[buf][tt][i] = aa;
+                s_aa[buf][tt][i] = l2k ? aa * g : aa * (g * kk);   // times k once it is normalised
+                if (OUT) s_q[buf][tt][i] = widen(pq[x]);
+            }
+        }
+#pragma unroll
+        for (int x = 0; x < EM; ++x) {
+            const int e = tid + x * NTH;
+            if (e < nt * CB) {
+                float g = widen(pw[x]);
+                if (logits) g = round_to<TIn>(prep_gate(g, ext));
+                s_m[buf][e / CB][e % CB] = g * widen(pv[x]);
+            }
+        }
+    };
+    if (len > 0) {
+        fetch(0);
+        commit(0, 0);
+    }
+    __syncthreads();
+    for (int base = 0, blk = 0; base < len; base += TB, ++blk) {
+        const int nt = min(TB, len - base), buf = blk & 1;
+        const bool more = base + TB < len;
+        if (more) fetch(base + TB);
         if (l2k) {   // k_t / ||k_t||, then a~ = (alpha g) (.) k
             for (int tt = tid; tt < nt; tt += NTH) {
                 float ss = 0.f;
-                for (int i = 0; i < DK; ++i) ss = fmaf(s_k[tt][i], s_k[tt][i], ss);
+                for (int i = 0; i < DK; ++i) ss = fmaf(s_k[buf][tt][i], s_k[buf][tt][i], ss);
                 s_ksc[tt] = prep_kscale(ss);
             }
             __syncthreads();
             for (int e = tid; e < nt * DK; e += NTH) {
                 const int tt = e / DK, i = e % DK;
-                const float kn = round_to<TIn>(s_k[tt][i] * s_ksc[tt]);
-                s_k[tt][i] = kn;
-                s_aa[tt][i] *= kn;
+                const float kn = round_to<TIn>(s_k[buf][tt][i] * s_ksc[tt]);
+                s_k[buf][tt][i] = kn;
+                s_aa[buf][tt][i] *= kn;
             }
             __syncthreads();
         }
         for (int tt = 0; tt < nt; ++tt) {
-            float r[CC][2];
+            // column pairs (2c, 2c + 1) go through the packed fp32 pipe: each
+            // lane of a pair gets the same fused multiply-add as the scalar form
+            float2 r[CC / 2][2];
 #pragma unroll
-            for (int c = 0; c < CC; ++c) r[c][0] = r[c][1] = 0.f;
+            for (int c = 0; c < CC / 2; ++c) r[c][0] = r[c][1] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int m = 0; m < NG; ++m) {
-                const float4 x = *reinterpret_cast<const float4 *>(&s_aa[tt][row(m, 0)]);
+                const float4 x = *reinterpret_cast<const float4 *>(&s_aa[buf][tt][row(m, 0)]);
 #pragma unroll
-                for (int c = 0; c < CC; ++c) {
-                    r[c][0] = fmaf(x.x, S[4 * m][c], r[c][0]);
-                    r[c][1] = fmaf(x.y, S[4 * m + 1][c], r[c][1]);
-                    r[c][0] = fmaf(x.z, S[4 * m + 2][c], r[c][0]);
-                    r[c][1] = fmaf(x.w, S[4 * m + 3][c], r[c][1]);
+                for (int c = 0; c < CC / 2; ++c) {
+                    r[c][0] = __ffma2_rn(make_float2(x.x, x.x), S2[4 * m][c], r[c][0]);
+                    r[c][1] = __ffma2_rn(make_float2(x.y, x.y), S2[4 * m + 1][c], r[c][1]);
+                    r[c][0] = __ffma2_rn(make_float2(x.z, x.z), S2[4 * m + 2][c], r[c][0]);
+                    r[c][1] = __ffma2_rn(make_float2(x.w, x.w), S2[4 * m + 3][c], r[c][1]);
                 }
             }
             float u[CC];
-            ld_cols<CC>(&s_m[tt][cl], u);
+            ld_cols<CC>(&s_m[buf][tt][cl], u);
 #pragma unroll
-            for (int c = 0; c < CC; ++c) u[c] -= group_sum<KS>(r[c][0] + r[c][1]);
-            float o[CC][2];
+            for (int c = 0; c < CC / 2; ++c) {
+                u[2 * c] -= group_sum<KS>(r[c][0].x + r[c][1].x);
+                u[2 * c + 1] -= group_sum<KS>(r[c][0].y + r[c][1].y);
+            }
+            float2 o[CC / 2][2];
 #pragma unroll
-            for (int c = 0; c < CC; ++c) o[c][0] = o[c][1] = 0.f;
+            for (int c = 0; c < CC / 2; ++c) o[c][0] = o[c][1] = make_float2(0.f, 0.f);
 #pragma unroll
             for (int m = 0; m < NG; ++m) {
-                const float4 av = *reinterpret_cast<const float4 *>(&s_al[tt][row(m, 0)]);
-                const float4 kv = *reinterpret_cast<const float4 *>(&s_k[tt][row(m, 0)]);
+                const float4 av = *reinterpret_cast<const float4 *>(&s_al[buf][tt][row(m, 0)]);
+                const float4 kv = *reinterpret_cast<const float4 *>(&s_k[buf][tt][row(m, 0)]);
                 const float a4[4] = {av.x, av.y, av.z, av.w}, k4[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
 #pragma unroll
-                    for (int c = 0; c < CC; ++c) S[4 * m + e][c] = fmaf(a4[e], S[4 * m + e][c], k4[e] * u[c]);
+                    for (int c = 0; c < CC / 2; ++c) {
+                        const float2 ku = __fmul2_rn(make_float2(k4[e], k4[e]), make_float2(u[2 * c], u[2 * c + 1]));
+                        S2[4 * m + e][c] = __ffma2_rn(make_float2(a4[e], a4[e]), S2[4 * m + e][c], ku);
+                    }
                 if (OUT) {
-                    const float4 qv = *reinterpret_cast<const float4 *>(&s_q[tt][row(m, 0)]);
+                    const float4 qv = *reinterpret_cast<const float4 *>(&s_q[buf][tt][row(m, 0)]);
                     const float q4[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
 #pragma unroll
-                        for (int c = 0; c < CC; ++c) o[c][e & 1] = fmaf(q4[e], S[4 * m + e][c], o[c][e & 1]);
+                        for (int c = 0; c < CC / 2; ++c)
+                            o[c][e & 1] = __ffma2_rn(make_float2(q4[e], q4[e]), S2[4 * m + e][c], o[c][e & 1]);
                 }
             }
             const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
             if (OUT) {
                 float ov[CC];
 #pragma unroll
-                for (int c = 0; c < CC; ++c) ov[c] = group_sum<KS>(o[c][0] + o[c][1]);
+                for (int c = 0; c < CC / 2; ++c) {
+                    ov[2 * c] = group_sum<KS>(o[c][0].x + o[c][1].x);
+                    ov[2 * c + 1] = group_sum<KS>(o[c][0].y + o[c][1].y);
+                }
                 if (p == 0) {
 #pragma unroll
                     for (int c = 0; c < CC; ++c) st_out((TIn *)a.o + tok * DV + j + c, ov[c]);
@@ -249,15 +266,17 @@ scan_fwd_kernel(FwdArgs a)
 #pragma unroll
                 for (int m = 0; m < NG; ++m)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) st_cols<CC>(dst + (size_t)row(m, e) * DV, S[4 * m + e]);
+                    for (int e = 0; e < 4; ++e) st_cols<CC>(dst + (size_t)row(m, e) * DV, S2[4 * m + e]);
             }
         }
+        if (more) commit(buf ^ 1, base + TB);
+        __syncthreads();   // block b consumed, block b+1 staged
     }
     if (a.sf) {
 #pragma unroll
         for (int m = 0; m < NG; ++m)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) st_cols<CC>(a.sf + soff + (size_t)row(m, e) * DV + j, S[4 * m + e]);
+            for (int e = 0; e < 4; ++e) st_cols<CC>(a.sf + soff + (size_t)row(m, e) * DV + j, S2[4 * m + e]);
     }
 }
 
