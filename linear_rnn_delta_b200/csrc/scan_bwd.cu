@@ -385,14 +385,19 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
     const size_t srow = (((size_t)n * a.H + h) * DK + i) * a.dv + (size_t)jb * DVB;
     float4 *scr = reinterpret_cast<float4 *>(g.scratch) + (size_t)blockIdx.x * (BC / CKP) * NQ * DK;
 
-    float S[DVB], G[DVB];
-    auto load_row = [&](float (&dst)[DVB], const float *src) {
+    // row i of S and G, as column pairs (2p, 2p + 1): elementwise work goes
+    // through the packed fp32 pipe, each lane with the scalar form's fused
+    // multiply-add in the scalar form's order
+    float2 S[DVB / 2], G[DVB / 2];
+    auto load_row = [&](float2 (&dst)[DVB / 2], const float *src) {
 #pragma unroll
         for (int c4 = 0; c4 < NQ; ++c4) {
             const float4 x = src ? reinterpret_cast<const float4 *>(src)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-            dst[4 * c4] = x.x; dst[4 * c4 + 1] = x.y; dst[4 * c4 + 2] = x.z; dst[4 * c4 + 3] = x.w;
+            dst[2 * c4] = make_float2(x.x, x.y);
+            dst[2 * c4 + 1] = make_float2(x.z, x.w);
         }
     };
+    auto dup = [](float x) { return make_float2(x, x); };
     auto tok_of = [&](int t) { return ((size_t)row0 + t) * a.H + h; };
     auto gate_raw = [&](size_t tok) { return vec_gate ? g1[tok * DK + i] : g1[tok]; };
     // column sums over the CTA's rows of x (destroyed); returns nothing, leaves the
@@ -465,12 +470,16 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
 #pragma unroll
                 for (int c4 = 0; c4 < NQ; ++c4)
                     scr[((size_t)(tt / CKP) * NQ + c4) * DK + i] =
-                        make_float4(S[4 * c4], S[4 * c4 + 1], S[4 * c4 + 2], S[4 * c4 + 3]);
+                        make_float4(S[2 * c4].x, S[2 * c4].y, S[2 * c4 + 1].x, S[2 * c4 + 1].y);
             }
             float x[DVB];
             const float aa = alpha_i * (e_i * k_i);   // alpha_i a~_i
 #pragma unroll
-            for (int j = 0; j < DVB; ++j) x[j] = aa * S[j];
+            for (int j2 = 0; j2 < DVB / 2; ++j2) {
+                const float2 t = __fmul2_rn(dup(aa), S[j2]);
+                x[2 * j2] = t.x;
+                x[2 * j2 + 1] = t.y;
+            }
             float *fin = column_sums(x);
             if (owner) {   // u_j = m_j - sum_i alpha_i a~_i S_ij
                 const float u = sW[tt * DVB + col] * sV[tt * DVB + col] - fin[col];
@@ -481,10 +490,8 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
 #pragma unroll
             for (int c4 = 0; c4 < NQ; ++c4) {
                 const float4 u4 = reinterpret_cast<const float4 *>(fin)[c4];
-                S[4 * c4] = fmaf(alpha_i, S[4 * c4], k_i * u4.x);
-                S[4 * c4 + 1] = fmaf(alpha_i, S[4 * c4 + 1], k_i * u4.y);
-                S[4 * c4 + 2] = fmaf(alpha_i, S[4 * c4 + 2], k_i * u4.z);
-                S[4 * c4 + 3] = fmaf(alpha_i, S[4 * c4 + 3], k_i * u4.w);
+                S[2 * c4] = __ffma2_rn(dup(alpha_i), S[2 * c4], __fmul2_rn(dup(k_i), make_float2(u4.x, u4.y)));
+                S[2 * c4 + 1] = __ffma2_rn(dup(alpha_i), S[2 * c4 + 1], __fmul2_rn(dup(k_i), make_float2(u4.z, u4.w)));
             }
         }
         __syncthreads();   // u_t of the chunk visible to every warp
@@ -536,7 +543,8 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
 #pragma unroll
                 for (int c4 = 0; c4 < NQ; ++c4) {
                     const float4 x = ckb[((size_t)buf * NQ + c4) * DK + i];
-                    S[4 * c4] = x.x; S[4 * c4 + 1] = x.y; S[4 * c4 + 2] = x.z; S[4 * c4 + 3] = x.w;
+                    S[2 * c4] = make_float2(x.x, x.y);
+                    S[2 * c4 + 1] = make_float2(x.z, x.w);
                 }
                 const float alpha_i = rsm[(r * 4 + 0) * DK + i], k_i = rsm[(r * 4 + 1) * DK + i];
                 const float q_i = rsm[(r * 4 + 2) * DK + i], e_i = rsm[(r * 4 + 3) * DK + i];
@@ -547,10 +555,10 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
 #pragma unroll
                         for (int c4 = 0; c4 < NQ; ++c4) {
                             const float4 u4 = u4p[c4];
-                            S[4 * c4] = fmaf(c_al[s], S[4 * c4], c_k[s] * u4.x);
-                            S[4 * c4 + 1] = fmaf(c_al[s], S[4 * c4 + 1], c_k[s] * u4.y);
-                            S[4 * c4 + 2] = fmaf(c_al[s], S[4 * c4 + 2], c_k[s] * u4.z);
-                            S[4 * c4 + 3] = fmaf(c_al[s], S[4 * c4 + 3], c_k[s] * u4.w);
+                            S[2 * c4] = __ffma2_rn(dup(c_al[s]), S[2 * c4],
+                                                   __fmul2_rn(dup(c_k[s]), make_float2(u4.x, u4.y)));
+                            S[2 * c4 + 1] = __ffma2_rn(dup(c_al[s]), S[2 * c4 + 1],
+                                                       __fmul2_rn(dup(c_k[s]), make_float2(u4.z, u4.w)));
                         }
                     }
                 }
@@ -559,24 +567,30 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                 const float4 *do4 = reinterpret_cast<const float4 *>(sDO + tt * DVB);
                 const float4 *u4p = reinterpret_cast<const float4 *>(sU + tt * DVB);
                 // G += q do^T;  row partials of S_t do (= alpha S_{t-1} do + k (u.do)) and G u
-                float sdo[2] = {0.f, 0.f}, udo[2] = {0.f, 0.f}, gu[2] = {0.f, 0.f};
+                // (partial sums over even and odd columns in .x and .y)
+                float2 sdo = make_float2(0.f, 0.f), udo = sdo, gu = sdo;
 #pragma unroll
                 for (int c4 = 0; c4 < NQ; ++c4) {
                     const float4 d4 = do4[c4], u4 = u4p[c4];
-                    const float dd[4] = {d4.x, d4.y, d4.z, d4.w}, uu[4] = {u4.x, u4.y, u4.z, u4.w};
+                    const float2 dd[2] = {make_float2(d4.x, d4.y), make_float2(d4.z, d4.w)};
+                    const float2 uu[2] = {make_float2(u4.x, u4.y), make_float2(u4.z, u4.w)};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 4 * c4 + e;
-                        G[j] = fmaf(q_i, dd[e], G[j]);
-                        sdo[e & 1] = fmaf(S[j], dd[e], sdo[e & 1]);
-                        udo[e & 1] = fmaf(uu[e], dd[e], udo[e & 1]);
-                        gu[e & 1] = fmaf(G[j], uu[e], gu[e & 1]);
+                    for (int e = 0; e < 2; ++e) {
+                        const int j2 = 2 * c4 + e;
+                        G[j2] = __ffma2_rn(dup(q_i), dd[e], G[j2]);
+                        sdo = __ffma2_rn(S[j2], dd[e], sdo);
+                        udo = __ffma2_rn(uu[e], dd[e], udo);
+                        gu = __ffma2_rn(G[j2], uu[e], gu);
                     }
                 }
                 // du_j = sum_i k_i G_ij
                 float x[DVB];
 #pragma unroll
-                for (int j = 0; j < DVB; ++j) x[j] = k_i * G[j];
+                for (int j2 = 0; j2 < DVB / 2; ++j2) {
+                    const float2 t = __fmul2_rn(dup(k_i), G[j2]);
+                    x[2 * j2] = t.x;
+                    x[2 * j2 + 1] = t.y;
+                }
                 float *fin = column_sums(x);
                 if (warp == 0) {   // per-column outputs: dv = w du;  GDN-2 dw = v du;  scalar gates: sum_j v_j du_j
                     float vdu = 0.f;
@@ -595,26 +609,26 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                 }
                 // dS' = G - a~ du^T;  dalpha = rowsum(S_{t-1} dS');  S_{t-1} du;  G <- Diag(alpha) dS'
                 const float at = e_i * k_i;
-                float sds[2] = {0.f, 0.f}, sdu[2] = {0.f, 0.f};
+                float2 sds = make_float2(0.f, 0.f), sdu = sds;
 #pragma unroll
                 for (int c4 = 0; c4 < NQ; ++c4) {
                     const float4 du4 = reinterpret_cast<const float4 *>(fin)[c4];
-                    const float du[4] = {du4.x, du4.y, du4.z, du4.w};
+                    const float2 du[2] = {make_float2(du4.x, du4.y), make_float2(du4.z, du4.w)};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 4 * c4 + e;
-                        G[j] = fmaf(-at, du[e], G[j]);
-                        sds[e & 1] = fmaf(S[j], G[j], sds[e & 1]);
-                        sdu[e & 1] = fmaf(S[j], du[e], sdu[e & 1]);
-                        G[j] *= alpha_i;
+                    for (int e = 0; e < 2; ++e) {
+                        const int j2 = 2 * c4 + e;
+                        G[j2] = __ffma2_rn(dup(-at), du[e], G[j2]);
+                        sds = __ffma2_rn(S[j2], G[j2], sds);
+                        sdu = __ffma2_rn(S[j2], du[e], sdu);
+                        G[j2] = __fmul2_rn(G[j2], dup(alpha_i));
                     }
                 }
                 // this CTA's parts (its value columns) of dq, dk, dalpha and k (.) da~, da~ = -Diag(alpha) S_{t-1} du
-                const float datp = -alpha_i * (sdu[0] + sdu[1]);
+                const float datp = -alpha_i * (sdu.x + sdu.y);
                 float *ring = smf + L::RING + ((size_t)((blk & 1) * RTB + pos) * 4) * DK;
-                ring[i] = fmaf(alpha_i, sdo[0] + sdo[1], k_i * (udo[0] + udo[1]));
-                ring[DK + i] = fmaf(e_i, datp, gu[0] + gu[1]);   // a~ = e (.) k: dk = G u + e da~
-                ring[2 * DK + i] = sds[0] + sds[1];
+                ring[i] = fmaf(alpha_i, sdo.x + sdo.y, k_i * (udo.x + udo.y));
+                ring[DK + i] = fmaf(e_i, datp, gu.x + gu.y);   // a~ = e (.) k: dk = G u + e da~
+                ring[2 * DK + i] = sds.x + sds.y;
                 ring[3 * DK + i] = k_i * datp;
                 if (i == 0) tokrow[(blk & 1) * RTB + pos] = t;
                 ++pos;
@@ -669,7 +683,7 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
     if (g.d_s0) {
         float4 *dst = reinterpret_cast<float4 *>(g.d_s0 + srow);
 #pragma unroll
-        for (int c4 = 0; c4 < NQ; ++c4) dst[c4] = make_float4(G[4 * c4], G[4 * c4 + 1], G[4 * c4 + 2], G[4 * c4 + 3]);
+        for (int c4 = 0; c4 < NQ; ++c4) dst[c4] = make_float4(G[2 * c4].x, G[2 * c4].y, G[2 * c4 + 1].x, G[2 * c4 + 1].y);
     }
     cl.sync();   // no CTA leaves while the cluster may still read its shared memory
 }
