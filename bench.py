@@ -105,6 +105,8 @@ def source_digest(paths) -> str:
 CHUNK_SOURCES = ["linear_rnn_delta_b200/csrc/chunk_fwd_sm100.cu", "linear_rnn_delta_b200/csrc/sm100.cuh",
                  "linear_rnn_delta_b200/csrc/common.cuh"]
 DECODE_SOURCES = ["linear_rnn_delta_b200/csrc/decode_step.cu", "linear_rnn_delta_b200/csrc/common.cuh"]
+BWD_SOURCES = ["linear_rnn_delta_b200/csrc/scan_fwd.cu", "linear_rnn_delta_b200/csrc/scan_bwd.cu",
+               "linear_rnn_delta_b200/csrc/scan_bwd.cuh", "linear_rnn_delta_b200/csrc/common.cuh"]
 
 
 def measured_traffic(name: str, sources) -> dict:
@@ -422,7 +424,8 @@ def run_backward_workload(inp, steps, warmup, world, rank):
             "value": alg["tokens"] * world * steps / total, "unit": UNIT, "ms_per_step": total / steps * 1e3,
             "p50_ms": pct(per, 50) * 1e3, "kernels_per_step": 2, "gpu_launches": 2 * steps,
             "roofline": {"bound": "alu", "achieved": tfs, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                         "frac": tfs / FP32_ALU_TFLOPS, "traffic": None,
+                         "frac": tfs / FP32_ALU_TFLOPS,
+                         "traffic": measured_traffic("backward_kda_4x16x4096", BWD_SOURCES).get("dram_bytes_per_launch"),
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz",
                          "alg_flops_per_launch": alg["flops"],
                          "kernel": "kda_chunk_bwd: checkpoint scan + cluster adjoint scan timed as one call"}}
