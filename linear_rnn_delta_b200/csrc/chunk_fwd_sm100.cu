@@ -86,8 +86,8 @@ constexpr uint32_t OFF_LA = OFF_F;            // level row factors: 128 rows x 1
 constexpr uint32_t OFF_LB = OFF_F + 32768;    // level column factors: 64 rows x 128 ch
 constexpr int TP = 68;                        // pitch (floats) of the fp32 A and T tiles: 16-byte rows
 constexpr uint32_t OFF_AF32 = OFF_F;          // A fp32 [64][TP]
-constexpr uint32_t OFF_TF32 = OFF_F + 17408;  // T fp32 [64][TP]; B operand tile of the T solve before
-constexpr uint32_t OFF_X = OFF_F + 34816;     // T_D, compact [64][16] fp32, of the T solve
+constexpr uint32_t OFF_TF32 = OFF_F + 17408;  // T fp32 [64][TP]
+constexpr uint32_t OFF_X = OFF_F + 34816;     // 32 x 32 fp32 scratch of the block solve
 constexpr uint32_t OFF_TBF = OFF_F + 38912;   // T Diag(e) / T Diag(w) bf16 64 x 64 K-major
 constexpr uint32_t OFF_PBF = OFF_F + 47104;   // P bf16 64 x 64 K-major
 constexpr uint32_t OFF_MISC = OFF_F + 55296;
@@ -99,8 +99,7 @@ constexpr uint32_t M_G1B = OFF_MISC + 6992, M_G2B = OFF_MISC + 7248;   // gates 
 constexpr uint32_t SMEM_USED = OFF_MISC + 7504;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // slack for aligning the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-static_assert((OFF_TBF & 1023) == 0 && (OFF_PBF & 1023) == 0 && (OFF_QA & 1023) == 0 && (OFF_TF32 & 1023) == 0,
-              "swizzle atoms");
+static_assert((OFF_TBF & 1023) == 0 && (OFF_PBF & 1023) == 0 && (OFF_QA & 1023) == 0, "swizzle atoms");
 
 // ---- TMEM columns ---------------------------------------------------------
 constexpr uint32_t TM_S = 0, TM_U = 128, TM_O = 192, TM_W = 256, TM_AP = 384;
@@ -502,183 +501,6 @@ __device__ __forceinline__ void scatter_level(uint8_t *pbf, float *Af, const flo
             else *reinterpret_cast<unsigned short *>(pbf + sw_elem(8192, r, s)) = bf16_bits(v[c]);
         }
     }
-}
-
-// ---- T = (I + A)^{-1} on the tensor cores --------------------------------------
-// A is strictly lower triangular (64 x 64, fp32).  Let T_D be the inverses of the
-// four 16 x 16 diagonal blocks of I + A (forward substitution, SIMT) and L the
-// rest of A (the blocks below them).  Then I + A = (I + L T_D) T_D^{-1}, and
-// R = L T_D is strictly block lower, so R^4 = 0 and
-//   T = T_D (I + R)^{-1} = T_D (I - R)(I + R^2) = V + V R^2,   V = T_D - T_D R.
-// Three rounds of tcgen05 kind::tf32 GEMMs (M = 128 with the A operand in
-// tensor memory, its lanes 64..127 unused; N = K = 64; fp32 accumulation) give
-// R; then R^2 and T_D R; then V R^2.  Operands are rounded to tf32 (nearest);
-// the sums V and V + V R^2 are formed in fp32.  tf32 carries 3 more mantissa
-// bits than the bf16 copies of T that W and U' are built from.
-//
-// Lanes 0..63 of tensor memory (rows of the 64 x 64 matrices) belong to the
-// warps of lane quarters 0 and 1: those threads ("row workers", row r, NC
-// columns from col0) move rows between tensor memory and shared memory; every
-// thread of the group writes the first B tile.  The B tile (16 KiB, 1024-byte
-// aligned, K-major 128-byte swizzled: B[n][k] = X[k][n] for the product Y X)
-// may overlay the A tile (read before the first barrier) and the T tile (written
-// after the last round).
-struct TcSolve {
-    const float *At;   // A fp32 [64][TP] (rows read in phase 1)
-    float *Tt;         // T fp32 [64][TP] (written in phase 4)
-    const float *Xd;   // T_D, compact [64][16]: row r holds T_D[r][16 (r/16) + c]
-    uint8_t *bt;       // B operand tile
-    uint32_t bt_s;     // its shared-memory address
-    uint32_t tbase;    // tensor memory base
-    uint32_t reg[4];   // four free 64-column regions of tensor memory
-    uint64_t *bar;     // commit barrier of the rounds
-};
-
-template <int NC>
-__device__ __forceinline__ void tm_store_cols(uint32_t taddr, const float *v)
-{
-#pragma unroll
-    for (int c16 = 0; c16 < NC / 16; ++c16) tmem_st16(taddr + c16 * 16, v + c16 * 16);
-}
-template <int NC>
-__device__ __forceinline__ void tm_load_cols(uint32_t taddr, float *v)
-{
-#pragma unroll
-    for (int c32 = 0; c32 < NC / 32; ++c32) tmem_ld32(taddr + c32 * 32, v + c32 * 32);
-    tmem_wait_ld();
-}
-
-// Row r of T_D from the compact layout: its 16 entries in the diagonal block.
-// Column col0 + c (col0 a multiple of 16) of the row is td[c & 15] when it falls
-// in row r's block, else 0.
-__device__ __forceinline__ void td_row(const float *Xd, int r, float (&td)[16])
-{
-#pragma unroll
-    for (int i = 0; i < 4; ++i) *reinterpret_cast<float4 *>(td + 4 * i) = *reinterpret_cast<const float4 *>(Xd + r * 16 + 4 * i);
-}
-__device__ __forceinline__ float td_col(const float (&td)[16], int r, int col0, int c)
-{
-    return ((col0 + c) >> 4) == (r >> 4) ? td[c & 15] : 0.f;
-}
-
-// NC: columns per row worker (64, or 32 when two warps share a lane quarter).
-// `sync` is the group's barrier; `wait_mma` waits for the last commit (and
-// fences); the group's thread 0 issues the MMAs.
-template <int NC, class Sync, class Wait>
-__device__ __forceinline__ void tc_tsolve(const TcSolve &s, int gtid, int gthreads, bool row_worker, int r,
-                                          int col0, uint32_t lane_field, Sync sync, Wait wait_mma)
-{
-    constexpr uint32_t ID = idesc_tf32(128, 64);
-    const uint32_t tl = s.tbase + lane_field;
-    float v[NC];
-    // ---- phase 1: A operands L (reg 0) and T_D (reg 1); then B = T_D^T
-    if (row_worker) {
-        const int b0 = r & ~15;
-#pragma unroll
-        for (int c4 = 0; c4 < NC / 4; ++c4) {
-            const float4 a4 = *reinterpret_cast<const float4 *>(s.At + r * TP + col0 + 4 * c4);
-            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[4 * c4 + i] = (col0 + 4 * c4 + i < b0) ? rna_tf32(av[i]) : 0.f;
-        }
-        tm_store_cols<NC>(tl + s.reg[0] + col0, v);
-        float td[16];
-        td_row(s.Xd, r, td);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) v[c] = rna_tf32(td_col(td, r, col0, c));
-        tm_store_cols<NC>(tl + s.reg[1] + col0, v);
-        tmem_wait_st();
-    }
-    sync();   // the A tile has been read: the B tile may overlay it
-    for (int e = gtid; e < 1024; e += gthreads) {
-        const int n = e >> 4, kc = e & 15;
-        float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-        if ((kc >> 2) == (n >> 4)) {
-            const float *x = s.Xd + (4 * kc) * 16 + (n & 15);
-            w = make_float4(rna_tf32(x[0]), rna_tf32(x[16]), rna_tf32(x[32]), rna_tf32(x[48]));
-        }
-        *reinterpret_cast<float4 *>(s.bt + sw_chunk(8192, n, kc)) = w;
-    }
-    fence_async_smem();
-    tc_fence_before();
-    sync();
-    if (gtid == 0) {   // R = L T_D -> reg 2
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ta(s.tbase + s.reg[2], s.tbase + s.reg[0] + kk * 8, dK(s.bt_s, 8192, kk), ID, kk > 0);
-        mma_commit(s.bar);
-    }
-    wait_mma();
-    // ---- phase 2: R rounded in place (A operand), B = R^T
-    if (row_worker) {
-        tm_load_cols<NC>(tl + s.reg[2] + col0, v);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            v[c] = rna_tf32(v[c]);
-            *reinterpret_cast<float *>(s.bt + sw_chunk(8192, col0 + c, r >> 2) + (r & 3) * 4) = v[c];
-        }
-        tm_store_cols<NC>(tl + s.reg[2] + col0, v);
-        tmem_wait_st();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    sync();
-    if (gtid == 0) {   // R^2 -> reg 0;  T_D R -> reg 3
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ta(s.tbase + s.reg[0], s.tbase + s.reg[2] + kk * 8, dK(s.bt_s, 8192, kk), ID, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ta(s.tbase + s.reg[3], s.tbase + s.reg[1] + kk * 8, dK(s.bt_s, 8192, kk), ID, kk > 0);
-        mma_commit(s.bar);
-    }
-    wait_mma();
-    // ---- phase 3: V = T_D - T_D R rounded (A operand, reg 1), B = (R^2)^T
-    if (row_worker) {
-        float td[16];
-        td_row(s.Xd, r, td);
-        tm_load_cols<NC>(tl + s.reg[3] + col0, v);
-#pragma unroll
-        for (int c = 0; c < NC; ++c) v[c] = rna_tf32(td_col(td, r, col0, c) - v[c]);
-        tm_store_cols<NC>(tl + s.reg[1] + col0, v);
-        tm_load_cols<NC>(tl + s.reg[0] + col0, v);
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-            *reinterpret_cast<float *>(s.bt + sw_chunk(8192, col0 + c, r >> 2) + (r & 3) * 4) = rna_tf32(v[c]);
-        tmem_wait_st();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    sync();
-    if (gtid == 0) {   // V R^2 -> reg 2
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-            mma_tf32_ta(s.tbase + s.reg[2], s.tbase + s.reg[1] + kk * 8, dK(s.bt_s, 8192, kk), ID, kk > 0);
-        mma_commit(s.bar);
-    }
-    wait_mma();
-    // ---- phase 4: T = V + V R^2 (V recomputed in fp32 as in phase 3) -> T tile
-    if (row_worker) {
-        float w[NC], td[16];
-        td_row(s.Xd, r, td);
-        tm_load_cols<NC>(tl + s.reg[3] + col0, v);
-        tm_load_cols<NC>(tl + s.reg[2] + col0, w);
-#pragma unroll
-        for (int c4 = 0; c4 < NC / 4; ++c4) {
-            float t4[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = 4 * c4 + i;
-                t4[i] = (td_col(td, r, col0, c) - v[c]) + w[c];
-            }
-            *reinterpret_cast<float4 *>(s.Tt + r * TP + col0 + 4 * c4) = make_float4(t4[0], t4[1], t4[2], t4[3]);
-        }
-    }
-    tc_fence_before();
-    sync();
 }
 
 // ---- exact path for ill-conditioned chunks ------------------------------------
@@ -1469,9 +1291,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
             group_sync(BAR_PREP, NPREP);
 
             // ===== 3. T = (I + A)^{-1} =============================================
-            // 16x16 diagonal blocks by forward substitution (one column per thread, fp32,
-            // A rows read four at a time) into the compact T_D tile; the rest on the tensor
-            // cores (tc_tsolve: T into the T tile, which serves as the B operand meanwhile).
+            // 16x16 diagonal blocks by forward substitution (one column per thread), then
+            // recursive doubling: T[16(I+1):, 16I:] = -D_{I+1} A_{I+1,I} D_I for I = 0, 2, and
+            // T[32:, :32] = -T2 A21 T1.  fp32 throughout; A rows read four at a time.
             if (ptid < 64) {
                 const int I = ptid >> 4, c = ptid & 15;
                 float xv[16];
@@ -1491,16 +1313,92 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                     xv[r2] = (r2 < c) ? 0.f : ((r2 == c) ? 1.f : -(acc0 + acc1));
                 }
 #pragma unroll
-                for (int r2 = 0; r2 < 16; ++r2) Xs[(16 * I + r2) * 16 + c] = xv[r2];
+                for (int r2 = 0; r2 < 16; ++r2) Tf[(16 * I + r2) * TP + 16 * I + c] = xv[r2];
+                for (int r2 = 0; r2 < 16 * I; ++r2) Tf[r2 * TP + 16 * I + c] = 0.f;  // above the block
             } else if (ptid < 64 + C) {   // meanwhile: the next item's gates
                 if (nxt.valid) fetch_gates(nxt, ptid - 64, par ^ 1u);
             }
             group_sync(BAR_PREP, NPREP);
-            {
-                const TcSolve ts{Af, Tf, Xs, sm + OFF_TF32, sb + OFF_TF32, tbase, {256u, 320u, 384u, 448u}, bar_pmma};
-                tc_tsolve<32>(ts, ptid, NPREP, quarter < 2, jrow, phalf * 32, lane_base,
-                              [&]() { group_sync(BAR_PREP, NPREP); }, wait_pmma);
+            {   // X = A_{I+1,I} D_I for I = 0, 2 (two outputs per thread)
+                const int r2 = (ptid >> 4) & 15, c2 = ptid & 15;
+                float acc[2] = {0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 av = *reinterpret_cast<const float4 *>(Af + (16 * I + 16 + r2) * TP + 16 * I + 4 * m4);
+                        const float *tcol = Tf + (16 * I + 4 * m4) * TP + 16 * I + c2;
+                        acc[blk] = fmaf(av.x, tcol[0], acc[blk]);
+                        acc[blk] = fmaf(av.y, tcol[TP], acc[blk]);
+                        acc[blk] = fmaf(av.z, tcol[2 * TP], acc[blk]);
+                        acc[blk] = fmaf(av.w, tcol[3 * TP], acc[blk]);
+                    }
+                }
+                Xs[ptid] = acc[0];
+                Xs[256 + ptid] = acc[1];
             }
+            group_sync(BAR_PREP, NPREP);
+            {   // T_{I+1,I} = -D_{I+1} X
+                const int r2 = (ptid >> 4) & 15, c2 = ptid & 15;
+                float acc[2] = {0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 tv = *reinterpret_cast<const float4 *>(Tf + (16 * I + 16 + r2) * TP + 16 * I + 16 + 4 * m4);
+                        const float *xcol = Xs + (blk << 8) + (4 * m4) * 16 + c2;
+                        acc[blk] = fmaf(tv.x, xcol[0], acc[blk]);
+                        acc[blk] = fmaf(tv.y, xcol[16], acc[blk]);
+                        acc[blk] = fmaf(tv.z, xcol[32], acc[blk]);
+                        acc[blk] = fmaf(tv.w, xcol[48], acc[blk]);
+                    }
+                }
+                Tf[(16 + r2) * TP + c2] = -acc[0];
+                Tf[(48 + r2) * TP + 32 + c2] = -acc[1];
+            }
+            group_sync(BAR_PREP, NPREP);
+            {   // X = A21 T1 (rows r0 + 8k, column c2)
+                const int r0 = ptid >> 5, c2 = ptid & 31;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *tcol = Tf + (4 * m4) * TP + c2;
+                    const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + r0 + 8 * k4) * TP + 4 * m4);
+                        acc[k4] = fmaf(av.x, t0v, acc[k4]);
+                        acc[k4] = fmaf(av.y, t1v, acc[k4]);
+                        acc[k4] = fmaf(av.z, t2v, acc[k4]);
+                        acc[k4] = fmaf(av.w, t3v, acc[k4]);
+                    }
+                }
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) Xs[(r0 + 8 * k4) * 32 + c2] = acc[k4];
+            }
+            group_sync(BAR_PREP, NPREP);
+            {   // T21 = -T2 X
+                const int r0 = ptid >> 5, c2 = ptid & 31;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *xcol = Xs + (4 * m4) * 32 + c2;
+                    const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const float4 tv = *reinterpret_cast<const float4 *>(Tf + (32 + r0 + 8 * k4) * TP + 32 + 4 * m4);
+                        acc[k4] = fmaf(tv.x, x0, acc[k4]);
+                        acc[k4] = fmaf(tv.y, x1, acc[k4]);
+                        acc[k4] = fmaf(tv.z, x2, acc[k4]);
+                        acc[k4] = fmaf(tv.w, x3, acc[k4]);
+                    }
+                }
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) Tf[(32 + r0 + 8 * k4) * TP + c2] = -acc[k4];
+            }
+            group_sync(BAR_PREP, NPREP);
 
             // ===== 4. W = T Diag(e) (row operand a~ part);  U'^T = M^T (T Diag(w))^T ==
             // T copies go through one bf16 tile: T Diag(e) for W, then (RDA only, whose two
@@ -1649,8 +1547,8 @@ constexpr uint32_t P2_QA = 65536;     // [a~'; Q'] 128-row K-major tile (A/P GEM
 constexpr uint32_t P2_AT = 98304;     // back: the a~' rows (2 panels x 64 rows), then -W'
 constexpr uint32_t P2_FR = 114688;    // front: band partials | level factors; then A fp32 and P bf16
 constexpr uint32_t P2_LA = P2_FR, P2_LB = P2_FR + 32768, P2_AF = P2_FR, P2_PBF = P2_FR + 17408;
-constexpr uint32_t P2_TB = 163840;    // back: A, the B operand of the T solve, then T, fp32 [64][TP]
-constexpr uint32_t P2_TBF = 181248;   // back: compact T_D [64][16] fp32 of the T solve, then T Diag(.) bf16
+constexpr uint32_t P2_TB = 163840;    // back: A, then T in place, fp32 [64][TP]
+constexpr uint32_t P2_TBF = 181248;   // back: the 32 x 32 scratch of the T solve, then T Diag(.) bf16
 constexpr uint32_t P2_X = P2_TBF;
 constexpr uint32_t P2_MT = 189440;    // front, GDN-2: v, then M = w (.) v in place
 constexpr uint32_t P2_MISC = 205824;
@@ -1668,7 +1566,7 @@ constexpr uint32_t P2_ALLOC = P2_MISC + 10352 + 1024;
 static_assert(P2_ALLOC <= 232448, "shared memory budget");
 static_assert(P2_FR + 40960 <= P2_TB && P2_LB + 16384 <= P2_TB && P2_PBF + 8192 <= P2_TB, "front region");
 static_assert(P2_TB + 64 * TP * 4 <= P2_TBF && P2_TBF + 8192 <= P2_MT && P2_MT + 16384 <= P2_MISC, "back region");
-static_assert(((P2_QA | P2_KB | P2_AT | P2_PBF | P2_TBF | P2_MT | P2_TB) & 1023) == 0, "swizzle atoms");
+static_assert(((P2_QA | P2_KB | P2_AT | P2_PBF | P2_TBF | P2_MT) & 1023) == 0, "swizzle atoms");
 static_assert(RAW_Q + 16384 <= RAW_K && RAW_K + 16384 <= P2_KB && P2_KB + 16384 <= RAW_A &&
               RAW_A + 16384 <= P2_QA && P2_QA + 32768 <= P2_AT && P2_AT + 16384 <= P2_FR, "tile map");
 static_assert((P2_META & 15) == 0 && (P2_BAR & 7) == 0, "alignment");
@@ -2336,44 +2234,127 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                 }
             }
 
-            // ===== 3. T = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution into the
-            // compact T_D tile, the rest on the tensor cores (tc_tsolve, T into TB, which holds A
-            // before and the B operand meanwhile)
-            if (btid < 64) {
+            // ===== 3. T = (I + A)^{-1}, in place: 16x16 diagonal blocks, then recursive doubling
+            {
                 float xv[16];
                 const int I = btid >> 4, c = btid & 15;
+                if (btid < 64) {
 #pragma unroll
-                for (int r2 = 0; r2 < 16; ++r2) {
-                    float arow[16];
+                    for (int r2 = 0; r2 < 16; ++r2) {
+                        float arow[16];
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<float4 *>(arow + 4 * q4) =
-                            *reinterpret_cast<const float4 *>(TB + (16 * I + r2) * TP + 16 * I + 4 * q4);
-                    float acc0 = 0.f, acc1 = 0.f;
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            *reinterpret_cast<float4 *>(arow + 4 * q4) =
+                                *reinterpret_cast<const float4 *>(TB + (16 * I + r2) * TP + 16 * I + 4 * q4);
+                        float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                    for (int s2 = 0; s2 < r2; ++s2) {
-                        if (s2 & 1) acc1 = fmaf(arow[s2], xv[s2], acc1);
-                        else acc0 = fmaf(arow[s2], xv[s2], acc0);
+                        for (int s2 = 0; s2 < r2; ++s2) {
+                            if (s2 & 1) acc1 = fmaf(arow[s2], xv[s2], acc1);
+                            else acc0 = fmaf(arow[s2], xv[s2], acc0);
+                        }
+                        xv[r2] = (r2 < c) ? 0.f : ((r2 == c) ? 1.f : -(acc0 + acc1));
                     }
-                    xv[r2] = (r2 < c) ? 0.f : ((r2 == c) ? 1.f : -(acc0 + acc1));
+                } else if (decoder) {   // meanwhile: the item four ahead
+                    ring_put(s_ring, j + 4, next_item_walk(a, N, nwork, wdec, ndec));
+                    wdec += gridDim.x;
                 }
+                group_sync(BAR_BACK, PF_BACK);   // every read of the diagonal blocks of A is done
+                if (btid < 64) {
 #pragma unroll
-                for (int r2 = 0; r2 < 16; ++r2) Xs[(16 * I + r2) * 16 + c] = xv[r2];
-            } else if (decoder) {   // meanwhile: the item four ahead
-                ring_put(s_ring, j + 4, next_item_walk(a, N, nwork, wdec, ndec));
-                wdec += gridDim.x;
+                    for (int r2 = 0; r2 < 16; ++r2) TB[(16 * I + r2) * TP + 16 * I + c] = xv[r2];
+                }
             }
             group_sync(BAR_BACK, PF_BACK);
-            {
-                const TcSolve ts{TB, TB, Xs, sm + P2_TB, sb + P2_TB, tbase, {0u, 64u, 192u, 256u}, bar_wmma};
-                tc_tsolve<64>(ts, btid, PF_BACK, bw < 2, quarter * 32 + lane, 0, lane_base,
-                              [&]() { group_sync(BAR_BACK, PF_BACK); },
-                              [&]() {
-                                  if (!mbar_wait_cycles(bar_wmma, ph_wmma, WAIT_CYCLES)) ok = false;
-                                  ph_wmma ^= 1;
-                                  tc_fence_after();
-                              });
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {   // X = A_{I+1,I} D_I for I = 0, 2
+                const int pt = btid + PF_BACK * pp;
+                const int r2 = (pt >> 4) & 15, c2 = pt & 15;
+                float acc[2] = {0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 av = *reinterpret_cast<const float4 *>(TB + (16 * I + 16 + r2) * TP + 16 * I + 4 * m4);
+                        const float *tcol = TB + (16 * I + 4 * m4) * TP + 16 * I + c2;
+                        acc[blk] = fmaf(av.x, tcol[0], acc[blk]);
+                        acc[blk] = fmaf(av.y, tcol[TP], acc[blk]);
+                        acc[blk] = fmaf(av.z, tcol[2 * TP], acc[blk]);
+                        acc[blk] = fmaf(av.w, tcol[3 * TP], acc[blk]);
+                    }
+                }
+                Xs[pt] = acc[0];
+                Xs[256 + pt] = acc[1];
             }
+            group_sync(BAR_BACK, PF_BACK);
+#pragma unroll 1
+            for (int pp = 0; pp < 2; ++pp) {   // T_{I+1,I} = -D_{I+1} X, over A_{I+1,I}
+                const int pt = btid + PF_BACK * pp;
+                const int r2 = (pt >> 4) & 15, c2 = pt & 15;
+                float acc[2] = {0.f, 0.f};
+#pragma unroll
+                for (int m4 = 0; m4 < 4; ++m4) {
+#pragma unroll
+                    for (int blk = 0; blk < 2; ++blk) {
+                        const int I = 2 * blk;
+                        const float4 tv = *reinterpret_cast<const float4 *>(TB + (16 * I + 16 + r2) * TP + 16 * I + 16 + 4 * m4);
+                        const float *xcol = Xs + (blk << 8) + (4 * m4) * 16 + c2;
+                        acc[blk] = fmaf(tv.x, xcol[0], acc[blk]);
+                        acc[blk] = fmaf(tv.y, xcol[16], acc[blk]);
+                        acc[blk] = fmaf(tv.z, xcol[32], acc[blk]);
+                        acc[blk] = fmaf(tv.w, xcol[48], acc[blk]);
+                    }
+                }
+                TB[(16 + r2) * TP + c2] = -acc[0];
+                TB[(48 + r2) * TP + 32 + c2] = -acc[1];
+            }
+            group_sync(BAR_BACK, PF_BACK);
+            {   // X = A21 T1: warp bw takes rows bw + 4i (i < 8), lane c2 column c2; a column of T1
+                // serves the warp's eight rows (each output summed in the fused kernel's order)
+                const int c2 = lane;
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *tcol = TB + (4 * m4) * TP + c2;
+                    const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 av = *reinterpret_cast<const float4 *>(TB + (32 + bw + 4 * i) * TP + 4 * m4);
+                        acc[i] = fmaf(av.x, t0v, acc[i]);
+                        acc[i] = fmaf(av.y, t1v, acc[i]);
+                        acc[i] = fmaf(av.z, t2v, acc[i]);
+                        acc[i] = fmaf(av.w, t3v, acc[i]);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) Xs[(bw + 4 * i) * 32 + c2] = acc[i];
+            }
+            group_sync(BAR_BACK, PF_BACK);
+            {   // T21 = -T2 X, over A21 (read by the previous phase); same row split
+                const int c2 = lane;
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+                for (int m4 = 0; m4 < 8; ++m4) {
+                    const float *xcol = Xs + (4 * m4) * 32 + c2;
+                    const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 tv =
+                            *reinterpret_cast<const float4 *>(TB + (32 + bw + 4 * i) * TP + 32 + 4 * m4);
+                        acc[i] = fmaf(tv.x, x0, acc[i]);
+                        acc[i] = fmaf(tv.y, x1, acc[i]);
+                        acc[i] = fmaf(tv.z, x2, acc[i]);
+                        acc[i] = fmaf(tv.w, x3, acc[i]);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) TB[(32 + bw + 4 * i) * TP + c2] = -acc[i];
+            }
+            group_sync(BAR_BACK, PF_BACK);
 
             // ===== 4. T Diag(e) -> W = T Diag(e) a~'; the exact-path decision; T Diag(w) for the slot
             const bool exact = !publish_and(write_t_copy(s_bg1, s_bg1, s_bg2) && well_a);
