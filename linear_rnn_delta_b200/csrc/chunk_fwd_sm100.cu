@@ -1559,8 +1559,8 @@ constexpr uint32_t P2_GAMC = P2_MISC + 7424;         // float [2][128]: Gamma_C 
 constexpr uint32_t P2_META = P2_MISC + 8448;         // back: Gamma_C fp32 [128], status word, epoch tag
 constexpr uint32_t P2_RING = P2_MISC + 8992;         // int [8][8]: decoded items
 constexpr uint32_t P2_FLAGS = P2_MISC + 9248;        // int [2] path flags by item parity, [1] abort
-constexpr uint32_t P2_BAR = P2_MISC + 9264;          // mbarriers: tma, v, pmma, wmma, full, taken
-constexpr uint32_t P2_TMEM = P2_MISC + 9312;
+constexpr uint32_t P2_BAR = P2_MISC + 9264;          // mbarriers: tma (alpha), v, pmma, wmma, full, taken, qk
+constexpr uint32_t P2_TMEM = P2_MISC + 9320;
 constexpr uint32_t P2_APART = P2_MISC + 9328;        // float [2][2][64]: |A| half-row sums by item parity
 constexpr uint32_t P2_ALLOC = P2_MISC + 10352 + 1024;
 static_assert(P2_ALLOC <= 232448, "shared memory budget");
@@ -1627,7 +1627,7 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
     int *s_flags = reinterpret_cast<int *>(sm + P2_FLAGS);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + P2_BAR);
     uint64_t *bar_tma = bars + 0, *bar_v = bars + 1, *bar_pmma = bars + 2, *bar_wmma = bars + 3;
-    uint64_t *bar_full = bars + 4, *bar_taken = bars + 5;
+    uint64_t *bar_full = bars + 4, *bar_taken = bars + 5, *bar_qk = bars + 6;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P2_TMEM);
     const __nv_bfloat16 *g1p = (const __nv_bfloat16 *)a.g1, *g2p = (const __nv_bfloat16 *)a.g2;
     const bool gdn2 = a.variant == GDN2;
@@ -1640,7 +1640,7 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
 
     if (warp == 0) tmem_alloc(s_tmem, 512);
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
         s_flags[2] = 0;   // abort
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -1665,15 +1665,22 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
         const int phalf = pw >> 2;
         const int jrow = quarter * 32 + lane;
         const int tg = ptid >> 5, cq = ptid & 31;
-        uint32_t ph_tma = 0, ph_v = 0, ph_pmma = 0, ph_taken = 0;
+        uint32_t ph_tma = 0, ph_qk = 0, ph_v = 0, ph_pmma = 0, ph_taken = 0;
         float *Af = reinterpret_cast<float *>(sm + P2_AF);
         float *s_apart = reinterpret_cast<float *>(sm + P2_APART);
+        // alpha first, on its own barrier: steps 0-1a need alpha only (and k, when keys are
+        // normalised in place), so q and k may still be in flight while they run
         auto issue_tma = [&](const Item &it) {
             const int g = it.row0 + it.c * C;
-            mbar_expect_tx(bar_tma, 3 * 16384);
-            tma_load_3d(sm + P2_RAW_Q, &P.tq, bar_tma, 0, it.h, g);
-            tma_load_3d(sm + P2_RAW_K, &P.tk, bar_tma, 0, it.h, g);
+            mbar_expect_tx(bar_tma, 16384);
             tma_load_3d(sm + P2_RAW_A, &P.ta, bar_tma, 0, it.h, g);
+            mbar_expect_tx(bar_qk, 2 * 16384);
+            tma_load_3d(sm + P2_RAW_Q, &P.tq, bar_qk, 0, it.h, g);
+            tma_load_3d(sm + P2_RAW_K, &P.tk, bar_qk, 0, it.h, g);
+        };
+        auto wait_qk = [&]() {
+            if (!mbar_wait_cycles(bar_qk, ph_qk, WAIT_CYCLES)) ok = false;
+            ph_qk ^= 1;
         };
         auto issue_tma_v = [&](const Item &it) {   // GDN-2: v into the M tile
             const int g = it.row0 + it.c * C;
@@ -1755,6 +1762,7 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
 
             if (!mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES)) ok = false;
             ph_tma ^= 1;
+            if (PREP && l2k) wait_qk();   // pass 0 rewrites k
             if (gdn2) {
                 if (!mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES)) ok = false;
                 ph_v ^= 1;
@@ -1880,6 +1888,7 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                 if (!mbar_wait_cycles(bar_taken, ph_taken, WAIT_CYCLES)) ok = false;
                 ph_taken ^= 1;
             }
+            if (!(PREP && l2k)) wait_qk();   // q and k, read from here on
 
             // ===== 1b. row operands, Kbar and the exact band of P
             if (fast) {
@@ -2129,6 +2138,7 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
         }
         if (!ok) {   // drain TMA still in flight (bounded)
             mbar_wait_cycles(bar_tma, ph_tma, WAIT_CYCLES);
+            mbar_wait_cycles(bar_qk, ph_qk, WAIT_CYCLES);
             if (gdn2) mbar_wait_cycles(bar_v, ph_v, WAIT_CYCLES);
         }
         if (lane == 0) bulk_wait_all();
@@ -2265,11 +2275,12 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                 }
             }
             group_sync(BAR_BACK, PF_BACK);
-#pragma unroll 1
-            for (int pp = 0; pp < 2; ++pp) {   // X = A_{I+1,I} D_I for I = 0, 2
-                const int pt = btid + PF_BACK * pp;
-                const int r2 = (pt >> 4) & 15, c2 = pt & 15;
-                float acc[2] = {0.f, 0.f};
+            // The merges give every output the fused kernel's multiply-add chain (same terms,
+            // same order); a thread owns two adjacent columns and runs both chains at once on
+            // the packed fp32 pipe.
+            {   // X = A_{I+1,I} D_I for I = 0, 2: thread (row r2, columns c2, c2 + 1) of both blocks
+                const int r2 = btid >> 3, c2 = (btid & 7) * 2;
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
 #pragma unroll
@@ -2277,21 +2288,19 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                         const int I = 2 * blk;
                         const float4 av = *reinterpret_cast<const float4 *>(TB + (16 * I + 16 + r2) * TP + 16 * I + 4 * m4);
                         const float *tcol = TB + (16 * I + 4 * m4) * TP + 16 * I + c2;
-                        acc[blk] = fmaf(av.x, tcol[0], acc[blk]);
-                        acc[blk] = fmaf(av.y, tcol[TP], acc[blk]);
-                        acc[blk] = fmaf(av.z, tcol[2 * TP], acc[blk]);
-                        acc[blk] = fmaf(av.w, tcol[3 * TP], acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(av.x, av.x), *reinterpret_cast<const float2 *>(tcol), acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(av.y, av.y), *reinterpret_cast<const float2 *>(tcol + TP), acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(av.z, av.z), *reinterpret_cast<const float2 *>(tcol + 2 * TP), acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(av.w, av.w), *reinterpret_cast<const float2 *>(tcol + 3 * TP), acc[blk]);
                     }
                 }
-                Xs[pt] = acc[0];
-                Xs[256 + pt] = acc[1];
+                *reinterpret_cast<float2 *>(Xs + r2 * 16 + c2) = acc[0];
+                *reinterpret_cast<float2 *>(Xs + 256 + r2 * 16 + c2) = acc[1];
             }
             group_sync(BAR_BACK, PF_BACK);
-#pragma unroll 1
-            for (int pp = 0; pp < 2; ++pp) {   // T_{I+1,I} = -D_{I+1} X, over A_{I+1,I}
-                const int pt = btid + PF_BACK * pp;
-                const int r2 = (pt >> 4) & 15, c2 = pt & 15;
-                float acc[2] = {0.f, 0.f};
+            {   // T_{I+1,I} = -D_{I+1} X, over A_{I+1,I}
+                const int r2 = btid >> 3, c2 = (btid & 7) * 2;
+                float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
 #pragma unroll
@@ -2299,60 +2308,68 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                         const int I = 2 * blk;
                         const float4 tv = *reinterpret_cast<const float4 *>(TB + (16 * I + 16 + r2) * TP + 16 * I + 16 + 4 * m4);
                         const float *xcol = Xs + (blk << 8) + (4 * m4) * 16 + c2;
-                        acc[blk] = fmaf(tv.x, xcol[0], acc[blk]);
-                        acc[blk] = fmaf(tv.y, xcol[16], acc[blk]);
-                        acc[blk] = fmaf(tv.z, xcol[32], acc[blk]);
-                        acc[blk] = fmaf(tv.w, xcol[48], acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(tv.x, tv.x), *reinterpret_cast<const float2 *>(xcol), acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(tv.y, tv.y), *reinterpret_cast<const float2 *>(xcol + 16), acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(tv.z, tv.z), *reinterpret_cast<const float2 *>(xcol + 32), acc[blk]);
+                        acc[blk] = __ffma2_rn(make_float2(tv.w, tv.w), *reinterpret_cast<const float2 *>(xcol + 48), acc[blk]);
                     }
                 }
-                TB[(16 + r2) * TP + c2] = -acc[0];
-                TB[(48 + r2) * TP + 32 + c2] = -acc[1];
+                *reinterpret_cast<float2 *>(TB + (16 + r2) * TP + c2) = make_float2(-acc[0].x, -acc[0].y);
+                *reinterpret_cast<float2 *>(TB + (48 + r2) * TP + 32 + c2) = make_float2(-acc[1].x, -acc[1].y);
             }
             group_sync(BAR_BACK, PF_BACK);
-            {   // X = A21 T1: warp bw takes rows bw + 4i (i < 8), lane c2 column c2; a column of T1
-                // serves the warp's eight rows (each output summed in the fused kernel's order)
-                const int c2 = lane;
-                float acc[8];
+            // level 32: warp bw takes rows bw + 4i, half-warp h the i in [4h, 4h + 4), lane pair
+            // columns c2, c2 + 1; a column pair of T1 (or X) serves the thread's four rows
+            const int hh = lane >> 4, cp = (lane & 15) * 2;
+            {   // X = A21 T1
+                float2 acc[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+                for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int m4 = 0; m4 < 8; ++m4) {
-                    const float *tcol = TB + (4 * m4) * TP + c2;
-                    const float t0v = tcol[0], t1v = tcol[TP], t2v = tcol[2 * TP], t3v = tcol[3 * TP];
+                    const float *tcol = TB + (4 * m4) * TP + cp;
+                    const float2 t0 = *reinterpret_cast<const float2 *>(tcol);
+                    const float2 t1 = *reinterpret_cast<const float2 *>(tcol + TP);
+                    const float2 t2 = *reinterpret_cast<const float2 *>(tcol + 2 * TP);
+                    const float2 t3 = *reinterpret_cast<const float2 *>(tcol + 3 * TP);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 av = *reinterpret_cast<const float4 *>(TB + (32 + bw + 4 * i) * TP + 4 * m4);
-                        acc[i] = fmaf(av.x, t0v, acc[i]);
-                        acc[i] = fmaf(av.y, t1v, acc[i]);
-                        acc[i] = fmaf(av.z, t2v, acc[i]);
-                        acc[i] = fmaf(av.w, t3v, acc[i]);
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = bw + 4 * (4 * hh + i);
+                        const float4 av = *reinterpret_cast<const float4 *>(TB + (32 + row) * TP + 4 * m4);
+                        acc[i] = __ffma2_rn(make_float2(av.x, av.x), t0, acc[i]);
+                        acc[i] = __ffma2_rn(make_float2(av.y, av.y), t1, acc[i]);
+                        acc[i] = __ffma2_rn(make_float2(av.z, av.z), t2, acc[i]);
+                        acc[i] = __ffma2_rn(make_float2(av.w, av.w), t3, acc[i]);
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) Xs[(bw + 4 * i) * 32 + c2] = acc[i];
+                for (int i = 0; i < 4; ++i) *reinterpret_cast<float2 *>(Xs + (bw + 4 * (4 * hh + i)) * 32 + cp) = acc[i];
             }
             group_sync(BAR_BACK, PF_BACK);
-            {   // T21 = -T2 X, over A21 (read by the previous phase); same row split
-                const int c2 = lane;
-                float acc[8];
+            {   // T21 = -T2 X, over A21 (read by the previous phase); same split
+                float2 acc[4];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+                for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int m4 = 0; m4 < 8; ++m4) {
-                    const float *xcol = Xs + (4 * m4) * 32 + c2;
-                    const float x0 = xcol[0], x1 = xcol[32], x2 = xcol[64], x3 = xcol[96];
+                    const float *xcol = Xs + (4 * m4) * 32 + cp;
+                    const float2 x0 = *reinterpret_cast<const float2 *>(xcol);
+                    const float2 x1 = *reinterpret_cast<const float2 *>(xcol + 32);
+                    const float2 x2 = *reinterpret_cast<const float2 *>(xcol + 64);
+                    const float2 x3 = *reinterpret_cast<const float2 *>(xcol + 96);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 tv =
-                            *reinterpret_cast<const float4 *>(TB + (32 + bw + 4 * i) * TP + 32 + 4 * m4);
-                        acc[i] = fmaf(tv.x, x0, acc[i]);
-                        acc[i] = fmaf(tv.y, x1, acc[i]);
-                        acc[i] = fmaf(tv.z, x2, acc[i]);
-                        acc[i] = fmaf(tv.w, x3, acc[i]);
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = bw + 4 * (4 * hh + i);
+                        const float4 tv = *reinterpret_cast<const float4 *>(TB + (32 + row) * TP + 32 + 4 * m4);
+                        acc[i] = __ffma2_rn(make_float2(tv.x, tv.x), x0, acc[i]);
+                        acc[i] = __ffma2_rn(make_float2(tv.y, tv.y), x1, acc[i]);
+                        acc[i] = __ffma2_rn(make_float2(tv.z, tv.z), x2, acc[i]);
+                        acc[i] = __ffma2_rn(make_float2(tv.w, tv.w), x3, acc[i]);
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) TB[(32 + bw + 4 * i) * TP + c2] = -acc[i];
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<float2 *>(TB + (32 + bw + 4 * (4 * hh + i)) * TP + cp) = make_float2(-acc[i].x, -acc[i].y);
             }
             group_sync(BAR_BACK, PF_BACK);
 
