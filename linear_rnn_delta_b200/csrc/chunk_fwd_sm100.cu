@@ -354,6 +354,13 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
             }
         }
     }
+    // channel pairs (0, 1) and (2, 3) on the packed fp32 pipe: the same product per channel
+    float2 sc2[2] = {make_float2(sc[0], sc[1]), make_float2(sc[2], sc[3])};
+    auto dot4 = [](const float (&u)[4], const float (&w)[4]) {   // (u0 w0 + u2 w2) + (u1 w1 + u3 w3)
+        const float2 t = __ffma2_rn(make_float2(u[2], u[3]), make_float2(w[2], w[3]),
+                                    __fmul2_rn(make_float2(u[0], u[1]), make_float2(w[0], w[1])));
+        return t.x + t.y;
+    };
 #pragma unroll UNROLL
     for (int i = 0; i < 8; ++i) {
         const int r = tg * 8 + i;
@@ -365,21 +372,26 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
         float e[4] = {1.f, 1.f, 1.f, 1.f};
         if (EVEC) erase_gate4(x, r, cq, e);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            sc[c] *= v ? al[c] : 1.f;
-            const float ek = EVEC ? e[c] * kv[c] : kv[c];
-            oa[c] = v ? sc[c] * ek : 0.f;
-            oq[c] = v ? sc[c] * qv[c] : 0.f;
-            kb[c] = v ? __fdividef(kv[c], sc[c]) : 0.f;
+        for (int pp = 0; pp < 2; ++pp) {
+            const int c = 2 * pp;
+            sc2[pp] = __fmul2_rn(sc2[pp], v ? make_float2(al[c], al[c + 1]) : make_float2(1.f, 1.f));
+            const float2 ek = EVEC ? __fmul2_rn(make_float2(e[c], e[c + 1]), make_float2(kv[c], kv[c + 1]))
+                                   : make_float2(kv[c], kv[c + 1]);
+            const float2 a2 = __fmul2_rn(sc2[pp], ek), q2 = __fmul2_rn(sc2[pp], make_float2(qv[c], qv[c + 1]));
+            oa[c] = v ? a2.x : 0.f;
+            oa[c + 1] = v ? a2.y : 0.f;
+            oq[c] = v ? q2.x : 0.f;
+            oq[c + 1] = v ? q2.y : 0.f;
+            kb[c] = v ? __fdividef(kv[c], sc2[pp].x) : 0.f;
+            kb[c + 1] = v ? __fdividef(kv[c + 1], sc2[pp].y) : 0.f;
         }
         *reinterpret_cast<uint2 *>(sm + x.qa + sw_half(16384, r, cq)) = pack4(oa);
         *reinterpret_cast<uint2 *>(sm + x.qa + sw_half(16384, 64 + r, cq)) = pack4(oq);
         *reinterpret_cast<uint2 *>(sm + x.kb + sw_half(8192, r, cq)) = pack4(kb);
         float *bp = band_part + r * (PBAND * 32) + lane;
-        bp[0] = oq[0] * kb[0] + oq[1] * kb[1] + oq[2] * kb[2] + oq[3] * kb[3];
+        bp[0] = dot4(oq, kb);
 #pragma unroll
-        for (int w = 1; w < PBAND; ++w)
-            bp[w * 32] = oq[0] * kw[4 - w][0] + oq[1] * kw[4 - w][1] + oq[2] * kw[4 - w][2] + oq[3] * kw[4 - w][3];
+        for (int w = 1; w < PBAND; ++w) bp[w * 32] = dot4(oq, kw[4 - w]);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             kw[0][c] = kw[1][c]; kw[1][c] = kw[2][c]; kw[2][c] = kw[3][c]; kw[3][c] = kb[c];
