@@ -89,6 +89,18 @@ def test_bwd_head_dims_no_initial_state(dk, dv):
     _check(inp, _bwd(inp, d_o, None), d_o, None)
 
 
+@pytest.mark.parametrize("dk", [16, 32, 64, 128])
+@pytest.mark.parametrize("dv", [16, 32, 64, 128])
+def test_bwd_every_head_size(dk, dv):
+    """Every (d_k, d_v): the checkpoint scan's states-only variant in each lane-group shape, and both
+    adjoint kernels (shared-memory at d_k = 16, cluster rows otherwise), over three checkpointed chunks
+    of packed documents."""
+    inp = W.make_chunk_inputs("kda", "extended", "f32", H=1, d_k=dk, d_v=dv, seed=90 + dk + dv,
+                              doc_lens=[130, 0, 21], init_state="random", init_std=0.2)
+    d_o, dsf = W.grad_outputs(inp, seed=90 + dk + dv)
+    _check(inp, _bwd(inp, d_o, dsf), d_o, dsf)
+
+
 def test_bwd_long_sequence_one_head():
     """1024 tokens (16 checkpointed chunks) on the KDA gates at d = 128."""
     inp = W.make_chunk_inputs("kda", "extended", "bf16", B=1, T=1024, H=1, d_k=128, d_v=128, seed=73,

@@ -64,6 +64,16 @@ def test_other_head_dims(dk, dv, dtype):
     _full_check(inp)
 
 
+@pytest.mark.parametrize("dk", [16, 32, 64, 128])
+@pytest.mark.parametrize("dv", [16, 32, 64, 128])
+def test_token_scan_every_head_size(dk, dv):
+    """Every (d_k, d_v) the token scan is instantiated for (its lane groups take 4, 8 or 16 lanes and 2
+    or 4 value columns, one or two CTAs per head), packed documents with a ragged tail, at 1e-4."""
+    inp = W.make_chunk_inputs("rda", "extended", "f32", H=2, d_k=dk, d_v=dv, seed=14 + dk + dv,
+                              doc_lens=[37, 0, 70], init_state="random", init_std=0.3)
+    _full_check(inp, FORCE_SCAN)
+
+
 @pytest.mark.parametrize("form", ["fused", "split"])
 @pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 129])
 def test_awkward_lengths_bf16(T, form):
