@@ -315,10 +315,13 @@ __device__ __forceinline__ void snapshot_state(const FwdArgs &a, uint32_t tlane,
 // (summed over the 32 lanes = 128 channels by band_reduce).
 // FULL: all 64 rows valid (no masking).  EVEC: channel-wise erase vector
 // (GDN-2).  UNROLL: rows per unrolled step (register budget permitting).
-template <bool FULL, bool EVEC, int UNROLL>
+// BPRE: the erase vector of the thread's 8 rows was loaded by the caller (raw
+// bf16 pairs in bpre; the loop is then unrolled fully) instead of row by row.
+template <bool FULL, bool EVEC, int UNROLL, bool BPRE = false>
 __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot, const float *gamc,
-                                          float *band_part, int tg, int cq, int lane)
+                                          float *band_part, int tg, int cq, int lane, const uint2 *bpre = nullptr)
 {
+    static_assert(!BPRE || (EVEC && UNROLL == 8), "prefetched erase vectors: full unroll");
     uint8_t *sm = x.sm;
     const int nvalid = x.nvalid;
     float pre[4] = {1.f, 1.f, 1.f, 1.f};
@@ -370,7 +373,15 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
         unpack4(raw_quad(sm, RAW_K, r, cq), kv);
         unpack4(raw_quad(sm, RAW_Q, r, cq), qv);
         float e[4] = {1.f, 1.f, 1.f, 1.f};
-        if (EVEC) erase_gate4(x, r, cq, e);
+        if (BPRE) {
+            unpack4(bpre[i], e);
+            if (x.logits) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) e[c] = round_bf16(prep_gate(e[c], x.ext));
+            }
+        } else if (EVEC) {
+            erase_gate4(x, r, cq, e);
+        }
 #pragma unroll
         for (int pp = 0; pp < 2; ++pp) {
             const int c = 2 * pp;
@@ -1762,13 +1773,14 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
             // (every thread: its 8 rows x 4 channels) are put in flight first
             uint32_t nge = 0, ngw = 0;
             if (ptid >= 64 && ptid < 64 + C) load_gates(nxt, ptid - 64, nge, ngw);
-            uint2 wraw[8];
+            uint2 wraw[8], braw[8];   // GDN-2: write and erase vectors of the thread's rows
             if (gdn2) {
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int r = tg * 8 + i;
-                    wraw[i] = r < nvalid ? *reinterpret_cast<const uint2 *>(g2p + ((rowbase + r) * H + h) * D + cq * 4)
-                                         : make_uint2(0u, 0u);
+                    const size_t off = ((rowbase + r) * H + h) * D + cq * 4;
+                    wraw[i] = r < nvalid ? *reinterpret_cast<const uint2 *>(g2p + off) : make_uint2(0u, 0u);
+                    braw[i] = r < nvalid ? *reinterpret_cast<const uint2 *>(g1p + off) : make_uint2(0u, 0u);
                 }
             }
 
@@ -1906,7 +1918,7 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
             if (fast) {
                 float *band_part = reinterpret_cast<float *>(sm + P2_FR);
                 if (nvalid == C) {
-                    if (gdn2) fast_rows<true, true, 4>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    if (gdn2) fast_rows<true, true, 8, true>(x, s_tot, gamc, band_part, tg, cq, lane, braw);
                     else fast_rows<true, false, 4>(x, s_tot, gamc, band_part, tg, cq, lane);
                 } else {
                     fast_rows<false, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
