@@ -1780,7 +1780,6 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                     const int r = tg * 8 + i;
                     const size_t off = ((rowbase + r) * H + h) * D + cq * 4;
                     wraw[i] = r < nvalid ? *reinterpret_cast<const uint2 *>(g2p + off) : make_uint2(0u, 0u);
-                    braw[i] = r < nvalid ? *reinterpret_cast<const uint2 *>(g1p + off) : make_uint2(0u, 0u);
                 }
             }
 
@@ -1878,6 +1877,14 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
                         for (int c = 0; c < 4; ++c) mv[c] = 0.f;
                     }
                     *pv = pack4(mv);
+                }
+            }
+            if (gdn2) {   // the erase vectors, read by the row sweep (w is consumed: its registers are free)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = tg * 8 + i;
+                    braw[i] = r < nvalid ? *reinterpret_cast<const uint2 *>(g1p + ((rowbase + r) * H + h) * D + cq * 4)
+                                         : make_uint2(0u, 0u);
                 }
             }
             if (lane == 0) bulk_wait_read();   // this group's stores of the previous item have read their tiles
