@@ -305,24 +305,23 @@ __device__ __forceinline__ void snapshot_state(const FwdArgs &a, uint32_t tlane,
     }
 }
 
-// Fast path, step 1b for the item (tg, cq): a backward sweep for Kbar, then one
-// forward sweep over the item's 8 rows.  With sc = Gamma_r / Gamma_C (|sc| >= 1
-// since every |alpha| <= 1):
+// Fast path, step 1b for the item (tg, cq): one forward sweep over the item's
+// 8 rows.  With sc = Gamma_r / Gamma_C (|sc| >= 1 since every |alpha| <= 1):
 //   row operands  Gamma a~ / Gamma_C = sc (.) a~,   Gamma q / Gamma_C = sc (.) q,
-//   Kbar_r = Lam_{C-1,r} (.) k_r   (Lam a product of the later rows' alpha: no division).
+//   Kbar_r = Lam_{C-1,r} (.) k_r = k_r / sc   (the divisor is bounded away from zero).
 // The band of P, P_{r,r-w} = sum_c (sc q)_{r,c} Kbar_{r-w,c} for w = 0..4, is
 // formed from these fp32 values: a window keeps Kbar of the four previous
 // rows, and each lane's 4-channel partial sums go to band_part[r][w][lane]
 // (summed over the 32 lanes = 128 channels by band_reduce).
 // FULL: all 64 rows valid (no masking).  EVEC: channel-wise erase vector
-// (GDN-2).  BPRE: the erase vector of the thread's 8 rows was loaded by the
-// caller (raw bf16 pairs in bpre) instead of row by row.  The row loops are
-// unrolled fully (Kbar of the 8 rows is held in registers).
-template <bool FULL, bool EVEC, bool BPRE = false>
+// (GDN-2).  UNROLL: rows per unrolled step (register budget permitting).
+// BPRE: the erase vector of the thread's 8 rows was loaded by the caller (raw
+// bf16 pairs in bpre; the loop is then unrolled fully) instead of row by row.
+template <bool FULL, bool EVEC, int UNROLL, bool BPRE = false>
 __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot, const float *gamc,
                                           float *band_part, int tg, int cq, int lane, const uint2 *bpre = nullptr)
 {
-    static_assert(!BPRE || EVEC, "prefetched erase vectors");
+    static_assert(!BPRE || (EVEC && UNROLL == 8), "prefetched erase vectors: full unroll");
     uint8_t *sm = x.sm;
     const int nvalid = x.nvalid;
     float pre[4] = {1.f, 1.f, 1.f, 1.f};
@@ -336,33 +335,9 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
     }
     const float4 gc4 = *reinterpret_cast<const float4 *>(gamc + cq * 4);
     float sc[4] = {pre[0] / gc4.x, pre[1] / gc4.y, pre[2] / gc4.z, pre[3] / gc4.w};
-    // Kbar_r = Lam_{C-1,r} (.) k_r, Lam_{C-1,r} the product of alpha over the valid rows after r:
-    // a backward sweep over the thread's 8 rows and the 4 before them (the band's window), from
-    // the later blocks' totals, by multiplications only
-    float kbv[8][4], kw[4][4];   // Kbar of the thread's rows; of rows 8tg-4 .. 8tg-1
+    float kw[4][4];   // Kbar of rows r-4 .. r-1
     {
-        float suf[4] = {1.f, 1.f, 1.f, 1.f};
-#pragma unroll
-        for (int g = 7; g > 0; --g) {
-            if (g <= tg) break;
-            float t4[4];
-            load_tot4(s_tot, g, cq, t4);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) suf[c] *= t4[c];
-        }
-#pragma unroll
-        for (int i = 7; i >= 0; --i) {
-            const int r = tg * 8 + i;
-            const bool v = FULL || r < nvalid;
-            float kv[4], av[4];
-            unpack4(raw_quad(sm, RAW_K, r, cq), kv);
-            unpack4(raw_quad(sm, RAW_A, r, cq), av);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                kbv[i][c] = v ? suf[c] * kv[c] : 0.f;
-                suf[c] *= v ? av[c] : 1.f;
-            }
-        }
+        float sb4[4] = {sc[0], sc[1], sc[2], sc[3]};   // Gamma_{8tg-1} / Gamma_C
 #pragma unroll
         for (int j = 3; j >= 0; --j) {
             const int rp = tg * 8 - 4 + j;
@@ -373,8 +348,8 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
                 const bool v = FULL || rp < nvalid;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    kw[j][c] = v ? suf[c] * kv[c] : 0.f;
-                    suf[c] *= v ? av[c] : 1.f;
+                    kw[j][c] = v ? __fdividef(kv[c], sb4[c]) : 0.f;
+                    sb4[c] = v ? __fdividef(sb4[c], av[c]) : sb4[c];
                 }
             } else {
 #pragma unroll
@@ -389,7 +364,7 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
                                     __fmul2_rn(make_float2(u[0], u[1]), make_float2(w[0], w[1])));
         return t.x + t.y;
     };
-#pragma unroll
+#pragma unroll UNROLL
     for (int i = 0; i < 8; ++i) {
         const int r = tg * 8 + i;
         const bool v = FULL || r < nvalid;
@@ -418,8 +393,8 @@ __device__ __forceinline__ void fast_rows(const ChunkCtx &x, const float *s_tot,
             oa[c + 1] = v ? a2.y : 0.f;
             oq[c] = v ? q2.x : 0.f;
             oq[c + 1] = v ? q2.y : 0.f;
-            kb[c] = kbv[i][c];
-            kb[c + 1] = kbv[i][c + 1];
+            kb[c] = v ? __fdividef(kv[c], sc2[pp].x) : 0.f;
+            kb[c + 1] = v ? __fdividef(kv[c + 1], sc2[pp].y) : 0.f;
         }
         *reinterpret_cast<uint2 *>(sm + x.qa + sw_half(16384, r, cq)) = pack4(oa);
         *reinterpret_cast<uint2 *>(sm + x.qa + sw_half(16384, 64 + r, cq)) = pack4(oq);
@@ -1137,10 +1112,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_kernel(const __grid_constant_
                 // one forward sweep per item; band partials to the F region, reduced after the A/P GEMM issue
                 float *band_part = reinterpret_cast<float *>(sm + OFF_F);
                 if (nvalid == C) {
-                    if (gdn2) fast_rows<true, true>(x, s_tot, gamc, band_part, tg, cq, lane);
-                    else fast_rows<true, false>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    if (gdn2) fast_rows<true, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    else fast_rows<true, false, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
                 } else {
-                    fast_rows<false, true>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    fast_rows<false, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
                 }
             } else {
             {
@@ -1950,10 +1925,10 @@ __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_const
             if (fast) {
                 float *band_part = reinterpret_cast<float *>(sm + P2_FR);
                 if (nvalid == C) {
-                    if (gdn2) fast_rows<true, true, true>(x, s_tot, gamc, band_part, tg, cq, lane, braw);
-                    else fast_rows<true, false>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    if (gdn2) fast_rows<true, true, 8, true>(x, s_tot, gamc, band_part, tg, cq, lane, braw);
+                    else fast_rows<true, false, 4>(x, s_tot, gamc, band_part, tg, cq, lane);
                 } else {
-                    fast_rows<false, true>(x, s_tot, gamc, band_part, tg, cq, lane);
+                    fast_rows<false, true, 1>(x, s_tot, gamc, band_part, tg, cq, lane);
                 }
             } else {
                 {
