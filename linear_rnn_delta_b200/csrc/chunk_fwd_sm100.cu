@@ -1632,6 +1632,9 @@ __device__ __forceinline__ Item ring_get(const int *ring, int k)
 template <bool PREP>
 __global__ void __launch_bounds__(PF_NT, 1) chunk_prep_kernel(const __grid_constant__ ChunkParams P)
 {
+    // the chain kernel may be scheduled now: it sets itself up on SMs this grid leaves and waits
+    // for this grid's completion before it reads a slot
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sb = smem_u32(sm);
@@ -2557,6 +2560,10 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
     // testing aid: this CTA never loads its first slot, so that waiting for it runs out
     const bool stall = P.debug_stall && blockIdx.x == 0;
     if (tid == 0) {
+        // launched as a programmatic dependent of the preparation kernel: the slots are complete
+        // and visible once this returns (at once when launched plainly).  Nothing else this
+        // kernel reads before its first slot is written by the preparation kernel.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         if (nchunks > 0 && !stall) issue_load(0, 0);
         if (nchunks > 1) issue_load(1, 1);
     }
@@ -2632,9 +2639,15 @@ __global__ void __launch_bounds__(CK_NT, 1) chunk_chain_kernel(const __grid_cons
                 float *sv = s + c32 * 32;
                 float t[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    t[e] = sv[e] * gamC[i0 + e];
-                    if (fast) sv[e] = t[e];
+                for (int e = 0; e < 32; e += 2) {   // column pairs on the packed fp32 pipe
+                    const float2 t2 = __fmul2_rn(make_float2(sv[e], sv[e + 1]),
+                                                 *reinterpret_cast<const float2 *>(gamC + i0 + e));
+                    t[e] = t2.x;
+                    t[e + 1] = t2.y;
+                    if (fast) {
+                        sv[e] = t2.x;
+                        sv[e + 1] = t2.y;
+                    }
                 }
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
@@ -2882,15 +2895,29 @@ cudaError_t launch_chunk_split_sm100(const FwdArgs &a, void *ws, cudaStream_t st
     p.epoch = epoch.fetch_add(1) + 1;   // a 32-bit tag: it repeats only after 2^32 split-form calls
     p.debug_stall = a.debug_stall;
     const long long nwork = (long long)p.nslots * a.H;
-    if (rows > 0 && nwork > 0) {
+    const bool prep = rows > 0 && nwork > 0;
+    if (prep) {
         const unsigned grid = (unsigned)std::min<long long>(nwork, num_sms);
         if (a.prep) chunk_prep_kernel<true><<<grid, PF_NT, P2_ALLOC, st>>>(p);
         else chunk_prep_kernel<false><<<grid, PF_NT, P2_ALLOC, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if (a.snap) chunk_chain_kernel<true><<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);
-    else chunk_chain_kernel<false><<<(unsigned)(N * a.H), CK_NT, CK_ALLOC, st>>>(p);
-    return cudaGetLastError();
+    // The chain kernel is a programmatic dependent of the preparation kernel (it may start its
+    // set-up while the preparation grid drains; its slot reads wait for that grid).  Only then:
+    // behind any other kernel its initial-state reads would not wait.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(N * a.H));
+    cfg.blockDim = dim3(CK_NT);
+    cfg.dynamicSmemBytes = CK_ALLOC;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = prep ? 1 : 0;
+    if (a.snap) e = cudaLaunchKernelEx(&cfg, chunk_chain_kernel<true>, p);
+    else e = cudaLaunchKernelEx(&cfg, chunk_chain_kernel<false>, p);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace kda
