@@ -265,13 +265,15 @@ int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
  * The gradient is that of the exact recurrence, in fp32 arithmetic (adjoint of
  * one step: G_{t-1} = Diag(alpha_t) (I - a~_t k_t^T) (G_t + q_t do_t^T)).  Two
  * launches on `stream`: a token scan stores the fp32 state after every 64
- * tokens; then a cluster of d_v/32 CTAs per (sequence, head) replays each
- * chunk from its checkpoint and walks it backwards.  Results are
- * deterministic (fixed summation order).
+ * tokens and the residual u_t = m_t - S_{t-1}^T Diag(alpha_t) a~_t of every
+ * token; then a cluster of d_v/32 CTAs per (sequence, head) replays each
+ * chunk from its checkpoint (with the stored u_t: the update alone) and walks
+ * it backwards.  Results are deterministic (fixed summation order).
  * workspace: caller-owned, 16-byte aligned, at least
  * kda_chunk_bwd_workspace_size(...) bytes: (N + ceil(B*T/64)) * H * d_k * d_v
- * * 4 for the checkpoints plus N * H * 16 * d_k * d_v * 4 (N * H * 64 * d_k *
- * d_v * 4 at d_k = 16) for the states kept during the replay.
+ * * 4 for the checkpoints, B * T * H * d_v * 4 for u_t, plus N * H * 16 * d_k
+ * * d_v * 4 (N * H * 64 * d_k * d_v * 4 at d_k = 16) for the states kept
+ * during the replay.
  * Errors: as kda_chunk_fwd; KDA_ERR_INVALID_ARG also for nonzero flags, a NULL
  * or misaligned gradient pointer (dg2 only for RDA and GDN-2) or a workspace
  * that is NULL, misaligned or too small.

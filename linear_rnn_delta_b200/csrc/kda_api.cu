@@ -294,13 +294,18 @@ extern "C" int kda_chunk_fwd_noalloc(int variant, int gate_range, int dtype,
 
 namespace {
 
-// Backward workspace: the forward's state snapshots (chunk slots) and each
-// CTA's per-chunk states.
-size_t bwd_workspace_bytes(const kda::FwdArgs &a)
+// Backward workspace: the forward's state snapshots (chunk slots), u_t of
+// every token, and each CTA's per-chunk states, in that order.
+size_t bwd_snap_bytes(const kda::FwdArgs &a)
 {
     const long long N = a.cu_seqlens ? a.num_seqs : a.B;
     const long long slots = N + ((long long)a.B * a.T + 63) / 64;
-    return (size_t)slots * a.H * a.dk * a.dv * sizeof(float) + kda::scan_bwd_scratch_bytes(a);
+    return (size_t)slots * a.H * a.dk * a.dv * sizeof(float);
+}
+size_t bwd_u_bytes(const kda::FwdArgs &a) { return (size_t)a.B * a.T * a.H * a.dv * sizeof(float); }
+size_t bwd_workspace_bytes(const kda::FwdArgs &a)
+{
+    return bwd_snap_bytes(a) + bwd_u_bytes(a) + kda::scan_bwd_scratch_bytes(a);
 }
 
 }  // namespace
@@ -354,16 +359,17 @@ extern "C" int kda_chunk_bwd(int variant, int gate_range, int dtype,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool bf16 = dtype == KDA_DTYPE_BF16;
     // 1. forward scan in fp32, keeping only the state after every 64 tokens (the checkpoints)
+    //    and u_t of every token
     a.o = nullptr;
     a.sf = nullptr;
     a.snap = static_cast<float *>(workspace);
-    const long long N = a.cu_seqlens ? a.num_seqs : a.B;
-    const size_t snap_bytes = (size_t)(N + ((long long)a.B * a.T + 63) / 64) * a.H * a.dk * a.dv * sizeof(float);
-    cudaError_t e = kda::launch_scan_fwd(a, bf16, st);
+    float *u_save = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + bwd_snap_bytes(a));
+    cudaError_t e = kda::launch_scan_checkpoints(a, u_save, bf16, st);
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd forward replay");
     // 2. adjoint scan
     kda::BwdArgs g{d_o, d_final_state, dq, dk, dv, dalpha, dg1, dg2, d_initial_state,
-                   reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + snap_bytes)};
+                   reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + bwd_snap_bytes(a) + bwd_u_bytes(a)),
+                   u_save};
     e = kda::launch_scan_bwd(a, g, bf16, st);
     if (e != cudaSuccess) return cuda_fail(e, "kda_chunk_bwd launch");
     return KDA_OK;

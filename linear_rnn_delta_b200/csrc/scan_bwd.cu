@@ -22,11 +22,13 @@
 // barrier.  The per-row results (dq, dk, dalpha, k (.) da~) are partial sums
 // over the CTA's columns; the cluster
 // adds them through distributed shared memory every 8 tokens, in a fixed order
-// (deterministic results).  The replay keeps S_{t-1} only every 4 tokens
+// (deterministic results).  The checkpoint scan also keeps u_t of every token,
+// so the replay of a chunk is the state update alone (no sum over key rows, no
+// barrier), bitwise the scan's own steps.  It keeps S_{t-1} only every 4 tokens
 // (global scratch) with u_t in shared memory; the backward walk recomputes the
 // states in between with the same fused multiply-adds, so they are bitwise
 // those of the replay.  d_k = 16 uses a plain shared-memory kernel (one CTA per
-// sequence and head).
+// sequence and head) that replays with its own sums.
 #include "scan_bwd.cuh"
 
 #include <cooperative_groups.h>
@@ -311,7 +313,7 @@ constexpr int RTB = 8;   // tokens per cross-CTA reduction block
 template <int DK, int DVB>
 struct RowSmem {
     static constexpr int NW = DK / 32;
-    static constexpr size_t U = 0;                               // [BC][DVB] u_t of the chunk
+    static constexpr size_t U = 0;                               // [BC][DVB] u_t of the chunk (from the scan)
     static constexpr size_t DO = U + (size_t)BC * DVB;           // [BC][DVB] do_t
     static constexpr size_t VV = DO + (size_t)BC * DVB;          // [BC][DVB] v_t
     static constexpr size_t WW = VV + (size_t)BC * DVB;          // [BC][DVB] write gate (scalar gates broadcast)
@@ -429,6 +431,7 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
         constexpr int SB = 8;   // elements per thread loaded before any is widened
         for (int e0 = i; e0 < nt * DVB; e0 += DK * SB) {
             TIn rv[SB], rw[SB], rd[SB];
+            float ru[SB];
 #pragma unroll
             for (int b = 0; b < SB; ++b) {
                 const int e = e0 + b * DK;
@@ -438,6 +441,7 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                     rv[b] = v[cj];
                     rw[b] = a.variant == KDA ? g1[tok] : (a.variant == RDA ? g2[tok] : g2[cj]);
                     rd[b] = dO[cj];
+                    ru[b] = g.u[cj];
                 }
             }
 #pragma unroll
@@ -447,6 +451,7 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                     sV[e] = widen(rv[b]);
                     sW[e] = widen(rw[b]);
                     sDO[e] = widen(rd[b]);
+                    sU[e] = ru[b];
                 }
             }
         }
@@ -454,17 +459,20 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                            : a.snap + (((size_t)(slot_base(a, n) + c - 1) * a.H + h) * DK + i) * a.dv +
                                  (size_t)jb * DVB);
         __syncthreads();
-        // ---- replay: u_t into shared memory, S_{t-1} every CKP tokens into scratch
-        TIn n_al = TIn(0.f), n_k = TIn(0.f), n_e = TIn(0.f);   // next token's row scalars, raw
+        // ---- replay: S_{t-1} every CKP tokens into scratch.  u_t comes from the checkpoint
+        // scan, so a step is the update S_ij = alpha_i S_ij + k_i u_j alone (the scan's own
+        // fused multiply-add: the replayed states are the scan's, bit for bit), with no sum
+        // over rows and no barrier
+        TIn n_al = TIn(0.f), n_k = TIn(0.f);   // next token's row scalars, raw
         if (nt > 0) {
             const size_t tok = tok_of(t0);
-            n_al = al[tok * DK + i]; n_k = k[tok * DK + i]; n_e = gate_raw(tok);
+            n_al = al[tok * DK + i]; n_k = k[tok * DK + i];
         }
         for (int tt = 0; tt < nt; ++tt) {
-            const float alpha_i = widen(n_al), k_i = widen(n_k), e_i = widen(n_e);
+            const float alpha_i = widen(n_al), k_i = widen(n_k);
             if (tt + 1 < nt) {
                 const size_t tok = tok_of(t0 + tt + 1);
-                n_al = al[tok * DK + i]; n_k = k[tok * DK + i]; n_e = gate_raw(tok);
+                n_al = al[tok * DK + i]; n_k = k[tok * DK + i];
             }
             if (tt % CKP == 0) {
 #pragma unroll
@@ -472,29 +480,15 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                     scr[((size_t)(tt / CKP) * NQ + c4) * DK + i] =
                         make_float4(S[2 * c4].x, S[2 * c4].y, S[2 * c4 + 1].x, S[2 * c4 + 1].y);
             }
-            float x[DVB];
-            const float aa = alpha_i * (e_i * k_i);   // alpha_i a~_i
-#pragma unroll
-            for (int j2 = 0; j2 < DVB / 2; ++j2) {
-                const float2 t = __fmul2_rn(dup(aa), S[j2]);
-                x[2 * j2] = t.x;
-                x[2 * j2 + 1] = t.y;
-            }
-            float *fin = column_sums(x);
-            if (owner) {   // u_j = m_j - sum_i alpha_i a~_i S_ij
-                const float u = sW[tt * DVB + col] * sV[tt * DVB + col] - fin[col];
-                fin[col] = u;
-                if (warp == 0) sU[tt * DVB + col] = u;
-            }
-            __syncwarp();
+            const float4 *u4p = reinterpret_cast<const float4 *>(sU + tt * DVB);
 #pragma unroll
             for (int c4 = 0; c4 < NQ; ++c4) {
-                const float4 u4 = reinterpret_cast<const float4 *>(fin)[c4];
+                const float4 u4 = u4p[c4];
                 S[2 * c4] = __ffma2_rn(dup(alpha_i), S[2 * c4], __fmul2_rn(dup(k_i), make_float2(u4.x, u4.y)));
                 S[2 * c4 + 1] = __ffma2_rn(dup(alpha_i), S[2 * c4 + 1], __fmul2_rn(dup(k_i), make_float2(u4.z, u4.w)));
             }
         }
-        __syncthreads();   // u_t of the chunk visible to every warp
+        __syncthreads();   // the replay is done (and its scratch stores ordered) before the walk reads them back
         // ---- backward walk, last token first, in groups of CKP tokens (one stored state each)
         const int ngrp = (nt + CKP - 1) / CKP;
         float4 *ckb = reinterpret_cast<float4 *>(smf + L::CKB);   // [2][NQ][DK]: each thread its own row

@@ -25,8 +25,10 @@
 // Token vectors are staged TB tokens at a time in shared memory, double
 // buffered, so the inner loop runs without barriers; optional input
 // preparation (gate activations, L2 norm of k) is applied while staging.  Without an output (the backward's
-// checkpoints) the readout is compiled out.
+// checkpoints) the readout is compiled out, and u_t of every token may be kept instead: with it the
+// backward replays a chunk from its checkpoint by the update alone, bitwise as this scan ran it.
 #include "common.cuh"
+#include "scan_bwd.cuh"
 
 namespace kda {
 namespace {
@@ -74,10 +76,11 @@ __device__ __forceinline__ float group_sum(float x)
 }
 
 // PREP: input preparation requested; OUT: o is written.  Without either, that
-// code is compiled out.
+// code is compiled out.  u_save (states-only variant, may be null): u_t, fp32,
+// in o's layout [B*T][H][d_v].
 template <int DK, int DV, typename TIn, bool PREP, bool OUT>
 __global__ void __launch_bounds__(ScanShape<DK, DV>::NTH)
-scan_fwd_kernel(FwdArgs a)
+scan_fwd_kernel(FwdArgs a, float *u_save)
 {
     using SH = ScanShape<DK, DV>;
     constexpr int KS = SH::KS, NG = SH::NG, CB = SH::CB, CC = SH::CC, NTH = SH::NTH, CTAS = SH::CTAS;
@@ -222,6 +225,13 @@ scan_fwd_kernel(FwdArgs a)
                 u[2 * c] -= group_sum<KS>(r[c][0].x + r[c][1].x);
                 u[2 * c + 1] -= group_sum<KS>(r[c][0].y + r[c][1].y);
             }
+            const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
+            if (!OUT && u_save && p == 0) {   // every lane of the group holds the same bits
+                float2 u2[CC / 2];
+#pragma unroll
+                for (int c = 0; c < CC / 2; ++c) u2[c] = make_float2(u[2 * c], u[2 * c + 1]);
+                st_cols<CC>(u_save + tok * DV + j, u2);
+            }
             float2 o[CC / 2][2];
 #pragma unroll
             for (int c = 0; c < CC / 2; ++c) o[c][0] = o[c][1] = make_float2(0.f, 0.f);
@@ -247,7 +257,6 @@ scan_fwd_kernel(FwdArgs a)
                             o[c][e & 1] = __ffma2_rn(make_float2(q4[e], q4[e]), S2[4 * m + e][c], o[c][e & 1]);
                 }
             }
-            const size_t tok = ((size_t)b * a.T + t0 + base + tt) * a.H + h;
             if (OUT) {
                 float ov[CC];
 #pragma unroll
@@ -283,48 +292,56 @@ scan_fwd_kernel(FwdArgs a)
 // Variants launched: with output, with or without input preparation; states
 // only (the backward's checkpoints), without preparation.
 template <int DK, int DV, typename TIn>
-void launch_typed(const FwdArgs &a, dim3 grid, cudaStream_t st)
+void launch_typed(const FwdArgs &a, float *u_save, dim3 grid, cudaStream_t st)
 {
     constexpr int NTH = ScanShape<DK, DV>::NTH;
-    if (a.prep) scan_fwd_kernel<DK, DV, TIn, true, true><<<grid, NTH, 0, st>>>(a);
-    else if (a.o) scan_fwd_kernel<DK, DV, TIn, false, true><<<grid, NTH, 0, st>>>(a);
-    else scan_fwd_kernel<DK, DV, TIn, false, false><<<grid, NTH, 0, st>>>(a);
+    if (a.prep) scan_fwd_kernel<DK, DV, TIn, true, true><<<grid, NTH, 0, st>>>(a, nullptr);
+    else if (a.o) scan_fwd_kernel<DK, DV, TIn, false, true><<<grid, NTH, 0, st>>>(a, nullptr);
+    else scan_fwd_kernel<DK, DV, TIn, false, false><<<grid, NTH, 0, st>>>(a, u_save);
 }
 
 template <int DK, int DV>
-cudaError_t launch_dims(const FwdArgs &a, bool bf16, cudaStream_t st)
+cudaError_t launch_dims(const FwdArgs &a, float *u_save, bool bf16, cudaStream_t st)
 {
     if (a.prep && !a.o) return cudaErrorInvalidValue;   // no such variant (and no caller)
     const int N = a.cu_seqlens ? a.num_seqs : a.B;
     const dim3 grid((unsigned)(N * a.H * ScanShape<DK, DV>::CTAS));
-    if (bf16) launch_typed<DK, DV, __nv_bfloat16>(a, grid, st);
-    else launch_typed<DK, DV, float>(a, grid, st);
+    if (bf16) launch_typed<DK, DV, __nv_bfloat16>(a, u_save, grid, st);
+    else launch_typed<DK, DV, float>(a, u_save, grid, st);
     return cudaGetLastError();
 }
 
 template <int DK>
-cudaError_t launch_dv(const FwdArgs &a, bool bf16, cudaStream_t st)
+cudaError_t launch_dv(const FwdArgs &a, float *u_save, bool bf16, cudaStream_t st)
 {
     switch (a.dv) {
-    case 16: return launch_dims<DK, 16>(a, bf16, st);
-    case 32: return launch_dims<DK, 32>(a, bf16, st);
-    case 64: return launch_dims<DK, 64>(a, bf16, st);
-    case 128: return launch_dims<DK, 128>(a, bf16, st);
+    case 16: return launch_dims<DK, 16>(a, u_save, bf16, st);
+    case 32: return launch_dims<DK, 32>(a, u_save, bf16, st);
+    case 64: return launch_dims<DK, 64>(a, u_save, bf16, st);
+    case 128: return launch_dims<DK, 128>(a, u_save, bf16, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_any(const FwdArgs &a, float *u_save, bool bf16, cudaStream_t st)
+{
+    switch (a.dk) {
+    case 16: return launch_dv<16>(a, u_save, bf16, st);
+    case 32: return launch_dv<32>(a, u_save, bf16, st);
+    case 64: return launch_dv<64>(a, u_save, bf16, st);
+    case 128: return launch_dv<128>(a, u_save, bf16, st);
     }
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_scan_fwd(const FwdArgs &a, bool bf16, cudaStream_t st)
+cudaError_t launch_scan_fwd(const FwdArgs &a, bool bf16, cudaStream_t st) { return launch_any(a, nullptr, bf16, st); }
+
+cudaError_t launch_scan_checkpoints(const FwdArgs &a, float *u_save, bool bf16, cudaStream_t st)
 {
-    switch (a.dk) {
-    case 16: return launch_dv<16>(a, bf16, st);
-    case 32: return launch_dv<32>(a, bf16, st);
-    case 64: return launch_dv<64>(a, bf16, st);
-    case 128: return launch_dv<128>(a, bf16, st);
-    }
-    return cudaErrorInvalidValue;
+    if (a.o || a.prep || !a.snap) return cudaErrorInvalidValue;   // the states-only variant
+    return launch_any(a, u_save, bf16, st);
 }
 
 }  // namespace kda

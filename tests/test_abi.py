@@ -213,11 +213,12 @@ def test_rank2_rejects_bad_arguments(lib, kw, code, detail):
 # ---- backward -------------------------------------------------------------------------------
 
 def test_bwd_workspace_size(lib):
-    # checkpoints: (N + ceil(B*T/64)) slots x H x d_k x d_v fp32, plus N*H*16*d_k*d_v fp32 replay states
+    # checkpoints: (N + ceil(B*T/64)) slots x H x d_k x d_v fp32, u_t: B*T*H*d_v fp32,
+    # plus N*H*16*d_k*d_v fp32 replay states
     assert lib.kda_chunk_bwd_workspace_size(0, 2, 100, 3, 128, 128, 0, 2) == \
-        (2 + 4) * 3 * 128 * 128 * 4 + 2 * 3 * 16 * 128 * 128 * 4
+        (2 + 4) * 3 * 128 * 128 * 4 + 2 * 100 * 3 * 128 * 4 + 2 * 3 * 16 * 128 * 128 * 4
     assert lib.kda_chunk_bwd_workspace_size(1, 1, 10, 1, 16, 32, 1, 3) == \
-        (3 + 1) * 1 * 16 * 32 * 4 + 3 * 1 * 64 * 16 * 32 * 4     # d_k = 16: every state of a chunk
+        (3 + 1) * 1 * 16 * 32 * 4 + 10 * 32 * 4 + 3 * 1 * 64 * 16 * 32 * 4     # d_k = 16: every state of a chunk
     assert lib.kda_chunk_bwd_workspace_size(0, 2, 100, 3, 48, 128, 0, 2) == 0
     assert lib.kda_chunk_bwd_workspace_size(0, 2, 100, 3, 128, 128, 1, 2) == 0   # cu_seqlens needs B == 1
 
