@@ -94,7 +94,7 @@ enum kda_status {
 /* KDA_FLAG_VALIDATE_RANGE -- before the work is launched, check on the device
  * that every gate lies in the declared range (alpha, and beta / e / GDN-2's b,
  * as kda_check_gates does; NaN fails) and that cu_seqlens keeps its contract
- * (as kda_check_seqlens does), and WAIT for the verdict: the call then
+ * (as kda_check_seqlens does), and WAIT for the outcome: the call then
  * synchronises `stream`.  A violation returns KDA_ERR_RANGE (gates) or
  * KDA_ERR_INVALID_ARG (cu_seqlens) and launches nothing.  With
  * KDA_FLAG_GATE_LOGITS only cu_seqlens is checked (logits have no range).

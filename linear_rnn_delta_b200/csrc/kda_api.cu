@@ -120,7 +120,7 @@ int chunk_args(kda::FwdArgs &a, int variant, int gate_range, int dtype, int B, i
 }
 
 // KDA_FLAG_VALIDATE_RANGE: check the gates against the declared range and
-// cu_seqlens against its contract on the device, wait for the verdict, and
+// cu_seqlens against its contract on the device, wait for the outcome, and
 // refuse the call (nothing launched) on a violation.  Gate logits are not
 // gates yet: with KDA_FLAG_GATE_LOGITS only cu_seqlens is checked.
 int validate(const kda::FwdArgs &a, int gate_range, int dtype, unsigned flags, cudaStream_t st)
