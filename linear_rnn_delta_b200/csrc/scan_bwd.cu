@@ -325,7 +325,8 @@ struct RowSmem {
     static constexpr size_t TOK = SRED + RTB * NW;               // [2][RTB] token index (int)
     static constexpr size_t CKB = TOK + 2 * RTB;                 // [2][DVB/4][DK] float4: a group's stored state
     static constexpr size_t RSM = CKB + 2 * (size_t)DVB * DK;    // [CKP][4][DK] row scalars of a group
-    static constexpr size_t FLOATS = RSM + (size_t)CKP * 4 * DK;
+    static constexpr size_t UDO = RSM + (size_t)CKP * 4 * DK;    // [BC] sum_j u_j do_j over the CTA's columns
+    static constexpr size_t FLOATS = UDO + BC;
 };
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
@@ -459,6 +460,18 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                            : a.snap + (((size_t)(slot_base(a, n) + c - 1) * a.H + h) * DK + i) * a.dv +
                                  (size_t)jb * DVB);
         __syncthreads();
+        if (i < nt) {   // per token: sum over the CTA's columns of u_j do_j (row-independent)
+            const float4 *d4p = reinterpret_cast<const float4 *>(sDO + i * DVB);
+            const float4 *u4p = reinterpret_cast<const float4 *>(sU + i * DVB);
+            float2 udo = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int c4 = 0; c4 < NQ; ++c4) {
+                const float4 d4 = d4p[c4], u4 = u4p[c4];
+                udo = __ffma2_rn(make_float2(u4.x, u4.y), make_float2(d4.x, d4.y), udo);
+                udo = __ffma2_rn(make_float2(u4.z, u4.w), make_float2(d4.z, d4.w), udo);
+            }
+            smf[L::UDO + i] = udo.x + udo.y;
+        }
         // ---- replay: S_{t-1} every CKP tokens into scratch.  u_t comes from the checkpoint
         // scan, so a step is the update S_ij = alpha_i S_ij + k_i u_j alone (the scan's own
         // fused multiply-add: the replayed states are the scan's, bit for bit), with no sum
@@ -560,9 +573,9 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                 const size_t tok = tok_of(t);
                 const float4 *do4 = reinterpret_cast<const float4 *>(sDO + tt * DVB);
                 const float4 *u4p = reinterpret_cast<const float4 *>(sU + tt * DVB);
-                // G += q do^T;  row partials of S_t do (= alpha S_{t-1} do + k (u.do)) and G u
-                // (partial sums over even and odd columns in .x and .y)
-                float2 sdo = make_float2(0.f, 0.f), udo = sdo, gu = sdo;
+                // G += q do^T;  row partials of S_t do (= alpha S_{t-1} do + k (u.do), u.do summed once
+                // per token above) and G u (partial sums over even and odd columns in .x and .y)
+                float2 sdo = make_float2(0.f, 0.f), gu = sdo;
 #pragma unroll
                 for (int c4 = 0; c4 < NQ; ++c4) {
                     const float4 d4 = do4[c4], u4 = u4p[c4];
@@ -573,7 +586,6 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                         const int j2 = 2 * c4 + e;
                         G[j2] = __ffma2_rn(dup(q_i), dd[e], G[j2]);
                         sdo = __ffma2_rn(S[j2], dd[e], sdo);
-                        udo = __ffma2_rn(uu[e], dd[e], udo);
                         gu = __ffma2_rn(G[j2], uu[e], gu);
                     }
                 }
@@ -620,7 +632,7 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                 // this CTA's parts (its value columns) of dq, dk, dalpha and k (.) da~, da~ = -Diag(alpha) S_{t-1} du
                 const float datp = -alpha_i * (sdu.x + sdu.y);
                 float *ring = smf + L::RING + ((size_t)((blk & 1) * RTB + pos) * 4) * DK;
-                ring[i] = fmaf(alpha_i, sdo.x + sdo.y, k_i * (udo.x + udo.y));
+                ring[i] = fmaf(alpha_i, sdo.x + sdo.y, k_i * smf[L::UDO + tt]);
                 ring[DK + i] = fmaf(e_i, datp, gu.x + gu.y);   // a~ = e (.) k: dk = G u + e da~
                 ring[2 * DK + i] = sds.x + sds.y;
                 ring[3 * DK + i] = k_i * datp;
