@@ -460,9 +460,9 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                            : a.snap + (((size_t)(slot_base(a, n) + c - 1) * a.H + h) * DK + i) * a.dv +
                                  (size_t)jb * DVB);
         __syncthreads();
-        if (i < nt) {   // per token: sum over the CTA's columns of u_j do_j (row-independent)
-            const float4 *d4p = reinterpret_cast<const float4 *>(sDO + i * DVB);
-            const float4 *u4p = reinterpret_cast<const float4 *>(sU + i * DVB);
+        for (int tt = i; tt < nt; tt += DK) {   // per token: sum over the CTA's columns of u_j do_j (row-independent)
+            const float4 *d4p = reinterpret_cast<const float4 *>(sDO + tt * DVB);
+            const float4 *u4p = reinterpret_cast<const float4 *>(sU + tt * DVB);
             float2 udo = make_float2(0.f, 0.f);
 #pragma unroll
             for (int c4 = 0; c4 < NQ; ++c4) {
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(DK) scan_bwd_rows_kernel(FwdArgs a, BwdArgs g)
                 udo = __ffma2_rn(make_float2(u4.x, u4.y), make_float2(d4.x, d4.y), udo);
                 udo = __ffma2_rn(make_float2(u4.z, u4.w), make_float2(d4.z, d4.w), udo);
             }
-            smf[L::UDO + i] = udo.x + udo.y;
+            smf[L::UDO + tt] = udo.x + udo.y;
         }
         // ---- replay: S_{t-1} every CKP tokens into scratch.  u_t comes from the checkpoint
         // scan, so a step is the update S_ij = alpha_i S_ij + k_i u_j alone (the scan's own
