@@ -83,14 +83,14 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def backward_algorithmic(inp) -> dict:
-    """Arithmetic of the backward as built, per head-token: the checkpoint scan
-    (u and the state update: 2 d_k d_v FMAs), the replay of each chunk (the same
-    2) and the adjoint step (G += q do^T, the row sums S do, G u, S dS', S du,
-    the column sum k^T G, dS' and G <- Diag(alpha) dS': 7.5 d_k d_v FMAs), i.e.
-    23 d_k d_v flops.  The recomputation of states between stored ones is not
-    counted."""
+    """Arithmetic the backward needs per head-token: one forward pass for the
+    states (u and the state update: 2 d_k d_v FMAs) and the adjoint step
+    (G += q do^T, the row sums S do, G u, S dS', S du, the column sum k^T G,
+    dS' and G <- Diag(alpha) dS': 7.5 d_k d_v FMAs), i.e. 19 d_k d_v flops.
+    Recomputation is not counted: neither the replay of each chunk from its
+    checkpoint nor the states between stored ones."""
     heads_tokens = inp.B * inp.T * inp.H
-    return {"tokens": inp.B * inp.T, "flops": 23.0 * inp.d_k * inp.d_v * heads_tokens}
+    return {"tokens": inp.B * inp.T, "flops": 19.0 * inp.d_k * inp.d_v * heads_tokens}
 
 
 def source_digest(paths) -> str:
